@@ -1,0 +1,243 @@
+"""ctypes binding for the plain-C CPU oracle (``kv4_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY.  The tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg
+of ``bench.py`` are the only callers; the product package never imports this module.  It
+shares no code with the CUDA library: the byte layout, the quantisers and the attention are
+all restated in ``kv4_oracle.c``.
+
+The oracle follows the method pages (KV4-RL, "Methodology in Plain English" paragraphs 2-3
+and "Key Contributions" item 4; SAW-INT4 section 2).  Arrays are NumPy; every call here is
+argument marshalling only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kv4_oracle.c")
+_HDR = os.path.join(_HERE, "kv4_oracle.h")
+LIB_PATH = os.path.join(_HERE, "liboracle_kv4.so")
+
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+          "-msse2", "-mfpmath=sse", "-fopenmp", "-Wall", "-Wextra"]
+
+RN, RD, RU = 0, 1, 2
+F32, BF16, F16 = 0, 1, 2
+REGIONAL, SINGLE = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``liboracle_kv4.so`` (skipped when up to date)."""
+    if not force and os.path.exists(LIB_PATH):
+        lib_t = os.path.getmtime(LIB_PATH)
+        if lib_t >= os.path.getmtime(_SRC) and lib_t >= os.path.getmtime(_HDR):
+            return LIB_PATH
+    tmp = LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.run(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+    os.replace(tmp, LIB_PATH)
+    return LIB_PATH
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "num_q_heads", "num_kv_heads", "head_dim", "page_size", "num_sinks",
+        "recent_window", "hadamard_block", "max_seqs")]
+
+
+@dataclass(frozen=True)
+class Config:
+    """Cache geometry (same meaning as the library's configuration record)."""
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    page_size: int
+    num_sinks: int
+    recent_window: int
+    hadamard_block: int
+    max_seqs: int
+
+    def c(self) -> _Cfg:
+        return _Cfg(self.num_q_heads, self.num_kv_heads, self.head_dim, self.page_size,
+                    self.num_sinks, self.recent_window, self.hadamard_block, self.max_seqs)
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        # KV4_ORACLE_LIB names an alternative build of this same source (the mutation test
+        # compiles deliberately broken copies and checks that the pins reject them).
+        path = os.environ.get("KV4_ORACLE_LIB") or build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        S = ctypes.c_size_t
+        cfgp = ctypes.POINTER(_Cfg)
+        L.orc_f32_to_f16.argtypes = [ctypes.c_float, I]
+        L.orc_f32_to_f16.restype = ctypes.c_uint16
+        L.orc_f16_to_f32.argtypes = [ctypes.c_uint16]
+        L.orc_f16_to_f32.restype = ctypes.c_float
+        L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        L.orc_bf16_to_f32.restype = ctypes.c_float
+        L.orc_fwht_f32.argtypes = [P, I, I]
+        L.orc_fwht_f64.argtypes = [P, I, I]
+        L.orc_quant_int4.argtypes = [P, I, P, P, P]
+        L.orc_quant_int8.argtypes = [P, I, P, P]
+        for n in ("orc_page_bytes", "orc_side_slot_bytes"):
+            getattr(L, n).argtypes = [cfgp]
+            getattr(L, n).restype = S
+        L.orc_side_tiles.argtypes = [cfgp]
+        L.orc_side_tiles.restype = I
+        for n in ("orc_k4_byte", "orc_v4_byte", "orc_p4_byte", "orc_k8_byte", "orc_v8_byte", "orc_s8_byte"):
+            getattr(L, n).argtypes = [cfgp, I, I, I, I]
+            getattr(L, n).restype = S
+        L.orc_side_row.argtypes = [cfgp, I]
+        L.orc_side_row.restype = I
+        L.orc_append.argtypes = [cfgp, P, P, I, P, I, P, I, P, P, P, P, I]
+        L.orc_append.restype = I
+        L.orc_dequant_seq.argtypes = [cfgp, P, P, P, I, I, I, P, P, P]
+        L.orc_dequant_seq.restype = I
+        L.orc_decode.argtypes = [cfgp, P, P, I, P, I, P, I, P, P, P, I, I, I, I]
+        L.orc_decode.restype = I
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# ---------------------------------------------------------------- scalar helpers
+
+def f32_to_f16(x: float, mode: int = RN) -> int:
+    return int(lib().orc_f32_to_f16(ctypes.c_float(float(x)), mode))
+
+
+def f16_to_f32(bits: int) -> float:
+    return float(lib().orc_f16_to_f32(ctypes.c_uint16(int(bits))))
+
+
+def bf16_to_f32(bits: int) -> float:
+    return float(lib().orc_bf16_to_f32(ctypes.c_uint16(int(bits))))
+
+
+def fwht_f32(x: np.ndarray, h: int) -> np.ndarray:
+    y = np.ascontiguousarray(x, dtype=np.float32).copy()
+    lib().orc_fwht_f32(_p(y), y.size, h)
+    return y
+
+
+def fwht_f64(x: np.ndarray, h: int) -> np.ndarray:
+    y = np.ascontiguousarray(x, dtype=np.float64).copy()
+    lib().orc_fwht_f64(_p(y), y.size, h)
+    return y
+
+
+def quant_int4(x: np.ndarray):
+    """Returns (codes uint8[D], scale_bits, zero_bits)."""
+    xf = np.ascontiguousarray(x, dtype=np.float32)
+    codes = np.zeros(xf.size, np.uint8)
+    sc = np.zeros(1, np.uint16)
+    zr = np.zeros(1, np.uint16)
+    lib().orc_quant_int4(_p(xf), xf.size, _p(codes), _p(sc), _p(zr))
+    return codes, int(sc[0]), int(zr[0])
+
+
+def quant_int8(x: np.ndarray):
+    """Returns (codes int8[D], scale_bits)."""
+    xf = np.ascontiguousarray(x, dtype=np.float32)
+    codes = np.zeros(xf.size, np.int8)
+    sc = np.zeros(1, np.uint16)
+    lib().orc_quant_int8(_p(xf), xf.size, _p(codes), _p(sc))
+    return codes, int(sc[0])
+
+
+# ---------------------------------------------------------------- cache-level calls
+
+def page_bytes(cfg: Config) -> int:
+    return int(lib().orc_page_bytes(ctypes.byref(cfg.c())))
+
+
+def side_slot_bytes(cfg: Config) -> int:
+    return int(lib().orc_side_slot_bytes(ctypes.byref(cfg.c())))
+
+
+def side_tiles(cfg: Config) -> int:
+    return int(lib().orc_side_tiles(ctypes.byref(cfg.c())))
+
+
+def byte_offset(kind: str, cfg: Config, a: int, g: int, r: int, e: int) -> int:
+    """kind in {k4, v4, p4, k8, v8, s8}; (a, g, r, e) = (page or slot, kv head, position in
+    page or side row, element or is_v)."""
+    return int(getattr(lib(), f"orc_{kind}_byte")(ctypes.byref(cfg.c()), a, g, r, e))
+
+
+def side_row(cfg: Config, pos: int) -> int:
+    return int(lib().orc_side_row(ctypes.byref(cfg.c()), pos))
+
+
+def _dtype_code(a: np.ndarray, declared: int | None) -> int:
+    if declared is not None:
+        return declared
+    if a.dtype == np.float32:
+        return F32
+    raise TypeError("uint16 inputs need an explicit dtype code (BF16 or F16)")
+
+
+def append(cfg: Config, pool: np.ndarray, side: np.ndarray, K: np.ndarray, V: np.ndarray,
+           seq_slot: np.ndarray, pos: np.ndarray, lens_after: np.ndarray, page_table: np.ndarray,
+           k_dtype: int | None = None, v_dtype: int | None = None) -> None:
+    """Append T tokens.  K, V: [T][Hkv][D] float32, or uint16 bit patterns with a dtype code."""
+    K = np.ascontiguousarray(K)
+    V = np.ascontiguousarray(V)
+    seq_slot = np.ascontiguousarray(seq_slot, np.int32)
+    pos = np.ascontiguousarray(pos, np.int32)
+    lens_after = np.ascontiguousarray(lens_after, np.int32)
+    page_table = np.ascontiguousarray(page_table, np.int32)
+    T = int(seq_slot.size)
+    rc = lib().orc_append(ctypes.byref(cfg.c()), _p(pool), _p(side), T, _p(K), _dtype_code(K, k_dtype),
+                          _p(V), _dtype_code(V, v_dtype), _p(seq_slot), _p(pos), _p(lens_after),
+                          _p(page_table), int(page_table.shape[1]))
+    if rc != 0:
+        raise RuntimeError(f"orc_append failed: {rc}")
+
+
+def dequant_seq(cfg: Config, pool: np.ndarray, side: np.ndarray, page_row: np.ndarray, slot: int,
+                L: int, g: int):
+    """Dense fp64 (khat [L][D], vhat [L][D], region [L]) of one (sequence, kv head)."""
+    D = cfg.head_dim
+    khat = np.zeros((L, D), np.float64)
+    vhat = np.zeros((L, D), np.float64)
+    region = np.zeros(L, np.int32)
+    page_row = np.ascontiguousarray(page_row, np.int32)
+    rc = lib().orc_dequant_seq(ctypes.byref(cfg.c()), _p(pool), _p(side), _p(page_row), slot, L, g,
+                               _p(khat), _p(vhat), _p(region))
+    if rc != 0:
+        raise RuntimeError(f"orc_dequant_seq failed: {rc}")
+    return khat, vhat, region
+
+
+def decode(cfg: Config, pool: np.ndarray, side: np.ndarray, q: np.ndarray, page_table: np.ndarray,
+           lens: np.ndarray, mode: int = REGIONAL, chunk_tokens: int = 0, reverse: bool = False,
+           q_dtype: int | None = None, nthreads: int = 1):
+    """Decode attention for B = len(lens) sequences; returns (out [B][Hq][D], lse [B][Hq])."""
+    q = np.ascontiguousarray(q)
+    lens = np.ascontiguousarray(lens, np.int32)
+    page_table = np.ascontiguousarray(page_table, np.int32)
+    B = int(lens.size)
+    out = np.zeros((B, cfg.num_q_heads, cfg.head_dim), np.float64)
+    lse = np.zeros((B, cfg.num_q_heads), np.float64)
+    rc = lib().orc_decode(ctypes.byref(cfg.c()), _p(pool), _p(side), B, _p(q), _dtype_code(q, q_dtype),
+                          _p(page_table), int(page_table.shape[1]), _p(lens), _p(out), _p(lse), mode,
+                          int(chunk_tokens), int(bool(reverse)), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"orc_decode failed: {rc}")
+    return out, lse

@@ -1,0 +1,98 @@
+"""Plant plausible mistakes in copies of the oracle (on the CPU) and check the pins catch them.
+
+Each mutant is one textual edit of ``oracle/kv4_oracle.c`` (a dropped term, a wrong sign,
+rounding mode, index or constant).  It is compiled to a temporary library and the full pin
+list runs against it in a child process; the mutant is "killed" when any pin fails (or the
+child crashes).  A surviving mutant means the pins do not constrain that part of the oracle.
+"""
+import os
+import subprocess
+import sys
+import tempfile
+from concurrent.futures import ThreadPoolExecutor
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "kv4_oracle.c")
+
+# (name, original text, replacement, occurrence index or None for all)
+MUTANTS = [
+    ("butterfly-sign", "x[j + st] = a - b;", "x[j + st] = b - a;", 0),
+    ("butterfly-f64-sign", "x[j + st] = a - b;", "x[j + st] = b - a;", 1),
+    ("zero-round-nearest", "orc_f32_to_f16(mn, ORC_RD)", "orc_f32_to_f16(mn, ORC_RN)", None),
+    ("scale-round-nearest", "orc_f32_to_f16(sq, ORC_RU)", "orc_f32_to_f16(sq, ORC_RN)", None),
+    ("int4-levels-16", "r / 15.0f", "r / 16.0f", None),
+    ("int4-truncate", "const float rq = rintf(t);", "const float rq = truncf(t);", None),
+    ("int8-levels-128", "a / 127.0f", "a / 128.0f", None),
+    ("int8-scale-round-nearest", "orc_f32_to_f16(a / 127.0f, ORC_RU)", "orc_f32_to_f16(a / 127.0f, ORC_RN)", None),
+    ("nibble-swap", "put_nibble(pool, orc_k4_byte(c, page, g, pp, e), e & 1, c4[e]);",
+     "put_nibble(pool, orc_k4_byte(c, page, g, pp, e), (e & 1) ^ 1, c4[e]);", None),
+    ("v4-pair-index", "4 * j + 2 * (r & 1) + (k >> 1)", "4 * j + 2 * ((r >> 1) & 1) + (k >> 1)", None),
+    ("k8-no-swizzle", "16 * ((e / 16) ^ (r & 1))", "16 * (e / 16)", None),
+    ("route-ring-strict", "p >= lens_after[b] - w", "p > lens_after[b] - w", None),
+    ("ring-row-no-offset", "row = s + p % w;", "row = p % w;", None),
+    ("q-rot-sqrt-norm", "qr[e] *= 1.0 / (double)h;", "qr[e] *= 1.0 / sqrt((double)h);", None),
+    ("q-not-rotated", "orc_fwht_f64(qr, D, h);", ";", None),
+    ("tau-wrong", "1.0 / sqrt((double)D)", "1.0 / (double)D", None),
+    ("merge-no-rescale-l", "l += parts[i].l * f;", "l += parts[i].l;", None),
+    ("merge-no-rescale-o", "out[e] += parts[i].o[e] * f;", "out[e] += parts[i].o[e];", None),
+    ("recent-begin-off-by-one", "const int r_begin = (L - w) > s ? (L - w) : s;",
+     "const int r_begin = (L - w + 1) > s ? (L - w + 1) : s;", None),
+    ("dequant-drop-zero", "kr[e] = kz + ks *", "kr[e] = ks *", None),
+    ("gqa-map", "(size_t)(g * G + i)", "(size_t)(g + i * Hkv)", None),
+    ("f16-no-subnormal", "if (E < -14) E = -14;", ";", None),
+    ("f16-ties-away", "(frac == 0.5 && fmod(n, 2.0) == 1.0)", "(frac == 0.5)", None),
+    ("single-softmax-max", "if (logit[j] > ps->m) ps->m = logit[j];", "if (logit[j] < ps->m) ps->m = logit[j];", None),
+]
+
+RUNNER = r"""
+import sys
+sys.path.insert(0, {root!r}); sys.path.insert(0, {tests!r})
+import oracle_pins as P
+for i, pin in enumerate(P.ALL_PINS):
+    try:
+        pin()
+    except Exception as e:
+        print("KILLED by pin", i, type(e).__name__)
+        sys.exit(3)
+print("SURVIVED")
+sys.exit(0)
+"""
+
+
+def _mutate(text: str, old: str, new: str, occ):
+    assert old in text, f"mutation anchor not found: {old!r}"
+    if occ is None:
+        return text.replace(old, new)
+    parts = text.split(old)
+    assert len(parts) > occ + 1, f"occurrence {occ} of {old!r} missing"
+    return old.join(parts[:occ + 1]) + new + old.join(parts[occ + 1:])
+
+
+def _run_mutant(tmp: str, name: str, old: str, new: str, occ) -> tuple[str, str]:
+    src = _mutate(open(SRC).read(), old, new, occ)
+    d = os.path.join(tmp, name)
+    os.makedirs(d)
+    csrc = os.path.join(d, "kv4_oracle.c")
+    with open(csrc, "w") as f:
+        f.write(src)
+    import shutil
+    shutil.copy(os.path.join(ROOT, "oracle", "kv4_oracle.h"), d)
+    so = os.path.join(d, "lib.so")
+    from oracle.oracle import CFLAGS
+    subprocess.run(["gcc", *[c for c in CFLAGS if c not in ("-Wall", "-Wextra")], "-o", so, csrc, "-lm"],
+                   check=True, capture_output=True)
+    env = dict(os.environ, KV4_ORACLE_LIB=so, OMP_NUM_THREADS="1")
+    r = subprocess.run([sys.executable, "-c", RUNNER.format(root=ROOT, tests=os.path.join(ROOT, "tests"))],
+                       env=env, capture_output=True, text=True, timeout=600)
+    return name, (r.stdout.strip().splitlines() or ["(crashed: %d)" % r.returncode])[-1]
+
+
+@pytest.mark.slow
+def test_every_mutant_is_killed():
+    with tempfile.TemporaryDirectory() as tmp:
+        with ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
+            results = list(ex.map(lambda m: _run_mutant(tmp, *m), MUTANTS))
+    survivors = [(n, r) for n, r in results if "SURVIVED" in r]
+    assert not survivors, f"mutants not caught by any pin: {survivors}"
