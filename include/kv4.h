@@ -1,0 +1,173 @@
+/*
+ * kv4.h -- C ABI of libkv4.so: a paged, calibration-free INT4 KV cache with an INT8 sink/recent
+ * side cache, and decode-step attention over it, for NVIDIA B200 (sm_100a).
+ *
+ * The method (page titles and sections it is defined in):
+ *   KV4-RL: Unlocking Faster Asynchronous Rollouts for RLVR with INT4 KV Cache Quantization
+ *     (ai.info summary), "Methodology in Plain English" paragraphs 2-3 and "Key Contributions"
+ *     item 4: every new K/V vector becomes one affine INT4 group per token-head vector with an
+ *     FP16 scale and offset, applied after the dot-product reduction; keys are stored in a
+ *     Hadamard-rotated basis and queries are rotated to match; the packed codes are read
+ *     directly by the attention kernel; an INT8 side cache holds the first s (sink) and the
+ *     most recent w positions; the INT4 and INT8 regions are attended as disjoint sets and
+ *     combined through regional softmax statistics.
+ *   SAW-INT4: System-Aware 4-Bit KV-Cache Quantization (gist.science summary), section 2:
+ *     token-wise INT4 in the unchanged paged buffers, block-diagonal Hadamard rotation with
+ *     block size h, rotation and quantisation fused in one kernel.
+ *
+ * Conventions the pages leave open (fixed here, identical in the test oracle):
+ *   - Hadamard: Sylvester order, unnormalised, on contiguous blocks of h elements (h a power
+ *     of two dividing head_dim; h = 1 means no rotation).  Keys are stored rotated; the query
+ *     is multiplied by H/h, so rotated query . rotated key = q . k.  Values are not rotated.
+ *   - INT4: zero = fp16 rounded toward -inf of min(x); scale = fp16 rounded toward +inf of
+ *     fl32(max(x) - zero)/15; code = clamp(rint((x - zero)/scale), 0, 15) in IEEE fp32;
+ *     x is reconstructed as zero + scale * code.
+ *   - INT8 (side cache): symmetric, scale = fp16 rounded toward +inf of max|x|/127,
+ *     code = clamp(rint(x/scale), -127, 127).
+ *   - Routing: every appended token is written to the INT4 pages; in addition position pos
+ *     goes to side row pos when pos < s, and to side row s + (pos mod w) when pos >= s and
+ *     pos >= lens_after[seq] - w.  Decode at length L reads sinks [0, min(s, L)) and recent
+ *     [max(s, L - w), L) from the side cache and the INT4 region [s, max(s, L - w)) from pages.
+ *   - Attention: q head j reads KV head j / (Hq/Hkv); softmax scale 1/sqrt(head_dim);
+ *     out is fp32, lse (optional) is m + ln(l) in natural log.
+ *
+ * Memory: the caller owns every device buffer (page pools, side cache, workspace, inputs,
+ * outputs) and the stream.  The library never allocates or frees device memory in these calls;
+ * kv4_cache_init allocates only the small host handle.  All launches are asynchronous on the
+ * given stream (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *
+ * Errors: arguments are validated on the host before anything is launched; a failed check
+ * returns a status and launches nothing.  A failed launch returns KV4_ERR_CUDA.  Device-side
+ * guards (page id outside the pool, a bounded wait that ran out) skip the access and set bits
+ * in a per-device error word read by kv4_get_device_error.  No kernel traps or spins forever.
+ */
+#ifndef KV4_H
+#define KV4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KV4_OK = 0,
+  KV4_ERR_INVALID_ARG = 1,  /* null pointer, negative size, index out of range          */
+  KV4_ERR_UNSUPPORTED = 2,  /* geometry outside the compiled variants (see kv4_config)  */
+  KV4_ERR_WORKSPACE = 3,    /* workspace missing or smaller than kv4_*_workspace_bytes  */
+  KV4_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed              */
+  KV4_ERR_DEVICE = 5        /* device-side guard fired (kv4_get_device_error has bits)  */
+} kv4_status;
+
+typedef enum { KV4_F32 = 0, KV4_BF16 = 1, KV4_F16 = 2 } kv4_dtype;
+
+/* Device error word bits (kv4_get_device_error). */
+#define KV4_DEVERR_PAGE_RANGE 0x1u  /* page-table entry outside [0, max_pages)            */
+#define KV4_DEVERR_WAIT_LIMIT 0x2u  /* a bounded wait for a bulk copy ran out             */
+#define KV4_DEVERR_LENGTH 0x4u      /* a length or position beyond the page-table row     */
+
+/*
+ * Cache geometry.  Supported: head_dim in {64, 128}; Hq/Hkv in {1, 2, 4}; page_size a
+ * multiple of 16; hadamard_block a power of two dividing head_dim; num_sinks >= 0,
+ * recent_window >= 0.  One page table (int32 [max_seqs][stride]) is shared by all layers, as in
+ * vLLM; page ids index a per-layer pool of max_pages pages.
+ */
+typedef struct {
+  int num_layers;
+  int num_q_heads;      /* Hq                                    */
+  int num_kv_heads;     /* Hkv                                   */
+  int head_dim;         /* D                                     */
+  int page_size;        /* P, positions per page                 */
+  int num_sinks;        /* s                                     */
+  int recent_window;    /* w                                     */
+  int hadamard_block;   /* h                                     */
+  int max_seqs;         /* sequence slots of the INT8 side cache */
+  int max_pages;        /* pages per layer pool                  */
+} kv4_config;
+
+typedef struct kv4_cache kv4_cache;  /* opaque host handle */
+
+/*
+ * Byte sizes the caller must allocate (all layers):
+ *   page pool:  num_layers * max_pages * Hkv * P * (D + 8)
+ *               (per token and KV head: D/2 bytes of K codes + D/2 of V codes + 2x fp16
+ *               scale/zero for K and for V; 4 + 32/D bits per element for D = 128 -> 4.25)
+ *   side cache: num_layers * max_seqs * Hkv * ceil((s + w)/16) * 16 * (2D + 4)
+ * Both must be 16-byte aligned.  Returns KV4_ERR_UNSUPPORTED for geometries outside the list.
+ */
+kv4_status kv4_query_sizes(const kv4_config* cfg, size_t* page_pool_bytes, size_t* side_cache_bytes);
+
+/* Bind caller-owned device buffers to a host handle (no device work).  *out receives the handle. */
+kv4_status kv4_cache_init(const kv4_config* cfg, void* page_pool, void* side_cache, kv4_cache** out);
+
+/* Free the host handle; caller memory is untouched.  NULL is ignored. */
+void kv4_cache_destroy(kv4_cache* cache);
+
+/*
+ * kv4_append: write T new tokens of one layer.  Fused per (token, KV head): block-Hadamard
+ * rotation of K, per-token affine INT4 quantisation of rotated K and of V, nibble packing into
+ * the token's page slot (page page_table[seq][pos / P], slot pos % P), and INT8 routing of
+ * sink/recent positions into the side cache.
+ *   K, V         device [T][Hkv][D] of k_dtype / v_dtype (KV4_F32 or KV4_BF16), contiguous
+ *   seq_slot     device int32 [T]: sequence slot of each token, in [0, max_seqs)
+ *   pos          device int32 [T]: position of each token in its sequence
+ *   lens_after   device int32 [max_seqs]: sequence length after this call (decides which
+ *                positions are "recent"); positions of one sequence must be distinct in a call
+ *   page_table   device int32 [max_seqs][stride]
+ * Device-side: a page id outside [0, max_pages) or pos / P >= stride sets an error bit and the
+ * token is skipped.
+ */
+kv4_status kv4_append(kv4_cache* cache, int layer, int T, const void* K, kv4_dtype k_dtype,
+                      const void* V, kv4_dtype v_dtype, const int32_t* seq_slot, const int32_t* pos,
+                      const int32_t* lens_after, const int32_t* page_table, int stride, void* stream);
+
+/* Workspace bytes kv4_decode_attn needs for a batch of B sequences (upper bound for any lens). */
+kv4_status kv4_decode_workspace_bytes(const kv4_cache* cache, int B, size_t* bytes);
+
+/*
+ * kv4_decode_attn: one decode step of attention for B sequences (row b of the batch is side-cache
+ * slot b) at lengths lens[b] (the just-appended token included).  Rotates each query once
+ * (H/h), streams the packed INT4 pages of [s, max(s, L-w)) and the INT8 rows of the sink and
+ * recent regions, and merges per-region / per-split softmax statistics.
+ *   q            device [B][Hq][D] of q_dtype (KV4_F32, KV4_BF16 or KV4_F16)
+ *   page_table   device int32 [>= B][stride];  lens device int32 [B] (0 gives out = 0, lse = -inf)
+ *   max_len_hint host upper bound of lens (0 = unknown); only sizes the grid
+ *   out          device fp32 [B][Hq][D];  lse device fp32 [B][Hq] or NULL
+ *   workspace    device scratch of at least kv4_decode_workspace_bytes(B) bytes, 16-byte aligned;
+ *                its contents need no initialisation and are overwritten
+ * Two launches on the stream (split-K partials, then their merge).
+ */
+kv4_status kv4_decode_attn(kv4_cache* cache, int layer, int B, const void* q, kv4_dtype q_dtype,
+                           const int32_t* page_table, int stride, const int32_t* lens, int max_len_hint,
+                           float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * BF16-KV baseline with the same page table and conventions, no quantisation and no rotation:
+ * a page holds Hkv head blocks of P * 4D bytes (bf16 K and V).  Used to measure the INT4
+ * speed-up on the same box.  kv4_bf16_query_sizes returns num_layers * max_pages * Hkv * P * 4D.
+ */
+kv4_status kv4_bf16_query_sizes(const kv4_config* cfg, size_t* page_pool_bytes);
+kv4_status kv4_bf16_cache_init(const kv4_config* cfg, void* page_pool, kv4_cache** out);
+kv4_status kv4_bf16_append(kv4_cache* cache, int layer, int T, const void* K, kv4_dtype k_dtype,
+                           const void* V, kv4_dtype v_dtype, const int32_t* seq_slot, const int32_t* pos,
+                           const int32_t* page_table, int stride, void* stream);
+kv4_status kv4_bf16_decode_workspace_bytes(const kv4_cache* cache, int B, size_t* bytes);
+kv4_status kv4_bf16_decode_attn(kv4_cache* cache, int layer, int B, const void* q, kv4_dtype q_dtype,
+                                const int32_t* page_table, int stride, const int32_t* lens,
+                                int max_len_hint, float* out, float* lse, void* workspace,
+                                size_t ws_bytes, void* stream);
+
+/* Read and clear the device error word of the current device (synchronises the device). */
+kv4_status kv4_get_device_error(uint32_t* bits);
+
+/* Number of kernels the library has launched since load (all devices). */
+uint64_t kv4_launch_count(void);
+
+const char* kv4_status_string(kv4_status status);
+int kv4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KV4_H */

@@ -1,0 +1,159 @@
+// kv4_device.cuh -- device helpers shared by the libkv4 kernels (sm_100a).
+//
+// Bulk (1-D TMA) copies with mbarrier completion, bounded mbarrier waits, the legacy
+// warp-level tensor-core MMA used for the tiny GQA contractions, and the register-level
+// conversions from packed INT4 / INT8 codes to fp16 MMA operands.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/kv4.h"
+
+namespace kv4 {
+
+// ------------------------------------------------------------------ shared-memory addressing
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ------------------------------------------------------------------ mbarrier + bulk copy
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Arrive once and add `bytes` to the barrier's expected transaction count.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+// One bulk copy global -> shared; completion is signalled on `bar` as `bytes` transactions.
+// src, dst and bytes must be multiples of 16 bytes.  Never multicast.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for phase `parity` of `bar`, giving up after about two seconds (global timer) or 2^26
+// polls, whichever comes first.  On expiry the error bit is set and false is returned; the
+// caller then stops consuming and drains.  No kernel of this library spins without a bound.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint32_t kWaitLimitPolls = 1u << 26;
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1; it < kWaitLimitPolls; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) break;
+  }
+  atomicOr(err, KV4_DEVERR_WAIT_LIMIT);
+  return false;
+}
+
+// ------------------------------------------------------------------ tensor-core MMA (m16n8k16)
+
+// D = A(16x16, row) * B(16x8, col) + C, fp16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ------------------------------------------------------------------ code -> fp16 conversions
+
+// Two INT4 codes of a 32-bit word, the nibbles at bits 4k and 16+4k, become the fp16 pair
+// (1 + c/16): the code is moved into the top four fraction bits of the fp16 1.0 pattern.
+// The value is exact, and the MMA result is corrected afterwards (x = 1 + c/16 means
+// c = 16 x - 16), which keeps the offset small next to the signal.
+template <int K>
+__device__ __forceinline__ uint32_t nib2h(uint32_t w) {
+  uint32_t t;
+  if constexpr (K == 0)
+    t = w << 6;
+  else if constexpr (K == 1)
+    t = w << 2;
+  else if constexpr (K == 2)
+    t = w >> 2;
+  else
+    t = w >> 6;
+  return (t & 0x03C003C0u) | 0x3C003C00u;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Bytes 0 and 1 (SEL = 0x4140) or 2 and 3 (SEL = 0x4342) of a word of signed INT8 codes that
+// was XOR-ed with 0x80808080, widened to the exact fp16 pair (c0, c1): 0x64 in the high byte
+// makes 1024 + (c + 128); subtracting 1152 leaves c.
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t i8x2_to_h2(uint32_t biased) {
+  const uint32_t h = prmt(biased, 0x64646464u, SEL);
+  __half2 v = *reinterpret_cast<const __half2*>(&h);
+  v = __hsub2(v, __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));  // 1152
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
+  return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+}
+
+__device__ __forceinline__ uint32_t pack_bf2(__nv_bfloat16 lo, __nv_bfloat16 hi) {
+  return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+}
+
+// ------------------------------------------------------------------ input loads
+
+__device__ __forceinline__ float load_as_f32(const void* base, int dtype, size_t i) {
+  if (dtype == KV4_F32) return reinterpret_cast<const float*>(base)[i];
+  if (dtype == KV4_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
+  return __half2float(reinterpret_cast<const __half*>(base)[i]);
+}
+
+}  // namespace kv4

@@ -1,0 +1,61 @@
+// kv4_internal.h -- host-side launch interfaces between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/kv4.h"
+
+namespace kv4 {
+
+struct AppendArgs {
+  uint8_t* pool;          // layer base of the INT4 page pool (or BF16 pool)
+  uint8_t* side;          // layer base of the INT8 side cache (INT4 cache only)
+  const void* K;
+  const void* V;
+  int k_dtype, v_dtype;
+  const int32_t* seq_slot;
+  const int32_t* pos;
+  const int32_t* lens_after;
+  const int32_t* page_table;
+  int stride;
+  int T, Hkv, P, s, w, h, max_seqs, max_pages, nt8;
+  size_t page_bytes, side_slot_bytes;
+  uint32_t* err;
+};
+
+struct DecodeArgs {
+  const uint8_t* pool;
+  const uint8_t* side;
+  const void* q;
+  int q_dtype;
+  const int32_t* page_table;
+  int stride;
+  const int32_t* lens;
+  int B, Hq, Hkv, P, s, w, h, max_pages, nt8;
+  size_t page_bytes, side_slot_bytes;
+  float* part;            // split partials [num_slots][G][D + 2]
+  float* out;
+  float* lse;
+  float qscale;           // softmax scale in log2 units: log2(e) / sqrt(D)
+  int W;                  // warps launched by the partial kernel
+  uint32_t* err;
+};
+
+// Launchers return cudaSuccess or the launch error.  `grid_ctas` is filled with the CTA count
+// used (decode), so the host can size and check the workspace.
+cudaError_t launch_append_int4(const AppendArgs& a, int D, cudaStream_t st);
+cudaError_t launch_append_bf16(const AppendArgs& a, int D, cudaStream_t st);
+
+int decode_warps_per_cta();
+int bf16_decode_warps_per_cta();
+size_t decode_smem_bytes(int D, int G);
+size_t bf16_decode_smem_bytes(int D, int G);
+cudaError_t launch_decode_int4(DecodeArgs a, int D, int G, int ctas, cudaStream_t st);
+cudaError_t launch_decode_bf16(DecodeArgs a, int D, int G, int ctas, cudaStream_t st);
+
+// Counts every kernel launch the library issues.
+void note_launches(int n);
+
+}  // namespace kv4

@@ -1,0 +1,303 @@
+"""ctypes binding of libkv4.so (C ABI in include/kv4.h).
+
+Each function has the name of the C entry point it wraps and only marshals arguments: torch
+CUDA tensors become device pointers, streams become cudaStream_t handles, and a non-OK status
+raises ``KV4Error``.  All computation happens in the CUDA kernels of libkv4.so; there is no
+fallback path, and importing this module fails loudly when the library is missing.
+
+``Cache`` and ``BF16Cache`` are conveniences that allocate the caller-owned buffers with torch
+(PyTorch is used here for device memory and streams only).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkv4.so")
+
+KV4_OK, KV4_ERR_INVALID_ARG, KV4_ERR_UNSUPPORTED, KV4_ERR_WORKSPACE, KV4_ERR_CUDA, KV4_ERR_DEVICE = range(6)
+KV4_F32, KV4_BF16, KV4_F16 = 0, 1, 2
+KV4_DEVERR_PAGE_RANGE, KV4_DEVERR_WAIT_LIMIT, KV4_DEVERR_LENGTH = 0x1, 0x2, 0x4
+
+# every entry point declared in include/kv4.h
+SYMBOLS = (
+    "kv4_query_sizes", "kv4_cache_init", "kv4_cache_destroy", "kv4_append", "kv4_decode_workspace_bytes",
+    "kv4_decode_attn", "kv4_bf16_query_sizes", "kv4_bf16_cache_init", "kv4_bf16_append",
+    "kv4_bf16_decode_workspace_bytes", "kv4_bf16_decode_attn", "kv4_get_device_error", "kv4_launch_count",
+    "kv4_status_string", "kv4_version",
+)
+
+
+class KV4Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        self.status = status
+
+
+class kv4_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "num_layers", "num_q_heads", "num_kv_heads", "head_dim", "page_size", "num_sinks",
+        "recent_window", "hadamard_block", "max_seqs", "max_pages")]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with `python -m int4_kv_cache_append_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, S, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64
+    cfgp = ctypes.POINTER(kv4_config)
+    i32p = ctypes.c_void_p
+    sig = {
+        "kv4_query_sizes": (I, [cfgp, ctypes.POINTER(S), ctypes.POINTER(S)]),
+        "kv4_cache_init": (I, [cfgp, P, P, ctypes.POINTER(P)]),
+        "kv4_cache_destroy": (None, [P]),
+        "kv4_append": (I, [P, I, I, P, I, P, I, i32p, i32p, i32p, i32p, I, P]),
+        "kv4_decode_workspace_bytes": (I, [P, I, ctypes.POINTER(S)]),
+        "kv4_decode_attn": (I, [P, I, I, P, I, i32p, I, i32p, I, P, P, P, S, P]),
+        "kv4_bf16_query_sizes": (I, [cfgp, ctypes.POINTER(S)]),
+        "kv4_bf16_cache_init": (I, [cfgp, P, ctypes.POINTER(P)]),
+        "kv4_bf16_append": (I, [P, I, I, P, I, P, I, i32p, i32p, i32p, I, P]),
+        "kv4_bf16_decode_workspace_bytes": (I, [P, I, ctypes.POINTER(S)]),
+        "kv4_bf16_decode_attn": (I, [P, I, I, P, I, i32p, I, i32p, I, P, P, P, S, P]),
+        "kv4_get_device_error": (I, [ctypes.POINTER(ctypes.c_uint32)]),
+        "kv4_launch_count": (U, []),
+        "kv4_status_string": (ctypes.c_char_p, [I]),
+        "kv4_version": (I, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.kv4_status_string(status).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != KV4_OK:
+        raise KV4Error(fn, status)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("device tensor expected")
+    if not t.is_contiguous():
+        raise ValueError("contiguous tensor expected")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def dtype_code(t: torch.Tensor) -> int:
+    return {torch.float32: KV4_F32, torch.bfloat16: KV4_BF16, torch.float16: KV4_F16}[t.dtype]
+
+
+# ------------------------------------------------------------------------ C entry points
+
+def kv4_query_sizes(cfg: kv4_config) -> tuple[int, int]:
+    pool, side = ctypes.c_size_t(), ctypes.c_size_t()
+    _check("kv4_query_sizes", lib.kv4_query_sizes(ctypes.byref(cfg), ctypes.byref(pool), ctypes.byref(side)))
+    return pool.value, side.value
+
+
+def kv4_cache_init(cfg: kv4_config, page_pool, side_cache) -> int:
+    h = ctypes.c_void_p()
+    _check("kv4_cache_init", lib.kv4_cache_init(ctypes.byref(cfg), _ptr(page_pool), _ptr(side_cache), ctypes.byref(h)))
+    return h.value
+
+
+def kv4_cache_destroy(handle: int) -> None:
+    lib.kv4_cache_destroy(handle)
+
+
+def kv4_append(handle, layer, T, K, k_dtype, V, v_dtype, seq_slot, pos, lens_after, page_table, stride, stream=None):
+    _check("kv4_append", lib.kv4_append(handle, layer, T, _ptr(K), k_dtype, _ptr(V), v_dtype, _ptr(seq_slot), _ptr(pos),
+                                        _ptr(lens_after), _ptr(page_table), stride, _stream(stream)))
+
+
+def kv4_decode_workspace_bytes(handle, B) -> int:
+    n = ctypes.c_size_t()
+    _check("kv4_decode_workspace_bytes", lib.kv4_decode_workspace_bytes(handle, B, ctypes.byref(n)))
+    return n.value
+
+
+def kv4_decode_attn(handle, layer, B, q, q_dtype, page_table, stride, lens, max_len_hint, out, lse, workspace,
+                    ws_bytes, stream=None):
+    _check("kv4_decode_attn", lib.kv4_decode_attn(handle, layer, B, _ptr(q), q_dtype, _ptr(page_table), stride,
+                                                  _ptr(lens), max_len_hint, _ptr(out), _ptr(lse), _ptr(workspace),
+                                                  ws_bytes, _stream(stream)))
+
+
+def kv4_bf16_query_sizes(cfg: kv4_config) -> int:
+    pool = ctypes.c_size_t()
+    _check("kv4_bf16_query_sizes", lib.kv4_bf16_query_sizes(ctypes.byref(cfg), ctypes.byref(pool)))
+    return pool.value
+
+
+def kv4_bf16_cache_init(cfg: kv4_config, page_pool) -> int:
+    h = ctypes.c_void_p()
+    _check("kv4_bf16_cache_init", lib.kv4_bf16_cache_init(ctypes.byref(cfg), _ptr(page_pool), ctypes.byref(h)))
+    return h.value
+
+
+def kv4_bf16_append(handle, layer, T, K, k_dtype, V, v_dtype, seq_slot, pos, page_table, stride, stream=None):
+    _check("kv4_bf16_append", lib.kv4_bf16_append(handle, layer, T, _ptr(K), k_dtype, _ptr(V), v_dtype, _ptr(seq_slot),
+                                                  _ptr(pos), _ptr(page_table), stride, _stream(stream)))
+
+
+def kv4_bf16_decode_workspace_bytes(handle, B) -> int:
+    n = ctypes.c_size_t()
+    _check("kv4_bf16_decode_workspace_bytes", lib.kv4_bf16_decode_workspace_bytes(handle, B, ctypes.byref(n)))
+    return n.value
+
+
+def kv4_bf16_decode_attn(handle, layer, B, q, q_dtype, page_table, stride, lens, max_len_hint, out, lse, workspace,
+                         ws_bytes, stream=None):
+    _check("kv4_bf16_decode_attn", lib.kv4_bf16_decode_attn(handle, layer, B, _ptr(q), q_dtype, _ptr(page_table), stride,
+                                                            _ptr(lens), max_len_hint, _ptr(out), _ptr(lse),
+                                                            _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def kv4_get_device_error() -> int:
+    v = ctypes.c_uint32()
+    _check("kv4_get_device_error", lib.kv4_get_device_error(ctypes.byref(v)))
+    return v.value
+
+
+def kv4_launch_count() -> int:
+    return int(lib.kv4_launch_count())
+
+
+def kv4_version() -> int:
+    return int(lib.kv4_version())
+
+
+# ------------------------------------------------------------------------ conveniences
+
+@dataclass
+class Geometry:
+    num_layers: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    page_size: int
+    num_sinks: int
+    recent_window: int
+    hadamard_block: int
+    max_seqs: int
+    max_pages: int
+
+    def c(self) -> kv4_config:
+        return kv4_config(self.num_layers, self.num_q_heads, self.num_kv_heads, self.head_dim, self.page_size,
+                          self.num_sinks, self.recent_window, self.hadamard_block, self.max_seqs, self.max_pages)
+
+
+class Cache:
+    """INT4 cache with torch-allocated page pool and side cache (uint8 tensors)."""
+
+    def __init__(self, geo: Geometry, device="cuda", fill: int | None = None):
+        self.geo = geo
+        self.cfg = geo.c()
+        pool_b, side_b = kv4_query_sizes(self.cfg)
+        self.pool = torch.empty(max(pool_b, 16), dtype=torch.uint8, device=device)
+        self.side = torch.empty(max(side_b, 16), dtype=torch.uint8, device=device)
+        if fill is not None:
+            self.pool.fill_(fill)
+            self.side.fill_(fill)
+        self.handle = kv4_cache_init(self.cfg, self.pool, self.side)
+        self._ws = None
+
+    def layer_views(self, layer: int):
+        pool_b, side_b = kv4_query_sizes(self.cfg)
+        pl, sl = pool_b // self.geo.num_layers, side_b // self.geo.num_layers
+        return self.pool[layer * pl:(layer + 1) * pl], self.side[layer * sl:(layer + 1) * sl]
+
+    def append(self, layer, K, V, seq_slot, pos, lens_after, page_table, stream=None):
+        kv4_append(self.handle, layer, int(seq_slot.numel()), K, dtype_code(K), V, dtype_code(V), seq_slot, pos,
+                   lens_after, page_table, int(page_table.shape[1]), stream)
+
+    def workspace(self, B: int) -> torch.Tensor:
+        n = kv4_decode_workspace_bytes(self.handle, B)
+        if self._ws is None or self._ws.numel() < n:
+            self._ws = torch.empty(n, dtype=torch.uint8, device=self.pool.device)
+        return self._ws
+
+    def decode(self, layer, q, page_table, lens, out=None, lse=None, max_len_hint=0, workspace=None, stream=None):
+        B = int(lens.numel())
+        if out is None:
+            out = torch.empty((B, self.geo.num_q_heads, self.geo.head_dim), dtype=torch.float32, device=q.device)
+        ws = workspace if workspace is not None else self.workspace(B)
+        kv4_decode_attn(self.handle, layer, B, q, dtype_code(q), page_table, int(page_table.shape[1]), lens,
+                        max_len_hint, out, lse, ws, ws.numel(), stream)
+        return out
+
+    def close(self):
+        if self.handle:
+            kv4_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class BF16Cache:
+    """BF16-KV baseline cache (same page table conventions, bf16 K and V in the pages)."""
+
+    def __init__(self, geo: Geometry, device="cuda"):
+        self.geo = geo
+        self.cfg = geo.c()
+        self.pool = torch.empty(max(kv4_bf16_query_sizes(self.cfg), 16), dtype=torch.uint8, device=device)
+        self.handle = kv4_bf16_cache_init(self.cfg, self.pool)
+        self._ws = None
+
+    def append(self, layer, K, V, seq_slot, pos, page_table, stream=None):
+        kv4_bf16_append(self.handle, layer, int(seq_slot.numel()), K, dtype_code(K), V, dtype_code(V), seq_slot, pos,
+                        page_table, int(page_table.shape[1]), stream)
+
+    def workspace(self, B: int) -> torch.Tensor:
+        n = kv4_bf16_decode_workspace_bytes(self.handle, B)
+        if self._ws is None or self._ws.numel() < n:
+            self._ws = torch.empty(n, dtype=torch.uint8, device=self.pool.device)
+        return self._ws
+
+    def decode(self, layer, q, page_table, lens, out=None, lse=None, max_len_hint=0, workspace=None, stream=None):
+        B = int(lens.numel())
+        if out is None:
+            out = torch.empty((B, self.geo.num_q_heads, self.geo.head_dim), dtype=torch.float32, device=q.device)
+        ws = workspace if workspace is not None else self.workspace(B)
+        kv4_bf16_decode_attn(self.handle, layer, B, q, dtype_code(q), page_table, int(page_table.shape[1]), lens,
+                             max_len_hint, out, lse, ws, ws.numel(), stream)
+        return out
+
+    def close(self):
+        if self.handle:
+            kv4_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -211,10 +211,12 @@ void orc_quant_int8(const float* x, int D, int8_t* codes8, uint16_t* scale) {
  * Side cache of one layer: max_seqs slots x Hkv heads x ceil((s+w)/16) tile blocks of
  * 16*(2D+4) bytes; side row R lives in tile R/16, row r = R % 16:
  *   [0, 16D)         K int8 codes, row r at r*D, 16-byte unit u stored at unit u ^ (r & 1).
- *   [16D, 32D)       V int8 codes, rows 2p and 2p+1 interleaved byte by byte per pair of
+ *   [16D, 16D+32)    K fp16 scales, row r at 2r.
+ *   [16D+32, 32D+32) V int8 codes, rows 2p and 2p+1 interleaved byte by byte per pair of
  *                    elements, grouped like the INT4 V codes (16-byte halves swapped for odd
  *                    groups when a group is 32 bytes).
- *   [32D, 32D+32)    K fp16 scales, row r at 2r.   [32D+32, 32D+64)  V fp16 scales.
+ *   [32D+32, 32D+64) V fp16 scales, row r at 2r.
+ *   (so a tile is two equal halves, K then V, of 16D + 32 bytes each)
  * The pages leave the layout free ("token-wise INT4 ... without changing the tensor layout"
  * in [SAW-INT4 s2] refers to the paged buffers, which stay paged here).
  */
@@ -272,12 +274,12 @@ size_t orc_v8_byte(const orc_config* c, int slot, int g, int row, int e) {
   const int gq = e / dg, dd = e % dg;
   int b = (dd / 2) * 4 + (dd % 2) * 2 + (r & 1);
   if (ch8 >= 32) b ^= 16 * (gq & 1);
-  return tile8_base(c, slot, g, row) + (size_t)(16 * D + ((half * 8 + gq) * 4 + pl) * ch8 + b);
+  return tile8_base(c, slot, g, row) + (size_t)(16 * D + 32 + ((half * 8 + gq) * 4 + pl) * ch8 + b);
 }
 
 size_t orc_s8_byte(const orc_config* c, int slot, int g, int row, int is_v) {
   const int D = c->head_dim, r = row % 16;
-  return tile8_base(c, slot, g, row) + (size_t)(32 * D + 32 * is_v + 2 * r);
+  return tile8_base(c, slot, g, row) + (size_t)(16 * D + is_v * (16 * D + 32) + 2 * r);
 }
 
 int orc_side_row(const orc_config* c, int pos) {

@@ -363,7 +363,7 @@ def _brute_layout_decode(wl: W.Workload, pool, side, b: int, g: int, L: int):
             row = j if j < s else s + j % w
             base = (b * Hkv + g) * ntiles8 * tile8 + (row // 16) * tile8
             r = row % 16
-            ks, vs = f16(side, base + 32 * D + 2 * r), f16(side, base + 32 * D + 32 + 2 * r)
+            ks, vs = f16(side, base + 16 * D + 2 * r), f16(side, base + 32 * D + 32 + 2 * r)
             for e in range(D):
                 kb = base + r * D + 16 * ((e // 16) ^ (r & 1)) + e % 16
                 kh[j, e] = ks * np.int8(side[kb])
@@ -373,7 +373,7 @@ def _brute_layout_decode(wl: W.Workload, pool, side, b: int, g: int, L: int):
                 bb = (dd // 2) * 4 + (dd % 2) * 2 + (r & 1)
                 if ch8 >= 32:
                     bb ^= 16 * (gq & 1)
-                vb = base + 16 * D + ((half * 8 + gq) * 4 + pl) * ch8 + bb
+                vb = base + 16 * D + 32 + ((half * 8 + gq) * 4 + pl) * ch8 + bb
                 vh[j, e] = vs * np.int8(side[vb])
         else:
             page = wl.page_table[b, j // P]

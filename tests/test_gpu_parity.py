@@ -1,0 +1,191 @@
+"""GPU (C ABI) against the CPU oracle on the same seeded inputs.
+
+Append: the page pool and side cache bytes written by kv4_append equal the oracle's byte for
+byte (codes, fp16 scale/zero bits, INT8 routing, untouched bytes keep the 0xA5 fill).
+Decode: kv4_decode_attn output within max-abs 2e-3 and relative-L2 1e-3 of the fp64 oracle on
+the same dequantised cache, lse within 1e-4.
+"""
+import numpy as np
+import pytest
+import torch
+
+from int4_kv_cache_append_b200 import workload as W
+from oracle import oracle as O
+
+import kv4_testlib as T
+
+pytestmark = pytest.mark.gpu
+
+# (name, D, Hq, Hkv, P, s, w, h, lens, k_dtype, v_dtype, q_dtype)
+CASES = [
+    ("tiny-cfg", None, None, None, None, None, None, None, None, None, None, None),
+    ("d128-g4-bf16", 128, 8, 2, 16, 4, 16, 128, (300, 37, 1, 4, 5, 20, 21, 129), W.BF16, W.BF16, W.BF16),
+    ("d128-g4-p64-h32", 128, 8, 2, 64, 4, 48, 32, (333, 64, 65, 200), W.F32, W.BF16, W.BF16),
+    ("d64-g1-h1", 64, 2, 2, 16, 2, 8, 1, (50, 17, 3), W.F32, W.F32, W.F32),
+    ("d128-g2-no-side", 128, 4, 2, 32, 0, 0, 64, (96, 33, 7), W.BF16, W.BF16, W.BF16),
+    ("d128-g4-sinks-only", 128, 4, 1, 16, 8, 0, 16, (40, 8, 3), W.F32, W.F32, W.BF16),
+    ("d64-g4-recent-only", 64, 8, 2, 16, 0, 24, 64, (90, 24, 25, 2), W.BF16, W.F32, W.F32),
+    ("d128-g4-wide-s", 128, 4, 1, 16, 19, 13, 128, (100, 19, 20, 31, 32, 33), W.BF16, W.BF16, W.BF16),
+]
+
+
+def make(case):
+    name, D, Hq, Hkv, P, s, w, h, lens, kd, vd, qd = case
+    if name == "tiny-cfg":
+        return W.tiny_cfg()
+    return W.make_workload(name, 17, 1, len(lens), Hq, Hkv, D, P, s, w, h, lambda r: list(lens), kd, vd, qd, 2, 20.0)
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+@pytest.mark.parametrize("step_by_step", [False, True], ids=["prefill", "stepwise"])
+def test_append_bit_exact(case, step_by_step):
+    wl = make(case)
+    if step_by_step and wl.lens.max() > 160:
+        wl.lens = np.minimum(wl.lens, 160).astype(np.int32)
+    gc = T.gpu_cache_from_host_inputs(wl, step_by_step=step_by_step)
+    cfg, pool, side = T.oracle_cache(wl, step_by_step=step_by_step)
+    gp, gs = gc.layer_views(0)
+    gp = gp.cpu().numpy()
+    gs = gs.cpu().numpy()
+    assert gp.size == pool.size and gs.size == side.size
+    bad = np.nonzero(gp != pool)[0]
+    assert bad.size == 0, f"page pool differs at {bad.size} bytes, first {bad[:8]}"
+    bad = np.nonzero(gs != side)[0]
+    assert bad.size == 0, f"side cache differs at {bad.size} bytes, first {bad[:8]}"
+    from int4_kv_cache_append_b200 import kv4
+    assert kv4.kv4_get_device_error() == 0
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_decode_matches_oracle(case):
+    wl = make(case)
+    gc = T.gpu_cache_from_host_inputs(wl)
+    cfg, pool, side = T.oracle_cache(wl)
+    q = wl.q_input(0)
+    ref, ref_lse = T.oracle_decode(wl, cfg, pool, side, q)
+    out, lse = T.gpu_decode(gc, wl, q)
+    T.assert_close(out, ref, lse, ref_lse, what=case[0])
+    # the regional merge equals one softmax over the whole dequantised cache
+    single, _ = T.oracle_decode(wl, cfg, pool, side, q, mode=O.SINGLE)
+    T.assert_close(out, single, what=case[0] + " vs single softmax")
+    from int4_kv_cache_append_b200 import kv4
+    assert kv4.kv4_get_device_error() == 0
+
+
+def test_decode_on_oracle_built_cache():
+    """The decode kernel alone: bytes written by the oracle, uploaded, decoded on the GPU."""
+    wl = make(CASES[1])
+    cfg, pool, side = T.oracle_cache(wl)
+    from int4_kv_cache_append_b200 import kv4
+    gc = kv4.Cache(T.geometry(wl))
+    gp, gs = gc.layer_views(0)
+    gp.copy_(torch.from_numpy(pool))
+    gs.copy_(torch.from_numpy(side))
+    q = wl.q_input(0)
+    ref, ref_lse = T.oracle_decode(wl, cfg, pool, side, q)
+    out, lse = T.gpu_decode(gc, wl, q)
+    T.assert_close(out, ref, lse, ref_lse, what="oracle-built cache")
+
+
+def test_decode_split_count_invariance():
+    """Different grid sizes (hence different split points) give the same result within tolerance."""
+    wl = W.make_workload("split", 23, 1, 3, 8, 2, 128, 16, 4, 32, 128, lambda r: [900, 517, 64],
+                         W.BF16, W.BF16, W.BF16, 4, 15.0)
+    gc = T.gpu_cache_from_host_inputs(wl)
+    cfg, pool, side = T.oracle_cache(wl)
+    q = wl.q_input(0)
+    ref, ref_lse = T.oracle_decode(wl, cfg, pool, side, q)
+    outs = []
+    for hint in (0, 1, 16, 64, 900):
+        out, lse = T.gpu_decode(gc, wl, q, max_len_hint=hint)
+        T.assert_close(out, ref, lse, ref_lse, what=f"hint {hint}")
+        outs.append(out)
+    for o in outs[1:]:
+        assert np.abs(o - outs[0]).max() <= 1e-4
+
+
+def test_page_permutation_invariance():
+    """Moving pages to other physical slots (table updated) gives bit-identical outputs."""
+    wl = make(CASES[1])
+    q = wl.q_input(0)
+    gc = T.gpu_cache_from_host_inputs(wl)
+    out1, lse1 = T.gpu_decode(gc, wl, q)
+    rng = np.random.default_rng(99)
+    perm = rng.permutation(wl.num_pages).astype(np.int32)
+    wl2 = W.Workload(**{**wl.__dict__, "page_table": np.where(wl.page_table >= 0, perm[wl.page_table], 0).astype(np.int32)})
+    gc2 = T.gpu_cache_from_host_inputs(wl2)
+    out2, lse2 = T.gpu_decode(gc2, wl2, q)
+    assert np.array_equal(out1, out2) and np.array_equal(lse1, lse2)
+
+
+def test_zero_length_and_single_token():
+    wl = W.make_workload("edge", 29, 1, 4, 8, 2, 128, 16, 4, 16, 128, lambda r: [1, 0, 2, 23],
+                         W.BF16, W.BF16, W.BF16, 2, 20.0)
+    gc = T.gpu_cache_from_host_inputs(wl)
+    cfg, pool, side = T.oracle_cache(wl)
+    q = wl.q_input(0)
+    ref, ref_lse = T.oracle_decode(wl, cfg, pool, side, q)
+    out, lse = T.gpu_decode(gc, wl, q)
+    assert np.all(out[1] == 0) and np.all(np.isneginf(lse[1]))
+    T.assert_close(out, ref, lse, ref_lse, what="edge lengths")
+    # L = 1: the output is the single (INT8) value exactly up to fp32 rounding
+    _, vd, _ = O.dequant_seq(cfg, pool, side, wl.page_table[0], 0, 1, 0)
+    assert np.abs(out[0, 0] - vd[0]).max() <= 1e-5 * max(1.0, np.abs(vd[0]).max())
+
+
+def test_out_of_range_page_sets_error_bit_without_fault():
+    """A page id outside the pool is caught by the kernels' guards: the access is skipped and
+    the device error word reports it (the process and the context stay healthy)."""
+    from int4_kv_cache_append_b200 import kv4
+    wl = make(CASES[1])
+    gc = T.gpu_cache_from_host_inputs(wl)
+    assert kv4.kv4_get_device_error() == 0
+    bad = wl.page_table.copy()
+    bad[0, 5] = wl.num_pages + 1000
+    q = T.to_dev(wl.q_input(0))
+    lens = torch.from_numpy(wl.lens).cuda()
+    gc.decode(0, q, torch.from_numpy(bad).cuda(), lens)
+    torch.cuda.synchronize()
+    assert kv4.kv4_get_device_error() & kv4.KV4_DEVERR_PAGE_RANGE
+    out, _ = T.gpu_decode(gc, wl, wl.q_input(0))
+    assert np.isfinite(out).all()
+
+
+def _bf16_reference(wl, lens, q_host):
+    """fp64 attention over bf16-rounded K/V (no rotation, no quantisation)."""
+    out = np.zeros((len(lens), wl.Hq, wl.D))
+    lse = np.zeros((len(lens), wl.Hq))
+    q = W.bf16_to_f32(q_host).astype(np.float64) if q_host.dtype == np.uint16 else q_host.astype(np.float64)
+    for b, L in enumerate(lens):
+        if L == 0:
+            lse[b] = -np.inf
+            continue
+        K, V = wl.kv_inputs(0, np.full(L, b, np.int32), np.arange(L, dtype=np.int32))
+        K = W.bf16_to_f32(K if K.dtype == np.uint16 else W.bf16_bits(K)).astype(np.float64)
+        V = W.bf16_to_f32(V if V.dtype == np.uint16 else W.bf16_bits(V)).astype(np.float64)
+        for j in range(wl.Hq):
+            g = j // wl.G
+            lg = K[:, g] @ q[b, j] / np.sqrt(wl.D)
+            p = np.exp(lg - lg.max())
+            out[b, j] = (p[:, None] * V[:, g]).sum(0) / p.sum()
+            lse[b, j] = lg.max() + np.log(p.sum())
+    return out, lse
+
+
+@pytest.mark.parametrize("case", [CASES[1], CASES[2], CASES[3]], ids=[CASES[i][0] for i in (1, 2, 3)])
+def test_bf16_baseline_matches_reference(case):
+    from int4_kv_cache_append_b200 import kv4
+    wl = make(case)
+    bc = kv4.BF16Cache(T.geometry(wl))
+    b, p = T.prefill_tokens(wl.lens)
+    K, V = wl.kv_inputs(0, b, p)
+    pt = torch.from_numpy(wl.page_table).cuda()
+    bc.append(0, T.to_dev(K), T.to_dev(V), torch.from_numpy(b).cuda(), torch.from_numpy(p).cuda(), pt)
+    q = wl.q_input(0)
+    lse = torch.empty((wl.B, wl.Hq), device="cuda")
+    out = bc.decode(0, T.to_dev(q), pt, torch.from_numpy(wl.lens).cuda(), lse=lse)
+    ref, ref_lse = _bf16_reference(wl, wl.lens, q)
+    # fp32 queries enter as bf16 hi/lo halves (about 16 bits): a looser logit tolerance applies
+    loose = q.dtype != np.uint16
+    T.assert_close(out.cpu().numpy(), ref, lse.cpu().numpy(), ref_lse, atol=2e-2 if loose else 2e-3,
+                   rel_l2=5e-3 if loose else 1e-3, lse_atol=1e-3 if loose else 1e-4, what="bf16 " + case[0])

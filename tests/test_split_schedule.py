@@ -1,0 +1,95 @@
+"""A Python model of the flattened split-K schedule of the decode kernels, checked on the CPU.
+
+The decode kernel gives warp w the tiles whose first slot lies in [w*Q, (w+1)*Q) of the
+sequence of all slots (per sequence b, per KV head g: the INT8 segment of ceil((s+w)/16) tiles
+of 2 slots, then the INT4 segment of the 16-position tiles covering [s, max(s, L-w))), writes one
+partial per (warp, segment) at index warp + segment_id, and the merge kernel reads, for each
+segment, the partials of warps floor(first_slot/Q) .. floor(last_tile_start/Q).  This model
+restates that arithmetic and checks its invariants for many length mixes and grid sizes:
+every tile processed exactly once, partial indices unique and inside the workspace, the merge
+reads exactly the partials that were written, and every bulk-copy source lies inside its buffer.
+"""
+import numpy as np
+import pytest
+
+
+def seg_info(L, s, w, nt8):
+    n8 = nt8 if L > 0 else 0
+    m_end = max(s, L - w)
+    t4a = s >> 4
+    n4 = ((m_end - 1) >> 4) - t4a + 1 if m_end > s else 0
+    return n8, n4, t4a, m_end
+
+
+def model(lens, Hkv, s, w, P, stride, W):
+    nt8 = (s + w + 15) // 16
+    cap = stride * P
+    lens = [min(max(L, 0), cap) for L in lens]
+    # every tile: (start_slot, b, g, seg, i, nslots)
+    tiles = []
+    pos = 0
+    for b, L in enumerate(lens):
+        n8, n4, t4a, m_end = seg_info(L, s, w, nt8)
+        for g in range(Hkv):
+            for i in range(n8):
+                tiles.append((pos, b, g, 0, i, 2))
+                pos += 2
+            for i in range(n4):
+                tiles.append((pos, b, g, 1, i, 1))
+                pos += 1
+    total = pos
+    Q = max(2, -(-total // W)) if total else 2
+    owner = {}
+    written = set()
+    for (start, b, g, seg, i, n) in tiles:
+        w_ = start // Q
+        assert w_ < W
+        owner[(b, g, seg, i)] = w_
+        sid = 2 * (b * Hkv + g) + seg
+        written.add((w_ + sid, b, g, seg, w_))
+    # partial indices unique and within W + 2*B*Hkv
+    idx = [x[0] for x in written]
+    assert len(idx) == len(set(idx))
+    assert all(0 <= v < W + 2 * len(lens) * Hkv for v in idx)
+    # merge ranges
+    pos = 0
+    for b, L in enumerate(lens):
+        n8, n4, t4a, m_end = seg_info(L, s, w, nt8)
+        for g in range(Hkv):
+            for seg, cnt, tc in ((0, n8, 2), (1, n4, 1)):
+                cs = pos
+                ce = cs + cnt * tc
+                pos = ce
+                if ce <= cs:
+                    continue
+                sid = 2 * (b * Hkv + g) + seg
+                readers = set(range(cs // Q, (ce - tc) // Q + 1))
+                writers = {x[4] for x in written if x[1] == b and x[2] == g and x[3] == seg}
+                assert readers == writers, (b, g, seg, readers, writers)
+        # INT4 tiles address pages inside the page-table row
+        for i in range(n4):
+            ti = t4a + i
+            assert (ti * 16) // P < stride
+            assert ti * 16 < max(L, 1) + 15
+    return total
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_schedule_invariants(seed):
+    rng = np.random.default_rng(seed)
+    B = int(rng.integers(1, 40))
+    Hkv = int(rng.choice([1, 2, 8]))
+    s = int(rng.choice([0, 1, 4, 16, 19]))
+    w = int(rng.choice([0, 8, 32, 128]))
+    P = int(rng.choice([16, 32, 64]))
+    lens = rng.integers(0, 3000, size=B).tolist()
+    if seed % 5 == 0:
+        lens = [1, 0, s, s + 1, s + w, s + w + 1][:B] + lens[6:]
+    stride = max(1, (max(lens) + P - 1) // P)
+    for W in (1, 3, 8, 37, 296, 2368):
+        model(lens, Hkv, s, w, P, stride, W)
+
+
+def test_lengths_beyond_page_table_are_clamped():
+    # a length past stride*P is clamped to it (the merge kernel also raises a device error bit)
+    model([10_000, 5], 2, 4, 32, 16, 4, 64)
