@@ -298,6 +298,18 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_bf16_kernel(const Decod
       vw0[4 * u] = y0.x; vw0[4 * u + 1] = y0.y; vw0[4 * u + 2] = y0.z; vw0[4 * u + 3] = y0.w;
       vw1[4 * u] = y1.x; vw1[4 * u + 1] = y1.y; vw1[4 * u + 2] = y1.z; vw1[4 * u + 3] = y1.w;
     }
+    if (cons.i * 16 + 16 > L) {
+      // Partial last tile: slots past L were never written and may hold NaN patterns, which a
+      // zero weight does not cancel (0 * NaN); clear those positions in the A operand.
+      const int t0 = cons.i * 16 + 2 * tig;
+      const uint32_t m0 = (t0 < L ? 0x0000ffffu : 0u) | (t0 + 1 < L ? 0xffff0000u : 0u);
+      const uint32_t m1 = (t0 + 8 < L ? 0x0000ffffu : 0u) | (t0 + 9 < L ? 0xffff0000u : 0u);
+#pragma unroll
+      for (int x = 0; x < D / 8; ++x) {
+        vw0[x] &= m0;
+        vw1[x] &= m1;
+      }
+    }
 #pragma unroll
     for (int mb = 0; mb < NKB; ++mb) mma_bf16(oacc[mb], vw0[2 * mb], vw0[2 * mb + 1], vw1[2 * mb], vw1[2 * mb + 1], b0, b1);
     __syncwarp();
@@ -362,20 +374,19 @@ __global__ void __launch_bounds__(256) merge_bf16_kernel(const DecodeArgs a) {
 
 template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
-  const size_t smem = sizeof(SmemBF<D, G>);
+  const int smem = static_cast<int>(sizeof(SmemBF<D, G>));
+  static std::atomic<uint64_t> done[3];
   cudaError_t e;
-#define KV4_BF16_LAUNCH(QT)                                                                                      \
-  e = cudaFuncSetAttribute(decode_bf16_kernel<D, G, QT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-  if (e != cudaSuccess) return e;                                                                                \
-  decode_bf16_kernel<D, G, QT><<<ctas, kWarps * 32, smem, st>>>(a)
   if (a.q_dtype == KV4_F32) {
-    KV4_BF16_LAUNCH(KV4_F32);
+    if ((e = ensure_smem_limit(decode_bf16_kernel<D, G, KV4_F32>, smem, done[0])) != cudaSuccess) return e;
+    decode_bf16_kernel<D, G, KV4_F32><<<ctas, kWarps * 32, smem, st>>>(a);
   } else if (a.q_dtype == KV4_BF16) {
-    KV4_BF16_LAUNCH(KV4_BF16);
+    if ((e = ensure_smem_limit(decode_bf16_kernel<D, G, KV4_BF16>, smem, done[1])) != cudaSuccess) return e;
+    decode_bf16_kernel<D, G, KV4_BF16><<<ctas, kWarps * 32, smem, st>>>(a);
   } else {
-    KV4_BF16_LAUNCH(KV4_F16);
+    if ((e = ensure_smem_limit(decode_bf16_kernel<D, G, KV4_F16>, smem, done[2])) != cudaSuccess) return e;
+    decode_bf16_kernel<D, G, KV4_F16><<<ctas, kWarps * 32, smem, st>>>(a);
   }
-#undef KV4_BF16_LAUNCH
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   merge_bf16_kernel<D, G><<<(a.B * a.Hq + 7) / 8, 256, 0, st>>>(a);

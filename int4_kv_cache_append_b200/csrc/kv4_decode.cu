@@ -199,6 +199,14 @@ __device__ __forceinline__ uint32_t nib2h_rt(uint32_t w, int k) {
   return nib2h<3>(w);
 }
 
+// (1 + c/16) - 1.5 = (c - 8)/16, exact in fp16: centred V codes keep the PV accumulators near
+// the size of the result instead of carrying the affine offset through every tile.
+__device__ __forceinline__ uint32_t centred(uint32_t x) {
+  __half2 v = *reinterpret_cast<const __half2*>(&x);
+  v = __hsub2(v, __halves2half2(__ushort_as_half(0x3E00), __ushort_as_half(0x3E00)));  // 1.5
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 __device__ __forceinline__ __half split_part(float x, bool lo) {
   const __half hi = __float2half_rn(x);
   return lo ? __float2half_rn(x - __half2float(hi)) : hi;
@@ -531,7 +539,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
       const float vs1 = __half2float(__ushort_as_half(vp1 & 0xffff)), vz1 = __half2float(__ushort_as_half(vp1 >> 16));
       const float pv0 = v0 ? p0 * vs0 : 0.f, pv1 = v1 ? p1 * vs1 : 0.f;
       l_part += (v0 ? p0 : 0.f) + (v1 ? p1 : 0.f);
-      beta_part += (v0 ? p0 * (vz0 - 16.f * vs0) : 0.f) + (v1 ? p1 * (vz1 - 16.f * vs1) : 0.f);
+      // v^ = z + s c = (z + 8 s) + 16 s (c - 8)/16: the MMA sees the centred codes, the
+      // per-token constant goes to the scalar sum.
+      beta_part += (v0 ? p0 * (vz0 + 8.f * vs0) : 0.f) + (v1 ? p1 * (vz1 + 8.f * vs1) : 0.f);
       uint32_t b0, b1;
       pv_fragments(pv0, pv1, b0, b1);
       uint32_t vw0[WPC], vw1[WPC];
@@ -552,8 +562,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
 #pragma unroll
       for (int mb = 0; mb < NKB; ++mb) {
         const int j = mb >> 1, k0 = 2 * (mb & 1);
-        mma_f16(oacc[mb], nib2h_rt(vw0[j], k0), nib2h_rt(vw0[j], k0 + 1), nib2h_rt(vw1[j], k0),
-                nib2h_rt(vw1[j], k0 + 1), b0, b1);
+        mma_f16(oacc[mb], centred(nib2h_rt(vw0[j], k0)), centred(nib2h_rt(vw0[j], k0 + 1)),
+                centred(nib2h_rt(vw1[j], k0)), centred(nib2h_rt(vw1[j], k0 + 1)), b0, b1);
       }
     } else if (cons.half == 0) {
       // ----------------------------------------------------------- INT8 tile, K half
@@ -703,19 +713,17 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a) {
 
 template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
-  const size_t smem = sizeof(Smem<D, G>);
+  const int smem = static_cast<int>(sizeof(Smem<D, G>));
+  static std::atomic<uint64_t> done[3];
   cudaError_t e;
   if (a.q_dtype == KV4_F32) {
-    e = cudaFuncSetAttribute(decode_int4_kernel<D, G, KV4_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F32>, smem, done[0])) != cudaSuccess) return e;
     decode_int4_kernel<D, G, KV4_F32><<<ctas, kWarps * 32, smem, st>>>(a);
   } else if (a.q_dtype == KV4_BF16) {
-    e = cudaFuncSetAttribute(decode_int4_kernel<D, G, KV4_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_BF16>, smem, done[1])) != cudaSuccess) return e;
     decode_int4_kernel<D, G, KV4_BF16><<<ctas, kWarps * 32, smem, st>>>(a);
   } else {
-    e = cudaFuncSetAttribute(decode_int4_kernel<D, G, KV4_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F16>, smem, done[2])) != cudaSuccess) return e;
     decode_int4_kernel<D, G, KV4_F16><<<ctas, kWarps * 32, smem, st>>>(a);
   }
   e = cudaGetLastError();

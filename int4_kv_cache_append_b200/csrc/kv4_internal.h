@@ -2,6 +2,8 @@
 #pragma once
 
 #include <cuda_runtime.h>
+
+#include <atomic>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -57,5 +59,19 @@ cudaError_t launch_decode_bf16(DecodeArgs a, int D, int G, int ctas, cudaStream_
 
 // Counts every kernel launch the library issues.
 void note_launches(int n);
+
+// Raise a kernel's dynamic shared-memory limit once per device (not on every launch, so that
+// launches inside a CUDA-graph capture make no attribute calls).
+template <typename Kernel>
+cudaError_t ensure_smem_limit(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 }  // namespace kv4
