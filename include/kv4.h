@@ -158,6 +158,29 @@ kv4_status kv4_bf16_decode_attn(kv4_cache* cache, int layer, int B, const void* 
                                 int max_len_hint, float* out, float* lse, void* workspace,
                                 size_t ws_bytes, void* stream);
 
+/*
+ * kv4_decode_attn_static: kv4_decode_attn for callers that cannot allocate device memory -- code
+ * running inside another runtime's memory pool that forbids foreign allocations, a serving
+ * process that reserved all device memory up front for its page pools, or a caller that has no
+ * allocator of its own to size and keep a workspace.  The method pages have no counterpart; this
+ * is a deployment variant of the same decode.
+ * The split-K partials live in a static device array of KV4_STATIC_SCRATCH_BYTES per GPU, part of
+ * the library image and held by every GPU that loads libkv4.so until the process exits.  The
+ * call allocates and frees nothing.  Arguments and results are those of kv4_decode_attn minus the
+ * workspace.  A batch whose partials exceed the array (kv4_decode_workspace_bytes(B) >
+ * KV4_STATIC_SCRATCH_BYTES; about B > 350 for 8 KV heads, head_dim 128, 4 q heads per KV head on
+ * 148 SMs) returns KV4_ERR_WORKSPACE and launches nothing.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  All calls on one GPU share the
+ * array, which keeps the last call's contents; nothing in it needs clearing (every partial the
+ * merge reads is written earlier in the same call), but calls that overlap on the GPU (different
+ * streams, or another thread) race on it and must be serialised by the caller.
+ */
+#define KV4_STATIC_SCRATCH_BYTES (16u << 20)
+kv4_status kv4_decode_attn_static(kv4_cache* cache, int layer, int B, const void* q, kv4_dtype q_dtype,
+                                  const int32_t* page_table, int stride, const int32_t* lens, int max_len_hint,
+                                  float* out, float* lse, void* stream);
+
 /* Read and clear the device error word of the current device (synchronises the device). */
 kv4_status kv4_get_device_error(uint32_t* bits);
 

@@ -261,6 +261,39 @@ kv4_status kv4_decode_attn(kv4_cache* cache, int layer, int B, const void* q, kv
                        workspace, ws_bytes, stream);
 }
 
+// No-allocation decode: the split-K partials go to this file-scope device array instead of a
+// caller workspace.  In host code the name is only a stand-in, so its device address is looked
+// up per device (cudaGetSymbolAddress, with that device current) and passed to the kernels.
+static __device__ __align__(256) unsigned char g_kv4_static_scratch[KV4_STATIC_SCRATCH_BYTES];
+static void* g_static_scratch_ptr[kMaxDevices] = {};
+
+static bool static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_static_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_kv4_static_scratch) != cudaSuccess || !p) return false;
+    g_static_scratch_ptr[dev] = p;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return true;
+}
+
+kv4_status kv4_decode_attn_static(kv4_cache* cache, int layer, int B, const void* q, kv4_dtype q_dtype,
+                                  const int32_t* page_table, int stride, const int32_t* lens, int max_len_hint,
+                                  float* out, float* lse, void* stream) {
+  if (!cache || cache->format != FMT_INT4 || B < 0 || B > cache->cfg.max_seqs) return KV4_ERR_INVALID_ARG;
+  if (B == 0) return KV4_OK;
+  int sms = 0;
+  if (!device_info(nullptr, &sms)) return KV4_ERR_CUDA;
+  if (workspace_for(cache, B, decode_ctas_full(FMT_INT4, sms)) > KV4_STATIC_SCRATCH_BYTES) return KV4_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (!static_scratch_address(&scratch)) return KV4_ERR_CUDA;
+  return decode_common(cache, FMT_INT4, layer, B, q, q_dtype, page_table, stride, lens, max_len_hint, out, lse,
+                       scratch, KV4_STATIC_SCRATCH_BYTES, stream);
+}
+
 kv4_status kv4_bf16_query_sizes(const kv4_config* cfg, size_t* page_pool_bytes) {
   const kv4_status st = check_config(cfg);
   if (st != KV4_OK) return st;

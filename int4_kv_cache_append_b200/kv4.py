@@ -26,7 +26,7 @@ KV4_DEVERR_PAGE_RANGE, KV4_DEVERR_WAIT_LIMIT, KV4_DEVERR_LENGTH = 0x1, 0x2, 0x4
 # every entry point declared in include/kv4.h
 SYMBOLS = (
     "kv4_query_sizes", "kv4_cache_init", "kv4_cache_destroy", "kv4_append", "kv4_decode_workspace_bytes",
-    "kv4_decode_attn", "kv4_bf16_query_sizes", "kv4_bf16_cache_init", "kv4_bf16_append",
+    "kv4_decode_attn", "kv4_decode_attn_static", "kv4_bf16_query_sizes", "kv4_bf16_cache_init", "kv4_bf16_append",
     "kv4_bf16_decode_workspace_bytes", "kv4_bf16_decode_attn", "kv4_get_device_error", "kv4_launch_count",
     "kv4_status_string", "kv4_version",
 )
@@ -58,6 +58,7 @@ def _load():
         "kv4_append": (I, [P, I, I, P, I, P, I, i32p, i32p, i32p, i32p, I, P]),
         "kv4_decode_workspace_bytes": (I, [P, I, ctypes.POINTER(S)]),
         "kv4_decode_attn": (I, [P, I, I, P, I, i32p, I, i32p, I, P, P, P, S, P]),
+        "kv4_decode_attn_static": (I, [P, I, I, P, I, i32p, I, i32p, I, P, P, P]),
         "kv4_bf16_query_sizes": (I, [cfgp, ctypes.POINTER(S)]),
         "kv4_bf16_cache_init": (I, [cfgp, P, ctypes.POINTER(P)]),
         "kv4_bf16_append": (I, [P, I, I, P, I, P, I, i32p, i32p, i32p, I, P]),
@@ -145,6 +146,20 @@ def kv4_decode_attn(handle, layer, B, q, q_dtype, page_table, stride, lens, max_
     _check("kv4_decode_attn", lib.kv4_decode_attn(handle, layer, B, _ptr(q), q_dtype, _ptr(page_table), stride,
                                                   _ptr(lens), max_len_hint, _ptr(out), _ptr(lse), _ptr(workspace),
                                                   ws_bytes, _stream(stream)))
+
+
+def kv4_decode_attn_static(handle, layer, B, q, q_dtype, page_table, stride, lens, max_len_hint, out, lse,
+                           stream=None):
+    """kv4_decode_attn without a workspace argument, for callers that cannot allocate device
+    memory: the split partials use the library's static per-GPU scratch array
+    (KV4_STATIC_SCRATCH_BYTES = 16 MiB); larger batches are rejected with KV4_ERR_WORKSPACE.
+    Calls that overlap on one GPU share that array and must not run concurrently."""
+    _check("kv4_decode_attn_static", lib.kv4_decode_attn_static(handle, layer, B, _ptr(q), q_dtype, _ptr(page_table),
+                                                                stride, _ptr(lens), max_len_hint, _ptr(out), _ptr(lse),
+                                                                _stream(stream)))
+
+
+KV4_STATIC_SCRATCH_BYTES = 16 << 20
 
 
 def kv4_bf16_query_sizes(cfg: kv4_config) -> int:
