@@ -96,11 +96,18 @@ size_t align16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
 int decode_ctas_full(int format, int sms) { return format == FMT_INT4 ? 2 * sms : sms; }
 
+// Workspace layout: [counters: max_seqs * Hkv uint32, padded to 256 B][split partials].  The
+// counter region does not depend on B, so one workspace serves every batch size.
+size_t counter_bytes(const kv4_cache* c) {
+  const size_t n = static_cast<size_t>(c->cfg.max_seqs) * c->cfg.num_kv_heads * sizeof(uint32_t);
+  return (n + 255) & ~static_cast<size_t>(255);
+}
+
 size_t workspace_for(const kv4_cache* c, int B, int ctas) {
   const int G = c->cfg.num_q_heads / c->cfg.num_kv_heads;
   const int warps = ctas * (c->format == FMT_INT4 ? kv4::decode_warps_per_cta() : kv4::bf16_decode_warps_per_cta());
   const size_t segs = static_cast<size_t>(B) * c->cfg.num_kv_heads * (c->format == FMT_INT4 ? 2 : 1);
-  return align16((static_cast<size_t>(warps) + segs) * G * (c->cfg.head_dim + 2) * sizeof(float));
+  return counter_bytes(c) + align16((static_cast<size_t>(warps) + segs) * G * (c->cfg.head_dim + 4) * sizeof(float));
 }
 
 kv4_status append_common(kv4_cache* c, int fmt, int layer, int T, const void* K, kv4_dtype kd, const void* V,
@@ -172,6 +179,13 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
     if (want < ctas) ctas = static_cast<int>(want);
   }
   if (ws_bytes < workspace_for(c, B, ctas)) return KV4_ERR_WORKSPACE;
+  {
+    // work units are counted in 32 bits on the device: bound the worst case (every sequence at
+    // the page-table capacity)
+    const long long tiles = (static_cast<long long>(stride) * c->cfg.page_size + 15) / 16;
+    const long long units = static_cast<long long>(B) * c->cfg.num_kv_heads * (tiles + 2LL * c->nt8);
+    if (units >= (1LL << 31)) return KV4_ERR_UNSUPPORTED;
+  }
   kv4::DecodeArgs a{};
   a.pool = c->pool + static_cast<size_t>(layer) * c->pool_layer_bytes;
   a.side = c->side ? c->side + static_cast<size_t>(layer) * c->side_layer_bytes : nullptr;
@@ -191,11 +205,16 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
   a.nt8 = c->nt8;
   a.page_bytes = c->page_bytes;
   a.side_slot_bytes = c->side_slot_bytes;
-  a.part = static_cast<float*>(ws);
+  a.counters = static_cast<unsigned int*>(ws);
+  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + counter_bytes(c));
   a.out = out;
   a.lse = lse;
   a.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->cfg.head_dim)));
   a.err = err;
+  {
+    const int tpp = c->cfg.page_size / 16;
+    a.tp_shift = pow2(tpp) ? __builtin_ctz(static_cast<unsigned>(tpp)) : -1;
+  }
   const int G = c->cfg.num_q_heads / c->cfg.num_kv_heads;
   const cudaError_t e = fmt == FMT_INT4
                             ? kv4::launch_decode_int4(a, c->cfg.head_dim, G, ctas, static_cast<cudaStream_t>(stream))
@@ -267,13 +286,16 @@ kv4_status kv4_decode_attn(kv4_cache* cache, int layer, int B, const void* q, kv
 static __device__ __align__(256) unsigned char g_kv4_static_scratch[KV4_STATIC_SCRATCH_BYTES];
 static void* g_static_scratch_ptr[kMaxDevices] = {};
 
-static bool static_scratch_address(void** out) {
+// First use on a device: look up the array's address and zero it (the merge counters at its
+// start must begin at zero; every decode returns them to zero afterwards).
+static bool static_scratch_address(void** out, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_static_scratch_ptr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_kv4_static_scratch) != cudaSuccess || !p) return false;
+    if (cudaMemsetAsync(p, 0, KV4_STATIC_SCRATCH_BYTES, stream) != cudaSuccess) return false;
     g_static_scratch_ptr[dev] = p;
   }
   *out = g_static_scratch_ptr[dev];
@@ -289,7 +311,7 @@ kv4_status kv4_decode_attn_static(kv4_cache* cache, int layer, int B, const void
   if (!device_info(nullptr, &sms)) return KV4_ERR_CUDA;
   if (workspace_for(cache, B, decode_ctas_full(FMT_INT4, sms)) > KV4_STATIC_SCRATCH_BYTES) return KV4_ERR_WORKSPACE;
   void* scratch = nullptr;
-  if (!static_scratch_address(&scratch)) return KV4_ERR_CUDA;
+  if (!static_scratch_address(&scratch, static_cast<cudaStream_t>(stream))) return KV4_ERR_CUDA;
   return decode_common(cache, FMT_INT4, layer, B, q, q_dtype, page_table, stride, lens, max_len_hint, out, lse,
                        scratch, KV4_STATIC_SCRATCH_BYTES, stream);
 }

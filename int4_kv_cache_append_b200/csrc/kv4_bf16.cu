@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_bf16_kernel(const Decod
     for (int o = 4; o < 32; o <<= 1) l += __shfl_xor_sync(FULL, l, o);
     if (tig < G) {
       const long long sid = static_cast<long long>(c.b) * a.Hkv + c.g;
-      float* p = a.part + (static_cast<size_t>(wid + sid) * G + tig) * (D + 2);
+      float* p = a.part + (static_cast<size_t>(wid + sid) * G + tig) * kPartRow<D>;
 #pragma unroll
       for (int mb = 0; mb < NKB; ++mb) {
         const int d = Gm::DG * gq + 2 * mb;
@@ -354,7 +354,7 @@ __global__ void __launch_bounds__(256) merge_bf16_kernel(const DecodeArgs a) {
     const long long cs = bstart + g * n, ce = cs + n;
     const long long sid = static_cast<long long>(b) * a.Hkv + g;
     for (long long w = cs / Q; w <= (ce - 1) / Q; ++w) {
-      const float* p = a.part + (static_cast<size_t>(w + sid) * G + hi) * (D + 2);
+      const float* p = a.part + (static_cast<size_t>(w + sid) * G + hi) * kPartRow<D>;
       const float pm = p[D], pl = p[D + 1];
       if (!(pl > 0.f)) continue;
       const float mn = fmaxf(m, pm);

@@ -9,20 +9,24 @@
 //
 // Work decomposition (flattened split-K): every (sequence b, KV head g) has an INT8 segment of
 // ceil((s+w)/16) tiles and an INT4 segment of the 16-position tiles covering [s, max(s, L-w)).
-// A tile is one or two "slots" of at most 16*(D+8) bytes: an INT4 tile is one slot, an INT8 tile
-// two (its K half and its V half).  All slots of all segments form one sequence; warp w of the
-// launch takes the tiles whose first slot lies in [w*Q, (w+1)*Q), Q = ceil(total / warps), so
-// every warp streams the same number of bytes regardless of the length mix.  A warp writes one
-// partial (o, m, l) for every segment it touches, at index w + segment_id (unique because each
-// step along the sequence advances the warp, the segment, or both), and a second kernel merges
-// the partials of each (b, q head) with the LSE rule.
+// An INT4 tile costs 1 unit (16*(D+8) bytes), an INT8 tile 2 units (about twice the bytes).  All
+// tiles of all segments form one sequence of units; warp w of the launch takes the tiles whose
+// first unit lies in [w*Q, (w+1)*Q), Q = ceil(total / warps), so every warp streams about the
+// same number of bytes whatever the length mix.  A warp writes one partial (o, m, l) for every
+// segment it touches, at index w + segment_id (unique: each step along the sequence advances the
+// warp, the segment, or both), then counts it on the (b, g) counter; the warp that brings the
+// counter to the number of partials of (b, g) merges them with the LSE rule, writes out/lse and
+// returns the counter to zero.
 //
-// Per warp: a ring of kStages shared-memory stages fed by 1-D bulk copies (cp.async.bulk, one
-// per slot, issued by lane 0 kStages-1 slots ahead, completion on an mbarrier per stage).  The
-// G query heads of the KV group and hi/lo fp16 halves of each query form the 8 columns of an
-// m16n8k16 MMA: QK^T takes 16 positions x 16 dims per MMA with the codes as the A operand
-// converted in registers; PV takes 16 dims x 16 positions with the (p * scale) hi/lo halves as
-// the B operand.  Everything else (softmax, scale/offset, rescaling) runs in fp32 registers.
+// Per warp: kStages shared-memory stages of two tile blocks each, fed by 1-D bulk copies
+// (cp.async.bulk, issued by lane 0 kStages-1 slots ahead, completion on one mbarrier per stage).
+// A slot is two INT4 tiles (32 positions) or one INT8 tile (its K half and V half).  Slot
+// descriptors (sources, 32-row validity mask, segment index, last-slot flag) are computed 16 slots
+// at a time, one slot per lane, into a small ring, so the per-slot bookkeeping is a few
+// instructions.  The G query heads of the KV group and hi/lo fp16 halves of each query form the
+// 8 columns of an m16n8k16 MMA: QK^T takes 16 positions x 16 dims per MMA with the codes as the A
+// operand converted in registers; PV takes 16 dims x 16 positions with the (p * scale) hi/lo
+// halves as the B operand.  Softmax, scale/offset and rescaling run in fp32 registers.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -35,14 +39,21 @@ namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
 constexpr int kWarps = 8;
-constexpr int kStages = 4;
+constexpr int kStages = 3;
+constexpr int kChunk = 16;  // slots per descriptor fill
+constexpr int kRing = 32;   // descriptor ring (two chunks)
 constexpr float kNegInf = -__builtin_huge_valf();
 
-// ------------------------------------------------------------------ schedule (shared with merge)
+// ------------------------------------------------------------------ schedule
+//
+// Unit positions are 32-bit: the host refuses launches whose worst-case unit count
+// B * Hkv * (2 * nt8 + stride * P / 16) reaches 2^31.
+
+typedef unsigned int u32;
 
 struct SegInfo {
-  int n8;     // INT8 tiles (each 2 slots)
-  int n4;     // INT4 tiles (each 1 slot)
+  int n8;     // INT8 tiles (2 units each)
+  int n4;     // INT4 tiles (1 unit each)
   int t4a;    // first INT4 tile (absolute 16-position tile index)
   int m_end;  // INT4 region end position
   int L;
@@ -60,38 +71,39 @@ __device__ __forceinline__ SegInfo seg_info(int L, int s, int w, int nt8) {
   return r;
 }
 
-__device__ __forceinline__ long long head_cost(const SegInfo& si) { return 2LL * si.n8 + si.n4; }
+__device__ __forceinline__ u32 head_cost(const SegInfo& si) { return 2u * si.n8 + si.n4; }
 
-__device__ __forceinline__ long long warp_incl_scan(long long v, int lane) {
+__device__ __forceinline__ u32 seq_cost(const DecodeArgs& a, int cap, int b) {
+  return static_cast<u32>(a.Hkv) * head_cost(seg_info(clamp_len(a.lens[b], cap), a.s, a.w, a.nt8));
+}
+
+__device__ __forceinline__ u32 warp_incl_scan(u32 v, int lane) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const long long t = __shfl_up_sync(FULL, v, o);
+    const u32 t = __shfl_up_sync(FULL, v, o);
     if (lane >= o) v += t;
   }
   return v;
 }
 
-// Total slot count over all sequences (every lane gets the same value).
-__device__ long long total_cost(const DecodeArgs& a, int cap, int lane) {
-  long long run = 0;
+__device__ u32 total_cost(const DecodeArgs& a, int cap, int lane) {
+  u32 run = 0;
   for (int base = 0; base < a.B; base += 32) {
     const int b = base + lane;
-    long long c = 0;
-    if (b < a.B) c = a.Hkv * head_cost(seg_info(clamp_len(a.lens[b], cap), a.s, a.w, a.nt8));
+    const u32 c = b < a.B ? seq_cost(a, cap, b) : 0u;
     run += __shfl_sync(FULL, warp_incl_scan(c, lane), 31);
   }
   return run;
 }
 
-// Sequence containing slot position c (c < total); *bstart = first slot of that sequence.
-__device__ int find_seq(const DecodeArgs& a, int cap, int lane, long long c, long long* bstart) {
-  long long run = 0;
+// Sequence containing unit c (c < total); *bstart = first unit of that sequence.
+__device__ int find_seq(const DecodeArgs& a, int cap, int lane, u32 c, u32* bstart) {
+  u32 run = 0;
   for (int base = 0; base < a.B; base += 32) {
     const int b = base + lane;
-    long long cb = 0;
-    if (b < a.B) cb = a.Hkv * head_cost(seg_info(clamp_len(a.lens[b], cap), a.s, a.w, a.nt8));
-    const long long incl = warp_incl_scan(cb, lane);
-    const long long tot = __shfl_sync(FULL, incl, 31);
+    const u32 cb = b < a.B ? seq_cost(a, cap, b) : 0u;
+    const u32 incl = warp_incl_scan(cb, lane);
+    const u32 tot = __shfl_sync(FULL, incl, 31);
     if (c < run + tot) {
       const unsigned m = __ballot_sync(FULL, c < run + incl);
       const int l = __ffs(m) - 1;
@@ -104,26 +116,30 @@ __device__ int find_seq(const DecodeArgs& a, int cap, int lane, long long c, lon
   return a.B;
 }
 
-__device__ __forceinline__ long long quota(long long total, int W) {
-  long long q = (total + W - 1) / W;
-  return q < 2 ? 2 : q;
-}
+// Division by a per-launch constant d >= 2 for n < 2^31: q = umulhi(n, ceil(2^32 / d)) is
+// floor(n / d) or one more; one multiply-compare fixes it.
+struct FastDiv {
+  u32 d, m;
+  __device__ explicit FastDiv(u32 dd) : d(dd), m(static_cast<u32>(((1ull << 32) + dd - 1) / dd)) {}
+  __device__ __forceinline__ u32 div(u32 n) const {
+    u32 q = __umulhi(n, m);
+    if (q * d > n) --q;
+    return q;
+  }
+};
 
-// ------------------------------------------------------------------ slot cursor
-
+// Position in the tile sequence (warp-uniform): tile i of segment seg of (b, g).
 struct Cursor {
-  int b, g, seg;        // seg 0 = INT8 region, 1 = INT4 region
-  int i;                // tile index within the segment
-  int half;             // INT8 tiles: 0 = K half, 1 = V half
-  int n;                // tiles in the segment
-  long long cost;       // slot position
+  int b, g, seg;  // seg 0 = INT8 region, 1 = INT4 region
+  int i;          // tile index within the segment
+  int n;          // tiles in the segment
+  u32 cost;       // first unit of tile i
+  u32 cs8;        // first unit of the INT8 segment of (b, g)
   SegInfo si;
   bool valid;
 };
 
-__device__ __forceinline__ long long tile_start(const Cursor& c) { return c.seg == 0 ? c.cost - c.half : c.cost; }
-
-// Move to the next non-empty segment starting at (b, g, seg) (inclusive).
+// Move forward to the first non-empty segment at or after the current one.
 __device__ void settle(const DecodeArgs& a, int cap, Cursor& c) {
   while (true) {
     if (c.b >= a.B) {
@@ -133,11 +149,11 @@ __device__ void settle(const DecodeArgs& a, int cap, Cursor& c) {
     c.n = c.seg == 0 ? c.si.n8 : c.si.n4;
     if (c.i < c.n) return;
     c.i = 0;
-    c.half = 0;
     if (c.seg == 0) {
       c.seg = 1;
     } else {
       c.seg = 0;
+      c.cs8 += head_cost(c.si);
       if (++c.g == a.Hkv) {
         c.g = 0;
         if (++c.b < a.B) c.si = seg_info(clamp_len(a.lens[c.b], cap), a.s, a.w, a.nt8);
@@ -146,51 +162,187 @@ __device__ void settle(const DecodeArgs& a, int cap, Cursor& c) {
   }
 }
 
-__device__ __forceinline__ void advance(const DecodeArgs& a, int cap, Cursor& c) {
-  c.cost += 1;
-  if (c.seg == 0 && c.half == 0) {
-    c.half = 1;
-    return;
-  }
-  c.half = 0;
-  c.i += 1;
-  settle(a, cap, c);
+// Unit position of the cursor's tile (after settle moved it to another segment).
+__device__ __forceinline__ void recost(Cursor& c) {
+  c.cost = c.seg == 0 ? c.cs8 + 2u * c.i : c.cs8 + 2u * c.si.n8 + c.i;
 }
 
-// First slot of the first tile whose start is >= c0.
-__device__ Cursor cursor_at(const DecodeArgs& a, int cap, int lane, long long c0) {
+// First tile whose first unit is >= c0, in sequence b (first unit bstart).
+__device__ Cursor cursor_at(const DecodeArgs& a, int cap, int b, u32 bstart, u32 c0) {
   Cursor c;
-  long long bstart;
-  c.b = find_seq(a, cap, lane, c0, &bstart);
-  c.valid = c.b < a.B;
+  c.b = b;
+  c.valid = b < a.B;
   if (!c.valid) return c;
-  c.si = seg_info(clamp_len(a.lens[c.b], cap), a.s, a.w, a.nt8);
-  const long long ch = head_cost(c.si);
-  const long long off = c0 - bstart;
+  c.si = seg_info(clamp_len(a.lens[b], cap), a.s, a.w, a.nt8);
+  const u32 ch = head_cost(c.si);
+  const u32 off = c0 - bstart;
   c.g = static_cast<int>(off / ch);
-  const long long r = off - c.g * ch;
-  c.half = 0;
-  if (r < 2LL * c.si.n8) {
+  c.cs8 = bstart + static_cast<u32>(c.g) * ch;
+  const u32 r = off - static_cast<u32>(c.g) * ch;
+  if (r < 2u * c.si.n8) {
     c.seg = 0;
     c.i = static_cast<int>((r + 1) >> 1);
-    c.cost = c0 + (r & 1);
   } else {
     c.seg = 1;
-    c.i = static_cast<int>(r - 2LL * c.si.n8);
-    c.cost = c0;
+    c.i = static_cast<int>(r - 2u * c.si.n8);
   }
   settle(a, cap, c);
+  if (c.valid) recost(c);
   return c;
 }
 
-// ------------------------------------------------------------------ the partial kernel
+// Page-table column and tile-in-page of absolute tile ti (16 positions each).
+__device__ __forceinline__ void tile_page(const DecodeArgs& a, int ti, int* lp, int* tin) {
+  if (a.tp_shift >= 0) {
+    *lp = ti >> a.tp_shift;
+    *tin = ti & ((1 << a.tp_shift) - 1);
+  } else {
+    *lp = (ti * 16) / a.P;
+    *tin = ti - *lp * (a.P >> 4);
+  }
+}
 
-template <int D, int G>
+// ------------------------------------------------------------------ per-warp shared memory
+
+template <int D>
 struct Smem {
-  uint8_t ring[kWarps][kStages][Geo<D>::T4B];
-  float qbuf[kWarps][G][D];
+  uint8_t ring[kWarps][kStages][2 * Geo<D>::T4B];  // stage = two tile blocks
+  unsigned long long src[kWarps][kRing][2];          // bulk-copy sources of each slot (0 = none)
+  unsigned int mask[kWarps][kRing];                  // valid rows: tile A bits 0-15, tile B 16-31
+  unsigned int meta[kWarps][kRing];                  // kind | flags | segment index << 8
+  unsigned long long seg[kWarps][kRing];             // segment table: cs8 | seg<<32 | g<<33 | b<<41
   uint64_t bar[kWarps][kStages];
 };
+
+// slot meta word
+constexpr unsigned kKindInt4 = 0u, kKindInt8 = 1u, kKindNone = 2u;
+constexpr unsigned kMetaLast = 4u;  // last slot of its segment in this warp's stream
+constexpr unsigned kMetaTwo = 8u;   // INT4 slot with a second tile
+constexpr unsigned kMetaBad = 16u;  // a page id outside the pool (tile skipped)
+__device__ __forceinline__ unsigned meta_kind(unsigned m) { return m & 3u; }
+__device__ __forceinline__ unsigned meta_seg(unsigned m) { return (m >> 8) & (kRing - 1); }
+
+__device__ __forceinline__ unsigned long long pack_seg(int b, int g, int seg, u32 cs8) {
+  return static_cast<unsigned long long>(cs8) | (static_cast<unsigned long long>(seg) << 32) |
+         (static_cast<unsigned long long>(g) << 33) | (static_cast<unsigned long long>(b) << 41);
+}
+__device__ __forceinline__ u32 seg_cs8(unsigned long long e) { return static_cast<u32>(e); }
+__device__ __forceinline__ int seg_kind(unsigned long long e) { return static_cast<int>((e >> 32) & 1ull); }
+__device__ __forceinline__ int seg_g(unsigned long long e) { return static_cast<int>((e >> 33) & 255ull); }
+__device__ __forceinline__ int seg_b(unsigned long long e) { return static_cast<int>(e >> 41); }
+
+// Bits r (0..15) of the 16 rows starting at t0 whose index lies in [lo, hi).
+__device__ __forceinline__ unsigned range_bits(int lo, int hi, int t0) {
+  const int l = min(max(lo - t0, 0), 16), h = min(max(hi - t0, 0), 16);
+  return h > l ? (((1u << h) - 1u) & ~((1u << l) - 1u)) : 0u;
+}
+
+// Valid side rows of INT8 tile i for a sequence of length L: sink rows R < min(s, L); ring row
+// s + idx holds the recent position j in [max(s, L - w), L) with j mod w = idx, i.e. the cyclic
+// interval of idx starting at s mod w of length min(L - s, w); rows past s + w are padding.
+__device__ __forceinline__ unsigned side_tile_mask(int i, int L, int s, int w) {
+  const int t0 = 16 * i;
+  unsigned m = range_bits(0, min(s, L), t0);
+  if (L > s && w > 0) {
+    const int n = min(L - s, w);
+    if (n == w) {
+      m |= range_bits(s, s + w, t0);
+    } else {
+      const int a0 = s % w;
+      m |= range_bits(s + a0, s + min(w, a0 + n), t0);
+      if (a0 + n > w) m |= range_bits(s, s + (a0 + n - w), t0);
+    }
+  }
+  return m;
+}
+
+// Descriptors of the kChunk slots that follow cursor `c` (lane j < kChunk takes slot base + j),
+// written to ring position (base + j) % kRing, plus one segment-table entry per segment entered.
+// `c` is advanced past them; slots past the warp's stream get kind None.  `segno` counts the
+// segments this warp has entered.
+template <int D>
+__device__ void fill_descriptors(const DecodeArgs& a, int cap, u32 c1, Cursor& c, int lane,
+                                 Smem<D>& sm, int warp, int base, unsigned& segno) {
+  using Gm = Geo<D>;
+  unsigned long long s0 = 0ull, s1 = 0ull;
+  unsigned msk = 0u, meta = kKindNone;
+  int done = 0;
+  while (done < kChunk && c.valid && c.cost < c1) {
+    const unsigned sidx = segno & (kRing - 1);
+    if (lane == 0) sm.seg[warp][sidx] = pack_seg(c.b, c.g, c.seg, c.cs8);
+    int avail_tiles, avail_slots;
+    if (c.seg == 1) {
+      avail_tiles = static_cast<int>(min(static_cast<u32>(c.n - c.i), c1 - c.cost));
+      avail_slots = (avail_tiles + 1) >> 1;
+    } else {
+      avail_tiles = static_cast<int>(min(static_cast<u32>(c.n - c.i), (c1 - c.cost + 1) >> 1));
+      avail_slots = avail_tiles;
+    }
+    const int take = min(kChunk - done, avail_slots);
+    const int u = lane - done;
+    if (u >= 0 && u < take) {
+      meta = (sidx << 8) | ((take == avail_slots && u == take - 1) ? kMetaLast : 0u);
+      if (c.seg == 1) {
+        meta |= kKindInt4;
+        const int t0 = c.i + 2 * u;
+        const int nt = min(2, avail_tiles - 2 * u);
+        if (nt == 2) meta |= kMetaTwo;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (j < nt) {
+            const int ti = c.si.t4a + t0 + j;
+            int lp, tin;
+            tile_page(a, ti, &lp, &tin);
+            const int page = a.page_table[static_cast<size_t>(c.b) * a.stride + lp];
+            unsigned long long addr = 0ull;
+            if (page >= 0 && page < a.max_pages) {
+              addr = reinterpret_cast<unsigned long long>(a.pool + static_cast<size_t>(page) * a.page_bytes +
+                                                          static_cast<size_t>(c.g) * a.P * (D + 8) +
+                                                          static_cast<size_t>(tin) * Gm::T4B);
+              msk |= range_bits(a.s, c.si.m_end, 16 * ti) << (16 * j);
+            } else {
+              meta |= kMetaBad;
+            }
+            if (j == 0) s0 = addr; else s1 = addr;
+          }
+        }
+      } else {
+        meta |= kKindInt8;
+        const int ti = c.i + u;
+        s0 = reinterpret_cast<unsigned long long>(a.side + static_cast<size_t>(c.b) * a.side_slot_bytes +
+                                                  static_cast<size_t>(c.g) * a.nt8 * Gm::T8B +
+                                                  static_cast<size_t>(ti) * Gm::T8B);
+        s1 = s0 + Gm::H8B;
+        msk = side_tile_mask(ti, c.si.L, a.s, a.w);
+      }
+    }
+    // advance the cursor past the taken slots; at the end of the segment move to the next one.
+    // If the stream limit c1 cut the segment, the next tile starts at or past c1.
+    if (c.seg == 1) {
+      const int tiles = min(2 * take, avail_tiles);
+      c.i += tiles;
+      c.cost += static_cast<u32>(tiles);
+    } else {
+      c.i += take;
+      c.cost += 2u * take;
+    }
+    done += take;
+    if (c.i >= c.n) {
+      settle(a, cap, c);
+      ++segno;
+      if (c.valid) recost(c);
+    }
+  }
+  if (lane < kChunk) {
+    const int p = (base + lane) % kRing;
+    sm.src[warp][p][0] = s0;
+    sm.src[warp][p][1] = s1;
+    sm.mask[warp][p] = msk;
+    sm.meta[warp][p] = meta;
+  }
+}
+
+// ------------------------------------------------------------------ conversions
 
 __device__ __forceinline__ uint32_t nib2h_rt(uint32_t w, int k) {
   if (k == 0) return nib2h<0>(w);
@@ -199,17 +351,30 @@ __device__ __forceinline__ uint32_t nib2h_rt(uint32_t w, int k) {
   return nib2h<3>(w);
 }
 
-// (1 + c/16) - 1.5 = (c - 8)/16, exact in fp16: centred V codes keep the PV accumulators near
-// the size of the result instead of carrying the affine offset through every tile.
-__device__ __forceinline__ uint32_t centred(uint32_t x) {
-  __half2 v = *reinterpret_cast<const __half2*>(&x);
-  v = __hsub2(v, __halves2half2(__ushort_as_half(0x3E00), __ushort_as_half(0x3E00)));  // 1.5
+// V codes for the PV A operand: nibble k of each 16-bit half of word w (k = 0, 1 from w, k = 2, 3
+// from w >> 8) becomes the exact fp16 (c - 8) (even k) or 16 (c - 8) (odd k).  The factor 16 of
+// odd k is removed from the corresponding output rows at the end.
+template <int K>
+__device__ __forceinline__ uint32_t vcode(uint32_t w, uint32_t w8) {
+  const uint32_t src = K < 2 ? w : w8;
+  const uint32_t mask = (K & 1) ? 0x00F000F0u : 0x000F000Fu;
+  const uint32_t h = (src & mask) | 0x64006400u;
+  __half2 v = *reinterpret_cast<const __half2*>(&h);
+  const unsigned short off = (K & 1) ? 0x6480 : 0x6408;  // 1152 = 1024 + 16*8 or 1032 = 1024 + 8
+  v = __hsub2(v, __halves2half2(__ushort_as_half(off), __ushort_as_half(off)));
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ __half split_part(float x, bool lo) {
-  const __half hi = __float2half_rn(x);
-  return lo ? __float2half_rn(x - __half2float(hi)) : hi;
+// This lane's part of two fp32 values as an fp16 pair: the value truncated to 11 significant bits
+// (hi lanes) or the exact remainder rounded to fp16 (lo lanes); hi + lo carries ~22 bits.
+__device__ __forceinline__ uint32_t split_pair(float x0, float x1, bool lo) {
+  const float t0 = __uint_as_float(__float_as_uint(x0) & 0xFFFFE000u);
+  const float t1 = __uint_as_float(__float_as_uint(x1) & 0xFFFFE000u);
+  const float y0 = lo ? x0 - t0 : t0;
+  const float y1 = lo ? x1 - t1 : t1;
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(y1), "f"(y0));
+  return r;
 }
 
 __device__ __forceinline__ float exp2_fast(float x) {
@@ -218,38 +383,58 @@ __device__ __forceinline__ float exp2_fast(float x) {
   return y;
 }
 
-// Valid side rows for a sequence of length L: sink rows R < min(s, L); ring row s + i holds
-// the recent position j in [max(s, L-w), L) with j mod w = i.
-__device__ __forceinline__ bool side_row_valid(int R, int L, int s, int w) {
-  if (R < s) return R < L;
-  if (R >= s + w || L <= s) return false;
-  const int n = L - s;
-  if (n >= w) return true;
-  const int i = R - s;
-  int d = (i - s) % w;
-  if (d < 0) d += w;
-  return d < n;
-}
-
-template <int D, int G, int QT>
+template <int QT>
 __device__ __forceinline__ float load_q(const void* q, size_t i) {
   if constexpr (QT == KV4_F32) return reinterpret_cast<const float*>(q)[i];
   else if constexpr (QT == KV4_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(q)[i]);
   else return __half2float(reinterpret_cast<const __half*>(q)[i]);
 }
 
+__device__ __forceinline__ float half_lo(uint32_t w) { return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu))); }
+__device__ __forceinline__ float half_hi(uint32_t w) { return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16))); }
+
+template <int WPC>
+__device__ __forceinline__ void lds_words(const uint8_t* p, uint32_t (&w)[WPC]) {
+  if constexpr (WPC == 4) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    w[0] = u.x;
+    w[1] = u.y;
+    w[2] = u.z;
+    w[3] = u.w;
+  } else {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    w[0] = u.x;
+    w[1] = u.y;
+  }
+}
+
+// ------------------------------------------------------------------ the decode kernel
+
 template <int D, int G, int QT>
 __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const DecodeArgs a) {
   using Gm = Geo<D>;
   constexpr int NKB = Gm::NKB;
   constexpr int WPC = Gm::WPC;
+  constexpr int T4B = Gm::T4B;
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  Smem<D, G>& sm = *reinterpret_cast<Smem<D, G>*>(smem_raw);
+  Smem<D>& sm = *reinterpret_cast<Smem<D>*>(smem_raw);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tig = lane & 3;
   const int wid = blockIdx.x * kWarps + warp;
   const int cap = a.stride * a.P;
+  unsigned int* counters = a.counters;
+
+  // Sequences with no positions get out = 0, lse = -inf here (nothing else touches them).
+  for (int b = wid; b < a.B; b += a.W) {
+    const int Lraw = a.lens[b];
+    if (lane == 0 && Lraw > cap) atomicOr(a.err, KV4_DEVERR_LENGTH);
+    if (clamp_len(Lraw, cap) == 0) {
+      for (int e = lane; e < a.Hq * D; e += 32) a.out[static_cast<size_t>(b) * a.Hq * D + e] = 0.f;
+      if (a.lse)
+        for (int e = lane; e < a.Hq; e += 32) a.lse[static_cast<size_t>(b) * a.Hq + e] = kNegInf;
+    }
+  }
 
   uint64_t* bars = sm.bar[warp];
   if (lane == 0) {
@@ -258,58 +443,69 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
   }
   __syncwarp();
 
-  const long long total = total_cost(a, cap, lane);
-  const long long Q = quota(total, a.W);
-  const long long c0 = static_cast<long long>(wid) * Q;
-  if (c0 >= total) return;
-  const long long c1 = c0 + Q;
+  const u32 total = total_cost(a, cap, lane);
+  const u32 Q = max(2u, (total + a.W - 1) / static_cast<u32>(a.W));
+  const FastDiv divQ(Q);
+  const unsigned long long c0l = static_cast<unsigned long long>(wid) * Q;
+  if (c0l >= total) return;
+  const u32 c0 = static_cast<u32>(c0l);
+  const u32 c1 = c0 + Q;
+  u32 bstart;
+  const int b0 = find_seq(a, cap, lane, c0, &bstart);
+  Cursor dcur = cursor_at(a, cap, b0, bstart, c0);  // descriptor cursor, one chunk ahead
+  if (!dcur.valid || dcur.cost >= c1) return;
 
-  Cursor cons = cursor_at(a, cap, lane, c0);
-  if (!cons.valid || tile_start(cons) >= c1) return;
-  Cursor prod = cons;  // lane 0 uses it
-
-  // Issue the bulk copy of one slot into stage `st`.
-  auto issue = [&](const Cursor& c, int st) {
-    const void* src = nullptr;
-    uint32_t bytes;
-    if (c.seg == 1) {
-      const int ti = c.si.t4a + c.i;
-      const int lp = (ti * 16) / a.P;
-      const int page = a.page_table[static_cast<size_t>(c.b) * a.stride + lp];
-      bytes = Gm::T4B;
-      if (page >= 0 && page < a.max_pages)
-        src = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(c.g) * a.P * (D + 8) +
-              static_cast<size_t>((ti * 16 - lp * a.P) >> 4) * Gm::T4B;
-    } else {
-      bytes = Gm::H8B;
-      src = a.side + static_cast<size_t>(c.b) * a.side_slot_bytes + static_cast<size_t>(c.g) * a.nt8 * Gm::T8B +
-            static_cast<size_t>(c.i) * Gm::T8B + static_cast<size_t>(c.half) * Gm::H8B;
-    }
-    if (src) {
-      mbar_arrive_expect_tx(&bars[st], bytes);
-      bulk_g2s(sm.ring[warp][st], src, bytes, &bars[st]);
-    } else {
-      atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
-      mbar_arrive_expect_tx(&bars[st], 0);
-    }
-  };
-
-  // ---- per-(b, g) query state
-  uint32_t qf[NKB][2];
-  float sumq = 0.f, qinv = 1.f;
-  float* qb = &sm.qbuf[warp][0][0];
-
-  auto load_query = [&](int b, int g) {
-    // Rotate each query head of the group (H/h), scale to log2 softmax units, normalise by a
-    // power of two so that the fp16 hi/lo halves stay in the normal range.
+  // Query of the first (b, g): loads issued now, consumed after the first descriptors.
+  float qx[G][4];
+  auto load_q_regs = [&](int b, int g) {
     const bool act = lane < D / 4;
 #pragma unroll
     for (int i = 0; i < G; ++i) {
       const size_t q0 = (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G + i) * D + 4 * lane;
-      float x[4] = {0.f, 0.f, 0.f, 0.f};
-      if (act)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = load_q<D, G, QT>(a.q, q0 + e);
+      for (int e = 0; e < 4; ++e) qx[i][e] = act ? load_q<QT>(a.q, q0 + e) : 0.f;
+    }
+  };
+  load_q_regs(dcur.b, dcur.g);
+
+  unsigned segno = 0;
+  fill_descriptors<D>(a, cap, c1, dcur, lane, sm, warp, 0, segno);
+  __syncwarp();
+
+  // Issue the bulk copies of slot k into stage k % kStages (lane 0).  Returns false past the end.
+  auto issue = [&](int k) {
+    const int p = k % kRing;
+    const unsigned meta = sm.meta[warp][p];
+    if (meta_kind(meta) == kKindNone) return false;
+    const int st = k % kStages;
+    const unsigned long long s0 = sm.src[warp][p][0], s1 = sm.src[warp][p][1];
+    const uint32_t nb = meta_kind(meta) == kKindInt8 ? Gm::H8B : T4B;
+    const uint32_t bytes = (s0 ? nb : 0u) + (s1 ? nb : 0u);
+    if (meta & kMetaBad) atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
+    mbar_arrive_expect_tx(&bars[st], bytes);
+    if (s0) bulk_g2s(sm.ring[warp][st], reinterpret_cast<const void*>(s0), nb, &bars[st]);
+    if (s1) bulk_g2s(sm.ring[warp][st] + T4B, reinterpret_cast<const void*>(s1), nb, &bars[st]);
+    return true;
+  };
+
+  int issued = 0;
+  if (lane == 0)
+    for (int k = 0; k < kStages - 1; ++k)
+      if (issue(k)) ++issued;
+  issued = __shfl_sync(FULL, issued, 0);
+
+  // ---- per-(b, g) query state
+  uint32_t qf[NKB][2];
+  float sumq = 0.f, qinv = 1.f;
+
+  // Rotate the G query heads held in qx (H/h), scale to log2 softmax units, normalise each head
+  // by a power of two so that its fp16 hi/lo halves stay in the normal range, and build this
+  // lane's MMA B fragments through `scratch` (a free stage buffer).
+  auto build_query = [&](float* scratch) {
+    const bool act = lane < D / 4;
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      float* x = qx[i];
       const int h = a.h;
       if (h >= 2) {
         float u = x[0], v = x[1];
@@ -352,21 +548,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
       ex = max(min(ex, 100), -100);
       const float up = __int_as_float((127 + 14 - ex) << 23);
       const float down = __int_as_float((127 - 14 + ex) << 23);
-      float ps = 0.f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        x[e] *= up;
-        const __half hi = __float2half_rn(x[e]);
-        const __half lo = __float2half_rn(x[e] - __half2float(hi));
-        ps += __half2float(hi) + __half2float(lo);
-      }
-      if (act) *reinterpret_cast<float4*>(qb + i * D + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
-#pragma unroll
-      for (int o = 16; o; o >>= 1) ps += __shfl_xor_sync(FULL, ps, o);
-      if (tig == i) {
-        sumq = ps;
-        qinv = down;
-      }
+      if (act)
+        *reinterpret_cast<float4*>(scratch + i * D + 4 * lane) = make_float4(x[0] * up, x[1] * up, x[2] * up, x[3] * up);
+      if (tig == i) qinv = down;
     }
     __syncwarp();
     const int hh = gq >> 1;
@@ -375,22 +559,26 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
     for (int kb = 0; kb < NKB; ++kb) {
       const int W = WPC * tig + (kb >> 1), k0 = 2 * (kb & 1);
       if (hh < G) {
-        const float* qh = qb + hh * D;
-        qf[kb][0] = pack_h2(split_part(qh[8 * W + k0], lo), split_part(qh[8 * W + k0 + 4], lo));
-        qf[kb][1] = pack_h2(split_part(qh[8 * W + k0 + 1], lo), split_part(qh[8 * W + k0 + 5], lo));
+        const float* qh = scratch + hh * D + 8 * W + k0;
+        qf[kb][0] = split_pair(qh[0], qh[4], lo);
+        qf[kb][1] = split_pair(qh[1], qh[5], lo);
       } else {
         qf[kb][0] = 0u;
         qf[kb][1] = 0u;
       }
     }
+    // sum over the dims of head tig of the query exactly as the tensor core holds it (hi + lo):
+    // one MMA chain against an all-ones A operand.
+    float Sq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kb = 0; kb < NKB; ++kb) mma_f16(Sq, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u, qf[kb][0], qf[kb][1]);
+    sumq = Sq[0] + Sq[1];
     __syncwarp();
   };
 
   // ---- per-segment softmax state (head tig; lane-partial l and beta)
   float oacc[NKB][4];
   float m_run, l_part, beta_part;
-  float p_keep0 = 0.f, p_keep1 = 0.f;  // INT8: probabilities carried from the K half to the V half
-  bool v_keep0 = false, v_keep1 = false;
   auto reset = [&]() {
 #pragma unroll
     for (int mb = 0; mb < NKB; ++mb) oacc[mb][0] = oacc[mb][1] = oacc[mb][2] = oacc[mb][3] = 0.f;
@@ -399,30 +587,161 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
     beta_part = 0.f;
   };
 
-  auto flush = [&](const Cursor& c) {
+  // Write the partial of the segment `se` (a segment-table entry); if it completes its (b, g),
+  // merge and write out.
+  auto flush_and_merge = [&](unsigned long long se) {
+    const int cb = seg_b(se), cg = seg_g(se), cseg = seg_kind(se);
+    const u32 cs8 = seg_cs8(se);
+    const SegInfo si = seg_info(clamp_len(a.lens[cb], cap), a.s, a.w, a.nt8);
     float l = l_part, beta = beta_part;
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       l += __shfl_xor_sync(FULL, l, o);
       beta += __shfl_xor_sync(FULL, beta, o);
     }
+    const u32 sid = 2u * static_cast<u32>(cb * a.Hkv + cg) + static_cast<u32>(cseg);
     if (tig < G) {
-      const float fV = c.seg == 1 ? 16.f : 1.f;
-      const long long sid = 2LL * (static_cast<long long>(c.b) * a.Hkv + c.g) + c.seg;
-      float* p = a.part + (static_cast<size_t>(wid + sid) * G + tig) * (D + 2);
+      // INT4: even output rows carry (c - 8), odd rows 16 (c - 8); INT8 rows carry c.
+      const float f1 = cseg == 1 ? 0.0625f : 1.f;
+      float* p = a.part + (static_cast<size_t>(wid + sid) * G + tig) * kPartRow<D>;
 #pragma unroll
       for (int mb = 0; mb < NKB; ++mb) {
         const int d = Gm::DG * gq + 2 * mb;
         *reinterpret_cast<float2*>(p + d) =
-            make_float2(fV * (oacc[mb][0] + oacc[mb][1]) + beta, fV * (oacc[mb][2] + oacc[mb][3]) + beta);
+            make_float2((oacc[mb][0] + oacc[mb][1]) + beta, f1 * (oacc[mb][2] + oacc[mb][3]) + beta);
       }
       if (gq == 0) *reinterpret_cast<float2*>(p + D) = make_float2(m_run, l);
     }
+    // partials expected for (b, g): one per warp that owns a tile of each non-empty segment
+    const u32 cs4 = cs8 + 2u * si.n8;
+    const u32 w8a = divQ.div(cs8), w4a = divQ.div(cs4);
+    const u32 n8p_ = si.n8 ? divQ.div(cs4 - 2) - w8a + 1 : 0u;
+    const u32 n4p_ = si.n4 ? divQ.div(cs4 + si.n4 - 1) - w4a + 1 : 0u;
+    const unsigned expected = n8p_ + n4p_;
+    __syncwarp();
+    unsigned prev = 0;
+    if (lane == 0) prev = atomic_add_acq_rel(&counters[cb * a.Hkv + cg], 1u);
+    prev = __shfl_sync(FULL, prev, 0);
+    if (prev + 1 != expected) return;
+    __syncwarp();
+    // merge (b, g): lane j reads (m, l) of (head j / npart, partial j % npart), up to 32 pairs at
+    // once; the weighted rows are then summed with lanes over dims.
+    const int n8p = static_cast<int>(n8p_), npart = static_cast<int>(expected);
+    const u32 sid8 = 2u * static_cast<u32>(cb * a.Hkv + cg);
+    constexpr int PER = D / 32;
+    auto row_of = [&](int j, int hh) -> unsigned long long {
+      const u32 idx = j < n8p ? (w8a + j + sid8) : (w4a + (j - n8p) + sid8 + 1);
+      return (static_cast<unsigned long long>(idx) * G + hh) * kPartRow<D>;
+    };
+    auto write_out = [&](int hd, const float (&o)[PER], float Ls, float Mx) {
+      const int jq = cg * G + hd;
+      float* out = a.out + (static_cast<size_t>(cb) * a.Hq + jq) * D + lane * PER;
+      const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+      if constexpr (PER == 4)
+        *reinterpret_cast<float4*>(out) = make_float4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
+      else
+        *reinterpret_cast<float2*>(out) = make_float2(o[0] * inv, o[1] * inv);
+      if (a.lse && lane == 0)
+        a.lse[static_cast<size_t>(cb) * a.Hq + jq] = Ls > 0.f ? (Mx + log2f(Ls)) * 0.69314718055994531f : kNegInf;
+    };
+    auto accumulate = [&](float (&o)[PER], unsigned long long rt, float wt) {
+      const float* pr = a.part + rt + lane * PER;
+      if constexpr (PER == 4) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(pr));
+        o[0] += wt * v.x;
+        o[1] += wt * v.y;
+        o[2] += wt * v.z;
+        o[3] += wt * v.w;
+      } else {
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(pr));
+        o[0] += wt * v.x;
+        o[1] += wt * v.y;
+      }
+    };
+    if (npart * G <= 32) {
+      const int hh = lane / npart, j = lane - hh * npart;
+      float pm = kNegInf, pl = 0.f;
+      unsigned long long row = 0;
+      if (hh < G) {
+        row = row_of(j, hh);
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part + row + D));
+        pm = ml.x;
+        pl = ml.y;
+      }
+      const bool ok = pl > 0.f;
+      float mx = ok ? pm : kNegInf;
+      for (int hd = 0; hd < G; ++hd) {
+        float v = (hh == hd) ? mx : kNegInf;
+#pragma unroll
+        for (int sft = 16; sft; sft >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, sft));
+        if (hh == hd) mx = v;
+      }
+      const float wj = ok ? exp2f(pm - mx) : 0.f;
+      float lsum = wj * pl;
+      for (int hd = 0; hd < G; ++hd) {
+        float v = (hh == hd) ? lsum : 0.f;
+#pragma unroll
+        for (int sft = 16; sft; sft >>= 1) v += __shfl_xor_sync(FULL, v, sft);
+        if (hh == hd) lsum = v;
+      }
+      for (int hd = 0; hd < G; ++hd) {
+        float o[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[e] = 0.f;
+        for (int t = 0; t < npart; ++t) {
+          const int srcl = hd * npart + t;
+          const float wt = __shfl_sync(FULL, wj, srcl);
+          const unsigned long long rt = __shfl_sync(FULL, row, srcl);
+          if (wt != 0.f) accumulate(o, rt, wt);
+        }
+        write_out(hd, o, __shfl_sync(FULL, lsum, hd * npart), __shfl_sync(FULL, mx, hd * npart));
+      }
+    } else {
+      for (int hh = 0; hh < G; ++hh) {
+        float M = kNegInf, Lsum = 0.f;
+        float o[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[e] = 0.f;
+        for (int base = 0; base < npart; base += 32) {
+          const int j = base + lane;
+          float pm = kNegInf, pl = 0.f;
+          unsigned long long row = 0;
+          if (j < npart) {
+            row = row_of(j, hh);
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part + row + D));
+            pm = ml.x;
+            pl = ml.y;
+          }
+          const bool ok = pl > 0.f;
+          float mx = ok ? pm : kNegInf;
+#pragma unroll
+          for (int sft = 16; sft; sft >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, sft));
+          const float Mn = fmaxf(M, mx);
+          if (Mn == kNegInf) continue;
+          const float fo = M == kNegInf ? 0.f : exp2f(M - Mn);
+          const float wj = ok ? exp2f(pm - Mn) : 0.f;
+          float lj = wj * pl;
+#pragma unroll
+          for (int sft = 16; sft; sft >>= 1) lj += __shfl_xor_sync(FULL, lj, sft);
+          Lsum = Lsum * fo + lj;
+#pragma unroll
+          for (int e = 0; e < PER; ++e) o[e] *= fo;
+          const int cnt = min(32, npart - base);
+          for (int t = 0; t < cnt; ++t) {
+            const float wt = __shfl_sync(FULL, wj, t);
+            const unsigned long long rt = __shfl_sync(FULL, row, t);
+            if (wt != 0.f) accumulate(o, rt, wt);
+          }
+          M = Mn;
+        }
+        write_out(hh, o, Lsum, M);
+      }
+    }
+    if (lane == 0) counters[cb * a.Hkv + cg] = 0u;
   };
 
-  // Softmax update for this lane's two positions (gq and gq + 8) of head tig.
-  auto softmax_step = [&](float lg0, float lg1, float& p0, float& p1) {
-    float tm = fmaxf(lg0, lg1);
+  // Running-max update for this lane's logits of head tig (NL values), then their exponentials.
+  auto softmax_update = [&](float tm) {
     tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, 4));
     tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, 8));
     tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, 16));
@@ -441,135 +760,120 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
       beta_part *= alpha;
       m_run = mn;
     }
-    const float mu = m_run == kNegInf ? 0.f : m_run;
-    p0 = exp2_fast(lg0 - mu);
-    p1 = exp2_fast(lg1 - mu);
+    return m_run == kNegInf ? 0.f : m_run;
   };
 
-  // PV for one 16-position tile: B = hi/lo halves of pv (head gq>>1 of this lane's column).
+  // PV B operand: hi/lo halves of pv for head gq>>1 of this lane's column, positions 2tig, 2tig+1
+  // (b0) and 2tig+8, 2tig+9 (b1), gathered from the lanes that computed them.
   auto pv_fragments = [&](float pv0, float pv1, uint32_t& b0, uint32_t& b1) {
     const int hh = gq >> 1;
     const bool lo = gq & 1;
-    const int src0 = 8 * tig + (hh < 4 ? hh : 0), src1 = src0 + 4;
+    const int src0 = 8 * tig + hh, src1 = src0 + 4;
     const float x0 = __shfl_sync(FULL, pv0, src0), x1 = __shfl_sync(FULL, pv0, src1);
     const float x2 = __shfl_sync(FULL, pv1, src0), x3 = __shfl_sync(FULL, pv1, src1);
     if (hh < G) {
-      b0 = pack_h2(split_part(x0, lo), split_part(x1, lo));
-      b1 = pack_h2(split_part(x2, lo), split_part(x3, lo));
+      b0 = split_pair(x0, x1, lo);
+      b1 = split_pair(x2, x3, lo);
     } else {
       b0 = b1 = 0u;
     }
   };
 
-  // ---- pipeline
-  int issued = 0;
-  long long processed = 0;
-  if (lane == 0) {
-    for (int k = 0; k < kStages - 1; ++k) {
-      if (!prod.valid || tile_start(prod) >= c1) break;
-      issue(prod, k % kStages);
-      advance(a, cap, prod);
-      ++issued;
+  // QK^T of one INT4 tile block: logits (log2 units) of rows gq and gq + 8 for head tig.
+  auto qk_int4 = [&](const uint8_t* tb, bool v0, bool v1, float& lg0, float& lg1) {
+    uint32_t kw0[WPC], kw1[WPC];
+    lds_words<WPC>(tb + gq * (D / 2) + tig * Gm::CH, kw0);
+    lds_words<WPC>(tb + (gq + 8) * (D / 2) + tig * Gm::CH, kw1);
+    float S[4] = {0.f, 0.f, 0.f, 0.f}, S2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kb = 0; kb < NKB; ++kb) {
+      const int j = kb >> 1, k0 = 2 * (kb & 1);
+      if (kb & 1)
+        mma_f16(S2, nib2h_rt(kw0[j], k0), nib2h_rt(kw1[j], k0), nib2h_rt(kw0[j], k0 + 1), nib2h_rt(kw1[j], k0 + 1),
+                qf[kb][0], qf[kb][1]);
+      else
+        mma_f16(S, nib2h_rt(kw0[j], k0), nib2h_rt(kw1[j], k0), nib2h_rt(kw0[j], k0 + 1), nib2h_rt(kw1[j], k0 + 1),
+                qf[kb][0], qf[kb][1]);
     }
-  }
-  issued = __shfl_sync(FULL, issued, 0);
+    const uint32_t kp0 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 4 * gq);
+    const uint32_t kp1 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 4 * (gq + 8));
+    const float ks0 = half_lo(kp0), kz0 = half_hi(kp0), ks1 = half_lo(kp1), kz1 = half_hi(kp1);
+    // logit = (16 s R + (z - 16 s) sum(q)) / 2^e, R = sum_d q_d (1 + c_d / 16)
+    const float R0 = (S[0] + S2[0]) + (S[1] + S2[1]), R1 = (S[2] + S2[2]) + (S[3] + S2[3]);
+    lg0 = v0 ? (16.f * ks0 * R0 + (kz0 - 16.f * ks0) * sumq) * qinv : kNegInf;
+    lg1 = v1 ? (16.f * ks1 * R1 + (kz1 - 16.f * ks1) * sumq) * qinv : kNegInf;
+  };
 
+  // PV of one INT4 tile block with probabilities p0, p1 (rows gq, gq + 8 of head tig).
+  auto pv_int4 = [&](const uint8_t* tb, bool v0, bool v1, float p0, float p1) {
+    const uint32_t vp0 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 64 + 4 * gq);
+    const uint32_t vp1 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 64 + 4 * (gq + 8));
+    const float vs0 = half_lo(vp0), vz0 = half_hi(vp0), vs1 = half_lo(vp1), vz1 = half_hi(vp1);
+    l_part += (v0 ? p0 : 0.f) + (v1 ? p1 : 0.f);
+    // v^ = z + s c = (z + 8 s) + s (c - 8): the MMA sees the centred codes, the per-position
+    // constant goes to the scalar sum.
+    beta_part += (v0 ? p0 * (vz0 + 8.f * vs0) : 0.f) + (v1 ? p1 * (vz1 + 8.f * vs1) : 0.f);
+    uint32_t b0, b1;
+    pv_fragments(v0 ? p0 * vs0 : 0.f, v1 ? p1 * vs1 : 0.f, b0, b1);
+    uint32_t vw0[WPC], vw1[WPC];
+    const uint8_t* vb = tb + 8 * D;
+    lds_words<WPC>(vb + ((0 * 8 + gq) * 4 + tig) * Gm::CH, vw0);
+    lds_words<WPC>(vb + ((1 * 8 + gq) * 4 + tig) * Gm::CH, vw1);
+#pragma unroll
+    for (int j = 0; j < WPC; ++j) {
+      const uint32_t a8 = vw0[j] >> 8, c8 = vw1[j] >> 8;
+      // m-blocks 2j (nibbles 0, 1) and 2j + 1 (nibbles 2, 3)
+      mma_f16(oacc[2 * j], vcode<0>(vw0[j], a8), vcode<1>(vw0[j], a8), vcode<0>(vw1[j], c8), vcode<1>(vw1[j], c8),
+              b0, b1);
+      mma_f16(oacc[2 * j + 1], vcode<2>(vw0[j], a8), vcode<3>(vw0[j], a8), vcode<2>(vw1[j], c8),
+              vcode<3>(vw1[j], c8), b0, b1);
+    }
+  };
+
+  // ---- main loop over this warp's slots
   reset();
-  load_query(cons.b, cons.g);
+  build_query(reinterpret_cast<float*>(sm.ring[warp][kStages - 1]));  // stage kStages-1 is not in flight
+  int cur_bg;  // (b, g) whose query fragments are loaded
+  {
+    const unsigned long long se = sm.seg[warp][meta_seg(sm.meta[warp][0])];
+    cur_bg = seg_b(se) * a.Hkv + seg_g(se);
+  }
   bool failed = false;
   int k = 0;
   while (true) {
+    if ((k % kChunk) == 0) {
+      // descriptors of slots [k + kChunk, k + 2 kChunk) while this chunk is consumed
+      fill_descriptors<D>(a, cap, c1, dcur, lane, sm, warp, k + kChunk, segno);
+      __syncwarp();
+    }
     if (lane == 0) {
-      if (prod.valid && tile_start(prod) < c1) {
-        fence_proxy_async_smem();
-        issue(prod, (k + kStages - 1) % kStages);
-        advance(a, cap, prod);
-        ++issued;
-      }
+      fence_proxy_async_smem();
+      if (issue(k + kStages - 1)) ++issued;
     }
     const int st = k % kStages;
-    const bool ok = mbar_wait_bounded(&bars[st], (k / kStages) & 1, a.err);
+    const bool ok = mbar_wait_bounded(&bars[st], static_cast<uint32_t>((k / kStages) & 1), a.err);
     if (__any_sync(FULL, !ok)) {
       failed = true;
       break;
     }
     const uint8_t* buf = sm.ring[warp][st];
-    if (cons.seg == 1) {
-      // ----------------------------------------------------------- INT4 tile
-      const int ti = cons.si.t4a + cons.i;
-      const int lp = (ti * 16) / a.P;
-      const int page = a.page_table[static_cast<size_t>(cons.b) * a.stride + lp];
-      const bool page_ok = page >= 0 && page < a.max_pages;
-      const int pos0 = ti * 16 + gq, pos1 = pos0 + 8;
-      const bool v0 = page_ok && tig < G && pos0 >= a.s && pos0 < cons.si.m_end;
-      const bool v1 = page_ok && tig < G && pos1 >= a.s && pos1 < cons.si.m_end;
-      uint32_t kw0[WPC], kw1[WPC];
-      {
-        const uint8_t* k0p = buf + gq * (D / 2) + tig * Gm::CH;
-        const uint8_t* k1p = k0p + 8 * (D / 2);
-        if constexpr (WPC == 4) {
-          const uint4 u0 = *reinterpret_cast<const uint4*>(k0p), u1 = *reinterpret_cast<const uint4*>(k1p);
-          kw0[0] = u0.x; kw0[1] = u0.y; kw0[2] = u0.z; kw0[3] = u0.w;
-          kw1[0] = u1.x; kw1[1] = u1.y; kw1[2] = u1.z; kw1[3] = u1.w;
-        } else {
-          const uint2 u0 = *reinterpret_cast<const uint2*>(k0p), u1 = *reinterpret_cast<const uint2*>(k1p);
-          kw0[0] = u0.x; kw0[1] = u0.y;
-          kw1[0] = u1.x; kw1[1] = u1.y;
-        }
-      }
-      float S[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int kb = 0; kb < NKB; ++kb) {
-        const int j = kb >> 1, k0 = 2 * (kb & 1);
-        mma_f16(S, nib2h_rt(kw0[j], k0), nib2h_rt(kw1[j], k0), nib2h_rt(kw0[j], k0 + 1), nib2h_rt(kw1[j], k0 + 1),
-                qf[kb][0], qf[kb][1]);
-      }
-      const uint32_t kp0 = *reinterpret_cast<const uint32_t*>(buf + 16 * D + 4 * gq);
-      const uint32_t kp1 = *reinterpret_cast<const uint32_t*>(buf + 16 * D + 4 * (gq + 8));
-      const uint32_t vp0 = *reinterpret_cast<const uint32_t*>(buf + 16 * D + 64 + 4 * gq);
-      const uint32_t vp1 = *reinterpret_cast<const uint32_t*>(buf + 16 * D + 64 + 4 * (gq + 8));
-      const float ks0 = __half2float(__ushort_as_half(kp0 & 0xffff)), kz0 = __half2float(__ushort_as_half(kp0 >> 16));
-      const float ks1 = __half2float(__ushort_as_half(kp1 & 0xffff)), kz1 = __half2float(__ushort_as_half(kp1 >> 16));
-      // logit (log2 units) = (16 s R + (z - 16 s) sum(q)) / 2^e
-      const float lg0 = v0 ? (16.f * ks0 * (S[0] + S[1]) + (kz0 - 16.f * ks0) * sumq) * qinv : kNegInf;
-      const float lg1 = v1 ? (16.f * ks1 * (S[2] + S[3]) + (kz1 - 16.f * ks1) * sumq) * qinv : kNegInf;
-      float p0, p1;
-      softmax_step(lg0, lg1, p0, p1);
-      const float vs0 = __half2float(__ushort_as_half(vp0 & 0xffff)), vz0 = __half2float(__ushort_as_half(vp0 >> 16));
-      const float vs1 = __half2float(__ushort_as_half(vp1 & 0xffff)), vz1 = __half2float(__ushort_as_half(vp1 >> 16));
-      const float pv0 = v0 ? p0 * vs0 : 0.f, pv1 = v1 ? p1 * vs1 : 0.f;
-      l_part += (v0 ? p0 : 0.f) + (v1 ? p1 : 0.f);
-      // v^ = z + s c = (z + 8 s) + 16 s (c - 8)/16: the MMA sees the centred codes, the
-      // per-token constant goes to the scalar sum.
-      beta_part += (v0 ? p0 * (vz0 + 8.f * vs0) : 0.f) + (v1 ? p1 * (vz1 + 8.f * vs1) : 0.f);
-      uint32_t b0, b1;
-      pv_fragments(pv0, pv1, b0, b1);
-      uint32_t vw0[WPC], vw1[WPC];
-      {
-        const uint8_t* vb = buf + 8 * D;
-        const uint8_t* v0p = vb + ((0 * 8 + gq) * 4 + tig) * Gm::CH;
-        const uint8_t* v1p = vb + ((1 * 8 + gq) * 4 + tig) * Gm::CH;
-        if constexpr (WPC == 4) {
-          const uint4 u0 = *reinterpret_cast<const uint4*>(v0p), u1 = *reinterpret_cast<const uint4*>(v1p);
-          vw0[0] = u0.x; vw0[1] = u0.y; vw0[2] = u0.z; vw0[3] = u0.w;
-          vw1[0] = u1.x; vw1[1] = u1.y; vw1[2] = u1.z; vw1[3] = u1.w;
-        } else {
-          const uint2 u0 = *reinterpret_cast<const uint2*>(v0p), u1 = *reinterpret_cast<const uint2*>(v1p);
-          vw0[0] = u0.x; vw0[1] = u0.y;
-          vw1[0] = u1.x; vw1[1] = u1.y;
-        }
-      }
-#pragma unroll
-      for (int mb = 0; mb < NKB; ++mb) {
-        const int j = mb >> 1, k0 = 2 * (mb & 1);
-        mma_f16(oacc[mb], centred(nib2h_rt(vw0[j], k0)), centred(nib2h_rt(vw0[j], k0 + 1)),
-                centred(nib2h_rt(vw1[j], k0)), centred(nib2h_rt(vw1[j], k0 + 1)), b0, b1);
-      }
-    } else if (cons.half == 0) {
-      // ----------------------------------------------------------- INT8 tile, K half
-      const int R0 = cons.i * 16 + gq, R1 = R0 + 8;
-      const bool v0 = tig < G && side_row_valid(R0, cons.si.L, a.s, a.w);
-      const bool v1 = tig < G && side_row_valid(R1, cons.si.L, a.s, a.w);
+    const int p = k % kRing;
+    const unsigned meta = sm.meta[warp][p];
+    const unsigned msk = sm.mask[warp][p];
+    if (meta_kind(meta) == kKindInt4) {
+      // ----------------------------------------------------------- two INT4 tiles
+      const bool two = (meta & kMetaTwo) != 0;
+      const bool vA0 = tig < G && ((msk >> gq) & 1u), vA1 = tig < G && ((msk >> (gq + 8)) & 1u);
+      const bool vB0 = tig < G && ((msk >> (gq + 16)) & 1u), vB1 = tig < G && ((msk >> (gq + 24)) & 1u);
+      float lA0, lA1, lB0 = kNegInf, lB1 = kNegInf;
+      qk_int4(buf, vA0, vA1, lA0, lA1);
+      if (two) qk_int4(buf + T4B, vB0, vB1, lB0, lB1);
+      const float mu = softmax_update(fmaxf(fmaxf(lA0, lA1), fmaxf(lB0, lB1)));
+      pv_int4(buf, vA0, vA1, exp2_fast(lA0 - mu), exp2_fast(lA1 - mu));
+      if (two) pv_int4(buf + T4B, vB0, vB1, exp2_fast(lB0 - mu), exp2_fast(lB1 - mu));
+    } else {
+      // ----------------------------------------------------------- one INT8 tile (K half, V half)
+      const bool v0 = tig < G && ((msk >> gq) & 1u), v1 = tig < G && ((msk >> (gq + 8)) & 1u);
       constexpr int NW8 = 2 * WPC;  // int8 words per row chunk
       uint32_t kw0[NW8], kw1[NW8];
 #pragma unroll
@@ -595,24 +899,21 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
       const float ks1 = __half2float(*reinterpret_cast<const __half*>(buf + 16 * D + 2 * (gq + 8)));
       const float lg0 = v0 ? ks0 * (S[0] + S[1]) * qinv : kNegInf;
       const float lg1 = v1 ? ks1 * (S[2] + S[3]) * qinv : kNegInf;
-      softmax_step(lg0, lg1, p_keep0, p_keep1);
-      v_keep0 = v0;
-      v_keep1 = v1;
-      l_part += (v0 ? p_keep0 : 0.f) + (v1 ? p_keep1 : 0.f);
-    } else {
-      // ----------------------------------------------------------- INT8 tile, V half
-      const float vs0 = __half2float(*reinterpret_cast<const __half*>(buf + 16 * D + 2 * gq));
-      const float vs1 = __half2float(*reinterpret_cast<const __half*>(buf + 16 * D + 2 * (gq + 8)));
-      const float pv0 = v_keep0 ? p_keep0 * vs0 : 0.f, pv1 = v_keep1 ? p_keep1 * vs1 : 0.f;
+      const float mu = softmax_update(fmaxf(lg0, lg1));
+      const float p0 = exp2_fast(lg0 - mu), p1 = exp2_fast(lg1 - mu);
+      l_part += (v0 ? p0 : 0.f) + (v1 ? p1 : 0.f);
+      const uint8_t* vb = buf + T4B;  // V half
+      const float vs0 = __half2float(*reinterpret_cast<const __half*>(vb + 16 * D + 2 * gq));
+      const float vs1 = __half2float(*reinterpret_cast<const __half*>(vb + 16 * D + 2 * (gq + 8)));
       uint32_t b0, b1;
-      pv_fragments(pv0, pv1, b0, b1);
+      pv_fragments(v0 ? p0 * vs0 : 0.f, v1 ? p1 * vs1 : 0.f, b0, b1);
       constexpr int NW = Gm::CH8 / 4;  // words per pair chunk (8 or 4)
       uint32_t vw0[NW], vw1[NW];
 #pragma unroll
       for (int hv = 0; hv < NW / 4; ++hv) {
         const int phys = (Gm::CH8 >= 32) ? (hv ^ (gq & 1)) : hv;
-        const uint4 x0 = *reinterpret_cast<const uint4*>(buf + ((0 * 8 + gq) * 4 + tig) * Gm::CH8 + 16 * phys);
-        const uint4 x1 = *reinterpret_cast<const uint4*>(buf + ((1 * 8 + gq) * 4 + tig) * Gm::CH8 + 16 * phys);
+        const uint4 x0 = *reinterpret_cast<const uint4*>(vb + ((0 * 8 + gq) * 4 + tig) * Gm::CH8 + 16 * phys);
+        const uint4 x1 = *reinterpret_cast<const uint4*>(vb + ((1 * 8 + gq) * 4 + tig) * Gm::CH8 + 16 * phys);
         vw0[4 * hv] = x0.x; vw0[4 * hv + 1] = x0.y; vw0[4 * hv + 2] = x0.z; vw0[4 * hv + 3] = x0.w;
         vw1[4 * hv] = x1.x; vw1[4 * hv + 1] = x1.y; vw1[4 * hv + 2] = x1.z; vw1[4 * hv + 3] = x1.w;
       }
@@ -624,96 +925,34 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
       }
     }
     __syncwarp();
-    ++processed;
 
-    Cursor nxt = cons;
-    advance(a, cap, nxt);
-    const bool more = nxt.valid && tile_start(nxt) < c1;
-    const bool seg_change = !more || nxt.b != cons.b || nxt.g != cons.g || nxt.seg != cons.seg;
-    if (seg_change) {
-      flush(cons);
+    if (meta & kMetaLast) {
+      const unsigned long long se = sm.seg[warp][meta_seg(meta)];
+      flush_and_merge(se);
       reset();
-      if (more && (nxt.b != cons.b || nxt.g != cons.g)) load_query(nxt.b, nxt.g);
+      const unsigned nmeta = sm.meta[warp][(k + 1) % kRing];
+      if (meta_kind(nmeta) == kKindNone) break;  // end of this warp's stream
+      const unsigned long long ns = sm.seg[warp][meta_seg(nmeta)];
+      const int nbg = seg_b(ns) * a.Hkv + seg_g(ns);
+      if (nbg != cur_bg) {
+        cur_bg = nbg;
+        load_q_regs(seg_b(ns), seg_g(ns));
+        build_query(reinterpret_cast<float*>(sm.ring[warp][st]));  // this slot's stage is free now
+      }
     }
-    if (!more) break;
-    cons = nxt;
     ++k;
   }
   if (failed) {
     // A copy did not arrive in time: wait (bounded) for every copy this warp still has in
     // flight so none lands in shared memory after the CTA exits, then leave.
     issued = __shfl_sync(FULL, issued, 0);
-    for (long long j = processed; j < issued; ++j) {
-      const int st = static_cast<int>(j % kStages);
-      mbar_wait_bounded(&bars[st], static_cast<uint32_t>((j / kStages) & 1), a.err);
-    }
+    for (int j = k; j < issued; ++j) mbar_wait_bounded(&bars[j % kStages], static_cast<uint32_t>((j / kStages) & 1), a.err);
   }
-}
-
-// ------------------------------------------------------------------ merge kernel
-
-// One warp per (b, q head): LSE merge of the partials of the INT8 and INT4 segments.
-template <int D, int G>
-__global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int item = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
-  if (item >= a.B * a.Hq) return;
-  const int b = item / a.Hq, j = item - b * a.Hq;
-  const int g = j / G, hi = j - g * G;
-  const int cap = a.stride * a.P;
-  const long long total = total_cost(a, cap, lane);
-  const long long Q = quota(total, a.W);
-  long long bstart = 0;
-  // prefix of sequence b
-  {
-    long long run = 0;
-    for (int base = 0; base < b; base += 32) {
-      const int bb = base + lane;
-      long long c = 0;
-      if (bb < b) c = a.Hkv * head_cost(seg_info(clamp_len(a.lens[bb], cap), a.s, a.w, a.nt8));
-      run += __shfl_sync(FULL, warp_incl_scan(c, lane), 31);
-    }
-    bstart = run;
-  }
-  const int Lraw = a.lens[b];
-  const SegInfo si = seg_info(clamp_len(Lraw, cap), a.s, a.w, a.nt8);
-  if (lane == 0 && Lraw > cap) atomicOr(a.err, KV4_DEVERR_LENGTH);
-  const long long hstart = bstart + g * head_cost(si);
-
-  constexpr int PER = D / 32;
-  float o[PER];
-#pragma unroll
-  for (int e = 0; e < PER; ++e) o[e] = 0.f;
-  float m = kNegInf, l = 0.f;
-  for (int seg = 0; seg < 2; ++seg) {
-    const long long cs = hstart + (seg == 0 ? 0 : 2LL * si.n8);
-    const long long ce = cs + (seg == 0 ? 2LL * si.n8 : si.n4);
-    if (ce <= cs) continue;
-    const long long tc = seg == 0 ? 2 : 1;
-    const long long wf = cs / Q, wl = (ce - tc) / Q;
-    const long long sid = 2LL * (static_cast<long long>(b) * a.Hkv + g) + seg;
-    for (long long w = wf; w <= wl; ++w) {
-      const float* p = a.part + (static_cast<size_t>(w + sid) * G + hi) * (D + 2);
-      const float pm = p[D], pl = p[D + 1];
-      if (!(pl > 0.f)) continue;
-      const float mn = fmaxf(m, pm);
-      const float fo = m == kNegInf ? 0.f : exp2f(m - mn), fp = exp2f(pm - mn);
-      l = l * fo + pl * fp;
-#pragma unroll
-      for (int e = 0; e < PER; ++e) o[e] = o[e] * fo + p[lane * PER + e] * fp;
-      m = mn;
-    }
-  }
-  float* out = a.out + (static_cast<size_t>(b) * a.Hq + j) * D + lane * PER;
-  const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-  for (int e = 0; e < PER; ++e) out[e] = o[e] * inv;
-  if (a.lse && lane == 0) a.lse[static_cast<size_t>(b) * a.Hq + j] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : kNegInf;
 }
 
 template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
-  const int smem = static_cast<int>(sizeof(Smem<D, G>));
+  const int smem = static_cast<int>(sizeof(Smem<D>));
   static std::atomic<uint64_t> done[3];
   cudaError_t e;
   if (a.q_dtype == KV4_F32) {
@@ -726,10 +965,6 @@ cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
     if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F16>, smem, done[2])) != cudaSuccess) return e;
     decode_int4_kernel<D, G, KV4_F16><<<ctas, kWarps * 32, smem, st>>>(a);
   }
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const int items = a.B * a.Hq;
-  merge_kernel<D, G><<<(items + 7) / 8, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -738,13 +973,13 @@ cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
 int decode_warps_per_cta() { return kWarps; }
 
 size_t decode_smem_bytes(int D, int G) {
-  if (D == 128) return G == 4 ? sizeof(Smem<128, 4>) : G == 2 ? sizeof(Smem<128, 2>) : sizeof(Smem<128, 1>);
-  return G == 4 ? sizeof(Smem<64, 4>) : G == 2 ? sizeof(Smem<64, 2>) : sizeof(Smem<64, 1>);
+  (void)G;
+  return D == 128 ? sizeof(Smem<128>) : sizeof(Smem<64>);
 }
 
 cudaError_t launch_decode_int4(DecodeArgs a, int D, int G, int ctas, cudaStream_t st) {
   a.W = ctas * kWarps;
-  note_launches(2);
+  note_launches(1);
   if (D == 128) {
     if (G == 4) return launch_dg<128, 4>(a, ctas, st);
     if (G == 2) return launch_dg<128, 2>(a, ctas, st);

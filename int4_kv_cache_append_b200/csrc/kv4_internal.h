@@ -38,10 +38,12 @@ struct DecodeArgs {
   int B, Hq, Hkv, P, s, w, h, max_pages, nt8;
   size_t page_bytes, side_slot_bytes;
   float* part;            // split partials [num_slots][G][D + 2]
+  unsigned int* counters; // per (b, g) partial counters, zero between calls
   float* out;
   float* lse;
   float qscale;           // softmax scale in log2 units: log2(e) / sqrt(D)
   int W;                  // warps launched by the partial kernel
+  int tp_shift;           // log2(P / 16) when P / 16 is a power of two, else -1
   uint32_t* err;
 };
 

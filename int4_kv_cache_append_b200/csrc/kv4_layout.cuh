@@ -49,6 +49,11 @@ struct Geo {
   static constexpr int EPT = D / 4;           // BF16 elements per thread chunk
 };
 
+// Row of one split partial in the decode workspace: o[D] then (m, l), padded to a multiple of
+// four floats so that rows start on 16-byte boundaries.
+template <int D>
+constexpr int kPartRow = D + 4;
+
 __host__ __device__ constexpr int bf16_swz(int D, int a, int b) { return D == 128 ? ((a & 2) | (b & 1)) : (b & 1); }
 
 }  // namespace kv4

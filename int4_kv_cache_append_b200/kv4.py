@@ -253,7 +253,7 @@ class Cache:
     def workspace(self, B: int) -> torch.Tensor:
         n = kv4_decode_workspace_bytes(self.handle, B)
         if self._ws is None or self._ws.numel() < n:
-            self._ws = torch.empty(n, dtype=torch.uint8, device=self.pool.device)
+            self._ws = torch.zeros(n, dtype=torch.uint8, device=self.pool.device)  # zero once
         return self._ws
 
     def decode(self, layer, q, page_table, lens, out=None, lse=None, max_len_hint=0, workspace=None, stream=None):
@@ -294,7 +294,7 @@ class BF16Cache:
     def workspace(self, B: int) -> torch.Tensor:
         n = kv4_bf16_decode_workspace_bytes(self.handle, B)
         if self._ws is None or self._ws.numel() < n:
-            self._ws = torch.empty(n, dtype=torch.uint8, device=self.pool.device)
+            self._ws = torch.zeros(n, dtype=torch.uint8, device=self.pool.device)  # zero once
         return self._ws
 
     def decode(self, layer, q, page_table, lens, out=None, lse=None, max_len_hint=0, workspace=None, stream=None):
