@@ -64,15 +64,17 @@ def decode_sources_digest() -> str:
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per decode launch from a committed ncu summary, if taken on these sources."""
-    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on these sources.
+
+    profiles/decode_int4_traffic.txt holds lines `workload sources-digest bytes-per-launch`."""
+    p = os.path.join(ROOT, "profiles", "decode_int4_traffic.txt")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    e = d.get(workload)
-    if not e or e.get("sources") != decode_sources_digest():
-        return None
-    return e.get("traffic_bytes_per_launch")
+    for line in open(p):
+        f = line.split()
+        if len(f) == 3 and not line.startswith("#") and f[0] == workload and f[1] == decode_sources_digest():
+            return int(f[2])
+    return None
 
 
 class ClockSampler:
@@ -126,7 +128,10 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def dist_setup(args):
+def dist_setup(backend: str = "nccl"):
+    """One process per GPU under torchrun; the process group carries only the barrier and the
+    max-over-ranks timing reduction (no collective on the data path).  `gloo` is for the
+    CPU tests of this host logic."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -135,9 +140,12 @@ def dist_setup(args):
 
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
     return world, rank, local
 
 
@@ -146,9 +154,16 @@ def max_over_ranks(x: float, world: int) -> float:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, max_ms: float) -> float:
+    """Weak scaling: every rank processes the same units; the job rate is all ranks' units over the
+    slowest rank's time."""
+    return world * units_per_rank / (max_ms / 1e3)
 
 
 def barrier(world: int):
@@ -200,7 +215,7 @@ def cpu_baseline(wl, nseq: int = 16, min_seconds: float = 10.0):
         step(cores)
         reps += 1
         el = time.perf_counter() - t0
-        if el >= min_seconds or reps >= 50:
+        if el >= min_seconds or reps >= 5000:
             break
     return {"value": nseq * reps / el, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"first {nseq} of {wl.B} sequences (lengths {int(lens.min())}..{int(lens.max())}), "
@@ -214,7 +229,7 @@ def run_reference(args, world, rank):
     sys.path.insert(0, ROOT)
     from int4_kv_cache_append_b200 import workload as W
     wl = W.WORKLOADS[args.workload]()
-    nseq = 4
+    nseq = min(4, wl.B)
     step, lens = oracle_sample_setup(wl, nseq)
     cores = os.cpu_count() or 1
     for _ in range(args.warmup):
@@ -369,7 +384,7 @@ def run_kv4(args, world, rank, local):
     if err:
         raise RuntimeError(f"device error bits {err:#x} during the benchmark")
     total_ms = max_over_ranks(total_ms, world)
-    value = world * B * args.steps / (total_ms / 1e3)
+    value = whole_job_rate(B * args.steps, world, total_ms)
 
     kv_bytes = wl.kv_bytes_int4(lens)
     pt_bytes = int(4 * ((lens + wl.P - 1) // wl.P).sum())
@@ -379,7 +394,7 @@ def run_kv4(args, world, rank, local):
     achieved = alg_bytes / (dec_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": profiled_traffic(wl.name),
-            "kernel": "kv4_decode_attn (split-K partial kernel + merge kernel)",
+            "kernel": "decode_int4_kernel (kv4_decode_attn: split-K tiles + in-kernel merge, one launch)",
             "bytes_per_launch": alg_bytes, "kv_bytes_per_launch": kv_bytes, "decode_ms": round(dec_ms, 5),
             "peak_source": f"{peak_kind} MEASURED_PEAKS.json hbm_gbs" if peak_kind == "measured" else "fallback"}
     spec_frac = achieved / 8000.0
@@ -421,7 +436,7 @@ def run_kv4(args, world, rank, local):
         s1.record(stream)
         s1.synchronize()
         e2e_ms = max_over_ranks(s0.elapsed_time(s1), world)
-        e2e = {"value": world * B * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": whole_job_rate(B * args.e2e_steps, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                "path": "kv4.Cache.append + kv4.Cache.decode (C ABI) with pinned host inputs/outputs copied every step"}
 
@@ -437,11 +452,11 @@ def run_kv4(args, world, rank, local):
         b_total = max_over_ranks(b_total, world)
         bkv = wl.kv_bytes_bf16(lens)
         b_alg = bkv + pt_bytes + io_bytes
-        bf = {"value": world * B * args.steps / (b_total / 1e3), "unit": UNIT, "ms_per_step": b_total / args.steps,
+        bf = {"value": whole_job_rate(B * args.steps, world, b_total), "unit": UNIT, "ms_per_step": b_total / args.steps,
               "decode_ms": round(b_dec, 5), "kv_bytes_per_launch": bkv,
               "achieved_GBps": round(b_alg / (b_dec / 1e3) / 1e9, 1),
               "frac": round(b_alg / (b_dec / 1e3) / 1e9 / peak, 4),
-              "int4_speedup_step": round(value / (world * B * args.steps / (b_total / 1e3)), 3),
+              "int4_speedup_step": round(value / whole_job_rate(B * args.steps, world, b_total), 3),
               "int4_speedup_decode": round(b_dec / dec_ms, 3)}
         del bcache, bins
         torch.cuda.empty_cache()
@@ -467,9 +482,16 @@ def run_kv4(args, world, rank, local):
 
 def main():
     args = parse()
-    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        # the host-core oracle: rank 0 alone runs and prints; other ranks exit without work
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = run_reference(args, world, int(os.environ.get("RANK", "0")))
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, local = dist_setup("nccl")
     try:
-        line = run_reference(args, world, rank) if args.impl == "reference" else run_kv4(args, world, rank, local)
+        line = run_kv4(args, world, rank, local)
         if line is not None and rank == 0:
             print(json.dumps(line), flush=True)
     finally:

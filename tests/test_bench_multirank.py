@@ -1,0 +1,62 @@
+"""Host logic of `bench.py --gpus N` on 2 CPU ranks over gloo.
+
+Each rank runs its own batch (weak scaling); the only process-group traffic is a barrier and
+the max-over-ranks reduction of the timed region.  The reference (oracle) arm runs on rank 0
+alone.  No GPU is used.
+"""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank: int, world: int, port: int, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import argparse
+
+    import bench
+    import torch.distributed as dist
+    try:
+        w, r, _ = bench.dist_setup("gloo")
+        assert (w, r) == (world, rank)
+        bench.barrier(w)
+        ms = 10.0 + 5.0 * rank  # the slower rank decides the job time
+        mx = bench.max_over_ranks(ms, w)
+        rate = bench.whole_job_rate(64 * 100, w, mx)
+        args = argparse.Namespace(workload="tiny", steps=1, warmup=0)
+        line = bench.run_reference(args, w, r)
+        q.put((rank, mx, rate, None if line is None else (line["impl"], line["n_gpus"], line["cpu_baseline"]["kind"])))
+        dist.destroy_process_group()
+    except Exception as e:  # surface the failure to the parent
+        q.put((rank, "error", repr(e), None))
+
+
+def test_two_rank_max_timing_and_reference_on_rank0_only():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, mx, rate, ref in res:
+        assert mx != "error", rate
+        assert mx == pytest.approx(15.0)
+        assert rate == pytest.approx(2 * 64 * 100 / 0.015)
+    assert res[0][3] == ("reference", 2, "oracle")
+    assert res[1][3] is None
