@@ -344,16 +344,11 @@ __device__ void fill_descriptors(const DecodeArgs& a, int cap, u32 c1, Cursor& c
 
 // ------------------------------------------------------------------ conversions
 
-__device__ __forceinline__ uint32_t nib2h_rt(uint32_t w, int k) {
-  if (k == 0) return nib2h<0>(w);
-  if (k == 1) return nib2h<1>(w);
-  if (k == 2) return nib2h<2>(w);
-  return nib2h<3>(w);
-}
-
 // V codes for the PV A operand: nibble k of each 16-bit half of word w (k = 0, 1 from w, k = 2, 3
-// from w >> 8) becomes the exact fp16 (c - 8) (even k) or 16 (c - 8) (odd k).  The factor 16 of
-// odd k is removed from the corresponding output rows at the end.
+// from w8 = w >> 8) becomes the exact fp16 (c - 8) (even k) or 16 (c - 8) (odd k); the factor 16
+// of odd k is removed from the corresponding output rows when the partial is written.  V stays in
+// normal fp16: the (p * scale) operand is small, and subnormal codes against it lose accuracy in
+// the tensor-core accumulation over long sequences.
 template <int K>
 __device__ __forceinline__ uint32_t vcode(uint32_t w, uint32_t w8) {
   const uint32_t src = K < 2 ? w : w8;
@@ -496,7 +491,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
 
   // ---- per-(b, g) query state
   uint32_t qf[NKB][2];
-  float sumq = 0.f, qinv = 1.f;
+  float sumq = 0.f, qinv = 1.f, qinv20 = 1.f;  // sumq in units of 2^20
 
   // Rotate the G query heads held in qx (H/h), scale to log2 softmax units, normalise each head
   // by a power of two so that its fp16 hi/lo halves stay in the normal range, and build this
@@ -557,11 +552,13 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
     const bool lo = gq & 1;
 #pragma unroll
     for (int kb = 0; kb < NKB; ++kb) {
-      const int W = WPC * tig + (kb >> 1), k0 = 2 * (kb & 1);
+      // k-block kb of this lane: dims (d, d + 4) in b0 and (d + 2, d + 6) in b1 of the 8-dim group
+      // W, d = kb & 1, matching the nibble masks of the K code words in qk_int4.
+      const int W = WPC * tig + (kb >> 1);
       if (hh < G) {
-        const float* qh = scratch + hh * D + 8 * W + k0;
+        const float* qh = scratch + hh * D + 8 * W + (kb & 1);
         qf[kb][0] = split_pair(qh[0], qh[4], lo);
-        qf[kb][1] = split_pair(qh[1], qh[5], lo);
+        qf[kb][1] = split_pair(qh[2], qh[6], lo);
       } else {
         qf[kb][0] = 0u;
         qf[kb][1] = 0u;
@@ -572,7 +569,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
     float Sq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kb = 0; kb < NKB; ++kb) mma_f16(Sq, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u, qf[kb][0], qf[kb][1]);
-    sumq = Sq[0] + Sq[1];
+    sumq = (Sq[0] + Sq[1]) * 0x1p-20f;
+    qinv20 = qinv * 0x1p20f;
     __syncwarp();
   };
 
@@ -787,21 +785,23 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
     float S[4] = {0.f, 0.f, 0.f, 0.f}, S2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kb = 0; kb < NKB; ++kb) {
-      const int j = kb >> 1, k0 = 2 * (kb & 1);
+      // word j of a row holds dims 8W..8W+7, nibble n at bits 4n.  Every code is moved to bits
+      // 4-7 of its half (fp16 subnormal c * 2^-20): even kb takes dims 0, 4 (w << 4) and 2, 6
+      // (w >> 4), odd kb dims 1, 5 (w) and 3, 7 (w >> 8).
+      const int j = kb >> 1;
+      const uint32_t w0 = kw0[j], w1 = kw1[j];
       if (kb & 1)
-        mma_f16(S2, nib2h_rt(kw0[j], k0), nib2h_rt(kw1[j], k0), nib2h_rt(kw0[j], k0 + 1), nib2h_rt(kw1[j], k0 + 1),
-                qf[kb][0], qf[kb][1]);
+        mma_f16(S2, nib_hi(w0), nib_hi(w1), nib_hi(w0 >> 8), nib_hi(w1 >> 8), qf[kb][0], qf[kb][1]);
       else
-        mma_f16(S, nib2h_rt(kw0[j], k0), nib2h_rt(kw1[j], k0), nib2h_rt(kw0[j], k0 + 1), nib2h_rt(kw1[j], k0 + 1),
-                qf[kb][0], qf[kb][1]);
+        mma_f16(S, nib_hi(w0 << 4), nib_hi(w1 << 4), nib_hi(w0 >> 4), nib_hi(w1 >> 4), qf[kb][0], qf[kb][1]);
     }
     const uint32_t kp0 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 4 * gq);
     const uint32_t kp1 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 4 * (gq + 8));
     const float ks0 = half_lo(kp0), kz0 = half_hi(kp0), ks1 = half_lo(kp1), kz1 = half_hi(kp1);
-    // logit = (16 s R + (z - 16 s) sum(q)) / 2^e, R = sum_d q_d (1 + c_d / 16)
-    const float R0 = (S[0] + S2[0]) + (S[1] + S2[1]), R1 = (S[2] + S2[2]) + (S[3] + S2[3]);
-    lg0 = v0 ? (16.f * ks0 * R0 + (kz0 - 16.f * ks0) * sumq) * qinv : kNegInf;
-    lg1 = v1 ? (16.f * ks1 * R1 + (kz1 - 16.f * ks1) * sumq) * qinv : kNegInf;
+    // logit = (s q.c + z sum(q)) / 2^e with q.c = 2^20 R
+    const float R0 = (S[0] + S[1]) + (S2[0] + S2[1]), R1 = (S[2] + S[3]) + (S2[2] + S2[3]);
+    lg0 = v0 ? fmaf(ks0, R0, kz0 * sumq) * qinv20 : kNegInf;
+    lg1 = v1 ? fmaf(ks1, R1, kz1 * sumq) * qinv20 : kNegInf;
   };
 
   // PV of one INT4 tile block with probabilities p0, p1 (rows gq, gq + 8 of head tig).
@@ -890,7 +890,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
         const int j = kb >> 1;
         const uint32_t A0 = kw0[2 * j] ^ 0x80808080u, B0 = kw0[2 * j + 1] ^ 0x80808080u;
         const uint32_t A1 = kw1[2 * j] ^ 0x80808080u, B1 = kw1[2 * j + 1] ^ 0x80808080u;
-        const uint32_t sel = (kb & 1) ? 0x7362u : 0x5140u;
+        const uint32_t sel = (kb & 1) ? 0x7351u : 0x6240u;  // dims (d, d+4, d+2, d+6), d = kb & 1
         const uint32_t t0 = prmt(A0, B0, sel), t1 = prmt(A1, B1, sel);
         mma_f16(S, i8x2_to_h2<0x4140>(t0), i8x2_to_h2<0x4140>(t1), i8x2_to_h2<0x4342>(t0), i8x2_to_h2<0x4342>(t1),
                 qf[kb][0], qf[kb][1]);

@@ -118,23 +118,11 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1
 
 // ------------------------------------------------------------------ code -> fp16 conversions
 
-// Two INT4 codes of a 32-bit word, the nibbles at bits 4k and 16+4k, become the fp16 pair
-// (1 + c/16): the code is moved into the top four fraction bits of the fp16 1.0 pattern.
-// The value is exact, and the MMA result is corrected afterwards (x = 1 + c/16 means
-// c = 16 x - 16), which keeps the offset small next to the signal.
-template <int K>
-__device__ __forceinline__ uint32_t nib2h(uint32_t w) {
-  uint32_t t;
-  if constexpr (K == 0)
-    t = w << 6;
-  else if constexpr (K == 1)
-    t = w << 2;
-  else if constexpr (K == 2)
-    t = w >> 2;
-  else
-    t = w >> 6;
-  return (t & 0x03C003C0u) | 0x3C003C00u;
-}
+// The two INT4 codes at bits 4-7 and 20-23 of a word, as the fp16 pair of subnormals c * 2^-20
+// (a mask alone; exact).  The sm_100a tensor cores take subnormal fp16 operands, but measured
+// sums of such products carry errors near 2^-24 in absolute terms, so the other operand must be
+// large (the query, scaled to [2^14, 2^15)) for the products to keep full relative precision.
+__device__ __forceinline__ uint32_t nib_hi(uint32_t w) { return w & 0x00F000F0u; }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
