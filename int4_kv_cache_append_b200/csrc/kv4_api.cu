@@ -94,20 +94,25 @@ kv4_status dtype_ok_q(kv4_dtype d) {
 
 size_t align16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
-int decode_ctas_full(int format, int sms) { return format == FMT_INT4 ? 2 * sms : sms; }
+int decode_ctas_full(int format, int sms) { return format == FMT_INT4 ? kv4::decode_ctas_per_sm() * sms : sms; }
 
-// Workspace layout: [counters: max_seqs * Hkv uint32, padded to 256 B][split partials].  The
-// counter region does not depend on B, so one workspace serves every batch size.
-size_t counter_bytes(const kv4_cache* c) {
-  const size_t n = static_cast<size_t>(c->cfg.max_seqs) * c->cfg.num_kv_heads * sizeof(uint32_t);
+// Workspace layout: [counters][split partials].  Counters: max_seqs * Hkv per (sequence, KV head)
+// counters, then one per possible partial index (warps of the full grid + 2 * max_seqs * Hkv) for
+// the groups of the two-level merge; padded to 256 B.  The counter region depends only on the
+// configuration and the device, so one workspace serves every batch size and grid.
+size_t counter_bytes(const kv4_cache* c, int sms) {
+  const size_t bg = static_cast<size_t>(c->cfg.max_seqs) * c->cfg.num_kv_heads;
+  const int full_warps =
+      decode_ctas_full(c->format, sms) * (c->format == FMT_INT4 ? kv4::decode_warps_per_cta() : kv4::bf16_decode_warps_per_cta());
+  const size_t n = (bg + static_cast<size_t>(full_warps) + 2 * bg) * sizeof(uint32_t);
   return (n + 255) & ~static_cast<size_t>(255);
 }
 
-size_t workspace_for(const kv4_cache* c, int B, int ctas) {
+size_t workspace_for(const kv4_cache* c, int B, int ctas, int sms) {
   const int G = c->cfg.num_q_heads / c->cfg.num_kv_heads;
   const int warps = ctas * (c->format == FMT_INT4 ? kv4::decode_warps_per_cta() : kv4::bf16_decode_warps_per_cta());
   const size_t segs = static_cast<size_t>(B) * c->cfg.num_kv_heads * (c->format == FMT_INT4 ? 2 : 1);
-  return counter_bytes(c) + align16((static_cast<size_t>(warps) + segs) * G * (c->cfg.head_dim + 4) * sizeof(float));
+  return counter_bytes(c, sms) + align16((static_cast<size_t>(warps) + segs) * G * (c->cfg.head_dim + 4) * sizeof(float));
 }
 
 kv4_status append_common(kv4_cache* c, int fmt, int layer, int T, const void* K, kv4_dtype kd, const void* V,
@@ -178,7 +183,7 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
     if (want < 1) want = 1;
     if (want < ctas) ctas = static_cast<int>(want);
   }
-  if (ws_bytes < workspace_for(c, B, ctas)) return KV4_ERR_WORKSPACE;
+  if (ws_bytes < workspace_for(c, B, ctas, sms)) return KV4_ERR_WORKSPACE;
   {
     // work units are counted in 32 bits on the device: bound the worst case (every sequence at
     // the page-table capacity)
@@ -206,7 +211,8 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
   a.page_bytes = c->page_bytes;
   a.side_slot_bytes = c->side_slot_bytes;
   a.counters = static_cast<unsigned int*>(ws);
-  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + counter_bytes(c));
+  a.gcounters = static_cast<unsigned int*>(ws) + static_cast<size_t>(c->cfg.max_seqs) * c->cfg.num_kv_heads;
+  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + counter_bytes(c, sms));
   a.out = out;
   a.lse = lse;
   a.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->cfg.head_dim)));
@@ -269,7 +275,7 @@ kv4_status kv4_decode_workspace_bytes(const kv4_cache* cache, int B, size_t* byt
   if (!cache || cache->format != FMT_INT4 || B < 0 || !bytes) return KV4_ERR_INVALID_ARG;
   int sms = 0;
   if (!device_info(nullptr, &sms)) return KV4_ERR_CUDA;
-  *bytes = workspace_for(cache, B, decode_ctas_full(FMT_INT4, sms));
+  *bytes = workspace_for(cache, B, decode_ctas_full(FMT_INT4, sms), sms);
   return KV4_OK;
 }
 
@@ -309,7 +315,7 @@ kv4_status kv4_decode_attn_static(kv4_cache* cache, int layer, int B, const void
   if (B == 0) return KV4_OK;
   int sms = 0;
   if (!device_info(nullptr, &sms)) return KV4_ERR_CUDA;
-  if (workspace_for(cache, B, decode_ctas_full(FMT_INT4, sms)) > KV4_STATIC_SCRATCH_BYTES) return KV4_ERR_WORKSPACE;
+  if (workspace_for(cache, B, decode_ctas_full(FMT_INT4, sms), sms) > KV4_STATIC_SCRATCH_BYTES) return KV4_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (!static_scratch_address(&scratch, static_cast<cudaStream_t>(stream))) return KV4_ERR_CUDA;
   return decode_common(cache, FMT_INT4, layer, B, q, q_dtype, page_table, stride, lens, max_len_hint, out, lse,
@@ -355,7 +361,7 @@ kv4_status kv4_bf16_decode_workspace_bytes(const kv4_cache* cache, int B, size_t
   if (!cache || cache->format != FMT_BF16 || B < 0 || !bytes) return KV4_ERR_INVALID_ARG;
   int sms = 0;
   if (!device_info(nullptr, &sms)) return KV4_ERR_CUDA;
-  *bytes = workspace_for(cache, B, decode_ctas_full(FMT_BF16, sms));
+  *bytes = workspace_for(cache, B, decode_ctas_full(FMT_BF16, sms), sms);
   return KV4_OK;
 }
 

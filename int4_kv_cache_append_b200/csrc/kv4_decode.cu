@@ -30,6 +30,8 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "kv4_device.cuh"
 #include "kv4_internal.h"
 #include "kv4_layout.cuh"
@@ -38,10 +40,14 @@ namespace kv4 {
 namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
-constexpr int kWarps = 8;
-constexpr int kStages = 3;
+// One CTA of 16 warps per SM: the SM's warp schedulers favour the older of two co-resident CTAs,
+// so two 8-warp CTAs per SM finish unevenly; warps of one CTA progress at the same rate.
+constexpr int kWarps = 16;
+constexpr int kCtasPerSm = 1;
+constexpr int kStages = 2;
 constexpr int kChunk = 16;  // slots per descriptor fill
 constexpr int kRing = 32;   // descriptor ring (two chunks)
+constexpr int kGroup = 8;   // partials per group of the two-level merge
 constexpr float kNegInf = -__builtin_huge_valf();
 
 // ------------------------------------------------------------------ schedule
@@ -403,10 +409,135 @@ __device__ __forceinline__ void lds_words(const uint8_t* p, uint32_t (&w)[WPC]) 
   }
 }
 
+// ------------------------------------------------------------------ LSE merge of split partials
+
+// Where the rows of the partials of one (b, g) live: partial j (INT8-region owners first, then
+// INT4) has index w8a + j + sid8 (j < n8p) or w4a + (j - n8p) + sid8 + 1, and its G rows of
+// (o[D], m, l) start at index * G * kPartRow.
+struct PartRows {
+  int n8p;
+  u32 w8a, w4a, sid8;
+  __device__ __forceinline__ unsigned long long row(int j, int G, int stride) const {
+    const u32 idx = j < n8p ? (w8a + static_cast<u32>(j) + sid8) : (w4a + static_cast<u32>(j - n8p) + sid8 + 1u);
+    return static_cast<unsigned long long>(idx) * G * stride;
+  }
+};
+
+// LSE merge of the n partials j0, j0 + step, ... of one (b, g).  Pass 1 finds the per-head
+// maximum of m (lanes read the (m, l) of 32 (head, partial) pairs at a time).  Pass 2 walks the
+// n * G pairs head-major, 32 at a time: each lane weights one pair, exp2(m - M) and its share
+// of the per-head sum; the pairs' o rows are then read kInFlight at a time with independent
+// loads so that their latencies overlap (a pass over n rows costs about 1 + n G / kInFlight
+// round trips to L2).  dst = ~0 writes the normalised output and lse of query heads cg*G.. of
+// sequence cb; otherwise the merged rows (o, M, L) go to the rows at dst.
+template <int D, int G>
+__device__ __forceinline__ void merge_partials(float* part, float* outp, float* lsep, int Hq, int lane,
+                                               const PartRows pr, int n, int j0, int step, unsigned long long dst,
+                                               int cb, int cg) {
+  constexpr int PER = D / 32;
+  constexpr int kInFlight = 8;
+  constexpr int RS = kPartRow<D>;
+  using VecT = typename std::conditional<PER == 4, float4, float2>::type;
+  const int npairs = n * G;
+  float Mh[G], Lh[G], o[G][PER];
+#pragma unroll
+  for (int hd = 0; hd < G; ++hd) {
+    Mh[hd] = kNegInf;
+    Lh[hd] = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) o[hd][e] = 0.f;
+  }
+  for (int base = 0; base < npairs; base += 32) {
+    const int q = base + lane;
+    float v = kNegInf;
+    int hh = -1;
+    if (q < npairs) {
+      hh = q / n;
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(part + pr.row(j0 + (q - hh * n) * step, G, RS) + hh * RS + D));
+      if (ml.y > 0.f) v = ml.x;
+    }
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) {
+      float x = (hh == hd) ? v : kNegInf;
+#pragma unroll
+      for (int sft = 16; sft; sft >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, sft));
+      Mh[hd] = fmaxf(Mh[hd], x);
+    }
+  }
+  for (int base = 0; base < npairs; base += 32) {
+    const int q = base + lane;
+    float w = 0.f, wl = 0.f;
+    unsigned long long row = 0;
+    int hh = 0;
+    if (q < npairs) {
+      hh = q / n;
+      row = pr.row(j0 + (q - hh * n) * step, G, RS) + hh * RS;
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(part + row + D));
+      float mh = Mh[0];
+#pragma unroll
+      for (int hd = 1; hd < G; ++hd)
+        if (hh == hd) mh = Mh[hd];
+      if (ml.y > 0.f) {
+        w = exp2f(ml.x - mh);
+        wl = w * ml.y;
+      }
+    }
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) {
+      float x = (hh == hd) ? wl : 0.f;
+#pragma unroll
+      for (int sft = 16; sft; sft >>= 1) x += __shfl_xor_sync(FULL, x, sft);
+      Lh[hd] += x;
+    }
+    const int cnt = min(32, npairs - base);
+    for (int u0 = 0; u0 < cnt; u0 += kInFlight) {
+      VecT v[kInFlight];
+#pragma unroll
+      for (int u = 0; u < kInFlight; ++u) {
+        const unsigned long long rt = __shfl_sync(FULL, row, (u0 + u < cnt) ? u0 + u : 0);  // lane 0's row is valid
+        v[u] = __ldcg(reinterpret_cast<const VecT*>(part + rt + lane * PER));
+      }
+#pragma unroll
+      for (int u = 0; u < kInFlight; ++u) {
+        const float wt = (u0 + u < cnt) ? __shfl_sync(FULL, w, u0 + u) : 0.f;
+        const int ht = __shfl_sync(FULL, hh, (u0 + u < cnt) ? u0 + u : 0);
+        const float* vv = reinterpret_cast<const float*>(&v[u]);
+#pragma unroll
+        for (int hd = 0; hd < G; ++hd) {
+          const float ww = (ht == hd) ? wt : 0.f;
+#pragma unroll
+          for (int e = 0; e < PER; ++e) o[hd][e] = fmaf(ww, vv[e], o[hd][e]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int hd = 0; hd < G; ++hd) {
+    if (dst == ~0ull) {
+      const int jq = cg * G + hd;
+      float* out = outp + (static_cast<size_t>(cb) * Hq + jq) * D + lane * PER;
+      const float inv = Lh[hd] > 0.f ? 1.f / Lh[hd] : 0.f;
+      if constexpr (PER == 4)
+        *reinterpret_cast<float4*>(out) = make_float4(o[hd][0] * inv, o[hd][1] * inv, o[hd][2] * inv, o[hd][3] * inv);
+      else
+        *reinterpret_cast<float2*>(out) = make_float2(o[hd][0] * inv, o[hd][1] * inv);
+      if (lsep && lane == 0)
+        lsep[static_cast<size_t>(cb) * Hq + jq] = Lh[hd] > 0.f ? (Mh[hd] + log2f(Lh[hd])) * 0.69314718055994531f : kNegInf;
+    } else {
+      float* p = part + dst + hd * RS;
+      if constexpr (PER == 4)
+        *reinterpret_cast<float4*>(p + lane * PER) = make_float4(o[hd][0], o[hd][1], o[hd][2], o[hd][3]);
+      else
+        *reinterpret_cast<float2*>(p + lane * PER) = make_float2(o[hd][0], o[hd][1]);
+      if (lane == 0) *reinterpret_cast<float2*>(p + D) = make_float2(Mh[hd], Lh[hd]);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ the decode kernel
 
 template <int D, int G, int QT>
-__global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(const DecodeArgs a) {
   using Gm = Geo<D>;
   constexpr int NKB = Gm::NKB;
   constexpr int WPC = Gm::WPC;
@@ -610,132 +741,42 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_int4_kernel(const Decod
       }
       if (gq == 0) *reinterpret_cast<float2*>(p + D) = make_float2(m_run, l);
     }
-    // partials expected for (b, g): one per warp that owns a tile of each non-empty segment
+    // Partials of (b, g): one per warp that owns a tile of each non-empty segment, ordinal j in
+    // [0, npart) (INT8 owners first).  They are merged in two levels when there are more than
+    // kGroup: the last of each group of kGroup consecutive partials to arrive merges the group
+    // into the row of its first partial; the last group to finish merges the group rows.
     const u32 cs4 = cs8 + 2u * si.n8;
     const u32 w8a = divQ.div(cs8), w4a = divQ.div(cs4);
-    const u32 n8p_ = si.n8 ? divQ.div(cs4 - 2) - w8a + 1 : 0u;
-    const u32 n4p_ = si.n4 ? divQ.div(cs4 + si.n4 - 1) - w4a + 1 : 0u;
-    const unsigned expected = n8p_ + n4p_;
-    __syncwarp();
-    unsigned prev = 0;
-    if (lane == 0) prev = atomic_add_acq_rel(&counters[cb * a.Hkv + cg], 1u);
-    prev = __shfl_sync(FULL, prev, 0);
-    if (prev + 1 != expected) return;
-    __syncwarp();
-    // merge (b, g): lane j reads (m, l) of (head j / npart, partial j % npart), up to 32 pairs at
-    // once; the weighted rows are then summed with lanes over dims.
-    const int n8p = static_cast<int>(n8p_), npart = static_cast<int>(expected);
-    const u32 sid8 = 2u * static_cast<u32>(cb * a.Hkv + cg);
-    constexpr int PER = D / 32;
-    auto row_of = [&](int j, int hh) -> unsigned long long {
-      const u32 idx = j < n8p ? (w8a + j + sid8) : (w4a + (j - n8p) + sid8 + 1);
-      return (static_cast<unsigned long long>(idx) * G + hh) * kPartRow<D>;
+    const int n8p = si.n8 ? static_cast<int>(divQ.div(cs4 - 2) - w8a + 1) : 0;
+    const int n4p = si.n4 ? static_cast<int>(divQ.div(cs4 + si.n4 - 1) - w4a + 1) : 0;
+    const int npart = n8p + n4p;
+    const PartRows pr{n8p, w8a, w4a, 2u * static_cast<u32>(cb * a.Hkv + cg)};
+    const int jme = cseg == 0 ? static_cast<int>(static_cast<u32>(wid) - w8a)
+                              : n8p + static_cast<int>(static_cast<u32>(wid) - w4a);
+    const int ngroups = (npart + kGroup - 1) / kGroup;
+    unsigned* top = &counters[cb * a.Hkv + cg];
+    auto arrive = [&](unsigned* ctr) -> unsigned {
+      __syncwarp();
+      unsigned prev = 0;
+      if (lane == 0) prev = atomic_add_acq_rel(ctr, 1u);
+      prev = __shfl_sync(FULL, prev, 0);
+      __syncwarp();
+      return prev + 1;
     };
-    auto write_out = [&](int hd, const float (&o)[PER], float Ls, float Mx) {
-      const int jq = cg * G + hd;
-      float* out = a.out + (static_cast<size_t>(cb) * a.Hq + jq) * D + lane * PER;
-      const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-      if constexpr (PER == 4)
-        *reinterpret_cast<float4*>(out) = make_float4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
-      else
-        *reinterpret_cast<float2*>(out) = make_float2(o[0] * inv, o[1] * inv);
-      if (a.lse && lane == 0)
-        a.lse[static_cast<size_t>(cb) * a.Hq + jq] = Ls > 0.f ? (Mx + log2f(Ls)) * 0.69314718055994531f : kNegInf;
-    };
-    auto accumulate = [&](float (&o)[PER], unsigned long long rt, float wt) {
-      const float* pr = a.part + rt + lane * PER;
-      if constexpr (PER == 4) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(pr));
-        o[0] += wt * v.x;
-        o[1] += wt * v.y;
-        o[2] += wt * v.z;
-        o[3] += wt * v.w;
-      } else {
-        const float2 v = __ldcg(reinterpret_cast<const float2*>(pr));
-        o[0] += wt * v.x;
-        o[1] += wt * v.y;
-      }
-    };
-    if (npart * G <= 32) {
-      const int hh = lane / npart, j = lane - hh * npart;
-      float pm = kNegInf, pl = 0.f;
-      unsigned long long row = 0;
-      if (hh < G) {
-        row = row_of(j, hh);
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part + row + D));
-        pm = ml.x;
-        pl = ml.y;
-      }
-      const bool ok = pl > 0.f;
-      float mx = ok ? pm : kNegInf;
-      for (int hd = 0; hd < G; ++hd) {
-        float v = (hh == hd) ? mx : kNegInf;
-#pragma unroll
-        for (int sft = 16; sft; sft >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, sft));
-        if (hh == hd) mx = v;
-      }
-      const float wj = ok ? exp2f(pm - mx) : 0.f;
-      float lsum = wj * pl;
-      for (int hd = 0; hd < G; ++hd) {
-        float v = (hh == hd) ? lsum : 0.f;
-#pragma unroll
-        for (int sft = 16; sft; sft >>= 1) v += __shfl_xor_sync(FULL, v, sft);
-        if (hh == hd) lsum = v;
-      }
-      for (int hd = 0; hd < G; ++hd) {
-        float o[PER];
-#pragma unroll
-        for (int e = 0; e < PER; ++e) o[e] = 0.f;
-        for (int t = 0; t < npart; ++t) {
-          const int srcl = hd * npart + t;
-          const float wt = __shfl_sync(FULL, wj, srcl);
-          const unsigned long long rt = __shfl_sync(FULL, row, srcl);
-          if (wt != 0.f) accumulate(o, rt, wt);
-        }
-        write_out(hd, o, __shfl_sync(FULL, lsum, hd * npart), __shfl_sync(FULL, mx, hd * npart));
-      }
+    if (ngroups > 1) {
+      const int j0 = (jme / kGroup) * kGroup, gsize = min(kGroup, npart - j0);
+      const unsigned long long lead = pr.row(j0, G, kPartRow<D>);
+      unsigned* gc = a.gcounters + lead / (static_cast<unsigned long long>(G) * kPartRow<D>);
+      if (arrive(gc) != static_cast<unsigned>(gsize)) return;
+      merge_partials<D, G>(a.part, a.out, a.lse, a.Hq, lane, pr, gsize, j0, 1, lead, cb, cg);
+      if (lane == 0) *gc = 0u;
+      if (arrive(top) != static_cast<unsigned>(ngroups)) return;
+      merge_partials<D, G>(a.part, a.out, a.lse, a.Hq, lane, pr, ngroups, 0, kGroup, ~0ull, cb, cg);
     } else {
-      for (int hh = 0; hh < G; ++hh) {
-        float M = kNegInf, Lsum = 0.f;
-        float o[PER];
-#pragma unroll
-        for (int e = 0; e < PER; ++e) o[e] = 0.f;
-        for (int base = 0; base < npart; base += 32) {
-          const int j = base + lane;
-          float pm = kNegInf, pl = 0.f;
-          unsigned long long row = 0;
-          if (j < npart) {
-            row = row_of(j, hh);
-            const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part + row + D));
-            pm = ml.x;
-            pl = ml.y;
-          }
-          const bool ok = pl > 0.f;
-          float mx = ok ? pm : kNegInf;
-#pragma unroll
-          for (int sft = 16; sft; sft >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, sft));
-          const float Mn = fmaxf(M, mx);
-          if (Mn == kNegInf) continue;
-          const float fo = M == kNegInf ? 0.f : exp2f(M - Mn);
-          const float wj = ok ? exp2f(pm - Mn) : 0.f;
-          float lj = wj * pl;
-#pragma unroll
-          for (int sft = 16; sft; sft >>= 1) lj += __shfl_xor_sync(FULL, lj, sft);
-          Lsum = Lsum * fo + lj;
-#pragma unroll
-          for (int e = 0; e < PER; ++e) o[e] *= fo;
-          const int cnt = min(32, npart - base);
-          for (int t = 0; t < cnt; ++t) {
-            const float wt = __shfl_sync(FULL, wj, t);
-            const unsigned long long rt = __shfl_sync(FULL, row, t);
-            if (wt != 0.f) accumulate(o, rt, wt);
-          }
-          M = Mn;
-        }
-        write_out(hh, o, Lsum, M);
-      }
+      if (arrive(top) != static_cast<unsigned>(npart)) return;
+      merge_partials<D, G>(a.part, a.out, a.lse, a.Hq, lane, pr, npart, 0, 1, ~0ull, cb, cg);
     }
-    if (lane == 0) counters[cb * a.Hkv + cg] = 0u;
+    if (lane == 0) *top = 0u;
   };
 
   // Running-max update for this lane's logits of head tig (NL values), then their exponentials.
@@ -971,6 +1012,7 @@ cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
 }  // namespace
 
 int decode_warps_per_cta() { return kWarps; }
+int decode_ctas_per_sm() { return kCtasPerSm; }
 
 size_t decode_smem_bytes(int D, int G) {
   (void)G;

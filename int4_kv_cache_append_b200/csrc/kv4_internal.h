@@ -37,8 +37,9 @@ struct DecodeArgs {
   const int32_t* lens;
   int B, Hq, Hkv, P, s, w, h, max_pages, nt8;
   size_t page_bytes, side_slot_bytes;
-  float* part;            // split partials [num_slots][G][D + 2]
+  float* part;            // split partials [num_slots][G][D + 4]
   unsigned int* counters; // per (b, g) partial counters, zero between calls
+  unsigned int* gcounters;  // per partial-group counters, indexed by the group's first partial
   float* out;
   float* lse;
   float qscale;           // softmax scale in log2 units: log2(e) / sqrt(D)
@@ -53,6 +54,7 @@ cudaError_t launch_append_int4(const AppendArgs& a, int D, cudaStream_t st);
 cudaError_t launch_append_bf16(const AppendArgs& a, int D, cudaStream_t st);
 
 int decode_warps_per_cta();
+int decode_ctas_per_sm();
 int bf16_decode_warps_per_cta();
 size_t decode_smem_bytes(int D, int G);
 size_t bf16_decode_smem_bytes(int D, int G);
