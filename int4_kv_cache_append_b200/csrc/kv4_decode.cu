@@ -48,6 +48,7 @@ constexpr int kStages = 2;
 constexpr int kChunk = 16;  // slots per descriptor fill
 constexpr int kRing = 32;   // descriptor ring (two chunks)
 constexpr int kGroup = 8;   // partials per group of the two-level merge
+constexpr int kLensRegs = 8;  // sequence lengths held in registers by the schedule (B <= 256)
 constexpr float kNegInf = -__builtin_huge_valf();
 
 // ------------------------------------------------------------------ schedule
@@ -173,13 +174,13 @@ __device__ __forceinline__ void recost(Cursor& c) {
   c.cost = c.seg == 0 ? c.cs8 + 2u * c.i : c.cs8 + 2u * c.si.n8 + c.i;
 }
 
-// First tile whose first unit is >= c0, in sequence b (first unit bstart).
-__device__ Cursor cursor_at(const DecodeArgs& a, int cap, int b, u32 bstart, u32 c0) {
+// First tile whose first unit is >= c0, in sequence b (first unit bstart, raw length Lraw).
+__device__ Cursor cursor_at(const DecodeArgs& a, int cap, int b, u32 bstart, u32 c0, int Lraw) {
   Cursor c;
   c.b = b;
   c.valid = b < a.B;
   if (!c.valid) return c;
-  c.si = seg_info(clamp_len(a.lens[b], cap), a.s, a.w, a.nt8);
+  c.si = seg_info(clamp_len(Lraw, cap), a.s, a.w, a.nt8);
   const u32 ch = head_cost(c.si);
   const u32 off = c0 - bstart;
   c.g = static_cast<int>(off / ch);
@@ -541,6 +542,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   using Gm = Geo<D>;
   constexpr int NKB = Gm::NKB;
   constexpr int WPC = Gm::WPC;
+  constexpr int NK32 = D / 32;  // 32-dim blocks of the QK^T integer MMAs
   constexpr int T4B = Gm::T4B;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem<D>& sm = *reinterpret_cast<Smem<D>*>(smem_raw);
@@ -551,9 +553,31 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   const int cap = a.stride * a.P;
   unsigned int* counters = a.counters;
 
+  uint64_t* bars = sm.bar[warp];
+  if (lane == 0) {
+    for (int i = 0; i < kStages; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+  }
+
+  // Lengths: read once (one load per lane and 32 sequences, all in flight together) and kept in
+  // registers for the schedule when B <= 32 * kLensRegs; larger batches re-read them.
+  const bool cached = a.B <= 32 * kLensRegs;
+  int lr[kLensRegs];
+#pragma unroll
+  for (int r = 0; r < kLensRegs; ++r) {
+    const int b = 32 * r + lane;
+    lr[r] = (cached && b < a.B) ? a.lens[b] : 0;
+  }
+  auto cached_len = [&](int b) {  // raw length of sequence b (warp-uniform b < B <= 32 kLensRegs)
+    int v = lr[0];
+#pragma unroll
+    for (int r = 1; r < kLensRegs; ++r)
+      if ((b >> 5) == r) v = lr[r];
+    return __shfl_sync(FULL, v, b & 31);
+  };
   // Sequences with no positions get out = 0, lse = -inf here (nothing else touches them).
   for (int b = wid; b < a.B; b += a.W) {
-    const int Lraw = a.lens[b];
+    const int Lraw = cached ? cached_len(b) : a.lens[b];
     if (lane == 0 && Lraw > cap) atomicOr(a.err, KV4_DEVERR_LENGTH);
     if (clamp_len(Lraw, cap) == 0) {
       for (int e = lane; e < a.Hq * D; e += 32) a.out[static_cast<size_t>(b) * a.Hq * D + e] = 0.f;
@@ -561,24 +585,46 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
         for (int e = lane; e < a.Hq; e += 32) a.lse[static_cast<size_t>(b) * a.Hq + e] = kNegInf;
     }
   }
-
-  uint64_t* bars = sm.bar[warp];
-  if (lane == 0) {
-    for (int i = 0; i < kStages; ++i) mbar_init(&bars[i], 1);
-    fence_mbar_init();
-  }
   __syncwarp();
 
-  const u32 total = total_cost(a, cap, lane);
+  u32 total = 0;
+  if (cached) {
+#pragma unroll
+    for (int r = 0; r < kLensRegs; ++r)
+      if (32 * r < a.B) {
+        const u32 c = 32 * r + lane < a.B ? static_cast<u32>(a.Hkv) * head_cost(seg_info(clamp_len(lr[r], cap), a.s, a.w, a.nt8)) : 0u;
+        total += __shfl_sync(FULL, warp_incl_scan(c, lane), 31);
+      }
+  } else {
+    total = total_cost(a, cap, lane);
+  }
   const u32 Q = max(2u, (total + a.W - 1) / static_cast<u32>(a.W));
   const FastDiv divQ(Q);
   const unsigned long long c0l = static_cast<unsigned long long>(wid) * Q;
   if (c0l >= total) return;
   const u32 c0 = static_cast<u32>(c0l);
   const u32 c1 = c0 + Q;
-  u32 bstart;
-  const int b0 = find_seq(a, cap, lane, c0, &bstart);
-  Cursor dcur = cursor_at(a, cap, b0, bstart, c0);  // descriptor cursor, one chunk ahead
+  u32 bstart = 0;
+  int b0 = a.B;
+  if (cached) {
+    u32 run = 0;
+#pragma unroll
+    for (int r = 0; r < kLensRegs; ++r)
+      if (32 * r < a.B && b0 == a.B) {
+        const u32 cb = 32 * r + lane < a.B ? static_cast<u32>(a.Hkv) * head_cost(seg_info(clamp_len(lr[r], cap), a.s, a.w, a.nt8)) : 0u;
+        const u32 incl = warp_incl_scan(cb, lane);
+        const u32 tot = __shfl_sync(FULL, incl, 31);
+        if (c0 < run + tot) {
+          const int l = __ffs(__ballot_sync(FULL, c0 < run + incl)) - 1;
+          bstart = run + __shfl_sync(FULL, incl - cb, l);
+          b0 = 32 * r + l;
+        }
+        run += tot;
+      }
+  } else {
+    b0 = find_seq(a, cap, lane, c0, &bstart);
+  }
+  Cursor dcur = cursor_at(a, cap, b0, bstart, c0, b0 < a.B ? (cached ? cached_len(b0) : a.lens[b0]) : 0);
   if (!dcur.valid || dcur.cost >= c1) return;
 
   // Query of the first (b, g): loads issued now, consumed after the first descriptors.
@@ -621,18 +667,23 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   issued = __shfl_sync(FULL, issued, 0);
 
   // ---- per-(b, g) query state
-  uint32_t qf[NKB][2];
-  float sumq = 0.f, qinv = 1.f, qinv20 = 1.f;  // sumq in units of 2^20
+  // Query of head tig as the integer q_int = rint(q * 2^e) with |q_int| < 2^22, split into three
+  // signed base-256 digits; qd[j] holds the s8 B fragments of 32-dim block j: n-block A (columns
+  // 2h, 2h+1 = digits 2, 1 of head h), then n-block B (column 2h = digit 0 of head h).
+  uint32_t qd[NK32][4];
+  float sumq = 0.f, qinv = 1.f;  // sum of q_int over the dims of head tig; 2^-e
 
   // Rotate the G query heads held in qx (H/h), scale to log2 softmax units, normalise each head
   // by a power of two so that its fp16 hi/lo halves stay in the normal range, and build this
   // lane's MMA B fragments through `scratch` (a free stage buffer).
-  auto build_query = [&](float* scratch) {
+  auto build_query = [&](uint8_t* scratch) {
     const bool act = lane < D / 4;
+    const int h = a.h;
+    // Butterfly strides 1 and 2 within the lane, then 4 .. h/2 across lanes (lane xor stride/4),
+    // every stage over all G heads so that their shuffles overlap.
 #pragma unroll
     for (int i = 0; i < G; ++i) {
       float* x = qx[i];
-      const int h = a.h;
       if (h >= 2) {
         float u = x[0], v = x[1];
         x[0] = u + v;
@@ -651,57 +702,106 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
         x[1] = u + v;
         x[3] = u - v;
       }
-      for (int st = 4; st < h; st <<= 1) {
+    }
+#pragma unroll
+    for (int st = 4; st < D; st <<= 1) {
+      if (st < h) {
         const int m = st >> 2;
         const bool upper = (lane & m) != 0;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float o = __shfl_xor_sync(FULL, x[e], m);
-          x[e] = upper ? o - x[e] : x[e] + o;
-        }
+        for (int i = 0; i < G; ++i)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float o = __shfl_xor_sync(FULL, qx[i][e], m);
+            qx[i][e] = upper ? o - qx[i][e] : qx[i][e] + o;
+          }
       }
-      const float sc = a.qscale / static_cast<float>(h);
-      float amax = 0.f;
+    }
+    const float sc = a.qscale / static_cast<float>(h);
+    float amax[G];
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      amax[i] = 0.f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        x[e] *= sc;
-        amax = fmaxf(amax, fabsf(x[e]));
+        qx[i][e] *= sc;
+        amax[i] = fmaxf(amax[i], fabsf(qx[i][e]));
       }
+    }
 #pragma unroll
-      for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
-      // 2^(14 - floor(log2 amax)) puts max|q| in [2^14, 2^15).
-      int ex = amax > 0.f ? ((__float_as_int(amax) >> 23) & 0xff) - 127 : 0;
+    for (int o = 16; o; o >>= 1)
+#pragma unroll
+      for (int i = 0; i < G; ++i) amax[i] = fmaxf(amax[i], __shfl_xor_sync(FULL, amax[i], o));
+    int qsum[G];
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      // 2^(21 - floor(log2 amax)) puts max|q| in [2^21, 2^22).
+      int ex = amax[i] > 0.f ? ((__float_as_int(amax[i]) >> 23) & 0xff) - 127 : 0;
       ex = max(min(ex, 100), -100);
-      const float up = __int_as_float((127 + 14 - ex) << 23);
-      const float down = __int_as_float((127 - 14 + ex) << 23);
-      if (act)
-        *reinterpret_cast<float4*>(scratch + i * D + 4 * lane) = make_float4(x[0] * up, x[1] * up, x[2] * up, x[3] * up);
+      const float up = __int_as_float((127 + 21 - ex) << 23);
+      const float down = __int_as_float((127 - 21 + ex) << 23);
       if (tig == i) qinv = down;
-    }
-    __syncwarp();
-    const int hh = gq >> 1;
-    const bool lo = gq & 1;
+      // digits of the lane's dims 4 lane + e: q = d2 2^16 + d1 2^8 + d0, each in [-128, 127]; in
+      // the scratch each 8-dim group keeps its even dims in bytes 0-3 and odd dims in 4-7, the
+      // order in which the K code bytes of a group enter the MMA.
+      unsigned dg[3][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}};  // [digit][dims {0,2} | {1,3}] packed
+      qsum[i] = 0;
 #pragma unroll
-    for (int kb = 0; kb < NKB; ++kb) {
-      // k-block kb of this lane: dims (d, d + 4) in b0 and (d + 2, d + 6) in b1 of the 8-dim group
-      // W, d = kb & 1, matching the nibble masks of the K code words in qk_int4.
-      const int W = WPC * tig + (kb >> 1);
-      if (hh < G) {
-        const float* qh = scratch + hh * D + 8 * W + (kb & 1);
-        qf[kb][0] = split_pair(qh[0], qh[4], lo);
-        qf[kb][1] = split_pair(qh[2], qh[6], lo);
-      } else {
-        qf[kb][0] = 0u;
-        qf[kb][1] = 0u;
+      for (int e = 0; e < 4; ++e) {
+        const int qv = act ? __float2int_rn(qx[i][e] * up) : 0;
+        qsum[i] += qv;
+        const int d0 = ((qv + 128) & 255) - 128;
+        const int q1 = (qv - d0) >> 8;
+        const int d1 = ((q1 + 128) & 255) - 128;
+        const int d2 = (q1 - d1) >> 8;
+        const int sh = 8 * (e >> 1);
+        dg[0][e & 1] |= static_cast<unsigned>(d0 & 255) << sh;
+        dg[1][e & 1] |= static_cast<unsigned>(d1 & 255) << sh;
+        dg[2][e & 1] |= static_cast<unsigned>(d2 & 255) << sh;
+      }
+      if (act) {
+        // lane holds dims 0-3 (even lane) or 4-7 (odd lane) of group lane / 2: even dims go to
+        // bytes (0, 1) or (2, 3) of the group, odd dims to bytes (4, 5) or (6, 7).
+        const int gb = 8 * (lane >> 1) + 2 * (lane & 1);
+#pragma unroll
+        for (int dgt = 0; dgt < 3; ++dgt) {
+          uint8_t* row = scratch + (i * 3 + dgt) * D + gb;
+          *reinterpret_cast<unsigned short*>(row) = static_cast<unsigned short>(dg[dgt][0]);
+          *reinterpret_cast<unsigned short*>(row + 4) = static_cast<unsigned short>(dg[dgt][1]);
+        }
       }
     }
-    // sum over the dims of head tig of the query exactly as the tensor core holds it (hi + lo):
-    // one MMA chain against an all-ones A operand.
-    float Sq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int kb = 0; kb < NKB; ++kb) mma_f16(Sq, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u, qf[kb][0], qf[kb][1]);
-    sumq = (Sq[0] + Sq[1]) * 0x1p-20f;
-    qinv20 = qinv * 0x1p20f;
+    for (int o = 16; o; o >>= 1)
+#pragma unroll
+      for (int i = 0; i < G; ++i) qsum[i] += __shfl_xor_sync(FULL, qsum[i], o);
+#pragma unroll
+    for (int i = 0; i < G; ++i)
+      if (tig == i) sumq = static_cast<float>(qsum[i]);
+    __syncwarp();
+    // B fragments: lane (gq, tig) supplies column gq, bytes of its dims 32 tig + 8 j + (0, 2, 4, 6)
+    // (b0) and (1, 3, 5, 7) (b1).
+    const int hA = gq >> 1, digA = (gq & 1) ? 1 : 2;
+    const int hB = gq >> 1;
+    const bool useB = (gq & 1) == 0;
+#pragma unroll
+    for (int j = 0; j < NK32; ++j) {
+      const int grp = WPC * tig + j;
+      if (hA < G) {
+        const uint2 v = *reinterpret_cast<const uint2*>(scratch + (hA * 3 + digA) * D + 8 * grp);
+        qd[j][0] = v.x;
+        qd[j][1] = v.y;
+      } else {
+        qd[j][0] = qd[j][1] = 0u;
+      }
+      if (useB && hB < G) {
+        const uint2 v = *reinterpret_cast<const uint2*>(scratch + (hB * 3 + 0) * D + 8 * grp);
+        qd[j][2] = v.x;
+        qd[j][3] = v.y;
+      } else {
+        qd[j][2] = qd[j][3] = 0u;
+      }
+    }
     __syncwarp();
   };
 
@@ -823,26 +923,24 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     uint32_t kw0[WPC], kw1[WPC];
     lds_words<WPC>(tb + gq * (D / 2) + tig * Gm::CH, kw0);
     lds_words<WPC>(tb + (gq + 8) * (D / 2) + tig * Gm::CH, kw1);
-    float S[4] = {0.f, 0.f, 0.f, 0.f}, S2[4] = {0.f, 0.f, 0.f, 0.f};
+    int SA[4] = {0, 0, 0, 0}, SB[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int kb = 0; kb < NKB; ++kb) {
-      // word j of a row holds dims 8W..8W+7, nibble n at bits 4n.  Every code is moved to bits
-      // 4-7 of its half (fp16 subnormal c * 2^-20): even kb takes dims 0, 4 (w << 4) and 2, 6
-      // (w >> 4), odd kb dims 1, 5 (w) and 3, 7 (w >> 8).
-      const int j = kb >> 1;
-      const uint32_t w0 = kw0[j], w1 = kw1[j];
-      if (kb & 1)
-        mma_f16(S2, nib_hi(w0), nib_hi(w1), nib_hi(w0 >> 8), nib_hi(w1 >> 8), qf[kb][0], qf[kb][1]);
-      else
-        mma_f16(S, nib_hi(w0 << 4), nib_hi(w1 << 4), nib_hi(w0 >> 4), nib_hi(w1 >> 4), qf[kb][0], qf[kb][1]);
+    for (int j = 0; j < NK32; ++j) {
+      // word j of a row holds the codes of dims 8W..8W+7 (W = WPC tig + j), dim 8W + n at bits
+      // 4n: the low nibbles of its bytes are the even dims, the high nibbles the odd dims.
+      const uint32_t l0 = kw0[j] & 0x0F0F0F0Fu, h0 = (kw0[j] >> 4) & 0x0F0F0F0Fu;
+      const uint32_t l1 = kw1[j] & 0x0F0F0F0Fu, h1 = (kw1[j] >> 4) & 0x0F0F0F0Fu;
+      mma_u8s8(SA, l0, l1, h0, h1, qd[j][0], qd[j][1]);
+      mma_u8s8(SB, l0, l1, h0, h1, qd[j][2], qd[j][3]);
     }
     const uint32_t kp0 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 4 * gq);
     const uint32_t kp1 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 4 * (gq + 8));
     const float ks0 = half_lo(kp0), kz0 = half_hi(kp0), ks1 = half_lo(kp1), kz1 = half_hi(kp1);
-    // logit = (s q.c + z sum(q)) / 2^e with q.c = 2^20 R
-    const float R0 = (S[0] + S[1]) + (S2[0] + S2[1]), R1 = (S[2] + S[3]) + (S2[2] + S2[3]);
-    lg0 = v0 ? fmaf(ks0, R0, kz0 * sumq) * qinv20 : kNegInf;
-    lg1 = v1 ? fmaf(ks1, R1, kz1 * sumq) * qinv20 : kNegInf;
+    // logit = (s q_int.c + z sum(q_int)) 2^-e
+    const float R0 = fmaf(65536.f, static_cast<float>(SA[0]), fmaf(256.f, static_cast<float>(SA[1]), static_cast<float>(SB[0])));
+    const float R1 = fmaf(65536.f, static_cast<float>(SA[2]), fmaf(256.f, static_cast<float>(SA[3]), static_cast<float>(SB[2])));
+    lg0 = v0 ? fmaf(ks0, R0, kz0 * sumq) * qinv : kNegInf;
+    lg1 = v1 ? fmaf(ks1, R1, kz1 * sumq) * qinv : kNegInf;
   };
 
   // PV of one INT4 tile block with probabilities p0, p1 (rows gq, gq + 8 of head tig).
@@ -873,7 +971,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
 
   // ---- main loop over this warp's slots
   reset();
-  build_query(reinterpret_cast<float*>(sm.ring[warp][kStages - 1]));  // stage kStages-1 is not in flight
+  build_query(sm.ring[warp][kStages - 1]);  // stage kStages-1 is not in flight
   int cur_bg;  // (b, g) whose query fragments are loaded
   {
     const unsigned long long se = sm.seg[warp][meta_seg(sm.meta[warp][0])];
@@ -925,21 +1023,21 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
         kw0[4 * u] = x0.x; kw0[4 * u + 1] = x0.y; kw0[4 * u + 2] = x0.z; kw0[4 * u + 3] = x0.w;
         kw1[4 * u] = x1.x; kw1[4 * u + 1] = x1.y; kw1[4 * u + 2] = x1.z; kw1[4 * u + 3] = x1.w;
       }
-      float S[4] = {0.f, 0.f, 0.f, 0.f};
+      int SA[4] = {0, 0, 0, 0}, SB[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int kb = 0; kb < NKB; ++kb) {
-        const int j = kb >> 1;
-        const uint32_t A0 = kw0[2 * j] ^ 0x80808080u, B0 = kw0[2 * j + 1] ^ 0x80808080u;
-        const uint32_t A1 = kw1[2 * j] ^ 0x80808080u, B1 = kw1[2 * j + 1] ^ 0x80808080u;
-        const uint32_t sel = (kb & 1) ? 0x7351u : 0x6240u;  // dims (d, d+4, d+2, d+6), d = kb & 1
-        const uint32_t t0 = prmt(A0, B0, sel), t1 = prmt(A1, B1, sel);
-        mma_f16(S, i8x2_to_h2<0x4140>(t0), i8x2_to_h2<0x4140>(t1), i8x2_to_h2<0x4342>(t0), i8x2_to_h2<0x4342>(t1),
-                qf[kb][0], qf[kb][1]);
+      for (int j = 0; j < NK32; ++j) {
+        // words 2j, 2j + 1 of a row: dims 8W + 0..3 and 8W + 4..7; even dims, then odd dims
+        const uint32_t a0 = prmt(kw0[2 * j], kw0[2 * j + 1], 0x6420u), a2 = prmt(kw0[2 * j], kw0[2 * j + 1], 0x7531u);
+        const uint32_t a1 = prmt(kw1[2 * j], kw1[2 * j + 1], 0x6420u), a3 = prmt(kw1[2 * j], kw1[2 * j + 1], 0x7531u);
+        mma_s8s8(SA, a0, a1, a2, a3, qd[j][0], qd[j][1]);
+        mma_s8s8(SB, a0, a1, a2, a3, qd[j][2], qd[j][3]);
       }
       const float ks0 = __half2float(*reinterpret_cast<const __half*>(buf + 16 * D + 2 * gq));
       const float ks1 = __half2float(*reinterpret_cast<const __half*>(buf + 16 * D + 2 * (gq + 8)));
-      const float lg0 = v0 ? ks0 * (S[0] + S[1]) * qinv : kNegInf;
-      const float lg1 = v1 ? ks1 * (S[2] + S[3]) * qinv : kNegInf;
+      const float R0 = fmaf(65536.f, static_cast<float>(SA[0]), fmaf(256.f, static_cast<float>(SA[1]), static_cast<float>(SB[0])));
+      const float R1 = fmaf(65536.f, static_cast<float>(SA[2]), fmaf(256.f, static_cast<float>(SA[3]), static_cast<float>(SB[2])));
+      const float lg0 = v0 ? ks0 * R0 * qinv : kNegInf;
+      const float lg1 = v1 ? ks1 * R1 * qinv : kNegInf;
       const float mu = softmax_update(fmaxf(lg0, lg1));
       const float p0 = exp2_fast(lg0 - mu), p1 = exp2_fast(lg1 - mu);
       l_part += (v0 ? p0 : 0.f) + (v1 ? p1 : 0.f);
@@ -978,7 +1076,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
       if (nbg != cur_bg) {
         cur_bg = nbg;
         load_q_regs(seg_b(ns), seg_g(ns));
-        build_query(reinterpret_cast<float*>(sm.ring[warp][st]));  // this slot's stage is free now
+        build_query(sm.ring[warp][st]);  // this slot's stage is free now
       }
     }
     ++k;
