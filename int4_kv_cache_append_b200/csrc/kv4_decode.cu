@@ -424,13 +424,13 @@ struct PartRows {
   }
 };
 
-// LSE merge of the n partials j0, j0 + step, ... of one (b, g).  Pass 1 finds the per-head
-// maximum of m (lanes read the (m, l) of 32 (head, partial) pairs at a time).  Pass 2 walks the
-// n * G pairs head-major, 32 at a time: each lane weights one pair, exp2(m - M) and its share
-// of the per-head sum; the pairs' o rows are then read kInFlight at a time with independent
-// loads so that their latencies overlap (a pass over n rows costs about 1 + n G / kInFlight
-// round trips to L2).  dst = ~0 writes the normalised output and lse of query heads cg*G.. of
-// sequence cb; otherwise the merged rows (o, M, L) go to the rows at dst.
+// LSE merge of the n partials j0, j0 + step, ... of one (b, g), in one pass over the n * G
+// (head, partial) pairs taken head-major, 32 at a time: each lane reads the (m, l) of one pair;
+// the running per-head maximum M is raised to the block's maximum (rescaling what was summed so
+// far); each pair gets weight exp2(m - M), and the pairs' o rows are read kInFlight at a time
+// with independent loads so that their latencies overlap.  dst = ~0 writes the normalised
+// output and lse of query heads cg*G.. of sequence cb; otherwise the merged rows (o, M, L) go to
+// the rows at dst.
 template <int D, int G>
 __device__ __forceinline__ void merge_partials(float* part, float* outp, float* lsep, int Hq, int lane,
                                                const PartRows pr, int n, int j0, int step, unsigned long long dst,
@@ -450,42 +450,34 @@ __device__ __forceinline__ void merge_partials(float* part, float* outp, float* 
   }
   for (int base = 0; base < npairs; base += 32) {
     const int q = base + lane;
-    float v = kNegInf;
-    int hh = -1;
-    if (q < npairs) {
-      hh = q / n;
-      const float2 ml = __ldcg(reinterpret_cast<const float2*>(part + pr.row(j0 + (q - hh * n) * step, G, RS) + hh * RS + D));
-      if (ml.y > 0.f) v = ml.x;
-    }
-#pragma unroll
-    for (int hd = 0; hd < G; ++hd) {
-      float x = (hh == hd) ? v : kNegInf;
-#pragma unroll
-      for (int sft = 16; sft; sft >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, sft));
-      Mh[hd] = fmaxf(Mh[hd], x);
-    }
-  }
-  for (int base = 0; base < npairs; base += 32) {
-    const int q = base + lane;
-    float w = 0.f, wl = 0.f;
     unsigned long long row = 0;
     int hh = 0;
+    float2 ml = make_float2(kNegInf, 0.f);
     if (q < npairs) {
       hh = q / n;
       row = pr.row(j0 + (q - hh * n) * step, G, RS) + hh * RS;
-      const float2 ml = __ldcg(reinterpret_cast<const float2*>(part + row + D));
-      float mh = Mh[0];
-#pragma unroll
-      for (int hd = 1; hd < G; ++hd)
-        if (hh == hd) mh = Mh[hd];
-      if (ml.y > 0.f) {
-        w = exp2f(ml.x - mh);
-        wl = w * ml.y;
-      }
+      ml = __ldcg(reinterpret_cast<const float2*>(part + row + D));
     }
+    const bool live = q < npairs && ml.y > 0.f;
+    float mh = kNegInf;
 #pragma unroll
     for (int hd = 0; hd < G; ++hd) {
-      float x = (hh == hd) ? wl : 0.f;
+      float x = (live && hh == hd) ? ml.x : kNegInf;
+#pragma unroll
+      for (int sft = 16; sft; sft >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, sft));
+      if (x > Mh[hd]) {  // warp-uniform: rescale the head's sums to the new maximum
+        const float sc = Mh[hd] == kNegInf ? 0.f : exp2f(Mh[hd] - x);
+        Lh[hd] *= sc;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[hd][e] *= sc;
+        Mh[hd] = x;
+      }
+      if (hh == hd) mh = Mh[hd];
+    }
+    const float w = live ? exp2f(ml.x - mh) : 0.f;
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) {
+      float x = (hh == hd) ? w * ml.y : 0.f;
 #pragma unroll
       for (int sft = 16; sft; sft >>= 1) x += __shfl_xor_sync(FULL, x, sft);
       Lh[hd] += x;
