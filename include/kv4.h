@@ -134,12 +134,11 @@ kv4_status kv4_decode_workspace_bytes(const kv4_cache* cache, int B, size_t* byt
  *   page_table   device int32 [>= B][stride];  lens device int32 [B] (0 gives out = 0, lse = -inf)
  *   max_len_hint host upper bound of lens (0 = unknown); only sizes the grid
  *   out          device fp32 [B][Hq][D];  lse device fp32 [B][Hq] or NULL
- *   workspace    device scratch of at least kv4_decode_workspace_bytes(B) bytes, 16-byte aligned,
- *                zero-filled once before its first use (e.g. cudaMemsetAsync); it holds per
- *                (sequence, KV head) counters that every call returns to zero, so it stays ready
- *                for the next call of any batch size.  Re-zero it after a device-side error.
- * One launch on the stream: split-K partials, merged by the last warp to finish each
- * (sequence, KV head).
+ *   workspace    device scratch of at least kv4_decode_workspace_bytes(B) bytes, 16-byte aligned;
+ *                its contents need no initialisation and are dead after the call.
+ * Two launches on the stream: the split-K pass (one partial (o, m, l) per warp and segment it
+ * touches; a (sequence, KV head) covered by a single partial is written directly), then the LSE
+ * merge of the partials of every other (sequence, KV head).
  */
 kv4_status kv4_decode_attn(kv4_cache* cache, int layer, int B, const void* q, kv4_dtype q_dtype,
                            const int32_t* page_table, int stride, const int32_t* lens, int max_len_hint,
@@ -173,11 +172,10 @@ kv4_status kv4_bf16_decode_attn(kv4_cache* cache, int layer, int B, const void* 
  * workspace.  A batch whose partials exceed the array (kv4_decode_workspace_bytes(B) >
  * KV4_STATIC_SCRATCH_BYTES; about B > 350 for 8 KV heads, head_dim 128, 4 q heads per KV head on
  * 148 SMs) returns KV4_ERR_WORKSPACE and launches nothing.
- * The first call on a device looks up the array's device address (cudaGetSymbolAddress) and
- * zero-fills the array on the call's stream, with that device current; make that first call
- * before any stream capture.  All calls on one GPU share the array, which keeps the last call's
- * contents: every call returns its merge counters to zero and writes every partial its merge
- * reads, so nothing needs clearing between calls.  Calls that overlap on the
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  All calls on one GPU share
+ * the array; every call writes every partial its merge reads, so nothing needs clearing between
+ * calls.  Calls that overlap on the
  * GPU (different streams, or another thread) race on the array and must be serialised by the
  * caller.
  */

@@ -96,23 +96,13 @@ size_t align16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
 int decode_ctas_full(int format, int sms) { return format == FMT_INT4 ? kv4::decode_ctas_per_sm() * sms : sms; }
 
-// Workspace layout: [counters][split partials].  Counters: max_seqs * Hkv per (sequence, KV head)
-// counters, then one per possible partial index (warps of the full grid + 2 * max_seqs * Hkv) for
-// the groups of the two-level merge; padded to 256 B.  The counter region depends only on the
-// configuration and the device, so one workspace serves every batch size and grid.
-size_t counter_bytes(const kv4_cache* c, int sms) {
-  const size_t bg = static_cast<size_t>(c->cfg.max_seqs) * c->cfg.num_kv_heads;
-  const int full_warps =
-      decode_ctas_full(c->format, sms) * (c->format == FMT_INT4 ? kv4::decode_warps_per_cta() : kv4::bf16_decode_warps_per_cta());
-  const size_t n = (bg + static_cast<size_t>(full_warps) + 2 * bg) * sizeof(uint32_t);
-  return (n + 255) & ~static_cast<size_t>(255);
-}
-
-size_t workspace_for(const kv4_cache* c, int B, int ctas, int sms) {
+// Workspace: the split partials, one row group of G rows of (o[D], m, l) padded to D + 4 floats
+// per possible partial index (warps of the grid + 2 * B * Hkv segments).
+size_t workspace_for(const kv4_cache* c, int B, int ctas) {
   const int G = c->cfg.num_q_heads / c->cfg.num_kv_heads;
   const int warps = ctas * (c->format == FMT_INT4 ? kv4::decode_warps_per_cta() : kv4::bf16_decode_warps_per_cta());
   const size_t segs = static_cast<size_t>(B) * c->cfg.num_kv_heads * (c->format == FMT_INT4 ? 2 : 1);
-  return counter_bytes(c, sms) + align16((static_cast<size_t>(warps) + segs) * G * (c->cfg.head_dim + 4) * sizeof(float));
+  return align16((static_cast<size_t>(warps) + segs) * G * (c->cfg.head_dim + 4) * sizeof(float));
 }
 
 kv4_status append_common(kv4_cache* c, int fmt, int layer, int T, const void* K, kv4_dtype kd, const void* V,
@@ -183,7 +173,7 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
     if (want < 1) want = 1;
     if (want < ctas) ctas = static_cast<int>(want);
   }
-  if (ws_bytes < workspace_for(c, B, ctas, sms)) return KV4_ERR_WORKSPACE;
+  if (ws_bytes < workspace_for(c, B, ctas)) return KV4_ERR_WORKSPACE;
   {
     // work units are counted in 32 bits on the device: bound the worst case (every sequence at
     // the page-table capacity)
@@ -210,9 +200,7 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
   a.nt8 = c->nt8;
   a.page_bytes = c->page_bytes;
   a.side_slot_bytes = c->side_slot_bytes;
-  a.counters = static_cast<unsigned int*>(ws);
-  a.gcounters = static_cast<unsigned int*>(ws) + static_cast<size_t>(c->cfg.max_seqs) * c->cfg.num_kv_heads;
-  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + counter_bytes(c, sms));
+  a.part = static_cast<float*>(ws);
   a.out = out;
   a.lse = lse;
   a.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->cfg.head_dim)));
@@ -275,7 +263,7 @@ kv4_status kv4_decode_workspace_bytes(const kv4_cache* cache, int B, size_t* byt
   if (!cache || cache->format != FMT_INT4 || B < 0 || !bytes) return KV4_ERR_INVALID_ARG;
   int sms = 0;
   if (!device_info(nullptr, &sms)) return KV4_ERR_CUDA;
-  *bytes = workspace_for(cache, B, decode_ctas_full(FMT_INT4, sms), sms);
+  *bytes = workspace_for(cache, B, decode_ctas_full(FMT_INT4, sms));
   return KV4_OK;
 }
 
@@ -292,16 +280,14 @@ kv4_status kv4_decode_attn(kv4_cache* cache, int layer, int B, const void* q, kv
 static __device__ __align__(256) unsigned char g_kv4_static_scratch[KV4_STATIC_SCRATCH_BYTES];
 static void* g_static_scratch_ptr[kMaxDevices] = {};
 
-// First use on a device: look up the array's address and zero it (the merge counters at its
-// start must begin at zero; every decode returns them to zero afterwards).
-static bool static_scratch_address(void** out, cudaStream_t stream) {
+// First use on a device: look up the array's address (with that device current).
+static bool static_scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_static_scratch_ptr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_kv4_static_scratch) != cudaSuccess || !p) return false;
-    if (cudaMemsetAsync(p, 0, KV4_STATIC_SCRATCH_BYTES, stream) != cudaSuccess) return false;
     g_static_scratch_ptr[dev] = p;
   }
   *out = g_static_scratch_ptr[dev];
@@ -315,9 +301,9 @@ kv4_status kv4_decode_attn_static(kv4_cache* cache, int layer, int B, const void
   if (B == 0) return KV4_OK;
   int sms = 0;
   if (!device_info(nullptr, &sms)) return KV4_ERR_CUDA;
-  if (workspace_for(cache, B, decode_ctas_full(FMT_INT4, sms), sms) > KV4_STATIC_SCRATCH_BYTES) return KV4_ERR_WORKSPACE;
+  if (workspace_for(cache, B, decode_ctas_full(FMT_INT4, sms)) > KV4_STATIC_SCRATCH_BYTES) return KV4_ERR_WORKSPACE;
   void* scratch = nullptr;
-  if (!static_scratch_address(&scratch, static_cast<cudaStream_t>(stream))) return KV4_ERR_CUDA;
+  if (!static_scratch_address(&scratch)) return KV4_ERR_CUDA;
   return decode_common(cache, FMT_INT4, layer, B, q, q_dtype, page_table, stride, lens, max_len_hint, out, lse,
                        scratch, KV4_STATIC_SCRATCH_BYTES, stream);
 }
@@ -361,7 +347,7 @@ kv4_status kv4_bf16_decode_workspace_bytes(const kv4_cache* cache, int B, size_t
   if (!cache || cache->format != FMT_BF16 || B < 0 || !bytes) return KV4_ERR_INVALID_ARG;
   int sms = 0;
   if (!device_info(nullptr, &sms)) return KV4_ERR_CUDA;
-  *bytes = workspace_for(cache, B, decode_ctas_full(FMT_BF16, sms), sms);
+  *bytes = workspace_for(cache, B, decode_ctas_full(FMT_BF16, sms));
   return KV4_OK;
 }
 

@@ -14,19 +14,21 @@
 // first unit lies in [w*Q, (w+1)*Q), Q = ceil(total / warps), so every warp streams about the
 // same number of bytes whatever the length mix.  A warp writes one partial (o, m, l) for every
 // segment it touches, at index w + segment_id (unique: each step along the sequence advances the
-// warp, the segment, or both), then counts it on the (b, g) counter; the warp that brings the
-// counter to the number of partials of (b, g) merges them with the LSE rule, writes out/lse and
-// returns the counter to zero.
+// warp, the segment, or both); a second kernel (merge_int4_kernel) merges the partials of each
+// (b, g) with the LSE rule.  A (b, g) whose positions all fell to one warp segment is written
+// directly.  One CTA of 16 warps per SM.
 //
 // Per warp: kStages shared-memory stages of two tile blocks each, fed by 1-D bulk copies
 // (cp.async.bulk, issued by lane 0 kStages-1 slots ahead, completion on one mbarrier per stage).
 // A slot is two INT4 tiles (32 positions) or one INT8 tile (its K half and V half).  Slot
 // descriptors (sources, 32-row validity mask, segment index, last-slot flag) are computed 16 slots
 // at a time, one slot per lane, into a small ring, so the per-slot bookkeeping is a few
-// instructions.  The G query heads of the KV group and hi/lo fp16 halves of each query form the
-// 8 columns of an m16n8k16 MMA: QK^T takes 16 positions x 16 dims per MMA with the codes as the A
-// operand converted in registers; PV takes 16 dims x 16 positions with the (p * scale) hi/lo
-// halves as the B operand.  Softmax, scale/offset and rescaling run in fp32 registers.
+// instructions.  QK^T runs on 8-bit integer MMAs (m16n8k32): the INT4 key codes, unpacked to
+// bytes, are the A operand; the rotated query, rounded to a 22-bit integer and split into three
+// signed base-256 digits, is the B operand (G heads x 3 digits in two n-blocks), so q . c is exact
+// in int32.  PV runs on m16n8k16 fp16 MMAs: 16 dims x 16 positions with the centred V codes as the
+// A operand and the hi/lo fp16 halves of p * scale of the G heads as the 8 columns of B.  Softmax,
+// scale/offset and rescaling run in fp32 registers.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -47,7 +49,6 @@ constexpr int kCtasPerSm = 1;
 constexpr int kStages = 2;
 constexpr int kChunk = 16;  // slots per descriptor fill
 constexpr int kRing = 32;   // descriptor ring (two chunks)
-constexpr int kGroup = 8;   // partials per group of the two-level merge
 constexpr int kLensRegs = 8;  // sequence lengths held in registers by the schedule (B <= 256)
 constexpr float kNegInf = -__builtin_huge_valf();
 
@@ -424,109 +425,6 @@ struct PartRows {
   }
 };
 
-// LSE merge of the n partials j0, j0 + step, ... of one (b, g), in one pass over the n * G
-// (head, partial) pairs taken head-major, 32 at a time: each lane reads the (m, l) of one pair;
-// the running per-head maximum M is raised to the block's maximum (rescaling what was summed so
-// far); each pair gets weight exp2(m - M), and the pairs' o rows are read kInFlight at a time
-// with independent loads so that their latencies overlap.  dst = ~0 writes the normalised
-// output and lse of query heads cg*G.. of sequence cb; otherwise the merged rows (o, M, L) go to
-// the rows at dst.
-template <int D, int G>
-__device__ __forceinline__ void merge_partials(float* part, float* outp, float* lsep, int Hq, int lane,
-                                               const PartRows pr, int n, int j0, int step, unsigned long long dst,
-                                               int cb, int cg) {
-  constexpr int PER = D / 32;
-  constexpr int kInFlight = 8;
-  constexpr int RS = kPartRow<D>;
-  using VecT = typename std::conditional<PER == 4, float4, float2>::type;
-  const int npairs = n * G;
-  float Mh[G], Lh[G], o[G][PER];
-#pragma unroll
-  for (int hd = 0; hd < G; ++hd) {
-    Mh[hd] = kNegInf;
-    Lh[hd] = 0.f;
-#pragma unroll
-    for (int e = 0; e < PER; ++e) o[hd][e] = 0.f;
-  }
-  for (int base = 0; base < npairs; base += 32) {
-    const int q = base + lane;
-    unsigned long long row = 0;
-    int hh = 0;
-    float2 ml = make_float2(kNegInf, 0.f);
-    if (q < npairs) {
-      hh = q / n;
-      row = pr.row(j0 + (q - hh * n) * step, G, RS) + hh * RS;
-      ml = __ldcg(reinterpret_cast<const float2*>(part + row + D));
-    }
-    const bool live = q < npairs && ml.y > 0.f;
-    float mh = kNegInf;
-#pragma unroll
-    for (int hd = 0; hd < G; ++hd) {
-      float x = (live && hh == hd) ? ml.x : kNegInf;
-#pragma unroll
-      for (int sft = 16; sft; sft >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, sft));
-      if (x > Mh[hd]) {  // warp-uniform: rescale the head's sums to the new maximum
-        const float sc = Mh[hd] == kNegInf ? 0.f : exp2f(Mh[hd] - x);
-        Lh[hd] *= sc;
-#pragma unroll
-        for (int e = 0; e < PER; ++e) o[hd][e] *= sc;
-        Mh[hd] = x;
-      }
-      if (hh == hd) mh = Mh[hd];
-    }
-    const float w = live ? exp2f(ml.x - mh) : 0.f;
-#pragma unroll
-    for (int hd = 0; hd < G; ++hd) {
-      float x = (hh == hd) ? w * ml.y : 0.f;
-#pragma unroll
-      for (int sft = 16; sft; sft >>= 1) x += __shfl_xor_sync(FULL, x, sft);
-      Lh[hd] += x;
-    }
-    const int cnt = min(32, npairs - base);
-    for (int u0 = 0; u0 < cnt; u0 += kInFlight) {
-      VecT v[kInFlight];
-#pragma unroll
-      for (int u = 0; u < kInFlight; ++u) {
-        const unsigned long long rt = __shfl_sync(FULL, row, (u0 + u < cnt) ? u0 + u : 0);  // lane 0's row is valid
-        v[u] = __ldcg(reinterpret_cast<const VecT*>(part + rt + lane * PER));
-      }
-#pragma unroll
-      for (int u = 0; u < kInFlight; ++u) {
-        const float wt = (u0 + u < cnt) ? __shfl_sync(FULL, w, u0 + u) : 0.f;
-        const int ht = __shfl_sync(FULL, hh, (u0 + u < cnt) ? u0 + u : 0);
-        const float* vv = reinterpret_cast<const float*>(&v[u]);
-#pragma unroll
-        for (int hd = 0; hd < G; ++hd) {
-          const float ww = (ht == hd) ? wt : 0.f;
-#pragma unroll
-          for (int e = 0; e < PER; ++e) o[hd][e] = fmaf(ww, vv[e], o[hd][e]);
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int hd = 0; hd < G; ++hd) {
-    if (dst == ~0ull) {
-      const int jq = cg * G + hd;
-      float* out = outp + (static_cast<size_t>(cb) * Hq + jq) * D + lane * PER;
-      const float inv = Lh[hd] > 0.f ? 1.f / Lh[hd] : 0.f;
-      if constexpr (PER == 4)
-        *reinterpret_cast<float4*>(out) = make_float4(o[hd][0] * inv, o[hd][1] * inv, o[hd][2] * inv, o[hd][3] * inv);
-      else
-        *reinterpret_cast<float2*>(out) = make_float2(o[hd][0] * inv, o[hd][1] * inv);
-      if (lsep && lane == 0)
-        lsep[static_cast<size_t>(cb) * Hq + jq] = Lh[hd] > 0.f ? (Mh[hd] + log2f(Lh[hd])) * 0.69314718055994531f : kNegInf;
-    } else {
-      float* p = part + dst + hd * RS;
-      if constexpr (PER == 4)
-        *reinterpret_cast<float4*>(p + lane * PER) = make_float4(o[hd][0], o[hd][1], o[hd][2], o[hd][3]);
-      else
-        *reinterpret_cast<float2*>(p + lane * PER) = make_float2(o[hd][0], o[hd][1]);
-      if (lane == 0) *reinterpret_cast<float2*>(p + D) = make_float2(Mh[hd], Lh[hd]);
-    }
-  }
-}
-
 // ------------------------------------------------------------------ the decode kernel
 
 template <int D, int G, int QT>
@@ -543,7 +441,6 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   const int gq = lane >> 2, tig = lane & 3;
   const int wid = blockIdx.x * kWarps + warp;
   const int cap = a.stride * a.P;
-  unsigned int* counters = a.counters;
 
   uint64_t* bars = sm.bar[warp];
   if (lane == 0) {
@@ -808,9 +705,9 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     beta_part = 0.f;
   };
 
-  // Write the partial of the segment `se` (a segment-table entry); if it completes its (b, g),
-  // merge and write out.
-  auto flush_and_merge = [&](unsigned long long se) {
+  // Write the partial of the segment `se` (a segment-table entry).  The partials of (b, g) are
+  // merged by merge_int4_kernel; when this is the only partial of (b, g) it is the output.
+  auto flush = [&](unsigned long long se) {
     const int cb = seg_b(se), cg = seg_g(se), cseg = seg_kind(se);
     const u32 cs8 = seg_cs8(se);
     const SegInfo si = seg_info(clamp_len(a.lens[cb], cap), a.s, a.w, a.nt8);
@@ -820,55 +717,31 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
       l += __shfl_xor_sync(FULL, l, o);
       beta += __shfl_xor_sync(FULL, beta, o);
     }
+    const u32 cs4 = cs8 + 2u * si.n8;
+    const u32 w8a = divQ.div(cs8), w4a = divQ.div(cs4);
+    const u32 n8p = si.n8 ? divQ.div(cs4 - 2) - w8a + 1 : 0u;
+    const u32 n4p = si.n4 ? divQ.div(cs4 + si.n4 - 1) - w4a + 1 : 0u;
+    const bool only = n8p + n4p == 1u;
     const u32 sid = 2u * static_cast<u32>(cb * a.Hkv + cg) + static_cast<u32>(cseg);
     if (tig < G) {
       // INT4: even output rows carry (c - 8), odd rows 16 (c - 8); INT8 rows carry c.
       const float f1 = cseg == 1 ? 0.0625f : 1.f;
-      float* p = a.part + (static_cast<size_t>(wid + sid) * G + tig) * kPartRow<D>;
+      const float sc = only ? (l > 0.f ? 1.f / l : 0.f) : 1.f;
+      float* p = only ? a.out + (static_cast<size_t>(cb) * a.Hq + cg * G + tig) * D
+                      : a.part + (static_cast<size_t>(wid + sid) * G + tig) * kPartRow<D>;
 #pragma unroll
       for (int mb = 0; mb < NKB; ++mb) {
         const int d = Gm::DG * gq + 2 * mb;
-        *reinterpret_cast<float2*>(p + d) =
-            make_float2((oacc[mb][0] + oacc[mb][1]) + beta, f1 * (oacc[mb][2] + oacc[mb][3]) + beta);
+        *reinterpret_cast<float2*>(p + d) = make_float2(((oacc[mb][0] + oacc[mb][1]) + beta) * sc,
+                                                         (f1 * (oacc[mb][2] + oacc[mb][3]) + beta) * sc);
       }
-      if (gq == 0) *reinterpret_cast<float2*>(p + D) = make_float2(m_run, l);
+      if (gq == 0) {
+        if (!only)
+          *reinterpret_cast<float2*>(p + D) = make_float2(m_run, l);
+        else if (a.lse)
+          a.lse[static_cast<size_t>(cb) * a.Hq + cg * G + tig] = l > 0.f ? (m_run + log2f(l)) * 0.69314718055994531f : kNegInf;
+      }
     }
-    // Partials of (b, g): one per warp that owns a tile of each non-empty segment, ordinal j in
-    // [0, npart) (INT8 owners first).  They are merged in two levels when there are more than
-    // kGroup: the last of each group of kGroup consecutive partials to arrive merges the group
-    // into the row of its first partial; the last group to finish merges the group rows.
-    const u32 cs4 = cs8 + 2u * si.n8;
-    const u32 w8a = divQ.div(cs8), w4a = divQ.div(cs4);
-    const int n8p = si.n8 ? static_cast<int>(divQ.div(cs4 - 2) - w8a + 1) : 0;
-    const int n4p = si.n4 ? static_cast<int>(divQ.div(cs4 + si.n4 - 1) - w4a + 1) : 0;
-    const int npart = n8p + n4p;
-    const PartRows pr{n8p, w8a, w4a, 2u * static_cast<u32>(cb * a.Hkv + cg)};
-    const int jme = cseg == 0 ? static_cast<int>(static_cast<u32>(wid) - w8a)
-                              : n8p + static_cast<int>(static_cast<u32>(wid) - w4a);
-    const int ngroups = (npart + kGroup - 1) / kGroup;
-    unsigned* top = &counters[cb * a.Hkv + cg];
-    auto arrive = [&](unsigned* ctr) -> unsigned {
-      __syncwarp();
-      unsigned prev = 0;
-      if (lane == 0) prev = atomic_add_acq_rel(ctr, 1u);
-      prev = __shfl_sync(FULL, prev, 0);
-      __syncwarp();
-      return prev + 1;
-    };
-    if (ngroups > 1) {
-      const int j0 = (jme / kGroup) * kGroup, gsize = min(kGroup, npart - j0);
-      const unsigned long long lead = pr.row(j0, G, kPartRow<D>);
-      unsigned* gc = a.gcounters + lead / (static_cast<unsigned long long>(G) * kPartRow<D>);
-      if (arrive(gc) != static_cast<unsigned>(gsize)) return;
-      merge_partials<D, G>(a.part, a.out, a.lse, a.Hq, lane, pr, gsize, j0, 1, lead, cb, cg);
-      if (lane == 0) *gc = 0u;
-      if (arrive(top) != static_cast<unsigned>(ngroups)) return;
-      merge_partials<D, G>(a.part, a.out, a.lse, a.Hq, lane, pr, ngroups, 0, kGroup, ~0ull, cb, cg);
-    } else {
-      if (arrive(top) != static_cast<unsigned>(npart)) return;
-      merge_partials<D, G>(a.part, a.out, a.lse, a.Hq, lane, pr, npart, 0, 1, ~0ull, cb, cg);
-    }
-    if (lane == 0) *top = 0u;
   };
 
   // Running-max update for this lane's logits of head tig (NL values), then their exponentials.
@@ -1059,7 +932,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
 
     if (meta & kMetaLast) {
       const unsigned long long se = sm.seg[warp][meta_seg(meta)];
-      flush_and_merge(se);
+      flush(se);
       reset();
       const unsigned nmeta = sm.meta[warp][(k + 1) % kRing];
       if (meta_kind(nmeta) == kKindNone) break;  // end of this warp's stream
@@ -1081,6 +954,98 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   }
 }
 
+// ------------------------------------------------------------------ LSE merge kernel
+
+// One warp per (sequence b, query head j): recomputes the schedule of the decode launch (the same
+// unit sequence and quota Q over the same W warps) to find the partials of (b, j / G), and merges
+// head j % G of them with the LSE rule in one pass, 32 partials at a time: lanes read the (m, l)
+// of 32 partials, the running maximum is raised to their maximum (rescaling the sums so far), and
+// their o rows are read kInFlight at a time with independent loads.  (b, g) with at most one
+// partial were written by the decode kernel.
+template <int D, int G>
+__global__ void __launch_bounds__(256) merge_int4_kernel(const DecodeArgs a) {
+  constexpr int PER = D / 32;
+  constexpr int kInFlight = 16;
+  constexpr int RS = kPartRow<D>;
+  using VecT = typename std::conditional<PER == 4, float4, float2>::type;
+  const int lane = threadIdx.x & 31;
+  const int item = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  if (item >= a.B * a.Hq) return;
+  const int b = item / a.Hq, j = item - b * a.Hq;
+  const int g = j / G, hd = j - g * G;
+  const int cap = a.stride * a.P;
+  u32 run = 0, bstart = 0;
+#pragma unroll 4
+  for (int base = 0; base < a.B; base += 32) {
+    const int bb = base + lane;
+    const u32 c = bb < a.B ? seq_cost(a, cap, bb) : 0u;
+    const u32 incl = warp_incl_scan(c, lane);
+    if (b >= base && b < base + 32) bstart = run + __shfl_sync(FULL, incl - c, b - base);
+    run += __shfl_sync(FULL, incl, 31);
+  }
+  const u32 Q = max(2u, (run + a.W - 1) / static_cast<u32>(a.W));
+  const SegInfo si = seg_info(clamp_len(a.lens[b], cap), a.s, a.w, a.nt8);
+  const u32 cs8 = bstart + static_cast<u32>(g) * head_cost(si);
+  const u32 cs4 = cs8 + 2u * si.n8;
+  const u32 w8a = cs8 / Q, w4a = cs4 / Q;
+  const int n8p = si.n8 ? static_cast<int>((cs4 - 2) / Q - w8a + 1) : 0;
+  const int n4p = si.n4 ? static_cast<int>((cs4 + si.n4 - 1) / Q - w4a + 1) : 0;
+  const int n = n8p + n4p;
+  if (n <= 1) return;
+  const PartRows pr{n8p, w8a, w4a, 2u * static_cast<u32>(b * a.Hkv + g)};
+  float M = kNegInf, L = 0.f, o[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) o[e] = 0.f;
+  for (int base = 0; base < n; base += 32) {
+    const int t = base + lane;
+    unsigned long long row = 0;
+    float2 ml = make_float2(kNegInf, 0.f);
+    if (t < n) {
+      row = pr.row(t, G, RS) + hd * RS;
+      ml = __ldcg(reinterpret_cast<const float2*>(a.part + row + D));
+    }
+    const bool live = t < n && ml.y > 0.f;
+    float x = live ? ml.x : kNegInf;
+#pragma unroll
+    for (int sft = 16; sft; sft >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, sft));
+    if (x > M) {
+      const float sc = M == kNegInf ? 0.f : exp2f(M - x);
+      L *= sc;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) o[e] *= sc;
+      M = x;
+    }
+    const float w = live ? exp2f(ml.x - M) : 0.f;
+    float wl = w * ml.y;
+#pragma unroll
+    for (int sft = 16; sft; sft >>= 1) wl += __shfl_xor_sync(FULL, wl, sft);
+    L += wl;
+    const int cnt = min(32, n - base);
+    for (int u0 = 0; u0 < cnt; u0 += kInFlight) {
+      VecT v[kInFlight];
+#pragma unroll
+      for (int u = 0; u < kInFlight; ++u) {
+        const unsigned long long rt = __shfl_sync(FULL, row, (u0 + u < cnt) ? u0 + u : 0);  // lane 0's row is valid
+        v[u] = __ldcg(reinterpret_cast<const VecT*>(a.part + rt + lane * PER));
+      }
+#pragma unroll
+      for (int u = 0; u < kInFlight; ++u) {
+        const float wt = (u0 + u < cnt) ? __shfl_sync(FULL, w, u0 + u) : 0.f;
+        const float* vv = reinterpret_cast<const float*>(&v[u]);
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[e] = fmaf(wt, vv[e], o[e]);
+      }
+    }
+  }
+  float* out = a.out + (static_cast<size_t>(b) * a.Hq + j) * D + lane * PER;
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  if constexpr (PER == 4)
+    *reinterpret_cast<float4*>(out) = make_float4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
+  else
+    *reinterpret_cast<float2*>(out) = make_float2(o[0] * inv, o[1] * inv);
+  if (a.lse && lane == 0) a.lse[static_cast<size_t>(b) * a.Hq + j] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : kNegInf;
+}
+
 template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
   const int smem = static_cast<int>(sizeof(Smem<D>));
@@ -1096,6 +1061,9 @@ cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
     if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F16>, smem, done[2])) != cudaSuccess) return e;
     decode_int4_kernel<D, G, KV4_F16><<<ctas, kWarps * 32, smem, st>>>(a);
   }
+  cudaError_t le = cudaGetLastError();
+  if (le != cudaSuccess) return le;
+  merge_int4_kernel<D, G><<<(a.B * a.Hq + 7) / 8, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -1111,7 +1079,7 @@ size_t decode_smem_bytes(int D, int G) {
 
 cudaError_t launch_decode_int4(DecodeArgs a, int D, int G, int ctas, cudaStream_t st) {
   a.W = ctas * kWarps;
-  note_launches(1);
+  note_launches(2);
   if (D == 128) {
     if (G == 4) return launch_dg<128, 4>(a, ctas, st);
     if (G == 2) return launch_dg<128, 2>(a, ctas, st);

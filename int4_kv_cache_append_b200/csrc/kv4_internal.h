@@ -38,8 +38,6 @@ struct DecodeArgs {
   int B, Hq, Hkv, P, s, w, h, max_pages, nt8;
   size_t page_bytes, side_slot_bytes;
   float* part;            // split partials [num_slots][G][D + 4]
-  unsigned int* counters; // per (b, g) partial counters, zero between calls
-  unsigned int* gcounters;  // per partial-group counters, indexed by the group's first partial
   float* out;
   float* lse;
   float qscale;           // softmax scale in log2 units: log2(e) / sqrt(D)

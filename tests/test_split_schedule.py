@@ -4,19 +4,17 @@ The decode kernel gives warp w the tiles whose first slot lies in [w*Q, (w+1)*Q)
 sequence of all slots (per sequence b, per KV head g: the INT8 segment of ceil((s+w)/16) tiles
 of 2 slots, then the INT4 segment of the 16-position tiles covering [s, max(s, L-w))), writes one
 partial per (warp, segment) at index warp + segment_id, and the merge of (b, g) reads, for each
-segment, the partials of warps floor(first_slot/Q) .. floor(last_tile_start/Q).  The partials of
-(b, g) are numbered j = 0.. (INT8-segment writers first, then INT4) and merged in groups of
-K_GROUP consecutive partials, each group counted on the counter indexed by the partial index of
-its first member.  This model restates that arithmetic and checks its invariants for many length
-mixes and grid sizes: every tile processed exactly once, partial indices unique and inside the
-workspace, the merge reads exactly the partials that were written, each writer's ordinal is the
-one the kernel computes, group counter indices are unique and inside their region, and every
-bulk-copy source lies inside its buffer.
+segment, the partials of warps floor(first_slot/Q) .. floor(last_tile_start/Q).  The merge kernel
+numbers the partials of (b, g) j = 0.. (INT8-segment writers first, then INT4) and finds partial j
+at index w8a + j + sid8 (INT8) or w4a + (j - n8p) + sid8 + 1 (INT4).  This model restates that
+arithmetic and checks its invariants for many length mixes and grid sizes: every tile processed
+exactly once, partial indices unique and inside the workspace, the merge reads exactly the
+partials that were written (and finds each at the index its writer used), a (b, g) with a single
+partial is recognised as such by its writer, and every bulk-copy source lies inside its buffer.
 """
 import numpy as np
 import pytest
 
-K_GROUP = 8
 
 
 def seg_info(L, s, w, nt8):
@@ -58,7 +56,6 @@ def model(lens, Hkv, s, w, P, stride, W):
     assert len(idx) == len(set(idx))
     assert all(0 <= v < W + 2 * len(lens) * Hkv for v in idx)
     # merge ranges
-    group_counters = set()
     pos = 0
     for b, L in enumerate(lens):
         n8, n4, t4a, m_end = seg_info(L, s, w, nt8)
@@ -91,13 +88,7 @@ def model(lens, Hkv, s, w, P, stride, W):
                 seg, wr = (0, idx - sid8) if j < n8p else (1, idx - sid8 - 1)
                 jme = (wr - w8a) if seg == 0 else n8p + (wr - w4a)
                 assert jme == j
-            ngroups = -(-len(parts) // K_GROUP)
-            if ngroups > 1:
-                for k in range(ngroups):
-                    gidx = parts[k * K_GROUP]
-                    assert gidx not in group_counters
-                    assert 0 <= gidx < W + 2 * len(lens) * Hkv
-                    group_counters.add(gidx)
+            assert (len(parts) == 1) == (n8p + n4p == 1)
         # INT4 tiles address pages inside the page-table row
         for i in range(n4):
             ti = t4a + i
