@@ -96,13 +96,18 @@ size_t align16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
 int decode_ctas_full(int format, int sms) { return format == FMT_INT4 ? kv4::decode_ctas_per_sm() * sms : sms; }
 
-// Workspace: the split partials, one row group of G rows of (o[D], m, l) padded to D + 4 floats
-// per possible partial index (warps of the grid + 2 * B * Hkv segments).
+// Workspace: per (sequence, KV head) a 16-byte record of where its partials are (max_seqs * Hkv
+// records, INT4 format), then the split partials, one row group of G rows of (o[D], m, l) padded
+// to D + 4 floats per possible partial index (warps of the grid + 2 * B * Hkv segments).
+size_t meta_bytes(const kv4_cache* c) {
+  return c->format == FMT_INT4 ? static_cast<size_t>(c->cfg.max_seqs) * c->cfg.num_kv_heads * 16 : 0;
+}
+
 size_t workspace_for(const kv4_cache* c, int B, int ctas) {
   const int G = c->cfg.num_q_heads / c->cfg.num_kv_heads;
   const int warps = ctas * (c->format == FMT_INT4 ? kv4::decode_warps_per_cta() : kv4::bf16_decode_warps_per_cta());
   const size_t segs = static_cast<size_t>(B) * c->cfg.num_kv_heads * (c->format == FMT_INT4 ? 2 : 1);
-  return align16((static_cast<size_t>(warps) + segs) * G * (c->cfg.head_dim + 4) * sizeof(float));
+  return meta_bytes(c) + align16((static_cast<size_t>(warps) + segs) * G * (c->cfg.head_dim + 4) * sizeof(float));
 }
 
 kv4_status append_common(kv4_cache* c, int fmt, int layer, int T, const void* K, kv4_dtype kd, const void* V,
@@ -200,7 +205,8 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
   a.nt8 = c->nt8;
   a.page_bytes = c->page_bytes;
   a.side_slot_bytes = c->side_slot_bytes;
-  a.part = static_cast<float*>(ws);
+  a.meta = static_cast<unsigned int*>(ws);
+  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + meta_bytes(c));
   a.out = out;
   a.lse = lse;
   a.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->cfg.head_dim)));

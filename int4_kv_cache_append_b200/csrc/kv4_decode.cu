@@ -50,6 +50,7 @@ constexpr int kStages = 2;
 constexpr int kChunk = 16;  // slots per descriptor fill
 constexpr int kRing = 32;   // descriptor ring (two chunks)
 constexpr int kLensRegs = 8;  // sequence lengths held in registers by the schedule (B <= 256)
+constexpr int kMergeWideItems = 1184;  // up to this many (b, j), 4 merge warps each
 constexpr float kNegInf = -__builtin_huge_valf();
 
 // ------------------------------------------------------------------ schedule
@@ -441,6 +442,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   const int gq = lane >> 2, tig = lane & 3;
   const int wid = blockIdx.x * kWarps + warp;
   const int cap = a.stride * a.P;
+  pdl_launch_dependents();  // the merge kernel may be scheduled as SMs free up; it waits for this grid
 
   uint64_t* bars = sm.bar[warp];
   if (lane == 0) {
@@ -723,6 +725,8 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     const u32 n4p = si.n4 ? divQ.div(cs4 + si.n4 - 1) - w4a + 1 : 0u;
     const bool only = n8p + n4p == 1u;
     const u32 sid = 2u * static_cast<u32>(cb * a.Hkv + cg) + static_cast<u32>(cseg);
+    // where the merge finds the partials of (b, g); every writer of (b, g) stores the same record
+    if (lane == 0) *reinterpret_cast<uint4*>(a.meta + 4 * (cb * a.Hkv + cg)) = make_uint4(w8a, w4a, n8p, n4p);
     if (tig < G) {
       // INT4: even output rows carry (c - 8), odd rows 16 (c - 8); INT8 rows carry c.
       const float f1 = cseg == 1 ? 0.0625f : 1.f;
@@ -956,55 +960,51 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
 
 // ------------------------------------------------------------------ LSE merge kernel
 
-// One warp per (sequence b, query head j): recomputes the schedule of the decode launch (the same
-// unit sequence and quota Q over the same W warps) to find the partials of (b, j / G), and merges
-// head j % G of them with the LSE rule in one pass, 32 partials at a time: lanes read the (m, l)
-// of 32 partials, the running maximum is raised to their maximum (rescaling the sums so far), and
-// their o rows are read kInFlight at a time with independent loads.  (b, g) with at most one
-// partial were written by the decode kernel.
-template <int D, int G>
-__global__ void __launch_bounds__(256) merge_int4_kernel(const DecodeArgs a) {
+// Merge of the partials of (sequence b, query head j): MW warps per (b, j) (MW = 4 when the batch
+// has few (b, j), else 1 with 4 (b, j) per CTA).  The decode kernel left, per (b, g), where the n
+// partials are (meta); warp w of the MW merges head j % G of partials [w n / MW, (w+1) n / MW) in
+// one pass, 32 at a time: lanes read the (m, l) of 32 partials, the running maximum is raised to
+// their maximum (rescaling the sums so far), and their o rows are read kInFlight at a time with
+// independent loads.  With MW = 4, warp 0 combines the warps' (M, L, o) through shared memory.
+// (b, g) with at most one partial were written by the decode kernel; sequences of length 0 were
+// written by it too and have no meta.  Launched as a programmatic dependent of the decode kernel:
+// griddepcontrol.wait orders every read of its results after its completion.
+constexpr int kMergeThreads = 128;
+
+template <int D, int G, int MW>
+__global__ void __launch_bounds__(kMergeThreads) merge_int4_kernel(const DecodeArgs a) {
   constexpr int PER = D / 32;
   constexpr int kInFlight = 16;
   constexpr int RS = kPartRow<D>;
   using VecT = typename std::conditional<PER == 4, float4, float2>::type;
-  const int lane = threadIdx.x & 31;
-  const int item = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  __shared__ float smo[MW][D];
+  __shared__ float smM[MW], smL[MW];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = MW == 1 ? 0 : warp;                       // warp within the item
+  const int item = MW == 1 ? blockIdx.x * (kMergeThreads / 32) + warp : blockIdx.x;
   if (item >= a.B * a.Hq) return;
   const int b = item / a.Hq, j = item - b * a.Hq;
   const int g = j / G, hd = j - g * G;
   const int cap = a.stride * a.P;
-  u32 run = 0, bstart = 0;
-#pragma unroll 4
-  for (int base = 0; base < a.B; base += 32) {
-    const int bb = base + lane;
-    const u32 c = bb < a.B ? seq_cost(a, cap, bb) : 0u;
-    const u32 incl = warp_incl_scan(c, lane);
-    if (b >= base && b < base + 32) bstart = run + __shfl_sync(FULL, incl - c, b - base);
-    run += __shfl_sync(FULL, incl, 31);
-  }
-  const u32 Q = max(2u, (run + a.W - 1) / static_cast<u32>(a.W));
-  const SegInfo si = seg_info(clamp_len(a.lens[b], cap), a.s, a.w, a.nt8);
-  const u32 cs8 = bstart + static_cast<u32>(g) * head_cost(si);
-  const u32 cs4 = cs8 + 2u * si.n8;
-  const u32 w8a = cs8 / Q, w4a = cs4 / Q;
-  const int n8p = si.n8 ? static_cast<int>((cs4 - 2) / Q - w8a + 1) : 0;
-  const int n4p = si.n4 ? static_cast<int>((cs4 + si.n4 - 1) / Q - w4a + 1) : 0;
-  const int n = n8p + n4p;
-  if (n <= 1) return;
-  const PartRows pr{n8p, w8a, w4a, 2u * static_cast<u32>(b * a.Hkv + g)};
+  pdl_wait();
+  if (clamp_len(a.lens[b], cap) == 0) return;
+  const uint4 mt = *reinterpret_cast<const uint4*>(a.meta + 4 * (b * a.Hkv + g));
+  const int n8p = static_cast<int>(mt.z), n = static_cast<int>(mt.z + mt.w);
+  if (n <= 1) return;  // uniform over the item's warps
+  const PartRows pr{n8p, mt.x, mt.y, 2u * static_cast<u32>(b * a.Hkv + g)};
+  const int t0 = sub * n / MW, t1 = (sub + 1) * n / MW;
   float M = kNegInf, L = 0.f, o[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) o[e] = 0.f;
-  for (int base = 0; base < n; base += 32) {
+  for (int base = t0; base < t1; base += 32) {
     const int t = base + lane;
     unsigned long long row = 0;
     float2 ml = make_float2(kNegInf, 0.f);
-    if (t < n) {
+    if (t < t1) {
       row = pr.row(t, G, RS) + hd * RS;
       ml = __ldcg(reinterpret_cast<const float2*>(a.part + row + D));
     }
-    const bool live = t < n && ml.y > 0.f;
+    const bool live = t < t1 && ml.y > 0.f;
     float x = live ? ml.x : kNegInf;
 #pragma unroll
     for (int sft = 16; sft; sft >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, sft));
@@ -1020,7 +1020,7 @@ __global__ void __launch_bounds__(256) merge_int4_kernel(const DecodeArgs a) {
 #pragma unroll
     for (int sft = 16; sft; sft >>= 1) wl += __shfl_xor_sync(FULL, wl, sft);
     L += wl;
-    const int cnt = min(32, n - base);
+    const int cnt = min(32, t1 - base);
     for (int u0 = 0; u0 < cnt; u0 += kInFlight) {
       VecT v[kInFlight];
 #pragma unroll
@@ -1037,6 +1037,30 @@ __global__ void __launch_bounds__(256) merge_int4_kernel(const DecodeArgs a) {
       }
     }
   }
+  if constexpr (MW > 1) {
+#pragma unroll
+    for (int e = 0; e < PER; ++e) smo[sub][lane * PER + e] = o[e];
+    if (lane == 0) {
+      smM[sub] = M;
+      smL[sub] = L;
+    }
+    __syncthreads();
+    if (sub != 0) return;
+    M = kNegInf;
+#pragma unroll
+    for (int w = 0; w < MW; ++w)
+      if (smL[w] > 0.f) M = fmaxf(M, smM[w]);
+    L = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) o[e] = 0.f;
+#pragma unroll
+    for (int w = 0; w < MW; ++w) {
+      const float f = smL[w] > 0.f ? exp2f(smM[w] - M) : 0.f;
+      L += f * smL[w];
+#pragma unroll
+      for (int e = 0; e < PER; ++e) o[e] = fmaf(f, smo[w][lane * PER + e], o[e]);
+    }
+  }
   float* out = a.out + (static_cast<size_t>(b) * a.Hq + j) * D + lane * PER;
   const float inv = L > 0.f ? 1.f / L : 0.f;
   if constexpr (PER == 4)
@@ -1044,6 +1068,24 @@ __global__ void __launch_bounds__(256) merge_int4_kernel(const DecodeArgs a) {
   else
     *reinterpret_cast<float2*>(out) = make_float2(o[0] * inv, o[1] * inv);
   if (a.lse && lane == 0) a.lse[static_cast<size_t>(b) * a.Hq + j] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : kNegInf;
+}
+
+// Launch of the merge kernel as a programmatic dependent of the preceding decode kernel.
+template <int D, int G>
+cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t st) {
+  const int items = a.B * a.Hq;
+  const bool wide = items <= kMergeWideItems;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(wide ? items : (items + kMergeThreads / 32 - 1) / (kMergeThreads / 32)));
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return wide ? cudaLaunchKernelEx(&cfg, merge_int4_kernel<D, G, 4>, a) : cudaLaunchKernelEx(&cfg, merge_int4_kernel<D, G, 1>, a);
 }
 
 template <int D, int G>
@@ -1063,8 +1105,7 @@ cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
   }
   cudaError_t le = cudaGetLastError();
   if (le != cudaSuccess) return le;
-  merge_int4_kernel<D, G><<<(a.B * a.Hq + 7) / 8, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_merge<D, G>(a, st);
 }
 
 }  // namespace

@@ -116,6 +116,12 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Programmatic dependent launch: let the next kernel on the stream (launched with programmatic
+// stream serialisation) be scheduled before this grid ends; in that kernel, wait for the
+// preceding grid to complete with its memory operations visible.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // D += A B with 8-bit integer operands, int32 accumulation (exact): A 16x32 row-major (u8 or s8),
 // B 32x8 column-major (s8).
 __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,

@@ -38,6 +38,7 @@ struct DecodeArgs {
   int B, Hq, Hkv, P, s, w, h, max_pages, nt8;
   size_t page_bytes, side_slot_bytes;
   float* part;            // split partials [num_slots][G][D + 4]
+  unsigned int* meta;     // per (b, g): first INT8 / INT4 partial warps and their counts
   float* out;
   float* lse;
   float qscale;           // softmax scale in log2 units: log2(e) / sqrt(D)
