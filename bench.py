@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--no-bf16", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--overlap", action="store_true",
+                    help="decode builds its schedule while the append runs (kv4_set_decode_overlap 1)")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--soak-s", type=float, default=1.5, help="untimed identical steps sampled for clocks")
     return ap.parse_args()
@@ -377,6 +379,9 @@ def run_kv4(args, world, rank, local):
 
     # ---- INT4 cache (the product)
     cache, ins, bt, pt_ = setup(False)
+    # lens and page_table are written before the step, not by the append: the decode may build its
+    # schedule while the append runs
+    kv4.kv4_set_decode_overlap(cache.handle, args.overlap)
     append, decode, out, page_table, lens_t = make_steps(cache, ins, bt, pt_, False)
     total_ms, dec_ms, app_ms, launches, clocks = timed(append, decode, args.steps, args.warmup,
                                                        sampler=ClockSampler(uuid), soak_s=args.soak_s)
@@ -474,7 +479,8 @@ def run_kv4(args, world, rank, local):
                        "compute": "f16 tensor-core operands, f32 accumulate/softmax",
                        "l2": "inputs larger than L2: 4 resident layers cycled, 0.72 GB of KV between reuses",
                        "parallelism": f"dp{world} (independent batches per GPU, no collective)",
-                       "graph": not args.no_graph, "append_ms": round(app_ms, 5)},
+                       "graph": not args.no_graph, "decode_overlap": args.overlap,
+                       "append_ms": round(app_ms, 5)},
             "roofline": roof, "hbm_frac_of_spec_8TBps": round(spec_frac, 4), "gpu_launches": int(launches),
             "clocks": clocks, "e2e": e2e, "bf16_kv": bf, "cpu_baseline": cpu}
     return line if rank == 0 else None

@@ -145,6 +145,19 @@ kv4_status kv4_decode_attn(kv4_cache* cache, int layer, int B, const void* q, kv
                            float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * kv4_set_decode_overlap: how kv4_decode_attn of this cache starts (default 0).  Its kernel is
+ * always launched as a programmatic dependent of the preceding kernel on the stream, and the
+ * append kernel lets its dependent launch early.  With 0 the decode kernel reads nothing before
+ * the preceding kernel has completed: stream order exactly.  With 1 it builds its work schedule
+ * and first copy descriptors, reading lens and page_table only, while the preceding kernel runs,
+ * then waits for it before reading q or the cache or writing any output; lens and page_table
+ * must then not be written by the kernel that immediately precedes the decode on the stream
+ * (writes earlier in stream order are fine).  Returns KV4_ERR_INVALID_ARG for a NULL or BF16
+ * cache.
+ */
+kv4_status kv4_set_decode_overlap(kv4_cache* cache, int enable);
+
+/*
  * BF16-KV baseline with the same page table and conventions, no quantisation and no rotation:
  * a page holds Hkv head blocks of P * 4D bytes (bf16 K and V).  Used to measure the INT4
  * speed-up on the same box.  kv4_bf16_query_sizes returns num_layers * max_pages * Hkv * P * 4D.

@@ -37,6 +37,7 @@ struct kv4_cache {
   size_t side_slot_bytes;  // one sequence slot, all KV heads
   size_t side_layer_bytes;
   int nt8;
+  int overlap;  // kv4_set_decode_overlap
 };
 
 namespace kv4 {
@@ -213,7 +214,8 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
   a.err = err;
   {
     const int tpp = c->cfg.page_size / 16;
-    a.tp_shift = pow2(tpp) ? __builtin_ctz(static_cast<unsigned>(tpp)) : -1;
+    a.early = (fmt == FMT_INT4 && c->overlap) ? 1 : 0;
+  a.tp_shift = pow2(tpp) ? __builtin_ctz(static_cast<unsigned>(tpp)) : -1;
   }
   const int G = c->cfg.num_q_heads / c->cfg.num_kv_heads;
   const cudaError_t e = fmt == FMT_INT4
@@ -298,6 +300,12 @@ static bool static_scratch_address(void** out) {
   }
   *out = g_static_scratch_ptr[dev];
   return true;
+}
+
+kv4_status kv4_set_decode_overlap(kv4_cache* cache, int enable) {
+  if (!cache || cache->format != FMT_INT4) return KV4_ERR_INVALID_ARG;
+  cache->overlap = enable ? 1 : 0;
+  return KV4_OK;
 }
 
 kv4_status kv4_decode_attn_static(kv4_cache* cache, int layer, int B, const void* q, kv4_dtype q_dtype,

@@ -136,6 +136,7 @@ __device__ __forceinline__ uint32_t quant_int8(const float (&x)[4], bool act, ui
 template <int D, typename KT, typename VT>
 __global__ void __launch_bounds__(256) append_int4_kernel(AppendArgs a) {
   using Gm = Geo<D>;
+  pdl_launch_dependents();  // the decode kernel that follows may start its launch now
   const int gw = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= a.T * a.Hkv) return;

@@ -444,6 +444,10 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   const int cap = a.stride * a.P;
   pdl_launch_dependents();  // the merge kernel may be scheduled as SMs free up; it waits for this grid
 
+  // Launched as a programmatic dependent of the preceding kernel.  By default nothing is read
+  // before that kernel completes; with a.early the schedule and the first descriptors (which read
+  // only lens and page_table) are built first, and the wait comes before anything else.
+  if (!a.early) pdl_wait();
   uint64_t* bars = sm.bar[warp];
   if (lane == 0) {
     for (int i = 0; i < kStages; ++i) mbar_init(&bars[i], 1);
@@ -466,18 +470,6 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
       if ((b >> 5) == r) v = lr[r];
     return __shfl_sync(FULL, v, b & 31);
   };
-  // Sequences with no positions get out = 0, lse = -inf here (nothing else touches them).
-  for (int b = wid; b < a.B; b += a.W) {
-    const int Lraw = cached ? cached_len(b) : a.lens[b];
-    if (lane == 0 && Lraw > cap) atomicOr(a.err, KV4_DEVERR_LENGTH);
-    if (clamp_len(Lraw, cap) == 0) {
-      for (int e = lane; e < a.Hq * D; e += 32) a.out[static_cast<size_t>(b) * a.Hq * D + e] = 0.f;
-      if (a.lse)
-        for (int e = lane; e < a.Hq; e += 32) a.lse[static_cast<size_t>(b) * a.Hq + e] = kNegInf;
-    }
-  }
-  __syncwarp();
-
   u32 total = 0;
   if (cached) {
 #pragma unroll
@@ -492,7 +484,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   const u32 Q = max(2u, (total + a.W - 1) / static_cast<u32>(a.W));
   const FastDiv divQ(Q);
   const unsigned long long c0l = static_cast<unsigned long long>(wid) * Q;
-  if (c0l >= total) return;
+  const bool any = c0l < total;
   const u32 c0 = static_cast<u32>(c0l);
   const u32 c1 = c0 + Q;
   u32 bstart = 0;
@@ -515,10 +507,11 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   } else {
     b0 = find_seq(a, cap, lane, c0, &bstart);
   }
-  Cursor dcur = cursor_at(a, cap, b0, bstart, c0, b0 < a.B ? (cached ? cached_len(b0) : a.lens[b0]) : 0);
-  if (!dcur.valid || dcur.cost >= c1) return;
+  Cursor dcur = cursor_at(a, cap, b0, bstart, c0, (any && b0 < a.B) ? (cached ? cached_len(b0) : a.lens[b0]) : 0);
+  const bool active = any && dcur.valid && dcur.cost < c1;
 
-  // Query of the first (b, g): loads issued now, consumed after the first descriptors.
+  // Query of the first (b, g): loaded during the first descriptor fill, or after the wait on the
+  // preceding kernel when the schedule is built early.
   float qx[G][4];
   auto load_q_regs = [&](int b, int g) {
     const bool act = lane < D / 4;
@@ -529,11 +522,28 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
       for (int e = 0; e < 4; ++e) qx[i][e] = act ? load_q<QT>(a.q, q0 + e) : 0.f;
     }
   };
-  load_q_regs(dcur.b, dcur.g);
+  const int qb0 = dcur.b, qg0 = dcur.g;  // first (b, g); the fill below moves dcur on
+  if (active && !a.early) load_q_regs(qb0, qg0);  // in flight during the descriptor fill
 
   unsigned segno = 0;
-  fill_descriptors<D>(a, cap, c1, dcur, lane, sm, warp, 0, segno);
+  if (active) fill_descriptors<D>(a, cap, c1, dcur, lane, sm, warp, 0, segno);
   __syncwarp();
+  if (a.early) pdl_wait();
+
+  // Sequences with no positions get out = 0, lse = -inf here (nothing else touches them).
+  for (int b = wid; b < a.B; b += a.W) {
+    const int Lraw = cached ? cached_len(b) : a.lens[b];
+    if (lane == 0 && Lraw > cap) atomicOr(a.err, KV4_DEVERR_LENGTH);
+    if (clamp_len(Lraw, cap) == 0) {
+      for (int e = lane; e < a.Hq * D; e += 32) a.out[static_cast<size_t>(b) * a.Hq * D + e] = 0.f;
+      if (a.lse)
+        for (int e = lane; e < a.Hq; e += 32) a.lse[static_cast<size_t>(b) * a.Hq + e] = kNegInf;
+    }
+  }
+  __syncwarp();
+
+  if (!active) return;
+  if (a.early) load_q_regs(qb0, qg0);
 
   // Issue the bulk copies of slot k into stage k % kStages (lane 0).  Returns false past the end.
   auto issue = [&](int k) {
@@ -1092,19 +1102,28 @@ template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
   const int smem = static_cast<int>(sizeof(Smem<D>));
   static std::atomic<uint64_t> done[3];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   cudaError_t e;
   if (a.q_dtype == KV4_F32) {
     if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F32>, smem, done[0])) != cudaSuccess) return e;
-    decode_int4_kernel<D, G, KV4_F32><<<ctas, kWarps * 32, smem, st>>>(a);
+    e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_F32>, a);
   } else if (a.q_dtype == KV4_BF16) {
     if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_BF16>, smem, done[1])) != cudaSuccess) return e;
-    decode_int4_kernel<D, G, KV4_BF16><<<ctas, kWarps * 32, smem, st>>>(a);
+    e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_BF16>, a);
   } else {
     if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F16>, smem, done[2])) != cudaSuccess) return e;
-    decode_int4_kernel<D, G, KV4_F16><<<ctas, kWarps * 32, smem, st>>>(a);
+    e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_F16>, a);
   }
-  cudaError_t le = cudaGetLastError();
-  if (le != cudaSuccess) return le;
+  if (e != cudaSuccess) return e;
   return launch_merge<D, G>(a, st);
 }
 

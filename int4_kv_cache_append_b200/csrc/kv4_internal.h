@@ -44,6 +44,7 @@ struct DecodeArgs {
   float qscale;           // softmax scale in log2 units: log2(e) / sqrt(D)
   int W;                  // warps launched by the partial kernel
   int tp_shift;           // log2(P / 16) when P / 16 is a power of two, else -1
+  int early;              // build the schedule before waiting on the preceding kernel
   uint32_t* err;
 };
 

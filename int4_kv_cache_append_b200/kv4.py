@@ -26,7 +26,7 @@ KV4_DEVERR_PAGE_RANGE, KV4_DEVERR_WAIT_LIMIT, KV4_DEVERR_LENGTH = 0x1, 0x2, 0x4
 # every entry point declared in include/kv4.h
 SYMBOLS = (
     "kv4_query_sizes", "kv4_cache_init", "kv4_cache_destroy", "kv4_append", "kv4_decode_workspace_bytes",
-    "kv4_decode_attn", "kv4_decode_attn_static", "kv4_bf16_query_sizes", "kv4_bf16_cache_init", "kv4_bf16_append",
+    "kv4_decode_attn", "kv4_decode_attn_static", "kv4_set_decode_overlap", "kv4_bf16_query_sizes", "kv4_bf16_cache_init", "kv4_bf16_append",
     "kv4_bf16_decode_workspace_bytes", "kv4_bf16_decode_attn", "kv4_get_device_error", "kv4_launch_count",
     "kv4_status_string", "kv4_version",
 )
@@ -59,6 +59,7 @@ def _load():
         "kv4_decode_workspace_bytes": (I, [P, I, ctypes.POINTER(S)]),
         "kv4_decode_attn": (I, [P, I, I, P, I, i32p, I, i32p, I, P, P, P, S, P]),
         "kv4_decode_attn_static": (I, [P, I, I, P, I, i32p, I, i32p, I, P, P, P]),
+        "kv4_set_decode_overlap": (I, [P, I]),
         "kv4_bf16_query_sizes": (I, [cfgp, ctypes.POINTER(S)]),
         "kv4_bf16_cache_init": (I, [cfgp, P, ctypes.POINTER(P)]),
         "kv4_bf16_append": (I, [P, I, I, P, I, P, I, i32p, i32p, i32p, I, P]),
@@ -162,6 +163,12 @@ def kv4_decode_attn_static(handle, layer, B, q, q_dtype, page_table, stride, len
 KV4_STATIC_SCRATCH_BYTES = 16 << 20
 
 
+def kv4_set_decode_overlap(handle, enable: bool):
+    """With enable, the decode kernel builds its schedule from lens and page_table while the
+    preceding kernel on the stream runs (they must not be written by that kernel)."""
+    _check("kv4_set_decode_overlap", lib.kv4_set_decode_overlap(handle, 1 if enable else 0))
+
+
 def kv4_bf16_query_sizes(cfg: kv4_config) -> int:
     pool = ctypes.c_size_t()
     _check("kv4_bf16_query_sizes", lib.kv4_bf16_query_sizes(ctypes.byref(cfg), ctypes.byref(pool)))
@@ -253,7 +260,7 @@ class Cache:
     def workspace(self, B: int) -> torch.Tensor:
         n = kv4_decode_workspace_bytes(self.handle, B)
         if self._ws is None or self._ws.numel() < n:
-            self._ws = torch.zeros(n, dtype=torch.uint8, device=self.pool.device)  # zero once
+            self._ws = torch.empty(n, dtype=torch.uint8, device=self.pool.device)
         return self._ws
 
     def decode(self, layer, q, page_table, lens, out=None, lse=None, max_len_hint=0, workspace=None, stream=None):
@@ -294,7 +301,7 @@ class BF16Cache:
     def workspace(self, B: int) -> torch.Tensor:
         n = kv4_bf16_decode_workspace_bytes(self.handle, B)
         if self._ws is None or self._ws.numel() < n:
-            self._ws = torch.zeros(n, dtype=torch.uint8, device=self.pool.device)  # zero once
+            self._ws = torch.empty(n, dtype=torch.uint8, device=self.pool.device)
         return self._ws
 
     def decode(self, layer, q, page_table, lens, out=None, lse=None, max_len_hint=0, workspace=None, stream=None):

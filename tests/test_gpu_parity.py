@@ -189,3 +189,33 @@ def test_bf16_baseline_matches_reference(case):
     loose = q.dtype != np.uint16
     T.assert_close(out.cpu().numpy(), ref, lse.cpu().numpy(), ref_lse, atol=2e-2 if loose else 2e-3,
                    rel_l2=5e-3 if loose else 1e-3, lse_atol=1e-3 if loose else 1e-4, what="bf16 " + case[0])
+
+
+@pytest.mark.parametrize("overlap", [False, True], ids=["stream-order", "overlap"])
+def test_append_then_decode_on_one_stream(overlap):
+    """The decode kernel launched right after an append on the same stream (the append lets its
+    dependent launch early; with overlap the decode builds its schedule before waiting on the
+    append): the result is the oracle's, and identical with and without overlap."""
+    from int4_kv_cache_append_b200 import kv4
+    wl = make(CASES[1])
+    gc = T.gpu_cache_from_host_inputs(wl, lens=wl.lens - 1)  # every sequence short of its last token
+    cfg, pool, side = T.oracle_cache(wl)
+    q = wl.q_input(0)
+    ref, ref_lse = T.oracle_decode(wl, cfg, pool, side, q)
+    rows = np.nonzero(wl.lens > 0)[0].astype(np.int32)
+    pos = (wl.lens[rows] - 1).astype(np.int32)
+    K, V = wl.kv_inputs(0, rows, pos)
+    pt = torch.from_numpy(wl.page_table).cuda()
+    lens = torch.from_numpy(wl.lens).cuda()
+    kv4.kv4_set_decode_overlap(gc.handle, overlap)
+    outs = []
+    for _ in range(2):
+        gc.append(0, T.to_dev(K), T.to_dev(V), torch.from_numpy(rows).cuda(), torch.from_numpy(pos).cuda(), lens, pt)
+        lse = torch.empty((wl.B, wl.Hq), device="cuda")
+        out = gc.decode(0, T.to_dev(q), pt, lens, lse=lse)
+        torch.cuda.synchronize()
+        outs.append((out.cpu().numpy(), lse.cpu().numpy()))
+    kv4.kv4_set_decode_overlap(gc.handle, False)
+    T.assert_close(outs[0][0], ref, outs[0][1], ref_lse, what=f"append->decode overlap={overlap}")
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+    assert kv4.kv4_get_device_error() == 0
