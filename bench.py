@@ -399,7 +399,7 @@ def run_kv4(args, world, rank, local):
     achieved = alg_bytes / (dec_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": profiled_traffic(wl.name),
-            "kernel": "decode_int4_kernel (kv4_decode_attn: split-K tiles + in-kernel merge, one launch)",
+            "kernel": "decode_int4_kernel + merge_int4_kernel (kv4_decode_attn: split-K tiles, then LSE merge)",
             "bytes_per_launch": alg_bytes, "kv_bytes_per_launch": kv_bytes, "decode_ms": round(dec_ms, 5),
             "peak_source": f"{peak_kind} MEASURED_PEAKS.json hbm_gbs" if peak_kind == "measured" else "fallback"}
     spec_frac = achieved / 8000.0
@@ -476,7 +476,7 @@ def run_kv4(args, world, rank, local):
             "config": {"workload": wl.name, "B_per_gpu": B, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": wl.D, "P": wl.P,
                        "s": wl.s, "w": wl.w, "h": wl.h, "len_mean": round(float(lens.mean()), 1),
                        "len_max": maxlen, "kv_dtype": "int4 pages + int8 side cache",
-                       "compute": "f16 tensor-core operands, f32 accumulate/softmax",
+                       "compute": "QK^T int8 MMA (exact int32), PV f16 MMA with f32 accumulate, f32 softmax",
                        "l2": "inputs larger than L2: 4 resident layers cycled, 0.72 GB of KV between reuses",
                        "parallelism": f"dp{world} (independent batches per GPU, no collective)",
                        "graph": not args.no_graph, "decode_overlap": args.overlap,

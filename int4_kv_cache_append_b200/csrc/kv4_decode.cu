@@ -538,6 +538,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
       for (int e = lane; e < a.Hq * D; e += 32) a.out[static_cast<size_t>(b) * a.Hq * D + e] = 0.f;
       if (a.lse)
         for (int e = lane; e < a.Hq; e += 32) a.lse[static_cast<size_t>(b) * a.Hq + e] = kNegInf;
+      for (int g = lane; g < a.Hkv; g += 32) *reinterpret_cast<uint4*>(a.meta + 4 * (b * a.Hkv + g)) = make_uint4(0u, 0u, 0u, 0u);
     }
   }
   __syncwarp();
@@ -976,8 +977,8 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
 // one pass, 32 at a time: lanes read the (m, l) of 32 partials, the running maximum is raised to
 // their maximum (rescaling the sums so far), and their o rows are read kInFlight at a time with
 // independent loads.  With MW = 4, warp 0 combines the warps' (M, L, o) through shared memory.
-// (b, g) with at most one partial were written by the decode kernel; sequences of length 0 were
-// written by it too and have no meta.  Launched as a programmatic dependent of the decode kernel:
+// (b, g) with at most one partial, and sequences of length 0 (record of zeros), were written by
+// the decode kernel.  Launched as a programmatic dependent of the decode kernel:
 // griddepcontrol.wait orders every read of its results after its completion.
 constexpr int kMergeThreads = 128;
 
@@ -995,9 +996,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_int4_kernel(const DecodeA
   if (item >= a.B * a.Hq) return;
   const int b = item / a.Hq, j = item - b * a.Hq;
   const int g = j / G, hd = j - g * G;
-  const int cap = a.stride * a.P;
   pdl_wait();
-  if (clamp_len(a.lens[b], cap) == 0) return;
   const uint4 mt = *reinterpret_cast<const uint4*>(a.meta + 4 * (b * a.Hkv + g));
   const int n8p = static_cast<int>(mt.z), n = static_cast<int>(mt.z + mt.w);
   if (n <= 1) return;  // uniform over the item's warps
