@@ -238,6 +238,19 @@ def async_refill(B: int = 256) -> Workload:
                          F32, BF16, BF16, 2, 20.0)
 
 
+def async_refill_snapshot(B: int = 256) -> Workload:
+    """The async-refill shape drawn as a step of continuous refill rather than i.i.d. lengths:
+    B slots, ceil(Exp(6144)) response lengths capped at 32768, context lengths of the slots at a
+    random steady-state step (length-biased responses, uniform position; see concentration.py).
+    Other parameters as async_refill."""
+    from . import concentration as C
+
+    def lens(r):
+        return C.async_snapshot(C.exponential_lengths(6144.0, 32768), B, r, cap=32768)
+    return make_workload(f"async-refill-snapshot-B{B}", 5, 1, B, 32, 8, 128, 16, 4, 128, 64, lens,
+                         F32, BF16, BF16, 2, 20.0)
+
+
 def long_context() -> Workload:
     """4 sequences of 32K/64K/128K/128K, 32q/8kv, D=128, P=64, s=4, w=256, h=128."""
     return make_workload("long-context-32k-128k", 3, 1, 4, 32, 8, 128, 64, 4, 256, 128,
@@ -256,6 +269,7 @@ WORKLOADS = {
     "tiny": tiny_cfg,
     "qwen3-4b-decode": qwen3_4b_decode,
     "async-refill": async_refill,
+    "async-refill-snapshot": async_refill_snapshot,
     "long-context": long_context,
     "qwen3-8b-loop": qwen3_8b_loop,
 }

@@ -26,6 +26,9 @@ CASES = [
     ("d128-g4-sinks-only", 128, 4, 1, 16, 8, 0, 16, (40, 8, 3), W.F32, W.F32, W.BF16),
     ("d64-g4-recent-only", 64, 8, 2, 16, 0, 24, 64, (90, 24, 25, 2), W.BF16, W.F32, W.F32),
     ("d128-g4-wide-s", 128, 4, 1, 16, 19, 13, 128, (100, 19, 20, 31, 32, 33), W.BF16, W.BF16, W.BF16),
+    # KV8: no sinks and a recent window longer than every sequence, so every position is read
+    # from the INT8 side cache
+    ("d128-g4-kv8", 128, 8, 2, 16, 0, 208, 128, (200, 77, 1, 16, 17), W.BF16, W.BF16, W.BF16),
 ]
 
 
