@@ -145,6 +145,17 @@ kv4_status kv4_decode_attn(kv4_cache* cache, int layer, int B, const void* q, kv
                            float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * kv4_set_rotation_signs: randomised-sign Hadamard rotation for this cache (a precision variant;
+ * default: none).  Bit d of sign_bits (host array of ceil(head_dim / 32) words, bit d % 32 of word
+ * d / 32) negates key dimension d before the block Hadamard at append, and query dimension d
+ * before the query rotation at decode, so the rotation is H diag(s) with s in {+1, -1}; the
+ * attention is unchanged in exact arithmetic.  NULL clears it.  The signs are part of the stored
+ * format: set them before the first append to the cache and keep them.  Returns
+ * KV4_ERR_INVALID_ARG for a NULL or BF16 cache.
+ */
+kv4_status kv4_set_rotation_signs(kv4_cache* cache, const uint32_t* sign_bits);
+
+/*
  * kv4_set_decode_overlap: how kv4_decode_attn of this cache starts (default 0).  Its kernel is
  * always launched as a programmatic dependent of the preceding kernel on the stream, and the
  * append kernel lets its dependent launch early.  With 0 the decode kernel reads nothing before

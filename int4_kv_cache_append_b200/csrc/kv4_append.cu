@@ -158,6 +158,12 @@ __global__ void __launch_bounds__(256) append_int4_kernel(AppendArgs a) {
     load4<KT>(a.K, in0, k);
     load4<VT>(a.V, in0, v);
   }
+  {
+    // randomised-sign rotation: dims of set bits are negated first (exact: the sign bit flips)
+    const uint32_t sb = (a.signs[lane >> 3] >> (4 * (lane & 7))) & 15u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) k[e] = __uint_as_float(__float_as_uint(k[e]) ^ (((sb >> e) & 1u) << 31));
+  }
   hadamard4(k, lane, a.h);
 
   const int pp = pos % a.P, r = pp & 15;

@@ -581,6 +581,14 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   auto build_query = [&](uint8_t* scratch) {
     const bool act = lane < D / 4;
     const int h = a.h;
+    {
+      // the keys' randomised signs (lane holds dims 4 lane .. 4 lane + 3)
+      const uint32_t sb = act ? (a.signs[lane >> 3] >> (4 * (lane & 7))) & 15u : 0u;
+#pragma unroll
+      for (int i = 0; i < G; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) qx[i][e] = __uint_as_float(__float_as_uint(qx[i][e]) ^ (((sb >> e) & 1u) << 31));
+    }
     // Butterfly strides 1 and 2 within the lane, then 4 .. h/2 across lanes (lane xor stride/4),
     // every stage over all G heads so that their shuffles overlap.
 #pragma unroll

@@ -130,6 +130,16 @@ void orc_fwht_f32(float* x, int D, int h) {
         }
 }
 
+/* Randomised-sign variant (a precision variant of the rotation; signs all zero by default): the
+ * sign of dimension d is flipped first, so the stored basis is H diag(s). */
+static int orc_sign(const orc_config* c, int d) { return (int)((c->sign_bits[d >> 5] >> (d & 31)) & 1u); }
+
+void orc_rotate_key(const orc_config* c, float* x) {
+  for (int e = 0; e < c->head_dim; ++e)
+    if (orc_sign(c, e)) x[e] = -x[e];
+  orc_fwht_f32(x, c->head_dim, c->hadamard_block);
+}
+
 void orc_fwht_f64(double* x, int D, int h) {
   for (int b0 = 0; b0 < D; b0 += h)
     for (int st = 1; st < h; st <<= 1)
@@ -344,7 +354,7 @@ int orc_append(const orc_config* c, uint8_t* pool, uint8_t* side, int T, const v
         kf[e] = (float)load_elem(K, k_dtype, in0 + (size_t)e);
         vf[e] = (float)load_elem(V, v_dtype, in0 + (size_t)e);
       }
-      orc_fwht_f32(kf, D, c->hadamard_block);
+      orc_rotate_key(c, kf);
       uint16_t sc, zr;
       orc_quant_int4(kf, D, c4, &sc, &zr);
       for (int e = 0; e < D; ++e) put_nibble(pool, orc_k4_byte(c, page, g, pp, e), e & 1, c4[e]);
@@ -497,6 +507,8 @@ int orc_decode(const orc_config* c, const uint8_t* pool, const uint8_t* side, in
         const size_t qh = (size_t)b * (size_t)Hq + (size_t)(g * G + i);
         /* [KV4-RL Meth.2] queries rotated to match the stored key basis: (H q) / h. */
         for (int e = 0; e < D; ++e) qr[e] = load_elem(q, q_dtype, qh * (size_t)D + (size_t)e);
+        for (int e = 0; e < D; ++e)
+          if (orc_sign(c, e)) qr[e] = -qr[e];
         orc_fwht_f64(qr, D, h);
         for (int e = 0; e < D; ++e) qr[e] *= 1.0 / (double)h;
         for (int j = 0; j < L; ++j) {

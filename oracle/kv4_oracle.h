@@ -43,6 +43,8 @@ typedef struct {
   int recent_window;   /* w                                            */
   int hadamard_block;  /* h, power of two dividing D (1 = no rotation) */
   int max_seqs;        /* rows of the INT8 side cache                  */
+  uint32_t sign_bits[4]; /* randomised-sign rotation: bit d (word d / 32) negates dim d of the
+                            key and of the query before the Hadamard; all zero = plain H    */
 } orc_config;
 
 /* fp16 helpers (IEEE binary16), written from the format definition. */
@@ -54,6 +56,8 @@ float    orc_bf16_to_f32(uint16_t b);
 void orc_fwht_f32(float* x, int D, int h);
 /* Same transform in fp64 (used for the query rotation). */
 void orc_fwht_f64(double* x, int D, int h);
+/* The key rotation of the append: H diag(s) x, the configured signs, then orc_fwht_f32. */
+void orc_rotate_key(const orc_config* c, float* x);
 
 /* Per-vector quantisers.  codes4 holds one code (0..15) per element, unpacked. */
 void orc_quant_int4(const float* x, int D, uint8_t* codes4, uint16_t* scale, uint16_t* zero);

@@ -46,7 +46,7 @@ def build(force: bool = False) -> str:
 class _Cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "num_q_heads", "num_kv_heads", "head_dim", "page_size", "num_sinks",
-        "recent_window", "hadamard_block", "max_seqs")]
+        "recent_window", "hadamard_block", "max_seqs")] + [("sign_bits", ctypes.c_uint32 * 4)]
 
 
 @dataclass(frozen=True)
@@ -60,10 +60,12 @@ class Config:
     recent_window: int
     hadamard_block: int
     max_seqs: int
+    sign_bits: tuple = (0, 0, 0, 0)  # randomised-sign rotation (bit d negates dim d); zero = plain
 
     def c(self) -> _Cfg:
         return _Cfg(self.num_q_heads, self.num_kv_heads, self.head_dim, self.page_size,
-                    self.num_sinks, self.recent_window, self.hadamard_block, self.max_seqs)
+                    self.num_sinks, self.recent_window, self.hadamard_block, self.max_seqs,
+                    (ctypes.c_uint32 * 4)(*[int(x) & 0xFFFFFFFF for x in (list(self.sign_bits) + [0] * 4)[:4]]))
 
 
 _lib = None
@@ -88,6 +90,7 @@ def lib():
         L.orc_bf16_to_f32.restype = ctypes.c_float
         L.orc_fwht_f32.argtypes = [P, I, I]
         L.orc_fwht_f64.argtypes = [P, I, I]
+        L.orc_rotate_key.argtypes = [ctypes.POINTER(_Cfg), P]
         L.orc_quant_int4.argtypes = [P, I, P, P, P]
         L.orc_quant_int8.argtypes = [P, I, P, P]
         for n in ("orc_page_bytes", "orc_side_slot_bytes"):
@@ -132,6 +135,15 @@ def bf16_to_f32(bits: int) -> float:
 def fwht_f32(x: np.ndarray, h: int) -> np.ndarray:
     y = np.ascontiguousarray(x, dtype=np.float32).copy()
     lib().orc_fwht_f32(_p(y), y.size, h)
+    return y
+
+
+def rotate_key(cfg: "Config", x: np.ndarray) -> np.ndarray:
+    """The append's key rotation H diag(s) x (fp32)."""
+    y = np.ascontiguousarray(x, dtype=np.float32).copy()
+    assert y.size == cfg.head_dim
+    c = cfg.c()
+    lib().orc_rotate_key(ctypes.byref(c), _p(y))
     return y
 
 

@@ -281,10 +281,11 @@ def pin_layout_bijection():
 
 # ----------------------------------------------------------------------------- cache helpers
 
-def build_cache(wl: W.Workload, layer: int = 0, lens=None, step_by_step: bool = False, sentinel: int = 0xA5):
+def build_cache(wl: W.Workload, layer: int = 0, lens=None, step_by_step: bool = False, sentinel: int = 0xA5,
+                signs=(0, 0, 0, 0)):
     """Oracle cache for a workload: prefill every token in position order (one call for all
     tokens with lens_after = L, or one call per position with lens_after = pos + 1)."""
-    cfg = oracle_cfg(wl)
+    cfg = oracle_cfg(wl, signs)
     lens = np.asarray(wl.lens if lens is None else lens, np.int32)
     pool = np.full(O.page_bytes(cfg) * wl.num_pages, sentinel, np.uint8)
     side = np.full(O.side_slot_bytes(cfg) * wl.B, sentinel, np.uint8)
@@ -306,8 +307,8 @@ def build_cache(wl: W.Workload, layer: int = 0, lens=None, step_by_step: bool = 
     return cfg, pool, side
 
 
-def oracle_cfg(wl: W.Workload) -> O.Config:
-    return O.Config(wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h, wl.B)
+def oracle_cfg(wl: W.Workload, signs=(0, 0, 0, 0)) -> O.Config:
+    return O.Config(wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h, wl.B, tuple(signs))
 
 
 def small_workload(D=32, B=3, lens=(12, 7, 40), s=2, w=5, h=8, G=2, Hkv=2, P=16, seed=5,
@@ -457,17 +458,40 @@ def pin_regional_equals_single(seed: int = 41):
             assert np.abs(l1 - l2).max() <= 1e-12 * max(1.0, np.abs(l1).max())
 
 
+def sign_vector(words, D: int) -> np.ndarray:
+    return np.array([-1.0 if (int(words[d >> 5]) >> (d & 31)) & 1 else 1.0 for d in range(D)])
+
+
+def pin_signed_rotation_exact(seed: int = 53):
+    """The append's key rotation with randomised signs is H diag(s) x: on integer vectors the fp32
+    butterfly equals the explicit matrix product exactly."""
+    rng = np.random.default_rng(seed)
+    for D in (32, 64):
+        for h in (1, 8, D):
+            words = tuple(int(x) for x in rng.integers(0, 2**32, size=4, dtype=np.uint64))
+            cfg = O.Config(2, 1, D, 16, 2, 4, h, 1, words)
+            Hm = np.kron(np.eye(D // h), scipy.linalg.hadamard(h)).astype(np.float64)
+            S = sign_vector(words, D)
+            for _ in range(5):
+                x = rng.integers(-7, 8, size=D).astype(np.float32)
+                assert np.array_equal(O.rotate_key(cfg, x).astype(np.float64), Hm @ (S * x))
+
+
 def pin_rotation_invariance(seed: int = 51):
-    """tau * q_rot . khat_rot equals tau * q . (H^T khat_rot / h): the stored rotated keys seen
-    by the unrotated query through the inverse transform (H^T H = h I)."""
-    for h in (1, 8, 32):
+    """tau * q_rot . khat_rot equals tau * q . (diag(s) H^T khat_rot / h): the stored rotated keys
+    seen by the unrotated query through the inverse transform (H^T H = h I, s_d^2 = 1), with and
+    without randomised signs."""
+    rng = np.random.default_rng(seed)
+    for h, words in ((1, (0, 0, 0, 0)), (8, (0, 0, 0, 0)), (32, (0, 0, 0, 0)),
+                     (8, tuple(int(x) for x in rng.integers(0, 2**32, size=4, dtype=np.uint64))),
+                     (32, tuple(int(x) for x in rng.integers(0, 2**32, size=4, dtype=np.uint64)))):
         wl = small_workload(D=32, lens=(30,), B=1, s=2, w=4, h=h, seed=seed)
-        cfg, pool, side = build_cache(wl)
+        cfg, pool, side = build_cache(wl, signs=words)
         q = wl.q_input(0)
         out, _ = O.decode(cfg, pool, side, q, wl.page_table, wl.lens, mode=O.SINGLE)
         Hm = np.kron(np.eye(wl.D // h), scipy.linalg.hadamard(h)).astype(np.float64)
         kd, vd, _ = O.dequant_seq(cfg, pool, side, wl.page_table[0], 0, 30, 0)
-        k_unrot = kd @ Hm / h             # rows: (H^T khat) / h, H symmetric
+        k_unrot = (kd @ Hm / h) * sign_vector(words, wl.D)[None, :]  # rows: diag(s) H^T khat / h
         for i in range(wl.G):
             logits = k_unrot @ q[0, i].astype(np.float64) / np.sqrt(wl.D)
             p = np.exp(logits - logits.max())
@@ -518,5 +542,5 @@ ALL_PINS = [
     pin_quant_int4_constant, pin_quant_int8_bounds, pin_storage_bits, pin_layout_bijection,
     lambda: pin_routing(False), lambda: pin_routing(True), pin_brute_force,
     pin_append_vs_numpy_requant, pin_regional_equals_single, pin_rotation_invariance,
-    pin_special_cases,
+    pin_special_cases, pin_signed_rotation_exact,
 ]

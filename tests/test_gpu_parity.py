@@ -29,6 +29,10 @@ CASES = [
     # KV8: no sinks and a recent window longer than every sequence, so every position is read
     # from the INT8 side cache
     ("d128-g4-kv8", 128, 8, 2, 16, 0, 208, 128, (200, 77, 1, 16, 17), W.BF16, W.BF16, W.BF16),
+    # more than 256 sequences: the decode prologue reads the lengths from memory instead of
+    # keeping them in registers
+    ("d64-g2-b300", 64, 4, 2, 16, 4, 16, 64,
+     tuple(int(x) for x in np.random.default_rng(300).integers(0, 90, size=300)), W.BF16, W.BF16, W.BF16),
 ]
 
 
@@ -222,3 +226,26 @@ def test_append_then_decode_on_one_stream(overlap):
     T.assert_close(outs[0][0], ref, outs[0][1], ref_lse, what=f"append->decode overlap={overlap}")
     assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
     assert kv4.kv4_get_device_error() == 0
+
+
+@pytest.mark.parametrize("case_id", [1, 3], ids=["d128-h128", "d64-h1"])
+def test_randomised_sign_rotation(case_id):
+    """kv4_set_rotation_signs: keys stored in the H diag(s) basis are bit-exact against the oracle's
+    same reading, and the decode (query rotated with the same signs) matches it."""
+    from int4_kv_cache_append_b200 import kv4
+    wl = make(CASES[case_id])
+    words = [int(x) for x in np.random.default_rng(77 + case_id).integers(0, 2**32, size=4, dtype=np.uint64)]
+    words = words[:(wl.D + 31) // 32] + [0] * (4 - (wl.D + 31) // 32)
+    gc = T.gpu_cache_from_host_inputs(wl, signs=words)
+    cfg, pool, side = T.oracle_cache(wl, signs=words)
+    gp, gs = gc.layer_views(0)
+    assert np.array_equal(gp.cpu().numpy(), pool) and np.array_equal(gs.cpu().numpy(), side)
+    q = wl.q_input(0)
+    ref, ref_lse = T.oracle_decode(wl, cfg, pool, side, q)
+    out, lse = T.gpu_decode(gc, wl, q)
+    T.assert_close(out, ref, lse, ref_lse, what=f"signed rotation {CASES[case_id][0]}")
+    # without the signs the stored keys differ (the option is not a no-op)
+    plain = T.oracle_cache(wl)[1]
+    assert not np.array_equal(plain, pool)
+    assert kv4.kv4_get_device_error() == 0
+

@@ -34,6 +34,8 @@ MUTANTS = [
     ("ring-row-no-offset", "row = s + p % w;", "row = p % w;", None),
     ("q-rot-sqrt-norm", "qr[e] *= 1.0 / (double)h;", "qr[e] *= 1.0 / sqrt((double)h);", None),
     ("q-not-rotated", "orc_fwht_f64(qr, D, h);", ";", None),
+    ("q-signs-ignored", "if (orc_sign(c, e)) qr[e] = -qr[e];", ";", None),
+    ("k-signs-ignored", "if (orc_sign(c, e)) x[e] = -x[e];", ";", None),
     ("tau-wrong", "1.0 / sqrt((double)D)", "1.0 / (double)D", None),
     ("merge-no-rescale-l", "l += parts[i].l * f;", "l += parts[i].l;", None),
     ("merge-no-rescale-o", "out[e] += parts[i].o[e] * f;", "out[e] += parts[i].o[e];", None),
