@@ -156,6 +156,15 @@ kv4_status kv4_decode_attn(kv4_cache* cache, int layer, int B, const void* q, kv
 kv4_status kv4_set_rotation_signs(kv4_cache* cache, const uint32_t* sign_bits);
 
 /*
+ * kv4_set_value_rotation: store values in the keys' rotated basis too (a precision variant;
+ * default 0).  With 1 the append applies H diag(s) to V before quantising (INT4 and INT8 copies),
+ * and the decode's merge returns every output to the original basis, out = diag(s) H o / h.  This
+ * is part of the stored format: set it before the first append and keep it.  Returns
+ * KV4_ERR_INVALID_ARG for a NULL or BF16 cache.
+ */
+kv4_status kv4_set_value_rotation(kv4_cache* cache, int enable);
+
+/*
  * kv4_set_decode_overlap: how kv4_decode_attn of this cache starts (default 0).  Its kernel is
  * always launched as a programmatic dependent of the preceding kernel on the stream, and the
  * append kernel lets its dependent launch early.  With 0 the decode kernel reads nothing before

@@ -39,6 +39,7 @@ struct kv4_cache {
   int nt8;
   int overlap;        // kv4_set_decode_overlap
   uint32_t signs[4];  // kv4_set_rotation_signs
+  int rotate_v;       // kv4_set_value_rotation
 };
 
 namespace kv4 {
@@ -148,6 +149,7 @@ kv4_status append_common(kv4_cache* c, int fmt, int layer, int T, const void* K,
   a.page_bytes = c->page_bytes;
   a.side_slot_bytes = c->side_slot_bytes;
   for (int i = 0; i < 4; ++i) a.signs[i] = fmt == FMT_INT4 ? c->signs[i] : 0u;
+  a.rotate_v = fmt == FMT_INT4 ? c->rotate_v : 0;
   a.err = err;
   const cudaError_t e = fmt == FMT_INT4 ? kv4::launch_append_int4(a, c->cfg.head_dim, static_cast<cudaStream_t>(stream))
                                         : kv4::launch_append_bf16(a, c->cfg.head_dim, static_cast<cudaStream_t>(stream));
@@ -218,6 +220,7 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
     const int tpp = c->cfg.page_size / 16;
     a.early = (fmt == FMT_INT4 && c->overlap) ? 1 : 0;
   for (int i = 0; i < 4; ++i) a.signs[i] = c->signs[i];
+  a.rotate_v = fmt == FMT_INT4 ? c->rotate_v : 0;
   a.tp_shift = pow2(tpp) ? __builtin_ctz(static_cast<unsigned>(tpp)) : -1;
   }
   const int G = c->cfg.num_q_heads / c->cfg.num_kv_heads;
@@ -309,6 +312,12 @@ kv4_status kv4_set_rotation_signs(kv4_cache* cache, const uint32_t* sign_bits) {
   if (!cache || cache->format != FMT_INT4) return KV4_ERR_INVALID_ARG;
   const int words = (cache->cfg.head_dim + 31) / 32;
   for (int i = 0; i < 4; ++i) cache->signs[i] = (sign_bits && i < words) ? sign_bits[i] : 0u;
+  return KV4_OK;
+}
+
+kv4_status kv4_set_value_rotation(kv4_cache* cache, int enable) {
+  if (!cache || cache->format != FMT_INT4) return KV4_ERR_INVALID_ARG;
+  cache->rotate_v = enable ? 1 : 0;
   return KV4_OK;
 }
 

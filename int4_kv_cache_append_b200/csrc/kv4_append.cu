@@ -165,6 +165,12 @@ __global__ void __launch_bounds__(256) append_int4_kernel(AppendArgs a) {
     for (int e = 0; e < 4; ++e) k[e] = __uint_as_float(__float_as_uint(k[e]) ^ (((sb >> e) & 1u) << 31));
   }
   hadamard4(k, lane, a.h);
+  if (a.rotate_v) {  // value rotation: the same H diag(s) as the keys
+    const uint32_t sb = (a.signs[lane >> 3] >> (4 * (lane & 7))) & 15u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = __uint_as_float(__float_as_uint(v[e]) ^ (((sb >> e) & 1u) << 31));
+    hadamard4(v, lane, a.h);
+  }
 
   const int pp = pos % a.P, r = pp & 15;
   uint8_t* tile = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(g) * a.P * (D + 8) +

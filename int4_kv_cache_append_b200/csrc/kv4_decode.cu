@@ -742,7 +742,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     const u32 w8a = divQ.div(cs8), w4a = divQ.div(cs4);
     const u32 n8p = si.n8 ? divQ.div(cs4 - 2) - w8a + 1 : 0u;
     const u32 n4p = si.n4 ? divQ.div(cs4 + si.n4 - 1) - w4a + 1 : 0u;
-    const bool only = n8p + n4p == 1u;
+    const bool only = n8p + n4p == 1u && !a.rotate_v;  // rotated values: the merge rotates back
     const u32 sid = 2u * static_cast<u32>(cb * a.Hkv + cg) + static_cast<u32>(cseg);
     // where the merge finds the partials of (b, g); every writer of (b, g) stores the same record
     if (lane == 0) *reinterpret_cast<uint4*>(a.meta + 4 * (cb * a.Hkv + cg)) = make_uint4(w8a, w4a, n8p, n4p);
@@ -1007,7 +1007,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_int4_kernel(const DecodeA
   pdl_wait();
   const uint4 mt = *reinterpret_cast<const uint4*>(a.meta + 4 * (b * a.Hkv + g));
   const int n8p = static_cast<int>(mt.z), n = static_cast<int>(mt.z + mt.w);
-  if (n <= 1) return;  // uniform over the item's warps
+  if (n == 0 || (n == 1 && !a.rotate_v)) return;  // uniform over the item's warps
   const PartRows pr{n8p, mt.x, mt.y, 2u * static_cast<u32>(b * a.Hkv + g)};
   const int t0 = sub * n / MW, t1 = (sub + 1) * n / MW;
   float M = kNegInf, L = 0.f, o[PER];
@@ -1080,10 +1080,43 @@ __global__ void __launch_bounds__(kMergeThreads) merge_int4_kernel(const DecodeA
   }
   float* out = a.out + (static_cast<size_t>(b) * a.Hq + j) * D + lane * PER;
   const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) o[e] *= inv;
+  if (a.rotate_v) {
+    // values were stored as H diag(s) v: o = diag(s) H o_rot / h (lane holds dims PER lane + e)
+    const int h = a.h;
+#pragma unroll
+    for (int st = 1; st < PER; st <<= 1)
+      if (st < h)
+#pragma unroll
+        for (int e = 0; e < PER; ++e)
+          if ((e & st) == 0) {
+            const float x0 = o[e], x1 = o[e + st];
+            o[e] = x0 + x1;
+            o[e + st] = x0 - x1;
+          }
+#pragma unroll
+    for (int st = PER; st < D; st <<= 1)
+      if (st < h) {
+        const int m = st / PER;
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+          const float x = __shfl_xor_sync(FULL, o[e], m);
+          o[e] = upper ? x - o[e] : o[e] + x;
+        }
+      }
+    const float ih = 1.f / static_cast<float>(h);
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      const int d = lane * PER + e;
+      o[e] = __uint_as_float(__float_as_uint(o[e] * ih) ^ (((a.signs[d >> 5] >> (d & 31)) & 1u) << 31));
+    }
+  }
   if constexpr (PER == 4)
-    *reinterpret_cast<float4*>(out) = make_float4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
+    *reinterpret_cast<float4*>(out) = make_float4(o[0], o[1], o[2], o[3]);
   else
-    *reinterpret_cast<float2*>(out) = make_float2(o[0] * inv, o[1] * inv);
+    *reinterpret_cast<float2*>(out) = make_float2(o[0], o[1]);
   if (a.lse && lane == 0) a.lse[static_cast<size_t>(b) * a.Hq + j] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : kNegInf;
 }
 

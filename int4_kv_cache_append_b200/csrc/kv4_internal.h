@@ -25,6 +25,7 @@ struct AppendArgs {
   int T, Hkv, P, s, w, h, max_seqs, max_pages, nt8;
   size_t page_bytes, side_slot_bytes;
   uint32_t signs[4];      // bit d: key dim d negated before the rotation (randomised-sign Hadamard)
+  int rotate_v;           // values stored in the keys' rotated basis too
   uint32_t* err;
 };
 
@@ -47,6 +48,7 @@ struct DecodeArgs {
   int tp_shift;           // log2(P / 16) when P / 16 is a power of two, else -1
   int early;              // build the schedule before waiting on the preceding kernel
   uint32_t signs[4];      // bit d: query dim d negated before the rotation (as the keys)
+  int rotate_v;           // values stored rotated: outputs are rotated back by the merge kernel
   uint32_t* err;
 };
 

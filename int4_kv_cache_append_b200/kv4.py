@@ -26,7 +26,7 @@ KV4_DEVERR_PAGE_RANGE, KV4_DEVERR_WAIT_LIMIT, KV4_DEVERR_LENGTH = 0x1, 0x2, 0x4
 # every entry point declared in include/kv4.h
 SYMBOLS = (
     "kv4_query_sizes", "kv4_cache_init", "kv4_cache_destroy", "kv4_append", "kv4_decode_workspace_bytes",
-    "kv4_decode_attn", "kv4_decode_attn_static", "kv4_set_decode_overlap", "kv4_set_rotation_signs", "kv4_bf16_query_sizes", "kv4_bf16_cache_init", "kv4_bf16_append",
+    "kv4_decode_attn", "kv4_decode_attn_static", "kv4_set_decode_overlap", "kv4_set_rotation_signs", "kv4_set_value_rotation", "kv4_bf16_query_sizes", "kv4_bf16_cache_init", "kv4_bf16_append",
     "kv4_bf16_decode_workspace_bytes", "kv4_bf16_decode_attn", "kv4_get_device_error", "kv4_launch_count",
     "kv4_status_string", "kv4_version",
 )
@@ -61,6 +61,7 @@ def _load():
         "kv4_decode_attn_static": (I, [P, I, I, P, I, i32p, I, i32p, I, P, P, P]),
         "kv4_set_decode_overlap": (I, [P, I]),
         "kv4_set_rotation_signs": (I, [P, P]),
+        "kv4_set_value_rotation": (I, [P, I]),
         "kv4_bf16_query_sizes": (I, [cfgp, ctypes.POINTER(S)]),
         "kv4_bf16_cache_init": (I, [cfgp, P, ctypes.POINTER(P)]),
         "kv4_bf16_append": (I, [P, I, I, P, I, P, I, i32p, i32p, i32p, I, P]),
@@ -172,6 +173,11 @@ def kv4_set_rotation_signs(handle, sign_bits):
         return
     arr = (ctypes.c_uint32 * 4)(*[int(x) & 0xFFFFFFFF for x in list(sign_bits)[:4]])
     _check("kv4_set_rotation_signs", lib.kv4_set_rotation_signs(handle, ctypes.cast(arr, ctypes.c_void_p)))
+
+
+def kv4_set_value_rotation(handle, enable: bool):
+    """Store values rotated like the keys; outputs are rotated back.  Set before the first append."""
+    _check("kv4_set_value_rotation", lib.kv4_set_value_rotation(handle, 1 if enable else 0))
 
 
 def kv4_set_decode_overlap(handle, enable: bool):

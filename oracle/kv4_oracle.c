@@ -355,6 +355,7 @@ int orc_append(const orc_config* c, uint8_t* pool, uint8_t* side, int T, const v
         vf[e] = (float)load_elem(V, v_dtype, in0 + (size_t)e);
       }
       orc_rotate_key(c, kf);
+      if (c->rotate_values) orc_rotate_key(c, vf);
       uint16_t sc, zr;
       orc_quant_int4(kf, D, c4, &sc, &zr);
       for (int e = 0; e < D; ++e) put_nibble(pool, orc_k4_byte(c, page, g, pp, e), e & 1, c4[e]);
@@ -539,6 +540,11 @@ int orc_decode(const orc_config* c, const uint8_t* pool, const uint8_t* side, in
           region_stats(logit, vhat, D, m_end > s_end ? m_end : s_end, L, &parts[np++]);
         }
         merge_parts(parts, np, D, o, &lse_v);
+        if (c->rotate_values) {
+          /* the values were stored as H diag(s) v: back to the original basis, diag(s) H o / h */
+          orc_fwht_f64(o, D, h);
+          for (int e = 0; e < D; ++e) o[e] = (orc_sign(c, e) ? -o[e] : o[e]) / (double)h;
+        }
         if (lse) lse[qh] = lse_v;
       }
     }

@@ -45,6 +45,8 @@ typedef struct {
   int max_seqs;        /* rows of the INT8 side cache                  */
   uint32_t sign_bits[4]; /* randomised-sign rotation: bit d (word d / 32) negates dim d of the
                             key and of the query before the Hadamard; all zero = plain H    */
+  int rotate_values;     /* values stored rotated like the keys (H diag(s)); outputs rotated
+                            back as diag(s) H o / h                                          */
 } orc_config;
 
 /* fp16 helpers (IEEE binary16), written from the format definition. */
@@ -56,7 +58,8 @@ float    orc_bf16_to_f32(uint16_t b);
 void orc_fwht_f32(float* x, int D, int h);
 /* Same transform in fp64 (used for the query rotation). */
 void orc_fwht_f64(double* x, int D, int h);
-/* The key rotation of the append: H diag(s) x, the configured signs, then orc_fwht_f32. */
+/* The key rotation of the append: H diag(s) x, the configured signs, then orc_fwht_f32 (also the
+ * value rotation when rotate_values is set). */
 void orc_rotate_key(const orc_config* c, float* x);
 
 /* Per-vector quantisers.  codes4 holds one code (0..15) per element, unpacked. */

@@ -46,7 +46,8 @@ def build(force: bool = False) -> str:
 class _Cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "num_q_heads", "num_kv_heads", "head_dim", "page_size", "num_sinks",
-        "recent_window", "hadamard_block", "max_seqs")] + [("sign_bits", ctypes.c_uint32 * 4)]
+        "recent_window", "hadamard_block", "max_seqs")] + [("sign_bits", ctypes.c_uint32 * 4),
+                                                           ("rotate_values", ctypes.c_int)]
 
 
 @dataclass(frozen=True)
@@ -61,11 +62,13 @@ class Config:
     hadamard_block: int
     max_seqs: int
     sign_bits: tuple = (0, 0, 0, 0)  # randomised-sign rotation (bit d negates dim d); zero = plain
+    rotate_values: int = 0  # values stored rotated like the keys
 
     def c(self) -> _Cfg:
         return _Cfg(self.num_q_heads, self.num_kv_heads, self.head_dim, self.page_size,
                     self.num_sinks, self.recent_window, self.hadamard_block, self.max_seqs,
-                    (ctypes.c_uint32 * 4)(*[int(x) & 0xFFFFFFFF for x in (list(self.sign_bits) + [0] * 4)[:4]]))
+                    (ctypes.c_uint32 * 4)(*[int(x) & 0xFFFFFFFF for x in (list(self.sign_bits) + [0] * 4)[:4]]),
+                    int(self.rotate_values))
 
 
 _lib = None

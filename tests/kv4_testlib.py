@@ -34,13 +34,15 @@ def prefill_tokens(lens):
 
 
 def gpu_cache_from_host_inputs(wl: W.Workload, layer: int = 0, step_by_step: bool = False, fill: int = 0xA5,
-                               lens=None, signs=None):
+                               lens=None, signs=None, rotate_values: bool = False):
     """Append every token of the workload through kv4_append (inputs drawn on the host)."""
     from int4_kv_cache_append_b200 import kv4
     lens = np.asarray(wl.lens if lens is None else lens, np.int32)
     cache = kv4.Cache(geometry(wl), fill=fill)
     if signs is not None:
         kv4.kv4_set_rotation_signs(cache.handle, signs)
+    if rotate_values:
+        kv4.kv4_set_value_rotation(cache.handle, True)
     pt = torch.from_numpy(wl.page_table).cuda()
     if not step_by_step:
         b, p = prefill_tokens(lens)
@@ -60,8 +62,10 @@ def gpu_cache_from_host_inputs(wl: W.Workload, layer: int = 0, step_by_step: boo
     return cache
 
 
-def oracle_cache(wl: W.Workload, layer: int = 0, step_by_step: bool = False, lens=None, signs=None):
-    cfg = O.Config(wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h, wl.B, tuple(signs) if signs is not None else (0, 0, 0, 0))
+def oracle_cache(wl: W.Workload, layer: int = 0, step_by_step: bool = False, lens=None, signs=None,
+                 rotate_values: bool = False):
+    cfg = O.Config(wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h, wl.B,
+                   tuple(signs) if signs is not None else (0, 0, 0, 0), int(rotate_values))
     lens = np.asarray(wl.lens if lens is None else lens, np.int32)
     pool = np.full(O.page_bytes(cfg) * max(wl.num_pages, 1), 0xA5, np.uint8)
     side = np.full(O.side_slot_bytes(cfg) * wl.B, 0xA5, np.uint8)

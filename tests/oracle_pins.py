@@ -282,10 +282,10 @@ def pin_layout_bijection():
 # ----------------------------------------------------------------------------- cache helpers
 
 def build_cache(wl: W.Workload, layer: int = 0, lens=None, step_by_step: bool = False, sentinel: int = 0xA5,
-                signs=(0, 0, 0, 0)):
+                signs=(0, 0, 0, 0), rotate_values: int = 0):
     """Oracle cache for a workload: prefill every token in position order (one call for all
     tokens with lens_after = L, or one call per position with lens_after = pos + 1)."""
-    cfg = oracle_cfg(wl, signs)
+    cfg = oracle_cfg(wl, signs, rotate_values)
     lens = np.asarray(wl.lens if lens is None else lens, np.int32)
     pool = np.full(O.page_bytes(cfg) * wl.num_pages, sentinel, np.uint8)
     side = np.full(O.side_slot_bytes(cfg) * wl.B, sentinel, np.uint8)
@@ -307,8 +307,8 @@ def build_cache(wl: W.Workload, layer: int = 0, lens=None, step_by_step: bool = 
     return cfg, pool, side
 
 
-def oracle_cfg(wl: W.Workload, signs=(0, 0, 0, 0)) -> O.Config:
-    return O.Config(wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h, wl.B, tuple(signs))
+def oracle_cfg(wl: W.Workload, signs=(0, 0, 0, 0), rotate_values: int = 0) -> O.Config:
+    return O.Config(wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h, wl.B, tuple(signs), rotate_values)
 
 
 def small_workload(D=32, B=3, lens=(12, 7, 40), s=2, w=5, h=8, G=2, Hkv=2, P=16, seed=5,
@@ -499,6 +499,31 @@ def pin_rotation_invariance(seed: int = 51):
             assert np.abs(out[0, i] - ref).max() <= 1e-12 * max(1, np.abs(ref).max())
 
 
+def pin_value_rotation_invariance(seed: int = 57):
+    """With values stored rotated (H diag(s) v) the decode output, rotated back, equals attention
+    over the de-rotated dequantised values diag(s) H^T vhat_rot / h (and de-rotated keys)."""
+    rng = np.random.default_rng(seed)
+    for h in (1, 8, 32):
+        words = tuple(int(x) for x in rng.integers(0, 2**32, size=4, dtype=np.uint64))
+        wl = small_workload(D=32, lens=(30,), B=1, s=2, w=4, h=h, seed=seed)
+        cfg, pool, side = build_cache(wl, signs=words, rotate_values=1)
+        q = wl.q_input(0)
+        out, _ = O.decode(cfg, pool, side, q, wl.page_table, wl.lens, mode=O.SINGLE)
+        Hm = np.kron(np.eye(wl.D // h), scipy.linalg.hadamard(h)).astype(np.float64)
+        S = sign_vector(words, wl.D)[None, :]
+        kd, vd, _ = O.dequant_seq(cfg, pool, side, wl.page_table[0], 0, 30, 0)
+        k_unrot = (kd @ Hm / h) * S
+        v_unrot = (vd @ Hm / h) * S
+        for i in range(wl.G):
+            logits = k_unrot @ q[0, i].astype(np.float64) / np.sqrt(wl.D)
+            p = np.exp(logits - logits.max())
+            ref = (p[:, None] * v_unrot).sum(0) / p.sum()
+            assert np.abs(out[0, i] - ref).max() <= 1e-12 * max(1, np.abs(ref).max())
+        # the stored values are rotated: dequantised rows differ from the unrotated cache's
+        _, vd0, _ = O.dequant_seq(*build_cache(wl, signs=words), wl.page_table[0], 0, 30, 0)
+        assert not np.allclose(vd, vd0)
+
+
 def pin_special_cases(seed: int = 61):
     # L = 1: a single position -> out equals its dequantised value exactly
     wl = small_workload(lens=(1, 1), B=2, s=2, w=5, seed=seed)
@@ -542,5 +567,5 @@ ALL_PINS = [
     pin_quant_int4_constant, pin_quant_int8_bounds, pin_storage_bits, pin_layout_bijection,
     lambda: pin_routing(False), lambda: pin_routing(True), pin_brute_force,
     pin_append_vs_numpy_requant, pin_regional_equals_single, pin_rotation_invariance,
-    pin_special_cases, pin_signed_rotation_exact,
+    pin_special_cases, pin_signed_rotation_exact, pin_value_rotation_invariance,
 ]

@@ -249,3 +249,23 @@ def test_randomised_sign_rotation(case_id):
     assert not np.array_equal(plain, pool)
     assert kv4.kv4_get_device_error() == 0
 
+
+@pytest.mark.parametrize("case_id", [1, 3, 8], ids=["d128-h128", "d64-h1", "d128-kv8"])
+def test_value_rotation(case_id):
+    """kv4_set_value_rotation (with random signs): values stored in the keys' rotated basis are
+    bit-exact against the oracle's same reading, and the decode output, rotated back by the merge,
+    matches the oracle's."""
+    from int4_kv_cache_append_b200 import kv4
+    wl = make(CASES[case_id])
+    words = [int(x) for x in np.random.default_rng(91 + case_id).integers(0, 2**32, size=4, dtype=np.uint64)]
+    words = words[:(wl.D + 31) // 32] + [0] * (4 - (wl.D + 31) // 32)
+    gc = T.gpu_cache_from_host_inputs(wl, signs=words, rotate_values=True)
+    cfg, pool, side = T.oracle_cache(wl, signs=words, rotate_values=True)
+    gp, gs = gc.layer_views(0)
+    assert np.array_equal(gp.cpu().numpy(), pool) and np.array_equal(gs.cpu().numpy(), side)
+    q = wl.q_input(0)
+    ref, ref_lse = T.oracle_decode(wl, cfg, pool, side, q)
+    out, lse = T.gpu_decode(gc, wl, q)
+    T.assert_close(out, ref, lse, ref_lse, what=f"value rotation {CASES[case_id][0]}")
+    assert kv4.kv4_get_device_error() == 0
+

@@ -36,6 +36,8 @@ MUTANTS = [
     ("q-not-rotated", "orc_fwht_f64(qr, D, h);", ";", None),
     ("q-signs-ignored", "if (orc_sign(c, e)) qr[e] = -qr[e];", ";", None),
     ("k-signs-ignored", "if (orc_sign(c, e)) x[e] = -x[e];", ";", None),
+    ("v-rotation-not-undone", "if (c->rotate_values) {", "if (0) {", None),
+    ("v-rotation-no-signs", "(orc_sign(c, e) ? -o[e] : o[e]) / (double)h", "o[e] / (double)h", None),
     ("tau-wrong", "1.0 / sqrt((double)D)", "1.0 / (double)D", None),
     ("merge-no-rescale-l", "l += parts[i].l * f;", "l += parts[i].l;", None),
     ("merge-no-rescale-o", "out[e] += parts[i].o[e] * f;", "out[e] += parts[i].o[e];", None),

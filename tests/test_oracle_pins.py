@@ -77,5 +77,9 @@ def test_signed_rotation_exact():
     P.pin_signed_rotation_exact()
 
 
+def test_value_rotation_invariance():
+    P.pin_value_rotation_invariance()
+
+
 def test_special_cases():
     P.pin_special_cases()
