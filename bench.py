@@ -1,15 +1,18 @@
 #!/usr/bin/env python
-"""Benchmark: one decode step of INT4-KV attention (append + decode) on the Qwen3-4B-like
-workload (32 q / 8 KV heads, head_dim 128, bf16, B = 64 sequences with lognormal lengths of
-median 2048 capped at 8192, P = 16, s = 4, w = 128, h = 128), beside the BF16-KV kernel on the
-same box and the CPU oracle on the host cores.
+"""Benchmark: decode steps of INT4-KV attention (append + decode) beside the BF16-KV kernel on
+the same box and the CPU oracle on the host cores.  Default workload: Qwen3-4B-like (32 q / 8 KV
+heads, head_dim 128, bf16, B = 64 sequences with lognormal lengths of median 2048 capped at
+8192, P = 16, s = 4, w = 128, h = 128).
 
-A step = kv4_append of one new token per sequence (rotation, INT4 pack, INT8 routing) followed
-by kv4_decode_attn over the whole cache (INT4 region + INT8 sink/recent regions, split-K,
-regional merge).  Steps cycle over 4 resident layers (0.72 GB of KV between reuses, larger than
-the 126 MB L2).  Prints one JSON line.
+A layer call = kv4_append of one new token per sequence (rotation, INT4 pack, INT8 routing)
+followed by kv4_decode_attn over the whole cache (INT4 region + INT8 sink/recent regions,
+split-K, regional merge).  One-layer workloads: a step is one layer call, steps cycle over 4
+resident layers (0.72 GB of KV between reuses for the default, larger than the 126 MB L2).
+`--workload qwen3-8b-loop [--h 32|64|128]`: a step is all 36 layers, and every sequence grows by
+one token per step.  Each step is one CUDA graph (the decode a programmatic dependent of the
+append); a second loop times the kernels one by one for the roofline.  Prints one JSON line.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kv4|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kv4|reference] [--workload NAME]
 Under torchrun (N > 1) every rank runs its own batch on its own GPU (weak scaling, no
 collective on the data path); the time is the max over ranks.
 """
@@ -34,18 +37,31 @@ LAYERS = 4
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 2000; 64 for the growing 36-layer workload)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["kv4", "reference"], default="kv4")
     ap.add_argument("--workload", default="qwen3-4b-decode")
+    ap.add_argument("--h", type=int, default=None, help="Hadamard block of the 36-layer workload (32, 64, 128)")
     ap.add_argument("--no-bf16", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
-    ap.add_argument("--overlap", action="store_true",
-                    help="decode builds its schedule while the append runs (kv4_set_decode_overlap 1)")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="decode waits for the append before building its schedule (kv4_set_decode_overlap 0)")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--soak-s", type=float, default=1.5, help="untimed identical steps sampled for clocks")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if args.steps is None:
+        args.steps = 64 if args.workload == "qwen3-8b-loop" else 2000
+    return args
+
+
+def make_wl(args):
+    sys.path.insert(0, ROOT)
+    from int4_kv_cache_append_b200 import workload as W
+    fn = W.WORKLOADS[args.workload]
+    h = getattr(args, "h", None)
+    return fn(h=h) if h is not None else fn()
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -208,7 +224,9 @@ def oracle_sample_setup(wl, nseq: int):
     return step, lens
 
 
-def cpu_baseline(wl, nseq: int = 16, min_seconds: float = 10.0):
+def cpu_baseline(wl, nseq: int = 16, min_seconds: float = 10.0, per_step: int = 1):
+    """The oracle's append + decode of one layer per step on a sample of sequences; a step of
+    per_step layers costs per_step such steps (the layers are identical in shape)."""
     step, lens = oracle_sample_setup(wl, nseq)
     cores = os.cpu_count() or 1
     step(cores)  # warm
@@ -219,18 +237,19 @@ def cpu_baseline(wl, nseq: int = 16, min_seconds: float = 10.0):
         el = time.perf_counter() - t0
         if el >= min_seconds or reps >= 5000:
             break
-    return {"value": nseq * reps / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+    per = f", one layer timed, rate divided by the step's {per_step} layers" if per_step > 1 else ""
+    return {"value": nseq * reps / el / per_step, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"first {nseq} of {wl.B} sequences (lengths {int(lens.min())}..{int(lens.max())}), "
-                      f"append 1 token + decode per step, fp64 C oracle with OpenMP over (sequence, KV head), "
-                      f"{reps} steps in {el:.1f} s"}
+                      f"append 1 token + decode per layer, fp64 C oracle with OpenMP over (sequence, KV head), "
+                      f"{reps} layer-steps in {el:.1f} s{per}"}
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return None
     sys.path.insert(0, ROOT)
-    from int4_kv_cache_append_b200 import workload as W
-    wl = W.WORKLOADS[args.workload]()
+    wl = make_wl(args)
+    per_step = step_shape(wl)[0]
     nseq = min(4, wl.B)
     step, lens = oracle_sample_setup(wl, nseq)
     cores = os.cpu_count() or 1
@@ -240,11 +259,12 @@ def run_reference(args, world, rank):
     for _ in range(args.steps):
         step(cores)
     el = time.perf_counter() - t0
-    value = nseq * args.steps / el
+    value = nseq * args.steps / el / per_step
     sample = (f"each step: first {nseq} of {wl.B} sequences (lengths {int(lens.min())}..{int(lens.max())}), "
-              f"append 1 token + decode, fp64 C oracle, OpenMP over (sequence, KV head)")
+              f"append 1 token + decode of one layer, fp64 C oracle, OpenMP over (sequence, KV head)"
+              + (f"; rate divided by the step's {per_step} layers" if per_step > 1 else ""))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps * per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "B_sampled": nseq, "parallelism": "host cores"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
@@ -254,122 +274,186 @@ def run_reference(args, world, rank):
 
 # ----------------------------------------------------------------------------- GPU leg
 
+def step_shape(wl):
+    """(layers one step runs, resident layers, positions each sequence may still grow by).
+
+    One-layer workloads cycle over LAYERS resident layers, one layer per step, and append at the
+    same position every step.  A workload with more layers than that (the 36-layer append + decode
+    loop) runs every layer in one step, and its lengths grow by one token per step."""
+    grow = int((wl.max_lens - wl.lens).min())
+    if wl.layers > LAYERS:
+        return wl.layers, wl.layers, grow
+    return 1, LAYERS, grow
+
+
 def run_kv4(args, world, rank, local):
     import torch
     sys.path.insert(0, ROOT)
     from int4_kv_cache_append_b200 import harness as H, kv4
-    from int4_kv_cache_append_b200 import workload as W
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    wl = W.WORKLOADS[args.workload]()
+    wl = make_wl(args)
     B = wl.B
-    lens = wl.lens.astype(np.int32)
-    maxlen = int(lens.max())
+    lens0 = wl.lens.astype(np.int32)
+    per_step, resident, grow = step_shape(wl)
+    steps, warmup = args.steps, args.warmup
+    if grow and steps > grow:
+        raise SystemExit(f"{wl.name}: at most {grow} timed steps (page capacity for growth)")
+    maxlen = int(lens0.max()) + grow
     stream = torch.cuda.Stream(dev)
 
-    def setup(bf16: bool):
-        geo = H.geometry(wl, layers=LAYERS)
+    def setup(bf16: bool, layers: int):
+        geo = H.geometry(wl, layers=layers)
         cache = kv4.BF16Cache(geo, device=dev) if bf16 else kv4.Cache(geo, device=dev)
-        for layer in range(LAYERS):
-            H.prefill(cache, wl, layer, lens, upto=lens - 1, bf16_pool=bf16)
+        for layer in range(layers):
+            H.prefill(cache, wl, layer, lens0, upto=lens0 - 1, bf16_pool=bf16)
         factor = torch.from_numpy(wl.factor()).to(dev)
         bt = torch.arange(B, dtype=torch.int32, device=dev)
-        pt_ = torch.from_numpy(lens - 1).to(dev)
+        pos = torch.from_numpy(lens0 - 1).to(dev)
         ins = []
-        for layer in range(LAYERS):
-            K1, V1 = H.device_kv(wl, layer, bt, pt_, factor)
+        for layer in range(layers):
+            K1, V1 = H.device_kv(wl, layer, bt, pos, factor)
             ins.append((K1, V1, H.device_q(wl, layer, 0, dev)))
-        return cache, ins, bt, pt_
+        return cache, ins, bt
 
-    def make_steps(cache, ins, bt, pt_, bf16):
-        page_table = torch.from_numpy(wl.page_table).to(dev)
-        lens_t = torch.from_numpy(lens).to(dev)
-        out = torch.empty((B, wl.Hq, wl.D), dtype=torch.float32, device=dev)
-        ws = cache.workspace(B)
+    class Steps:
+        """Kernels of one layer (append, decode) and of one whole step, on `stream`.  `st` holds
+        the new token's position (row 0) and the length after it (row 1) of every sequence; a
+        growing workload advances both by one at the end of each step."""
 
-        def append(layer):
-            K1, V1, _ = ins[layer]
-            if bf16:
-                cache.append(layer, K1, V1, bt, pt_, page_table, stream=stream)
+        def __init__(self, cache, ins, bt, bf16, layers):
+            self.cache, self.ins, self.bt, self.bf16, self.layers = cache, ins, bt, bf16, layers
+            self.page_table = torch.from_numpy(wl.page_table).to(dev)
+            self.st0 = torch.from_numpy(np.stack([lens0 - 1, lens0])).to(dev)
+            self.st = self.st0.clone()
+            self.out = torch.empty((B, wl.Hq, wl.D), dtype=torch.float32, device=dev)
+            self.ws = cache.workspace(B)
+
+        def append(self, layer):
+            K1, V1, _ = self.ins[layer]
+            if self.bf16:
+                self.cache.append(layer, K1, V1, self.bt, self.st[0], self.page_table, stream=stream)
             else:
-                cache.append(layer, K1, V1, bt, pt_, lens_t, page_table, stream=stream)
+                self.cache.append(layer, K1, V1, self.bt, self.st[0], self.st[1], self.page_table, stream=stream)
 
-        def decode(layer):
-            cache.decode(layer, ins[layer][2], page_table, lens_t, out=out, max_len_hint=maxlen, workspace=ws,
-                         stream=stream)
+        def decode(self, layer):
+            self.cache.decode(layer, self.ins[layer][2], self.page_table, self.st[1], out=self.out,
+                              max_len_hint=maxlen, workspace=self.ws, stream=stream)
 
-        return append, decode, out, page_table, lens_t
+        def advance(self):
+            if grow:
+                self.st.add_(1)
 
-    def capture(fn_list):
-        graphs = []
-        n0 = kv4.kv4_launch_count()
+        def reset(self):
+            self.st.copy_(self.st0)
+
+        def step(self, i):
+            """Step i: every layer (multi-layer workloads) or resident layer i % layers."""
+            for layer in (range(self.layers) if per_step > 1 else [i % self.layers]):
+                self.append(layer)
+                self.decode(layer)
+            self.advance()
+
+    def capture(fns):
+        """One CUDA graph per callable (each warmed once outside capture, which sets kernel
+        attributes).  Returns the graphs and the library kernel launches one replay of each makes."""
+        graphs, counts = [], []
         with torch.cuda.stream(stream):
-            for fn in fn_list:
-                fn()  # warm (sets kernel attributes outside capture)
+            for fn in fns:
+                fn()
             stream.synchronize()
-            for fn in fn_list:
+            for fn in fns:
+                n0 = kv4.kv4_launch_count()
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=stream):
                     fn()
+                counts.append(kv4.kv4_launch_count() - n0)
                 graphs.append(g)
-        launches = (kv4.kv4_launch_count() - n0) // 2  # warm run + capture each counted once
-        return graphs, launches
+        return graphs, counts
 
-    def timed(append, decode, steps, warmup, sampler=None, soak_s=0.0):
+    def timed(S, steps, warmup, sampler=None, soak_s=0.0):
+        """Two timed loops of `steps` steps each, after `warmup` untimed ones.
+
+        Kernel loop: layer launches in turn (layer i % layers), each append and each decode as its
+        own graph with CUDA events between them -> the mean append and decode (decode + merge
+        kernels) durations.  Step loop: `steps` steps, each one graph holding the step's kernels
+        in stream order, the decode a programmatic dependent of the append before it -> the step
+        time.  Lengths are reset before each loop."""
+        L = S.layers
         if args.no_graph:
-            ga = [lambda l=l: append(l) for l in range(LAYERS)]
-            gd = [lambda l=l: decode(l) for l in range(LAYERS)]
-            run_a = lambda l: ga[l]()
-            run_d = lambda l: gd[l]()
+            run_a = S.append
+            run_d = S.decode
+            run_s = S.step
             n0 = kv4.kv4_launch_count()
-            append(0)
-            decode(0)
+            S.step(0)
             torch.cuda.synchronize(dev)
-            per_step = kv4.kv4_launch_count() - n0
+            launches_per_step = kv4.kv4_launch_count() - n0
         else:
-            gA, la = capture([lambda l=l: append(l) for l in range(LAYERS)])
-            gD, ld = capture([lambda l=l: decode(l) for l in range(LAYERS)])
-            per_step = (la + ld) // LAYERS
+            gA, _ = capture([lambda l=l: S.append(l) for l in range(L)])
+            gD, _ = capture([lambda l=l: S.decode(l) for l in range(L)])
+            n_graphs = 1 if per_step > 1 else L
+            gS, cS = capture([lambda i=i: S.step(i) for i in range(n_graphs)])
+            launches_per_step = cS[0]
             run_a = lambda l: gA[l].replay()
             run_d = lambda l: gD[l].replay()
+            run_s = lambda i: gS[i % n_graphs].replay()
+        adv = S.advance
         with torch.cuda.stream(stream):
+            S.reset()
             for i in range(warmup):
-                run_a(i % LAYERS)
-                run_d(i % LAYERS)
+                run_s(i)
+                if grow and (i + 1) % grow == 0:
+                    S.reset()
             stream.synchronize()
             if sampler:
                 sampler.start()
                 t_end = time.perf_counter() + soak_s
                 i = 0
+                S.reset()
                 while time.perf_counter() < t_end:
-                    run_a(i % LAYERS)
-                    run_d(i % LAYERS)
+                    run_s(i)
                     i += 1
-                    if i % 64 == 0:
+                    if grow and i % grow == 0:
+                        S.reset()
+                    if i % 16 == 0:
                         stream.synchronize()
                 stream.synchronize()
+            # kernel loop
+            S.reset()
             barrier(world)
             torch.cuda.synchronize(dev)
             ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+            for i in range(steps):
+                layer = i % L
+                ev[i][0].record(stream)
+                run_a(layer)
+                ev[i][1].record(stream)
+                run_d(layer)
+                ev[i][2].record(stream)
+                if layer == L - 1 or per_step == 1:
+                    adv()
+            torch.cuda.synchronize(dev)
+            dec_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
+            app_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+            kernel_loop_lens = [int(i // L) if per_step > 1 else i for i in range(steps)] if grow else [0]
+            # step loop
+            S.reset()
+            torch.cuda.synchronize(dev)
+            barrier(world)
+            torch.cuda.synchronize(dev)
             start = torch.cuda.Event(enable_timing=True)
             end = torch.cuda.Event(enable_timing=True)
             start.record(stream)
             for i in range(steps):
-                ev[i][0].record(stream)
-                run_a(i % LAYERS)
-                ev[i][1].record(stream)
-                run_d(i % LAYERS)
-                ev[i][2].record(stream)
+                run_s(i)
             end.record(stream)
             end.synchronize()
             torch.cuda.synchronize(dev)
         barrier(world)
         clocks = sampler.stop() if sampler else None
         total_ms = start.elapsed_time(end)
-        dec_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
-        app_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
-        return total_ms, dec_ms, app_ms, per_step * steps, clocks
+        return total_ms, dec_ms, app_ms, launches_per_step * steps, clocks, kernel_loop_lens
 
     uuid = None
     try:
@@ -378,21 +462,25 @@ def run_kv4(args, world, rank, local):
         pass
 
     # ---- INT4 cache (the product)
-    cache, ins, bt, pt_ = setup(False)
-    # lens and page_table are written before the step, not by the append: the decode may build its
-    # schedule while the append runs
-    kv4.kv4_set_decode_overlap(cache.handle, args.overlap)
-    append, decode, out, page_table, lens_t = make_steps(cache, ins, bt, pt_, False)
-    total_ms, dec_ms, app_ms, launches, clocks = timed(append, decode, args.steps, args.warmup,
-                                                       sampler=ClockSampler(uuid), soak_s=args.soak_s)
+    cache, ins, bt = setup(False, resident)
+    # lens and page_table are written before the step, never by the append: the decode may build
+    # its schedule while the append runs
+    kv4.kv4_set_decode_overlap(cache.handle, 0 if args.no_overlap else 1)
+    S = Steps(cache, ins, bt, False, resident)
+    total_ms, dec_ms, app_ms, launches, clocks, klens = timed(S, steps, warmup, sampler=ClockSampler(uuid),
+                                                               soak_s=args.soak_s)
     err = kv4.kv4_get_device_error()
     if err:
         raise RuntimeError(f"device error bits {err:#x} during the benchmark")
     total_ms = max_over_ranks(total_ms, world)
-    value = whole_job_rate(B * args.steps, world, total_ms)
+    value = whole_job_rate(B * steps, world, total_ms)
 
-    kv_bytes = wl.kv_bytes_int4(lens)
-    pt_bytes = int(4 * ((lens + wl.P - 1) // wl.P).sum())
+    # algorithmic bytes of one decode launch, averaged over the lengths the kernel loop saw
+    def alg_of(kv_fn):
+        kv = float(np.mean([kv_fn(lens0 + d) for d in klens]))
+        pt = float(np.mean([4 * ((lens0 + d + wl.P - 1) // wl.P).sum() for d in klens]))
+        return kv, pt
+    kv_bytes, pt_bytes = alg_of(wl.kv_bytes_int4)
     io_bytes = B * wl.Hq * wl.D * (2 + 4)  # bf16 q in, fp32 out
     alg_bytes = kv_bytes + pt_bytes + io_bytes
     peak, peak_kind = peaks()
@@ -400,30 +488,29 @@ def run_kv4(args, world, rank, local):
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": profiled_traffic(wl.name),
             "kernel": "decode_int4_kernel + merge_int4_kernel (kv4_decode_attn: split-K tiles, then LSE merge)",
-            "bytes_per_launch": alg_bytes, "kv_bytes_per_launch": kv_bytes, "decode_ms": round(dec_ms, 5),
+            "bytes_per_launch": int(alg_bytes), "kv_bytes_per_launch": int(kv_bytes), "decode_ms": round(dec_ms, 5),
             "peak_source": f"{peak_kind} MEASURED_PEAKS.json hbm_gbs" if peak_kind == "measured" else "fallback"}
     spec_frac = achieved / 8000.0
 
-    # ---- e2e through the public API with host buffers (pinned), every step.  Each step copies its
-    # inputs (q, K, V, slots, positions, lengths) from pinned host memory, runs append + decode
-    # through the C ABI and copies the output back.  Pipelined: inputs on an H2D stream and the
-    # output on a D2H stream, device buffers double-buffered and ordered by events, so the copies
-    # of one step overlap the kernels of the previous one.  The serial form (one stream) is
-    # reported beside it.
+    # ---- e2e through the public API with host buffers (pinned), every step.  Each step copies the
+    # inputs of every layer call it makes (q, K, V, slots, positions, lengths) from pinned host
+    # memory, runs append + decode through the C ABI and copies the (last layer's) output back.
+    # Pipelined: inputs on an H2D stream and the output on a D2H stream, device buffers
+    # double-buffered and ordered by events, so the copies of one step overlap the kernels of the
+    # previous one.  The serial form (one stream) is reported beside it.
     e2e = None
     if args.e2e_steps > 0:
-        K1, V1, q0 = ins[0]
-        hK = K1.cpu().pin_memory()
-        hV = V1.cpu().pin_memory()
-        hq = q0.cpu().pin_memory()
+        nl = per_step  # layer calls per step
+        hkv = [(ins[l][0].cpu().pin_memory(), ins[l][1].cpu().pin_memory(), ins[l][2].cpu().pin_memory())
+               for l in range(nl if per_step > 1 else 1)]
         hb = bt.cpu().pin_memory()
-        hp = pt_.cpu().pin_memory()
-        hl = lens_t.cpu().pin_memory()
-        hins = (hK, hV, hq, hb, hp, hl)
-        dbuf = [tuple(torch.empty_like(t, device=dev) for t in hins) + (torch.empty_like(out),) for _ in range(2)]
-        houts = [torch.empty_like(out, device="cpu").pin_memory() for _ in range(2)]
-        ws = cache.workspace(B)
-        h2d = sum(t.numel() * t.element_size() for t in hins)
+        nst = max(grow, 1)
+        hst = [torch.from_numpy(np.stack([lens0 - 1 + k, lens0 + k])).pin_memory() for k in range(nst)]
+        dbuf = [{"kvq": [tuple(torch.empty_like(t, device=dev) for t in h) for h in hkv],
+                 "b": torch.empty_like(hb, device=dev), "st": torch.empty_like(hst[0], device=dev),
+                 "out": torch.empty_like(S.out)} for _ in range(2)]
+        houts = [torch.empty_like(S.out, device="cpu").pin_memory() for _ in range(2)]
+        h2d = sum(t.numel() * t.element_size() for h in hkv for t in h) + hb.numel() * 4 + hst[0].numel() * 4
         d2h = houts[0].numel() * houts[0].element_size()
         up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         ev_in = [torch.cuda.Event() for _ in range(2)]
@@ -432,38 +519,45 @@ def run_kv4(args, world, rank, local):
         for e in ev_done + ev_out:
             e.record(stream)
 
-        def step_on(j, layer, pipelined):
-            dK, dV, dq, db, dp, dl, dout = dbuf[j]
+        def step_on(j, i, pipelined):
+            d = dbuf[j]
             cs = up if pipelined else stream
             if pipelined:
                 up.wait_event(ev_done[j])  # the step that last used buffer j has finished
             with torch.cuda.stream(cs):
-                for d_, h_ in zip((dK, dV, dq, db, dp, dl), hins):
-                    d_.copy_(h_, non_blocking=True)
+                for dd, hh in zip(d["kvq"], hkv):
+                    for d_, h_ in zip(dd, hh):
+                        d_.copy_(h_, non_blocking=True)
+                d["b"].copy_(hb, non_blocking=True)
+                d["st"].copy_(hst[i % nst], non_blocking=True)
             if pipelined:
                 ev_in[j].record(up)
                 stream.wait_event(ev_in[j])
                 stream.wait_event(ev_out[j])  # its previous output has been copied out
-            cache.append(layer, dK, dV, db, dp, dl, page_table, stream=stream)
-            cache.decode(layer, dq, page_table, dl, out=dout, max_len_hint=maxlen, workspace=ws, stream=stream)
+            layers = range(nl) if per_step > 1 else [i % resident]
+            for li, layer in enumerate(layers):
+                dK, dV, dq = d["kvq"][li if per_step > 1 else 0]
+                cache.append(layer, dK, dV, d["b"], d["st"][0], d["st"][1], S.page_table, stream=stream)
+                cache.decode(layer, dq, S.page_table, d["st"][1], out=d["out"], max_len_hint=maxlen,
+                             workspace=S.ws, stream=stream)
             if pipelined:
                 ev_done[j].record(stream)
                 down.wait_event(ev_done[j])
             with torch.cuda.stream(down if pipelined else stream):
-                houts[j].copy_(dout, non_blocking=True)
+                houts[j].copy_(d["out"], non_blocking=True)
             if pipelined:
                 ev_out[j].record(down)
 
         def run(pipelined):
-            for i in range(5):
-                step_on(i % 2, i % LAYERS, pipelined)
+            for i in range(3):
+                step_on(i % 2, i, pipelined)
             torch.cuda.synchronize(dev)
             barrier(world)
             s0 = torch.cuda.Event(enable_timing=True)
             s1 = torch.cuda.Event(enable_timing=True)
             s0.record(stream)
             for i in range(args.e2e_steps):
-                step_on(i % 2, i % LAYERS, pipelined)
+                step_on(i % 2, i, pipelined)
             if pipelined:
                 stream.wait_event(ev_out[(args.e2e_steps - 1) % 2])
             s1.record(stream)
@@ -475,46 +569,58 @@ def run_kv4(args, world, rank, local):
         e2e = {"value": whole_job_rate(B * args.e2e_steps, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                "e2e_serial": whole_job_rate(B * args.e2e_steps, world, serial_ms),
-               "path": "kv4.Cache.append + kv4.Cache.decode (C ABI); every step copies its inputs from pinned host "
-                       "memory and its output back; copies on H2D/D2H streams overlap the previous step's kernels "
-                       "(double-buffered); e2e_serial: the same on one stream"}
+               "path": "kv4.Cache.append + kv4.Cache.decode (C ABI) for every layer call of the step; every step "
+                       "copies the inputs of those calls from pinned host memory and the last output back; "
+                       "copies on H2D/D2H streams overlap the previous step's kernels (double-buffered); "
+                       "e2e_serial: the same on one stream"}
 
-    del cache, ins
+    del cache, ins, S
     torch.cuda.empty_cache()
 
-    # ---- BF16-KV baseline kernel on the same box
+    # ---- BF16-KV baseline kernel on the same box.  A multi-layer step is timed on LAYERS of its
+    # layers (BF16 KV of every layer would not fit) and scaled by per_step / LAYERS: the layers
+    # are identical in shape, so the per-layer cost is the same.
     bf = None
     if not args.no_bf16:
-        bcache, bins, bbt, bpt = setup(True)
-        bappend, bdecode, _, _, _ = make_steps(bcache, bins, bbt, bpt, True)
-        b_total, b_dec, b_app, _, _ = timed(bappend, bdecode, args.steps, args.warmup)
-        b_total = max_over_ranks(b_total, world)
-        bkv = wl.kv_bytes_bf16(lens)
+        bl = min(resident, LAYERS)
+        bcache, bins, bbt = setup(True, bl)
+        BS = Steps(bcache, bins, bbt, True, bl)
+        b_total, b_dec, b_app, _, _, bklens = timed(BS, steps, warmup)
+        scale = per_step / bl if per_step > 1 else 1.0
+        b_total = max_over_ranks(b_total, world) * scale
+        bkv = float(np.mean([wl.kv_bytes_bf16(lens0 + d) for d in bklens]))
         b_alg = bkv + pt_bytes + io_bytes
-        bf = {"value": whole_job_rate(B * args.steps, world, b_total), "unit": UNIT, "ms_per_step": b_total / args.steps,
-              "decode_ms": round(b_dec, 5), "kv_bytes_per_launch": bkv,
+        bf = {"value": whole_job_rate(B * steps, world, b_total), "unit": UNIT, "ms_per_step": b_total / steps,
+              "decode_ms": round(b_dec, 5), "kv_bytes_per_launch": int(bkv),
               "achieved_GBps": round(b_alg / (b_dec / 1e3) / 1e9, 1),
               "frac": round(b_alg / (b_dec / 1e3) / 1e9 / peak, 4),
-              "int4_speedup_step": round(value / whole_job_rate(B * args.steps, world, b_total), 3),
+              "int4_speedup_step": round(value / whole_job_rate(B * steps, world, b_total), 3),
               "int4_speedup_decode": round(b_dec / dec_ms, 3)}
-        del bcache, bins
+        if per_step > 1:
+            bf["layers_timed"] = f"{bl} of {per_step} layers per step, time scaled by {scale:g}"
+        del bcache, bins, BS
         torch.cuda.empty_cache()
 
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl)
+        cpu = cpu_baseline(wl, nseq=4 if per_step > 1 else 16, per_step=per_step)
 
-    line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
+    resident_gb = resident * kv_bytes / 1e9
+    line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": steps,
+            "warmup": warmup, "ms_per_step": round(total_ms / steps, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": wl.name, "B_per_gpu": B, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": wl.D, "P": wl.P,
-                       "s": wl.s, "w": wl.w, "h": wl.h, "len_mean": round(float(lens.mean()), 1),
-                       "len_max": maxlen, "kv_dtype": "int4 pages + int8 side cache",
+                       "s": wl.s, "w": wl.w, "h": wl.h, "len_mean": round(float(lens0.mean()), 1),
+                       "len_max": int(lens0.max()), "layers_per_step": per_step,
+                       "growth_per_step": 1 if grow else 0, "kv_dtype": "int4 pages + int8 side cache",
                        "compute": "QK^T int8 MMA (exact int32), PV f16 MMA with f32 accumulate, f32 softmax",
-                       "l2": "inputs larger than L2: 4 resident layers cycled, 0.72 GB of KV between reuses",
+                       "l2": f"inputs larger than L2: {resident} resident layers cycled, {resident_gb:.2f} GB of KV "
+                             f"between reuses",
                        "parallelism": f"dp{world} (independent batches per GPU, no collective)",
-                       "graph": not args.no_graph, "decode_overlap": args.overlap,
-                       "append_ms": round(app_ms, 5)},
+                       "graph": ("one graph per step (append -> decode programmatic edge)" if not args.no_graph
+                                 else False),
+                       "decode_overlap": not args.no_overlap, "append_ms": round(app_ms, 5),
+                       "timing": "step loop (value) and kernel loop (decode_ms, append_ms), each `steps` long"},
             "roofline": roof, "hbm_frac_of_spec_8TBps": round(spec_frac, 4), "gpu_launches": int(launches),
             "clocks": clocks, "e2e": e2e, "bf16_kv": bf, "cpu_baseline": cpu}
     return line if rank == 0 else None

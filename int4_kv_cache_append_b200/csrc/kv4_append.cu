@@ -22,6 +22,7 @@ namespace kv4 {
 namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
+constexpr int kAppendThreads = 1024;
 
 template <typename T>
 __device__ __forceinline__ void load4(const void* base, size_t i, float (&x)[4]);
@@ -134,29 +135,33 @@ __device__ __forceinline__ uint32_t quant_int8(const float (&x)[4], bool act, ui
 }
 
 template <int D, typename KT, typename VT>
-__global__ void __launch_bounds__(256) append_int4_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(kAppendThreads) append_int4_kernel(AppendArgs a) {
   using Gm = Geo<D>;
   pdl_launch_dependents();  // the decode kernel that follows may start its launch now
   const int gw = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= a.T * a.Hkv) return;
   const int t = gw / a.Hkv, g = gw - t * a.Hkv;
-  const int b = a.seq_slot[t], pos = a.pos[t];
-  if (b < 0 || b >= a.max_seqs || pos < 0 || pos / a.P >= a.stride) {
-    if (lane == 0) atomicOr(a.err, KV4_DEVERR_LENGTH);
-    return;
-  }
-  const int page = a.page_table[static_cast<size_t>(b) * a.stride + pos / a.P];
-  if (page < 0 || page >= a.max_pages) {
-    if (lane == 0) atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
-    return;
-  }
+  // Three dependent round trips at most: {token's slot and position, its K and V} -> {page-table
+  // entry, length after the call} -> stores.  K and V are read before the checks (every t < T is
+  // a valid input row).
   const bool act = lane < D / 4;
   float k[4] = {0.f, 0.f, 0.f, 0.f}, v[4] = {0.f, 0.f, 0.f, 0.f};
   const size_t in0 = (static_cast<size_t>(t) * a.Hkv + g) * D + 4 * lane;
   if (act) {
     load4<KT>(a.K, in0, k);
     load4<VT>(a.V, in0, v);
+  }
+  const int b = a.seq_slot[t], pos = a.pos[t];
+  if (b < 0 || b >= a.max_seqs || pos < 0 || pos / a.P >= a.stride) {
+    if (lane == 0) atomicOr(a.err, KV4_DEVERR_LENGTH);
+    return;
+  }
+  const int page = a.page_table[static_cast<size_t>(b) * a.stride + pos / a.P];
+  const int len_after = a.w > 0 && pos >= a.s ? a.lens_after[b] : 0;
+  if (page < 0 || page >= a.max_pages) {
+    if (lane == 0) atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
+    return;
   }
   {
     // randomised-sign rotation: dims of set bits are negated first (exact: the sign bit flips)
@@ -195,7 +200,7 @@ __global__ void __launch_bounds__(256) append_int4_kernel(AppendArgs a) {
   int row = -1;
   if (pos < a.s)
     row = pos;
-  else if (a.w > 0 && pos >= a.lens_after[b] - a.w)
+  else if (a.w > 0 && pos >= len_after - a.w)
     row = a.s + pos % a.w;
   if (row < 0) return;
   uint8_t* t8 = a.side + static_cast<size_t>(b) * a.side_slot_bytes +
@@ -225,7 +230,7 @@ __global__ void __launch_bounds__(256) append_int4_kernel(AppendArgs a) {
 
 // BF16 baseline pool append: K and V stored as bf16 (no rotation, no quantisation).
 template <int D, typename KT, typename VT>
-__global__ void __launch_bounds__(256) append_bf16_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(kAppendThreads) append_bf16_kernel(AppendArgs a) {
   using Gm = Geo<D>;
   const int gw = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
@@ -271,8 +276,10 @@ __global__ void __launch_bounds__(256) append_bf16_kernel(AppendArgs a) {
 
 template <int D, bool BF16_POOL>
 cudaError_t dispatch_types(const AppendArgs& a, cudaStream_t st) {
+  // Few large blocks: a block of this kernel keeps the following decode kernel's block (which
+  // needs a whole SM) off its SM until it exits.
   const int warps = a.T * a.Hkv;
-  const dim3 grid((warps + 7) / 8), block(256);
+  const dim3 grid((warps + kAppendThreads / 32 - 1) / (kAppendThreads / 32)), block(kAppendThreads);
   const bool kf = a.k_dtype == KV4_F32, vf = a.v_dtype == KV4_F32;
   if (BF16_POOL) {
     if (kf && vf) KV4_APPEND_LAUNCH(append_bf16_kernel, float, float);

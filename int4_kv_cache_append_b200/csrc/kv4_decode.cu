@@ -220,6 +220,8 @@ struct Smem {
   unsigned int mask[kWarps][kRing];                  // valid rows: tile A bits 0-15, tile B 16-31
   unsigned int meta[kWarps][kRing];                  // kind | flags | segment index << 8
   unsigned long long seg[kWarps][kRing];             // segment table: cs8 | seg<<32 | g<<33 | b<<41
+  Cursor cur[kWarps];                                // descriptor cursor between fills
+  unsigned segno[kWarps];                            // segments entered so far
   uint64_t bar[kWarps][kStages];
 };
 
@@ -527,6 +529,11 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
 
   unsigned segno = 0;
   if (active) fill_descriptors<D>(a, cap, c1, dcur, lane, sm, warp, 0, segno);
+  // the cursor waits in shared memory between fills (its registers are free in the main loop)
+  if (lane == 0) {
+    sm.cur[warp] = dcur;
+    sm.segno[warp] = segno;
+  }
   __syncwarp();
   if (a.early) pdl_wait();
 
@@ -712,6 +719,9 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
         qd[j][2] = qd[j][3] = 0u;
       }
     }
+    // the scratch is a ring stage that a bulk copy (async proxy) refills later: order this lane's
+    // generic accesses to it before that copy
+    fence_proxy_async_smem();
     __syncwarp();
   };
 
@@ -760,14 +770,16 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
       }
       if (gq == 0) {
         if (!only)
-          *reinterpret_cast<float2*>(p + D) = make_float2(m_run, l);
+          *reinterpret_cast<float2*>(p + D) = make_float2(m_run * qinv, l);
         else if (a.lse)
-          a.lse[static_cast<size_t>(cb) * a.Hq + cg * G + tig] = l > 0.f ? (m_run + log2f(l)) * 0.69314718055994531f : kNegInf;
+          a.lse[static_cast<size_t>(cb) * a.Hq + cg * G + tig] = l > 0.f ? (m_run * qinv + log2f(l)) * 0.69314718055994531f : kNegInf;
       }
     }
   };
 
-  // Running-max update for this lane's logits of head tig (NL values), then their exponentials.
+  // Running-max update for this lane's logits of head tig.  Logits and the running max m_run are
+  // kept unscaled (log2 units times 2^e, e the query's power-of-two normalisation); the returned
+  // offset -m_run 2^-e makes exp2(fmaf(logit, qinv, offset)) the probability.
   auto softmax_update = [&](float tm) {
     tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, 4));
     tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, 8));
@@ -775,7 +787,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     const float mn = fmaxf(m_run, tm);
     const bool grow = mn > m_run;
     if (__any_sync(FULL, grow)) {
-      const float alpha = grow ? (m_run == kNegInf ? 0.f : exp2_fast(m_run - mn)) : 1.f;
+      const float alpha = grow ? (m_run == kNegInf ? 0.f : exp2_fast((m_run - mn) * qinv)) : 1.f;
 #pragma unroll
       for (int mb = 0; mb < NKB; ++mb) {
         oacc[mb][0] *= alpha;
@@ -787,8 +799,9 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
       beta_part *= alpha;
       m_run = mn;
     }
-    return m_run == kNegInf ? 0.f : m_run;
+    return m_run == kNegInf ? 0.f : -m_run * qinv;
   };
+  auto prob = [&](float lg, float off) { return exp2_fast(fmaf(lg, qinv, off)); };
 
   // PV B operand: hi/lo halves of pv for head gq>>1 of this lane's column, positions 2tig, 2tig+1
   // (b0) and 2tig+8, 2tig+9 (b1), gathered from the lanes that computed them.
@@ -824,11 +837,12 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     const uint32_t kp0 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 4 * gq);
     const uint32_t kp1 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 4 * (gq + 8));
     const float ks0 = half_lo(kp0), kz0 = half_hi(kp0), ks1 = half_lo(kp1), kz1 = half_hi(kp1);
-    // logit = (s q_int.c + z sum(q_int)) 2^-e
-    const float R0 = fmaf(65536.f, static_cast<float>(SA[0]), fmaf(256.f, static_cast<float>(SA[1]), static_cast<float>(SB[0])));
-    const float R1 = fmaf(65536.f, static_cast<float>(SA[2]), fmaf(256.f, static_cast<float>(SA[3]), static_cast<float>(SB[2])));
-    lg0 = v0 ? fmaf(ks0, R0, kz0 * sumq) * qinv : kNegInf;
-    lg1 = v1 ? fmaf(ks1, R1, kz1 * sumq) * qinv : kNegInf;
+    // logit 2^e = s q_int.c + z sum(q_int), q_int.c = 2^16 S2 + (2^8 S1 + S0); the bracket is
+    // below 2^26 in magnitude and exact in int32
+    const float R0 = fmaf(65536.f, static_cast<float>(SA[0]), static_cast<float>(SA[1] * 256 + SB[0]));
+    const float R1 = fmaf(65536.f, static_cast<float>(SA[2]), static_cast<float>(SA[3] * 256 + SB[2]));
+    lg0 = v0 ? fmaf(ks0, R0, kz0 * sumq) : kNegInf;
+    lg1 = v1 ? fmaf(ks1, R1, kz1 * sumq) : kNegInf;
   };
 
   // PV of one INT4 tile block with probabilities p0, p1 (rows gq, gq + 8 of head tig).
@@ -870,13 +884,17 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   while (true) {
     if ((k % kChunk) == 0) {
       // descriptors of slots [k + kChunk, k + 2 kChunk) while this chunk is consumed
-      fill_descriptors<D>(a, cap, c1, dcur, lane, sm, warp, k + kChunk, segno);
+      Cursor fc = sm.cur[warp];
+      unsigned fs = sm.segno[warp];
+      __syncwarp();
+      fill_descriptors<D>(a, cap, c1, fc, lane, sm, warp, k + kChunk, fs);
+      if (lane == 0) {
+        sm.cur[warp] = fc;
+        sm.segno[warp] = fs;
+      }
       __syncwarp();
     }
-    if (lane == 0) {
-      fence_proxy_async_smem();
-      if (issue(k + kStages - 1)) ++issued;
-    }
+    if (lane == 0 && issue(k + kStages - 1)) ++issued;
     const int st = k % kStages;
     const bool ok = mbar_wait_bounded(&bars[st], static_cast<uint32_t>((k / kStages) & 1), a.err);
     if (__any_sync(FULL, !ok)) {
@@ -889,15 +907,25 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     const unsigned msk = sm.mask[warp][p];
     if (meta_kind(meta) == kKindInt4) {
       // ----------------------------------------------------------- two INT4 tiles
-      const bool two = (meta & kMetaTwo) != 0;
-      const bool vA0 = tig < G && ((msk >> gq) & 1u), vA1 = tig < G && ((msk >> (gq + 8)) & 1u);
-      const bool vB0 = tig < G && ((msk >> (gq + 16)) & 1u), vB1 = tig < G && ((msk >> (gq + 24)) & 1u);
       float lA0, lA1, lB0 = kNegInf, lB1 = kNegInf;
-      qk_int4(buf, vA0, vA1, lA0, lA1);
-      if (two) qk_int4(buf + T4B, vB0, vB1, lB0, lB1);
-      const float mu = softmax_update(fmaxf(fmaxf(lA0, lA1), fmaxf(lB0, lB1)));
-      pv_int4(buf, vA0, vA1, exp2_fast(lA0 - mu), exp2_fast(lA1 - mu));
-      if (two) pv_int4(buf + T4B, vB0, vB1, exp2_fast(lB0 - mu), exp2_fast(lB1 - mu));
+      if (msk == 0xFFFFFFFFu) {
+        // both tiles present with all 32 rows valid (the common case): no row masking.  Lanes of
+        // absent heads (tig >= G) compute finite values that nothing reads.
+        qk_int4(buf, true, true, lA0, lA1);
+        qk_int4(buf + T4B, true, true, lB0, lB1);
+        const float off = softmax_update(fmaxf(fmaxf(lA0, lA1), fmaxf(lB0, lB1)));
+        pv_int4(buf, true, true, prob(lA0, off), prob(lA1, off));
+        pv_int4(buf + T4B, true, true, prob(lB0, off), prob(lB1, off));
+      } else {
+        const bool two = (meta & kMetaTwo) != 0;
+        const bool vA0 = tig < G && ((msk >> gq) & 1u), vA1 = tig < G && ((msk >> (gq + 8)) & 1u);
+        const bool vB0 = tig < G && ((msk >> (gq + 16)) & 1u), vB1 = tig < G && ((msk >> (gq + 24)) & 1u);
+        qk_int4(buf, vA0, vA1, lA0, lA1);
+        if (two) qk_int4(buf + T4B, vB0, vB1, lB0, lB1);
+        const float off = softmax_update(fmaxf(fmaxf(lA0, lA1), fmaxf(lB0, lB1)));
+        pv_int4(buf, vA0, vA1, prob(lA0, off), prob(lA1, off));
+        if (two) pv_int4(buf + T4B, vB0, vB1, prob(lB0, off), prob(lB1, off));
+      }
     } else {
       // ----------------------------------------------------------- one INT8 tile (K half, V half)
       const bool v0 = tig < G && ((msk >> gq) & 1u), v1 = tig < G && ((msk >> (gq + 8)) & 1u);
@@ -922,12 +950,13 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
       }
       const float ks0 = __half2float(*reinterpret_cast<const __half*>(buf + 16 * D + 2 * gq));
       const float ks1 = __half2float(*reinterpret_cast<const __half*>(buf + 16 * D + 2 * (gq + 8)));
-      const float R0 = fmaf(65536.f, static_cast<float>(SA[0]), fmaf(256.f, static_cast<float>(SA[1]), static_cast<float>(SB[0])));
-      const float R1 = fmaf(65536.f, static_cast<float>(SA[2]), fmaf(256.f, static_cast<float>(SA[3]), static_cast<float>(SB[2])));
-      const float lg0 = v0 ? ks0 * R0 * qinv : kNegInf;
-      const float lg1 = v1 ? ks1 * R1 * qinv : kNegInf;
-      const float mu = softmax_update(fmaxf(lg0, lg1));
-      const float p0 = exp2_fast(lg0 - mu), p1 = exp2_fast(lg1 - mu);
+      // |2^8 S1 + S0| < 2^31 for 8-bit codes
+      const float R0 = fmaf(65536.f, static_cast<float>(SA[0]), static_cast<float>(SA[1] * 256 + SB[0]));
+      const float R1 = fmaf(65536.f, static_cast<float>(SA[2]), static_cast<float>(SA[3] * 256 + SB[2]));
+      const float lg0 = v0 ? ks0 * R0 : kNegInf;
+      const float lg1 = v1 ? ks1 * R1 : kNegInf;
+      const float off = softmax_update(fmaxf(lg0, lg1));
+      const float p0 = prob(lg0, off), p1 = prob(lg1, off);
       l_part += (v0 ? p0 : 0.f) + (v1 ? p1 : 0.f);
       const uint8_t* vb = buf + T4B;  // V half
       const float vs0 = __half2float(*reinterpret_cast<const __half*>(vb + 16 * D + 2 * gq));

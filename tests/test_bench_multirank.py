@@ -60,3 +60,16 @@ def test_two_rank_max_timing_and_reference_on_rank0_only():
         assert rate == pytest.approx(2 * 64 * 100 / 0.015)
     assert res[0][3] == ("reference", 2, "oracle")
     assert res[1][3] is None
+
+
+def test_step_shape_of_the_workloads():
+    """One-layer workloads cycle 4 resident layers at fixed lengths; the 36-layer loop runs all of
+    its layers per step and may grow by the page capacity it was built with."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from int4_kv_cache_append_b200 import workload as W
+    assert bench.step_shape(W.qwen3_4b_decode()) == (1, 4, 0)
+    for h in (32, 64, 128):
+        wl = W.qwen3_8b_loop(h=h)
+        assert wl.h == h
+        assert bench.step_shape(wl) == (36, 36, 64)

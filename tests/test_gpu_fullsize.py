@@ -49,7 +49,7 @@ def _oracle_one(wl: W.Workload, b: int, g: int, layer: int = 0):
     return cfg, pool, side, out[0], lse[0]
 
 
-@pytest.mark.parametrize("name", ["qwen3-4b-decode", "async-refill", "long-context"])
+@pytest.mark.parametrize("name", ["qwen3-4b-decode", "async-refill", "long-context", "qwen3-8b-loop"])
 def test_fullsize_sampled_parity(name):
     from int4_kv_cache_append_b200 import harness as H, kv4
     wl = W.WORKLOADS[name]()
