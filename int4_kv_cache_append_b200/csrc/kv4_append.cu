@@ -184,8 +184,21 @@ __global__ void __launch_bounds__(kAppendThreads) append_int4_kernel(AppendArgs 
   const uint32_t kc = quant_int4(k, act, &ksz);
   const uint32_t vc = quant_int4(v, act, &vsz);
   if (act) {
-    // K: elements 4l..4l+3 are bytes 2l, 2l+1 of row r.
-    *reinterpret_cast<uint16_t*>(tile + r * (D / 2) + 2 * lane) = static_cast<uint16_t>(kc);
+    // K: row r shares pair-row r % 8 with row r ^ 8 (low nibbles rows 0-7, high nibbles rows
+    // 8-15), so its nibbles are merged in with atomics (another token of the tile may be written
+    // by another warp of this launch).  Elements 4l, 4l+2 go to bytes 2(l&1), 2(l&1)+1 of word 0
+    // of 8-byte group l/2, elements 4l+1, 4l+3 to the same bytes of word 1.
+    const int pr = r & 7, hi4 = 4 * (r >> 3);
+    const int gb = 8 * (lane >> 1);                                    // group byte in the pair-row
+    const int unit = (gb >> 4) ^ (D >= 128 ? (pr & 1) : 0);
+    uint32_t* w0 = reinterpret_cast<uint32_t*>(tile + pr * D + 16 * unit + (gb & 15));
+    const int sh = 16 * (lane & 1) + hi4;                              // bit of byte 2(l&1)
+    const uint32_t e0 = kc & 15u, e1 = (kc >> 4) & 15u, e2 = (kc >> 8) & 15u, e3 = (kc >> 12) & 15u;
+    const uint32_t clear = ~((0xFu << sh) | (0xFu << (sh + 8)));
+    atomicAnd(w0, clear);
+    atomicOr(w0, (e0 << sh) | (e2 << (sh + 8)));
+    atomicAnd(w0 + 1, clear);
+    atomicOr(w0 + 1, (e1 << sh) | (e3 << (sh + 8)));
     // V: 16-bit chunk of quad Q = l.
     const int Q = lane, p = r >> 1, half = p >> 2, pl = p & 3;
     const int off = ((half * 8 + Q / Gm::WPC) * 4 + pl) * Gm::CH + 4 * (Q % Gm::WPC) + 2 * (r & 1);

@@ -126,10 +126,11 @@ __device__ int find_seq(const DecodeArgs& a, int cap, int lane, u32 c, u32* bsta
 }
 
 // Division by a per-launch constant d >= 2 for n < 2^31: q = umulhi(n, ceil(2^32 / d)) is
-// floor(n / d) or one more; one multiply-compare fixes it.
+// floor(n / d) or one more; one multiply-compare fixes it.  ceil(2^32 / d) = floor((2^32 - 1) / d)
+// + 1 for every d >= 2, a 32-bit division.
 struct FastDiv {
   u32 d, m;
-  __device__ explicit FastDiv(u32 dd) : d(dd), m(static_cast<u32>(((1ull << 32) + dd - 1) / dd)) {}
+  __device__ explicit FastDiv(u32 dd) : d(dd), m(0xFFFFFFFFu / dd + 1u) {}
   __device__ __forceinline__ u32 div(u32 n) const {
     u32 q = __umulhi(n, m);
     if (q * d > n) --q;
@@ -821,24 +822,33 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
 
   // QK^T of one INT4 tile block: logits (log2 units) of rows gq and gq + 8 for head tig.
   auto qk_int4 = [&](const uint8_t* tb, bool v0, bool v1, float& lg0, float& lg1) {
-    uint32_t kw0[WPC], kw1[WPC];
-    lds_words<WPC>(tb + gq * (D / 2) + tig * Gm::CH, kw0);
-    lds_words<WPC>(tb + (gq + 8) * (D / 2) + tig * Gm::CH, kw1);
+    // pair-row gq holds rows gq (low nibbles) and gq + 8 (high nibbles); this lane's 8-dim
+    // groups 4 tig .. 4 tig + 3 are 8 W bytes at 8 W tig (16-byte halves swapped for odd gq
+    // when D = 128): per group, word 0 = its even dims, word 1 = its odd dims
+    uint32_t kw[2 * WPC];
+    if constexpr (D == 128) {
+      const int sw = gq & 1;
+      lds_words<4>(tb + gq * D + 16 * ((2 * tig) ^ sw), *reinterpret_cast<uint32_t(*)[4]>(&kw[0]));
+      lds_words<4>(tb + gq * D + 16 * ((2 * tig + 1) ^ sw), *reinterpret_cast<uint32_t(*)[4]>(&kw[4]));
+    } else {
+      lds_words<4>(tb + gq * D + 16 * tig, *reinterpret_cast<uint32_t(*)[4]>(&kw[0]));
+    }
     int SA[4] = {0, 0, 0, 0}, SB[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int j = 0; j < NK32; ++j) {
-      // word j of a row holds the codes of dims 8W..8W+7 (W = WPC tig + j), dim 8W + n at bits
-      // 4n: the low nibbles of its bytes are the even dims, the high nibbles the odd dims.
-      const uint32_t l0 = kw0[j] & 0x0F0F0F0Fu, h0 = (kw0[j] >> 4) & 0x0F0F0F0Fu;
-      const uint32_t l1 = kw1[j] & 0x0F0F0F0Fu, h1 = (kw1[j] >> 4) & 0x0F0F0F0Fu;
-      mma_u8s8(SA, l0, l1, h0, h1, qd[j][0], qd[j][1]);
-      mma_u8s8(SB, l0, l1, h0, h1, qd[j][2], qd[j][3]);
+      // A fragment: row gq = low nibbles, row gq + 8 = high nibbles kept in place (16 c, the
+      // factor is removed from that row's logit below); k 0-15 even dims, k 16-31 odd dims
+      const uint32_t e = kw[2 * j], o = kw[2 * j + 1];
+      const uint32_t a0 = e & 0x0F0F0F0Fu, a1 = e & 0xF0F0F0F0u;
+      const uint32_t a2 = o & 0x0F0F0F0Fu, a3 = o & 0xF0F0F0F0u;
+      mma_u8s8(SA, a0, a1, a2, a3, qd[j][0], qd[j][1]);
+      mma_u8s8(SB, a0, a1, a2, a3, qd[j][2], qd[j][3]);
     }
     const uint32_t kp0 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 4 * gq);
     const uint32_t kp1 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 4 * (gq + 8));
-    const float ks0 = half_lo(kp0), kz0 = half_hi(kp0), ks1 = half_lo(kp1), kz1 = half_hi(kp1);
+    const float ks0 = half_lo(kp0), kz0 = half_hi(kp0), ks1 = half_lo(kp1) * 0.0625f, kz1 = half_hi(kp1);
     // logit 2^e = s q_int.c + z sum(q_int), q_int.c = 2^16 S2 + (2^8 S1 + S0); the bracket is
-    // below 2^26 in magnitude and exact in int32
+    // below 2^30 in magnitude and exact in int32 (row gq + 8: 16 q_int.c, hence s / 16)
     const float R0 = fmaf(65536.f, static_cast<float>(SA[0]), static_cast<float>(SA[1] * 256 + SB[0]));
     const float R1 = fmaf(65536.f, static_cast<float>(SA[2]), static_cast<float>(SA[3] * 256 + SB[2]));
     lg0 = v0 ? fmaf(ks0, R0, kz0 * sumq) : kNegInf;

@@ -9,7 +9,11 @@
 //
 // INT4 page pool (one layer): page = Hkv head blocks of P*(D+8) bytes; head block = P/16 tiles
 // of T4B = 16*(D+8) bytes; in a tile (row r = position % 16):
-//   [0, 8D)            K codes, row-major: byte r*D/2 + e/2, low nibble = even element.
+//   [0, 8D)            K codes in 8 pair-rows of D bytes: pair-row p = r % 8 holds row p in the
+//                      low nibbles and row p + 8 in the high nibbles, one byte per element e:
+//                      byte 8*(e/8) + 4*(e%2) + (e%8)/2 (even elements, then odd, per 8-group);
+//                      for D = 128 the 16-byte halves of each 32 bytes are swapped in odd
+//                      pair-rows.  A decode lane's unpack is then one mask per four codes.
 //   [8D, 16D)          V codes: 16-bit chunk (r, quad Q) holds elements 4Q..4Q+3 (4Q+k in bits
 //                      4k..4k+3); rows 2p, 2p+1 share a 32-bit word (2p low half); word groups
 //                      at byte ((half*8 + Q/WPC)*4 + (p&3))*CH + 4*(Q%WPC), half = p>>2.

@@ -210,8 +210,11 @@ void orc_quant_int8(const float* x, int D, int8_t* codes8, uint16_t* scale) {
 /*
  * Page pool of one layer: pages of P positions; a page holds Hkv head blocks of P*(D+8)
  * bytes; a head block holds P/16 tile blocks of 16*(D+8) bytes, one per 16 positions:
- *   [0, 8D)          K codes, row r (position in tile) at r*D/2, element e in byte e/2,
- *                    low nibble for even e.
+ *   [0, 8D)          K codes in 8 pair-rows of D bytes: pair-row p holds rows p (low nibbles)
+ *                    and p + 8 (high nibbles), one byte per element.  In a pair-row, element e
+ *                    is in 8-byte group e/8, byte (e%8)/2 for even e and 4 + (e%8)/2 for odd e;
+ *                    for D >= 128 the two 16-byte halves of every 32 bytes are swapped in odd
+ *                    pair-rows.
  *   [8D, 16D)        V codes in 16-bit chunks: chunk (r, Q) holds elements 4Q..4Q+3 of row r
  *                    (element 4Q+k in byte k/2, low nibble for even k); the chunks of rows
  *                    2p and 2p+1 sit side by side in one 32-bit word, and words are grouped
@@ -246,8 +249,16 @@ static size_t tile4_base(const orc_config* c, int page, int g, int pp) {
 }
 
 size_t orc_k4_byte(const orc_config* c, int page, int g, int pp, int e) {
-  const int D = c->head_dim, r = pp % 16;
-  return tile4_base(c, page, g, pp) + (size_t)r * (size_t)(D / 2) + (size_t)(e / 2);
+  const int D = c->head_dim, pr = (pp % 16) & 7;
+  const int b = 8 * (e / 8) + (e % 2) * 4 + (e % 8) / 2;  /* byte within the pair-row */
+  const int unit = (b / 16) ^ (D >= 128 ? (pr & 1) : 0);
+  return tile4_base(c, page, g, pp) + (size_t)pr * (size_t)D + (size_t)(16 * unit + b % 16);
+}
+
+int orc_k4_high(const orc_config* c, int pp, int e) {
+  (void)c;
+  (void)e;
+  return (pp % 16) >> 3;
 }
 
 size_t orc_v4_byte(const orc_config* c, int page, int g, int pp, int e) {
@@ -358,7 +369,7 @@ int orc_append(const orc_config* c, uint8_t* pool, uint8_t* side, int T, const v
       if (c->rotate_values) orc_rotate_key(c, vf);
       uint16_t sc, zr;
       orc_quant_int4(kf, D, c4, &sc, &zr);
-      for (int e = 0; e < D; ++e) put_nibble(pool, orc_k4_byte(c, page, g, pp, e), e & 1, c4[e]);
+      for (int e = 0; e < D; ++e) put_nibble(pool, orc_k4_byte(c, page, g, pp, e), orc_k4_high(c, pp, e), c4[e]);
       put_u16(pool, orc_p4_byte(c, page, g, pp, 0), sc);
       put_u16(pool, orc_p4_byte(c, page, g, pp, 0) + 2, zr);
       orc_quant_int4(vf, D, c4, &sc, &zr);
@@ -418,7 +429,7 @@ int orc_dequant_seq(const orc_config* c, const uint8_t* pool, const uint8_t* sid
       const double vs = (double)orc_f16_to_f32(get_u16(pool, vp));
       const double vz = (double)orc_f16_to_f32(get_u16(pool, vp + 2));
       for (int e = 0; e < D; ++e) {
-        kr[e] = kz + ks * (double)get_nibble(pool, orc_k4_byte(c, page, g, pp, e), e & 1);
+        kr[e] = kz + ks * (double)get_nibble(pool, orc_k4_byte(c, page, g, pp, e), orc_k4_high(c, pp, e));
         vr[e] = vz + vs * (double)get_nibble(pool, orc_v4_byte(c, page, g, pp, e), e & 1);
       }
     }

@@ -73,6 +73,9 @@ int    orc_side_tiles(const orc_config* c);          /* 16-row tiles per (slot, 
 
 /* Byte offsets inside one layer's page pool / side cache (exposed for the layout pins). */
 size_t orc_k4_byte(const orc_config* c, int page, int g, int pos_in_page, int elem);
+/* 1 when element elem of the K codes at pos_in_page is the high nibble of its byte (rows 8-15
+ * of a tile), else 0.  V codes: the high nibble holds the odd elements (elem & 1). */
+int    orc_k4_high(const orc_config* c, int pos_in_page, int elem);
 size_t orc_v4_byte(const orc_config* c, int page, int g, int pos_in_page, int elem);
 size_t orc_p4_byte(const orc_config* c, int page, int g, int pos_in_page, int is_v);
 size_t orc_k8_byte(const orc_config* c, int slot, int g, int row, int elem);

@@ -104,6 +104,8 @@ def lib():
         for n in ("orc_k4_byte", "orc_v4_byte", "orc_p4_byte", "orc_k8_byte", "orc_v8_byte", "orc_s8_byte"):
             getattr(L, n).argtypes = [cfgp, I, I, I, I]
             getattr(L, n).restype = S
+        L.orc_k4_high.argtypes = [cfgp, I, I]
+        L.orc_k4_high.restype = I
         L.orc_side_row.argtypes = [cfgp, I]
         L.orc_side_row.restype = I
         L.orc_append.argtypes = [cfgp, P, P, I, P, I, P, I, P, P, P, P, I]
@@ -193,6 +195,14 @@ def byte_offset(kind: str, cfg: Config, a: int, g: int, r: int, e: int) -> int:
     """kind in {k4, v4, p4, k8, v8, s8}; (a, g, r, e) = (page or slot, kv head, position in
     page or side row, element or is_v)."""
     return int(getattr(lib(), f"orc_{kind}_byte")(ctypes.byref(cfg.c()), a, g, r, e))
+
+
+def nibble_high(kind: str, cfg: Config, r: int, e: int) -> int:
+    """1 if element e of the INT4 codes at position-in-page r is the high nibble of the byte
+    byte_offset(kind, ...) names (kind k4 or v4), else 0."""
+    if kind == "k4":
+        return int(lib().orc_k4_high(ctypes.byref(cfg.c()), r, e))
+    return e & 1
 
 
 def side_row(cfg: Config, pos: int) -> int:

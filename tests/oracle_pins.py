@@ -259,8 +259,8 @@ def pin_layout_bijection():
         for g in range(Hkv):
             for pp in range(P):
                 for e in range(D):
-                    nib[2 * O.byte_offset("k4", cfg, 1, g, pp, e) - 2 * pb + (e & 1)] += 1
-                    nib[2 * O.byte_offset("v4", cfg, 1, g, pp, e) - 2 * pb + (e & 1)] += 1
+                    nib[2 * O.byte_offset("k4", cfg, 1, g, pp, e) - 2 * pb + O.nibble_high("k4", cfg, pp, e)] += 1
+                    nib[2 * O.byte_offset("v4", cfg, 1, g, pp, e) - 2 * pb + O.nibble_high("v4", cfg, pp, e)] += 1
                 for isv in (0, 1):
                     off = O.byte_offset("p4", cfg, 1, g, pp, isv) - pb
                     nib[2 * off:2 * off + 8] += 1
@@ -384,8 +384,14 @@ def _brute_layout_decode(wl: W.Workload, pool, side, b: int, g: int, L: int):
             ks, kz = f16(pool, base + 16 * D + 4 * r), f16(pool, base + 16 * D + 4 * r + 2)
             vs, vz = f16(pool, base + 16 * D + 64 + 4 * r), f16(pool, base + 16 * D + 64 + 4 * r + 2)
             for e in range(D):
-                byte = pool[base + r * (D // 2) + e // 2]
-                kh[j, e] = kz + ks * ((byte >> 4) if e & 1 else (byte & 15))
+                # K: pair-row r % 8 of D bytes, row r in the low (r < 8) or high nibble; element e
+                # in 8-byte group e // 8 (even elements first); 16-byte halves of each 32 bytes
+                # swapped in odd pair-rows when D >= 128
+                pr = r % 8
+                bi = 8 * (e // 8) + (e % 2) * 4 + (e % 8) // 2
+                unit = (bi // 16) ^ ((pr % 2) if D >= 128 else 0)
+                byte = pool[base + pr * D + 16 * unit + bi % 16]
+                kh[j, e] = kz + ks * ((byte >> 4) if r >= 8 else (byte & 15))
                 Q, k = e // 4, e % 4
                 wpc = D // 32
                 p_ = r >> 1
@@ -398,8 +404,9 @@ def _brute_layout_decode(wl: W.Workload, pool, side, b: int, g: int, L: int):
 def pin_brute_force(seed: int = 21):
     """Tiny cases: the oracle's decode against a direct fp64 triple loop with an explicit
     Hadamard matrix, on a cache read back through an independent layout decoder."""
-    for (lens, s, w, h, G) in (((12, 7, 3), 2, 5, 8, 2), ((11, 1, 9), 0, 4, 32, 1), ((10, 12, 5), 3, 0, 4, 2)):
-        wl = small_workload(lens=lens, s=s, w=w, h=h, G=G, seed=seed)
+    for (lens, s, w, h, G, D) in (((12, 7, 3), 2, 5, 8, 2, 32), ((11, 1, 9), 0, 4, 32, 1, 32),
+                                  ((10, 12, 5), 3, 0, 4, 2, 32), ((21, 3), 1, 2, 16, 1, 128)):
+        wl = small_workload(D=D, lens=lens, s=s, w=w, h=h, G=G, seed=seed)
         cfg, pool, side = build_cache(wl)
         q = wl.q_input(0)
         out, lse = O.decode(cfg, pool, side, q, wl.page_table, wl.lens)
@@ -436,8 +443,8 @@ def pin_append_vs_numpy_requant(seed: int = 31):
                 for isv, x in ((0, kr), (1, V[j, g])):
                     codes, sc, zr = _requant_int4_numpy(x)
                     kind = "v4" if isv else "k4"
-                    got = np.array([(pool[O.byte_offset(kind, cfg, page, g, pp, e)] >> (4 * (e & 1))) & 15
-                                    for e in range(wl.D)])
+                    got = np.array([(pool[O.byte_offset(kind, cfg, page, g, pp, e)]
+                                     >> (4 * O.nibble_high(kind, cfg, pp, e))) & 15 for e in range(wl.D)])
                     assert np.array_equal(got, codes), (b, j, g, isv)
                     off = O.byte_offset("p4", cfg, page, g, pp, isv)
                     assert int(pool[off]) | (int(pool[off + 1]) << 8) == sc

@@ -26,8 +26,9 @@ MUTANTS = [
     ("int4-truncate", "const float rq = rintf(t);", "const float rq = truncf(t);", None),
     ("int8-levels-128", "a / 127.0f", "a / 128.0f", None),
     ("int8-scale-round-nearest", "orc_f32_to_f16(a / 127.0f, ORC_RU)", "orc_f32_to_f16(a / 127.0f, ORC_RN)", None),
-    ("nibble-swap", "put_nibble(pool, orc_k4_byte(c, page, g, pp, e), e & 1, c4[e]);",
-     "put_nibble(pool, orc_k4_byte(c, page, g, pp, e), (e & 1) ^ 1, c4[e]);", None),
+    ("nibble-swap", "put_nibble(pool, orc_k4_byte(c, page, g, pp, e), orc_k4_high(c, pp, e), c4[e]);",
+     "put_nibble(pool, orc_k4_byte(c, page, g, pp, e), orc_k4_high(c, pp, e) ^ 1, c4[e]);", None),
+    ("k4-pair-row-no-swizzle", "(b / 16) ^ (D >= 128 ? (pr & 1) : 0)", "(b / 16)", None),
     ("v4-pair-index", "4 * j + 2 * (r & 1) + (k >> 1)", "4 * j + 2 * ((r >> 1) & 1) + (k >> 1)", None),
     ("k8-no-swizzle", "16 * ((e / 16) ^ (r & 1))", "16 * (e / 16)", None),
     ("route-ring-strict", "p >= lens_after[b] - w", "p > lens_after[b] - w", None),

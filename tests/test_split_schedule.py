@@ -116,3 +116,26 @@ def test_schedule_invariants(seed):
 def test_lengths_beyond_page_table_are_clamped():
     # a length past stride*P is clamped to it (the merge kernel also raises a device error bit)
     model([10_000, 5], 2, 4, 32, 16, 4, 64)
+
+
+def test_fast_division_multiplier():
+    """The decode kernel divides by the per-launch unit count Q >= 2 as umulhi(n, m) with
+    m = floor((2^32 - 1) / Q) + 1, corrected by one multiply-compare.  m equals ceil(2^32 / Q)
+    for every Q >= 2, and the corrected quotient is exact for n < 2^31."""
+    import numpy as np
+    rng = np.random.default_rng(5)
+    # Q < 2^31: the unit total is below 2^31 (the host refuses larger launches)
+    ds = [2, 3, 4, 7, 8, 1000, 1024, 65535, 65536, 2**30 + 3, 2**31 - 1]
+    ds += [int(x) for x in rng.integers(2, 2**31, size=200)]
+    for d in ds:
+        m = (2**32 - 1) // d + 1
+        assert m == -(-2**32 // d)
+        assert m < 2**32
+        ns = [0, 1, d - 1, d, d + 1, 2**31 - 1] + [int(x) for x in rng.integers(0, 2**31, size=50)]
+        for n in ns:
+            if n >= 2**31:
+                continue
+            q = (n * m) >> 32                 # umulhi
+            if (q * d) & 0xFFFFFFFF > n:      # 32-bit product, as in the kernel (q d < 2^32 here)
+                q -= 1
+            assert q == n // d, (n, d)
