@@ -43,6 +43,9 @@ def parse():
     ap.add_argument("--impl", choices=["kv4", "reference"], default="kv4")
     ap.add_argument("--workload", default="qwen3-4b-decode")
     ap.add_argument("--h", type=int, default=None, help="Hadamard block of the 36-layer workload (32, 64, 128)")
+    ap.add_argument("--sinks", type=int, default=None, help="override s, the INT8 sink positions")
+    ap.add_argument("--recent", type=int, default=None,
+                    help="override w, the INT8 recent window (-1: every position, i.e. all-INT8 KV8)")
     ap.add_argument("--no-bf16", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
@@ -61,7 +64,15 @@ def make_wl(args):
     from int4_kv_cache_append_b200 import workload as W
     fn = W.WORKLOADS[args.workload]
     h = getattr(args, "h", None)
-    return fn(h=h) if h is not None else fn()
+    wl = fn(h=h) if h is not None else fn()
+    # sink / recent budgets (KV4-RL "Main Findings": s/w sweep; KV8 = every position in INT8)
+    s, w = getattr(args, "sinks", None), getattr(args, "recent", None)
+    if s is not None or w is not None:
+        import dataclasses
+        s = wl.s if s is None else s
+        w = wl.w if w is None else (int(wl.max_lens.max()) if w < 0 else w)
+        wl = dataclasses.replace(wl, s=s, w=w, name=f"{wl.name}-s{s}-w{w}")
+    return wl
 
 
 # ----------------------------------------------------------------------------- helpers

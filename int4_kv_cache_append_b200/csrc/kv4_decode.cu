@@ -70,10 +70,21 @@ struct SegInfo {
 
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
 
+// Side tiles visited: those up to the highest side row that holds a position.  Until the recent
+// ring has wrapped (L - s + (s mod w) <= w) that row is below L + (s mod w), so short sequences
+// (and the all-INT8 configuration, w >= every length) read only the tiles they fill.
+__device__ __forceinline__ int side_tiles_used(int L, int s, int w, int nt8) {
+  if (L <= 0) return 0;
+  if (L <= s) return min(nt8, (L + 15) >> 4);
+  if (w <= 0 || L - s >= w) return nt8;
+  const int top = s + (s % w) + (L - s);  // one past the last ring row, if not wrapped
+  return top <= s + w ? min(nt8, (top + 15) >> 4) : nt8;
+}
+
 __device__ __forceinline__ SegInfo seg_info(int L, int s, int w, int nt8) {
   SegInfo r;
   r.L = L;
-  r.n8 = L > 0 ? nt8 : 0;
+  r.n8 = side_tiles_used(L, s, w, nt8);
   r.m_end = max(s, L - w);
   r.t4a = s >> 4;
   r.n4 = (r.m_end > s) ? ((r.m_end - 1) >> 4) - r.t4a + 1 : 0;

@@ -17,8 +17,28 @@ import pytest
 
 
 
+def side_tiles_used(L, s, w, nt8):
+    if L <= 0:
+        return 0
+    if L <= s:
+        return min(nt8, (L + 15) // 16)
+    if w <= 0 or L - s >= w:
+        return nt8
+    top = s + s % w + (L - s)
+    return min(nt8, (top + 15) // 16) if top <= s + w else nt8
+
+
+def side_rows_used(L, s, w):
+    """Side rows holding a position at length L: sinks j < min(s, L) at row j, recent
+    j in [max(s, L - w), L) at row s + j mod w."""
+    rows = set(range(min(s, L)))
+    if w > 0:
+        rows |= {s + j % w for j in range(max(s, L - w), L)}
+    return rows
+
+
 def seg_info(L, s, w, nt8):
-    n8 = nt8 if L > 0 else 0
+    n8 = side_tiles_used(L, s, w, nt8)
     m_end = max(s, L - w)
     t4a = s >> 4
     n4 = ((m_end - 1) >> 4) - t4a + 1 if m_end > s else 0
@@ -89,6 +109,8 @@ def model(lens, Hkv, s, w, P, stride, W):
                 jme = (wr - w8a) if seg == 0 else n8p + (wr - w4a)
                 assert jme == j
             assert (len(parts) == 1) == (n8p + n4p == 1)
+        # the visited side tiles hold every side row in use
+        assert all(r < 16 * n8 for r in side_rows_used(L, s, w))
         # INT4 tiles address pages inside the page-table row
         for i in range(n4):
             ti = t4a + i
@@ -108,6 +130,10 @@ def test_schedule_invariants(seed):
     lens = rng.integers(0, 3000, size=B).tolist()
     if seed % 5 == 0:
         lens = [1, 0, s, s + 1, s + w, s + w + 1][:B] + lens[6:]
+    if seed % 5 == 1:  # short sequences and the all-INT8 configuration (w above every length)
+        lens = rng.integers(0, 2 * (s + w) + 3, size=B).tolist()
+    if seed % 7 == 3:
+        s, w = 0, int(max(lens)) + int(rng.integers(0, 40))
     stride = max(1, (max(lens) + P - 1) // P)
     for W in (1, 3, 8, 37, 296, 2368):
         model(lens, Hkv, s, w, P, stride, W)
@@ -139,3 +165,18 @@ def test_fast_division_multiplier():
             if (q * d) & 0xFFFFFFFF > n:      # 32-bit product, as in the kernel (q d < 2^32 here)
                 q -= 1
             assert q == n // d, (n, d)
+
+
+def test_side_tiles_used_cover_every_side_row():
+    """Exhaustive over small budgets: the side tiles a decode visits hold every side row in use,
+    and a sequence whose ring has not wrapped visits no tile past its last used row."""
+    for s in range(0, 40, 3):
+        for w in (0, 1, 5, 16, 17, 40):
+            nt8 = (s + w + 15) // 16
+            for L in range(0, 2 * (s + w) + 20):
+                n8 = side_tiles_used(L, s, w, nt8)
+                rows = side_rows_used(L, s, w)
+                assert 0 <= n8 <= nt8
+                assert all(r < 16 * n8 for r in rows), (s, w, L)
+                if rows and n8 < nt8:
+                    assert n8 == (max(rows) + 16) // 16, (s, w, L)
