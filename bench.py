@@ -506,56 +506,82 @@ def run_kv4(args, world, rank, local):
     # ---- e2e through the public API with host buffers (pinned), every step.  Each step copies the
     # inputs of every layer call it makes (q, K, V, slots, positions, lengths) from pinned host
     # memory, runs append + decode through the C ABI and copies the (last layer's) output back.
-    # Pipelined: inputs on an H2D stream and the output on a D2H stream, device buffers
-    # double-buffered and ordered by events, so the copies of one step overlap the kernels of the
-    # previous one.  The serial form (one stream) is reported beside it.
+    # The step's static inputs sit in one pinned buffer (one H2D copy), positions and lengths in a
+    # second small one (they change every step of a growing workload); the C entry points are
+    # called directly with device addresses.  Pipelined: inputs on an H2D stream and the output
+    # on a D2H stream, device buffers double-buffered and ordered by events, so the copies of one
+    # step overlap the kernels of the previous one.  The serial form (one stream) is reported
+    # beside it.
     e2e = None
     if args.e2e_steps > 0:
         nl = per_step  # layer calls per step
-        hkv = [(ins[l][0].cpu().pin_memory(), ins[l][1].cpu().pin_memory(), ins[l][2].cpu().pin_memory())
-               for l in range(nl if per_step > 1 else 1)]
-        hb = bt.cpu().pin_memory()
+        nsets = nl if per_step > 1 else 1
+        parts = []  # (host tensor, offset) of the static inputs
+        off = 0
+        for l in range(nsets):
+            for t in (ins[l][0], ins[l][1], ins[l][2]):
+                parts.append((t.cpu().contiguous(), off))
+                off += (t.numel() * t.element_size() + 255) // 256 * 256
+        hb = bt.cpu()
+        parts.append((hb, off))
+        off += (hb.numel() * 4 + 255) // 256 * 256
+        hpack = torch.empty(off, dtype=torch.uint8).pin_memory()
+        for t, o in parts:
+            nb = t.numel() * t.element_size()
+            hpack[o:o + nb].copy_(t.view(-1).view(torch.uint8))
         nst = max(grow, 1)
         hst = [torch.from_numpy(np.stack([lens0 - 1 + k, lens0 + k])).pin_memory() for k in range(nst)]
-        dbuf = [{"kvq": [tuple(torch.empty_like(t, device=dev) for t in h) for h in hkv],
-                 "b": torch.empty_like(hb, device=dev), "st": torch.empty_like(hst[0], device=dev),
-                 "out": torch.empty_like(S.out)} for _ in range(2)]
+        dpack = [torch.empty_like(hpack, device=dev) for _ in range(2)]
+        dst = [torch.empty_like(hst[0], device=dev) for _ in range(2)]
+        douts = [torch.empty_like(S.out) for _ in range(2)]
         houts = [torch.empty_like(S.out, device="cpu").pin_memory() for _ in range(2)]
-        h2d = sum(t.numel() * t.element_size() for h in hkv for t in h) + hb.numel() * 4 + hst[0].numel() * 4
+        h2d = sum(t.numel() * t.element_size() for t, _ in parts) + hst[0].numel() * 4
         d2h = houts[0].numel() * houts[0].element_size()
+        kd, vd, qd = kv4.dtype_code(ins[0][0]), kv4.dtype_code(ins[0][1]), kv4.dtype_code(ins[0][2])
+        ws = S.ws
+        pt_ptr, stride = S.page_table.data_ptr(), int(S.page_table.shape[1])
+        calls = []  # per buffer: the (append args, decode args) of every layer call
+        for j in range(2):
+            base = dpack[j].data_ptr()
+            slot_p = base + parts[-1][1]
+            pos_p, len_p = dst[j].data_ptr(), dst[j].data_ptr() + 4 * B
+            cj = []
+            for li, layer in enumerate(range(nl) if per_step > 1 else [None]):
+                kp, vp, qp = (base + parts[3 * li + x][1] for x in range(3))
+                cj.append((kp, vp, qp, slot_p, pos_p, len_p))
+            calls.append(cj)
+        handle = cache.handle
         up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        sh_main = stream.cuda_stream
         ev_in = [torch.cuda.Event() for _ in range(2)]
         ev_done = [torch.cuda.Event() for _ in range(2)]
         ev_out = [torch.cuda.Event() for _ in range(2)]
         for e in ev_done + ev_out:
             e.record(stream)
+        lib = kv4.lib
 
         def step_on(j, i, pipelined):
-            d = dbuf[j]
-            cs = up if pipelined else stream
             if pipelined:
                 up.wait_event(ev_done[j])  # the step that last used buffer j has finished
-            with torch.cuda.stream(cs):
-                for dd, hh in zip(d["kvq"], hkv):
-                    for d_, h_ in zip(dd, hh):
-                        d_.copy_(h_, non_blocking=True)
-                d["b"].copy_(hb, non_blocking=True)
-                d["st"].copy_(hst[i % nst], non_blocking=True)
+            with torch.cuda.stream(up if pipelined else stream):
+                dpack[j].copy_(hpack, non_blocking=True)
+                dst[j].copy_(hst[i % nst], non_blocking=True)
             if pipelined:
                 ev_in[j].record(up)
                 stream.wait_event(ev_in[j])
                 stream.wait_event(ev_out[j])  # its previous output has been copied out
             layers = range(nl) if per_step > 1 else [i % resident]
-            for li, layer in enumerate(layers):
-                dK, dV, dq = d["kvq"][li if per_step > 1 else 0]
-                cache.append(layer, dK, dV, d["b"], d["st"][0], d["st"][1], S.page_table, stream=stream)
-                cache.decode(layer, dq, S.page_table, d["st"][1], out=d["out"], max_len_hint=maxlen,
-                             workspace=S.ws, stream=stream)
+            for (kp, vp, qp, slot_p, pos_p, len_p), layer in zip(calls[j] * (1 if per_step > 1 else 1), layers):
+                st_ = lib.kv4_append(handle, layer, B, kp, kd, vp, vd, slot_p, pos_p, len_p, pt_ptr, stride, sh_main)
+                sd_ = lib.kv4_decode_attn(handle, layer, B, qp, qd, pt_ptr, stride, len_p, maxlen,
+                                          douts[j].data_ptr(), None, ws.data_ptr(), ws.numel(), sh_main)
+                if st_ or sd_:
+                    raise RuntimeError(f"kv4 call failed: append {st_}, decode {sd_}")
             if pipelined:
                 ev_done[j].record(stream)
                 down.wait_event(ev_done[j])
             with torch.cuda.stream(down if pipelined else stream):
-                houts[j].copy_(d["out"], non_blocking=True)
+                houts[j].copy_(douts[j], non_blocking=True)
             if pipelined:
                 ev_out[j].record(down)
 
@@ -580,10 +606,10 @@ def run_kv4(args, world, rank, local):
         e2e = {"value": whole_job_rate(B * args.e2e_steps, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                "e2e_serial": whole_job_rate(B * args.e2e_steps, world, serial_ms),
-               "path": "kv4.Cache.append + kv4.Cache.decode (C ABI) for every layer call of the step; every step "
-                       "copies the inputs of those calls from pinned host memory and the last output back; "
-                       "copies on H2D/D2H streams overlap the previous step's kernels (double-buffered); "
-                       "e2e_serial: the same on one stream"}
+               "path": "kv4_append + kv4_decode_attn (C ABI) for every layer call of the step; every step copies "
+                       "the inputs of those calls from pinned host memory (one packed buffer, plus positions and "
+                       "lengths) and the last output back; copies on H2D/D2H streams overlap the previous step's "
+                       "kernels (double-buffered); e2e_serial: the same on one stream"}
 
     del cache, ins, S
     torch.cuda.empty_cache()

@@ -22,7 +22,7 @@ namespace kv4 {
 namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
-constexpr int kAppendThreads = 1024;
+constexpr int kAppendThreads = 256;
 
 template <typename T>
 __device__ __forceinline__ void load4(const void* base, size_t i, float (&x)[4]);
@@ -289,8 +289,9 @@ __global__ void __launch_bounds__(kAppendThreads) append_bf16_kernel(AppendArgs 
 
 template <int D, bool BF16_POOL>
 cudaError_t dispatch_types(const AppendArgs& a, cudaStream_t st) {
-  // Few large blocks: a block of this kernel keeps the following decode kernel's block (which
-  // needs a whole SM) off its SM until it exits.
+  // 8-warp blocks: a block of this kernel keeps the following decode kernel's block (which needs a
+  // whole SM) off its SM until it exits, but spreading the append over more SMs ends it sooner,
+  // and that measured better for the whole step than fewer 32-warp blocks (0.0606 vs 0.0633 ms).
   const int warps = a.T * a.Hkv;
   const dim3 grid((warps + kAppendThreads / 32 - 1) / (kAppendThreads / 32)), block(kAppendThreads);
   const bool kf = a.k_dtype == KV4_F32, vf = a.v_dtype == KV4_F32;
