@@ -208,6 +208,7 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
   a.h = fmt == FMT_INT4 ? c->cfg.hadamard_block : 1;
   a.max_pages = c->cfg.max_pages;
   a.nt8 = c->nt8;
+  a.smw = a.w > 0 ? a.s % a.w : 0;
   a.page_bytes = c->page_bytes;
   a.side_slot_bytes = c->side_slot_bytes;
   a.meta = static_cast<unsigned int*>(ws);

@@ -70,21 +70,25 @@ struct SegInfo {
 
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
 
-// Side tiles visited: those up to the highest side row that holds a position.  Until the recent
-// ring has wrapped (L - s + (s mod w) <= w) that row is below L + (s mod w), so short sequences
-// (and the all-INT8 configuration, w >= every length) read only the tiles they fill.
-__device__ __forceinline__ int side_tiles_used(int L, int s, int w, int nt8) {
-  if (L <= 0) return 0;
-  if (L <= s) return min(nt8, (L + 15) >> 4);
-  if (w <= 0 || L - s >= w) return nt8;
-  const int top = s + (s % w) + (L - s);  // one past the last ring row, if not wrapped
-  return top <= s + w ? min(nt8, (top + 15) >> 4) : nt8;
+// Side tiles visited: those up to the highest side row that holds a position.  Position j < s
+// is row j; position j >= s is row s + (j mod w), so until the recent ring wraps
+// (L + (s mod w) <= s + w) the rows in use end at L + (s mod w) (at L when L <= s): short
+// sequences, and the all-INT8 configuration (w >= every length), read only the tiles they fill.
+// smw = s mod w, precomputed on the host (0 when w = 0, which always gives nt8 for L > s).
+__device__ __forceinline__ int side_tiles_used(int L, int s, int w, int nt8, int smw) {
+  const int top = L <= s ? L : L + smw;
+  return L <= 0 ? 0 : (top <= s + w ? (top + 15) >> 4 : nt8);
 }
 
-__device__ __forceinline__ SegInfo seg_info(int L, int s, int w, int nt8) {
+// T8: side caches larger than kTightSideTiles tiles (long recent windows, the all-INT8
+// configuration) visit only the side tiles in use; smaller ones visit all of theirs (a few tiles,
+// masked), which keeps this bound out of the common kernels' code.
+constexpr int kTightSideTiles = 16;
+template <bool T8>
+__device__ __forceinline__ SegInfo seg_info(int L, int s, int w, int nt8, int smw) {
   SegInfo r;
   r.L = L;
-  r.n8 = side_tiles_used(L, s, w, nt8);
+  r.n8 = T8 ? side_tiles_used(L, s, w, nt8, smw) : (L > 0 ? nt8 : 0);
   r.m_end = max(s, L - w);
   r.t4a = s >> 4;
   r.n4 = (r.m_end > s) ? ((r.m_end - 1) >> 4) - r.t4a + 1 : 0;
@@ -93,8 +97,9 @@ __device__ __forceinline__ SegInfo seg_info(int L, int s, int w, int nt8) {
 
 __device__ __forceinline__ u32 head_cost(const SegInfo& si) { return 2u * si.n8 + si.n4; }
 
+template <bool T8>
 __device__ __forceinline__ u32 seq_cost(const DecodeArgs& a, int cap, int b) {
-  return static_cast<u32>(a.Hkv) * head_cost(seg_info(clamp_len(a.lens[b], cap), a.s, a.w, a.nt8));
+  return static_cast<u32>(a.Hkv) * head_cost(seg_info<T8>(clamp_len(a.lens[b], cap), a.s, a.w, a.nt8, a.smw));
 }
 
 __device__ __forceinline__ u32 warp_incl_scan(u32 v, int lane) {
@@ -106,22 +111,24 @@ __device__ __forceinline__ u32 warp_incl_scan(u32 v, int lane) {
   return v;
 }
 
+template <bool T8>
 __device__ u32 total_cost(const DecodeArgs& a, int cap, int lane) {
   u32 run = 0;
   for (int base = 0; base < a.B; base += 32) {
     const int b = base + lane;
-    const u32 c = b < a.B ? seq_cost(a, cap, b) : 0u;
+    const u32 c = b < a.B ? seq_cost<T8>(a, cap, b) : 0u;
     run += __shfl_sync(FULL, warp_incl_scan(c, lane), 31);
   }
   return run;
 }
 
 // Sequence containing unit c (c < total); *bstart = first unit of that sequence.
+template <bool T8>
 __device__ int find_seq(const DecodeArgs& a, int cap, int lane, u32 c, u32* bstart) {
   u32 run = 0;
   for (int base = 0; base < a.B; base += 32) {
     const int b = base + lane;
-    const u32 cb = b < a.B ? seq_cost(a, cap, b) : 0u;
+    const u32 cb = b < a.B ? seq_cost<T8>(a, cap, b) : 0u;
     const u32 incl = warp_incl_scan(cb, lane);
     const u32 tot = __shfl_sync(FULL, incl, 31);
     if (c < run + tot) {
@@ -161,6 +168,7 @@ struct Cursor {
 };
 
 // Move forward to the first non-empty segment at or after the current one.
+template <bool T8>
 __device__ void settle(const DecodeArgs& a, int cap, Cursor& c) {
   while (true) {
     if (c.b >= a.B) {
@@ -177,7 +185,7 @@ __device__ void settle(const DecodeArgs& a, int cap, Cursor& c) {
       c.cs8 += head_cost(c.si);
       if (++c.g == a.Hkv) {
         c.g = 0;
-        if (++c.b < a.B) c.si = seg_info(clamp_len(a.lens[c.b], cap), a.s, a.w, a.nt8);
+        if (++c.b < a.B) c.si = seg_info<T8>(clamp_len(a.lens[c.b], cap), a.s, a.w, a.nt8, a.smw);
       }
     }
   }
@@ -189,12 +197,13 @@ __device__ __forceinline__ void recost(Cursor& c) {
 }
 
 // First tile whose first unit is >= c0, in sequence b (first unit bstart, raw length Lraw).
+template <bool T8>
 __device__ Cursor cursor_at(const DecodeArgs& a, int cap, int b, u32 bstart, u32 c0, int Lraw) {
   Cursor c;
   c.b = b;
   c.valid = b < a.B;
   if (!c.valid) return c;
-  c.si = seg_info(clamp_len(Lraw, cap), a.s, a.w, a.nt8);
+  c.si = seg_info<T8>(clamp_len(Lraw, cap), a.s, a.w, a.nt8, a.smw);
   const u32 ch = head_cost(c.si);
   const u32 off = c0 - bstart;
   c.g = static_cast<int>(off / ch);
@@ -207,7 +216,7 @@ __device__ Cursor cursor_at(const DecodeArgs& a, int cap, int b, u32 bstart, u32
     c.seg = 1;
     c.i = static_cast<int>(r - 2u * c.si.n8);
   }
-  settle(a, cap, c);
+  settle<T8>(a, cap, c);
   if (c.valid) recost(c);
   return c;
 }
@@ -283,7 +292,7 @@ __device__ __forceinline__ unsigned side_tile_mask(int i, int L, int s, int w) {
 // written to ring position (base + j) % kRing, plus one segment-table entry per segment entered.
 // `c` is advanced past them; slots past the warp's stream get kind None.  `segno` counts the
 // segments this warp has entered.
-template <int D>
+template <int D, bool T8>
 __device__ void fill_descriptors(const DecodeArgs& a, int cap, u32 c1, Cursor& c, int lane,
                                  Smem<D>& sm, int warp, int base, unsigned& segno) {
   using Gm = Geo<D>;
@@ -351,7 +360,7 @@ __device__ void fill_descriptors(const DecodeArgs& a, int cap, u32 c1, Cursor& c
     }
     done += take;
     if (c.i >= c.n) {
-      settle(a, cap, c);
+      settle<T8>(a, cap, c);
       ++segno;
       if (c.valid) recost(c);
     }
@@ -442,7 +451,7 @@ struct PartRows {
 
 // ------------------------------------------------------------------ the decode kernel
 
-template <int D, int G, int QT>
+template <int D, int G, int QT, bool T8>
 __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(const DecodeArgs a) {
   using Gm = Geo<D>;
   constexpr int NKB = Gm::NKB;
@@ -489,11 +498,11 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
 #pragma unroll
     for (int r = 0; r < kLensRegs; ++r)
       if (32 * r < a.B) {
-        const u32 c = 32 * r + lane < a.B ? static_cast<u32>(a.Hkv) * head_cost(seg_info(clamp_len(lr[r], cap), a.s, a.w, a.nt8)) : 0u;
+        const u32 c = 32 * r + lane < a.B ? static_cast<u32>(a.Hkv) * head_cost(seg_info<T8>(clamp_len(lr[r], cap), a.s, a.w, a.nt8, a.smw)) : 0u;
         total += __shfl_sync(FULL, warp_incl_scan(c, lane), 31);
       }
   } else {
-    total = total_cost(a, cap, lane);
+    total = total_cost<T8>(a, cap, lane);
   }
   const u32 Q = max(2u, (total + a.W - 1) / static_cast<u32>(a.W));
   const FastDiv divQ(Q);
@@ -508,7 +517,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
 #pragma unroll
     for (int r = 0; r < kLensRegs; ++r)
       if (32 * r < a.B && b0 == a.B) {
-        const u32 cb = 32 * r + lane < a.B ? static_cast<u32>(a.Hkv) * head_cost(seg_info(clamp_len(lr[r], cap), a.s, a.w, a.nt8)) : 0u;
+        const u32 cb = 32 * r + lane < a.B ? static_cast<u32>(a.Hkv) * head_cost(seg_info<T8>(clamp_len(lr[r], cap), a.s, a.w, a.nt8, a.smw)) : 0u;
         const u32 incl = warp_incl_scan(cb, lane);
         const u32 tot = __shfl_sync(FULL, incl, 31);
         if (c0 < run + tot) {
@@ -519,9 +528,9 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
         run += tot;
       }
   } else {
-    b0 = find_seq(a, cap, lane, c0, &bstart);
+    b0 = find_seq<T8>(a, cap, lane, c0, &bstart);
   }
-  Cursor dcur = cursor_at(a, cap, b0, bstart, c0, (any && b0 < a.B) ? (cached ? cached_len(b0) : a.lens[b0]) : 0);
+  Cursor dcur = cursor_at<T8>(a, cap, b0, bstart, c0, (any && b0 < a.B) ? (cached ? cached_len(b0) : a.lens[b0]) : 0);
   const bool active = any && dcur.valid && dcur.cost < c1;
 
   // Query of the first (b, g): loaded during the first descriptor fill, or after the wait on the
@@ -540,7 +549,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   if (active && !a.early) load_q_regs(qb0, qg0);  // in flight during the descriptor fill
 
   unsigned segno = 0;
-  if (active) fill_descriptors<D>(a, cap, c1, dcur, lane, sm, warp, 0, segno);
+  if (active) fill_descriptors<D, T8>(a, cap, c1, dcur, lane, sm, warp, 0, segno);
   // the cursor waits in shared memory between fills (its registers are free in the main loop)
   if (lane == 0) {
     sm.cur[warp] = dcur;
@@ -753,7 +762,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   auto flush = [&](unsigned long long se) {
     const int cb = seg_b(se), cg = seg_g(se), cseg = seg_kind(se);
     const u32 cs8 = seg_cs8(se);
-    const SegInfo si = seg_info(clamp_len(a.lens[cb], cap), a.s, a.w, a.nt8);
+    const SegInfo si = seg_info<T8>(clamp_len(a.lens[cb], cap), a.s, a.w, a.nt8, a.smw);
     float l = l_part, beta = beta_part;
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
@@ -908,7 +917,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
       Cursor fc = sm.cur[warp];
       unsigned fs = sm.segno[warp];
       __syncwarp();
-      fill_descriptors<D>(a, cap, c1, fc, lane, sm, warp, k + kChunk, fs);
+      fill_descriptors<D, T8>(a, cap, c1, fc, lane, sm, warp, k + kChunk, fs);
       if (lane == 0) {
         sm.cur[warp] = fc;
         sm.segno[warp] = fs;
@@ -1191,7 +1200,7 @@ cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t st) {
 template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
   const int smem = static_cast<int>(sizeof(Smem<D>));
-  static std::atomic<uint64_t> done[3];
+  static std::atomic<uint64_t> done[6];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ctas));
   cfg.blockDim = dim3(kWarps * 32);
@@ -1203,15 +1212,28 @@ cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (a.q_dtype == KV4_F32) {
-    if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F32>, smem, done[0])) != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_F32>, a);
-  } else if (a.q_dtype == KV4_BF16) {
-    if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_BF16>, smem, done[1])) != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_BF16>, a);
+  if (a.nt8 > kTightSideTiles) {
+    if (a.q_dtype == KV4_F32) {
+      if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F32, true>, smem, done[3])) != cudaSuccess) return e;
+      e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_F32, true>, a);
+    } else if (a.q_dtype == KV4_BF16) {
+      if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_BF16, true>, smem, done[4])) != cudaSuccess) return e;
+      e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_BF16, true>, a);
+    } else {
+      if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F16, true>, smem, done[5])) != cudaSuccess) return e;
+      e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_F16, true>, a);
+    }
   } else {
-    if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F16>, smem, done[2])) != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_F16>, a);
+    if (a.q_dtype == KV4_F32) {
+      if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F32, false>, smem, done[0])) != cudaSuccess) return e;
+      e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_F32, false>, a);
+    } else if (a.q_dtype == KV4_BF16) {
+      if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_BF16, false>, smem, done[1])) != cudaSuccess) return e;
+      e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_BF16, false>, a);
+    } else {
+      if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F16, false>, smem, done[2])) != cudaSuccess) return e;
+      e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_F16, false>, a);
+    }
   }
   if (e != cudaSuccess) return e;
   return launch_merge<D, G>(a, st);

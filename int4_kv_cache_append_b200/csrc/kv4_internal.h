@@ -38,6 +38,7 @@ struct DecodeArgs {
   int stride;
   const int32_t* lens;
   int B, Hq, Hkv, P, s, w, h, max_pages, nt8;
+  int smw;  // s mod w (0 when w = 0): where the recent ring starts being filled
   size_t page_bytes, side_slot_bytes;
   float* part;            // split partials [num_slots][G][D + 4]
   unsigned int* meta;     // per (b, g): first INT8 / INT4 partial warps and their counts

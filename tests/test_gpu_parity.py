@@ -29,6 +29,10 @@ CASES = [
     # KV8: no sinks and a recent window longer than every sequence, so every position is read
     # from the INT8 side cache
     ("d128-g4-kv8", 128, 8, 2, 16, 0, 208, 128, (200, 77, 1, 16, 17), W.BF16, W.BF16, W.BF16),
+    # side caches of more than 16 tiles: the decode visits only the side tiles in use (all-INT8
+    # with a window longer than every sequence; sinks with a long ring that wraps for some)
+    ("d64-g2-kv8-long-window", 64, 4, 2, 16, 0, 400, 64, (350, 77, 1, 16, 17, 260), W.BF16, W.BF16, W.BF16),
+    ("d128-g4-long-ring", 128, 8, 2, 16, 5, 300, 128, (20, 306, 400, 3, 305, 290), W.BF16, W.BF16, W.BF16),
     # more than 256 sequences: the decode prologue reads the lengths from memory instead of
     # keeping them in registers
     ("d64-g2-b300", 64, 4, 2, 16, 4, 16, 64,

@@ -18,14 +18,11 @@ import pytest
 
 
 def side_tiles_used(L, s, w, nt8):
-    if L <= 0:
-        return 0
-    if L <= s:
-        return min(nt8, (L + 15) // 16)
-    if w <= 0 or L - s >= w:
-        return nt8
-    top = s + s % w + (L - s)
-    return min(nt8, (top + 15) // 16) if top <= s + w else nt8
+    """The kernel's rule: tiles up to one past the last side row in use while the recent ring has
+    not wrapped (rows end at L + (s mod w), or at L when L <= s), else all nt8."""
+    smw = s % w if w > 0 else 0
+    top = L if L <= s else L + smw
+    return 0 if L <= 0 else ((top + 15) // 16 if top <= s + w else nt8)
 
 
 def side_rows_used(L, s, w):
@@ -37,8 +34,11 @@ def side_rows_used(L, s, w):
     return rows
 
 
+TIGHT_SIDE_TILES = 16  # side caches with more tiles visit only the tiles in use
+
+
 def seg_info(L, s, w, nt8):
-    n8 = side_tiles_used(L, s, w, nt8)
+    n8 = side_tiles_used(L, s, w, nt8) if nt8 > TIGHT_SIDE_TILES else (nt8 if L > 0 else 0)
     m_end = max(s, L - w)
     t4a = s >> 4
     n4 = ((m_end - 1) >> 4) - t4a + 1 if m_end > s else 0
@@ -132,8 +132,11 @@ def test_schedule_invariants(seed):
         lens = [1, 0, s, s + 1, s + w, s + w + 1][:B] + lens[6:]
     if seed % 5 == 1:  # short sequences and the all-INT8 configuration (w above every length)
         lens = rng.integers(0, 2 * (s + w) + 3, size=B).tolist()
-    if seed % 7 == 3:
+    if seed % 7 == 3:  # all-INT8: a side cache of more than 16 tiles, visited only where filled
         s, w = 0, int(max(lens)) + int(rng.integers(0, 40))
+    if seed % 7 == 5:  # sinks and a long recent window (ring wraps for the longest sequences)
+        s, w = int(rng.integers(1, 20)), int(rng.choice([300, 700]))
+        lens = rng.integers(0, s + 2 * w, size=B).tolist()
     stride = max(1, (max(lens) + P - 1) // P)
     for W in (1, 3, 8, 37, 296, 2368):
         model(lens, Hkv, s, w, P, stride, W)
