@@ -8,7 +8,8 @@
 // disjoint regions whose softmax statistics (running max, sum) are merged.
 //
 // Work decomposition (flattened split-K): every (sequence b, KV head g) has an INT8 segment of
-// ceil((s+w)/16) tiles and an INT4 segment of the 16-position tiles covering [s, max(s, L-w)).
+// ceil((s+w)/16) tiles (with a side cache over 16 tiles, only the tiles in use) and an INT4
+// segment of the 16-position tiles covering [s, max(s, L-w)).
 // An INT4 tile costs 1 unit (16*(D+8) bytes), an INT8 tile 2 units (about twice the bytes).  All
 // tiles of all segments form one sequence of units; warp w of the launch takes the tiles whose
 // first unit lies in [w*Q, (w+1)*Q), Q = ceil(total / warps), so every warp streams about the
@@ -24,9 +25,9 @@
 // descriptors (sources, 32-row validity mask, segment index, last-slot flag) are computed 16 slots
 // at a time, one slot per lane, into a small ring, so the per-slot bookkeeping is a few
 // instructions.  QK^T runs on 8-bit integer MMAs (m16n8k32): the INT4 key codes, unpacked to
-// bytes, are the A operand; the rotated query, rounded to a 22-bit integer and split into three
-// signed base-256 digits, is the B operand (G heads x 3 digits in two n-blocks), so q . c is exact
-// in int32.  PV runs on m16n8k16 fp16 MMAs: 16 dims x 16 positions with the centred V codes as the
+// bytes by masks (pair-rows: rows r and r + 8 share a byte), are the A operand; the rotated
+// query, rounded to a 22-bit integer and split into three signed base-256 digits, is the B
+// operand (G heads x 3 digits in two n-blocks), so q . c is exact in int32.  PV runs on m16n8k16 fp16 MMAs: 16 dims x 16 positions with the centred V codes as the
 // A operand and the hi/lo fp16 halves of p * scale of the G heads as the 8 columns of B.  Softmax,
 // scale/offset and rescaling run in fp32 registers.
 #include <cuda_bf16.h>

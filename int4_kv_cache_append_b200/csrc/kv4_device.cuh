@@ -63,15 +63,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Device-scope atomic add with acquire-release ordering: the caller's earlier writes (and those
-// of lanes ordered before it by __syncwarp) are visible to whoever reads the incremented value,
-// and that reader sees every write released by earlier increments.
-__device__ __forceinline__ unsigned atomic_add_acq_rel(unsigned* p, unsigned v) {
-  unsigned old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -159,20 +150,8 @@ __device__ __forceinline__ uint32_t i8x2_to_h2(uint32_t biased) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
-  return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
-}
-
 __device__ __forceinline__ uint32_t pack_bf2(__nv_bfloat16 lo, __nv_bfloat16 hi) {
   return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
-}
-
-// ------------------------------------------------------------------ input loads
-
-__device__ __forceinline__ float load_as_f32(const void* base, int dtype, size_t i) {
-  if (dtype == KV4_F32) return reinterpret_cast<const float*>(base)[i];
-  if (dtype == KV4_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
-  return __half2float(reinterpret_cast<const __half*>(base)[i]);
 }
 
 }  // namespace kv4
