@@ -628,7 +628,7 @@ def run_kv4(args, world, rank, local):
         bkv = float(np.mean([wl.kv_bytes_bf16(lens0 + d) for d in bklens]))
         b_alg = bkv + pt_bytes + io_bytes
         bf = {"value": whole_job_rate(B * steps, world, b_total), "unit": UNIT, "ms_per_step": b_total / steps,
-              "decode_ms": round(b_dec, 5), "kv_bytes_per_launch": int(bkv),
+              "decode_ms": round(b_dec, 5), "append_ms": round(b_app, 5), "kv_bytes_per_launch": int(bkv),
               "achieved_GBps": round(b_alg / (b_dec / 1e3) / 1e9, 1),
               "frac": round(b_alg / (b_dec / 1e3) / 1e9 / peak, 4),
               "int4_speedup_step": round(value / whole_job_rate(B * steps, world, b_total), 3),

@@ -73,3 +73,20 @@ def test_step_shape_of_the_workloads():
         wl = W.qwen3_8b_loop(h=h)
         assert wl.h == h
         assert bench.step_shape(wl) == (36, 36, 64)
+
+
+def test_sink_recent_overrides():
+    """--sinks/--recent replace a workload's s and w (recent -1: every position, KV8) and name the
+    workload after them; the lengths and pages are unchanged."""
+    import argparse
+    sys.path.insert(0, ROOT)
+    import bench
+    base = bench.make_wl(argparse.Namespace(workload="qwen3-4b-decode", h=None, sinks=None, recent=None))
+    kv8 = bench.make_wl(argparse.Namespace(workload="qwen3-4b-decode", h=None, sinks=0, recent=-1))
+    assert (kv8.s, kv8.w) == (0, int(base.max_lens.max()))
+    assert kv8.name == f"{base.name}-s0-w{kv8.w}"
+    assert (kv8.lens == base.lens).all() and (kv8.page_table == base.page_table).all()
+    # every position read from the side cache: 2D + 4 bytes per token and KV head
+    assert kv8.kv_bytes_int4() == base.Hkv * int(base.lens.astype(int).sum()) * (2 * base.D + 4)
+    sw = bench.make_wl(argparse.Namespace(workload="qwen3-4b-decode", h=None, sinks=144, recent=0))
+    assert (sw.s, sw.w) == (144, 0)
