@@ -546,7 +546,7 @@ def run_kv4(args, world, rank, local):
             slot_p = base + parts[-1][1]
             pos_p, len_p = dst[j].data_ptr(), dst[j].data_ptr() + 4 * B
             cj = []
-            for li, layer in enumerate(range(nl) if per_step > 1 else [None]):
+            for li in range(nsets):
                 kp, vp, qp = (base + parts[3 * li + x][1] for x in range(3))
                 cj.append((kp, vp, qp, slot_p, pos_p, len_p))
             calls.append(cj)
@@ -571,7 +571,7 @@ def run_kv4(args, world, rank, local):
                 stream.wait_event(ev_in[j])
                 stream.wait_event(ev_out[j])  # its previous output has been copied out
             layers = range(nl) if per_step > 1 else [i % resident]
-            for (kp, vp, qp, slot_p, pos_p, len_p), layer in zip(calls[j] * (1 if per_step > 1 else 1), layers):
+            for (kp, vp, qp, slot_p, pos_p, len_p), layer in zip(calls[j], layers):
                 st_ = lib.kv4_append(handle, layer, B, kp, kd, vp, vd, slot_p, pos_p, len_p, pt_ptr, stride, sh_main)
                 sd_ = lib.kv4_decode_attn(handle, layer, B, qp, qd, pt_ptr, stride, len_p, maxlen,
                                           douts[j].data_ptr(), None, ws.data_ptr(), ws.numel(), sh_main)
