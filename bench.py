@@ -1,6 +1,6 @@
 #!/usr/bin/env python
 """Benchmark: decode steps of INT4-KV attention (append + decode) beside the BF16-KV kernel on
-the same box and the CPU oracle on the host cores.  Default workload: Qwen3-4B-like (32 q / 8 KV
+the same GPU and the CPU oracle on the host cores.  Default workload: Qwen3-4B-like (32 q / 8 KV
 heads, head_dim 128, bf16, B = 64 sequences with lognormal lengths of median 2048 capped at
 8192, P = 16, s = 4, w = 128, h = 128).
 
@@ -614,7 +614,7 @@ def run_kv4(args, world, rank, local):
     del cache, ins, S
     torch.cuda.empty_cache()
 
-    # ---- BF16-KV baseline kernel on the same box.  A multi-layer step is timed on LAYERS of its
+    # ---- BF16-KV baseline kernel on the same GPU.  A multi-layer step is timed on LAYERS of its
     # layers (BF16 KV of every layer would not fit) and scaled by per_step / LAYERS: the layers
     # are identical in shape, so the per-layer cost is the same.
     bf = None

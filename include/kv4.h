@@ -17,8 +17,10 @@
  *
  * Conventions the pages leave open (fixed here, identical in the test oracle):
  *   - Hadamard: Sylvester order, unnormalised, on contiguous blocks of h elements (h a power
- *     of two dividing head_dim; h = 1 means no rotation).  Keys are stored rotated; the query
- *     is multiplied by H/h, so rotated query . rotated key = q . k.  Values are not rotated.
+ *     of two dividing head_dim; h = 1 means no rotation), optionally after a per-dimension sign
+ *     flip (kv4_set_rotation_signs).  Keys are stored rotated; the query is multiplied by the
+ *     same rotation over h, so rotated query . rotated key = q . k.  Values are stored as given
+ *     unless kv4_set_value_rotation is on (then rotated too, and outputs rotated back).
  *   - INT4: zero = fp16 rounded toward -inf of min(x); scale = fp16 rounded toward +inf of
  *     fl32(max(x) - zero)/15; code = clamp(rint((x - zero)/scale), 0, 15) in IEEE fp32;
  *     x is reconstructed as zero + scale * code.
@@ -180,7 +182,7 @@ kv4_status kv4_set_decode_overlap(kv4_cache* cache, int enable);
 /*
  * BF16-KV baseline with the same page table and conventions, no quantisation and no rotation:
  * a page holds Hkv head blocks of P * 4D bytes (bf16 K and V).  Used to measure the INT4
- * speed-up on the same box.  kv4_bf16_query_sizes returns num_layers * max_pages * Hkv * P * 4D.
+ * speed-up on the same GPU.  kv4_bf16_query_sizes returns num_layers * max_pages * Hkv * P * 4D.
  */
 kv4_status kv4_bf16_query_sizes(const kv4_config* cfg, size_t* page_pool_bytes);
 kv4_status kv4_bf16_cache_init(const kv4_config* cfg, void* page_pool, kv4_cache** out);
