@@ -24,8 +24,11 @@
  *   R2 keys are stored rotated and unnormalised; the query uses (H q) / h, so the product of
  *      rotated query and rotated key equals q . k.  Values are not rotated.
  *   R3 INT4: zero = fp16 rounded down of min, scale = fp16 rounded up of (max - zero)/15,
- *      code = clamp(rint((x - zero)/scale), 0, 15) in fp32; scale 0 gives all-zero codes.
- *   R4 INT8: symmetric, scale = fp16 rounded up of max|x|/127, code = clamp(rint(x/scale), +-127).
+ *      code = clamp(rint((x - zero)/scale), 0, 15) in fp32; scale 0 gives all-zero codes; a
+ *      non-finite zero or scale (values beyond the fp16 range) gives all-zero codes and is
+ *      reported by the append.
+ *   R4 INT8: symmetric, scale = fp16 rounded up of max|x|/127, code = clamp(rint(x/scale), +-127);
+ *      a non-finite scale is treated as in R3.
  *   R5 routing: every token gets INT4 codes; in addition pos < s goes to sink row pos, and
  *      pos >= s with pos >= lens_after - w goes to ring row s + (pos mod w).
  *   R6 byte layout of pages and of the side cache: see the orc_*_byte functions.
@@ -156,7 +159,7 @@ void orc_fwht_f64(double* x, int D, int h) {
 /* [KV4-RL Meth.2]: one affine INT4 group per token-head vector with an FP16 scale and
  * offset; x is reconstructed as zero + scale * code.  Minimum and maximum are taken as
  * values (a zero result is +0). */
-void orc_quant_int4(const float* x, int D, uint8_t* codes4, uint16_t* scale, uint16_t* zero) {
+int orc_quant_int4(const float* x, int D, uint8_t* codes4, uint16_t* scale, uint16_t* zero) {
   float mn = x[0], mx = x[0];
   for (int i = 1; i < D; ++i) {
     if (x[i] < mn) mn = x[i];
@@ -170,9 +173,12 @@ void orc_quant_int4(const float* x, int D, uint8_t* codes4, uint16_t* scale, uin
   const float sq = r / 15.0f;
   const uint16_t sb = orc_f32_to_f16(sq, ORC_RU);
   const float sf = orc_f16_to_f32(sb);
+  /* R3 range: a vector whose offset or scale is not a finite fp16 (its values reach beyond the
+   * fp16 range) keeps its non-finite parameters and all-zero codes, and is reported. */
+  const int out_of_range = !isfinite(zf) || !isfinite(sf);
   for (int i = 0; i < D; ++i) {
     int c = 0;
-    if (sf != 0.0f) {
+    if (sf != 0.0f && !out_of_range) {
       const float t = (x[i] - zf) / sf;
       const float rq = rintf(t);    /* default rounding mode: nearest, ties to even */
       c = (int)rq;
@@ -183,10 +189,11 @@ void orc_quant_int4(const float* x, int D, uint8_t* codes4, uint16_t* scale, uin
   }
   *scale = sb;
   *zero = zb;
+  return out_of_range;
 }
 
 /* INT8 side-cache format (R4): the pages name INT8 only; symmetric per vector. */
-void orc_quant_int8(const float* x, int D, int8_t* codes8, uint16_t* scale) {
+int orc_quant_int8(const float* x, int D, int8_t* codes8, uint16_t* scale) {
   float a = 0.0f;
   for (int i = 0; i < D; ++i) {
     const float ax = fabsf(x[i]);
@@ -194,9 +201,10 @@ void orc_quant_int8(const float* x, int D, int8_t* codes8, uint16_t* scale) {
   }
   const uint16_t sb = orc_f32_to_f16(a / 127.0f, ORC_RU);
   const float sf = orc_f16_to_f32(sb);
+  const int out_of_range = !isfinite(sf); /* as for INT4: zero codes, reported */
   for (int i = 0; i < D; ++i) {
     int c = 0;
-    if (sf != 0.0f) {
+    if (sf != 0.0f && !out_of_range) {
       c = (int)rintf(x[i] / sf);
       if (c < -127) c = -127;
       if (c > 127) c = 127;
@@ -204,6 +212,7 @@ void orc_quant_int8(const float* x, int D, int8_t* codes8, uint16_t* scale) {
     codes8[i] = (int8_t)c;
   }
   *scale = sb;
+  return out_of_range;
 }
 
 /* ------------------------------------------------------------------ layout (R6) */
@@ -303,12 +312,6 @@ size_t orc_s8_byte(const orc_config* c, int slot, int g, int row, int is_v) {
   return tile8_base(c, slot, g, row) + (size_t)(16 * D + is_v * (16 * D + 32) + 2 * r);
 }
 
-int orc_side_row(const orc_config* c, int pos) {
-  if (pos < c->num_sinks) return pos;
-  if (c->recent_window > 0) return c->num_sinks + pos % c->recent_window;
-  return -1;
-}
-
 static int config_ok(const orc_config* c) {
   const int D = c->head_dim, h = c->hadamard_block;
   if (c->num_kv_heads <= 0 || c->num_q_heads <= 0 || c->num_q_heads % c->num_kv_heads) return 0;
@@ -355,6 +358,7 @@ int orc_append(const orc_config* c, uint8_t* pool, uint8_t* side, int T, const v
   uint8_t* c4 = (uint8_t*)malloc((size_t)D);
   int8_t* c8 = (int8_t*)malloc((size_t)D);
   if (!kf || !vf || !c4 || !c8) return -2;
+  int range = 0;
   for (int t = 0; t < T; ++t) {
     const int b = seq_slot[t], p = pos[t];
     const int page = page_table[(size_t)b * (size_t)stride + (size_t)(p / P)];
@@ -368,11 +372,11 @@ int orc_append(const orc_config* c, uint8_t* pool, uint8_t* side, int T, const v
       orc_rotate_key(c, kf);
       if (c->rotate_values) orc_rotate_key(c, vf);
       uint16_t sc, zr;
-      orc_quant_int4(kf, D, c4, &sc, &zr);
+      range |= orc_quant_int4(kf, D, c4, &sc, &zr);
       for (int e = 0; e < D; ++e) put_nibble(pool, orc_k4_byte(c, page, g, pp, e), orc_k4_high(c, pp, e), c4[e]);
       put_u16(pool, orc_p4_byte(c, page, g, pp, 0), sc);
       put_u16(pool, orc_p4_byte(c, page, g, pp, 0) + 2, zr);
-      orc_quant_int4(vf, D, c4, &sc, &zr);
+      range |= orc_quant_int4(vf, D, c4, &sc, &zr);
       for (int e = 0; e < D; ++e) put_nibble(pool, orc_v4_byte(c, page, g, pp, e), e & 1, c4[e]);
       put_u16(pool, orc_p4_byte(c, page, g, pp, 1), sc);
       put_u16(pool, orc_p4_byte(c, page, g, pp, 1) + 2, zr);
@@ -384,10 +388,10 @@ int orc_append(const orc_config* c, uint8_t* pool, uint8_t* side, int T, const v
         row = s + p % w;
       if (row >= 0) {
         uint16_t s8;
-        orc_quant_int8(kf, D, c8, &s8);
+        range |= orc_quant_int8(kf, D, c8, &s8);
         for (int e = 0; e < D; ++e) side[orc_k8_byte(c, b, g, row, e)] = (uint8_t)c8[e];
         put_u16(side, orc_s8_byte(c, b, g, row, 0), s8);
-        orc_quant_int8(vf, D, c8, &s8);
+        range |= orc_quant_int8(vf, D, c8, &s8);
         for (int e = 0; e < D; ++e) side[orc_v8_byte(c, b, g, row, e)] = (uint8_t)c8[e];
         put_u16(side, orc_s8_byte(c, b, g, row, 1), s8);
       }
@@ -397,7 +401,7 @@ int orc_append(const orc_config* c, uint8_t* pool, uint8_t* side, int T, const v
   free(vf);
   free(c4);
   free(c8);
-  return 0;
+  return range ? ORC_APPEND_RANGE : 0;
 }
 
 /* ------------------------------------------------------------------ dequantise */

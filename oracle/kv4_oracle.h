@@ -62,9 +62,10 @@ void orc_fwht_f64(double* x, int D, int h);
  * value rotation when rotate_values is set). */
 void orc_rotate_key(const orc_config* c, float* x);
 
-/* Per-vector quantisers.  codes4 holds one code (0..15) per element, unpacked. */
-void orc_quant_int4(const float* x, int D, uint8_t* codes4, uint16_t* scale, uint16_t* zero);
-void orc_quant_int8(const float* x, int D, int8_t* codes8, uint16_t* scale);
+/* Per-vector quantisers.  codes4 holds one code (0..15) per element, unpacked.  Both return 1
+ * when a parameter is not a finite fp16 (the codes are then all zero), else 0. */
+int orc_quant_int4(const float* x, int D, uint8_t* codes4, uint16_t* scale, uint16_t* zero);
+int orc_quant_int8(const float* x, int D, int8_t* codes8, uint16_t* scale);
 
 /* Storage sizes. */
 size_t orc_page_bytes(const orc_config* c);          /* one page, all KV heads             */
@@ -81,11 +82,11 @@ size_t orc_p4_byte(const orc_config* c, int page, int g, int pos_in_page, int is
 size_t orc_k8_byte(const orc_config* c, int slot, int g, int row, int elem);
 size_t orc_v8_byte(const orc_config* c, int slot, int g, int row, int elem);
 size_t orc_s8_byte(const orc_config* c, int slot, int g, int row, int is_v);
-/* Side-cache row that holds position pos (sink row or ring row); -1 if not routed. */
-int    orc_side_row(const orc_config* c, int pos);
 
 /* Append T tokens (K, V [T][Hkv][D], element type k_dtype / v_dtype) into host copies of
- * one layer's page pool and side cache.  Returns 0 or a negative error code. */
+ * one layer's page pool and side cache.  Returns 0, ORC_APPEND_RANGE when some vector's fp16
+ * scale or offset was not finite (stored with zero codes), or a negative error code. */
+enum { ORC_APPEND_RANGE = 1 };
 int orc_append(const orc_config* c, uint8_t* pool, uint8_t* side, int T,
                const void* K, int k_dtype, const void* V, int v_dtype,
                const int32_t* seq_slot, const int32_t* pos, const int32_t* lens_after,

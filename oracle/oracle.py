@@ -95,7 +95,9 @@ def lib():
         L.orc_fwht_f64.argtypes = [P, I, I]
         L.orc_rotate_key.argtypes = [ctypes.POINTER(_Cfg), P]
         L.orc_quant_int4.argtypes = [P, I, P, P, P]
+        L.orc_quant_int4.restype = I
         L.orc_quant_int8.argtypes = [P, I, P, P]
+        L.orc_quant_int8.restype = I
         for n in ("orc_page_bytes", "orc_side_slot_bytes"):
             getattr(L, n).argtypes = [cfgp]
             getattr(L, n).restype = S
@@ -106,8 +108,6 @@ def lib():
             getattr(L, n).restype = S
         L.orc_k4_high.argtypes = [cfgp, I, I]
         L.orc_k4_high.restype = I
-        L.orc_side_row.argtypes = [cfgp, I]
-        L.orc_side_row.restype = I
         L.orc_append.argtypes = [cfgp, P, P, I, P, I, P, I, P, P, P, P, I]
         L.orc_append.restype = I
         L.orc_dequant_seq.argtypes = [cfgp, P, P, P, I, I, I, P, P, P]
@@ -158,23 +158,24 @@ def fwht_f64(x: np.ndarray, h: int) -> np.ndarray:
     return y
 
 
-def quant_int4(x: np.ndarray):
-    """Returns (codes uint8[D], scale_bits, zero_bits)."""
+def quant_int4(x: np.ndarray, with_flag: bool = False):
+    """Returns (codes uint8[D], scale_bits, zero_bits), plus the out-of-range flag (a scale or
+    zero that is not a finite fp16; the codes are then zero) when with_flag is set."""
     xf = np.ascontiguousarray(x, dtype=np.float32)
     codes = np.zeros(xf.size, np.uint8)
     sc = np.zeros(1, np.uint16)
     zr = np.zeros(1, np.uint16)
-    lib().orc_quant_int4(_p(xf), xf.size, _p(codes), _p(sc), _p(zr))
-    return codes, int(sc[0]), int(zr[0])
+    flag = lib().orc_quant_int4(_p(xf), xf.size, _p(codes), _p(sc), _p(zr))
+    return (codes, int(sc[0]), int(zr[0]), bool(flag)) if with_flag else (codes, int(sc[0]), int(zr[0]))
 
 
-def quant_int8(x: np.ndarray):
-    """Returns (codes int8[D], scale_bits)."""
+def quant_int8(x: np.ndarray, with_flag: bool = False):
+    """Returns (codes int8[D], scale_bits), plus the out-of-range flag when with_flag is set."""
     xf = np.ascontiguousarray(x, dtype=np.float32)
     codes = np.zeros(xf.size, np.int8)
     sc = np.zeros(1, np.uint16)
-    lib().orc_quant_int8(_p(xf), xf.size, _p(codes), _p(sc))
-    return codes, int(sc[0])
+    flag = lib().orc_quant_int8(_p(xf), xf.size, _p(codes), _p(sc))
+    return (codes, int(sc[0]), bool(flag)) if with_flag else (codes, int(sc[0]))
 
 
 # ---------------------------------------------------------------- cache-level calls
@@ -205,10 +206,6 @@ def nibble_high(kind: str, cfg: Config, r: int, e: int) -> int:
     return e & 1
 
 
-def side_row(cfg: Config, pos: int) -> int:
-    return int(lib().orc_side_row(ctypes.byref(cfg.c()), pos))
-
-
 def _dtype_code(a: np.ndarray, declared: int | None) -> int:
     if declared is not None:
         return declared
@@ -219,8 +216,9 @@ def _dtype_code(a: np.ndarray, declared: int | None) -> int:
 
 def append(cfg: Config, pool: np.ndarray, side: np.ndarray, K: np.ndarray, V: np.ndarray,
            seq_slot: np.ndarray, pos: np.ndarray, lens_after: np.ndarray, page_table: np.ndarray,
-           k_dtype: int | None = None, v_dtype: int | None = None) -> None:
-    """Append T tokens.  K, V: [T][Hkv][D] float32, or uint16 bit patterns with a dtype code."""
+           k_dtype: int | None = None, v_dtype: int | None = None) -> bool:
+    """Append T tokens.  K, V: [T][Hkv][D] float32, or uint16 bit patterns with a dtype code.
+    Returns True when some vector's fp16 scale or offset was not finite (stored with zero codes)."""
     K = np.ascontiguousarray(K)
     V = np.ascontiguousarray(V)
     seq_slot = np.ascontiguousarray(seq_slot, np.int32)
@@ -231,8 +229,9 @@ def append(cfg: Config, pool: np.ndarray, side: np.ndarray, K: np.ndarray, V: np
     rc = lib().orc_append(ctypes.byref(cfg.c()), _p(pool), _p(side), T, _p(K), _dtype_code(K, k_dtype),
                           _p(V), _dtype_code(V, v_dtype), _p(seq_slot), _p(pos), _p(lens_after),
                           _p(page_table), int(page_table.shape[1]))
-    if rc != 0:
+    if rc < 0:
         raise RuntimeError(f"orc_append failed: {rc}")
+    return rc == 1
 
 
 def dequant_seq(cfg: Config, pool: np.ndarray, side: np.ndarray, page_row: np.ndarray, slot: int,

@@ -183,7 +183,7 @@ def _requant_int4_numpy(x: np.ndarray):
     if float(s) < float(sq):
         s = _f16_up(s)
     sf = np.float32(s)
-    if sf == 0:
+    if sf == 0 or not (np.isfinite(sf) and np.isfinite(zf)):
         codes = np.zeros(x.size, np.uint8)
     else:
         t = ((x - zf).astype(np.float32) / sf).astype(np.float32)
@@ -219,6 +219,55 @@ def pin_quant_int4_constant():
         codes, sc, zr = O.quant_int4(x)
         if float(np.float16(v)) == v:
             assert np.all(_f16(zr) + _f16(sc) * codes == v)
+
+
+def pin_quant_range(seed: int = 17):
+    """Vectors beyond the fp16 range: the largest fp16 <= min is -inf below -65504, the smallest
+    fp16 >= (max - zero)/15 is +inf above 65504 (IEEE directed rounding of an overflow); such a
+    vector gets all-zero codes and the out-of-range flag.  At the edge of the range the parameters
+    are finite, the flag is clear and the reconstruction bound holds."""
+    rng = np.random.default_rng(seed)
+    big = np.float32(np.finfo(np.float16).max)  # 65504
+    for D in (64, 128):
+        x = rng.normal(0, 1, D).astype(np.float32)
+        x[5] = -1.0e6  # zero overflows to -inf
+        codes, sc, zr, bad = O.quant_int4(x, with_flag=True)
+        assert bad and zr == 0xFC00 and sc == 0x7C00 and not codes.any(), (hex(sc), hex(zr))
+        x = np.abs(rng.normal(0, 1, D)).astype(np.float32)
+        x[7] = 1.0e6  # (max - zero)/15 = 66667 > 65504: scale overflows to +inf
+        codes, sc, zr, bad = O.quant_int4(x, with_flag=True)
+        z = _f16(zr)
+        assert bad and sc == 0x7C00 and np.isfinite(z) and z <= x.min() < float(_f16_up(np.float16(z)))
+        assert not codes.any()
+        # INT8: max|x| / 127 stays finite up to 127 * 65504
+        c8, s8, bad8 = O.quant_int8(x, with_flag=True)
+        assert not bad8 and _f16(s8) >= 1.0e6 / 127
+        x8 = x.copy()
+        x8[7] = 1.0e7
+        c8, s8, bad8 = O.quant_int8(x8, with_flag=True)
+        assert bad8 and s8 == 0x7C00 and not c8.any()
+        # the edge: min = -65504 exactly, range inside fp16 -> finite parameters, no flag
+        x = rng.normal(0, 1, D).astype(np.float32)
+        x[3] = -big
+        codes, sc, zr, bad = O.quant_int4(x, with_flag=True)
+        assert not bad and zr == 0xFBFF and np.isfinite(_f16(sc))
+        rec = _f16(zr) + _f16(sc) * codes.astype(np.float64)
+        assert np.all(np.abs(x.astype(np.float64) - rec) <= _f16(sc) / 2 + 4 * np.spacing(big))
+
+
+def pin_append_range_flag(seed: int = 19):
+    """The append reports a token whose parameters overflowed, and only then."""
+    wl = small_workload(lens=(9,), B=1, s=2, w=3, h=8, seed=seed)
+    cfg = oracle_cfg(wl)
+    pool = np.zeros(O.page_bytes(cfg) * wl.num_pages, np.uint8)
+    side = np.zeros(O.side_slot_bytes(cfg) * wl.B, np.uint8)
+    b = np.zeros(9, np.int32)
+    p = np.arange(9, dtype=np.int32)
+    K, V = wl.kv_inputs(0, b, p)
+    assert not O.append(cfg, pool, side, K, V, b, p, wl.lens, wl.page_table)
+    V = V.copy()
+    V[4, 1, 3] = 2.0e6
+    assert O.append(cfg, pool, side, K, V, b, p, wl.lens, wl.page_table)
 
 
 def pin_quant_int8_bounds(seed: int = 13, n: int = 300):
@@ -574,5 +623,6 @@ ALL_PINS = [
     pin_quant_int4_constant, pin_quant_int8_bounds, pin_storage_bits, pin_layout_bijection,
     lambda: pin_routing(False), lambda: pin_routing(True), pin_brute_force,
     pin_append_vs_numpy_requant, pin_regional_equals_single, pin_rotation_invariance,
-    pin_special_cases, pin_signed_rotation_exact, pin_value_rotation_invariance,
+    pin_special_cases, pin_signed_rotation_exact, pin_value_rotation_invariance, pin_quant_range,
+    pin_append_range_flag,
 ]

@@ -48,6 +48,8 @@ MUTANTS = [
     ("gqa-map", "(size_t)(g * G + i)", "(size_t)(g + i * Hkv)", None),
     ("f16-no-subnormal", "if (E < -14) E = -14;", ";", None),
     ("f16-ties-away", "(frac == 0.5 && fmod(n, 2.0) == 1.0)", "(frac == 0.5)", None),
+    ("int4-range-unreported", "  return out_of_range;\n}", "  return 0;\n}", 0),
+    ("int8-range-unreported", "  return out_of_range;\n}", "  return 0;\n}", 1),
     ("single-softmax-max", "if (logit[j] > ps->m) ps->m = logit[j];", "if (logit[j] < ps->m) ps->m = logit[j];", None),
 ]
 

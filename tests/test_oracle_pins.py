@@ -83,3 +83,11 @@ def test_value_rotation_invariance():
 
 def test_special_cases():
     P.pin_special_cases()
+
+
+def test_quantiser_range_overflow():
+    P.pin_quant_range()
+
+
+def test_append_reports_range_overflow():
+    P.pin_append_range_flag()
