@@ -68,6 +68,12 @@ typedef enum { KV4_F32 = 0, KV4_BF16 = 1, KV4_F16 = 2 } kv4_dtype;
 #define KV4_DEVERR_PAGE_RANGE 0x1u  /* page-table entry outside [0, max_pages)            */
 #define KV4_DEVERR_WAIT_LIMIT 0x2u  /* a bounded wait for a bulk copy ran out             */
 #define KV4_DEVERR_LENGTH 0x4u      /* a length or position beyond the page-table row     */
+#define KV4_DEVERR_RANGE 0x8u       /* an appended vector's fp16 scale or offset overflowed: its
+                                       values reach beyond the fp16 range; the vector was stored
+                                       with all-zero codes and its non-finite parameters        */
+#define KV4_DEVERR_RECORD 0x10u     /* the merge found a split-partial record pointing outside the
+                                       workspace (left by a decode that stopped early) and
+                                       skipped it                                               */
 
 /*
  * Cache geometry.  Supported: head_dim in {64, 128}; Hq/Hkv in {1, 2, 4}; page_size a
@@ -180,6 +186,18 @@ kv4_status kv4_set_value_rotation(kv4_cache* cache, int enable);
 kv4_status kv4_set_decode_overlap(kv4_cache* cache, int enable);
 
 /*
+ * kv4_debug_force_wait_timeout: a test hook for the device-side failure path (default 0, leave
+ * it off in production).  With 1, every kv4_decode_attn of this cache makes each warp of the
+ * split-K kernel wait, with a 1 ms limit, on a barrier that nothing arrives on: the wait runs
+ * out, the warp sets KV4_DEVERR_WAIT_LIMIT, waits (bounded) for the bulk copies it already has
+ * in flight, and returns.  The merge kernel then finds no fresh partial records: records that
+ * point outside the workspace are skipped with KV4_DEVERR_RECORD.  That call's out and lse are
+ * undefined; the context stays usable, and a call with 0 decodes normally.  Returns
+ * KV4_ERR_INVALID_ARG for a NULL or BF16 cache.
+ */
+kv4_status kv4_debug_force_wait_timeout(kv4_cache* cache, int enable);
+
+/*
  * BF16-KV baseline with the same page table and conventions, no quantisation and no rotation:
  * a page holds Hkv head blocks of P * 4D bytes (bf16 K and V).  Used to measure the INT4
  * speed-up on the same GPU.  kv4_bf16_query_sizes returns num_layers * max_pages * Hkv * P * 4D.
@@ -204,9 +222,11 @@ kv4_status kv4_bf16_decode_attn(kv4_cache* cache, int layer, int B, const void* 
  * The split-K partials live in a static device array of KV4_STATIC_SCRATCH_BYTES per GPU, part of
  * the library image and held by every GPU that loads libkv4.so until the process exits.  The
  * call allocates and frees nothing.  Arguments and results are those of kv4_decode_attn minus the
- * workspace.  A batch whose partials exceed the array (kv4_decode_workspace_bytes(B) >
- * KV4_STATIC_SCRATCH_BYTES; about B > 350 for 8 KV heads, head_dim 128, 4 q heads per KV head on
- * 148 SMs) returns KV4_ERR_WORKSPACE and launches nothing.
+ * workspace.  The limit: a call is accepted when kv4_decode_workspace_bytes(cache, B) <=
+ * KV4_STATIC_SCRATCH_BYTES, else it returns KV4_ERR_WORKSPACE and launches nothing.  That size
+ * holds one 16-byte record per (sequence slot, KV head) of the cache (max_seqs * Hkv * 16 bytes,
+ * so the limit shrinks as max_seqs grows) plus the split partials of B sequences; for 8 KV heads,
+ * head_dim 128, 4 q heads per KV head on 148 SMs and max_seqs = B it admits B <= 347.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
  * device current; make that first call before any stream capture.  All calls on one GPU share
  * the array; every call writes every partial its merge reads, so nothing needs clearing between

@@ -40,6 +40,7 @@ struct kv4_cache {
   int overlap;        // kv4_set_decode_overlap
   uint32_t signs[4];  // kv4_set_rotation_signs
   int rotate_v;       // kv4_set_value_rotation
+  int stall_test;     // kv4_debug_force_wait_timeout
 };
 
 namespace kv4 {
@@ -174,8 +175,6 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
   int ctas = full;
   if (max_len_hint > 0) {
     // Enough CTAs that each warp gets at least ~16 slots of the hinted upper bound.
-    const long long D = c->cfg.head_dim;
-    (void)D;
     const long long tiles = (static_cast<long long>(max_len_hint) + 15) / 16;
     const long long slots = static_cast<long long>(B) * c->cfg.num_kv_heads * (tiles + (fmt == FMT_INT4 ? 2LL * c->nt8 : 0));
     const int warps = fmt == FMT_INT4 ? kv4::decode_warps_per_cta() : kv4::bf16_decode_warps_per_cta();
@@ -217,13 +216,14 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
   a.lse = lse;
   a.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->cfg.head_dim)));
   a.err = err;
-  {
-    const int tpp = c->cfg.page_size / 16;
-    a.early = (fmt == FMT_INT4 && c->overlap) ? 1 : 0;
+  a.early = (fmt == FMT_INT4 && c->overlap) ? 1 : 0;
   for (int i = 0; i < 4; ++i) a.signs[i] = c->signs[i];
   a.rotate_v = fmt == FMT_INT4 ? c->rotate_v : 0;
+  const int tpp = c->cfg.page_size / 16;
   a.tp_shift = pow2(tpp) ? __builtin_ctz(static_cast<unsigned>(tpp)) : -1;
-  }
+  // The wait-limit test runs every warp's first wait out after 1 ms; the normal limit is 2 s.
+  a.stall_test = (fmt == FMT_INT4 && c->stall_test) ? 1 : 0;
+  a.wait_ns = a.stall_test ? 1000000ull : 2000000000ull;
   const int G = c->cfg.num_q_heads / c->cfg.num_kv_heads;
   const cudaError_t e = fmt == FMT_INT4
                             ? kv4::launch_decode_int4(a, c->cfg.head_dim, G, ctas, static_cast<cudaStream_t>(stream))
@@ -325,6 +325,12 @@ kv4_status kv4_set_value_rotation(kv4_cache* cache, int enable) {
 kv4_status kv4_set_decode_overlap(kv4_cache* cache, int enable) {
   if (!cache || cache->format != FMT_INT4) return KV4_ERR_INVALID_ARG;
   cache->overlap = enable ? 1 : 0;
+  return KV4_OK;
+}
+
+kv4_status kv4_debug_force_wait_timeout(kv4_cache* cache, int enable) {
+  if (!cache || cache->format != FMT_INT4) return KV4_ERR_INVALID_ARG;
+  cache->stall_test = enable ? 1 : 0;
   return KV4_OK;
 }
 

@@ -89,8 +89,10 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // INT4 codes of the lane's 4 elements packed as elements 0..3 in bits 0..15 (4 bits each);
-// *sz receives (fp16 scale bits) | (fp16 zero bits << 16).
-__device__ __forceinline__ uint32_t quant_int4(const float (&x)[4], bool act, uint32_t* sz) {
+// *sz receives (fp16 scale bits) | (fp16 zero bits << 16).  A vector whose zero or scale is not a
+// finite fp16 (values beyond the fp16 range) keeps those parameters, gets all-zero codes and sets
+// *bad (warp-uniform: the parameters come from warp reductions).
+__device__ __forceinline__ uint32_t quant_int4(const float (&x)[4], bool act, uint32_t* sz, bool* bad) {
   float mn = act ? fminf(fminf(x[0], x[1]), fminf(x[2], x[3])) : __int_as_float(0x7f800000);
   float mx = act ? fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])) : __int_as_float(0xff800000);
   mn = __fadd_rn(warp_min(mn), 0.0f);
@@ -100,11 +102,12 @@ __device__ __forceinline__ uint32_t quant_int4(const float (&x)[4], bool act, ui
   const float r = __fsub_rn(mx, zf);
   const __half sh = __float2half_ru(__fdiv_rn(r, 15.0f));
   const float sf = __half2float(sh);
+  *bad = !(isfinite(zf) && isfinite(sf));
   uint32_t packed = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     int c = 0;
-    if (sf != 0.0f) {
+    if (sf != 0.0f && !*bad) {
       c = static_cast<int>(rintf(__fdiv_rn(__fsub_rn(x[i], zf), sf)));
       c = min(max(c, 0), 15);
     }
@@ -114,17 +117,19 @@ __device__ __forceinline__ uint32_t quant_int4(const float (&x)[4], bool act, ui
   return packed;
 }
 
-// Symmetric INT8 codes of the lane's 4 elements (bytes 0..3), fp16 scale bits in *sc.
-__device__ __forceinline__ uint32_t quant_int8(const float (&x)[4], bool act, uint16_t* sc) {
+// Symmetric INT8 codes of the lane's 4 elements (bytes 0..3), fp16 scale bits in *sc; a scale
+// that is not a finite fp16 gives all-zero codes and sets *bad, as for INT4.
+__device__ __forceinline__ uint32_t quant_int8(const float (&x)[4], bool act, uint16_t* sc, bool* bad) {
   float a = act ? fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3]))) : 0.0f;
   a = warp_max(a);
   const __half sh = __float2half_ru(__fdiv_rn(a, 127.0f));
   const float sf = __half2float(sh);
+  *bad = !isfinite(sf);
   uint32_t packed = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     int c = 0;
-    if (sf != 0.0f) {
+    if (sf != 0.0f && !*bad) {
       c = static_cast<int>(rintf(__fdiv_rn(x[i], sf)));
       c = min(max(c, -127), 127);
     }
@@ -181,8 +186,10 @@ __global__ void __launch_bounds__(kAppendThreads) append_int4_kernel(AppendArgs 
   uint8_t* tile = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(g) * a.P * (D + 8) +
                   static_cast<size_t>(pp >> 4) * Gm::T4B;
   uint32_t ksz, vsz;
-  const uint32_t kc = quant_int4(k, act, &ksz);
-  const uint32_t vc = quant_int4(v, act, &vsz);
+  bool kbad, vbad;
+  const uint32_t kc = quant_int4(k, act, &ksz, &kbad);
+  const uint32_t vc = quant_int4(v, act, &vsz, &vbad);
+  if (lane == 0 && (kbad || vbad)) atomicOr(a.err, KV4_DEVERR_RANGE);
   if (act) {
     // K: row r shares pair-row r % 8 with row r ^ 8 (low nibbles rows 0-7, high nibbles rows
     // 8-15), so its nibbles are merged in with atomics (another token of the tile may be written
@@ -220,8 +227,10 @@ __global__ void __launch_bounds__(kAppendThreads) append_int4_kernel(AppendArgs 
                 static_cast<size_t>(g) * a.nt8 * Gm::T8B + static_cast<size_t>(row >> 4) * Gm::T8B;
   const int r8 = row & 15;
   uint16_t ks, vs;
-  const uint32_t k8 = quant_int8(k, act, &ks);
-  const uint32_t v8 = quant_int8(v, act, &vs);
+  bool kbad8, vbad8;
+  const uint32_t k8 = quant_int8(k, act, &ks, &kbad8);
+  const uint32_t v8 = quant_int8(v, act, &vs, &vbad8);
+  if (lane == 0 && (kbad8 || vbad8)) atomicOr(a.err, KV4_DEVERR_RANGE);
   if (act) {
     const int e = 4 * lane;
     *reinterpret_cast<uint32_t*>(t8 + r8 * D + 16 * ((e >> 4) ^ (r8 & 1)) + (e & 15)) = k8;

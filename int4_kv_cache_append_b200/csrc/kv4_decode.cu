@@ -245,6 +245,7 @@ struct Smem {
   Cursor cur[kWarps];                                // descriptor cursor between fills
   unsigned segno[kWarps];                            // segments entered so far
   uint64_t bar[kWarps][kStages];
+  uint64_t stall[kWarps];  // never arrived on: the wait-limit test (kv4_debug_force_wait_timeout)
 };
 
 // slot meta word
@@ -475,6 +476,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   uint64_t* bars = sm.bar[warp];
   if (lane == 0) {
     for (int i = 0; i < kStages; ++i) mbar_init(&bars[i], 1);
+    mbar_init(&sm.stall[warp], 1);
     fence_mbar_init();
   }
 
@@ -910,9 +912,11 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     const unsigned long long se = sm.seg[warp][meta_seg(sm.meta[warp][0])];
     cur_bg = seg_b(se) * a.Hkv + seg_g(se);
   }
-  bool failed = false;
+  // The wait-limit test: a wait on a barrier that nothing arrives on runs out, and the warp takes
+  // the failure path below with its first copies in flight.
+  bool failed = a.stall_test && !mbar_wait_bounded(&sm.stall[warp], 0u, a.err, a.wait_ns);
   int k = 0;
-  while (true) {
+  while (!failed) {
     if ((k % kChunk) == 0) {
       // descriptors of slots [k + kChunk, k + 2 kChunk) while this chunk is consumed
       Cursor fc = sm.cur[warp];
@@ -927,7 +931,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     }
     if (lane == 0 && issue(k + kStages - 1)) ++issued;
     const int st = k % kStages;
-    const bool ok = mbar_wait_bounded(&bars[st], static_cast<uint32_t>((k / kStages) & 1), a.err);
+    const bool ok = mbar_wait_bounded(&bars[st], static_cast<uint32_t>((k / kStages) & 1), a.err, a.wait_ns);
     if (__any_sync(FULL, !ok)) {
       failed = true;
       break;
@@ -1033,7 +1037,8 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     // A copy did not arrive in time: wait (bounded) for every copy this warp still has in
     // flight so none lands in shared memory after the CTA exits, then leave.
     issued = __shfl_sync(FULL, issued, 0);
-    for (int j = k; j < issued; ++j) mbar_wait_bounded(&bars[j % kStages], static_cast<uint32_t>((j / kStages) & 1), a.err);
+    for (int j = k; j < issued; ++j)
+      mbar_wait_bounded(&bars[j % kStages], static_cast<uint32_t>((j / kStages) & 1), a.err, a.wait_ns);
   }
 }
 
@@ -1066,6 +1071,18 @@ __global__ void __launch_bounds__(kMergeThreads) merge_int4_kernel(const DecodeA
   const int g = j / G, hd = j - g * G;
   pdl_wait();
   const uint4 mt = *reinterpret_cast<const uint4*>(a.meta + 4 * (b * a.Hkv + g));
+  {
+    // A record whose partial rows fall outside the workspace can only be left over from a decode
+    // that stopped early (a wait that ran out): report it and write no output from it.
+    const unsigned long long rows = static_cast<unsigned long long>(a.W) + 2ull * a.B * a.Hkv;
+    const unsigned long long sid8 = 2ull * (b * a.Hkv + g);
+    const bool bad8 = mt.z && static_cast<unsigned long long>(mt.x) + mt.z + sid8 > rows;
+    const bool bad4 = mt.w && static_cast<unsigned long long>(mt.y) + mt.w + sid8 + 1ull > rows;
+    if (bad8 || bad4 || mt.z > rows || mt.w > rows) {
+      if (lane == 0 && sub == 0) atomicOr(a.err, KV4_DEVERR_RECORD);
+      return;
+    }
+  }
   const int n8p = static_cast<int>(mt.z), n = static_cast<int>(mt.z + mt.w);
   if (n == 0 || (n == 1 && !a.rotate_v)) return;  // uniform over the item's warps
   const PartRows pr{n8p, mt.x, mt.y, 2u * static_cast<u32>(b * a.Hkv + g)};

@@ -69,18 +69,21 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// Wait for phase `parity` of `bar`, giving up after about two seconds (global timer) or 2^26
-// polls, whichever comes first.  On expiry the error bit is set and false is returned; the
-// caller then stops consuming and drains.  No kernel of this library spins without a bound.
+// Wait for phase `parity` of `bar`, giving up after `limit_ns` of global time (two seconds by
+// default) or 2^26 polls, whichever comes first.  On expiry the error bit is set and false is
+// returned; the caller then stops consuming and drains.  No kernel of this library spins without
+// a bound.  The clock is read every 16 polls, so with the suspend hint the wait ends at most
+// about 16 hints past the limit.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kWaitLimitPolls = 1u << 26;
 
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* err) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1; it < kWaitLimitPolls; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) break;
+    if ((it & 15u) == 0u && global_timer_ns() - t0 > limit_ns) break;
   }
   atomicOr(err, KV4_DEVERR_WAIT_LIMIT);
   return false;

@@ -50,6 +50,8 @@ struct DecodeArgs {
   int early;              // build the schedule before waiting on the preceding kernel
   uint32_t signs[4];      // bit d: query dim d negated before the rotation (as the keys)
   int rotate_v;           // values stored rotated: outputs are rotated back by the merge kernel
+  int stall_test;         // kv4_debug_force_wait_timeout: every warp's first wait runs out
+  uint64_t wait_ns;       // bounded-wait limit of the bulk-copy waits
   uint32_t* err;
 };
 

@@ -21,14 +21,15 @@ LIB_PATH = os.path.join(_HERE, "libkv4.so")
 
 KV4_OK, KV4_ERR_INVALID_ARG, KV4_ERR_UNSUPPORTED, KV4_ERR_WORKSPACE, KV4_ERR_CUDA, KV4_ERR_DEVICE = range(6)
 KV4_F32, KV4_BF16, KV4_F16 = 0, 1, 2
-KV4_DEVERR_PAGE_RANGE, KV4_DEVERR_WAIT_LIMIT, KV4_DEVERR_LENGTH = 0x1, 0x2, 0x4
+KV4_DEVERR_PAGE_RANGE, KV4_DEVERR_WAIT_LIMIT, KV4_DEVERR_LENGTH, KV4_DEVERR_RANGE, KV4_DEVERR_RECORD = 0x1, 0x2, 0x4, 0x8, 0x10
 
 # every entry point declared in include/kv4.h
 SYMBOLS = (
     "kv4_query_sizes", "kv4_cache_init", "kv4_cache_destroy", "kv4_append", "kv4_decode_workspace_bytes",
-    "kv4_decode_attn", "kv4_decode_attn_static", "kv4_set_decode_overlap", "kv4_set_rotation_signs", "kv4_set_value_rotation", "kv4_bf16_query_sizes", "kv4_bf16_cache_init", "kv4_bf16_append",
-    "kv4_bf16_decode_workspace_bytes", "kv4_bf16_decode_attn", "kv4_get_device_error", "kv4_launch_count",
-    "kv4_status_string", "kv4_version",
+    "kv4_decode_attn", "kv4_decode_attn_static", "kv4_set_decode_overlap", "kv4_debug_force_wait_timeout",
+    "kv4_set_rotation_signs", "kv4_set_value_rotation", "kv4_bf16_query_sizes", "kv4_bf16_cache_init",
+    "kv4_bf16_append", "kv4_bf16_decode_workspace_bytes", "kv4_bf16_decode_attn", "kv4_get_device_error",
+    "kv4_launch_count", "kv4_status_string", "kv4_version",
 )
 
 
@@ -60,6 +61,7 @@ def _load():
         "kv4_decode_attn": (I, [P, I, I, P, I, i32p, I, i32p, I, P, P, P, S, P]),
         "kv4_decode_attn_static": (I, [P, I, I, P, I, i32p, I, i32p, I, P, P, P]),
         "kv4_set_decode_overlap": (I, [P, I]),
+        "kv4_debug_force_wait_timeout": (I, [P, I]),
         "kv4_set_rotation_signs": (I, [P, P]),
         "kv4_set_value_rotation": (I, [P, I]),
         "kv4_bf16_query_sizes": (I, [cfgp, ctypes.POINTER(S)]),
@@ -184,6 +186,12 @@ def kv4_set_decode_overlap(handle, enable: bool):
     """With enable, the decode kernel builds its schedule from lens and page_table while the
     preceding kernel on the stream runs (they must not be written by that kernel)."""
     _check("kv4_set_decode_overlap", lib.kv4_set_decode_overlap(handle, 1 if enable else 0))
+
+
+def kv4_debug_force_wait_timeout(handle, enable: bool):
+    """Test hook: with enable, the decode's bounded waits are made to run out (1 ms limit), so the
+    device-side failure path runs and KV4_DEVERR_WAIT_LIMIT is reported.  Off by default."""
+    _check("kv4_debug_force_wait_timeout", lib.kv4_debug_force_wait_timeout(handle, 1 if enable else 0))
 
 
 def kv4_bf16_query_sizes(cfg: kv4_config) -> int:

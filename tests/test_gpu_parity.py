@@ -273,3 +273,96 @@ def test_value_rotation(case_id):
     T.assert_close(out, ref, lse, ref_lse, what=f"value rotation {CASES[case_id][0]}")
     assert kv4.kv4_get_device_error() == 0
 
+
+
+@pytest.mark.parametrize("case_id", [1, 3], ids=["d128-g4", "d64-g1"])
+def test_decode_f16_query(case_id):
+    """fp16 queries (KV4_F16): the kernel widens them exactly, like the oracle's fp16 input path."""
+    from int4_kv_cache_append_b200 import kv4
+    wl = make(CASES[case_id])
+    gc = T.gpu_cache_from_host_inputs(wl)
+    cfg, pool, side = T.oracle_cache(wl)
+    q32 = W.query_values(W.stream_key(wl.seed, W.KIND_Q, 0), wl.B, wl.Hq, wl.D)
+    qbits = np.ascontiguousarray(q32.astype(np.float16).view(np.uint16))
+    ref, ref_lse = O.decode(cfg, pool, side, qbits, wl.page_table, wl.lens, q_dtype=O.F16)
+    qd = torch.from_numpy(qbits.view(np.int16)).cuda().view(torch.float16)
+    lse = torch.empty((wl.B, wl.Hq), device="cuda")
+    out = gc.decode(0, qd, torch.from_numpy(wl.page_table).cuda(), torch.from_numpy(wl.lens).cuda(), lse=lse)
+    torch.cuda.synchronize()
+    T.assert_close(out.cpu().numpy(), ref, lse.cpu().numpy(), ref_lse, what=f"fp16 q {CASES[case_id][0]}")
+    # the fp16 query is not the bf16 one: the two oracle results differ
+    qb = np.ascontiguousarray(W.bf16_bits(q32))
+    other, _ = O.decode(cfg, pool, side, qb, wl.page_table, wl.lens, q_dtype=O.BF16)
+    assert not np.allclose(other, ref, rtol=0, atol=1e-7)
+    assert kv4.kv4_get_device_error() == 0
+
+
+def test_range_overflow_sets_error_bit():
+    """A key element of 1e6 (spread by the rotation, the vector's minimum is below -65504: its fp16
+    offset is -inf) and a value element of 2e6 ((max - zero)/15 above 65504: scale +inf): the append
+    stores both vectors with all-zero codes and their non-finite parameters, byte for byte as the
+    oracle does, and reports KV4_DEVERR_RANGE; the other vectors are unaffected."""
+    from int4_kv_cache_append_b200 import kv4
+    wl = W.make_workload("range", 37, 1, 2, 8, 2, 128, 16, 4, 16, 64, lambda r: [40, 25],
+                         W.F32, W.F32, W.F32, 2, 20.0)
+    b, p = T.prefill_tokens(wl.lens)
+    K, V = wl.kv_inputs(0, b, p)
+    K = K.copy()
+    V = V.copy()
+    K[3, 1, 17] = 1.0e6   # position 3 of sequence 0: a sink (also in the side cache)
+    V[45, 0, 5] = 2.0e6   # position 5 of sequence 1: INT4 only
+    gc = kv4.Cache(T.geometry(wl), fill=0xA5)
+    pt = torch.from_numpy(wl.page_table).cuda()
+    assert kv4.kv4_get_device_error() == 0
+    gc.append(0, T.to_dev(K), T.to_dev(V), torch.from_numpy(b).cuda(), torch.from_numpy(p).cuda(),
+              torch.from_numpy(wl.lens).cuda(), pt)
+    torch.cuda.synchronize()
+    assert kv4.kv4_get_device_error() & kv4.KV4_DEVERR_RANGE
+    cfg = O.Config(wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h, wl.B)
+    pool = np.full(O.page_bytes(cfg) * wl.num_pages, 0xA5, np.uint8)
+    side = np.full(O.side_slot_bytes(cfg) * wl.B, 0xA5, np.uint8)
+    assert O.append(cfg, pool, side, K, V, b, p, wl.lens, wl.page_table)
+    gp, gs = gc.layer_views(0)
+    assert np.array_equal(gp.cpu().numpy(), pool) and np.array_equal(gs.cpu().numpy(), side)
+    # the flagged key's stored offset is -inf, the flagged value's scale +inf
+    off = O.byte_offset("p4", cfg, int(wl.page_table[0, 0]), 1, 3, 0)
+    assert int(pool[off + 2]) | (int(pool[off + 3]) << 8) == 0xFC00
+    off = O.byte_offset("p4", cfg, int(wl.page_table[1, 0]), 0, 5, 1)
+    assert int(pool[off]) | (int(pool[off + 1]) << 8) == 0x7C00
+    # without the planted elements nothing is reported
+    K0, V0 = wl.kv_inputs(0, b, p)
+    gc.append(0, T.to_dev(K0), T.to_dev(V0), torch.from_numpy(b).cuda(), torch.from_numpy(p).cuda(),
+              torch.from_numpy(wl.lens).cuda(), pt)
+    torch.cuda.synchronize()
+    assert kv4.kv4_get_device_error() == 0
+
+
+def test_wait_limit_failure_path_reports_and_recovers():
+    """The device-side failure path of the bounded waits, made to run with the test hook (no
+    invalid copy involved): every decode warp's first wait is on a barrier that nothing arrives
+    on, runs out after its 1 ms limit, sets KV4_DEVERR_WAIT_LIMIT, waits for its copies in flight
+    and returns.  The merge kernel then meets the workspace's stale records (0xA5 fill), which
+    point outside the workspace, skips them and reports KV4_DEVERR_RECORD.  The context stays
+    usable: with the hook off the next decode matches the oracle and reports nothing."""
+    from int4_kv_cache_append_b200 import kv4
+    wl = make(CASES[1])
+    gc = T.gpu_cache_from_host_inputs(wl)
+    assert kv4.kv4_get_device_error() == 0
+    q_host = wl.q_input(0)
+    pt = torch.from_numpy(wl.page_table).cuda()
+    lens = torch.from_numpy(wl.lens).cuda()
+    ws = torch.full((kv4.kv4_decode_workspace_bytes(gc.handle, wl.B),), 0xA5, dtype=torch.uint8, device="cuda")
+    kv4.kv4_debug_force_wait_timeout(gc.handle, True)
+    try:
+        gc.decode(0, T.to_dev(q_host), pt, lens, workspace=ws)
+        torch.cuda.synchronize()
+    finally:
+        kv4.kv4_debug_force_wait_timeout(gc.handle, False)
+    err = kv4.kv4_get_device_error()
+    assert err & kv4.KV4_DEVERR_WAIT_LIMIT, hex(err)
+    assert err & kv4.KV4_DEVERR_RECORD, hex(err)
+    cfg, pool, side = T.oracle_cache(wl)
+    ref, ref_lse = T.oracle_decode(wl, cfg, pool, side, q_host)
+    out, lse = T.gpu_decode(gc, wl, q_host)
+    T.assert_close(out, ref, lse, ref_lse, what="decode after the wait-limit path")
+    assert kv4.kv4_get_device_error() == 0
