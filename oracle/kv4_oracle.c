@@ -32,6 +32,10 @@
  *   R5 routing: every token gets INT4 codes; in addition pos < s goes to sink row pos, and
  *      pos >= s with pos >= lens_after - w goes to ring row s + (pos mod w).
  *   R6 byte layout of pages and of the side cache: see the orc_*_byte functions.
+ *   R8 bf16 values (value_format 1, the K-INT4 / V-BF16 precision variant): keys exactly as
+ *      above; values are not quantised but stored as bf16 (nearest-even from fp32, the input
+ *      itself for bf16 inputs) in the pages and, for sink/recent positions, in the side cache,
+ *      beside the INT8 keys.
  *   R7 attention: q head j reads kv head j / (Hq/Hkv); softmax scale 1/sqrt(D); regions are
  *      sinks [0, min(s,L)), INT4 [s, max(s, L-w)), recent [max(s, L-w), L).
  */
@@ -110,6 +114,17 @@ float orc_bf16_to_f32(uint16_t b) {
   float f;
   memcpy(&f, &u, 4);
   return f;
+}
+
+/* Round a binary32 value to bfloat16 (8 exponent bits, 7 fraction bits: the upper half of the
+ * binary32 pattern), nearest with ties to even, from the format definition: the dropped 16 bits
+ * are compared with half of the kept quantum.  Finite inputs only (the library's precondition). */
+uint16_t orc_f32_to_bf16(float x) {
+  uint32_t u;
+  memcpy(&u, &x, 4);
+  const uint32_t hi = u >> 16, lo = u & 0xFFFFu;
+  const uint32_t up = lo > 0x8000u || (lo == 0x8000u && (hi & 1u));
+  return (uint16_t)(hi + up);
 }
 
 static double load_elem(const void* base, int dtype, size_t i) {
@@ -242,19 +257,33 @@ int orc_quant_int8(const float* x, int D, int8_t* codes8, uint16_t* scale) {
  * The pages leave the layout free ("token-wise INT4 ... without changing the tensor layout"
  * in [SAW-INT4 s2] refers to the paged buffers, which stay paged here).
  */
+/* Bytes of one position of one KV head in a page: INT4 values D/2 + 4 (K codes, V codes, two
+ * (scale, zero) pairs); bf16 values (value_format 1) D/2 + 4 + 2D (K codes and parameters, V as
+ * bf16).  In the side cache: INT8 values 2D + 4 (K and V codes, two scales); bf16 values 3D + 2
+ * (K codes and scale, V as bf16). */
+static size_t pos4_bytes(const orc_config* c) {
+  const size_t D = (size_t)c->head_dim;
+  return c->value_format ? D / 2 + 4 + 2 * D : D + 8;
+}
+
+static size_t pos8_bytes(const orc_config* c) {
+  const size_t D = (size_t)c->head_dim;
+  return c->value_format ? 3 * D + 2 : 2 * D + 4;
+}
+
 size_t orc_page_bytes(const orc_config* c) {
-  return (size_t)c->num_kv_heads * (size_t)c->page_size * (size_t)(c->head_dim + 8);
+  return (size_t)c->num_kv_heads * (size_t)c->page_size * pos4_bytes(c);
 }
 
 int orc_side_tiles(const orc_config* c) { return (c->num_sinks + c->recent_window + 15) / 16; }
 
 size_t orc_side_slot_bytes(const orc_config* c) {
-  return (size_t)c->num_kv_heads * (size_t)orc_side_tiles(c) * 16u * (size_t)(2 * c->head_dim + 4);
+  return (size_t)c->num_kv_heads * (size_t)orc_side_tiles(c) * 16u * pos8_bytes(c);
 }
 
 static size_t tile4_base(const orc_config* c, int page, int g, int pp) {
-  const size_t D = (size_t)c->head_dim, P = (size_t)c->page_size;
-  return (size_t)page * orc_page_bytes(c) + (size_t)g * P * (D + 8) + (size_t)(pp / 16) * 16u * (D + 8);
+  const size_t P = (size_t)c->page_size, pb = pos4_bytes(c);
+  return (size_t)page * orc_page_bytes(c) + (size_t)g * P * pb + (size_t)(pp / 16) * 16u * pb;
 }
 
 size_t orc_k4_byte(const orc_config* c, int page, int g, int pp, int e) {
@@ -282,12 +311,32 @@ size_t orc_v4_byte(const orc_config* c, int page, int g, int pp, int e) {
 
 size_t orc_p4_byte(const orc_config* c, int page, int g, int pp, int is_v) {
   const int D = c->head_dim, r = pp % 16;
+  if (c->value_format) return tile4_base(c, page, g, pp) + (size_t)(8 * D + 4 * r); /* K only */
   return tile4_base(c, page, g, pp) + (size_t)(16 * D + 64 * is_v + 4 * r);
 }
 
+/* bf16 values (value_format 1): a 16-row block of V in the order the PV tensor-core fragments
+ * read it.  Rows 2p and 2p+1 are a pair; elements are grouped in D/8 groups of D/8; for pair p
+ * (half = p / 4) and group gq a chunk of D/2 bytes at ((half*8 + gq)*4 + p%4) * D/2 holds the
+ * words (V[2p][e], V[2p+1][e]) for the elements e of the group in order, and the 16-byte units of
+ * the chunk are permuted by u -> u ^ swz (swz = (p%4 & 2) | (gq & 1) when a chunk has 4 units,
+ * gq & 1 when it has 2, 0 when it has 1). */
+static size_t vbf_off(int D, int r, int e) {
+  const int p = r >> 1, half = p >> 2, pl = p & 3;
+  const int dg = D / 8, gq = e / dg, m = e % dg;
+  const int units = D / 32;
+  const int swz = units >= 4 ? ((pl & 2) | (gq & 1)) : (units >= 2 ? (gq & 1) : 0);
+  const int u = (m * 4) / 16, within = (m * 4) % 16;
+  return (size_t)(((half * 8 + gq) * 4 + pl) * (D / 2) + 16 * (u ^ swz) + within + 2 * (r & 1));
+}
+
+size_t orc_vb_byte(const orc_config* c, int page, int g, int pp, int e) {
+  const int D = c->head_dim;
+  return tile4_base(c, page, g, pp) + (size_t)(8 * D + 64) + vbf_off(D, pp % 16, e);
+}
+
 static size_t tile8_base(const orc_config* c, int slot, int g, int row) {
-  const size_t D = (size_t)c->head_dim;
-  const size_t t8 = 16u * (2 * D + 4);
+  const size_t t8 = 16u * pos8_bytes(c);
   return (size_t)slot * orc_side_slot_bytes(c) + (size_t)g * (size_t)orc_side_tiles(c) * t8 +
          (size_t)(row / 16) * t8;
 }
@@ -312,6 +361,11 @@ size_t orc_s8_byte(const orc_config* c, int slot, int g, int row, int is_v) {
   return tile8_base(c, slot, g, row) + (size_t)(16 * D + is_v * (16 * D + 32) + 2 * r);
 }
 
+size_t orc_vb8_byte(const orc_config* c, int slot, int g, int row, int e) {
+  const int D = c->head_dim;
+  return tile8_base(c, slot, g, row) + (size_t)(16 * D + 32) + vbf_off(D, row % 16, e);
+}
+
 static int config_ok(const orc_config* c) {
   const int D = c->head_dim, h = c->hadamard_block;
   if (c->num_kv_heads <= 0 || c->num_q_heads <= 0 || c->num_q_heads % c->num_kv_heads) return 0;
@@ -319,6 +373,8 @@ static int config_ok(const orc_config* c) {
   if (c->page_size <= 0 || c->page_size % 16) return 0;
   if (c->num_sinks < 0 || c->recent_window < 0 || c->max_seqs <= 0) return 0;
   if (h <= 0 || (h & (h - 1)) || D % h) return 0;
+  if (c->value_format != 0 && c->value_format != 1) return 0;
+  if (c->value_format && c->rotate_values) return 0; /* bf16 values are stored as given */
   return 1;
 }
 
@@ -376,10 +432,15 @@ int orc_append(const orc_config* c, uint8_t* pool, uint8_t* side, int T, const v
       for (int e = 0; e < D; ++e) put_nibble(pool, orc_k4_byte(c, page, g, pp, e), orc_k4_high(c, pp, e), c4[e]);
       put_u16(pool, orc_p4_byte(c, page, g, pp, 0), sc);
       put_u16(pool, orc_p4_byte(c, page, g, pp, 0) + 2, zr);
-      range |= orc_quant_int4(vf, D, c4, &sc, &zr);
-      for (int e = 0; e < D; ++e) put_nibble(pool, orc_v4_byte(c, page, g, pp, e), e & 1, c4[e]);
-      put_u16(pool, orc_p4_byte(c, page, g, pp, 1), sc);
-      put_u16(pool, orc_p4_byte(c, page, g, pp, 1) + 2, zr);
+      if (c->value_format) {
+        /* bf16 values: the value itself, rounded to bf16 (exact for bf16 inputs) */
+        for (int e = 0; e < D; ++e) put_u16(pool, orc_vb_byte(c, page, g, pp, e), orc_f32_to_bf16(vf[e]));
+      } else {
+        range |= orc_quant_int4(vf, D, c4, &sc, &zr);
+        for (int e = 0; e < D; ++e) put_nibble(pool, orc_v4_byte(c, page, g, pp, e), e & 1, c4[e]);
+        put_u16(pool, orc_p4_byte(c, page, g, pp, 1), sc);
+        put_u16(pool, orc_p4_byte(c, page, g, pp, 1) + 2, zr);
+      }
 
       int row = -1;
       if (p < s)
@@ -391,9 +452,13 @@ int orc_append(const orc_config* c, uint8_t* pool, uint8_t* side, int T, const v
         range |= orc_quant_int8(kf, D, c8, &s8);
         for (int e = 0; e < D; ++e) side[orc_k8_byte(c, b, g, row, e)] = (uint8_t)c8[e];
         put_u16(side, orc_s8_byte(c, b, g, row, 0), s8);
-        range |= orc_quant_int8(vf, D, c8, &s8);
-        for (int e = 0; e < D; ++e) side[orc_v8_byte(c, b, g, row, e)] = (uint8_t)c8[e];
-        put_u16(side, orc_s8_byte(c, b, g, row, 1), s8);
+        if (c->value_format) {
+          for (int e = 0; e < D; ++e) put_u16(side, orc_vb8_byte(c, b, g, row, e), orc_f32_to_bf16(vf[e]));
+        } else {
+          range |= orc_quant_int8(vf, D, c8, &s8);
+          for (int e = 0; e < D; ++e) side[orc_v8_byte(c, b, g, row, e)] = (uint8_t)c8[e];
+          put_u16(side, orc_s8_byte(c, b, g, row, 1), s8);
+        }
       }
     }
   }
@@ -419,22 +484,28 @@ int orc_dequant_seq(const orc_config* c, const uint8_t* pool, const uint8_t* sid
       region[j] = j < s_end ? 0 : 2;
       const int row = j < s ? j : s + j % w;
       const double ks = (double)orc_f16_to_f32(get_u16(side, orc_s8_byte(c, slot, g, row, 0)));
-      const double vs = (double)orc_f16_to_f32(get_u16(side, orc_s8_byte(c, slot, g, row, 1)));
-      for (int e = 0; e < D; ++e) {
-        kr[e] = ks * (double)(int8_t)side[orc_k8_byte(c, slot, g, row, e)];
-        vr[e] = vs * (double)(int8_t)side[orc_v8_byte(c, slot, g, row, e)];
+      for (int e = 0; e < D; ++e) kr[e] = ks * (double)(int8_t)side[orc_k8_byte(c, slot, g, row, e)];
+      if (c->value_format) {
+        for (int e = 0; e < D; ++e) vr[e] = (double)orc_bf16_to_f32(get_u16(side, orc_vb8_byte(c, slot, g, row, e)));
+      } else {
+        const double vs = (double)orc_f16_to_f32(get_u16(side, orc_s8_byte(c, slot, g, row, 1)));
+        for (int e = 0; e < D; ++e) vr[e] = vs * (double)(int8_t)side[orc_v8_byte(c, slot, g, row, e)];
       }
     } else {
       region[j] = 1;
       const int page = page_row[j / P], pp = j % P;
-      const size_t kp = orc_p4_byte(c, page, g, pp, 0), vp = orc_p4_byte(c, page, g, pp, 1);
+      const size_t kp = orc_p4_byte(c, page, g, pp, 0);
       const double ks = (double)orc_f16_to_f32(get_u16(pool, kp));
       const double kz = (double)orc_f16_to_f32(get_u16(pool, kp + 2));
-      const double vs = (double)orc_f16_to_f32(get_u16(pool, vp));
-      const double vz = (double)orc_f16_to_f32(get_u16(pool, vp + 2));
-      for (int e = 0; e < D; ++e) {
+      for (int e = 0; e < D; ++e)
         kr[e] = kz + ks * (double)get_nibble(pool, orc_k4_byte(c, page, g, pp, e), orc_k4_high(c, pp, e));
-        vr[e] = vz + vs * (double)get_nibble(pool, orc_v4_byte(c, page, g, pp, e), e & 1);
+      if (c->value_format) {
+        for (int e = 0; e < D; ++e) vr[e] = (double)orc_bf16_to_f32(get_u16(pool, orc_vb_byte(c, page, g, pp, e)));
+      } else {
+        const size_t vp = orc_p4_byte(c, page, g, pp, 1);
+        const double vs = (double)orc_f16_to_f32(get_u16(pool, vp));
+        const double vz = (double)orc_f16_to_f32(get_u16(pool, vp + 2));
+        for (int e = 0; e < D; ++e) vr[e] = vz + vs * (double)get_nibble(pool, orc_v4_byte(c, page, g, pp, e), e & 1);
       }
     }
   }

@@ -47,12 +47,16 @@ typedef struct {
                             key and of the query before the Hadamard; all zero = plain H    */
   int rotate_values;     /* values stored rotated like the keys (H diag(s)); outputs rotated
                             back as diag(s) H o / h                                          */
+  int value_format;      /* 0: INT4 values (INT8 in the side cache); 1: values stored as bf16 in
+                            the pages and the side cache (keys as in format 0); with 1,
+                            rotate_values must be 0                                          */
 } orc_config;
 
 /* fp16 helpers (IEEE binary16), written from the format definition. */
 uint16_t orc_f32_to_f16(float x, int mode);
 float    orc_f16_to_f32(uint16_t h);
 float    orc_bf16_to_f32(uint16_t b);
+uint16_t orc_f32_to_bf16(float x);  /* nearest, ties to even */
 
 /* Block-diagonal Sylvester Hadamard, unnormalised, fp32 butterfly in ascending stride order. */
 void orc_fwht_f32(float* x, int D, int h);
@@ -82,6 +86,10 @@ size_t orc_p4_byte(const orc_config* c, int page, int g, int pos_in_page, int is
 size_t orc_k8_byte(const orc_config* c, int slot, int g, int row, int elem);
 size_t orc_v8_byte(const orc_config* c, int slot, int g, int row, int elem);
 size_t orc_s8_byte(const orc_config* c, int slot, int g, int row, int is_v);
+/* value_format 1: byte of the bf16 value element elem (2 bytes, little-endian) in a page tile /
+ * in a side-cache row.  orc_p4_byte then names the K parameters only (is_v ignored). */
+size_t orc_vb_byte(const orc_config* c, int page, int g, int pos_in_page, int elem);
+size_t orc_vb8_byte(const orc_config* c, int slot, int g, int row, int elem);
 
 /* Append T tokens (K, V [T][Hkv][D], element type k_dtype / v_dtype) into host copies of
  * one layer's page pool and side cache.  Returns 0, ORC_APPEND_RANGE when some vector's fp16

@@ -47,7 +47,8 @@ class _Cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "num_q_heads", "num_kv_heads", "head_dim", "page_size", "num_sinks",
         "recent_window", "hadamard_block", "max_seqs")] + [("sign_bits", ctypes.c_uint32 * 4),
-                                                           ("rotate_values", ctypes.c_int)]
+                                                           ("rotate_values", ctypes.c_int),
+                                                           ("value_format", ctypes.c_int)]
 
 
 @dataclass(frozen=True)
@@ -63,12 +64,13 @@ class Config:
     max_seqs: int
     sign_bits: tuple = (0, 0, 0, 0)  # randomised-sign rotation (bit d negates dim d); zero = plain
     rotate_values: int = 0  # values stored rotated like the keys
+    value_format: int = 0  # 0: INT4 values; 1: bf16 values (keys as in 0)
 
     def c(self) -> _Cfg:
         return _Cfg(self.num_q_heads, self.num_kv_heads, self.head_dim, self.page_size,
                     self.num_sinks, self.recent_window, self.hadamard_block, self.max_seqs,
                     (ctypes.c_uint32 * 4)(*[int(x) & 0xFFFFFFFF for x in (list(self.sign_bits) + [0] * 4)[:4]]),
-                    int(self.rotate_values))
+                    int(self.rotate_values), int(self.value_format))
 
 
 _lib = None
@@ -103,7 +105,10 @@ def lib():
             getattr(L, n).restype = S
         L.orc_side_tiles.argtypes = [cfgp]
         L.orc_side_tiles.restype = I
-        for n in ("orc_k4_byte", "orc_v4_byte", "orc_p4_byte", "orc_k8_byte", "orc_v8_byte", "orc_s8_byte"):
+        L.orc_f32_to_bf16.argtypes = [ctypes.c_float]
+        L.orc_f32_to_bf16.restype = ctypes.c_uint16
+        for n in ("orc_k4_byte", "orc_v4_byte", "orc_p4_byte", "orc_k8_byte", "orc_v8_byte", "orc_s8_byte",
+                  "orc_vb_byte", "orc_vb8_byte"):
             getattr(L, n).argtypes = [cfgp, I, I, I, I]
             getattr(L, n).restype = S
         L.orc_k4_high.argtypes = [cfgp, I, I]
@@ -135,6 +140,10 @@ def f16_to_f32(bits: int) -> float:
 
 def bf16_to_f32(bits: int) -> float:
     return float(lib().orc_bf16_to_f32(ctypes.c_uint16(int(bits))))
+
+
+def f32_to_bf16(x: float) -> int:
+    return int(lib().orc_f32_to_bf16(ctypes.c_float(float(x))))
 
 
 def fwht_f32(x: np.ndarray, h: int) -> np.ndarray:
@@ -193,8 +202,8 @@ def side_tiles(cfg: Config) -> int:
 
 
 def byte_offset(kind: str, cfg: Config, a: int, g: int, r: int, e: int) -> int:
-    """kind in {k4, v4, p4, k8, v8, s8}; (a, g, r, e) = (page or slot, kv head, position in
-    page or side row, element or is_v)."""
+    """kind in {k4, v4, p4, k8, v8, s8, vb, vb8}; (a, g, r, e) = (page or slot, kv head, position
+    in page or side row, element or is_v).  vb / vb8: bf16 values (value_format 1)."""
     return int(getattr(lib(), f"orc_{kind}_byte")(ctypes.byref(cfg.c()), a, g, r, e))
 
 

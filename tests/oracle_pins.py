@@ -328,13 +328,83 @@ def pin_layout_bijection():
         assert np.all(own == 1), (D, np.unique(own, return_counts=True))
 
 
+def _bf16_rne(x: np.ndarray) -> np.ndarray:
+    """fp32 -> bfloat16 bit patterns, nearest with ties to even, on the integer bits."""
+    u = np.ascontiguousarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def pin_bf16_rounding(seed: int = 23):
+    """orc_f32_to_bf16 is round-to-nearest-even on the 16 dropped bits: random finite patterns,
+    exact halfway cases of both parities, and values already in bf16."""
+    rng = np.random.default_rng(seed)
+    bits = rng.integers(0, 2**32, size=20000, dtype=np.uint64).astype(np.uint32)
+    x = bits.view(np.float32)
+    x = x[np.isfinite(x)]
+    half = (np.arange(-300, 300, dtype=np.int64) << 16 | 0x8000).astype(np.uint32).view(np.float32)
+    exact = (rng.integers(0, 2**16, size=500).astype(np.uint32) << 16).view(np.float32)
+    for arr in (x, half[np.isfinite(half)], exact[np.isfinite(exact)]):
+        want = _bf16_rne(arr)
+        got = np.array([O.f32_to_bf16(float(v)) for v in arr], np.uint16)
+        assert np.array_equal(got, want), np.nonzero(got != want)[0][:5]
+
+
+def pin_layout_bijection_bf16_values():
+    """bf16 values (value_format 1): every byte of a page tile (K nibbles, K parameters, V bf16)
+    and of a side tile (K int8, K scale, V bf16) is owned by exactly one item."""
+    for D, P, Hkv, s, w in ((64, 16, 2, 4, 32), (128, 32, 1, 3, 10), (32, 16, 1, 2, 5)):
+        cfg = O.Config(Hkv, Hkv, D, P, s, w, 1, 2, value_format=1)
+        pb = O.page_bytes(cfg)
+        assert pb == Hkv * P * (D // 2 + 4 + 2 * D)
+        nib = np.zeros(2 * pb, np.int32)
+        for g in range(Hkv):
+            for pp in range(P):
+                for e in range(D):
+                    nib[2 * O.byte_offset("k4", cfg, 1, g, pp, e) - 2 * pb + O.nibble_high("k4", cfg, pp, e)] += 1
+                    off = O.byte_offset("vb", cfg, 1, g, pp, e) - pb
+                    nib[2 * off:2 * off + 4] += 1
+                off = O.byte_offset("p4", cfg, 1, g, pp, 0) - pb
+                nib[2 * off:2 * off + 8] += 1
+        assert np.all(nib == 1), (D, P, np.unique(nib, return_counts=True))
+        sb = O.side_slot_bytes(cfg)
+        assert sb == Hkv * O.side_tiles(cfg) * 16 * (3 * D + 2)
+        own = np.zeros(sb, np.int32)
+        for g in range(Hkv):
+            for row in range(O.side_tiles(cfg) * 16):
+                for e in range(D):
+                    own[O.byte_offset("k8", cfg, 1, g, row, e) - sb] += 1
+                    off = O.byte_offset("vb8", cfg, 1, g, row, e) - sb
+                    own[off:off + 2] += 1
+                off = O.byte_offset("s8", cfg, 1, g, row, 0) - sb
+                own[off:off + 2] += 1
+        assert np.all(own == 1), (D, np.unique(own, return_counts=True))
+
+
+def pin_bf16_values_exact(seed: int = 29):
+    """With bf16 values the dequantised values are the inputs rounded to bf16 (nearest even), in
+    every region, and the keys dequantise exactly as in the INT4-value format."""
+    for dt in (W.F32, W.BF16):
+        wl = small_workload(D=64, lens=(40, 9, 70), s=3, w=8, h=16, seed=seed, dt=dt)
+        cfg, pool, side = build_cache(wl, value_format=1)
+        cfg0, pool0, side0 = build_cache(wl)
+        for b, L in enumerate(wl.lens):
+            _, V = wl.kv_inputs(0, np.full(L, b, np.int32), np.arange(L, dtype=np.int32))
+            vb = V if V.dtype == np.uint16 else _bf16_rne(V)
+            want = (vb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            for g in range(wl.Hkv):
+                kd, vd, _ = O.dequant_seq(cfg, pool, side, wl.page_table[b], b, L, g)
+                kd0, _, _ = O.dequant_seq(cfg0, pool0, side0, wl.page_table[b], b, L, g)
+                assert np.array_equal(vd, want[:, g]), (dt, b, g)
+                assert np.array_equal(kd, kd0), (dt, b, g)
+
+
 # ----------------------------------------------------------------------------- cache helpers
 
 def build_cache(wl: W.Workload, layer: int = 0, lens=None, step_by_step: bool = False, sentinel: int = 0xA5,
-                signs=(0, 0, 0, 0), rotate_values: int = 0):
+                signs=(0, 0, 0, 0), rotate_values: int = 0, value_format: int = 0):
     """Oracle cache for a workload: prefill every token in position order (one call for all
     tokens with lens_after = L, or one call per position with lens_after = pos + 1)."""
-    cfg = oracle_cfg(wl, signs, rotate_values)
+    cfg = oracle_cfg(wl, signs, rotate_values, value_format)
     lens = np.asarray(wl.lens if lens is None else lens, np.int32)
     pool = np.full(O.page_bytes(cfg) * wl.num_pages, sentinel, np.uint8)
     side = np.full(O.side_slot_bytes(cfg) * wl.B, sentinel, np.uint8)
@@ -356,8 +426,8 @@ def build_cache(wl: W.Workload, layer: int = 0, lens=None, step_by_step: bool = 
     return cfg, pool, side
 
 
-def oracle_cfg(wl: W.Workload, signs=(0, 0, 0, 0), rotate_values: int = 0) -> O.Config:
-    return O.Config(wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h, wl.B, tuple(signs), rotate_values)
+def oracle_cfg(wl: W.Workload, signs=(0, 0, 0, 0), rotate_values: int = 0, value_format: int = 0) -> O.Config:
+    return O.Config(wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h, wl.B, tuple(signs), rotate_values, value_format)
 
 
 def small_workload(D=32, B=3, lens=(12, 7, 40), s=2, w=5, h=8, G=2, Hkv=2, P=16, seed=5,
@@ -398,13 +468,29 @@ def pin_routing(step_by_step: bool):
 
 # ----------------------------------------------------------------------------- decode
 
-def _brute_layout_decode(wl: W.Workload, pool, side, b: int, g: int, L: int):
+def _vbf(buf, base: int, D: int, r: int, e: int) -> float:
+    """bf16 value element e of row r of a 16-row V block starting at base: rows 2p, 2p+1 form a
+    pair, element group gq = e // (D/8); the pair's group chunk (D/2 bytes) sits at chunk index
+    (p // 4) * 32 + gq * 4 + p % 4 and holds per element the pair's two bf16 (row 2p first); its
+    16-byte units are permuted by xor with (p%4 & 2 | gq & 1) for 4 units, gq & 1 for 2."""
+    p, dg = r // 2, D // 8
+    gq, m = divmod(e, dg)
+    units = D // 32
+    swz = ((p % 4) & 2 | (gq & 1)) if units >= 4 else ((gq & 1) if units >= 2 else 0)
+    chunk = base + (((p // 4) * 8 + gq) * 4 + p % 4) * (D // 2)
+    byte = chunk + 16 * ((4 * m) // 16 ^ swz) + (4 * m) % 16 + 2 * (r % 2)
+    bits = int(buf[byte]) | (int(buf[byte + 1]) << 8)
+    return float(np.array([bits << 16], np.uint32).view(np.float32)[0])
+
+
+def _brute_layout_decode(wl: W.Workload, pool, side, b: int, g: int, L: int, value_format: int = 0):
     """Independent restatement of the byte layout (written from the layout description, not
     from the C code) returning dense fp64 (khat rotated basis, vhat)."""
     D, P, s, w, Hkv = wl.D, wl.P, wl.s, wl.w, wl.Hkv
-    tile4 = 16 * (D + 8)
+    vbf = value_format == 1
+    tile4 = 16 * (D // 2 + 4 + 2 * D) if vbf else 16 * (D + 8)
     ntiles8 = (s + w + 15) // 16
-    tile8 = 16 * (2 * D + 4)
+    tile8 = 16 * (3 * D + 2) if vbf else 16 * (2 * D + 4)
     kh = np.zeros((L, D))
     vh = np.zeros((L, D))
     f16 = lambda buf, off: float(np.frombuffer(bytes(buf[off:off + 2]), np.float16)[0])
@@ -413,10 +499,14 @@ def _brute_layout_decode(wl: W.Workload, pool, side, b: int, g: int, L: int):
             row = j if j < s else s + j % w
             base = (b * Hkv + g) * ntiles8 * tile8 + (row // 16) * tile8
             r = row % 16
-            ks, vs = f16(side, base + 16 * D + 2 * r), f16(side, base + 32 * D + 32 + 2 * r)
+            ks = f16(side, base + 16 * D + 2 * r)
+            vs = 0.0 if vbf else f16(side, base + 32 * D + 32 + 2 * r)
             for e in range(D):
                 kb = base + r * D + 16 * ((e // 16) ^ (r & 1)) + e % 16
                 kh[j, e] = ks * np.int8(side[kb])
+                if vbf:
+                    vh[j, e] = _vbf(side, base + 16 * D + 32, D, r, e)
+                    continue
                 p_, half, pl = (r >> 1), (r >> 1) >> 2, (r >> 1) & 3
                 dg, ch8 = D // 8, D // 4
                 gq, dd = e // dg, e % dg
@@ -428,10 +518,12 @@ def _brute_layout_decode(wl: W.Workload, pool, side, b: int, g: int, L: int):
         else:
             page = wl.page_table[b, j // P]
             pp = j % P
-            base = page * Hkv * P * (D + 8) + g * P * (D + 8) + (pp // 16) * tile4
+            base = page * Hkv * P * (tile4 // 16) + g * P * (tile4 // 16) + (pp // 16) * tile4
             r = pp % 16
-            ks, kz = f16(pool, base + 16 * D + 4 * r), f16(pool, base + 16 * D + 4 * r + 2)
-            vs, vz = f16(pool, base + 16 * D + 64 + 4 * r), f16(pool, base + 16 * D + 64 + 4 * r + 2)
+            kpar = base + (8 * D if vbf else 16 * D) + 4 * r
+            ks, kz = f16(pool, kpar), f16(pool, kpar + 2)
+            if not vbf:
+                vs, vz = f16(pool, base + 16 * D + 64 + 4 * r), f16(pool, base + 16 * D + 64 + 4 * r + 2)
             for e in range(D):
                 # K: pair-row r % 8 of D bytes, row r in the low (r < 8) or high nibble; element e
                 # in 8-byte group e // 8 (even elements first); 16-byte halves of each 32 bytes
@@ -441,6 +533,9 @@ def _brute_layout_decode(wl: W.Workload, pool, side, b: int, g: int, L: int):
                 unit = (bi // 16) ^ ((pr % 2) if D >= 128 else 0)
                 byte = pool[base + pr * D + 16 * unit + bi % 16]
                 kh[j, e] = kz + ks * ((byte >> 4) if r >= 8 else (byte & 15))
+                if vbf:
+                    vh[j, e] = _vbf(pool, base + 8 * D + 64, D, r, e)
+                    continue
                 Q, k = e // 4, e % 4
                 wpc = D // 32
                 p_ = r >> 1
@@ -452,17 +547,19 @@ def _brute_layout_decode(wl: W.Workload, pool, side, b: int, g: int, L: int):
 
 def pin_brute_force(seed: int = 21):
     """Tiny cases: the oracle's decode against a direct fp64 triple loop with an explicit
-    Hadamard matrix, on a cache read back through an independent layout decoder."""
-    for (lens, s, w, h, G, D) in (((12, 7, 3), 2, 5, 8, 2, 32), ((11, 1, 9), 0, 4, 32, 1, 32),
-                                  ((10, 12, 5), 3, 0, 4, 2, 32), ((21, 3), 1, 2, 16, 1, 128)):
+    Hadamard matrix, on a cache read back through an independent layout decoder (INT4 values,
+    and bf16 values for the last two cases)."""
+    for (lens, s, w, h, G, D, vf) in (((12, 7, 3), 2, 5, 8, 2, 32, 0), ((11, 1, 9), 0, 4, 32, 1, 32, 0),
+                                      ((10, 12, 5), 3, 0, 4, 2, 32, 0), ((21, 3), 1, 2, 16, 1, 128, 0),
+                                      ((19, 6, 2), 2, 4, 8, 2, 64, 1), ((21, 3), 1, 2, 16, 1, 128, 1)):
         wl = small_workload(D=D, lens=lens, s=s, w=w, h=h, G=G, seed=seed)
-        cfg, pool, side = build_cache(wl)
+        cfg, pool, side = build_cache(wl, value_format=vf)
         q = wl.q_input(0)
         out, lse = O.decode(cfg, pool, side, q, wl.page_table, wl.lens)
         Hm = np.kron(np.eye(wl.D // h), scipy.linalg.hadamard(h)).astype(np.float64)
         for b, L in enumerate(wl.lens):
             for g in range(wl.Hkv):
-                kh, vh = _brute_layout_decode(wl, pool, side, b, g, L)
+                kh, vh = _brute_layout_decode(wl, pool, side, b, g, L, value_format=vf)
                 kd, vd, _ = O.dequant_seq(cfg, pool, side, wl.page_table[b], b, L, g)
                 assert np.array_equal(kh, kd) and np.array_equal(vh, vd)
                 for i in range(G):
@@ -624,5 +721,5 @@ ALL_PINS = [
     lambda: pin_routing(False), lambda: pin_routing(True), pin_brute_force,
     pin_append_vs_numpy_requant, pin_regional_equals_single, pin_rotation_invariance,
     pin_special_cases, pin_signed_rotation_exact, pin_value_rotation_invariance, pin_quant_range,
-    pin_append_range_flag,
+    pin_append_range_flag, pin_bf16_rounding, pin_layout_bijection_bf16_values, pin_bf16_values_exact,
 ]

@@ -90,3 +90,20 @@ def test_sink_recent_overrides():
     assert kv8.kv_bytes_int4() == base.Hkv * int(base.lens.astype(int).sum()) * (2 * base.D + 4)
     sw = bench.make_wl(argparse.Namespace(workload="qwen3-4b-decode", h=None, sinks=144, recent=0))
     assert (sw.s, sw.w) == (144, 0)
+
+
+def test_hadamard_override_of_one_layer_workloads():
+    """--h on a one-layer workload (the naive-INT4 h = 1 line beside h = 128) renames it and keeps
+    everything else."""
+    import argparse
+
+    import bench
+    from int4_kv_cache_append_b200 import workload as W
+    base = W.qwen3_4b_decode()
+    wl = bench.make_wl(argparse.Namespace(workload="qwen3-4b-decode", h=1, sinks=None, recent=None))
+    assert wl.h == 1 and wl.name == base.name + "-h1"
+    assert (wl.lens == base.lens).all() and (wl.page_table == base.page_table).all()
+    loop = bench.make_wl(argparse.Namespace(workload="qwen3-8b-loop", h=64, sinks=None, recent=None))
+    assert loop.h == 64 and loop.layers == 36
+    names = [n for n, _, _ in bench.PER_CONFIG]
+    assert {"tiny", "qwen3-4b-decode", "async-refill", "long-context"} <= set(names)

@@ -50,6 +50,14 @@ MUTANTS = [
     ("f16-ties-away", "(frac == 0.5 && fmod(n, 2.0) == 1.0)", "(frac == 0.5)", None),
     ("int4-range-unreported", "  return out_of_range;\n}", "  return 0;\n}", 0),
     ("int8-range-unreported", "  return out_of_range;\n}", "  return 0;\n}", 1),
+    ("bf16-truncate", "const uint32_t up = lo > 0x8000u || (lo == 0x8000u && (hi & 1u));",
+     "const uint32_t up = 0;", None),
+    ("bf16-ties-away", "const uint32_t up = lo > 0x8000u || (lo == 0x8000u && (hi & 1u));",
+     "const uint32_t up = lo >= 0x8000u;", None),
+    ("vbf-no-swizzle", "const int swz = units >= 4 ? ((pl & 2) | (gq & 1)) : (units >= 2 ? (gq & 1) : 0);",
+     "const int swz = 0;", None),
+    ("vbf-pair-rows", "return (size_t)(((half * 8 + gq) * 4 + pl) * (D / 2) + 16 * (u ^ swz) + within + 2 * (r & 1));",
+     "return (size_t)(((half * 8 + gq) * 4 + pl) * (D / 2) + 16 * (u ^ swz) + within + 2 * ((r >> 1) & 1));", None),
     ("single-softmax-max", "if (logit[j] > ps->m) ps->m = logit[j];", "if (logit[j] < ps->m) ps->m = logit[j];", None),
 ]
 

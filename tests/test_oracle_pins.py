@@ -91,3 +91,15 @@ def test_quantiser_range_overflow():
 
 def test_append_reports_range_overflow():
     P.pin_append_range_flag()
+
+
+def test_bf16_rounding():
+    P.pin_bf16_rounding()
+
+
+def test_bf16_value_layout_is_a_bijection():
+    P.pin_layout_bijection_bf16_values()
+
+
+def test_bf16_values_stored_exactly():
+    P.pin_bf16_values_exact()
