@@ -1,16 +1,20 @@
 #!/usr/bin/env python
 """Benchmark: decode steps of INT4-KV attention (append + decode) beside the BF16-KV kernel on
-the same GPU and the CPU oracle on the host cores.  Default workload: Qwen3-4B-like (32 q / 8 KV
-heads, head_dim 128, bf16, B = 64 sequences with lognormal lengths of median 2048 capped at
-8192, P = 16, s = 4, w = 128, h = 128).
+the same GPU and the CPU oracle on the host cores.  Default workload: the Qwen3-8B-like 36-layer
+decode loop (32 q / 8 KV heads, head_dim 128, bf16, B = 128 sequences with lengths U{1024..16384}
+growing by one token per step, P = 16, s = 16, w = 128, h = 128; about 44 GB of cache), the
+largest configuration that fits one GPU.
 
 A layer call = kv4_append of one new token per sequence (rotation, INT4 pack, INT8 routing)
 followed by kv4_decode_attn over the whole cache (INT4 region + INT8 sink/recent regions,
-split-K, regional merge).  One-layer workloads: a step is one layer call, steps cycle over 4
-resident layers (0.72 GB of KV between reuses for the default, larger than the 126 MB L2).
-`--workload qwen3-8b-loop [--h 32|64|128]`: a step is all 36 layers, and every sequence grows by
-one token per step.  Each step is one CUDA graph (the decode a programmatic dependent of the
-append); a second loop times the kernels one by one for the roofline.  Prints one JSON line.
+split-K, regional merge).  The 36-layer workload: a step is all 36 layer calls, and every
+sequence grows by one token per step.  One-layer workloads (`--workload qwen3-4b-decode |
+async-refill | long-context | tiny ...`): a step is one layer call, steps cycle over 4 resident
+layers (inputs larger than the 126 MB L2).  Each step is one CUDA graph (the decode a
+programmatic dependent of the append); a second loop times the kernels one by one for the
+roofline.  At N = 1 the line also carries `per_config`: the one-layer workloads measured in the
+same process (decode time, roofline fraction, BF16-KV decode time, clocks; h = 1 beside h = 128).
+Prints one JSON line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kv4|reference] [--workload NAME]
 Under torchrun (N > 1) every rank runs its own batch on its own GPU (weak scaling, no
@@ -32,6 +36,17 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "INT4-KV decode attn: seq-steps/s and HBM GB/s (% of roofline) vs BF16-KV"
 UNIT = "seq-steps/s"
 LAYERS = 4
+# sequences of the bench workload in the CPU oracle sample (the reference arm and the
+# cpu_baseline leg time the same sample)
+SAMPLE_SEQS = 8
+INPUTS = ("synthetic, seeded: K, V, q are Irwin-Hall N(0,1) stand-ins (sum of 12 uniforms minus 6, "
+          "tails cut at +-6) with fixed outlier channels per KV head")
+# one-layer workloads measured beside the default line: (name, overrides, note); overrides: h
+# (Hadamard block), values ("bf16": the K-INT4 / V-BF16 variant)
+PER_CONFIG = (("tiny", {}, "37 KB of KV per decode: bound by launch and fixed cost, not by HBM"),
+              ("qwen3-4b-decode", {}, None), ("qwen3-4b-decode", {"h": 1}, "h = 1: no rotation (naive INT4)"),
+              ("async-refill", {}, None), ("async-refill", {"values": "bf16"}, "K-INT4 / V-BF16: bf16 values"),
+              ("long-context", {}, None), ("long-context", {"h": 1}, "h = 1: no rotation (naive INT4)"))
 
 
 def parse():
@@ -41,34 +56,47 @@ def parse():
                     help="timed steps (default 2000; 64 for the growing 36-layer workload)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["kv4", "reference"], default="kv4")
-    ap.add_argument("--workload", default="qwen3-4b-decode")
+    ap.add_argument("--workload", default="qwen3-8b-loop")
     ap.add_argument("--h", type=int, default=None, help="Hadamard block of the 36-layer workload (32, 64, 128)")
     ap.add_argument("--sinks", type=int, default=None, help="override s, the INT8 sink positions")
     ap.add_argument("--recent", type=int, default=None,
                     help="override w, the INT8 recent window (-1: every position, i.e. all-INT8 KV8)")
+    ap.add_argument("--values", choices=["int4", "bf16"], default="int4",
+                    help="value storage: INT4 (KV4) or bf16 (the K-INT4 / V-BF16 variant)")
     ap.add_argument("--no-bf16", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-overlap", action="store_true",
                     help="decode waits for the append before building its schedule (kv4_set_decode_overlap 0)")
-    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--e2e-steps", type=int, default=None, help="default 200 (20 for the 36-layer workload)")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the one-layer workloads beside the line")
+    ap.add_argument("--per-config-steps", type=int, default=300)
     ap.add_argument("--soak-s", type=float, default=1.5, help="untimed identical steps sampled for clocks")
     args = ap.parse_args()
     if args.steps is None:
         args.steps = 64 if args.workload == "qwen3-8b-loop" else 2000
+    if args.e2e_steps is None:
+        args.e2e_steps = 20 if args.workload == "qwen3-8b-loop" else 200
     return args
 
 
 def make_wl(args):
     sys.path.insert(0, ROOT)
+    import dataclasses
     from int4_kv_cache_append_b200 import workload as W
     fn = W.WORKLOADS[args.workload]
     h = getattr(args, "h", None)
-    wl = fn(h=h) if h is not None else fn()
+    if h is not None and args.workload == "qwen3-8b-loop":
+        wl = fn(h=h)
+    else:
+        wl = fn()
+        if h is not None and h != wl.h:
+            wl = dataclasses.replace(wl, h=h, name=f"{wl.name}-h{h}")
+    if getattr(args, "values", "int4") == "bf16":
+        wl = dataclasses.replace(wl, value_format=1, name=f"{wl.name}-vbf16")
     # sink / recent budgets (KV4-RL "Main Findings": s/w sweep; KV8 = every position in INT8)
     s, w = getattr(args, "sinks", None), getattr(args, "recent", None)
     if s is not None or w is not None:
-        import dataclasses
         s = wl.s if s is None else s
         w = wl.w if w is None else (int(wl.max_lens.max()) if w < 0 else w)
         wl = dataclasses.replace(wl, s=s, w=w, name=f"{wl.name}-s{s}-w{w}")
@@ -204,7 +232,9 @@ def barrier(world: int):
 # ----------------------------------------------------------------------------- CPU oracle leg
 
 def oracle_sample_setup(wl, nseq: int):
-    """Host cache of the first nseq sequences, filled up to L-1 (untimed), plus the step inputs."""
+    """Host cache of the first nseq sequences, filled up to L-1 (untimed), plus the step inputs.
+    Returns step(nthreads) (one layer call: append of one token per sequence, then the decode),
+    its two halves append() and decode(nthreads), and the sample's lengths."""
     sys.path.insert(0, ROOT)
     from oracle import oracle as O
     from int4_kv_cache_append_b200 import workload as W
@@ -228,31 +258,49 @@ def oracle_sample_setup(wl, nseq: int):
     qd = O.BF16 if wl.q_dtype == W.BF16 else O.F32
     pt = np.ascontiguousarray(wl.page_table[:nseq])
 
-    def step(nthreads):
+    def append():
         O.append(cfg, pool, side, K1, V1, bs, ps, lens, pt, kd, vd)
+
+    def decode(nthreads):
         O.decode(cfg, pool, side, q, pt, lens, q_dtype=qd, nthreads=nthreads)
 
-    return step, lens
+    def step(nthreads):
+        append()
+        decode(nthreads)
+
+    return step, append, decode, lens
 
 
-def cpu_baseline(wl, nseq: int = 16, min_seconds: float = 10.0, per_step: int = 1):
-    """The oracle's append + decode of one layer per step on a sample of sequences; a step of
-    per_step layers costs per_step such steps (the layers are identical in shape)."""
-    step, lens = oracle_sample_setup(wl, nseq)
-    cores = os.cpu_count() or 1
-    step(cores)  # warm
+def _time_reps(fn, min_seconds: float, max_reps: int = 5000):
+    fn()  # warm
     reps, t0 = 0, time.perf_counter()
     while True:
-        step(cores)
+        fn()
         reps += 1
         el = time.perf_counter() - t0
-        if el >= min_seconds or reps >= 5000:
-            break
-    per = f", one layer timed, rate divided by the step's {per_step} layers" if per_step > 1 else ""
+        if el >= min_seconds or reps >= max_reps:
+            return reps, el
+
+
+def cpu_baseline(wl, nseq: int = SAMPLE_SEQS, min_seconds: float = 8.0, per_step: int = 1):
+    """The oracle's append + decode of one layer per step on a sample of sequences, on all host
+    cores (OpenMP over (sequence, KV head) in the decode) and on one thread; the append (one
+    thread) and the decode are also timed alone.  A step of per_step layers costs per_step such
+    layer-steps (the layers are identical in shape)."""
+    step, append, decode, lens = oracle_sample_setup(wl, nseq)
+    cores = os.cpu_count() or 1
+    reps, el = _time_reps(lambda: step(cores), min_seconds)
+    reps1, el1 = _time_reps(lambda: step(1), min_seconds)
+    repa, ela = _time_reps(append, min(2.0, min_seconds))
+    repd, eld = _time_reps(lambda: decode(cores), min(4.0, min_seconds))
+    per = f"; rate divided by the step's {per_step} layers" if per_step > 1 else ""
     return {"value": nseq * reps / el / per_step, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "single_thread": {"value": nseq * reps1 / el1 / per_step, "unit": UNIT, "cores": 1},
+            "append_ms_per_layer": round(1e3 * ela / repa, 3), "decode_ms_per_layer": round(1e3 * eld / repd, 3),
             "sample": f"first {nseq} of {wl.B} sequences (lengths {int(lens.min())}..{int(lens.max())}), "
-                      f"append 1 token + decode per layer, fp64 C oracle with OpenMP over (sequence, KV head), "
-                      f"{reps} layer-steps in {el:.1f} s{per}"}
+                      f"one layer call (append 1 token per sequence + decode), fp64 C oracle, OpenMP over "
+                      f"(sequence, KV head) in the decode; {reps} layer calls in {el:.1f} s on {cores} threads, "
+                      f"{reps1} in {el1:.1f} s on one{per}"}
 
 
 def run_reference(args, world, rank):
@@ -261,8 +309,8 @@ def run_reference(args, world, rank):
     sys.path.insert(0, ROOT)
     wl = make_wl(args)
     per_step = step_shape(wl)[0]
-    nseq = min(4, wl.B)
-    step, lens = oracle_sample_setup(wl, nseq)
+    nseq = min(SAMPLE_SEQS, wl.B)
+    step, _, _, lens = oracle_sample_setup(wl, nseq)
     cores = os.cpu_count() or 1
     for _ in range(args.warmup):
         step(cores)
@@ -272,12 +320,13 @@ def run_reference(args, world, rank):
     el = time.perf_counter() - t0
     value = nseq * args.steps / el / per_step
     sample = (f"each step: first {nseq} of {wl.B} sequences (lengths {int(lens.min())}..{int(lens.max())}), "
-              f"append 1 token + decode of one layer, fp64 C oracle, OpenMP over (sequence, KV head)"
+              f"one layer call (append 1 token per sequence + decode), fp64 C oracle, OpenMP over "
+              f"(sequence, KV head) in the decode; the same sample as the kv4 line's cpu_baseline"
               + (f"; rate divided by the step's {per_step} layers" if per_step > 1 else ""))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps * per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "B_sampled": nseq, "parallelism": "host cores"},
+            "config": {"workload": wl.name, "B_sampled": nseq, "parallelism": "host cores", "inputs": INPUTS},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     return line
@@ -297,25 +346,27 @@ def step_shape(wl):
     return 1, LAYERS, grow
 
 
-def run_kv4(args, world, rank, local):
+def run_kv4(args, world, rank, local, wl=None, light=False):
+    """The bench line of one workload.  light: a workload measured beside the line (per_config):
+    args.per_config_steps steps after 5 warm-up steps, no e2e leg and no CPU baseline."""
     import torch
     sys.path.insert(0, ROOT)
     from int4_kv_cache_append_b200 import harness as H, kv4
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    wl = make_wl(args)
+    wl = make_wl(args) if wl is None else wl
     B = wl.B
     lens0 = wl.lens.astype(np.int32)
     per_step, resident, grow = step_shape(wl)
-    steps, warmup = args.steps, args.warmup
+    steps, warmup = (args.per_config_steps, 5) if light else (args.steps, args.warmup)
     if grow and steps > grow:
         raise SystemExit(f"{wl.name}: at most {grow} timed steps (page capacity for growth)")
     maxlen = int(lens0.max()) + grow
     stream = torch.cuda.Stream(dev)
 
     def setup(bf16: bool, layers: int):
-        geo = H.geometry(wl, layers=layers)
+        geo = H.geometry(wl, layers=layers, value_format=0 if bf16 else wl.value_format)
         cache = kv4.BF16Cache(geo, device=dev) if bf16 else kv4.Cache(geo, device=dev)
         for layer in range(layers):
             H.prefill(cache, wl, layer, lens0, upto=lens0 - 1, bf16_pool=bf16)
@@ -479,7 +530,7 @@ def run_kv4(args, world, rank, local):
     kv4.kv4_set_decode_overlap(cache.handle, 0 if args.no_overlap else 1)
     S = Steps(cache, ins, bt, False, resident)
     total_ms, dec_ms, app_ms, launches, clocks, klens = timed(S, steps, warmup, sampler=ClockSampler(uuid),
-                                                               soak_s=args.soak_s)
+                                                               soak_s=0.3 if light else args.soak_s)
     err = kv4.kv4_get_device_error()
     if err:
         raise RuntimeError(f"device error bits {err:#x} during the benchmark")
@@ -513,7 +564,7 @@ def run_kv4(args, world, rank, local):
     # step overlap the kernels of the previous one.  The serial form (one stream) is reported
     # beside it.
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and not light:
         nl = per_step  # layer calls per step
         nsets = nl if per_step > 1 else 1
         parts = []  # (host tensor, offset) of the static inputs
@@ -639,17 +690,19 @@ def run_kv4(args, world, rank, local):
         torch.cuda.empty_cache()
 
     cpu = None
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, nseq=4 if per_step > 1 else 16, per_step=per_step)
+    if world == 1 and rank == 0 and not args.no_cpu_baseline and not light:
+        cpu = cpu_baseline(wl, nseq=min(SAMPLE_SEQS, wl.B), per_step=per_step)
 
     resident_gb = resident * kv_bytes / 1e9
     line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": steps,
             "warmup": warmup, "ms_per_step": round(total_ms / steps, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": wl.name, "B_per_gpu": B, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": wl.D, "P": wl.P,
+            "config": {"workload": wl.name, "inputs": INPUTS, "B_per_gpu": B, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": wl.D, "P": wl.P,
                        "s": wl.s, "w": wl.w, "h": wl.h, "len_mean": round(float(lens0.mean()), 1),
                        "len_max": int(lens0.max()), "layers_per_step": per_step,
-                       "growth_per_step": 1 if grow else 0, "kv_dtype": "int4 pages + int8 side cache",
+                       "growth_per_step": 1 if grow else 0,
+                       "kv_dtype": ("int4 K + bf16 V pages, int8 K + bf16 V side cache" if wl.value_format
+                                    else "int4 pages + int8 side cache"),
                        "compute": "QK^T int8 MMA (exact int32), PV f16 MMA with f32 accumulate, f32 softmax",
                        "l2": f"inputs larger than L2: {resident} resident layers cycled, {resident_gb:.2f} GB of KV "
                              f"between reuses",
@@ -661,6 +714,22 @@ def run_kv4(args, world, rank, local):
             "roofline": roof, "hbm_frac_of_spec_8TBps": round(spec_frac, 4), "gpu_launches": int(launches),
             "clocks": clocks, "e2e": e2e, "bf16_kv": bf, "cpu_baseline": cpu}
     return line if rank == 0 else None
+
+
+def per_config_record(line: dict, note: str | None) -> dict:
+    """The figures of a one-layer workload's line that go into the default line's per_config."""
+    r, b, c = line["roofline"], line["bf16_kv"], line["config"]
+    rec = {"decode_ms": r["decode_ms"], "bytes_per_launch": r["bytes_per_launch"], "achieved_GBps": r["achieved"],
+           "frac": r["frac"], "peak": r["peak"], "frac_of_spec_8TBps": line["hbm_frac_of_spec_8TBps"],
+           "append_ms": c["append_ms"], "ms_per_step": line["ms_per_step"], "value": line["value"],
+           "B": c["B_per_gpu"], "len_mean": c["len_mean"], "len_max": c["len_max"], "s": c["s"], "w": c["w"],
+           "h": c["h"], "P": c["P"], "steps": line["steps"], "clocks": line["clocks"]}
+    if b:
+        rec.update({"bf16_decode_ms": b["decode_ms"], "bf16_frac": b["frac"],
+                    "int4_over_bf16_decode": b["int4_speedup_decode"]})
+    if note:
+        rec["note"] = note
+    return rec
 
 
 def main():
@@ -675,6 +744,20 @@ def main():
     world, rank, local = dist_setup("nccl")
     try:
         line = run_kv4(args, world, rank, local)
+        if line is not None and rank == 0 and world == 1 and not args.no_per_config:
+            # the other configurations, one after the other in this process (N = 1 only)
+            import dataclasses
+
+            from int4_kv_cache_append_b200 import workload as W
+            per = {}
+            for name, over, note in PER_CONFIG:
+                wl = W.WORKLOADS[name]()
+                if "h" in over:
+                    wl = dataclasses.replace(wl, h=over["h"], name=f"{wl.name}-h{over['h']}")
+                if over.get("values") == "bf16":
+                    wl = dataclasses.replace(wl, value_format=1, name=f"{wl.name}-vbf16")
+                per[wl.name] = per_config_record(run_kv4(args, world, rank, local, wl=wl, light=True), note)
+            line["per_config"] = per
         if line is not None and rank == 0:
             print(json.dumps(line), flush=True)
     finally:

@@ -75,11 +75,18 @@ typedef enum { KV4_F32 = 0, KV4_BF16 = 1, KV4_F16 = 2 } kv4_dtype;
                                        workspace (left by a decode that stopped early) and
                                        skipped it                                               */
 
+/* Value storage formats (kv4_config.value_format). */
+#define KV4_VALUES_INT4 0  /* values as per-token affine INT4 (INT8 in the side cache): KV4       */
+#define KV4_VALUES_BF16 1  /* values kept in bf16 in the pages and the side cache, keys as in KV4 */
+
 /*
  * Cache geometry.  Supported: head_dim in {64, 128}; Hq/Hkv in {1, 2, 4}; page_size a
  * multiple of 16; hadamard_block a power of two dividing head_dim; num_sinks >= 0,
  * recent_window >= 0.  One page table (int32 [max_seqs][stride]) is shared by all layers, as in
- * vLLM; page ids index a per-layer pool of max_pages pages.
+ * vLLM; page ids index a per-layer pool of max_pages pages.  value_format selects the value
+ * storage (KV4-RL, "Main Findings", compares KV4, KV8 and BF16 KV budgets; the K-INT4 / V-BF16
+ * variant keeps the INT4 keys and leaves the values unquantised): KV4_VALUES_INT4 (0, the
+ * default of a zeroed struct) or KV4_VALUES_BF16 (1).
  */
 typedef struct {
   int num_layers;
@@ -92,6 +99,7 @@ typedef struct {
   int hadamard_block;   /* h                                     */
   int max_seqs;         /* sequence slots of the INT8 side cache */
   int max_pages;        /* pages per layer pool                  */
+  int value_format;     /* KV4_VALUES_INT4 or KV4_VALUES_BF16    */
 } kv4_config;
 
 typedef struct kv4_cache kv4_cache;  /* opaque host handle */
@@ -100,8 +108,11 @@ typedef struct kv4_cache kv4_cache;  /* opaque host handle */
  * Byte sizes the caller must allocate (all layers):
  *   page pool:  num_layers * max_pages * Hkv * P * (D + 8)
  *               (per token and KV head: D/2 bytes of K codes + D/2 of V codes + 2x fp16
- *               scale/zero for K and for V; 4 + 32/D bits per element for D = 128 -> 4.25)
+ *               scale/zero for K and for V; 4 + 32/D bits per element for D = 128 -> 4.25,
+ *               the storage KV4-RL, "Methodology in Plain English" paragraph 2, states)
  *   side cache: num_layers * max_seqs * Hkv * ceil((s + w)/16) * 16 * (2D + 4)
+ * With KV4_VALUES_BF16 a position takes D/2 + 4 + 2D bytes in a page (K codes and parameters,
+ * bf16 V) and 3D + 2 in the side cache (INT8 K and its scale, bf16 V).
  * Both must be 16-byte aligned.  Returns KV4_ERR_UNSUPPORTED for geometries outside the list.
  */
 kv4_status kv4_query_sizes(const kv4_config* cfg, size_t* page_pool_bytes, size_t* side_cache_bytes);
@@ -116,7 +127,12 @@ void kv4_cache_destroy(kv4_cache* cache);
  * kv4_append: write T new tokens of one layer.  Fused per (token, KV head): block-Hadamard
  * rotation of K, per-token affine INT4 quantisation of rotated K and of V, nibble packing into
  * the token's page slot (page page_table[seq][pos / P], slot pos % P), and INT8 routing of
- * sink/recent positions into the side cache.
+ * sink/recent positions into the side cache.  The method of KV4-RL (ai.info summary),
+ * "Methodology in Plain English" paragraphs 2-3 (every new K/V vector quantised on the fly to one
+ * affine INT4 group with fp16 scale and offset, keys in a Hadamard-rotated basis, an INT8 side
+ * cache for the first s and the most recent w positions), and of SAW-INT4 (gist.science
+ * summary), section 2 (block-diagonal rotation in blocks of h, fused with quantisation in one
+ * kernel).
  *   K, V         device [T][Hkv][D] of k_dtype / v_dtype (KV4_F32 or KV4_BF16), contiguous
  *   seq_slot     device int32 [T]: sequence slot of each token, in [0, max_seqs)
  *   pos          device int32 [T]: position of each token in its sequence
@@ -124,7 +140,8 @@ void kv4_cache_destroy(kv4_cache* cache);
  *                positions are "recent"); positions of one sequence must be distinct in a call
  *   page_table   device int32 [max_seqs][stride]
  * Device-side: a page id outside [0, max_pages) or pos / P >= stride sets an error bit and the
- * token is skipped.
+ * token is skipped; a vector whose fp16 scale or offset overflows sets KV4_DEVERR_RANGE (stored
+ * with zero codes).  With KV4_VALUES_BF16 the values are stored as bf16 (nearest even) instead.
  */
 kv4_status kv4_append(kv4_cache* cache, int layer, int T, const void* K, kv4_dtype k_dtype,
                       const void* V, kv4_dtype v_dtype, const int32_t* seq_slot, const int32_t* pos,
@@ -137,24 +154,31 @@ kv4_status kv4_decode_workspace_bytes(const kv4_cache* cache, int B, size_t* byt
  * kv4_decode_attn: one decode step of attention for B sequences (row b of the batch is side-cache
  * slot b) at lengths lens[b] (the just-appended token included).  Rotates each query once
  * (H/h), streams the packed INT4 pages of [s, max(s, L-w)) and the INT8 rows of the sink and
- * recent regions, and merges per-region / per-split softmax statistics.
+ * recent regions, and merges per-region / per-split softmax statistics.  This is the decode of
+ * KV4-RL (ai.info summary), "Methodology in Plain English" paragraphs 2-3 and "Key
+ * Contributions" item 4: packed codes read directly, scale and offset applied after the
+ * dot-product reduction, queries rotated to the keys' basis, sink and recent regions from the
+ * INT8 side cache attended as disjoint regions merged with their softmax statistics.
  *   q            device [B][Hq][D] of q_dtype (KV4_F32, KV4_BF16 or KV4_F16)
  *   page_table   device int32 [>= B][stride];  lens device int32 [B] (0 gives out = 0, lse = -inf)
  *   max_len_hint host upper bound of lens (0 = unknown); only sizes the grid
  *   out          device fp32 [B][Hq][D];  lse device fp32 [B][Hq] or NULL
  *   workspace    device scratch of at least kv4_decode_workspace_bytes(B) bytes, 16-byte aligned;
- *                its contents need no initialisation and are dead after the call.
+ *                its contents need no initialisation and are dead after the call.  Calls that
+ *                overlap on the GPU must not share a workspace.
  * Two launches on the stream: the split-K pass (one partial (o, m, l) per warp and segment it
- * touches; a (sequence, KV head) covered by a single partial is written directly), then the LSE
- * merge of the partials of every other (sequence, KV head).
+ * touches; a warp that holds a whole INT8 region and the start of the INT4 region of a
+ * (sequence, KV head) runs one softmax across both; a (sequence, KV head) covered by a single
+ * partial is written directly), then the LSE merge of the partials of every other (sequence,
+ * KV head).
  */
 kv4_status kv4_decode_attn(kv4_cache* cache, int layer, int B, const void* q, kv4_dtype q_dtype,
                            const int32_t* page_table, int stride, const int32_t* lens, int max_len_hint,
                            float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
- * kv4_set_rotation_signs: randomised-sign Hadamard rotation for this cache (a precision variant;
- * default: none).  Bit d of sign_bits (host array of ceil(head_dim / 32) words, bit d % 32 of word
+ * kv4_set_rotation_signs: randomised-sign Hadamard rotation for this cache (a precision variant of
+ * SAW-INT4's block-diagonal rotation, gist.science summary section 2; default: none).  Bit d of sign_bits (host array of ceil(head_dim / 32) words, bit d % 32 of word
  * d / 32) negates key dimension d before the block Hadamard at append, and query dimension d
  * before the query rotation at decode, so the rotation is H diag(s) with s in {+1, -1}; the
  * attention is unchanged in exact arithmetic.  NULL clears it.  The signs are part of the stored
@@ -164,8 +188,9 @@ kv4_status kv4_decode_attn(kv4_cache* cache, int layer, int B, const void* q, kv
 kv4_status kv4_set_rotation_signs(kv4_cache* cache, const uint32_t* sign_bits);
 
 /*
- * kv4_set_value_rotation: store values in the keys' rotated basis too (a precision variant;
- * default 0).  With 1 the append applies H diag(s) to V before quantising (INT4 and INT8 copies),
+ * kv4_set_value_rotation: store values in the keys' rotated basis too (a precision variant of the
+ * rotation of KV4-RL, "Methodology in Plain English" paragraph 2, which rotates keys only;
+ * default 0).  Not available with KV4_VALUES_BF16 (returns KV4_ERR_INVALID_ARG).  With 1 the append applies H diag(s) to V before quantising (INT4 and INT8 copies),
  * and the decode's merge returns every output to the original basis, out = diag(s) H o / h.  This
  * is part of the stored format: set it before the first append and keep it.  Returns
  * KV4_ERR_INVALID_ARG for a NULL or BF16 cache.
@@ -198,7 +223,8 @@ kv4_status kv4_set_decode_overlap(kv4_cache* cache, int enable);
 kv4_status kv4_debug_force_wait_timeout(kv4_cache* cache, int enable);
 
 /*
- * BF16-KV baseline with the same page table and conventions, no quantisation and no rotation:
+ * BF16-KV baseline (KV4-RL, "Main Findings", quotes its speed-ups against BF16 KV) with the same
+ * page table and conventions, no quantisation and no rotation:
  * a page holds Hkv head blocks of P * 4D bytes (bf16 K and V).  Used to measure the INT4
  * speed-up on the same GPU.  kv4_bf16_query_sizes returns num_layers * max_pages * Hkv * P * 4D.
  */

@@ -81,14 +81,16 @@ kv4_status check_config(const kv4_config* c) {
   if (c->page_size % 16) return KV4_ERR_UNSUPPORTED;
   if (!pow2(c->hadamard_block) || c->head_dim % c->hadamard_block) return KV4_ERR_INVALID_ARG;
   if (c->num_sinks > (1 << 20) || c->recent_window > (1 << 20)) return KV4_ERR_UNSUPPORTED;
+  if (c->value_format != KV4_VALUES_INT4 && c->value_format != KV4_VALUES_BF16) return KV4_ERR_INVALID_ARG;
   return KV4_OK;
 }
 
 void sizes(const kv4_config* c, size_t* page_bytes, size_t* side_slot, int* nt8) {
   const size_t D = static_cast<size_t>(c->head_dim);
-  *page_bytes = static_cast<size_t>(c->num_kv_heads) * static_cast<size_t>(c->page_size) * (D + 8);
+  const bool vbf = c->value_format == KV4_VALUES_BF16;
+  *page_bytes = static_cast<size_t>(c->num_kv_heads) * static_cast<size_t>(c->page_size) * (vbf ? D / 2 + 4 + 2 * D : D + 8);
   *nt8 = (c->num_sinks + c->recent_window + 15) / 16;
-  *side_slot = static_cast<size_t>(c->num_kv_heads) * static_cast<size_t>(*nt8) * 16u * (2 * D + 4);
+  *side_slot = static_cast<size_t>(c->num_kv_heads) * static_cast<size_t>(*nt8) * 16u * (vbf ? 3 * D + 2 : 2 * D + 4);
 }
 
 kv4_status dtype_ok_kv(kv4_dtype d) { return (d == KV4_F32 || d == KV4_BF16) ? KV4_OK : KV4_ERR_INVALID_ARG; }
@@ -151,6 +153,7 @@ kv4_status append_common(kv4_cache* c, int fmt, int layer, int T, const void* K,
   a.side_slot_bytes = c->side_slot_bytes;
   for (int i = 0; i < 4; ++i) a.signs[i] = fmt == FMT_INT4 ? c->signs[i] : 0u;
   a.rotate_v = fmt == FMT_INT4 ? c->rotate_v : 0;
+  a.vbf = (fmt == FMT_INT4 && c->cfg.value_format == KV4_VALUES_BF16) ? 1 : 0;
   a.err = err;
   const cudaError_t e = fmt == FMT_INT4 ? kv4::launch_append_int4(a, c->cfg.head_dim, static_cast<cudaStream_t>(stream))
                                         : kv4::launch_append_bf16(a, c->cfg.head_dim, static_cast<cudaStream_t>(stream));
@@ -219,6 +222,7 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
   a.early = (fmt == FMT_INT4 && c->overlap) ? 1 : 0;
   for (int i = 0; i < 4; ++i) a.signs[i] = c->signs[i];
   a.rotate_v = fmt == FMT_INT4 ? c->rotate_v : 0;
+  a.vbf = (fmt == FMT_INT4 && c->cfg.value_format == KV4_VALUES_BF16) ? 1 : 0;
   const int tpp = c->cfg.page_size / 16;
   a.tp_shift = pow2(tpp) ? __builtin_ctz(static_cast<unsigned>(tpp)) : -1;
   // The wait-limit test runs every warp's first wait out after 1 ms; the normal limit is 2 s.
@@ -318,6 +322,7 @@ kv4_status kv4_set_rotation_signs(kv4_cache* cache, const uint32_t* sign_bits) {
 
 kv4_status kv4_set_value_rotation(kv4_cache* cache, int enable) {
   if (!cache || cache->format != FMT_INT4) return KV4_ERR_INVALID_ARG;
+  if (enable && cache->cfg.value_format == KV4_VALUES_BF16) return KV4_ERR_INVALID_ARG;
   cache->rotate_v = enable ? 1 : 0;
   return KV4_OK;
 }
@@ -364,6 +369,7 @@ kv4_status kv4_bf16_cache_init(const kv4_config* cfg, void* page_pool, kv4_cache
   kv4_cache* c = new (std::nothrow) kv4_cache();
   if (!c) return KV4_ERR_INVALID_ARG;
   c->cfg = *cfg;
+  c->cfg.value_format = KV4_VALUES_INT4;  // the baseline pool stores K and V in bf16 whatever the field says
   c->format = FMT_BF16;
   c->pool = static_cast<uint8_t*>(page_pool);
   c->side = nullptr;

@@ -139,9 +139,22 @@ __device__ __forceinline__ uint32_t quant_int8(const float (&x)[4], bool act, ui
   return packed;
 }
 
-template <int D, typename KT, typename VT>
+// Offset of value element e of row r in a 16-row bf16 V block (the BF16 pool's V order).
+template <int D>
+__device__ __forceinline__ int vbf_offset(int r, int e) {
+  using Gm = Geo<D>;
+  const int p = r >> 1, half = p >> 2, pl = p & 3;
+  const int gq = e / Gm::DG, m = e % Gm::DG, uu = m >> 2;
+  return ((half * 8 + gq) * 4 + pl) * (D / 2) + ((uu ^ bf16_swz(D, pl, gq)) << 4) + (m & 3) * 4 + (r & 1) * 2;
+}
+
+// VB: values kept as bf16 (KV4_VALUES_BF16) instead of INT4 / INT8.
+template <int D, typename KT, typename VT, bool VB>
 __global__ void __launch_bounds__(kAppendThreads) append_int4_kernel(AppendArgs a) {
   using Gm = Geo<D>;
+  constexpr int PB = VB ? D / 2 + 4 + 2 * D : D + 8;  // bytes of one position of one head in a page
+  constexpr int KPO = VB ? 8 * D : 16 * D;             // K parameters in a page tile
+  constexpr int T8 = VB ? Gm::T8V : Gm::T8B;           // side tile
   pdl_launch_dependents();  // the decode kernel that follows may start its launch now
   const int gw = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
@@ -183,12 +196,13 @@ __global__ void __launch_bounds__(kAppendThreads) append_int4_kernel(AppendArgs 
   }
 
   const int pp = pos % a.P, r = pp & 15;
-  uint8_t* tile = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(g) * a.P * (D + 8) +
-                  static_cast<size_t>(pp >> 4) * Gm::T4B;
-  uint32_t ksz, vsz;
-  bool kbad, vbad;
+  uint8_t* tile = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(g) * a.P * PB +
+                  static_cast<size_t>(pp >> 4) * (16 * PB);
+  uint32_t ksz, vsz = 0;
+  bool kbad, vbad = false;
   const uint32_t kc = quant_int4(k, act, &ksz, &kbad);
-  const uint32_t vc = quant_int4(v, act, &vsz, &vbad);
+  uint32_t vc = 0;
+  if constexpr (!VB) vc = quant_int4(v, act, &vsz, &vbad);
   if (lane == 0 && (kbad || vbad)) atomicOr(a.err, KV4_DEVERR_RANGE);
   if (act) {
     // K: row r shares pair-row r % 8 with row r ^ 8 (low nibbles rows 0-7, high nibbles rows
@@ -206,14 +220,21 @@ __global__ void __launch_bounds__(kAppendThreads) append_int4_kernel(AppendArgs 
     atomicOr(w0, (e0 << sh) | (e2 << (sh + 8)));
     atomicAnd(w0 + 1, clear);
     atomicOr(w0 + 1, (e1 << sh) | (e3 << (sh + 8)));
-    // V: 16-bit chunk of quad Q = l.
-    const int Q = lane, p = r >> 1, half = p >> 2, pl = p & 3;
-    const int off = ((half * 8 + Q / Gm::WPC) * 4 + pl) * Gm::CH + 4 * (Q % Gm::WPC) + 2 * (r & 1);
-    *reinterpret_cast<uint16_t*>(tile + 8 * D + off) = static_cast<uint16_t>(vc);
+    if constexpr (VB) {
+      // V as bf16 (nearest even), elements 4l..4l+3
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<__nv_bfloat16*>(tile + Gm::VBO + vbf_offset<D>(r, 4 * lane + i)) = __float2bfloat16_rn(v[i]);
+    } else {
+      // V: 16-bit chunk of quad Q = l.
+      const int Q = lane, p = r >> 1, half = p >> 2, pl = p & 3;
+      const int off = ((half * 8 + Q / Gm::WPC) * 4 + pl) * Gm::CH + 4 * (Q % Gm::WPC) + 2 * (r & 1);
+      *reinterpret_cast<uint16_t*>(tile + 8 * D + off) = static_cast<uint16_t>(vc);
+    }
   }
   if (lane == 0) {
-    *reinterpret_cast<uint32_t*>(tile + 16 * D + 4 * r) = ksz;
-    *reinterpret_cast<uint32_t*>(tile + 16 * D + 64 + 4 * r) = vsz;
+    *reinterpret_cast<uint32_t*>(tile + KPO + 4 * r) = ksz;
+    if constexpr (!VB) *reinterpret_cast<uint32_t*>(tile + 16 * D + 64 + 4 * r) = vsz;
   }
 
   // INT8 side cache: sinks and the recent window (warp-uniform decision).
@@ -224,13 +245,25 @@ __global__ void __launch_bounds__(kAppendThreads) append_int4_kernel(AppendArgs 
     row = a.s + pos % a.w;
   if (row < 0) return;
   uint8_t* t8 = a.side + static_cast<size_t>(b) * a.side_slot_bytes +
-                static_cast<size_t>(g) * a.nt8 * Gm::T8B + static_cast<size_t>(row >> 4) * Gm::T8B;
+                static_cast<size_t>(g) * a.nt8 * T8 + static_cast<size_t>(row >> 4) * T8;
   const int r8 = row & 15;
-  uint16_t ks, vs;
-  bool kbad8, vbad8;
+  uint16_t ks, vs = 0;
+  bool kbad8, vbad8 = false;
   const uint32_t k8 = quant_int8(k, act, &ks, &kbad8);
-  const uint32_t v8 = quant_int8(v, act, &vs, &vbad8);
+  uint32_t v8 = 0;
+  if constexpr (!VB) v8 = quant_int8(v, act, &vs, &vbad8);
   if (lane == 0 && (kbad8 || vbad8)) atomicOr(a.err, KV4_DEVERR_RANGE);
+  if constexpr (VB) {
+    if (act) {
+      const int e = 4 * lane;
+      *reinterpret_cast<uint32_t*>(t8 + r8 * D + 16 * ((e >> 4) ^ (r8 & 1)) + (e & 15)) = k8;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<__nv_bfloat16*>(t8 + Gm::VB8O + vbf_offset<D>(r8, e + i)) = __float2bfloat16_rn(v[i]);
+    }
+    if (lane == 0) *reinterpret_cast<uint16_t*>(t8 + 16 * D + 2 * r8) = ks;
+    return;
+  }
   if (act) {
     const int e = 4 * lane;
     *reinterpret_cast<uint32_t*>(t8 + r8 * D + 16 * ((e >> 4) ^ (r8 & 1)) + (e & 15)) = k8;
@@ -295,6 +328,11 @@ __global__ void __launch_bounds__(kAppendThreads) append_bf16_kernel(AppendArgs 
 }
 
 #define KV4_APPEND_LAUNCH(KERN, KT, VT) KERN<D, KT, VT><<<grid, block, 0, st>>>(a)
+#define KV4_APPEND_LAUNCH4(KT, VT)                                   \
+  do {                                                               \
+    if (a.vbf) append_int4_kernel<D, KT, VT, true><<<grid, block, 0, st>>>(a); \
+    else append_int4_kernel<D, KT, VT, false><<<grid, block, 0, st>>>(a);      \
+  } while (0)
 
 template <int D, bool BF16_POOL>
 cudaError_t dispatch_types(const AppendArgs& a, cudaStream_t st) {
@@ -310,15 +348,16 @@ cudaError_t dispatch_types(const AppendArgs& a, cudaStream_t st) {
     else if (vf) KV4_APPEND_LAUNCH(append_bf16_kernel, __nv_bfloat16, float);
     else KV4_APPEND_LAUNCH(append_bf16_kernel, __nv_bfloat16, __nv_bfloat16);
   } else {
-    if (kf && vf) KV4_APPEND_LAUNCH(append_int4_kernel, float, float);
-    else if (kf) KV4_APPEND_LAUNCH(append_int4_kernel, float, __nv_bfloat16);
-    else if (vf) KV4_APPEND_LAUNCH(append_int4_kernel, __nv_bfloat16, float);
-    else KV4_APPEND_LAUNCH(append_int4_kernel, __nv_bfloat16, __nv_bfloat16);
+    if (kf && vf) KV4_APPEND_LAUNCH4(float, float);
+    else if (kf) KV4_APPEND_LAUNCH4(float, __nv_bfloat16);
+    else if (vf) KV4_APPEND_LAUNCH4(__nv_bfloat16, float);
+    else KV4_APPEND_LAUNCH4(__nv_bfloat16, __nv_bfloat16);
   }
   return cudaGetLastError();
 }
 
 #undef KV4_APPEND_LAUNCH
+#undef KV4_APPEND_LAUNCH4
 
 }  // namespace
 

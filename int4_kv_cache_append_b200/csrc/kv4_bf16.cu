@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_bf16_kernel(const Decod
       const uint8_t* src = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(c.g) * a.P * 4 * D +
                            static_cast<size_t>((c.i * 16 - lp * a.P) >> 4) * Gm::TBF;
       mbar_arrive_expect_tx(&bars[st], Gm::TBF);
-      bulk_g2s(sm.ring[warp][st], src, Gm::TBF, &bars[st]);
+      bulk_g2s_hint(sm.ring[warp][st], src, Gm::TBF, &bars[st], l2_policy_evict_first());
     } else {
       atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
       mbar_arrive_expect_tx(&bars[st], 0);

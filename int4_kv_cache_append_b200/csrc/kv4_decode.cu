@@ -48,10 +48,9 @@ constexpr unsigned FULL = 0xffffffffu;
 constexpr int kWarps = 16;
 constexpr int kCtasPerSm = 1;
 constexpr int kStages = 2;
-constexpr int kChunk = 16;  // slots per descriptor fill
+constexpr int kChunk = 16;  // slots per descriptor fill (a fill of 32 measured slower on short batches)
 constexpr int kRing = 32;   // descriptor ring (two chunks)
 constexpr int kLensRegs = 8;  // sequence lengths held in registers by the schedule (B <= 256)
-constexpr int kMergeWideItems = 1184;  // up to this many (b, j), 4 merge warps each
 constexpr float kNegInf = -__builtin_huge_valf();
 
 // ------------------------------------------------------------------ schedule
@@ -96,11 +95,17 @@ __device__ __forceinline__ SegInfo seg_info(int L, int s, int w, int nt8, int sm
   return r;
 }
 
-__device__ __forceinline__ u32 head_cost(const SegInfo& si) { return 2u * si.n8 + si.n4; }
+// Cost units of an INT8 side tile: 2 with INT4 values (its bytes are about twice an INT4 tile's),
+// 1 with bf16 values (a side tile and a page tile then move about the same bytes).
+template <bool VB>
+constexpr u32 kU8 = VB ? 1u : 2u;
 
-template <bool T8>
+template <bool VB>
+__device__ __forceinline__ u32 head_cost(const SegInfo& si) { return kU8<VB> * si.n8 + si.n4; }
+
+template <bool T8, bool VB>
 __device__ __forceinline__ u32 seq_cost(const DecodeArgs& a, int cap, int b) {
-  return static_cast<u32>(a.Hkv) * head_cost(seg_info<T8>(clamp_len(a.lens[b], cap), a.s, a.w, a.nt8, a.smw));
+  return static_cast<u32>(a.Hkv) * head_cost<VB>(seg_info<T8>(clamp_len(a.lens[b], cap), a.s, a.w, a.nt8, a.smw));
 }
 
 __device__ __forceinline__ u32 warp_incl_scan(u32 v, int lane) {
@@ -112,24 +117,24 @@ __device__ __forceinline__ u32 warp_incl_scan(u32 v, int lane) {
   return v;
 }
 
-template <bool T8>
+template <bool T8, bool VB>
 __device__ u32 total_cost(const DecodeArgs& a, int cap, int lane) {
   u32 run = 0;
   for (int base = 0; base < a.B; base += 32) {
     const int b = base + lane;
-    const u32 c = b < a.B ? seq_cost<T8>(a, cap, b) : 0u;
+    const u32 c = b < a.B ? seq_cost<T8, VB>(a, cap, b) : 0u;
     run += __shfl_sync(FULL, warp_incl_scan(c, lane), 31);
   }
   return run;
 }
 
 // Sequence containing unit c (c < total); *bstart = first unit of that sequence.
-template <bool T8>
+template <bool T8, bool VB>
 __device__ int find_seq(const DecodeArgs& a, int cap, int lane, u32 c, u32* bstart) {
   u32 run = 0;
   for (int base = 0; base < a.B; base += 32) {
     const int b = base + lane;
-    const u32 cb = b < a.B ? seq_cost<T8>(a, cap, b) : 0u;
+    const u32 cb = b < a.B ? seq_cost<T8, VB>(a, cap, b) : 0u;
     const u32 incl = warp_incl_scan(cb, lane);
     const u32 tot = __shfl_sync(FULL, incl, 31);
     if (c < run + tot) {
@@ -169,7 +174,7 @@ struct Cursor {
 };
 
 // Move forward to the first non-empty segment at or after the current one.
-template <bool T8>
+template <bool T8, bool VB>
 __device__ void settle(const DecodeArgs& a, int cap, Cursor& c) {
   while (true) {
     if (c.b >= a.B) {
@@ -183,7 +188,7 @@ __device__ void settle(const DecodeArgs& a, int cap, Cursor& c) {
       c.seg = 1;
     } else {
       c.seg = 0;
-      c.cs8 += head_cost(c.si);
+      c.cs8 += head_cost<VB>(c.si);
       if (++c.g == a.Hkv) {
         c.g = 0;
         if (++c.b < a.B) c.si = seg_info<T8>(clamp_len(a.lens[c.b], cap), a.s, a.w, a.nt8, a.smw);
@@ -193,32 +198,33 @@ __device__ void settle(const DecodeArgs& a, int cap, Cursor& c) {
 }
 
 // Unit position of the cursor's tile (after settle moved it to another segment).
+template <bool VB>
 __device__ __forceinline__ void recost(Cursor& c) {
-  c.cost = c.seg == 0 ? c.cs8 + 2u * c.i : c.cs8 + 2u * c.si.n8 + c.i;
+  c.cost = c.seg == 0 ? c.cs8 + kU8<VB> * c.i : c.cs8 + kU8<VB> * c.si.n8 + c.i;
 }
 
 // First tile whose first unit is >= c0, in sequence b (first unit bstart, raw length Lraw).
-template <bool T8>
+template <bool T8, bool VB>
 __device__ Cursor cursor_at(const DecodeArgs& a, int cap, int b, u32 bstart, u32 c0, int Lraw) {
   Cursor c;
   c.b = b;
   c.valid = b < a.B;
   if (!c.valid) return c;
   c.si = seg_info<T8>(clamp_len(Lraw, cap), a.s, a.w, a.nt8, a.smw);
-  const u32 ch = head_cost(c.si);
+  const u32 ch = head_cost<VB>(c.si);
   const u32 off = c0 - bstart;
   c.g = static_cast<int>(off / ch);
   c.cs8 = bstart + static_cast<u32>(c.g) * ch;
   const u32 r = off - static_cast<u32>(c.g) * ch;
-  if (r < 2u * c.si.n8) {
+  if (r < kU8<VB> * c.si.n8) {
     c.seg = 0;
-    c.i = static_cast<int>((r + 1) >> 1);
+    c.i = static_cast<int>(VB ? r : (r + 1) >> 1);
   } else {
     c.seg = 1;
-    c.i = static_cast<int>(r - 2u * c.si.n8);
+    c.i = static_cast<int>(r - kU8<VB> * c.si.n8);
   }
-  settle<T8>(a, cap, c);
-  if (c.valid) recost(c);
+  settle<T8, VB>(a, cap, c);
+  if (c.valid) recost<VB>(c);
   return c;
 }
 
@@ -235,13 +241,18 @@ __device__ __forceinline__ void tile_page(const DecodeArgs& a, int ti, int* lp, 
 
 // ------------------------------------------------------------------ per-warp shared memory
 
-template <int D>
+// Stage of the shared-memory ring: two INT4 page tiles or one INT8 side tile; with bf16 values
+// one page tile or one side tile (the larger).
+template <int D, bool VB>
+constexpr int kStageBytes = VB ? Geo<D>::T8V : 2 * Geo<D>::T4B;
+
+template <int D, bool VB>
 struct Smem {
-  uint8_t ring[kWarps][kStages][2 * Geo<D>::T4B];  // stage = two tile blocks
-  unsigned long long src[kWarps][kRing][2];          // bulk-copy sources of each slot (0 = none)
-  unsigned int mask[kWarps][kRing];                  // valid rows: tile A bits 0-15, tile B 16-31
-  unsigned int meta[kWarps][kRing];                  // kind | flags | segment index << 8
-  unsigned long long seg[kWarps][kRing];             // segment table: cs8 | seg<<32 | g<<33 | b<<41
+  uint8_t ring[kWarps][kStages][kStageBytes<D, VB>];
+  unsigned long long src[kWarps][kRing][2];      // bulk-copy sources of each slot (0 = none)
+  unsigned int mask[kWarps][kRing];              // valid rows: tile A bits 0-15, tile B 16-31
+  unsigned int meta[kWarps][kRing];              // kind | flags | segment index << 8
+  unsigned long long seg[kWarps][kRing];         // segment table: cs8 | seg<<32 | g<<33 | b<<41
   Cursor cur[kWarps];                                // descriptor cursor between fills
   unsigned segno[kWarps];                            // segments entered so far
   uint64_t bar[kWarps][kStages];
@@ -294,10 +305,13 @@ __device__ __forceinline__ unsigned side_tile_mask(int i, int L, int s, int w) {
 // written to ring position (base + j) % kRing, plus one segment-table entry per segment entered.
 // `c` is advanced past them; slots past the warp's stream get kind None.  `segno` counts the
 // segments this warp has entered.
-template <int D, bool T8>
+template <int D, bool T8, bool VB>
 __device__ void fill_descriptors(const DecodeArgs& a, int cap, u32 c1, Cursor& c, int lane,
-                                 Smem<D>& sm, int warp, int base, unsigned& segno) {
+                                 Smem<D, VB>& sm, int warp, int base, unsigned& segno) {
   using Gm = Geo<D>;
+  constexpr int TPS = VB ? 1 : 2;                         // page tiles per slot
+  constexpr int T4 = VB ? Gm::T4V : Gm::T4B;              // page tile bytes
+  constexpr int TS = VB ? Gm::T8V : Gm::T8B;              // side tile bytes
   unsigned long long s0 = 0ull, s1 = 0ull;
   unsigned msk = 0u, meta = kKindNone;
   int done = 0;
@@ -307,9 +321,9 @@ __device__ void fill_descriptors(const DecodeArgs& a, int cap, u32 c1, Cursor& c
     int avail_tiles, avail_slots;
     if (c.seg == 1) {
       avail_tiles = static_cast<int>(min(static_cast<u32>(c.n - c.i), c1 - c.cost));
-      avail_slots = (avail_tiles + 1) >> 1;
+      avail_slots = VB ? avail_tiles : (avail_tiles + 1) >> 1;
     } else {
-      avail_tiles = static_cast<int>(min(static_cast<u32>(c.n - c.i), (c1 - c.cost + 1) >> 1));
+      avail_tiles = static_cast<int>(min(static_cast<u32>(c.n - c.i), VB ? c1 - c.cost : (c1 - c.cost + 1) >> 1));
       avail_slots = avail_tiles;
     }
     const int take = min(kChunk - done, avail_slots);
@@ -318,11 +332,11 @@ __device__ void fill_descriptors(const DecodeArgs& a, int cap, u32 c1, Cursor& c
       meta = (sidx << 8) | ((take == avail_slots && u == take - 1) ? kMetaLast : 0u);
       if (c.seg == 1) {
         meta |= kKindInt4;
-        const int t0 = c.i + 2 * u;
-        const int nt = min(2, avail_tiles - 2 * u);
+        const int t0 = c.i + TPS * u;
+        const int nt = min(TPS, avail_tiles - TPS * u);
         if (nt == 2) meta |= kMetaTwo;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
+        for (int j = 0; j < TPS; ++j) {
           if (j < nt) {
             const int ti = c.si.t4a + t0 + j;
             int lp, tin;
@@ -331,8 +345,8 @@ __device__ void fill_descriptors(const DecodeArgs& a, int cap, u32 c1, Cursor& c
             unsigned long long addr = 0ull;
             if (page >= 0 && page < a.max_pages) {
               addr = reinterpret_cast<unsigned long long>(a.pool + static_cast<size_t>(page) * a.page_bytes +
-                                                          static_cast<size_t>(c.g) * a.P * (D + 8) +
-                                                          static_cast<size_t>(tin) * Gm::T4B);
+                                                          static_cast<size_t>(c.g) * (a.P / 16) * T4 +
+                                                          static_cast<size_t>(tin) * T4);
               msk |= range_bits(a.s, c.si.m_end, 16 * ti) << (16 * j);
             } else {
               meta |= kMetaBad;
@@ -344,27 +358,27 @@ __device__ void fill_descriptors(const DecodeArgs& a, int cap, u32 c1, Cursor& c
         meta |= kKindInt8;
         const int ti = c.i + u;
         s0 = reinterpret_cast<unsigned long long>(a.side + static_cast<size_t>(c.b) * a.side_slot_bytes +
-                                                  static_cast<size_t>(c.g) * a.nt8 * Gm::T8B +
-                                                  static_cast<size_t>(ti) * Gm::T8B);
-        s1 = s0 + Gm::H8B;
+                                                  static_cast<size_t>(c.g) * a.nt8 * TS +
+                                                  static_cast<size_t>(ti) * TS);
+        s1 = VB ? 0ull : s0 + Gm::H8B;  // bf16 values: the side tile is one copy
         msk = side_tile_mask(ti, c.si.L, a.s, a.w);
       }
     }
     // advance the cursor past the taken slots; at the end of the segment move to the next one.
     // If the stream limit c1 cut the segment, the next tile starts at or past c1.
     if (c.seg == 1) {
-      const int tiles = min(2 * take, avail_tiles);
+      const int tiles = min(TPS * take, avail_tiles);
       c.i += tiles;
       c.cost += static_cast<u32>(tiles);
     } else {
       c.i += take;
-      c.cost += 2u * take;
+      c.cost += kU8<VB> * take;
     }
     done += take;
     if (c.i >= c.n) {
-      settle<T8>(a, cap, c);
+      settle<T8, VB>(a, cap, c);
       ++segno;
-      if (c.valid) recost(c);
+      if (c.valid) recost<VB>(c);
     }
   }
   if (lane < kChunk) {
@@ -383,15 +397,22 @@ __device__ void fill_descriptors(const DecodeArgs& a, int cap, u32 c1, Cursor& c
 // of odd k is removed from the corresponding output rows when the partial is written.  V stays in
 // normal fp16: the (p * scale) operand is small, and subnormal codes against it lose accuracy in
 // the tensor-core accumulation over long sequences.
+// Written as one lop3 (mask and magic exponent) and one packed fp16 subtraction: the same steps
+// through the half2 intrinsics measured about 30 more integer-pipe instructions per tile.
 template <int K>
 __device__ __forceinline__ uint32_t vcode(uint32_t w, uint32_t w8) {
   const uint32_t src = K < 2 ? w : w8;
-  const uint32_t mask = (K & 1) ? 0x00F000F0u : 0x000F000Fu;
-  const uint32_t h = (src & mask) | 0x64006400u;
-  __half2 v = *reinterpret_cast<const __half2*>(&h);
-  const unsigned short off = (K & 1) ? 0x6480 : 0x6408;  // 1152 = 1024 + 16*8 or 1032 = 1024 + 8
-  v = __hsub2(v, __halves2half2(__ushort_as_half(off), __ushort_as_half(off)));
-  return *reinterpret_cast<uint32_t*>(&v);
+  uint32_t h, r;
+  if constexpr ((K & 1) != 0) {
+    // (src & 0x00F000F0) | 0x64006400 = 1024 + 16 c; minus 1152 = 1024 + 16 * 8
+    asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xea;" : "=r"(h) : "r"(src));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(0x64806480u));
+  } else {
+    // (src & 0x000F000F) | 0x64006400 = 1024 + c; minus 1032 = 1024 + 8
+    asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xea;" : "=r"(h) : "r"(src));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(0x64086408u));
+  }
+  return r;
 }
 
 // This lane's part of two fp32 values as an fp16 pair: the value truncated to 11 significant bits
@@ -403,6 +424,18 @@ __device__ __forceinline__ uint32_t split_pair(float x0, float x1, bool lo) {
   const float y1 = lo ? x1 - t1 : t1;
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(y1), "f"(y0));
+  return r;
+}
+
+// The bf16 counterpart of split_pair (bf16 values): the value truncated to 8 significant bits (hi
+// lanes) or the remainder rounded to bf16 (lo lanes); hi + lo carries ~16 bits.
+__device__ __forceinline__ uint32_t split_pair_bf16(float x0, float x1, bool lo) {
+  const float t0 = __uint_as_float(__float_as_uint(x0) & 0xFFFF0000u);
+  const float t1 = __uint_as_float(__float_as_uint(x1) & 0xFFFF0000u);
+  const float y0 = lo ? x0 - t0 : t0;
+  const float y1 = lo ? x1 - t1 : t1;
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(y1), "f"(y0));
   return r;
 }
 
@@ -453,21 +486,25 @@ struct PartRows {
 
 // ------------------------------------------------------------------ the decode kernel
 
-template <int D, int G, int QT, bool T8>
+// VB: values stored as bf16 (KV4_VALUES_BF16): one page tile per slot, PV on bf16 MMAs with the
+// probabilities as bf16 hi/lo halves, no value scale or offset.
+template <int D, int G, int QT, bool T8, bool VB>
 __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(const DecodeArgs a) {
   using Gm = Geo<D>;
   constexpr int NKB = Gm::NKB;
   constexpr int WPC = Gm::WPC;
   constexpr int NK32 = D / 32;  // 32-dim blocks of the QK^T integer MMAs
   constexpr int T4B = Gm::T4B;
+  constexpr int KPO = VB ? 8 * D : 16 * D;  // K {scale, zero} in a page tile
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  Smem<D>& sm = *reinterpret_cast<Smem<D>*>(smem_raw);
+  Smem<D, VB>& sm = *reinterpret_cast<Smem<D, VB>*>(smem_raw);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tig = lane & 3;
   const int wid = blockIdx.x * kWarps + warp;
   const int cap = a.stride * a.P;
-  pdl_launch_dependents();  // the merge kernel may be scheduled as SMs free up; it waits for this grid
+  // No early griddepcontrol.launch_dependents: the merge kernel launches when this grid completes.
+  // Launched early, its waiting CTAs sat beside this kernel's warps and slowed them (1-2 %).
 
   // Launched as a programmatic dependent of the preceding kernel.  By default nothing is read
   // before that kernel completes; with a.early the schedule and the first descriptors (which read
@@ -501,11 +538,11 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
 #pragma unroll
     for (int r = 0; r < kLensRegs; ++r)
       if (32 * r < a.B) {
-        const u32 c = 32 * r + lane < a.B ? static_cast<u32>(a.Hkv) * head_cost(seg_info<T8>(clamp_len(lr[r], cap), a.s, a.w, a.nt8, a.smw)) : 0u;
+        const u32 c = 32 * r + lane < a.B ? static_cast<u32>(a.Hkv) * head_cost<VB>(seg_info<T8>(clamp_len(lr[r], cap), a.s, a.w, a.nt8, a.smw)) : 0u;
         total += __shfl_sync(FULL, warp_incl_scan(c, lane), 31);
       }
   } else {
-    total = total_cost<T8>(a, cap, lane);
+    total = total_cost<T8, VB>(a, cap, lane);
   }
   const u32 Q = max(2u, (total + a.W - 1) / static_cast<u32>(a.W));
   const FastDiv divQ(Q);
@@ -520,7 +557,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
 #pragma unroll
     for (int r = 0; r < kLensRegs; ++r)
       if (32 * r < a.B && b0 == a.B) {
-        const u32 cb = 32 * r + lane < a.B ? static_cast<u32>(a.Hkv) * head_cost(seg_info<T8>(clamp_len(lr[r], cap), a.s, a.w, a.nt8, a.smw)) : 0u;
+        const u32 cb = 32 * r + lane < a.B ? static_cast<u32>(a.Hkv) * head_cost<VB>(seg_info<T8>(clamp_len(lr[r], cap), a.s, a.w, a.nt8, a.smw)) : 0u;
         const u32 incl = warp_incl_scan(cb, lane);
         const u32 tot = __shfl_sync(FULL, incl, 31);
         if (c0 < run + tot) {
@@ -531,9 +568,9 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
         run += tot;
       }
   } else {
-    b0 = find_seq<T8>(a, cap, lane, c0, &bstart);
+    b0 = find_seq<T8, VB>(a, cap, lane, c0, &bstart);
   }
-  Cursor dcur = cursor_at<T8>(a, cap, b0, bstart, c0, (any && b0 < a.B) ? (cached ? cached_len(b0) : a.lens[b0]) : 0);
+  Cursor dcur = cursor_at<T8, VB>(a, cap, b0, bstart, c0, (any && b0 < a.B) ? (cached ? cached_len(b0) : a.lens[b0]) : 0);
   const bool active = any && dcur.valid && dcur.cost < c1;
 
   // Query of the first (b, g): loaded during the first descriptor fill, or after the wait on the
@@ -552,7 +589,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   if (active && !a.early) load_q_regs(qb0, qg0);  // in flight during the descriptor fill
 
   unsigned segno = 0;
-  if (active) fill_descriptors<D, T8>(a, cap, c1, dcur, lane, sm, warp, 0, segno);
+  if (active) fill_descriptors<D, T8, VB>(a, cap, c1, dcur, lane, sm, warp, 0, segno);
   // the cursor waits in shared memory between fills (its registers are free in the main loop)
   if (lane == 0) {
     sm.cur[warp] = dcur;
@@ -584,12 +621,15 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     if (meta_kind(meta) == kKindNone) return false;
     const int st = k % kStages;
     const unsigned long long s0 = sm.src[warp][p][0], s1 = sm.src[warp][p][1];
-    const uint32_t nb = meta_kind(meta) == kKindInt8 ? Gm::H8B : T4B;
+    const uint32_t nb = meta_kind(meta) == kKindInt8 ? (VB ? Gm::T8V : Gm::H8B) : (VB ? Gm::T4V : T4B);
     const uint32_t bytes = (s0 ? nb : 0u) + (s1 ? nb : 0u);
     if (meta & kMetaBad) atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
     mbar_arrive_expect_tx(&bars[st], bytes);
-    if (s0) bulk_g2s(sm.ring[warp][st], reinterpret_cast<const void*>(s0), nb, &bars[st]);
-    if (s1) bulk_g2s(sm.ring[warp][st] + T4B, reinterpret_cast<const void*>(s1), nb, &bars[st]);
+    // the cache is read once per decode: evict it first from L2, so that lens, the page table,
+    // the queries and the split partials stay there
+    const uint64_t pol = l2_policy_evict_first();
+    if (s0) bulk_g2s_hint(sm.ring[warp][st], reinterpret_cast<const void*>(s0), nb, &bars[st], pol);
+    if (s1) bulk_g2s_hint(sm.ring[warp][st] + T4B, reinterpret_cast<const void*>(s1), nb, &bars[st], pol);
     return true;
   };
 
@@ -648,13 +688,13 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     for (int st = 4; st < D; st <<= 1) {
       if (st < h) {
         const int m = st >> 2;
-        const bool upper = (lane & m) != 0;
+        const float sgn = (lane & m) ? -1.f : 1.f;  // upper half of the pair: o - x, lower: x + o
 #pragma unroll
         for (int i = 0; i < G; ++i)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float o = __shfl_xor_sync(FULL, qx[i][e], m);
-            qx[i][e] = upper ? o - qx[i][e] : qx[i][e] + o;
+            qx[i][e] = fmaf(qx[i][e], sgn, o);  // exact: one rounding of o -+ x
           }
       }
     }
@@ -760,29 +800,42 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     beta_part = 0.f;
   };
 
+  // Which warps hold the partials of (b, g) (segment-table entry se of either segment): the
+  // first INT8 / INT4 warps and their counts.  When one warp holds the whole INT8 segment and
+  // the start of the INT4 segment, it runs one softmax across both regions (continuation) and
+  // writes no INT8 partial: the INT8 count is then 0.  Every warp computes the same record.
+  auto pair_split = [&](unsigned long long se, u32& w8a, u32& w4a, u32& n8p, u32& n4p) {
+    const int cb = seg_b(se);
+    const u32 cs8 = seg_cs8(se);
+    const SegInfo si = seg_info<T8>(clamp_len(a.lens[cb], cap), a.s, a.w, a.nt8, a.smw);
+    const u32 cs4 = cs8 + kU8<VB> * si.n8;
+    w8a = divQ.div(cs8);
+    w4a = divQ.div(cs4);
+    n8p = si.n8 ? divQ.div(cs4 - kU8<VB>) - w8a + 1 : 0u;
+    n4p = si.n4 ? divQ.div(cs4 + si.n4 - 1) - w4a + 1 : 0u;
+    if (n8p == 1u && n4p >= 1u && w8a == w4a) n8p = 0u;
+  };
+
   // Write the partial of the segment `se` (a segment-table entry).  The partials of (b, g) are
   // merged by merge_int4_kernel; when this is the only partial of (b, g) it is the output.
   auto flush = [&](unsigned long long se) {
     const int cb = seg_b(se), cg = seg_g(se), cseg = seg_kind(se);
-    const u32 cs8 = seg_cs8(se);
-    const SegInfo si = seg_info<T8>(clamp_len(a.lens[cb], cap), a.s, a.w, a.nt8, a.smw);
     float l = l_part, beta = beta_part;
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       l += __shfl_xor_sync(FULL, l, o);
       beta += __shfl_xor_sync(FULL, beta, o);
     }
-    const u32 cs4 = cs8 + 2u * si.n8;
-    const u32 w8a = divQ.div(cs8), w4a = divQ.div(cs4);
-    const u32 n8p = si.n8 ? divQ.div(cs4 - 2) - w8a + 1 : 0u;
-    const u32 n4p = si.n4 ? divQ.div(cs4 + si.n4 - 1) - w4a + 1 : 0u;
+    u32 w8a, w4a, n8p, n4p;
+    pair_split(se, w8a, w4a, n8p, n4p);
     const bool only = n8p + n4p == 1u && !a.rotate_v;  // rotated values: the merge rotates back
     const u32 sid = 2u * static_cast<u32>(cb * a.Hkv + cg) + static_cast<u32>(cseg);
     // where the merge finds the partials of (b, g); every writer of (b, g) stores the same record
     if (lane == 0) *reinterpret_cast<uint4*>(a.meta + 4 * (cb * a.Hkv + cg)) = make_uint4(w8a, w4a, n8p, n4p);
     if (tig < G) {
-      // INT4: even output rows carry (c - 8), odd rows 16 (c - 8); INT8 rows carry c.
-      const float f1 = cseg == 1 ? 0.0625f : 1.f;
+      // INT4: even output rows carry (c - 8), odd rows 16 (c - 8); INT8 rows carry c; bf16 values
+      // carry the values.
+      const float f1 = (cseg == 1 && !VB) ? 0.0625f : 1.f;
       const float sc = only ? (l > 0.f ? 1.f / l : 0.f) : 1.f;
       float* p = only ? a.out + (static_cast<size_t>(cb) * a.Hq + cg * G + tig) * D
                       : a.part + (static_cast<size_t>(wid + sid) * G + tig) * kPartRow<D>;
@@ -800,6 +853,8 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
       }
     }
   };
+
+
 
   // Running-max update for this lane's logits of head tig.  Logits and the running max m_run are
   // kept unscaled (log2 units times 2^e, e the query's power-of-two normalisation); the returned
@@ -836,11 +891,43 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     const float x0 = __shfl_sync(FULL, pv0, src0), x1 = __shfl_sync(FULL, pv0, src1);
     const float x2 = __shfl_sync(FULL, pv1, src0), x3 = __shfl_sync(FULL, pv1, src1);
     if (hh < G) {
-      b0 = split_pair(x0, x1, lo);
-      b1 = split_pair(x2, x3, lo);
+      b0 = VB ? split_pair_bf16(x0, x1, lo) : split_pair(x0, x1, lo);
+      b1 = VB ? split_pair_bf16(x2, x3, lo) : split_pair(x2, x3, lo);
     } else {
       b0 = b1 = 0u;
     }
+  };
+
+  // PV of one 16-row block of bf16 values (bf16 values) with probabilities p0, p1 (rows gq, gq + 8
+  // of head tig).  Rows whose bit in `rows` is clear are zeroed in the A operand: their bytes may
+  // be stale (a zero weight does not cancel a NaN pattern).
+  auto pv_bf16 = [&](const uint8_t* vb, bool v0, bool v1, float p0, float p1, unsigned rows) {
+    const float w0 = v0 ? p0 : 0.f, w1 = v1 ? p1 : 0.f;
+    l_part += w0 + w1;
+    uint32_t b0, b1;
+    pv_fragments(w0, w1, b0, b1);
+    constexpr int UPC = D / 32;
+    uint32_t vw0[D / 8], vw1[D / 8];
+#pragma unroll
+    for (int u = 0; u < UPC; ++u) {
+      const int uu = u ^ bf16_swz(D, tig, gq);
+      const uint4 y0 = *reinterpret_cast<const uint4*>(vb + ((0 * 8 + gq) * 4 + tig) * (D / 2) + 16 * uu);
+      const uint4 y1 = *reinterpret_cast<const uint4*>(vb + ((1 * 8 + gq) * 4 + tig) * (D / 2) + 16 * uu);
+      vw0[4 * u] = y0.x; vw0[4 * u + 1] = y0.y; vw0[4 * u + 2] = y0.z; vw0[4 * u + 3] = y0.w;
+      vw1[4 * u] = y1.x; vw1[4 * u + 1] = y1.y; vw1[4 * u + 2] = y1.z; vw1[4 * u + 3] = y1.w;
+    }
+    if (rows != 0xFFFFu) {
+      const int t0 = 2 * tig;
+      const uint32_t m0 = (((rows >> t0) & 1u) ? 0x0000ffffu : 0u) | (((rows >> (t0 + 1)) & 1u) ? 0xffff0000u : 0u);
+      const uint32_t m1 = (((rows >> (t0 + 8)) & 1u) ? 0x0000ffffu : 0u) | (((rows >> (t0 + 9)) & 1u) ? 0xffff0000u : 0u);
+#pragma unroll
+      for (int x = 0; x < D / 8; ++x) {
+        vw0[x] &= m0;
+        vw1[x] &= m1;
+      }
+    }
+#pragma unroll
+    for (int mb = 0; mb < NKB; ++mb) mma_bf16(oacc[mb], vw0[2 * mb], vw0[2 * mb + 1], vw1[2 * mb], vw1[2 * mb + 1], b0, b1);
   };
 
   // QK^T of one INT4 tile block: logits (log2 units) of rows gq and gq + 8 for head tig.
@@ -867,8 +954,8 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
       mma_u8s8(SA, a0, a1, a2, a3, qd[j][0], qd[j][1]);
       mma_u8s8(SB, a0, a1, a2, a3, qd[j][2], qd[j][3]);
     }
-    const uint32_t kp0 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 4 * gq);
-    const uint32_t kp1 = *reinterpret_cast<const uint32_t*>(tb + 16 * D + 4 * (gq + 8));
+    const uint32_t kp0 = *reinterpret_cast<const uint32_t*>(tb + KPO + 4 * gq);
+    const uint32_t kp1 = *reinterpret_cast<const uint32_t*>(tb + KPO + 4 * (gq + 8));
     const float ks0 = half_lo(kp0), kz0 = half_hi(kp0), ks1 = half_lo(kp1) * 0.0625f, kz1 = half_hi(kp1);
     // logit 2^e = s q_int.c + z sum(q_int), q_int.c = 2^16 S2 + (2^8 S1 + S0); the bracket is
     // below 2^30 in magnitude and exact in int32 (row gq + 8: 16 q_int.c, hence s / 16)
@@ -917,19 +1004,21 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
   bool failed = a.stall_test && !mbar_wait_bounded(&sm.stall[warp], 0u, a.err, a.wait_ns);
   int k = 0;
   while (!failed) {
+    // the next slot's copies first: its descriptor is in the chunk being consumed, and the fill
+    // below (page-table loads) then overlaps copies in flight
+    if (lane == 0 && issue(k + kStages - 1)) ++issued;
     if ((k % kChunk) == 0) {
       // descriptors of slots [k + kChunk, k + 2 kChunk) while this chunk is consumed
       Cursor fc = sm.cur[warp];
       unsigned fs = sm.segno[warp];
       __syncwarp();
-      fill_descriptors<D, T8>(a, cap, c1, fc, lane, sm, warp, k + kChunk, fs);
+      fill_descriptors<D, T8, VB>(a, cap, c1, fc, lane, sm, warp, k + kChunk, fs);
       if (lane == 0) {
         sm.cur[warp] = fc;
         sm.segno[warp] = fs;
       }
       __syncwarp();
     }
-    if (lane == 0 && issue(k + kStages - 1)) ++issued;
     const int st = k % kStages;
     const bool ok = mbar_wait_bounded(&bars[st], static_cast<uint32_t>((k / kStages) & 1), a.err, a.wait_ns);
     if (__any_sync(FULL, !ok)) {
@@ -940,7 +1029,20 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
     const int p = k % kRing;
     const unsigned meta = sm.meta[warp][p];
     const unsigned msk = sm.mask[warp][p];
-    if (meta_kind(meta) == kKindInt4) {
+    if (VB && meta_kind(meta) == kKindInt4) {
+      // ----------------------------------------------------------- one page tile, bf16 values
+      float l0, l1;
+      if (msk == 0xFFFFu) {
+        qk_int4(buf, true, true, l0, l1);
+        const float off = softmax_update(fmaxf(l0, l1));
+        pv_bf16(buf + Gm::VBO, true, true, prob(l0, off), prob(l1, off), 0xFFFFu);
+      } else {
+        const bool v0 = tig < G && ((msk >> gq) & 1u), v1 = tig < G && ((msk >> (gq + 8)) & 1u);
+        qk_int4(buf, v0, v1, l0, l1);
+        const float off = softmax_update(fmaxf(l0, l1));
+        pv_bf16(buf + Gm::VBO, v0, v1, prob(l0, off), prob(l1, off), msk);
+      }
+    } else if (meta_kind(meta) == kKindInt4) {
       // ----------------------------------------------------------- two INT4 tiles
       float lA0, lA1, lB0 = kNegInf, lB1 = kNegInf;
       if (msk == 0xFFFFFFFFu) {
@@ -992,35 +1094,57 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
       const float lg1 = v1 ? ks1 * R1 : kNegInf;
       const float off = softmax_update(fmaxf(lg0, lg1));
       const float p0 = prob(lg0, off), p1 = prob(lg1, off);
-      l_part += (v0 ? p0 : 0.f) + (v1 ? p1 : 0.f);
-      const uint8_t* vb = buf + T4B;  // V half
-      const float vs0 = __half2float(*reinterpret_cast<const __half*>(vb + 16 * D + 2 * gq));
-      const float vs1 = __half2float(*reinterpret_cast<const __half*>(vb + 16 * D + 2 * (gq + 8)));
-      uint32_t b0, b1;
-      pv_fragments(v0 ? p0 * vs0 : 0.f, v1 ? p1 * vs1 : 0.f, b0, b1);
-      constexpr int NW = Gm::CH8 / 4;  // words per pair chunk (8 or 4)
-      uint32_t vw0[NW], vw1[NW];
+      if constexpr (VB) {
+        pv_bf16(buf + Gm::VB8O, v0, v1, p0, p1, msk);
+      } else {
+        l_part += (v0 ? p0 : 0.f) + (v1 ? p1 : 0.f);
+        const uint8_t* vb = buf + T4B;  // V half
+        const float vs0 = __half2float(*reinterpret_cast<const __half*>(vb + 16 * D + 2 * gq));
+        const float vs1 = __half2float(*reinterpret_cast<const __half*>(vb + 16 * D + 2 * (gq + 8)));
+        uint32_t b0, b1;
+        pv_fragments(v0 ? p0 * vs0 : 0.f, v1 ? p1 * vs1 : 0.f, b0, b1);
+        constexpr int NW = Gm::CH8 / 4;  // words per pair chunk (8 or 4)
+        uint32_t vw0[NW], vw1[NW];
 #pragma unroll
-      for (int hv = 0; hv < NW / 4; ++hv) {
-        const int phys = (Gm::CH8 >= 32) ? (hv ^ (gq & 1)) : hv;
-        const uint4 x0 = *reinterpret_cast<const uint4*>(vb + ((0 * 8 + gq) * 4 + tig) * Gm::CH8 + 16 * phys);
-        const uint4 x1 = *reinterpret_cast<const uint4*>(vb + ((1 * 8 + gq) * 4 + tig) * Gm::CH8 + 16 * phys);
-        vw0[4 * hv] = x0.x; vw0[4 * hv + 1] = x0.y; vw0[4 * hv + 2] = x0.z; vw0[4 * hv + 3] = x0.w;
-        vw1[4 * hv] = x1.x; vw1[4 * hv + 1] = x1.y; vw1[4 * hv + 2] = x1.z; vw1[4 * hv + 3] = x1.w;
-      }
+        for (int hv = 0; hv < NW / 4; ++hv) {
+          const int phys = (Gm::CH8 >= 32) ? (hv ^ (gq & 1)) : hv;
+          const uint4 x0 = *reinterpret_cast<const uint4*>(vb + ((0 * 8 + gq) * 4 + tig) * Gm::CH8 + 16 * phys);
+          const uint4 x1 = *reinterpret_cast<const uint4*>(vb + ((1 * 8 + gq) * 4 + tig) * Gm::CH8 + 16 * phys);
+          vw0[4 * hv] = x0.x; vw0[4 * hv + 1] = x0.y; vw0[4 * hv + 2] = x0.z; vw0[4 * hv + 3] = x0.w;
+          vw1[4 * hv] = x1.x; vw1[4 * hv + 1] = x1.y; vw1[4 * hv + 2] = x1.z; vw1[4 * hv + 3] = x1.w;
+        }
 #pragma unroll
-      for (int mb = 0; mb < NKB; ++mb) {
-        const uint32_t w0 = vw0[mb] ^ 0x80808080u, w1 = vw1[mb] ^ 0x80808080u;
-        mma_f16(oacc[mb], i8x2_to_h2<0x4140>(w0), i8x2_to_h2<0x4342>(w0), i8x2_to_h2<0x4140>(w1),
-                i8x2_to_h2<0x4342>(w1), b0, b1);
+        for (int mb = 0; mb < NKB; ++mb) {
+          const uint32_t w0 = vw0[mb] ^ 0x80808080u, w1 = vw1[mb] ^ 0x80808080u;
+          mma_f16(oacc[mb], i8x2_to_h2<0x4140>(w0), i8x2_to_h2<0x4342>(w0), i8x2_to_h2<0x4140>(w1),
+                  i8x2_to_h2<0x4342>(w1), b0, b1);
+        }
       }
     }
     __syncwarp();
 
     if (meta & kMetaLast) {
       const unsigned long long se = sm.seg[warp][meta_seg(meta)];
-      flush(se);
-      reset();
+      bool cont = false;  // region continuation into the INT4 segment of the same (b, g)
+      if (seg_kind(se) == 0) {
+        u32 w8a, w4a, n8p, n4p;
+        pair_split(se, w8a, w4a, n8p, n4p);
+        cont = n8p == 0u && n4p >= 1u && w4a == static_cast<u32>(wid);
+      }
+      if (cont) {
+        // INT4 slots accumulate their odd output rows 16x (removed when the partial is written):
+        // bring the INT8 region's rows to that convention
+        if constexpr (!VB) {
+#pragma unroll
+          for (int mb = 0; mb < NKB; ++mb) {
+            oacc[mb][2] *= 16.f;
+            oacc[mb][3] *= 16.f;
+          }
+        }
+      } else {
+        flush(se);
+        reset();
+      }
       const unsigned nmeta = sm.meta[warp][(k + 1) % kRing];
       if (meta_kind(nmeta) == kKindNone) break;  // end of this warp's stream
       const unsigned long long ns = sm.seg[warp][meta_seg(nmeta)];
@@ -1044,21 +1168,22 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_int4_kernel(co
 
 // ------------------------------------------------------------------ LSE merge kernel
 
-// Merge of the partials of (sequence b, query head j): MW warps per (b, j) (MW = 4 when the batch
-// has few (b, j), else 1 with 4 (b, j) per CTA).  The decode kernel left, per (b, g), where the n
-// partials are (meta); warp w of the MW merges head j % G of partials [w n / MW, (w+1) n / MW) in
-// one pass, 32 at a time: lanes read the (m, l) of 32 partials, the running maximum is raised to
-// their maximum (rescaling the sums so far), and their o rows are read kInFlight at a time with
-// independent loads.  With MW = 4, warp 0 combines the warps' (M, L, o) through shared memory.
-// (b, g) with at most one partial, and sequences of length 0 (record of zeros), were written by
-// the decode kernel.  Launched as a programmatic dependent of the decode kernel:
-// griddepcontrol.wait orders every read of its results after its completion.
+// Merge of the partials of (sequence b, query head j): MW warps per (b, j), MW chosen on the host
+// so that a warp has at most kMergeBatch partials (MW = 1: four (b, j) per CTA of 4 warps; else one
+// (b, j) per CTA of MW warps).  The decode kernel left, per (b, g), where the n partials are
+// (meta); warp w of the MW merges head j % G of partials [w n / MW, (w+1) n / MW) in one pass of
+// batches of kMergeBatch rows, each batch one round trip.  With MW > 1, warp 0 combines the
+// warps' (M, L, o) through shared memory.  (b, g) with at most one partial, and sequences of
+// length 0 (record of zeros), were written by the decode kernel.  Launched as a programmatic
+// dependent of the decode kernel: griddepcontrol.wait orders every read of its results after its
+// completion.
 constexpr int kMergeThreads = 128;
+constexpr int kMergeBatch = 16;
 
 template <int D, int G, int MW>
-__global__ void __launch_bounds__(kMergeThreads) merge_int4_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(MW == 1 ? kMergeThreads : 32 * MW) merge_int4_kernel(const DecodeArgs a) {
   constexpr int PER = D / 32;
-  constexpr int kInFlight = 16;
+  constexpr int kInFlight = kMergeBatch;
   constexpr int RS = kPartRow<D>;
   using VecT = typename std::conditional<PER == 4, float4, float2>::type;
   __shared__ float smo[MW][D];
@@ -1090,45 +1215,34 @@ __global__ void __launch_bounds__(kMergeThreads) merge_int4_kernel(const DecodeA
   float M = kNegInf, L = 0.f, o[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) o[e] = 0.f;
-  for (int base = t0; base < t1; base += 32) {
-    const int t = base + lane;
-    unsigned long long row = 0;
-    float2 ml = make_float2(kNegInf, 0.f);
-    if (t < t1) {
-      row = pr.row(t, G, RS) + hd * RS;
-      ml = __ldcg(reinterpret_cast<const float2*>(a.part + row + D));
+  // One pass, kInFlight partials at a time: every lane loads its slice of each row together with
+  // the row's (m, l) (the same address in every lane), so a batch costs one memory round trip; the
+  // running maximum is raised partial by partial (warp-uniform).
+  for (int base = t0; base < t1; base += kInFlight) {
+    VecT v[kInFlight];
+    float2 ml[kInFlight];
+#pragma unroll
+    for (int u = 0; u < kInFlight; ++u) {
+      const int t = base + u < t1 ? base + u : t0;  // past the end: reload the first row, unused
+      const unsigned long long row = pr.row(t, G, RS) + hd * RS;
+      v[u] = __ldcg(reinterpret_cast<const VecT*>(a.part + row + lane * PER));
+      ml[u] = __ldcg(reinterpret_cast<const float2*>(a.part + row + D));
     }
-    const bool live = t < t1 && ml.y > 0.f;
-    float x = live ? ml.x : kNegInf;
 #pragma unroll
-    for (int sft = 16; sft; sft >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, sft));
-    if (x > M) {
-      const float sc = M == kNegInf ? 0.f : exp2f(M - x);
-      L *= sc;
+    for (int u = 0; u < kInFlight; ++u) {
+      if (base + u >= t1 || !(ml[u].y > 0.f)) continue;
+      if (ml[u].x > M) {
+        const float sc = M == kNegInf ? 0.f : exp2f(M - ml[u].x);
+        L *= sc;
 #pragma unroll
-      for (int e = 0; e < PER; ++e) o[e] *= sc;
-      M = x;
-    }
-    const float w = live ? exp2f(ml.x - M) : 0.f;
-    float wl = w * ml.y;
-#pragma unroll
-    for (int sft = 16; sft; sft >>= 1) wl += __shfl_xor_sync(FULL, wl, sft);
-    L += wl;
-    const int cnt = min(32, t1 - base);
-    for (int u0 = 0; u0 < cnt; u0 += kInFlight) {
-      VecT v[kInFlight];
-#pragma unroll
-      for (int u = 0; u < kInFlight; ++u) {
-        const unsigned long long rt = __shfl_sync(FULL, row, (u0 + u < cnt) ? u0 + u : 0);  // lane 0's row is valid
-        v[u] = __ldcg(reinterpret_cast<const VecT*>(a.part + rt + lane * PER));
+        for (int e = 0; e < PER; ++e) o[e] *= sc;
+        M = ml[u].x;
       }
+      const float w = exp2f(ml[u].x - M);
+      L = fmaf(w, ml[u].y, L);
+      const float* vv = reinterpret_cast<const float*>(&v[u]);
 #pragma unroll
-      for (int u = 0; u < kInFlight; ++u) {
-        const float wt = (u0 + u < cnt) ? __shfl_sync(FULL, w, u0 + u) : 0.f;
-        const float* vv = reinterpret_cast<const float*>(&v[u]);
-#pragma unroll
-        for (int e = 0; e < PER; ++e) o[e] = fmaf(wt, vv[e], o[e]);
-      }
+      for (int e = 0; e < PER; ++e) o[e] = fmaf(w, vv[e], o[e]);
     }
   }
   if constexpr (MW > 1) {
@@ -1201,10 +1315,12 @@ __global__ void __launch_bounds__(kMergeThreads) merge_int4_kernel(const DecodeA
 template <int D, int G>
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t st) {
   const int items = a.B * a.Hq;
-  const bool wide = items <= kMergeWideItems;
+  // partials of an average (b, g): its share of the split warps, plus the two segment ends
+  const long long per = static_cast<long long>(a.W) / (static_cast<long long>(a.B) * a.Hkv) + 2;
+  const int mw = per <= kMergeBatch ? 1 : per <= 4 * kMergeBatch ? 4 : per <= 8 * kMergeBatch ? 8 : 16;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(wide ? items : (items + kMergeThreads / 32 - 1) / (kMergeThreads / 32)));
-  cfg.blockDim = dim3(kMergeThreads);
+  cfg.gridDim = dim3(static_cast<unsigned>(mw > 1 ? items : (items + kMergeThreads / 32 - 1) / (kMergeThreads / 32)));
+  cfg.blockDim = dim3(mw > 1 ? 32 * mw : kMergeThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -1212,17 +1328,40 @@ cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return wide ? cudaLaunchKernelEx(&cfg, merge_int4_kernel<D, G, 4>, a) : cudaLaunchKernelEx(&cfg, merge_int4_kernel<D, G, 1>, a);
+  switch (mw) {
+    case 1: return cudaLaunchKernelEx(&cfg, merge_int4_kernel<D, G, 1>, a);
+    case 4: return cudaLaunchKernelEx(&cfg, merge_int4_kernel<D, G, 4>, a);
+    case 8: return cudaLaunchKernelEx(&cfg, merge_int4_kernel<D, G, 8>, a);
+    default: return cudaLaunchKernelEx(&cfg, merge_int4_kernel<D, G, 16>, a);
+  }
+}
+
+// One instantiation of the split-K kernel, launched as a programmatic dependent (its dynamic
+// shared-memory limit raised once per device).
+template <int D, int G, int QT, bool T8, bool VB>
+cudaError_t launch_variant(const cudaLaunchConfig_t& cfg0, const DecodeArgs& a, std::atomic<uint64_t>& done) {
+  const int smem = static_cast<int>(sizeof(Smem<D, VB>));
+  cudaError_t e = ensure_smem_limit(decode_int4_kernel<D, G, QT, T8, VB>, smem, done);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = cfg0;
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  return cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, QT, T8, VB>, a);
+}
+
+template <int D, int G, int QT>
+cudaError_t launch_qt(const cudaLaunchConfig_t& cfg, const DecodeArgs& a, std::atomic<uint64_t>* done) {
+  // bf16 values: every side tile is visited (masked), so one kernel serves every side-cache size
+  if (a.vbf) return launch_variant<D, G, QT, false, true>(cfg, a, done[2]);
+  if (a.nt8 > kTightSideTiles) return launch_variant<D, G, QT, true, false>(cfg, a, done[1]);
+  return launch_variant<D, G, QT, false, false>(cfg, a, done[0]);
 }
 
 template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
-  const int smem = static_cast<int>(sizeof(Smem<D>));
-  static std::atomic<uint64_t> done[6];
+  static std::atomic<uint64_t> done[3][3];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ctas));
   cfg.blockDim = dim3(kWarps * 32);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1230,29 +1369,9 @@ cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (a.nt8 > kTightSideTiles) {
-    if (a.q_dtype == KV4_F32) {
-      if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F32, true>, smem, done[3])) != cudaSuccess) return e;
-      e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_F32, true>, a);
-    } else if (a.q_dtype == KV4_BF16) {
-      if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_BF16, true>, smem, done[4])) != cudaSuccess) return e;
-      e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_BF16, true>, a);
-    } else {
-      if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F16, true>, smem, done[5])) != cudaSuccess) return e;
-      e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_F16, true>, a);
-    }
-  } else {
-    if (a.q_dtype == KV4_F32) {
-      if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F32, false>, smem, done[0])) != cudaSuccess) return e;
-      e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_F32, false>, a);
-    } else if (a.q_dtype == KV4_BF16) {
-      if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_BF16, false>, smem, done[1])) != cudaSuccess) return e;
-      e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_BF16, false>, a);
-    } else {
-      if ((e = ensure_smem_limit(decode_int4_kernel<D, G, KV4_F16, false>, smem, done[2])) != cudaSuccess) return e;
-      e = cudaLaunchKernelEx(&cfg, decode_int4_kernel<D, G, KV4_F16, false>, a);
-    }
-  }
+  if (a.q_dtype == KV4_F32) e = launch_qt<D, G, KV4_F32>(cfg, a, done[0]);
+  else if (a.q_dtype == KV4_BF16) e = launch_qt<D, G, KV4_BF16>(cfg, a, done[1]);
+  else e = launch_qt<D, G, KV4_F16>(cfg, a, done[2]);
   if (e != cudaSuccess) return e;
   return launch_merge<D, G>(a, st);
 }
@@ -1264,7 +1383,7 @@ int decode_ctas_per_sm() { return kCtasPerSm; }
 
 size_t decode_smem_bytes(int D, int G) {
   (void)G;
-  return D == 128 ? sizeof(Smem<128>) : sizeof(Smem<64>);
+  return D == 128 ? sizeof(Smem<128, true>) : sizeof(Smem<64, true>);
 }
 
 cudaError_t launch_decode_int4(DecodeArgs a, int D, int G, int ctas, cudaStream_t st) {

@@ -26,6 +26,7 @@ struct AppendArgs {
   size_t page_bytes, side_slot_bytes;
   uint32_t signs[4];      // bit d: key dim d negated before the rotation (randomised-sign Hadamard)
   int rotate_v;           // values stored in the keys' rotated basis too
+  int vbf;                // values stored as bf16 (KV4_VALUES_BF16)
   uint32_t* err;
 };
 
@@ -50,6 +51,7 @@ struct DecodeArgs {
   int early;              // build the schedule before waiting on the preceding kernel
   uint32_t signs[4];      // bit d: query dim d negated before the rotation (as the keys)
   int rotate_v;           // values stored rotated: outputs are rotated back by the merge kernel
+  int vbf;                // values stored as bf16 (KV4_VALUES_BF16)
   int stall_test;         // kv4_debug_force_wait_timeout: every warp's first wait runs out
   uint64_t wait_ns;       // bounded-wait limit of the bulk-copy waits
   uint32_t* err;

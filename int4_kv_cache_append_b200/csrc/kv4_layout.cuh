@@ -28,6 +28,11 @@
 //                      c[2p][d+1], c[2p+1][d+1]) for d = gq*D/8 + 2m; 16-byte halves of the
 //                      chunk swapped when CH8 = 32 and gq is odd.
 //   [H8B+16D, T8B)     V fp16 scale per row.
+// bf16 values (KV4_VALUES_BF16): a page tile is T4V = 16*(D/2 + 4 + 2D) bytes:
+//   [0, 8D)            K codes as above;  [8D, 8D+64)  K {scale, zero} per row;
+//   [8D+64, 40D+64)    V bf16 in the BF16 pool's V order (below).
+// and a side tile T8V = 16*(3D + 2) bytes: [0, 16D+32) K int8 codes and scales as above, then
+// [16D+32, 48D+32) V bf16 in the same order.
 // BF16 pool (baseline): page = Hkv head blocks of P/16 tiles of 64*D bytes:
 //   [0, 32D)   K bf16 row-major; row r, thread chunk c = e/(D/4) of D/2 bytes, 16-byte unit u of
 //              the chunk stored at unit u ^ sw(c, r).
@@ -50,6 +55,10 @@ struct Geo {
   static constexpr int DG = D / 8;            // dims per thread group
   static constexpr int NKB = D / 16;          // MMA k-blocks (QK) and m-blocks (PV)
   static constexpr int TBF = 64 * D;          // BF16 tile block
+  static constexpr int T4V = 40 * D + 64;      // page tile with bf16 values
+  static constexpr int T8V = 48 * D + 32;      // side tile with bf16 values
+  static constexpr int VBO = 8 * D + 64;       // bf16 values in a page tile
+  static constexpr int VB8O = 16 * D + 32;     // bf16 values in a side tile
   static constexpr int EPT = D / 4;           // BF16 elements per thread chunk
 };
 

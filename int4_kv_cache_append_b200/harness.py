@@ -13,8 +13,9 @@ from . import kv4
 from . import workload as W
 
 
-def geometry(wl: W.Workload, layers: int | None = None) -> kv4.Geometry:
-    return kv4.Geometry(layers or wl.layers, wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h, wl.B, max(wl.num_pages, 1))
+def geometry(wl: W.Workload, layers: int | None = None, value_format: int = kv4.KV4_VALUES_INT4) -> kv4.Geometry:
+    return kv4.Geometry(layers or wl.layers, wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h, wl.B, max(wl.num_pages, 1),
+                        value_format)
 
 
 def token_list(lens: np.ndarray, upto=None):

@@ -39,10 +39,13 @@ class KV4Error(RuntimeError):
         self.status = status
 
 
+KV4_VALUES_INT4, KV4_VALUES_BF16 = 0, 1
+
+
 class kv4_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "num_layers", "num_q_heads", "num_kv_heads", "head_dim", "page_size", "num_sinks",
-        "recent_window", "hadamard_block", "max_seqs", "max_pages")]
+        "recent_window", "hadamard_block", "max_seqs", "max_pages", "value_format")]
 
 
 def _load():
@@ -252,10 +255,12 @@ class Geometry:
     hadamard_block: int
     max_seqs: int
     max_pages: int
+    value_format: int = KV4_VALUES_INT4
 
     def c(self) -> kv4_config:
         return kv4_config(self.num_layers, self.num_q_heads, self.num_kv_heads, self.head_dim, self.page_size,
-                          self.num_sinks, self.recent_window, self.hadamard_block, self.max_seqs, self.max_pages)
+                          self.num_sinks, self.recent_window, self.hadamard_block, self.max_seqs, self.max_pages,
+                          self.value_format)
 
 
 class Cache:

@@ -139,6 +139,7 @@ class Workload:
     outliers: np.ndarray = field(repr=False)     # [Hkv][n_outlier] channel ids
     page_table: np.ndarray = field(repr=False)   # [B][stride] int32
     num_pages: int = 0
+    value_format: int = 0                        # 0: INT4 values, 1: bf16 values (K-INT4 / V-BF16)
 
     @property
     def G(self) -> int:
@@ -174,11 +175,14 @@ class Workload:
 
     def kv_bytes_int4(self, lens: np.ndarray | None = None) -> int:
         """Algorithmic KV bytes one decode reads: INT4 region codes + fp16 params, INT8 region
-        codes + fp16 scales, K and V, all KV heads."""
+        codes + fp16 scales, K and V, all KV heads (bf16 values: 2D bytes of V per position in
+        both regions instead of the V codes and parameters)."""
         L = np.asarray(self.lens if lens is None else lens, np.int64)
         n4 = np.maximum(0, L - self.s - self.w)
         n8 = np.minimum(L, self.s + self.w)
-        return int(self.Hkv * (n4 * (self.D + 8) + n8 * (2 * self.D + 4)).sum())
+        D = self.D
+        b4, b8 = (D // 2 + 4 + 2 * D, 3 * D + 2) if self.value_format else (D + 8, 2 * D + 4)
+        return int(self.Hkv * (n4 * b4 + n8 * b8).sum())
 
     def kv_bytes_bf16(self, lens: np.ndarray | None = None) -> int:
         L = np.asarray(self.lens if lens is None else lens, np.int64)

@@ -21,10 +21,10 @@ def to_dev(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
 
 
-def geometry(wl: W.Workload, max_seqs: int | None = None, layers: int | None = None):
+def geometry(wl: W.Workload, max_seqs: int | None = None, layers: int | None = None, value_format: int = 0):
     from int4_kv_cache_append_b200 import kv4
     return kv4.Geometry(layers or wl.layers, wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h,
-                        max_seqs or wl.B, max(wl.num_pages, 1))
+                        max_seqs or wl.B, max(wl.num_pages, 1), value_format)
 
 
 def prefill_tokens(lens):
@@ -34,11 +34,11 @@ def prefill_tokens(lens):
 
 
 def gpu_cache_from_host_inputs(wl: W.Workload, layer: int = 0, step_by_step: bool = False, fill: int = 0xA5,
-                               lens=None, signs=None, rotate_values: bool = False):
+                               lens=None, signs=None, rotate_values: bool = False, value_format: int = 0):
     """Append every token of the workload through kv4_append (inputs drawn on the host)."""
     from int4_kv_cache_append_b200 import kv4
     lens = np.asarray(wl.lens if lens is None else lens, np.int32)
-    cache = kv4.Cache(geometry(wl), fill=fill)
+    cache = kv4.Cache(geometry(wl, value_format=value_format), fill=fill)
     if signs is not None:
         kv4.kv4_set_rotation_signs(cache.handle, signs)
     if rotate_values:
@@ -63,9 +63,9 @@ def gpu_cache_from_host_inputs(wl: W.Workload, layer: int = 0, step_by_step: boo
 
 
 def oracle_cache(wl: W.Workload, layer: int = 0, step_by_step: bool = False, lens=None, signs=None,
-                 rotate_values: bool = False):
+                 rotate_values: bool = False, value_format: int = 0):
     cfg = O.Config(wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h, wl.B,
-                   tuple(signs) if signs is not None else (0, 0, 0, 0), int(rotate_values))
+                   tuple(signs) if signs is not None else (0, 0, 0, 0), int(rotate_values), int(value_format))
     lens = np.asarray(wl.lens if lens is None else lens, np.int32)
     pool = np.full(O.page_bytes(cfg) * max(wl.num_pages, 1), 0xA5, np.uint8)
     side = np.full(O.side_slot_bytes(cfg) * wl.B, 0xA5, np.uint8)

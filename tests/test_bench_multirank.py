@@ -106,4 +106,8 @@ def test_hadamard_override_of_one_layer_workloads():
     loop = bench.make_wl(argparse.Namespace(workload="qwen3-8b-loop", h=64, sinks=None, recent=None))
     assert loop.h == 64 and loop.layers == 36
     names = [n for n, _, _ in bench.PER_CONFIG]
+    vb = bench.make_wl(argparse.Namespace(workload="async-refill", h=None, sinks=None, recent=None, values="bf16"))
+    assert vb.value_format == 1 and vb.name.endswith("-vbf16")
+    base3 = W.async_refill()
+    assert vb.kv_bytes_int4() > base3.kv_bytes_int4()
     assert {"tiny", "qwen3-4b-decode", "async-refill", "long-context"} <= set(names)

@@ -337,7 +337,8 @@ def test_range_overflow_sets_error_bit():
     assert kv4.kv4_get_device_error() == 0
 
 
-def test_wait_limit_failure_path_reports_and_recovers():
+@pytest.mark.parametrize("case_id", [1, 11], ids=["b8", "b300"])
+def test_wait_limit_failure_path_reports_and_recovers(case_id):
     """The device-side failure path of the bounded waits, made to run with the test hook (no
     invalid copy involved): every decode warp's first wait is on a barrier that nothing arrives
     on, runs out after its 1 ms limit, sets KV4_DEVERR_WAIT_LIMIT, waits for its copies in flight
@@ -345,7 +346,7 @@ def test_wait_limit_failure_path_reports_and_recovers():
     point outside the workspace, skips them and reports KV4_DEVERR_RECORD.  The context stays
     usable: with the hook off the next decode matches the oracle and reports nothing."""
     from int4_kv_cache_append_b200 import kv4
-    wl = make(CASES[1])
+    wl = make(CASES[case_id])
     gc = T.gpu_cache_from_host_inputs(wl)
     assert kv4.kv4_get_device_error() == 0
     q_host = wl.q_input(0)
@@ -366,3 +367,52 @@ def test_wait_limit_failure_path_reports_and_recovers():
     out, lse = T.gpu_decode(gc, wl, q_host)
     T.assert_close(out, ref, lse, ref_lse, what="decode after the wait-limit path")
     assert kv4.kv4_get_device_error() == 0
+
+
+# K-INT4 / V-BF16: keys as in KV4, values stored as bf16 in the pages and the side cache
+VBF_CASES = [CASES[1], CASES[3], CASES[7], CASES[8], CASES[10], CASES[11]]
+
+
+@pytest.mark.parametrize("case", VBF_CASES, ids=[c[0] for c in VBF_CASES])
+@pytest.mark.parametrize("step_by_step", [False, True], ids=["prefill", "stepwise"])
+def test_bf16_values_append_bit_exact(case, step_by_step):
+    from int4_kv_cache_append_b200 import kv4
+    wl = make(case)
+    if step_by_step and wl.lens.max() > 160:
+        wl.lens = np.minimum(wl.lens, 160).astype(np.int32)
+    gc = T.gpu_cache_from_host_inputs(wl, step_by_step=step_by_step, value_format=1)
+    cfg, pool, side = T.oracle_cache(wl, step_by_step=step_by_step, value_format=1)
+    gp, gs = gc.layer_views(0)
+    gp, gs = gp.cpu().numpy(), gs.cpu().numpy()
+    assert gp.size == pool.size and gs.size == side.size
+    bad = np.nonzero(gp != pool)[0]
+    assert bad.size == 0, f"page pool differs at {bad.size} bytes, first {bad[:8]}"
+    bad = np.nonzero(gs != side)[0]
+    assert bad.size == 0, f"side cache differs at {bad.size} bytes, first {bad[:8]}"
+    assert kv4.kv4_get_device_error() == 0
+
+
+@pytest.mark.parametrize("case", VBF_CASES, ids=[c[0] for c in VBF_CASES])
+def test_bf16_values_decode_matches_oracle(case):
+    from int4_kv_cache_append_b200 import kv4
+    wl = make(case)
+    gc = T.gpu_cache_from_host_inputs(wl, value_format=1)
+    cfg, pool, side = T.oracle_cache(wl, value_format=1)
+    q = wl.q_input(0)
+    ref, ref_lse = T.oracle_decode(wl, cfg, pool, side, q)
+    out, lse = T.gpu_decode(gc, wl, q)
+    T.assert_close(out, ref, lse, ref_lse, what="bf16 values " + case[0])
+    single, _ = T.oracle_decode(wl, cfg, pool, side, q, mode=O.SINGLE)
+    T.assert_close(out, single, what="bf16 values " + case[0] + " vs single softmax")
+    # split points do not change the result beyond the tolerance
+    out2, lse2 = T.gpu_decode(gc, wl, q, max_len_hint=1)
+    T.assert_close(out2, ref, lse2, ref_lse, what="bf16 values, one CTA")
+    assert kv4.kv4_get_device_error() == 0
+
+
+def test_bf16_values_reject_value_rotation():
+    from int4_kv_cache_append_b200 import kv4
+    wl = make(CASES[1])
+    gc = kv4.Cache(T.geometry(wl, value_format=1))
+    with pytest.raises(kv4.KV4Error):
+        kv4.kv4_set_value_rotation(gc.handle, True)
