@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--impl", choices=["kv4", "reference"], default="kv4")
     ap.add_argument("--workload", default="qwen3-8b-loop")
     ap.add_argument("--h", type=int, default=None, help="Hadamard block of the 36-layer workload (32, 64, 128)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layers of the 36-layer workload (fewer for a small profiler capture: every layer's "
+                         "launch is the same, only the resident KV shrinks)")
     ap.add_argument("--sinks", type=int, default=None, help="override s, the INT8 sink positions")
     ap.add_argument("--recent", type=int, default=None,
                     help="override w, the INT8 recent window (-1: every position, i.e. all-INT8 KV8)")
@@ -86,9 +89,17 @@ def make_wl(args):
     from int4_kv_cache_append_b200 import workload as W
     fn = W.WORKLOADS[args.workload]
     h = getattr(args, "h", None)
-    if h is not None and args.workload == "qwen3-8b-loop":
-        wl = fn(h=h)
+    nl = getattr(args, "layers", None)
+    if args.workload == "qwen3-8b-loop" and (h is not None or nl is not None):
+        kw = {"h": h} if h is not None else {}
+        if nl is not None:
+            kw["layers"] = nl
+        wl = fn(**kw)
+        if nl is not None:
+            wl = dataclasses.replace(wl, name=f"{wl.name}-{nl}layers")
     else:
+        if nl is not None:
+            raise SystemExit("--layers applies to the 36-layer workload only")
         wl = fn()
         if h is not None and h != wl.h:
             wl = dataclasses.replace(wl, h=h, name=f"{wl.name}-h{h}")
@@ -341,7 +352,7 @@ def step_shape(wl):
     same position every step.  A workload with more layers than that (the 36-layer append + decode
     loop) runs every layer in one step, and its lengths grow by one token per step."""
     grow = int((wl.max_lens - wl.lens).min())
-    if wl.layers > LAYERS:
+    if wl.layers > 1:
         return wl.layers, wl.layers, grow
     return 1, LAYERS, grow
 
