@@ -140,6 +140,7 @@ class Workload:
     page_table: np.ndarray = field(repr=False)   # [B][stride] int32
     num_pages: int = 0
     value_format: int = 0                        # 0: INT4 values, 1: bf16 values (K-INT4 / V-BF16)
+    rope_outliers: bool = False                  # outliers as whole RoPE blocks, queries scaled alike
 
     @property
     def G(self) -> int:
@@ -150,9 +151,14 @@ class Workload:
         return int(self.page_table.shape[1])
 
     def factor(self) -> np.ndarray:
+        """Per-channel multiplier [Hkv][D] of the K and V inputs.  With rope_outliers an outlier
+        channel o takes its rotary partner (o + D/2) mod D along, so the outlier is a whole
+        two-dimensional RoPE block, as rotary position embedding makes it in real keys."""
         f = np.ones((self.Hkv, self.D), np.float32)
         for g in range(self.Hkv):
             f[g, self.outliers[g]] = np.float32(self.outlier_scale)
+            if self.rope_outliers:
+                f[g, (self.outliers[g] + self.D // 2) % self.D] = np.float32(self.outlier_scale)
         return f
 
     def kv_inputs(self, layer: int, b: np.ndarray, pos: np.ndarray):
@@ -169,6 +175,8 @@ class Workload:
     def q_input(self, layer: int, step: int = 0, rows: np.ndarray | None = None):
         """Queries [B][Hq][D] (or only the given rows) as fp32 or bf16 bits."""
         q = query_values(stream_key(self.seed, KIND_Q, layer, step), self.B, self.Hq, self.D)
+        if self.rope_outliers:  # queries carry the same block outliers as the keys of their head
+            q = (q * np.repeat(self.factor(), self.G, axis=0)[None]).astype(np.float32)
         if rows is not None:
             q = q[np.asarray(rows)]
         return bf16_bits(q) if self.q_dtype == BF16 else q.astype(np.float32)

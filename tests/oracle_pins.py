@@ -723,3 +723,8 @@ ALL_PINS = [
     pin_special_cases, pin_signed_rotation_exact, pin_value_rotation_invariance, pin_quant_range,
     pin_append_range_flag, pin_bf16_rounding, pin_layout_bijection_bf16_values, pin_bf16_values_exact,
 ]
+
+# the mixed bit-width key cache's pins run with the rest (the mutation test runs ALL_PINS)
+import gtq_pins as _G  # noqa: E402
+
+ALL_PINS = ALL_PINS + list(_G.GTQ_PINS)

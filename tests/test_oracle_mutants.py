@@ -1,7 +1,7 @@
 """Plant plausible mistakes in copies of the oracle (on the CPU) and check the pins catch them.
 
-Each mutant is one textual edit of ``oracle/kv4_oracle.c`` (a dropped term, a wrong sign,
-rounding mode, index or constant).  It is compiled to a temporary library and the full pin
+Each mutant is one textual edit of ``oracle/kv4_oracle.c`` or ``oracle/gtq_oracle.c`` (a dropped
+term, a wrong sign, rounding mode, index or constant).  It is compiled to a temporary library and the full pin
 list runs against it in a child process; the mutant is "killed" when any pin fails (or the
 child crashes).  A surviving mutant means the pins do not constrain that part of the oracle.
 """
@@ -14,7 +14,8 @@ from concurrent.futures import ThreadPoolExecutor
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-SRC = os.path.join(ROOT, "oracle", "kv4_oracle.c")
+ORACLE = os.path.join(ROOT, "oracle")
+FILES = ("kv4_oracle.c", "gtq_oracle.c", "kv4_oracle.h", "gtq_oracle.h")
 
 # (name, original text, replacement, occurrence index or None for all)
 MUTANTS = [
@@ -61,6 +62,31 @@ MUTANTS = [
     ("single-softmax-max", "if (logit[j] > ps->m) ps->m = logit[j];", "if (logit[j] < ps->m) ps->m = logit[j];", None),
 ]
 
+# mutants of the mixed bit-width key cache (gtq_oracle.c)
+GTQ_MUTANTS = [
+    ("gtq-gain-2-per-bit", "ldexp(energy[b], -2 * (int)widths[b]); /* E * 4^-w, exact */",
+     "ldexp(energy[b], -(int)widths[b]);", None),
+    ("gtq-ties-to-highest", "if (best < 0 || gain > best_gain) {", "if (best < 0 || gain >= best_gain) {", None),
+    ("gtq-cap-7", "if (widths[b] >= 8) continue;", "if (widths[b] >= 7) continue;", None),
+    ("gtq-adjacent-pairs", "gtq_load(K, k_dtype, row + (size_t)(b + nb));", "gtq_load(K, k_dtype, row + (size_t)(b ^ 1));", None),
+    ("gtq-energy-one-coordinate", "e = e + (x0 * x0 + x1 * x1);", "e = e + x0 * x0;", None),
+    ("gtq-scale-mean-not-rms", "(float)sqrt(energy[b] / (2.0 * (double)T))", "(float)(energy[b] / (2.0 * (double)T))", None),
+    ("gtq-key-scale-round-nearest", "const uint16_t sb = orc_f32_to_f16(m, ORC_RU);", "const uint16_t sb = orc_f32_to_f16(m, ORC_RN);", None),
+    ("gtq-key-ignores-sigma", "const float a = fabsf(x[i]) / sc[i];", "const float a = fabsf(x[i]);", None),
+    ("gtq-key-round-not-floor", "const float f = floorf(u);", "const float f = rintf(u);", None),
+    ("gtq-key-levels-off", "(t + 1.0f) * (float)(1 << (w - 1))", "(t + 1.0f) * (float)(1 << w)", None),
+    ("gtq-key-recon-midpoint", "(ldexp(2.0 * code + 1.0, -w) - 1.0)", "(ldexp(2.0 * code, -w) - 1.0)", None),
+    ("gtq-w0-not-zero", "if (w == 0) return 0.0;", "if (w == 0) return (double)orc_f16_to_f32(scale) * (double)sigma;", None),
+    ("gtq-value-levels-2w", "const int top = (1 << bits) - 1;", "const int top = (1 << bits);", 0),
+    ("gtq-value-zero-round-nearest", "const uint16_t zb = orc_f32_to_f16(mn, ORC_RD);", "const uint16_t zb = orc_f32_to_f16(mn, ORC_RN);", None),
+    ("gtq-pack-msb-first", "row[n >> 3] |= (uint8_t)(1u << (n & 7));", "row[n >> 3] |= (uint8_t)(0x80u >> (n & 7));", None),
+    ("gtq-value-rows-after-params", "return tile_base(c, page, g) + (size_t)c->page_size * orc_gtq_key_row_bytes(c) +\n         (size_t)pp * orc_gtq_value_row_bytes(c);",
+     "return tile_base(c, page, g) + (size_t)c->page_size * (orc_gtq_key_row_bytes(c) + 8) +\n         (size_t)pp * orc_gtq_value_row_bytes(c);", None),
+    ("gtq-param-order", "put16(pool + orc_gtq_param(c, page, g, pp) + 4, z);", "put16(pool + orc_gtq_param(c, page, g, pp) + 6, z);", None),
+    ("gtq-block-of-coordinate", "wc[i] = widths[(size_t)g * (size_t)nb + (size_t)(i % nb)];", "wc[i] = widths[(size_t)g * (size_t)nb + (size_t)(i / 2)];", None),
+    ("gtq-softmax-scale", "const double tau = 1.0 / sqrt((double)D);", "const double tau = 1.0 / (double)D;", None),
+]
+
 RUNNER = r"""
 import sys
 sys.path.insert(0, {root!r}); sys.path.insert(0, {tests!r})
@@ -85,18 +111,19 @@ def _mutate(text: str, old: str, new: str, occ):
     return old.join(parts[:occ + 1]) + new + old.join(parts[occ + 1:])
 
 
-def _run_mutant(tmp: str, name: str, old: str, new: str, occ) -> tuple[str, str]:
-    src = _mutate(open(SRC).read(), old, new, occ)
+def _run_mutant(tmp: str, fname: str, name: str, old: str, new: str, occ) -> tuple[str, str]:
     d = os.path.join(tmp, name)
     os.makedirs(d)
-    csrc = os.path.join(d, "kv4_oracle.c")
-    with open(csrc, "w") as f:
-        f.write(src)
-    import shutil
-    shutil.copy(os.path.join(ROOT, "oracle", "kv4_oracle.h"), d)
+    for f in FILES:
+        text = open(os.path.join(ORACLE, f)).read()
+        if f == fname:
+            text = _mutate(text, old, new, occ)
+        with open(os.path.join(d, f), "w") as out:
+            out.write(text)
     so = os.path.join(d, "lib.so")
     from oracle.oracle import CFLAGS
-    subprocess.run(["gcc", *[c for c in CFLAGS if c not in ("-Wall", "-Wextra")], "-o", so, csrc, "-lm"],
+    srcs = [os.path.join(d, f) for f in FILES if f.endswith(".c")]
+    subprocess.run(["gcc", *[c for c in CFLAGS if c not in ("-Wall", "-Wextra")], "-o", so, *srcs, "-lm"],
                    check=True, capture_output=True)
     env = dict(os.environ, KV4_ORACLE_LIB=so, OMP_NUM_THREADS="1")
     r = subprocess.run([sys.executable, "-c", RUNNER.format(root=ROOT, tests=os.path.join(ROOT, "tests"))],
@@ -108,6 +135,7 @@ def _run_mutant(tmp: str, name: str, old: str, new: str, occ) -> tuple[str, str]
 def test_every_mutant_is_killed():
     with tempfile.TemporaryDirectory() as tmp:
         with ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
-            results = list(ex.map(lambda m: _run_mutant(tmp, *m), MUTANTS))
+            jobs = [("kv4_oracle.c", *m) for m in MUTANTS] + [("gtq_oracle.c", *m) for m in GTQ_MUTANTS]
+            results = list(ex.map(lambda m: _run_mutant(tmp, *m), jobs))
     survivors = [(n, r) for n, r in results if "SURVIVED" in r]
     assert not survivors, f"mutants not caught by any pin: {survivors}"
