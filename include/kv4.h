@@ -59,7 +59,9 @@ typedef enum {
   KV4_ERR_UNSUPPORTED = 2,  /* geometry outside the compiled variants (see kv4_config)  */
   KV4_ERR_WORKSPACE = 3,    /* workspace missing or smaller than kv4_*_workspace_bytes  */
   KV4_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed              */
-  KV4_ERR_DEVICE = 5        /* device-side guard fired (kv4_get_device_error has bits)  */
+  KV4_ERR_DEVICE = 5,       /* device-side guard fired (kv4_get_device_error has bits)  */
+  KV4_ERR_NO_ALLOCATION = 6 /* mixed bit-width keys: the layer has no block allocation yet
+                               (kv4_allocate_key_bits or kv4_set_key_allocation)          */
 } kv4_status;
 
 typedef enum { KV4_F32 = 0, KV4_BF16 = 1, KV4_F16 = 2 } kv4_dtype;
@@ -75,9 +77,12 @@ typedef enum { KV4_F32 = 0, KV4_BF16 = 1, KV4_F16 = 2 } kv4_dtype;
                                        workspace (left by a decode that stopped early) and
                                        skipped it                                               */
 
-/* Value storage formats (kv4_config.value_format). */
+/* Storage formats (kv4_config.value_format). */
 #define KV4_VALUES_INT4 0  /* values as per-token affine INT4 (INT8 in the side cache): KV4       */
 #define KV4_VALUES_BF16 1  /* values kept in bf16 in the pages and the side cache, keys as in KV4 */
+#define KV4_KEYS_MIXED 2   /* mixed bit-width keys allocated per RoPE block, values at value_bits
+                              ("RoPE-Aware Bit Allocation for KV-Cache Quantization", abstract);
+                              see kv4_allocate_key_bits                                          */
 
 /*
  * Cache geometry.  Supported: head_dim in {64, 128}; Hq/Hkv in {1, 2, 4}; page_size a
@@ -86,7 +91,11 @@ typedef enum { KV4_F32 = 0, KV4_BF16 = 1, KV4_F16 = 2 } kv4_dtype;
  * vLLM; page ids index a per-layer pool of max_pages pages.  value_format selects the value
  * storage (KV4-RL, "Main Findings", compares KV4, KV8 and BF16 KV budgets; the K-INT4 / V-BF16
  * variant keeps the INT4 keys and leaves the values unquantised): KV4_VALUES_INT4 (0, the
- * default of a zeroed struct) or KV4_VALUES_BF16 (1).
+ * default of a zeroed struct) or KV4_VALUES_BF16 (1).  KV4_KEYS_MIXED (2) selects the mixed
+ * bit-width key cache instead: keys take key_bits bits per dimension on average (1..8), split
+ * over the RoPE blocks of each KV head by kv4_allocate_key_bits; values take value_bits bits per
+ * dimension (2, 3, 4 or 8); it has no side cache and no rotation (num_sinks = recent_window = 0,
+ * hadamard_block = 1).  key_bits and value_bits are ignored by the other formats.
  */
 typedef struct {
   int num_layers;
@@ -99,7 +108,9 @@ typedef struct {
   int hadamard_block;   /* h                                     */
   int max_seqs;         /* sequence slots of the INT8 side cache */
   int max_pages;        /* pages per layer pool                  */
-  int value_format;     /* KV4_VALUES_INT4 or KV4_VALUES_BF16    */
+  int value_format;     /* KV4_VALUES_INT4, KV4_VALUES_BF16 or KV4_KEYS_MIXED */
+  int key_bits;         /* KV4_KEYS_MIXED: average key bits per dimension      */
+  int value_bits;       /* KV4_KEYS_MIXED: value bits per dimension            */
 } kv4_config;
 
 typedef struct kv4_cache kv4_cache;  /* opaque host handle */
@@ -113,6 +124,11 @@ typedef struct kv4_cache kv4_cache;  /* opaque host handle */
  *   side cache: num_layers * max_seqs * Hkv * ceil((s + w)/16) * 16 * (2D + 4)
  * With KV4_VALUES_BF16 a position takes D/2 + 4 + 2D bytes in a page (K codes and parameters,
  * bf16 V) and 3D + 2 in the side cache (INT8 K and its scale, bf16 V).
+ * With KV4_KEYS_MIXED a position takes key_bits*D/8 + value_bits*D/8 + 8 bytes in a page (the
+ * packed key and value codes and four fp16: key scale, 0, value zero, value range; a page of one
+ * KV head holds P key rows, then P value rows, then P records, heads in order), the side cache is
+ * empty, and the page pool ends with num_layers * Hkv block-allocation records of
+ * ceil16(5 D / 2) bytes (D/2 fp32 block scales, then D/2 uint8 block widths).
  * Both must be 16-byte aligned.  Returns KV4_ERR_UNSUPPORTED for geometries outside the list.
  */
 kv4_status kv4_query_sizes(const kv4_config* cfg, size_t* page_pool_bytes, size_t* side_cache_bytes);
@@ -142,6 +158,14 @@ void kv4_cache_destroy(kv4_cache* cache);
  * Device-side: a page id outside [0, max_pages) or pos / P >= stride sets an error bit and the
  * token is skipped; a vector whose fp16 scale or offset overflows sets KV4_DEVERR_RANGE (stored
  * with zero codes).  With KV4_VALUES_BF16 the values are stored as bf16 (nearest even) instead.
+ * With KV4_KEYS_MIXED ("RoPE-Aware Bit Allocation for KV-Cache Quantization", abstract; the
+ * layer's allocation from kv4_allocate_key_bits): a key gets one fp16 scale s, rounded up, of
+ * max |x_j| / sigma_j over coordinates with bits, and coordinate j of width w the code
+ * clamp(floor((x_j / (sigma_j s) + 1) 2^(w-1)), 0, 2^w - 1) (reconstructed as
+ * s sigma_j ((2 code + 1) 2^-w - 1); 0 for w = 0); a value gets the per-token affine code of the
+ * INT4 cache at value_bits bits (fp16 zero rounded down, fp16 range rounded up, code =
+ * rint((x - zero) / (range / (2^b - 1)))); codes packed in coordinate order, least significant
+ * bit first; lens_after is not read.
  */
 kv4_status kv4_append(kv4_cache* cache, int layer, int T, const void* K, kv4_dtype k_dtype,
                       const void* V, kv4_dtype v_dtype, const int32_t* seq_slot, const int32_t* pos,
@@ -171,6 +195,9 @@ kv4_status kv4_decode_workspace_bytes(const kv4_cache* cache, int B, size_t* byt
  * (sequence, KV head) runs one softmax across both; a (sequence, KV head) covered by a single
  * partial is written directly), then the LSE merge of the partials of every other (sequence,
  * KV head).
+ * With KV4_KEYS_MIXED the layer's packed pages over [0, L) are attended as one region (no side
+ * cache, no rotation) with the keys and values reconstructed as kv4_append describes; two
+ * launches as well (split-K pass over 16-position tiles, LSE merge).
  */
 kv4_status kv4_decode_attn(kv4_cache* cache, int layer, int B, const void* q, kv4_dtype q_dtype,
                            const int32_t* page_table, int stride, const int32_t* lens, int max_len_hint,
@@ -221,6 +248,30 @@ kv4_status kv4_set_decode_overlap(kv4_cache* cache, int enable);
  * KV4_ERR_INVALID_ARG for a NULL or BF16 cache.
  */
 kv4_status kv4_debug_force_wait_timeout(kv4_cache* cache, int enable);
+
+/*
+ * Mixed bit-width keys (KV4_KEYS_MIXED): the block allocation of one layer.  "RoPE-Aware Bit
+ * Allocation for KV-Cache Quantization" (searcharxiv abstract): under RoPE a key's share of a
+ * later logit is a sum over its two-dimensional frequency blocks, so for every layer and KV head a
+ * label-free energy score is taken per RoPE block and integer bit widths are handed out greedily
+ * by marginal gain under the key budget.  Conventions: block b of a head is the rotate-half pair
+ * of coordinates (b, b + D/2); its score E_b is the fp64 sum of k[b]^2 + k[b + D/2]^2 over the
+ * given keys in order; its scale is sigma_b = sqrt(E_b / 2T) rounded to fp32 (1 when E_b = 0);
+ * starting from 0 bits, one bit at a time goes to the block of largest E_b 4^-w_b below 8 bits
+ * (lowest block on ties) until the blocks hold key_bits * D / 2 bits.
+ *
+ * kv4_allocate_key_bits scores the T keys K [T][Hkv][D] (KV4_F32, KV4_BF16 or KV4_F16, device
+ * memory) and writes the allocation of every KV head of the layer, all on the device (one
+ * kernel, one thread block per KV head summing in key order: about T * 10 ns).  Later appends of
+ * the layer quantise with it; re-allocating does not re-encode what is already stored.
+ * kv4_set_key_allocation copies a caller's allocation (host arrays widths [Hkv][D/2], each <= 8
+ * with D/2-sums of key_bits * D / 2, and sigma [Hkv][D/2], positive and finite) to the device;
+ * kv4_get_key_allocation copies the layer's allocation back to host arrays and synchronises the
+ * stream.  Append and decode of a layer without an allocation return KV4_ERR_NO_ALLOCATION.
+ */
+kv4_status kv4_allocate_key_bits(kv4_cache* cache, int layer, int T, const void* K, kv4_dtype k_dtype, void* stream);
+kv4_status kv4_set_key_allocation(kv4_cache* cache, int layer, const uint8_t* widths, const float* sigma, void* stream);
+kv4_status kv4_get_key_allocation(kv4_cache* cache, int layer, uint8_t* widths, float* sigma, void* stream);
 
 /*
  * BF16-KV baseline (KV4-RL, "Main Findings", quotes its speed-ups against BF16 KV) with the same

@@ -22,7 +22,7 @@ COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-shared"
           "-Xptxas", "-v"]
 
 LIBS = {
-    "libkv4.so": ["kv4_api.cu", "kv4_append.cu", "kv4_decode.cu", "kv4_bf16.cu"],
+    "libkv4.so": ["kv4_api.cu", "kv4_append.cu", "kv4_decode.cu", "kv4_bf16.cu", "kv4_mixed.cu"],
     "libkv4gen.so": ["kv4gen.cu"],
 }
 

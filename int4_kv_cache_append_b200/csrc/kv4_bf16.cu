@@ -1,9 +1,9 @@
 // kv4_bf16.cu -- BF16-KV paged decode attention: the baseline the INT4 cache is measured
 // against (KV4-RL, "Main Findings": speedups are quoted relative to BF16 KV).
 //
-// Same structure as the INT4 decode (flattened split-K over 16-position tiles, one bulk copy per
-// tile into a per-warp shared-memory ring, m16n8k16 MMA with the GQA group's query heads as the
-// N columns, LSE merge), but K and V are bf16 in the pages, so the MMA operands are read as-is.
+// Flattened split-K over 16-position tiles (kv4_splitk.cuh), one bulk copy per tile into a
+// per-warp shared-memory ring, m16n8k16 MMA with the GQA group's query heads as the N columns,
+// LSE merge; K and V are bf16 in the pages, so the MMA operands are read as-is.
 // Queries enter as bf16 hi/lo halves (exact for bf16 queries); P enters as bf16 hi/lo halves.
 #include <cuda_bf16.h>
 #include <math.h>
@@ -11,6 +11,7 @@
 #include "kv4_device.cuh"
 #include "kv4_internal.h"
 #include "kv4_layout.cuh"
+#include "kv4_splitk.cuh"
 
 namespace kv4 {
 namespace {
@@ -20,67 +21,11 @@ constexpr int kWarps = 8;
 constexpr int kStages = 3;
 constexpr float kNegInf = -__builtin_huge_valf();
 
-__device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
-__device__ __forceinline__ long long seq_cost(const DecodeArgs& a, int L) { return static_cast<long long>(a.Hkv) * ((L + 15) >> 4); }
-
-__device__ __forceinline__ long long warp_incl_scan(long long v, int lane) {
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const long long t = __shfl_up_sync(FULL, v, o);
-    if (lane >= o) v += t;
-  }
-  return v;
-}
-
-__device__ long long prefix_cost(const DecodeArgs& a, int cap, int lane, int upto) {
-  long long run = 0;
-  for (int base = 0; base < upto; base += 32) {
-    const int b = base + lane;
-    const long long c = b < upto ? seq_cost(a, clamp_len(a.lens[b], cap)) : 0;
-    run += __shfl_sync(FULL, warp_incl_scan(c, lane), 31);
-  }
-  return run;
-}
-
-__device__ int find_seq(const DecodeArgs& a, int cap, int lane, long long c, long long* bstart) {
-  long long run = 0;
-  for (int base = 0; base < a.B; base += 32) {
-    const int b = base + lane;
-    const long long cb = b < a.B ? seq_cost(a, clamp_len(a.lens[b], cap)) : 0;
-    const long long incl = warp_incl_scan(cb, lane);
-    const long long tot = __shfl_sync(FULL, incl, 31);
-    if (c < run + tot) {
-      const unsigned m = __ballot_sync(FULL, c < run + incl);
-      const int l = __ffs(m) - 1;
-      *bstart = run + __shfl_sync(FULL, incl - cb, l);
-      return base + l;
-    }
-    run += tot;
-  }
-  *bstart = run;
-  return a.B;
-}
-
-__device__ __forceinline__ long long quota(long long total, int W) {
-  const long long q = (total + W - 1) / W;
-  return q < 1 ? 1 : q;
-}
-
-struct Cur {
-  int b, g, i, n;
-  bool valid;
-};
-
-__device__ __forceinline__ void settle(const DecodeArgs& a, int cap, Cur& c) {
-  while (c.b < a.B && c.i >= c.n) {
-    c.i = 0;
-    if (++c.g == a.Hkv) {
-      c.g = 0;
-      if (++c.b < a.B) c.n = (clamp_len(a.lens[c.b], cap) + 15) >> 4;
-    }
-  }
-  c.valid = c.b < a.B;
-}
+using splitk::clamp_len;
+using splitk::Cur;
+using splitk::prefix_cost;
+using splitk::quota;
+using splitk::settle;
 
 template <int D, int G>
 struct SmemBF {
@@ -125,17 +70,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_bf16_kernel(const Decod
   if (c0 >= total) return;
   const long long c1 = c0 + Q < total ? c0 + Q : total;
 
-  Cur cons;
-  {
-    long long bstart;
-    cons.b = find_seq(a, cap, lane, c0, &bstart);
-    const int L = clamp_len(a.lens[cons.b], cap);
-    cons.n = (L + 15) >> 4;
-    const long long off = c0 - bstart;
-    cons.g = static_cast<int>(off / cons.n);
-    cons.i = static_cast<int>(off - static_cast<long long>(cons.g) * cons.n);
-    cons.valid = true;
-  }
+  Cur cons = splitk::cursor_at(a, cap, lane, c0);
   Cur prod = cons;
   const long long nslots = c1 - c0;
 
@@ -333,46 +268,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_bf16_kernel(const Decod
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(256) merge_bf16_kernel(const DecodeArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int item = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
-  if (item >= a.B * a.Hq) return;
-  const int b = item / a.Hq, j = item - b * a.Hq;
-  const int g = j / G, hi = j - g * G;
-  const int cap = a.stride * a.P;
-  const long long total = prefix_cost(a, cap, lane, a.B);
-  const long long Q = quota(total, a.W);
-  const long long bstart = prefix_cost(a, cap, lane, b);
-  const int L = clamp_len(a.lens[b], cap);
-  const long long n = (L + 15) >> 4;
-  constexpr int PER = D / 32;
-  float o[PER];
-#pragma unroll
-  for (int e = 0; e < PER; ++e) o[e] = 0.f;
-  float m = kNegInf, l = 0.f;
-  if (n > 0) {
-    const long long cs = bstart + g * n, ce = cs + n;
-    const long long sid = static_cast<long long>(b) * a.Hkv + g;
-    for (long long w = cs / Q; w <= (ce - 1) / Q; ++w) {
-      const float* p = a.part + (static_cast<size_t>(w + sid) * G + hi) * kPartRow<D>;
-      const float pm = p[D], pl = p[D + 1];
-      if (!(pl > 0.f)) continue;
-      const float mn = fmaxf(m, pm);
-      const float fo = m == kNegInf ? 0.f : exp2f(m - mn), fp = exp2f(pm - mn);
-      l = l * fo + pl * fp;
-#pragma unroll
-      for (int e = 0; e < PER; ++e) o[e] = o[e] * fo + p[lane * PER + e] * fp;
-      m = mn;
-    }
-  }
-  float* out = a.out + (static_cast<size_t>(b) * a.Hq + j) * D + lane * PER;
-  const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-  for (int e = 0; e < PER; ++e) out[e] = o[e] * inv;
-  if (a.lse && lane == 0) a.lse[static_cast<size_t>(b) * a.Hq + j] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : kNegInf;
-}
-
-template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
   const int smem = static_cast<int>(sizeof(SmemBF<D, G>));
   static std::atomic<uint64_t> done[3];
@@ -389,7 +284,7 @@ cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  merge_bf16_kernel<D, G><<<(a.B * a.Hq + 7) / 8, 256, 0, st>>>(a);
+  splitk::merge_kernel<D, G><<<(a.B * a.Hq + 7) / 8, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 

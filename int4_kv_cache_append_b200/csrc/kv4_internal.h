@@ -27,7 +27,21 @@ struct AppendArgs {
   uint32_t signs[4];      // bit d: key dim d negated before the rotation (randomised-sign Hadamard)
   int rotate_v;           // values stored in the keys' rotated basis too
   int vbf;                // values stored as bf16 (KV4_VALUES_BF16)
+  // mixed bit-width keys (KV4_KEYS_MIXED)
+  const uint8_t* alloc;   // this layer's block allocation records (per KV head: sigma, widths)
+  int kbits, vbits;       // key bits per dimension (average), value bits per dimension
   uint32_t* err;
+};
+
+// Mixed bit-width key cache: one layer's block allocation is Hkv records of D/2 fp32 block scales
+// followed by D/2 uint8 widths, padded to 16 bytes; the records of all layers follow the pages.
+__host__ __device__ inline size_t mixed_alloc_record_bytes(int D) { return (static_cast<size_t>(D) / 2 * 5 + 15) & ~static_cast<size_t>(15); }
+
+struct ScoreArgs {
+  const void* K;          // [T][Hkv][D] keys to score
+  int k_dtype;
+  int T, Hkv, kbits;
+  uint8_t* alloc;         // this layer's allocation records (written)
 };
 
 struct DecodeArgs {
@@ -54,6 +68,9 @@ struct DecodeArgs {
   int vbf;                // values stored as bf16 (KV4_VALUES_BF16)
   int stall_test;         // kv4_debug_force_wait_timeout: every warp's first wait runs out
   uint64_t wait_ns;       // bounded-wait limit of the bulk-copy waits
+  // mixed bit-width keys (KV4_KEYS_MIXED)
+  const uint8_t* alloc;   // this layer's block allocation records
+  int kbits, vbits;       // key bits per dimension (average), value bits per dimension
   uint32_t* err;
 };
 
@@ -69,6 +86,12 @@ size_t decode_smem_bytes(int D, int G);
 size_t bf16_decode_smem_bytes(int D, int G);
 cudaError_t launch_decode_int4(DecodeArgs a, int D, int G, int ctas, cudaStream_t st);
 cudaError_t launch_decode_bf16(DecodeArgs a, int D, int G, int ctas, cudaStream_t st);
+
+// Mixed bit-width key cache (RoPE-block bit allocation): scoring + allocation, append, decode.
+cudaError_t launch_mixed_score(const ScoreArgs& a, int D, cudaStream_t st);
+cudaError_t launch_append_mixed(const AppendArgs& a, int D, cudaStream_t st);
+int mixed_decode_warps_per_cta();
+cudaError_t launch_decode_mixed(DecodeArgs a, int D, int G, int ctas, cudaStream_t st);
 
 // Counts every kernel launch the library issues.
 void note_launches(int n);

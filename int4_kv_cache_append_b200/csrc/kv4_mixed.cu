@@ -1,0 +1,669 @@
+// kv4_mixed.cu -- the mixed bit-width key cache: RoPE-block energy scoring and greedy bit
+// allocation, the fused append (block-scaled key codes and affine value codes, bit-packed into
+// the page slot), and decode attention over the packed pages.
+//
+// Method: "RoPE-Aware Bit Allocation for KV-Cache Quantization" (searcharxiv abstract).  Under
+// RoPE a key's share of a later logit is a sum over its two-dimensional frequency blocks, so the
+// key budget is split per block: for every layer and KV head a label-free energy score is taken
+// per RoPE block and integer bit widths are handed out greedily by marginal gain; the cache is
+// served from packed pages (the abstract's K3V3 serving path).  Conventions the abstract leaves
+// open (identical in the test oracle):
+//   - block b of a head is the rotate-half coordinate pair (b, b + D/2); its score is the fp64 sum
+//     over the scored keys of k[b]^2 + k[b + D/2]^2 in key order; its scale sigma_b is
+//     sqrt(score / 2T) rounded to fp32 (1 for a zero score);
+//   - one more bit for a block of score E at w bits gains E 4^-w; bits go one at a time to the
+//     largest gain (lowest block on ties), at most 8 per block, key_bits * D / 2 in all;
+//   - a key gets one fp16 scale s = rounded up of max |x_j| / sigma_j over coordinates with
+//     bits, and coordinate j of width w the mid-rise code floor((x_j / (sigma_j s) + 1) 2^(w-1))
+//     clamped to [0, 2^w - 1], reconstructed as s sigma_j ((2 code + 1) 2^-w - 1) (0 for w = 0);
+//   - a value gets the per-token affine code of the INT4 cache at value_bits bits: fp16 zero
+//     rounded down, fp16 range rounded up, code = rint((x - zero) / (range / (2^b - 1)));
+//   - codes are packed in coordinate order, least significant bit first, as one little-endian
+//     bit stream per vector; a page tile of one KV head holds P key rows, P value rows and P
+//     8-byte records (key scale, 0, value zero, value range), tiles ordered (page, head).
+//
+// Decode: the same flattened split-K as the BF16 baseline (16-position tiles of one (sequence, KV
+// head), three bulk copies per tile into a per-warp ring, LSE merge).  QK^T runs on m16n8k16 fp16
+// MMAs: the integer codes are exact fp16 A operands, the query enters as q_j sigma_j 2^(1-w_j) in
+// hi/lo fp16 halves (columns 2h, 2h+1 of the 8 N columns), and the code-independent part
+// sum_j q_j sigma_j (2^-w_j - 1) is added per head; the MMA's k index is permuted so that each
+// lane reads one contiguous bit range of a key row.  PV multiplies the value codes (exact fp16)
+// by p * step in hi/lo halves and adds sum_t p_t zero_t.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <math.h>
+
+#include "kv4_device.cuh"
+#include "kv4_internal.h"
+#include "kv4_layout.cuh"
+#include "kv4_splitk.cuh"
+
+namespace kv4 {
+namespace {
+
+constexpr unsigned FULL = 0xffffffffu;
+constexpr float kNegInf = -__builtin_huge_valf();
+constexpr int kAppendThreads = 256;
+
+__device__ __forceinline__ float load_elem(const void* base, int dtype, size_t i) {
+  if (dtype == KV4_F32) return reinterpret_cast<const float*>(base)[i];
+  if (dtype == KV4_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
+  return __half2float(reinterpret_cast<const __half*>(base)[i]);
+}
+
+template <int D>
+__device__ __forceinline__ const float* rec_sigma(const uint8_t* alloc, int g) {
+  return reinterpret_cast<const float*>(alloc + static_cast<size_t>(g) * mixed_alloc_record_bytes(D));
+}
+template <int D>
+__device__ __forceinline__ const uint8_t* rec_width(const uint8_t* alloc, int g) {
+  return alloc + static_cast<size_t>(g) * mixed_alloc_record_bytes(D) + (D / 2) * 4;
+}
+
+// ------------------------------------------------------------------ scoring + allocation
+
+// One block per KV head, one thread per RoPE block: the fp64 score in key order (so the
+// allocation, an integer decision, is the oracle's bit for bit), the block scale, then the greedy.
+template <int D>
+__global__ void __launch_bounds__(D / 2) mixed_score_kernel(ScoreArgs a) {
+  constexpr int NB = D / 2;
+  __shared__ double energy[NB];
+  const int g = blockIdx.x, b = threadIdx.x;
+  double e = 0.0;
+  for (int t = 0; t < a.T; ++t) {
+    const size_t row = (static_cast<size_t>(t) * a.Hkv + g) * D;
+    const double x0 = static_cast<double>(load_elem(a.K, a.k_dtype, row + b));
+    const double x1 = static_cast<double>(load_elem(a.K, a.k_dtype, row + b + NB));
+    e = __dadd_rn(e, __dadd_rn(__dmul_rn(x0, x0), __dmul_rn(x1, x1)));
+  }
+  energy[b] = e;
+  float* sigma = reinterpret_cast<float*>(a.alloc + static_cast<size_t>(g) * mixed_alloc_record_bytes(D));
+  uint8_t* width = a.alloc + static_cast<size_t>(g) * mixed_alloc_record_bytes(D) + NB * 4;
+  sigma[b] = (e > 0.0 && a.T > 0) ? __double2float_rn(__dsqrt_rn(__ddiv_rn(e, 2.0 * static_cast<double>(a.T)))) : 1.0f;
+  __syncthreads();
+  if (b == 0) {
+    uint8_t w[NB];
+    for (int i = 0; i < NB; ++i) w[i] = 0;
+    const int steps = a.kbits * NB;
+    for (int s = 0; s < steps; ++s) {
+      int best = -1;
+      double best_gain = 0.0;
+      for (int i = 0; i < NB; ++i) {
+        if (w[i] >= 8) continue;
+        const double gain = scalbn(energy[i], -2 * static_cast<int>(w[i]));  // E 4^-w, exact
+        if (best < 0 || gain > best_gain) {
+          best = i;
+          best_gain = gain;
+        }
+      }
+      w[best] += 1;
+    }
+    for (int i = 0; i < NB; ++i) width[i] = w[i];
+  }
+}
+
+// ------------------------------------------------------------------ append
+
+// Add `code` (w bits) at bit `o` of a row held as 32-bit words in shared memory.
+__device__ __forceinline__ void put_bits(uint32_t* row, int o, uint32_t code, int w) {
+  if (w == 0) return;
+  const int wi = o >> 5, sh = o & 31;
+  atomicOr(&row[wi], code << sh);
+  if (sh + w > 32) atomicOr(&row[wi + 1], code >> (32 - sh));
+}
+
+// One warp per (token, KV head); lane l holds coordinates l + 32 i.  Row buffers: per warp two
+// rows of up to D bytes (8 bits per coordinate) plus a guard word.
+template <int D>
+__global__ void __launch_bounds__(kAppendThreads) append_mixed_kernel(AppendArgs a) {
+  constexpr int NB = D / 2, NI = D / 32, RW = D / 4 + 1;
+  __shared__ uint32_t rows[kAppendThreads / 32][2][RW];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gw = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  if (gw >= a.T * a.Hkv) return;
+  const int t = gw / a.Hkv, g = gw - t * a.Hkv;
+  const int b = a.seq_slot[t], pos = a.pos[t];
+  if (b < 0 || b >= a.max_seqs || pos < 0 || pos / a.P >= a.stride) {
+    if (lane == 0) atomicOr(a.err, KV4_DEVERR_LENGTH);
+    return;
+  }
+  const int page = a.page_table[static_cast<size_t>(b) * a.stride + pos / a.P];
+  if (page < 0 || page >= a.max_pages) {
+    if (lane == 0) atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
+    return;
+  }
+  const float* sig = rec_sigma<D>(a.alloc, g);
+  const uint8_t* wid = rec_width<D>(a.alloc, g);
+  float k[NI], v[NI], sg[NI];
+  int w[NI];
+  const size_t in0 = (static_cast<size_t>(t) * a.Hkv + g) * D;
+#pragma unroll
+  for (int i = 0; i < NI; ++i) {
+    const int j = lane + 32 * i;
+    k[i] = load_elem(a.K, a.k_dtype, in0 + j);
+    v[i] = load_elem(a.V, a.v_dtype, in0 + j);
+    sg[i] = sig[j % NB];
+    w[i] = wid[j % NB];
+  }
+  uint32_t* krow = rows[warp][0];
+  uint32_t* vrow = rows[warp][1];
+  for (int i = lane; i < RW; i += 32) krow[i] = vrow[i] = 0u;
+
+  // bit offsets of the lane's coordinates: exclusive prefix of the block widths (coordinate j is
+  // block j mod D/2; the second half of the row starts after key_bits * D / 2 bits)
+  int pre[NI];
+  {
+    int run = 0;
+#pragma unroll
+    for (int c = 0; c < NB / 32; ++c) {
+      int x = w[c];  // block lane + 32 c is coordinate lane + 32 c
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(FULL, x, o);
+        if (lane >= o) x += y;
+      }
+      pre[c] = run + x - w[c];
+      run += __shfl_sync(FULL, x, 31);
+    }
+#pragma unroll
+    for (int i = NB / 32; i < NI; ++i) pre[i] = run + pre[i - NB / 32];
+  }
+
+  // key: one fp16 scale over the block-standardised coordinates that have bits
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < NI; ++i)
+    if (w[i] > 0) m = fmaxf(m, __fdiv_rn(fabsf(k[i]), sg[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+  const __half ksh = __float2half_ru(m);
+  const float sf = __half2float(ksh);
+  const bool kbad = !isfinite(sf);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < NI; ++i) {
+    uint32_t c = 0u;
+    if (w[i] > 0 && sf != 0.f && !kbad) {
+      const int top = (1 << w[i]) - 1;
+      const float d = __fmul_rn(sg[i], sf);
+      const float tq = __fdiv_rn(k[i], d);
+      const float u = __fmul_rn(__fadd_rn(tq, 1.0f), static_cast<float>(1 << (w[i] - 1)));
+      const float f = floorf(u);
+      c = f < 0.f ? 0u : (f > static_cast<float>(top) ? static_cast<uint32_t>(top) : static_cast<uint32_t>(f));
+    }
+    put_bits(krow, pre[i], c, w[i]);
+  }
+
+  // value: per-token affine code at vbits
+  float mn = v[0], mx = v[0];
+#pragma unroll
+  for (int i = 1; i < NI; ++i) {
+    mn = fminf(mn, v[i]);
+    mx = fmaxf(mx, v[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+  }
+  mn = mn + 0.0f;
+  mx = mx + 0.0f;
+  const __half vzh = __float2half_rd(mn);
+  const float zf = __half2float(vzh);
+  const __half vrh = __float2half_ru(__fsub_rn(mx, zf));
+  const float rf = __half2float(vrh);
+  const bool vbad = !isfinite(zf) || !isfinite(rf);
+  const int vtop = (1 << a.vbits) - 1;
+#pragma unroll
+  for (int i = 0; i < NI; ++i) {
+    uint32_t c = 0u;
+    if (rf != 0.f && !vbad) {
+      const float step = __fdiv_rn(rf, static_cast<float>(vtop));
+      const float r = rintf(__fdiv_rn(__fsub_rn(v[i], zf), step));
+      c = r < 0.f ? 0u : (r > static_cast<float>(vtop) ? static_cast<uint32_t>(vtop) : static_cast<uint32_t>(r));
+    }
+    put_bits(vrow, (lane + 32 * i) * a.vbits, c, a.vbits);
+  }
+  if (lane == 0 && (kbad || vbad)) atomicOr(a.err, KV4_DEVERR_RANGE);
+  __syncwarp();
+
+  const int KR = a.kbits * D / 8, VR = a.vbits * D / 8, pp = pos % a.P;
+  uint8_t* tile = a.pool + static_cast<size_t>(page) * a.page_bytes +
+                  static_cast<size_t>(g) * static_cast<size_t>(a.P) * (KR + VR + 8);
+  uint32_t* kdst = reinterpret_cast<uint32_t*>(tile + static_cast<size_t>(pp) * KR);
+  uint32_t* vdst = reinterpret_cast<uint32_t*>(tile + static_cast<size_t>(a.P) * KR + static_cast<size_t>(pp) * VR);
+  for (int i = lane; i < KR / 4; i += 32) kdst[i] = krow[i];
+  for (int i = lane; i < VR / 4; i += 32) vdst[i] = vrow[i];
+  if (lane == 0) {
+    const unsigned long long rec =
+        static_cast<unsigned long long>(__half_as_ushort(ksh)) |
+        (static_cast<unsigned long long>(__half_as_ushort(vzh)) << 32) |
+        (static_cast<unsigned long long>(__half_as_ushort(vrh)) << 48);
+    *reinterpret_cast<unsigned long long*>(tile + static_cast<size_t>(a.P) * (KR + VR) + static_cast<size_t>(pp) * 8) = rec;
+  }
+}
+
+// ------------------------------------------------------------------ decode
+
+constexpr int kWarps = 8;
+constexpr int kStages = 3;
+
+template <int D, int VB>
+struct MixedGeo {
+  static constexpr int NK = D / 16;              // k steps of QK^T, m blocks of PV
+  static constexpr int VR = VB * D / 8;          // value row bytes
+  static constexpr int VO = 16 * D;              // value rows in a stage (key rows hold <= D bytes)
+  static constexpr int PO = VO + 16 * VR;        // parameter records in a stage
+  static constexpr int STAGE = PO + 128;
+  static constexpr int DPL = D / 8;              // value dims per lane (PV rows gq, gq + 8)
+  static constexpr int WIN = DPL * VB;           // value bits per lane and token
+  static constexpr int NWA = (WIN + 31) / 32;    // aligned window words
+  static_assert(STAGE % 16 == 0, "stage size");
+};
+
+template <int D, int G, int VB>
+struct SmemMixed {
+  uint8_t ring[kWarps][kStages][MixedGeo<D, VB>::STAGE];
+  float qbuf[kWarps][G][D];
+  uint32_t ktab[kWarps][D];  // coordinate tig * D/4 + r at [4 r + tig]: bit offset | width << 16
+  uint64_t bar[kWarps][kStages];
+};
+
+__device__ __forceinline__ float exp2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// fp16 pair (x0, x1) or the pair of their fp16 rounding remainders
+__device__ __forceinline__ uint32_t split_h2(float x0, float x1, bool lo) {
+  const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+  __half r0 = h0, r1 = h1;
+  if (lo) {
+    r0 = __float2half_rn(x0 - __half2float(h0));
+    r1 = __float2half_rn(x1 - __half2float(h1));
+  }
+  return static_cast<uint32_t>(__half_as_ushort(r0)) | (static_cast<uint32_t>(__half_as_ushort(r1)) << 16);
+}
+
+// two integer codes (< 2048) as the exact fp16 pair (c0, c1): 1024 + c in the 0x6400 exponent, minus 1024
+__device__ __forceinline__ uint32_t codes_h2(uint32_t c0, uint32_t c1) {
+  const uint32_t h = c0 | (c1 << 16) | 0x64006400u;
+  __half2 v = *reinterpret_cast<const __half2*>(&h);
+  v = __hsub2(v, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// bits [p, p + w) of a bit array held in words aw (p and w compile-time after unrolling)
+template <int NW>
+__device__ __forceinline__ uint32_t take_bits(const uint32_t (&aw)[NW], int p, int w) {
+  const int wi = p >> 5, sh = p & 31;
+  uint32_t x = aw[wi] >> sh;
+  if (sh + w > 32 && wi + 1 < NW) x |= aw[wi + 1] << (32 - sh);
+  return x & ((1u << w) - 1u);
+}
+
+template <int D, int G, int VB>
+__global__ void __launch_bounds__(kWarps * 32, 1) decode_mixed_kernel(const DecodeArgs a) {
+  using MG = MixedGeo<D, VB>;
+  constexpr int NK = MG::NK, NB = D / 2, Q4 = D / 4;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  SmemMixed<D, G, VB>& sm = *reinterpret_cast<SmemMixed<D, G, VB>*>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tig = lane & 3;
+  const int wid = blockIdx.x * kWarps + warp;
+  const int cap = a.stride * a.P;
+  const int KR = a.kbits * D / 8;
+  const size_t tile_bytes = static_cast<size_t>(a.P) * (KR + MG::VR + 8);
+  uint64_t* bars = sm.bar[warp];
+  if (lane == 0) {
+    for (int i = 0; i < kStages; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  const long long total = splitk::prefix_cost(a, cap, lane, a.B);
+  const long long Q = splitk::quota(total, a.W);
+  const long long c0 = static_cast<long long>(wid) * Q;
+  if (c0 >= total) return;
+  const long long c1 = c0 + Q < total ? c0 + Q : total;
+  splitk::Cur cons = splitk::cursor_at(a, cap, lane, c0);
+  splitk::Cur prod = cons;
+  const long long nslots = c1 - c0;
+  const uint32_t stage_tx = static_cast<uint32_t>(16 * KR + 16 * MG::VR + 128);
+
+  auto issue = [&](const splitk::Cur& c, int st) {
+    const int lp = (c.i * 16) / a.P;
+    const int page = a.page_table[static_cast<size_t>(c.b) * a.stride + lp];
+    if (page >= 0 && page < a.max_pages) {
+      const int r0 = c.i * 16 - lp * a.P;
+      const uint8_t* tile = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(c.g) * tile_bytes;
+      uint8_t* dst = sm.ring[warp][st];
+      const uint64_t pol = l2_policy_evict_first();
+      mbar_arrive_expect_tx(&bars[st], stage_tx);
+      bulk_g2s_hint(dst, tile + static_cast<size_t>(r0) * KR, 16 * KR, &bars[st], pol);
+      bulk_g2s_hint(dst + MG::VO, tile + static_cast<size_t>(a.P) * KR + static_cast<size_t>(r0) * MG::VR, 16 * MG::VR,
+                    &bars[st], pol);
+      bulk_g2s_hint(dst + MG::PO, tile + static_cast<size_t>(a.P) * (KR + MG::VR) + static_cast<size_t>(r0) * 8, 128,
+                    &bars[st], pol);
+    } else {
+      atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
+      mbar_arrive_expect_tx(&bars[st], 0);
+    }
+  };
+
+  // Per (sequence, KV head): the key bit table, the scaled query fragments and the constant part
+  // of each head's logit.
+  uint32_t qf[NK][2];
+  float cst = 0.f, inv_scale = 1.f;
+  float* qb = &sm.qbuf[warp][0][0];
+  uint32_t* ktab = sm.ktab[warp];
+  auto load_query = [&](int b, int g) {
+    const float* sig = rec_sigma<D>(a.alloc, g);
+    const uint8_t* wid8 = rec_width<D>(a.alloc, g);
+    // exclusive prefix of the block widths; coordinate j >= D/2 starts after kbits * D/2 bits
+    int wv[NB / 32], pre[NB / 32];
+    int run = 0;
+#pragma unroll
+    for (int c = 0; c < NB / 32; ++c) {
+      wv[c] = wid8[lane + 32 * c];
+      int x = wv[c];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(FULL, x, o);
+        if (lane >= o) x += y;
+      }
+      pre[c] = run + x - wv[c];
+      run += __shfl_sync(FULL, x, 31);
+    }
+    float csum[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) csum[h] = 0.f;
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+      const int j = lane + 32 * i, c = (j % NB) / 32;
+      const int w = wv[c];
+      const int off = (j >= NB ? run : 0) + pre[c];
+      ktab[4 * (j % Q4) + j / Q4] = static_cast<uint32_t>(off) | (static_cast<uint32_t>(w) << 16);
+      const float sgm = sig[j % NB];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const size_t qi = (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G + h) * D + j;
+        const float qs = load_elem(a.q, a.q_dtype, qi) * sgm * a.qscale;
+        const float qq = w > 0 ? qs * __int_as_float((128 - w) << 23) : 0.f;      // qs 2^(1-w)
+        if (w > 0) csum[h] += qs * (__int_as_float((127 - w) << 23) - 1.0f);      // qs (2^-w - 1)
+        qb[h * D + j] = qq;
+        amax = fmaxf(amax, fabsf(qq));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) csum[h] += __shfl_xor_sync(FULL, csum[h], o);
+    cst = 0.f;
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+      if (tig == h) cst = csum[h];
+    // a power of two that brings the largest query weight near 2^8 (fp16 hi/lo keep ~22 bits)
+    int ex = 0;
+    if (amax > 0.f) frexpf(amax, &ex);
+    const float scale = ldexpf(1.f, 8 - ex);
+    inv_scale = ldexpf(1.f, ex - 8);
+    __syncwarp();
+    const int hh = gq >> 1;
+    const bool lo = gq & 1;
+#pragma unroll
+    for (int kb = 0; kb < NK; ++kb) {
+      const int j0 = tig * Q4 + 4 * kb;
+      if (hh < G) {
+        const float* qh = qb + hh * D;
+        qf[kb][0] = split_h2(qh[j0] * scale, qh[j0 + 1] * scale, lo);
+        qf[kb][1] = split_h2(qh[j0 + 2] * scale, qh[j0 + 3] * scale, lo);
+      } else {
+        qf[kb][0] = qf[kb][1] = 0u;
+      }
+    }
+    __syncwarp();
+  };
+
+  float oacc[NK][4];
+  float m_run, l_part, pz;
+  auto reset = [&]() {
+#pragma unroll
+    for (int mb = 0; mb < NK; ++mb) oacc[mb][0] = oacc[mb][1] = oacc[mb][2] = oacc[mb][3] = 0.f;
+    m_run = kNegInf;
+    l_part = 0.f;
+    pz = 0.f;
+  };
+  auto flush = [&](const splitk::Cur& c) {
+    float l = l_part, z = pz;
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l += __shfl_xor_sync(FULL, l, o);
+      z += __shfl_xor_sync(FULL, z, o);
+    }
+    if (tig < G) {
+      const long long sid = static_cast<long long>(c.b) * a.Hkv + c.g;
+      float* p = a.part + (static_cast<size_t>(wid + sid) * G + tig) * kPartRow<D>;
+#pragma unroll
+      for (int mb = 0; mb < NK; ++mb) {
+        const int d = MG::DPL * gq + 2 * mb;
+        *reinterpret_cast<float2*>(p + d) = make_float2(oacc[mb][0] + oacc[mb][1] + z, oacc[mb][2] + oacc[mb][3] + z);
+      }
+      if (gq == 0) *reinterpret_cast<float2*>(p + D) = make_float2(m_run, l);
+    }
+  };
+
+  int issued = 0;
+  if (lane == 0) {
+    for (int k = 0; k < kStages - 1 && k < nslots; ++k) {
+      issue(prod, k);
+      ++prod.i;
+      splitk::settle(a, cap, prod);
+      ++issued;
+    }
+  }
+  reset();
+  load_query(cons.b, cons.g);
+  bool failed = false;
+  long long k = 0;
+  for (; k < nslots; ++k) {
+    if (lane == 0 && issued < nslots) {
+      fence_proxy_async_smem();
+      issue(prod, static_cast<int>((k + kStages - 1) % kStages));
+      ++prod.i;
+      splitk::settle(a, cap, prod);
+      ++issued;
+    }
+    const int st = static_cast<int>(k % kStages);
+    const bool ok = mbar_wait_bounded(&bars[st], static_cast<uint32_t>((k / kStages) & 1), a.err);
+    if (__any_sync(FULL, !ok)) {
+      failed = true;
+      break;
+    }
+    const uint8_t* buf = sm.ring[warp][st];
+    const int lp = (cons.i * 16) / a.P;
+    const int page = a.page_table[static_cast<size_t>(cons.b) * a.stride + lp];
+    const bool page_ok = page >= 0 && page < a.max_pages;
+    const int L = splitk::clamp_len(a.lens[cons.b], cap);
+    const int i0 = cons.i * 16;
+    const bool v0 = page_ok && tig < G && i0 + gq < L, v1 = page_ok && tig < G && i0 + gq + 8 < L;
+
+    // QK^T.  Lane (gq, tig) reads, in rows gq and gq + 8, the coordinates tig * D/4 + [0, D/4):
+    // k index (2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9) of step kb is coordinate tig * D/4 + 4 kb
+    // + (0, 1, 2, 3), and the query fragments use the same map.
+    const uint32_t* r0w = reinterpret_cast<const uint32_t*>(buf + gq * KR);
+    const uint32_t* r1w = reinterpret_cast<const uint32_t*>(buf + (gq + 8) * KR);
+    float S[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kb = 0; kb < NK; ++kb) {
+      uint32_t c0v[4], c1v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t ent = ktab[4 * (4 * kb + e) + tig];
+        const int off = static_cast<int>(ent & 0xffffu), w = static_cast<int>(ent >> 16);
+        const int wi = off >> 5, sh = off & 31;
+        const uint32_t mask = (1u << w) - 1u;
+        c0v[e] = __funnelshift_r(r0w[wi], r0w[wi + 1], sh) & mask;
+        c1v[e] = __funnelshift_r(r1w[wi], r1w[wi + 1], sh) & mask;
+      }
+      mma_f16(S, codes_h2(c0v[0], c0v[1]), codes_h2(c1v[0], c1v[1]), codes_h2(c0v[2], c0v[3]),
+              codes_h2(c1v[2], c1v[3]), qf[kb][0], qf[kb][1]);
+    }
+    const __half* prm = reinterpret_cast<const __half*>(buf + MG::PO);
+    const float s0 = v0 ? __half2float(prm[4 * gq]) : 0.f, s1 = v1 ? __half2float(prm[4 * (gq + 8)]) : 0.f;
+    const float lg0 = v0 ? s0 * fmaf(S[0] + S[1], inv_scale, cst) : kNegInf;
+    const float lg1 = v1 ? s1 * fmaf(S[2] + S[3], inv_scale, cst) : kNegInf;
+
+    float tm = fmaxf(lg0, lg1);
+    tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, 4));
+    tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, 8));
+    tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, 16));
+    const float mn = fmaxf(m_run, tm);
+    const bool grow = mn > m_run;
+    if (__any_sync(FULL, grow)) {
+      const float alpha = grow ? (m_run == kNegInf ? 0.f : exp2_fast(m_run - mn)) : 1.f;
+#pragma unroll
+      for (int mb = 0; mb < NK; ++mb) {
+        oacc[mb][0] *= alpha;
+        oacc[mb][1] *= alpha;
+        oacc[mb][2] *= alpha;
+        oacc[mb][3] *= alpha;
+      }
+      l_part *= alpha;
+      pz *= alpha;
+      m_run = mn;
+    }
+    const float mu = m_run == kNegInf ? 0.f : m_run;
+    const float p0 = v0 ? exp2_fast(lg0 - mu) : 0.f, p1 = v1 ? exp2_fast(lg1 - mu) : 0.f;
+    l_part += p0 + p1;
+    if (v0) pz = fmaf(p0, __half2float(prm[4 * gq + 2]), pz);
+    if (v1) pz = fmaf(p1, __half2float(prm[4 * (gq + 8) + 2]), pz);
+
+    // PV.  B: p * step of tokens (2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9) for column gq = (head
+    // gq / 2, hi or lo half); A: value codes of dims gq * D/8 + [0, D/8) (rows gq and gq + 8 of
+    // m block mb are dims gq * D/8 + 2 mb and + 1) for the same tokens.
+    const int hh = gq >> 1;
+    const bool lo = gq & 1;
+    const int src0 = 8 * tig + hh, src1 = src0 + 4;
+    const float x0 = __shfl_sync(FULL, p0, src0), x1 = __shfl_sync(FULL, p0, src1);
+    const float x2 = __shfl_sync(FULL, p1, src0), x3 = __shfl_sync(FULL, p1, src1);
+    const int tk[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
+    const float vstep = 1.0f / static_cast<float>((1 << VB) - 1);
+    float ps[4];
+    const float xs[4] = {x0, x1, x2, x3};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const bool vt = page_ok && i0 + tk[u] < L;
+      ps[u] = vt ? xs[u] * (__half2float(prm[4 * tk[u] + 3]) * vstep) : 0.f;
+    }
+    uint32_t b0 = 0u, b1 = 0u;
+    if (hh < G) {
+      b0 = split_h2(ps[0], ps[1], lo);
+      b1 = split_h2(ps[2], ps[3], lo);
+    }
+    // value codes of the lane's dims for its four tokens
+    uint32_t cv[4][MG::DPL];
+    const int bit0 = gq * MG::WIN;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t* vr = reinterpret_cast<const uint32_t*>(buf + MG::VO + tk[u] * MG::VR);
+      uint32_t raw[MG::NWA + 1], aw[MG::NWA];
+#pragma unroll
+      for (int x = 0; x <= MG::NWA; ++x) raw[x] = vr[(bit0 >> 5) + x];
+#pragma unroll
+      for (int x = 0; x < MG::NWA; ++x) aw[x] = __funnelshift_r(raw[x], raw[x + 1], bit0 & 31);
+#pragma unroll
+      for (int d = 0; d < MG::DPL; ++d) cv[u][d] = take_bits(aw, d * VB, VB);
+    }
+    // Slots past L (or of a bad page) hold arbitrary bytes, but their codes are finite integers
+    // and their B entries are exactly zero, so they add nothing.
+#pragma unroll
+    for (int mb = 0; mb < NK; ++mb)
+      mma_f16(oacc[mb], codes_h2(cv[0][2 * mb], cv[1][2 * mb]), codes_h2(cv[0][2 * mb + 1], cv[1][2 * mb + 1]),
+              codes_h2(cv[2][2 * mb], cv[3][2 * mb]), codes_h2(cv[2][2 * mb + 1], cv[3][2 * mb + 1]), b0, b1);
+    __syncwarp();
+
+    splitk::Cur nxt = cons;
+    ++nxt.i;
+    splitk::settle(a, cap, nxt);
+    const bool more = k + 1 < nslots;
+    if (!more || nxt.b != cons.b || nxt.g != cons.g) {
+      flush(cons);
+      reset();
+      if (more) load_query(nxt.b, nxt.g);
+    }
+    cons = nxt;
+  }
+  if (failed) {
+    issued = __shfl_sync(FULL, issued, 0);
+    for (long long j = k; j < issued; ++j)
+      mbar_wait_bounded(&bars[j % kStages], static_cast<uint32_t>((j / kStages) & 1), a.err);
+  }
+}
+
+template <int D, int G, int VB>
+cudaError_t launch_dgv(const DecodeArgs& a, int ctas, cudaStream_t st) {
+  const int smem = static_cast<int>(sizeof(SmemMixed<D, G, VB>));
+  static std::atomic<uint64_t> done;
+  cudaError_t e = ensure_smem_limit(decode_mixed_kernel<D, G, VB>, smem, done);
+  if (e != cudaSuccess) return e;
+  decode_mixed_kernel<D, G, VB><<<ctas, kWarps * 32, smem, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  splitk::merge_kernel<D, G><<<(a.B * a.Hq + 7) / 8, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, int G>
+cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
+  switch (a.vbits) {
+    case 2: return launch_dgv<D, G, 2>(a, ctas, st);
+    case 3: return launch_dgv<D, G, 3>(a, ctas, st);
+    case 4: return launch_dgv<D, G, 4>(a, ctas, st);
+    case 8: return launch_dgv<D, G, 8>(a, ctas, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int D>
+cudaError_t launch_append_d(const AppendArgs& a, cudaStream_t st) {
+  const int warps = a.T * a.Hkv;
+  append_mixed_kernel<D><<<(warps + kAppendThreads / 32 - 1) / (kAppendThreads / 32), kAppendThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_mixed_score(const ScoreArgs& a, int D, cudaStream_t st) {
+  note_launches(1);
+  if (D == 128) mixed_score_kernel<128><<<a.Hkv, 64, 0, st>>>(a);
+  else mixed_score_kernel<64><<<a.Hkv, 32, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_mixed(const AppendArgs& a, int D, cudaStream_t st) {
+  if (a.T <= 0) return cudaSuccess;
+  note_launches(1);
+  return D == 128 ? launch_append_d<128>(a, st) : launch_append_d<64>(a, st);
+}
+
+int mixed_decode_warps_per_cta() { return kWarps; }
+
+cudaError_t launch_decode_mixed(DecodeArgs a, int D, int G, int ctas, cudaStream_t st) {
+  a.W = ctas * kWarps;
+  note_launches(2);
+  if (D == 128) {
+    if (G == 4) return launch_dg<128, 4>(a, ctas, st);
+    if (G == 2) return launch_dg<128, 2>(a, ctas, st);
+    return launch_dg<128, 1>(a, ctas, st);
+  }
+  if (G == 4) return launch_dg<64, 4>(a, ctas, st);
+  if (G == 2) return launch_dg<64, 2>(a, ctas, st);
+  return launch_dg<64, 1>(a, ctas, st);
+}
+
+}  // namespace kv4

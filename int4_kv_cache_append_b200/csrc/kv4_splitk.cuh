@@ -1,0 +1,145 @@
+// kv4_splitk.cuh -- the flattened split-K schedule shared by the single-region decode kernels (the
+// BF16 baseline and the mixed bit-width key cache): every (sequence, KV head) is cut into
+// 16-position tiles, the tiles of all pairs are laid end to end in (sequence, head, tile) order,
+// and warp w of W takes the w-th run of ceil(total / W) of them.  A warp writes one partial row
+// group (o[D], m, l) per (sequence, head) segment it touches, at index w + b * Hkv + g (unique:
+// consecutive warps overlap in at most one segment); the merge kernel finds the warps that
+// covered a pair from the same arithmetic and combines their partials by log-sum-exp.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "kv4_internal.h"
+#include "kv4_layout.cuh"
+
+namespace kv4 {
+namespace splitk {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr float kNegInfF = -__builtin_huge_valf();
+
+__device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
+__device__ __forceinline__ long long seq_cost(const DecodeArgs& a, int L) {
+  return static_cast<long long>(a.Hkv) * ((L + 15) >> 4);
+}
+
+__device__ __forceinline__ long long warp_incl_scan(long long v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long t = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += t;
+  }
+  return v;
+}
+
+// tiles of sequences [0, upto)
+__device__ __forceinline__ long long prefix_cost(const DecodeArgs& a, int cap, int lane, int upto) {
+  long long run = 0;
+  for (int base = 0; base < upto; base += 32) {
+    const int b = base + lane;
+    const long long c = b < upto ? seq_cost(a, clamp_len(a.lens[b], cap)) : 0;
+    run += __shfl_sync(kFull, warp_incl_scan(c, lane), 31);
+  }
+  return run;
+}
+
+// the sequence holding flattened tile c, and the index of its first tile
+__device__ __forceinline__ int find_seq(const DecodeArgs& a, int cap, int lane, long long c, long long* bstart) {
+  long long run = 0;
+  for (int base = 0; base < a.B; base += 32) {
+    const int b = base + lane;
+    const long long cb = b < a.B ? seq_cost(a, clamp_len(a.lens[b], cap)) : 0;
+    const long long incl = warp_incl_scan(cb, lane);
+    const long long tot = __shfl_sync(kFull, incl, 31);
+    if (c < run + tot) {
+      const unsigned m = __ballot_sync(kFull, c < run + incl);
+      const int l = __ffs(m) - 1;
+      *bstart = run + __shfl_sync(kFull, incl - cb, l);
+      return base + l;
+    }
+    run += tot;
+  }
+  *bstart = run;
+  return a.B;
+}
+
+__device__ __forceinline__ long long quota(long long total, int W) {
+  const long long q = (total + W - 1) / W;
+  return q < 1 ? 1 : q;
+}
+
+// position in the flattened order: sequence b, KV head g, tile i of n
+struct Cur {
+  int b, g, i, n;
+  bool valid;
+};
+
+__device__ __forceinline__ void settle(const DecodeArgs& a, int cap, Cur& c) {
+  while (c.b < a.B && c.i >= c.n) {
+    c.i = 0;
+    if (++c.g == a.Hkv) {
+      c.g = 0;
+      if (++c.b < a.B) c.n = (clamp_len(a.lens[c.b], cap) + 15) >> 4;
+    }
+  }
+  c.valid = c.b < a.B;
+}
+
+// The cursor of flattened tile c0.
+__device__ __forceinline__ Cur cursor_at(const DecodeArgs& a, int cap, int lane, long long c0) {
+  Cur c;
+  long long bstart;
+  c.b = find_seq(a, cap, lane, c0, &bstart);
+  const int L = clamp_len(a.lens[c.b], cap);
+  c.n = (L + 15) >> 4;
+  const long long off = c0 - bstart;
+  c.g = static_cast<int>(off / c.n);
+  c.i = static_cast<int>(off - static_cast<long long>(c.g) * c.n);
+  c.valid = true;
+  return c;
+}
+
+// One warp per (sequence, query head): combine the partials of the warps that covered the pair.
+template <int D, int G>
+__global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int item = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  if (item >= a.B * a.Hq) return;
+  const int b = item / a.Hq, j = item - b * a.Hq;
+  const int g = j / G, hi = j - g * G;
+  const int cap = a.stride * a.P;
+  const long long total = prefix_cost(a, cap, lane, a.B);
+  const long long Q = quota(total, a.W);
+  const long long bstart = prefix_cost(a, cap, lane, b);
+  const int L = clamp_len(a.lens[b], cap);
+  const long long n = (L + 15) >> 4;
+  constexpr int PER = D / 32;
+  float o[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) o[e] = 0.f;
+  float m = kNegInfF, l = 0.f;
+  if (n > 0) {
+    const long long cs = bstart + g * n, ce = cs + n;
+    const long long sid = static_cast<long long>(b) * a.Hkv + g;
+    for (long long w = cs / Q; w <= (ce - 1) / Q; ++w) {
+      const float* p = a.part + (static_cast<size_t>(w + sid) * G + hi) * kPartRow<D>;
+      const float pm = p[D], pl = p[D + 1];
+      if (!(pl > 0.f)) continue;
+      const float mn = fmaxf(m, pm);
+      const float fo = m == kNegInfF ? 0.f : exp2f(m - mn), fp = exp2f(pm - mn);
+      l = l * fo + pl * fp;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) o[e] = o[e] * fo + p[lane * PER + e] * fp;
+      m = mn;
+    }
+  }
+  float* out = a.out + (static_cast<size_t>(b) * a.Hq + j) * D + lane * PER;
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) out[e] = o[e] * inv;
+  if (a.lse && lane == 0) a.lse[static_cast<size_t>(b) * a.Hq + j] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : kNegInfF;
+}
+
+}  // namespace splitk
+}  // namespace kv4

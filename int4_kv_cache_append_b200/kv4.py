@@ -19,7 +19,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkv4.so")
 
-KV4_OK, KV4_ERR_INVALID_ARG, KV4_ERR_UNSUPPORTED, KV4_ERR_WORKSPACE, KV4_ERR_CUDA, KV4_ERR_DEVICE = range(6)
+(KV4_OK, KV4_ERR_INVALID_ARG, KV4_ERR_UNSUPPORTED, KV4_ERR_WORKSPACE, KV4_ERR_CUDA, KV4_ERR_DEVICE,
+ KV4_ERR_NO_ALLOCATION) = range(7)
 KV4_F32, KV4_BF16, KV4_F16 = 0, 1, 2
 KV4_DEVERR_PAGE_RANGE, KV4_DEVERR_WAIT_LIMIT, KV4_DEVERR_LENGTH, KV4_DEVERR_RANGE, KV4_DEVERR_RECORD = 0x1, 0x2, 0x4, 0x8, 0x10
 
@@ -29,7 +30,8 @@ SYMBOLS = (
     "kv4_decode_attn", "kv4_decode_attn_static", "kv4_set_decode_overlap", "kv4_debug_force_wait_timeout",
     "kv4_set_rotation_signs", "kv4_set_value_rotation", "kv4_bf16_query_sizes", "kv4_bf16_cache_init",
     "kv4_bf16_append", "kv4_bf16_decode_workspace_bytes", "kv4_bf16_decode_attn", "kv4_get_device_error",
-    "kv4_launch_count", "kv4_status_string", "kv4_version",
+    "kv4_launch_count", "kv4_status_string", "kv4_version", "kv4_allocate_key_bits", "kv4_set_key_allocation",
+    "kv4_get_key_allocation",
 )
 
 
@@ -39,13 +41,13 @@ class KV4Error(RuntimeError):
         self.status = status
 
 
-KV4_VALUES_INT4, KV4_VALUES_BF16 = 0, 1
+KV4_VALUES_INT4, KV4_VALUES_BF16, KV4_KEYS_MIXED = 0, 1, 2
 
 
 class kv4_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "num_layers", "num_q_heads", "num_kv_heads", "head_dim", "page_size", "num_sinks",
-        "recent_window", "hadamard_block", "max_seqs", "max_pages", "value_format")]
+        "recent_window", "hadamard_block", "max_seqs", "max_pages", "value_format", "key_bits", "value_bits")]
 
 
 def _load():
@@ -76,6 +78,9 @@ def _load():
         "kv4_launch_count": (U, []),
         "kv4_status_string": (ctypes.c_char_p, [I]),
         "kv4_version": (I, []),
+        "kv4_allocate_key_bits": (I, [P, I, I, P, I, P]),
+        "kv4_set_key_allocation": (I, [P, I, P, P, P]),
+        "kv4_get_key_allocation": (I, [P, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -197,6 +202,32 @@ def kv4_debug_force_wait_timeout(handle, enable: bool):
     _check("kv4_debug_force_wait_timeout", lib.kv4_debug_force_wait_timeout(handle, 1 if enable else 0))
 
 
+def kv4_allocate_key_bits(handle, layer, T, K, k_dtype, stream=None):
+    """Mixed bit-width keys: score the T keys K [T][Hkv][D] per RoPE block and allocate the layer's
+    key bits on the device."""
+    _check("kv4_allocate_key_bits", lib.kv4_allocate_key_bits(handle, layer, T, _ptr(K), k_dtype, _stream(stream)))
+
+
+def kv4_set_key_allocation(handle, layer, widths, sigma, stream=None):
+    """Mixed bit-width keys: set a layer's allocation from host arrays widths uint8 [Hkv][D/2] and
+    sigma float32 [Hkv][D/2] (NumPy)."""
+    import numpy as np
+    w = np.ascontiguousarray(widths, np.uint8)
+    sg = np.ascontiguousarray(sigma, np.float32)
+    _check("kv4_set_key_allocation", lib.kv4_set_key_allocation(handle, layer, w.ctypes.data_as(ctypes.c_void_p),
+                                                                sg.ctypes.data_as(ctypes.c_void_p), _stream(stream)))
+
+
+def kv4_get_key_allocation(handle, layer, Hkv, D, stream=None):
+    """Mixed bit-width keys: (widths uint8 [Hkv][D/2], sigma float32 [Hkv][D/2]) of a layer."""
+    import numpy as np
+    w = np.zeros((Hkv, D // 2), np.uint8)
+    sg = np.zeros((Hkv, D // 2), np.float32)
+    _check("kv4_get_key_allocation", lib.kv4_get_key_allocation(handle, layer, w.ctypes.data_as(ctypes.c_void_p),
+                                                                sg.ctypes.data_as(ctypes.c_void_p), _stream(stream)))
+    return w, sg
+
+
 def kv4_bf16_query_sizes(cfg: kv4_config) -> int:
     pool = ctypes.c_size_t()
     _check("kv4_bf16_query_sizes", lib.kv4_bf16_query_sizes(ctypes.byref(cfg), ctypes.byref(pool)))
@@ -256,11 +287,20 @@ class Geometry:
     max_seqs: int
     max_pages: int
     value_format: int = KV4_VALUES_INT4
+    key_bits: int = 0      # KV4_KEYS_MIXED only
+    value_bits: int = 0    # KV4_KEYS_MIXED only
 
     def c(self) -> kv4_config:
         return kv4_config(self.num_layers, self.num_q_heads, self.num_kv_heads, self.head_dim, self.page_size,
                           self.num_sinks, self.recent_window, self.hadamard_block, self.max_seqs, self.max_pages,
-                          self.value_format)
+                          self.value_format, self.key_bits, self.value_bits)
+
+    def page_bytes(self) -> int:
+        """Bytes of one page (all KV heads) of one layer."""
+        D, P, H = self.head_dim, self.page_size, self.num_kv_heads
+        if self.value_format == KV4_KEYS_MIXED:
+            return H * P * ((self.key_bits + self.value_bits) * D // 8 + 8)
+        return H * P * (D // 2 + 4 + 2 * D if self.value_format == KV4_VALUES_BF16 else D + 8)
 
 
 class Cache:
@@ -279,9 +319,17 @@ class Cache:
         self._ws = None
 
     def layer_views(self, layer: int):
+        """(pages of the layer, side cache of the layer) as uint8 views."""
         pool_b, side_b = kv4_query_sizes(self.cfg)
-        pl, sl = pool_b // self.geo.num_layers, side_b // self.geo.num_layers
+        pl, sl = self.geo.page_bytes() * self.geo.max_pages, side_b // self.geo.num_layers
         return self.pool[layer * pl:(layer + 1) * pl], self.side[layer * sl:(layer + 1) * sl]
+
+    def allocate_key_bits(self, layer, K, stream=None):
+        """Mixed bit-width keys: allocate the layer's key bits from keys K [T][Hkv][D]."""
+        kv4_allocate_key_bits(self.handle, layer, int(K.shape[0]), K, dtype_code(K), stream)
+
+    def key_allocation(self, layer):
+        return kv4_get_key_allocation(self.handle, layer, self.geo.num_kv_heads, self.geo.head_dim)
 
     def append(self, layer, K, V, seq_slot, pos, lens_after, page_table, stream=None):
         kv4_append(self.handle, layer, int(seq_slot.numel()), K, dtype_code(K), V, dtype_code(V), seq_slot, pos,
