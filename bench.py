@@ -46,7 +46,10 @@ INPUTS = ("synthetic, seeded: K, V, q are Irwin-Hall N(0,1) stand-ins (sum of 12
 PER_CONFIG = (("tiny", {}, "37 KB of KV per decode: bound by launch and fixed cost, not by HBM"),
               ("qwen3-4b-decode", {}, None), ("qwen3-4b-decode", {"h": 1}, "h = 1: no rotation (naive INT4)"),
               ("async-refill", {}, None), ("async-refill", {"values": "bf16"}, "K-INT4 / V-BF16: bf16 values"),
-              ("long-context", {}, None), ("long-context", {"h": 1}, "h = 1: no rotation (naive INT4)"))
+              ("long-context", {}, None), ("long-context", {"h": 1}, "h = 1: no rotation (naive INT4)"),
+              ("async-refill", {"mixed": (3, 3)}, "mixed bit-width keys K3V3 (RoPE-block bit allocation)"),
+              ("async-refill", {"mixed": (4, 4)}, "mixed bit-width keys K4V4: the bytes of the INT4 cache"),
+              ("long-context", {"mixed": (3, 3)}, "mixed bit-width keys K3V3 (RoPE-block bit allocation)"))
 
 
 def parse():
@@ -66,6 +69,9 @@ def parse():
                     help="override w, the INT8 recent window (-1: every position, i.e. all-INT8 KV8)")
     ap.add_argument("--values", choices=["int4", "bf16"], default="int4",
                     help="value storage: INT4 (KV4) or bf16 (the K-INT4 / V-BF16 variant)")
+    ap.add_argument("--mixed", default=None, metavar="KB,VB",
+                    help="mixed bit-width key cache with KB average key bits and VB value bits per dimension "
+                         "(RoPE-block bit allocation; no side cache, no rotation)")
     ap.add_argument("--no-bf16", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
@@ -105,6 +111,9 @@ def make_wl(args):
             wl = dataclasses.replace(wl, h=h, name=f"{wl.name}-h{h}")
     if getattr(args, "values", "int4") == "bf16":
         wl = dataclasses.replace(wl, value_format=1, name=f"{wl.name}-vbf16")
+    if getattr(args, "mixed", None):
+        kb, vb = (int(x) for x in args.mixed.split(","))
+        wl = mixed_variant(wl, kb, vb)
     # sink / recent budgets (KV4-RL "Main Findings": s/w sweep; KV8 = every position in INT8)
     s, w = getattr(args, "sinks", None), getattr(args, "recent", None)
     if s is not None or w is not None:
@@ -112,6 +121,15 @@ def make_wl(args):
         w = wl.w if w is None else (int(wl.max_lens.max()) if w < 0 else w)
         wl = dataclasses.replace(wl, s=s, w=w, name=f"{wl.name}-s{s}-w{w}")
     return wl
+
+
+def mixed_variant(wl, kb: int, vb: int):
+    """The workload on the mixed bit-width key cache: keys at kb bits per dimension on average,
+    split over RoPE blocks; values at vb bits; outliers on whole RoPE blocks (queries alike); no
+    side cache and no rotation."""
+    import dataclasses
+    return dataclasses.replace(wl, s=0, w=0, h=1, value_format=2, key_bits=kb, value_bits=vb, rope_outliers=True,
+                               name=f"{wl.name}-k{kb}v{vb}")
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -380,7 +398,8 @@ def run_kv4(args, world, rank, local, wl=None, light=False):
         geo = H.geometry(wl, layers=layers, value_format=0 if bf16 else wl.value_format)
         cache = kv4.BF16Cache(geo, device=dev) if bf16 else kv4.Cache(geo, device=dev)
         for layer in range(layers):
-            H.prefill(cache, wl, layer, lens0, upto=lens0 - 1, bf16_pool=bf16)
+            H.prefill(cache, wl, layer, lens0, upto=lens0 - 1, bf16_pool=bf16,
+                      allocate=not bf16 and wl.value_format == kv4.KV4_KEYS_MIXED)
         factor = torch.from_numpy(wl.factor()).to(dev)
         bt = torch.arange(B, dtype=torch.int32, device=dev)
         pos = torch.from_numpy(lens0 - 1).to(dev)
@@ -538,7 +557,9 @@ def run_kv4(args, world, rank, local, wl=None, light=False):
     cache, ins, bt = setup(False, resident)
     # lens and page_table are written before the step, never by the append: the decode may build
     # its schedule while the append runs
-    kv4.kv4_set_decode_overlap(cache.handle, 0 if args.no_overlap else 1)
+    mixed = wl.value_format == kv4.KV4_KEYS_MIXED
+    if not mixed:
+        kv4.kv4_set_decode_overlap(cache.handle, 0 if args.no_overlap else 1)
     S = Steps(cache, ins, bt, False, resident)
     total_ms, dec_ms, app_ms, launches, clocks, klens = timed(S, steps, warmup, sampler=ClockSampler(uuid),
                                                                soak_s=0.3 if light else args.soak_s)
@@ -560,7 +581,8 @@ def run_kv4(args, world, rank, local, wl=None, light=False):
     achieved = alg_bytes / (dec_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": profiled_traffic(wl.name),
-            "kernel": "decode_int4_kernel + merge_int4_kernel (kv4_decode_attn: split-K tiles, then LSE merge)",
+            "kernel": ("decode_mixed_kernel + merge_kernel (kv4_decode_attn on the mixed bit-width key cache)" if mixed
+                       else "decode_int4_kernel + merge_int4_kernel (kv4_decode_attn: split-K tiles, then LSE merge)"),
             "bytes_per_launch": int(alg_bytes), "kv_bytes_per_launch": int(kv_bytes), "decode_ms": round(dec_ms, 5),
             "peak_source": f"{peak_kind} MEASURED_PEAKS.json hbm_gbs" if peak_kind == "measured" else "fallback"}
     spec_frac = achieved / 8000.0
@@ -712,9 +734,12 @@ def run_kv4(args, world, rank, local, wl=None, light=False):
                        "s": wl.s, "w": wl.w, "h": wl.h, "len_mean": round(float(lens0.mean()), 1),
                        "len_max": int(lens0.max()), "layers_per_step": per_step,
                        "growth_per_step": 1 if grow else 0,
-                       "kv_dtype": ("int4 K + bf16 V pages, int8 K + bf16 V side cache" if wl.value_format
+                       "kv_dtype": (f"packed K{wl.key_bits} (RoPE-block widths) V{wl.value_bits} pages" if mixed
+                                    else "int4 K + bf16 V pages, int8 K + bf16 V side cache" if wl.value_format
                                     else "int4 pages + int8 side cache"),
-                       "compute": "QK^T int8 MMA (exact int32), PV f16 MMA with f32 accumulate, f32 softmax",
+                       "compute": ("QK^T and PV f16 MMA on integer codes with hi/lo f16 weights, f32 accumulate, "
+                                   "f32 softmax" if mixed else
+                                   "QK^T int8 MMA (exact int32), PV f16 MMA with f32 accumulate, f32 softmax"),
                        "l2": f"inputs larger than L2: {resident} resident layers cycled, {resident_gb:.2f} GB of KV "
                              f"between reuses",
                        "parallelism": f"dp{world} (independent batches per GPU, no collective)",
@@ -767,6 +792,8 @@ def main():
                     wl = dataclasses.replace(wl, h=over["h"], name=f"{wl.name}-h{over['h']}")
                 if over.get("values") == "bf16":
                     wl = dataclasses.replace(wl, value_format=1, name=f"{wl.name}-vbf16")
+                if "mixed" in over:
+                    wl = mixed_variant(wl, *over["mixed"])
                 per[wl.name] = per_config_record(run_kv4(args, world, rank, local, wl=wl, light=True), note)
             line["per_config"] = per
         if line is not None and rank == 0:

@@ -125,7 +125,12 @@ kv4_status dtype_ok_q(kv4_dtype d) {
 
 size_t align16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
-int decode_ctas_full(int format, int sms) { return format == FMT_INT4 ? kv4::decode_ctas_per_sm() * sms : sms; }
+int decode_ctas_full(const kv4_cache* c, int sms) {
+  if (c->format == FMT_INT4) return kv4::decode_ctas_per_sm() * sms;
+  if (c->format == FMT_MIXED)
+    return kv4::mixed_decode_ctas_per_sm(c->cfg.head_dim, c->cfg.num_q_heads / c->cfg.num_kv_heads, c->cfg.value_bits) * sms;
+  return sms;
+}
 
 int warps_per_cta(int format) {
   return format == FMT_INT4 ? kv4::decode_warps_per_cta()
@@ -217,7 +222,7 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
   uint32_t* err = nullptr;
   int sms = 0;
   if (!device_info(&err, &sms)) return KV4_ERR_CUDA;
-  const int full = decode_ctas_full(fmt, sms);
+  const int full = decode_ctas_full(c, sms);
   int ctas = full;
   if (max_len_hint > 0) {
     // Enough CTAs that each warp gets at least ~16 slots of the hinted upper bound.
@@ -343,7 +348,7 @@ kv4_status kv4_decode_workspace_bytes(const kv4_cache* cache, int B, size_t* byt
   if (!cache || own_format(cache) != cache->format || B < 0 || !bytes) return KV4_ERR_INVALID_ARG;
   int sms = 0;
   if (!device_info(nullptr, &sms)) return KV4_ERR_CUDA;
-  *bytes = workspace_for(cache, B, decode_ctas_full(cache->format, sms));
+  *bytes = workspace_for(cache, B, decode_ctas_full(cache, sms));
   return KV4_OK;
 }
 
@@ -482,7 +487,7 @@ kv4_status kv4_decode_attn_static(kv4_cache* cache, int layer, int B, const void
   if (B == 0) return KV4_OK;
   int sms = 0;
   if (!device_info(nullptr, &sms)) return KV4_ERR_CUDA;
-  if (workspace_for(cache, B, decode_ctas_full(cache->format, sms)) > KV4_STATIC_SCRATCH_BYTES) return KV4_ERR_WORKSPACE;
+  if (workspace_for(cache, B, decode_ctas_full(cache, sms)) > KV4_STATIC_SCRATCH_BYTES) return KV4_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (!static_scratch_address(&scratch)) return KV4_ERR_CUDA;
   return decode_common(cache, cache->format, layer, B, q, q_dtype, page_table, stride, lens, max_len_hint, out, lse,
@@ -529,7 +534,7 @@ kv4_status kv4_bf16_decode_workspace_bytes(const kv4_cache* cache, int B, size_t
   if (!cache || cache->format != FMT_BF16 || B < 0 || !bytes) return KV4_ERR_INVALID_ARG;
   int sms = 0;
   if (!device_info(nullptr, &sms)) return KV4_ERR_CUDA;
-  *bytes = workspace_for(cache, B, decode_ctas_full(FMT_BF16, sms));
+  *bytes = workspace_for(cache, B, decode_ctas_full(cache, sms));
   return KV4_OK;
 }
 

@@ -33,6 +33,8 @@
 #include <cuda_fp16.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "kv4_device.cuh"
 #include "kv4_internal.h"
 #include "kv4_layout.cuh"
@@ -265,7 +267,10 @@ template <int D, int G, int VB>
 struct SmemMixed {
   uint8_t ring[kWarps][kStages][MixedGeo<D, VB>::STAGE];
   float qbuf[kWarps][G][D];
-  uint32_t ktab[kWarps][D];  // coordinate tig * D/4 + r at [4 r + tig]: bit offset | width << 16
+  // key extraction table per (k step kb, lane group tig): the four codes of coordinates
+  // tig * D/4 + 4 kb + (0..3) lie in one 32-bit window of the bit stream starting at bit off0:
+  // words [0, 4) their offsets in the window, [4, 8) their masks, word 8 off0
+  uint32_t ktab[kWarps][D / 16][4][12];
   uint64_t bar[kWarps][kStages];
 };
 
@@ -286,9 +291,9 @@ __device__ __forceinline__ uint32_t split_h2(float x0, float x1, bool lo) {
   return static_cast<uint32_t>(__half_as_ushort(r0)) | (static_cast<uint32_t>(__half_as_ushort(r1)) << 16);
 }
 
-// two integer codes (< 2048) as the exact fp16 pair (c0, c1): 1024 + c in the 0x6400 exponent, minus 1024
+// two integer codes (< 1024) as the exact fp16 pair (c0, c1): 1024 + c in the 0x6400 exponent, minus 1024
 __device__ __forceinline__ uint32_t codes_h2(uint32_t c0, uint32_t c1) {
-  const uint32_t h = c0 | (c1 << 16) | 0x64006400u;
+  const uint32_t h = prmt(c0, c1, 0x5410u) | 0x64006400u;
   __half2 v = *reinterpret_cast<const __half2*>(&h);
   v = __hsub2(v, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
   return *reinterpret_cast<uint32_t*>(&v);
@@ -304,7 +309,7 @@ __device__ __forceinline__ uint32_t take_bits(const uint32_t (&aw)[NW], int p, i
 }
 
 template <int D, int G, int VB>
-__global__ void __launch_bounds__(kWarps * 32, 1) decode_mixed_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const DecodeArgs a) {
   using MG = MixedGeo<D, VB>;
   constexpr int NK = MG::NK, NB = D / 2, Q4 = D / 4;
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -357,7 +362,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_mixed_kernel(const Deco
   uint32_t qf[NK][2];
   float cst = 0.f, inv_scale = 1.f;
   float* qb = &sm.qbuf[warp][0][0];
-  uint32_t* ktab = sm.ktab[warp];
+  uint32_t* ktab = &sm.ktab[warp][0][0][0];
   auto load_query = [&](int b, int g) {
     const float* sig = rec_sigma<D>(a.alloc, g);
     const uint8_t* wid8 = rec_width<D>(a.alloc, g);
@@ -385,7 +390,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_mixed_kernel(const Deco
       const int j = lane + 32 * i, c = (j % NB) / 32;
       const int w = wv[c];
       const int off = (j >= NB ? run : 0) + pre[c];
-      ktab[4 * (j % Q4) + j / Q4] = static_cast<uint32_t>(off) | (static_cast<uint32_t>(w) << 16);
+      const int off0 = __shfl_sync(FULL, off, lane & ~3);  // first coordinate of the group of four
+      {
+        const int r = j % Q4, kb = r >> 2, e = r & 3;
+        uint32_t* ent = ktab + (kb * 4 + j / Q4) * 12;
+        ent[e] = static_cast<uint32_t>(off - off0);
+        ent[4 + e] = (1u << w) - 1u;
+        if (e == 0) ent[8] = static_cast<uint32_t>(off);
+      }
       const float sgm = sig[j % NB];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -500,18 +512,16 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_mixed_kernel(const Deco
     float S[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kb = 0; kb < NK; ++kb) {
-      uint32_t c0v[4], c1v[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t ent = ktab[4 * (4 * kb + e) + tig];
-        const int off = static_cast<int>(ent & 0xffffu), w = static_cast<int>(ent >> 16);
-        const int wi = off >> 5, sh = off & 31;
-        const uint32_t mask = (1u << w) - 1u;
-        c0v[e] = __funnelshift_r(r0w[wi], r0w[wi + 1], sh) & mask;
-        c1v[e] = __funnelshift_r(r1w[wi], r1w[wi + 1], sh) & mask;
-      }
-      mma_f16(S, codes_h2(c0v[0], c0v[1]), codes_h2(c1v[0], c1v[1]), codes_h2(c0v[2], c0v[3]),
-              codes_h2(c1v[2], c1v[3]), qf[kb][0], qf[kb][1]);
+      const uint32_t* ent = ktab + (kb * 4 + tig) * 12;
+      const uint4 R = *reinterpret_cast<const uint4*>(ent);
+      const uint4 M = *reinterpret_cast<const uint4*>(ent + 4);
+      const uint32_t off0 = ent[8];
+      const int wi = static_cast<int>(off0 >> 5), sh = static_cast<int>(off0 & 31u);
+      const uint32_t x0 = __funnelshift_r(r0w[wi], r0w[wi + 1], sh);
+      const uint32_t x1 = __funnelshift_r(r1w[wi], r1w[wi + 1], sh);
+      mma_f16(S, codes_h2(x0 & M.x, (x0 >> R.y) & M.y), codes_h2(x1 & M.x, (x1 >> R.y) & M.y),
+              codes_h2((x0 >> R.z) & M.z, (x0 >> R.w) & M.w), codes_h2((x1 >> R.z) & M.z, (x1 >> R.w) & M.w),
+              qf[kb][0], qf[kb][1]);
     }
     const __half* prm = reinterpret_cast<const __half*>(buf + MG::PO);
     const float s0 = v0 ? __half2float(prm[4 * gq]) : 0.f, s1 = v1 ? __half2float(prm[4 * (gq + 8)]) : 0.f;
@@ -565,26 +575,28 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_mixed_kernel(const Deco
       b0 = split_h2(ps[0], ps[1], lo);
       b1 = split_h2(ps[2], ps[3], lo);
     }
-    // value codes of the lane's dims for its four tokens
-    uint32_t cv[4][MG::DPL];
+    // the lane's value bits (dims gq * D/8 + [0, D/8)) of its four tokens, aligned to bit 0
+    uint32_t aw[4][MG::NWA];
     const int bit0 = gq * MG::WIN;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const uint32_t* vr = reinterpret_cast<const uint32_t*>(buf + MG::VO + tk[u] * MG::VR);
-      uint32_t raw[MG::NWA + 1], aw[MG::NWA];
+      uint32_t raw[MG::NWA + 1];
 #pragma unroll
       for (int x = 0; x <= MG::NWA; ++x) raw[x] = vr[(bit0 >> 5) + x];
 #pragma unroll
-      for (int x = 0; x < MG::NWA; ++x) aw[x] = __funnelshift_r(raw[x], raw[x + 1], bit0 & 31);
-#pragma unroll
-      for (int d = 0; d < MG::DPL; ++d) cv[u][d] = take_bits(aw, d * VB, VB);
+      for (int x = 0; x < MG::NWA; ++x) aw[u][x] = __funnelshift_r(raw[x], raw[x + 1], bit0 & 31);
     }
     // Slots past L (or of a bad page) hold arbitrary bytes, but their codes are finite integers
     // and their B entries are exactly zero, so they add nothing.
 #pragma unroll
-    for (int mb = 0; mb < NK; ++mb)
-      mma_f16(oacc[mb], codes_h2(cv[0][2 * mb], cv[1][2 * mb]), codes_h2(cv[0][2 * mb + 1], cv[1][2 * mb + 1]),
-              codes_h2(cv[2][2 * mb], cv[3][2 * mb]), codes_h2(cv[2][2 * mb + 1], cv[3][2 * mb + 1]), b0, b1);
+    for (int mb = 0; mb < NK; ++mb) {
+      const int p0 = 2 * mb * VB, p1 = p0 + VB;
+      mma_f16(oacc[mb], codes_h2(take_bits(aw[0], p0, VB), take_bits(aw[1], p0, VB)),
+              codes_h2(take_bits(aw[0], p1, VB), take_bits(aw[1], p1, VB)),
+              codes_h2(take_bits(aw[2], p0, VB), take_bits(aw[3], p0, VB)),
+              codes_h2(take_bits(aw[2], p1, VB), take_bits(aw[3], p1, VB)), b0, b1);
+    }
     __syncwarp();
 
     splitk::Cur nxt = cons;
@@ -652,6 +664,27 @@ cudaError_t launch_append_mixed(const AppendArgs& a, int D, cudaStream_t st) {
 }
 
 int mixed_decode_warps_per_cta() { return kWarps; }
+
+// Two CTAs per SM where their shared memory fits (it does for value_bits <= 4), else one.
+int mixed_decode_ctas_per_sm(int D, int G, int VB) {
+  size_t bytes = 0;
+  auto pick = [&](auto d, auto g) {
+    constexpr int DD = decltype(d)::value, GG = decltype(g)::value;
+    bytes = VB == 2 ? sizeof(SmemMixed<DD, GG, 2>) : VB == 3 ? sizeof(SmemMixed<DD, GG, 3>)
+            : VB == 4 ? sizeof(SmemMixed<DD, GG, 4>) : sizeof(SmemMixed<DD, GG, 8>);
+  };
+  using I128 = std::integral_constant<int, 128>;
+  using I64 = std::integral_constant<int, 64>;
+  using G1 = std::integral_constant<int, 1>;
+  using G2 = std::integral_constant<int, 2>;
+  using G4 = std::integral_constant<int, 4>;
+  if (D == 128) {
+    if (G == 4) pick(I128{}, G4{}); else if (G == 2) pick(I128{}, G2{}); else pick(I128{}, G1{});
+  } else {
+    if (G == 4) pick(I64{}, G4{}); else if (G == 2) pick(I64{}, G2{}); else pick(I64{}, G1{});
+  }
+  return 2 * (bytes + 1024) <= 227u * 1024u ? 2 : 1;
+}
 
 cudaError_t launch_decode_mixed(DecodeArgs a, int D, int G, int ctas, cudaStream_t st) {
   a.W = ctas * kWarps;

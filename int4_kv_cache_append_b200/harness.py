@@ -14,8 +14,9 @@ from . import workload as W
 
 
 def geometry(wl: W.Workload, layers: int | None = None, value_format: int = kv4.KV4_VALUES_INT4) -> kv4.Geometry:
+    mixed = value_format == kv4.KV4_KEYS_MIXED
     return kv4.Geometry(layers or wl.layers, wl.Hq, wl.Hkv, wl.D, wl.P, wl.s, wl.w, wl.h, wl.B, max(wl.num_pages, 1),
-                        value_format)
+                        value_format, wl.key_bits if mixed else 0, wl.value_bits if mixed else 0)
 
 
 def token_list(lens: np.ndarray, upto=None):
@@ -38,8 +39,10 @@ def device_kv(wl: W.Workload, layer: int, b: torch.Tensor, p: torch.Tensor, fact
 
 
 def prefill(cache, wl: W.Workload, layer: int, lens: np.ndarray, upto=None, chunk: int = 65536,
-            bf16_pool: bool = False):
-    """Append positions [0, upto_b) of every sequence (lens_after = lens) in chunks."""
+            bf16_pool: bool = False, allocate: bool = False):
+    """Append positions [0, upto_b) of every sequence (lens_after = lens) in chunks.  allocate
+    (mixed bit-width keys): the layer's key bits are first allocated from the keys of the first
+    chunk (up to `chunk` prefill tokens, in sequence order)."""
     dev = cache.pool.device
     b_all, p_all = token_list(lens, upto)
     factor = torch.from_numpy(wl.factor()).to(dev)
@@ -49,6 +52,8 @@ def prefill(cache, wl: W.Workload, layer: int, lens: np.ndarray, upto=None, chun
         b = torch.from_numpy(b_all[i:i + chunk]).to(dev)
         p = torch.from_numpy(p_all[i:i + chunk]).to(dev)
         K, V = device_kv(wl, layer, b, p, factor)
+        if allocate and i == 0:
+            cache.allocate_key_bits(layer, K)
         if bf16_pool:
             cache.append(layer, K, V, b, p, pt)
         else:

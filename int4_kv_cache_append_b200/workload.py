@@ -141,6 +141,8 @@ class Workload:
     num_pages: int = 0
     value_format: int = 0                        # 0: INT4 values, 1: bf16 values (K-INT4 / V-BF16)
     rope_outliers: bool = False                  # outliers as whole RoPE blocks, queries scaled alike
+    key_bits: int = 0                            # value_format 2 (mixed bit-width keys): average key bits
+    value_bits: int = 0                          # value_format 2: value bits per dimension
 
     @property
     def G(self) -> int:
@@ -186,6 +188,8 @@ class Workload:
         codes + fp16 scales, K and V, all KV heads (bf16 values: 2D bytes of V per position in
         both regions instead of the V codes and parameters)."""
         L = np.asarray(self.lens if lens is None else lens, np.int64)
+        if self.value_format == 2:  # mixed bit-width keys: packed K and V codes + 8 bytes, every position
+            return int(self.Hkv * L.sum() * ((self.key_bits + self.value_bits) * self.D // 8 + 8))
         n4 = np.maximum(0, L - self.s - self.w)
         n8 = np.minimum(L, self.s + self.w)
         D = self.D
