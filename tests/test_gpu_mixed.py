@@ -236,3 +236,83 @@ def test_range_overflow_sets_error_bit():
     assert O.gtq_append(cfg, widths, sigma, pool, K, V, b, p, wl.page_table, O.F32, O.F32)
     pages, _ = cache.layer_views(0)
     assert np.array_equal(pages.cpu().numpy()[:pool.size], pool)
+
+
+def _oracle_one_mixed(wl, kb, vb, widths, sigma, b, g):
+    """Oracle cache (identity page table) and decode of sequence b of a full-size workload, only
+    KV head g populated, with the given allocation."""
+    L = int(wl.lens[b])
+    npages = (L + wl.P - 1) // wl.P
+    cfg = O.GtqConfig(wl.Hq, wl.Hkv, wl.D, wl.P, kb, vb)
+    pool = np.full(O.gtq_sizes(cfg)["page_bytes"] * npages, 0xA5, np.uint8)
+    f = wl.factor()
+    pos = np.arange(L, dtype=np.int64)
+    idx = ((b * W.POS_STRIDE + pos[:, None]) * wl.Hkv + g) * wl.D + np.arange(wl.D)[None, :]
+    K = np.zeros((L, wl.Hkv, wl.D), np.float32)
+    V = np.zeros((L, wl.Hkv, wl.D), np.float32)
+    K[:, g] = W.normal_f32(W.stream_key(wl.seed, W.KIND_K, 0), idx).reshape(L, wl.D) * f[g][None]
+    V[:, g] = W.normal_f32(W.stream_key(wl.seed, W.KIND_V, 0), idx).reshape(L, wl.D) * f[g][None]
+    kd = vd = O.F32
+    if wl.k_dtype == W.BF16:
+        K, kd = W.bf16_bits(K), O.BF16
+    if wl.v_dtype == W.BF16:
+        V, vd = W.bf16_bits(V), O.BF16
+    pt = np.arange(npages, dtype=np.int32)[None, :]
+    O.gtq_append(cfg, widths, sigma, pool, K, V, np.zeros(L, np.int32), pos.astype(np.int32), pt, kd, vd)
+    q = wl.q_input(0, 0, rows=[b])
+    out, lse = O.gtq_decode(cfg, widths, sigma, pool, q, pt, np.array([L], np.int32),
+                            q_dtype=O.BF16 if q.dtype == np.uint16 else O.F32)
+    return cfg, pool, out[0], lse[0]
+
+
+@pytest.mark.parametrize("name", ["async-refill", "long-context"])
+def test_fullsize_mixed_sampled_parity(name):
+    """The bench's K3V3 workloads at full size, in its launch configuration: the allocation from
+    4096 host-drawn keys equals the oracle's; sampled (sequence, KV head) pairs are recomputed by
+    the oracle one by one (page bytes bit-exact, outputs within the tolerance)."""
+    from int4_kv_cache_append_b200 import harness as H, kv4
+    kb, vb = 3, 3
+    wl = dataclasses.replace(W.WORKLOADS[name](), s=0, w=0, h=1, value_format=2, key_bits=kb, value_bits=vb,
+                             rope_outliers=True)
+    cache = kv4.Cache(H.geometry(wl, value_format=kv4.KV4_KEYS_MIXED), fill=0xA5)
+    b_all, p_all = H.token_list(wl.lens)
+    n = min(4096, b_all.size)
+    Ka, _ = wl.kv_inputs(0, b_all[:n], p_all[:n])
+    cache.allocate_key_bits(0, T.to_dev(Ka))
+    kdc = O.BF16 if wl.k_dtype == W.BF16 else O.F32
+    E = O.gtq_energy(Ka, kdc)
+    widths = np.stack([O.gtq_allocate(E[g], kb) for g in range(wl.Hkv)])
+    sigma = np.stack([O.gtq_scales(E[g], n) for g in range(wl.Hkv)])
+    w_gpu, s_gpu = cache.key_allocation(0)
+    assert np.array_equal(w_gpu, widths) and np.array_equal(s_gpu.view(np.uint32), sigma.view(np.uint32))
+    H.prefill(cache, wl, 0, wl.lens)
+    q = T.to_dev(wl.q_input(0))
+    lse = torch.empty((wl.B, wl.Hq), device="cuda")
+    out = cache.decode(0, q, torch.from_numpy(wl.page_table).cuda(), torch.from_numpy(wl.lens).cuda(), lse=lse,
+                       max_len_hint=int(wl.lens.max()))
+    torch.cuda.synchronize()
+    assert kv4.kv4_get_device_error() == 0
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    assert np.isfinite(out).all()
+    order = np.argsort(wl.lens, kind="stable")
+    picks = [(int(order[0]), 0), (int(order[len(order) // 2]), wl.Hkv // 2), (int(order[-1]), wl.Hkv - 1)]
+    if name == "long-context":
+        picks = [(0, 3), (3, 6)]
+    pages, _ = cache.layer_views(0)
+    tile = wl.P * ((kb + vb) * wl.D // 8 + 8)
+    for b, g in picks:
+        ocfg, opool, oout, olse = _oracle_one_mixed(wl, kb, vb, widths, sigma, b, g)
+        pb = O.gtq_sizes(ocfg)["page_bytes"]
+        L = int(wl.lens[b])
+        for lp in range((L + wl.P - 1) // wl.P):
+            page = int(wl.page_table[b, lp])
+            got = pages[page * pb + g * tile: page * pb + (g + 1) * tile].cpu().numpy()
+            want = opool[lp * pb + g * tile: lp * pb + (g + 1) * tile]
+            assert np.array_equal(got, want), f"{name}: seq {b} head {g} page {lp} differs"
+        G = wl.Hq // wl.Hkv
+        # The logits here reach several hundred (x20 RoPE-block outliers in both q and k), and the
+        # decode forms them from query weights kept to ~22 bits (fp16 hi/lo halves), so the lse
+        # bound grows with its magnitude: 1e-4 + 2^-20 |lse|.
+        lse_tol = 1e-4 + 2.0 ** -20 * float(np.abs(olse[g * G:(g + 1) * G]).max())
+        T.assert_close(out[b, g * G:(g + 1) * G], oout[g * G:(g + 1) * G], lse[b, g * G:(g + 1) * G],
+                       olse[g * G:(g + 1) * G], lse_atol=lse_tol, what=f"{name} seq {b} head {g}")
