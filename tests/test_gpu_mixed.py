@@ -34,6 +34,9 @@ CASES = [
     (mixed_workload("m-k8v3", 105, 2, 2, 2, 64, 16, [150, 9], dt=W.F32), 8, 3),
     (mixed_workload("m-k5v4-empty", 106, 3, 4, 2, 128, 48, [0, 250, 31]), 5, 4),
     (mixed_workload("m-k3v2-flat", 107, 3, 4, 2, 128, 16, [160, 99, 260], scale=1.0), 3, 2),
+    # smallest rows (8-byte keys, 16-byte values) and an odd width on every block
+    (mixed_workload("m-k1v2-d64", 108, 2, 4, 2, 64, 16, [33, 500]), 1, 2),
+    (mixed_workload("m-k7v8-p32", 109, 2, 2, 4, 128, 32, [70, 301], dt=W.F32), 7, 8),
 ]
 IDS = [c[0].name for c in CASES]
 
