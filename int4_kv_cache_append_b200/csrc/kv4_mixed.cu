@@ -308,6 +308,29 @@ __device__ __forceinline__ uint32_t take_bits(const uint32_t (&aw)[NW], int p, i
   return x & ((1u << w) - 1u);
 }
 
+// Value widths whose fields never straddle a byte: the PV operands are cut out with byte
+// permutes and masks, each field keeping its position s within its byte (code * 2^s), and the
+// partial's rows are scaled back by 2^-s at the flush.
+template <int VB>
+constexpr bool kSwarV = VB == 2 || VB == 4 || VB == 8;
+
+// bit position within its byte of the value field of lane dim d
+template <int VB>
+__host__ __device__ constexpr int swar_shift(int d) { return (d * VB) & 7; }
+
+// (code of dim d of token t0, same of t1) * 2^swar_shift(d) as an exact fp16 pair
+template <int VB, int NW>
+__device__ __forceinline__ uint32_t swar_pair(const uint32_t (&w0)[NW], const uint32_t (&w1)[NW], int d) {
+  const int byte = (d * VB) >> 3, sh = swar_shift<VB>(d);
+  const uint32_t sel = static_cast<uint32_t>((byte & 3) | ((4 + (byte & 3)) << 8));
+  const uint32_t x = prmt(w0[byte >> 2], w1[byte >> 2], sel);
+  const uint32_t m = ((1u << VB) - 1u) << sh;
+  const uint32_t h = (x & (m | (m << 16))) | 0x64006400u;
+  __half2 v = *reinterpret_cast<const __half2*>(&h);
+  v = __hsub2(v, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 template <int D, int G, int VB>
 __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const DecodeArgs a) {
   using MG = MixedGeo<D, VB>;
@@ -463,7 +486,11 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
 #pragma unroll
       for (int mb = 0; mb < NK; ++mb) {
         const int d = MG::DPL * gq + 2 * mb;
-        *reinterpret_cast<float2*>(p + d) = make_float2(oacc[mb][0] + oacc[mb][1] + z, oacc[mb][2] + oacc[mb][3] + z);
+        // byte-aligned value widths left the codes of dims 2 mb, 2 mb + 1 at 2^s (exact)
+        const float f0 = kSwarV<VB> ? 1.0f / static_cast<float>(1 << swar_shift<VB>(2 * mb)) : 1.0f;
+        const float f1 = kSwarV<VB> ? 1.0f / static_cast<float>(1 << swar_shift<VB>(2 * mb + 1)) : 1.0f;
+        *reinterpret_cast<float2*>(p + d) =
+            make_float2(fmaf(oacc[mb][0] + oacc[mb][1], f0, z), fmaf(oacc[mb][2] + oacc[mb][3], f1, z));
       }
       if (gq == 0) *reinterpret_cast<float2*>(p + D) = make_float2(m_run, l);
     }
@@ -591,11 +618,18 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
     // and their B entries are exactly zero, so they add nothing.
 #pragma unroll
     for (int mb = 0; mb < NK; ++mb) {
-      const int p0 = 2 * mb * VB, p1 = p0 + VB;
-      mma_f16(oacc[mb], codes_h2(take_bits(aw[0], p0, VB), take_bits(aw[1], p0, VB)),
-              codes_h2(take_bits(aw[0], p1, VB), take_bits(aw[1], p1, VB)),
-              codes_h2(take_bits(aw[2], p0, VB), take_bits(aw[3], p0, VB)),
-              codes_h2(take_bits(aw[2], p1, VB), take_bits(aw[3], p1, VB)), b0, b1);
+      if constexpr (kSwarV<VB>) {
+        // byte-aligned fields: one prmt puts byte k of two tokens' windows into the two halves,
+        // one mask keeps a field with the 0x6400 exponent, one subtraction leaves code * 2^s
+        mma_f16(oacc[mb], swar_pair<VB>(aw[0], aw[1], 2 * mb), swar_pair<VB>(aw[0], aw[1], 2 * mb + 1),
+                swar_pair<VB>(aw[2], aw[3], 2 * mb), swar_pair<VB>(aw[2], aw[3], 2 * mb + 1), b0, b1);
+      } else {
+        const int p0 = 2 * mb * VB, p1 = p0 + VB;
+        mma_f16(oacc[mb], codes_h2(take_bits(aw[0], p0, VB), take_bits(aw[1], p0, VB)),
+                codes_h2(take_bits(aw[0], p1, VB), take_bits(aw[1], p1, VB)),
+                codes_h2(take_bits(aw[2], p0, VB), take_bits(aw[3], p0, VB)),
+                codes_h2(take_bits(aw[2], p1, VB), take_bits(aw[3], p1, VB)), b0, b1);
+      }
     }
     __syncwarp();
 
