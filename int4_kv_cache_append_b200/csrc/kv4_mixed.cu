@@ -271,6 +271,7 @@ struct SmemMixed {
   // tig * D/4 + 4 kb + (0..3) lie in one 32-bit window of the bit stream starting at bit off0:
   // words [0, 4) their offsets in the window, [4, 8) their masks, word 8 off0
   uint32_t ktab[kWarps][D / 16][4][12];
+  uint32_t stage_ok[kWarps][kStages];  // 1 when the stage's page id was inside the pool
   uint64_t bar[kWarps][kStages];
 };
 
@@ -360,23 +361,31 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
   const long long nslots = c1 - c0;
   const uint32_t stage_tx = static_cast<uint32_t>(16 * KR + 16 * MG::VR + 128);
 
+  // Called by the whole warp: every lane reads the same page-table entry (one request); lane 0
+  // arms the barrier and records whether the page is valid, then lanes 0, 1 and 2 each start one
+  // of the tile's three bulk copies (keys, values, parameter records).
   auto issue = [&](const splitk::Cur& c, int st) {
     const int lp = (c.i * 16) / a.P;
     const int page = a.page_table[static_cast<size_t>(c.b) * a.stride + lp];
-    if (page >= 0 && page < a.max_pages) {
+    const bool ok = page >= 0 && page < a.max_pages;
+    if (lane == 0) {
+      sm.stage_ok[warp][st] = ok ? 1u : 0u;
+      if (!ok) atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
+      mbar_arrive_expect_tx(&bars[st], ok ? stage_tx : 0u);
+    }
+    __syncwarp();
+    if (ok && lane < 3) {
       const int r0 = c.i * 16 - lp * a.P;
       const uint8_t* tile = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(c.g) * tile_bytes;
       uint8_t* dst = sm.ring[warp][st];
       const uint64_t pol = l2_policy_evict_first();
-      mbar_arrive_expect_tx(&bars[st], stage_tx);
-      bulk_g2s_hint(dst, tile + static_cast<size_t>(r0) * KR, 16 * KR, &bars[st], pol);
-      bulk_g2s_hint(dst + MG::VO, tile + static_cast<size_t>(a.P) * KR + static_cast<size_t>(r0) * MG::VR, 16 * MG::VR,
-                    &bars[st], pol);
-      bulk_g2s_hint(dst + MG::PO, tile + static_cast<size_t>(a.P) * (KR + MG::VR) + static_cast<size_t>(r0) * 8, 128,
-                    &bars[st], pol);
-    } else {
-      atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
-      mbar_arrive_expect_tx(&bars[st], 0);
+      if (lane == 0) bulk_g2s_hint(dst, tile + static_cast<size_t>(r0) * KR, 16 * KR, &bars[st], pol);
+      else if (lane == 1)
+        bulk_g2s_hint(dst + MG::VO, tile + static_cast<size_t>(a.P) * KR + static_cast<size_t>(r0) * MG::VR,
+                      16 * MG::VR, &bars[st], pol);
+      else
+        bulk_g2s_hint(dst + MG::PO, tile + static_cast<size_t>(a.P) * (KR + MG::VR) + static_cast<size_t>(r0) * 8, 128,
+                      &bars[st], pol);
     }
   };
 
@@ -496,21 +505,20 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
     }
   };
 
-  int issued = 0;
-  if (lane == 0) {
-    for (int k = 0; k < kStages - 1 && k < nslots; ++k) {
-      issue(prod, k);
-      ++prod.i;
-      splitk::settle(a, cap, prod);
-      ++issued;
-    }
+  int issued = 0;  // warp-uniform
+  for (int k = 0; k < kStages - 1 && k < nslots; ++k) {
+    issue(prod, k);
+    ++prod.i;
+    splitk::settle(a, cap, prod);
+    ++issued;
   }
   reset();
   load_query(cons.b, cons.g);
+  int Lseg = splitk::clamp_len(a.lens[cons.b], cap);  // length of the consumer's sequence
   bool failed = false;
   long long k = 0;
   for (; k < nslots; ++k) {
-    if (lane == 0 && issued < nslots) {
+    if (issued < nslots) {
       fence_proxy_async_smem();
       issue(prod, static_cast<int>((k + kStages - 1) % kStages));
       ++prod.i;
@@ -524,10 +532,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
       break;
     }
     const uint8_t* buf = sm.ring[warp][st];
-    const int lp = (cons.i * 16) / a.P;
-    const int page = a.page_table[static_cast<size_t>(cons.b) * a.stride + lp];
-    const bool page_ok = page >= 0 && page < a.max_pages;
-    const int L = splitk::clamp_len(a.lens[cons.b], cap);
+    const bool page_ok = sm.stage_ok[warp][st] != 0u;
+    const int L = Lseg;
     const int i0 = cons.i * 16;
     const bool v0 = page_ok && tig < G && i0 + gq < L, v1 = page_ok && tig < G && i0 + gq + 8 < L;
 
@@ -640,12 +646,14 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
     if (!more || nxt.b != cons.b || nxt.g != cons.g) {
       flush(cons);
       reset();
-      if (more) load_query(nxt.b, nxt.g);
+      if (more) {
+        load_query(nxt.b, nxt.g);
+        if (nxt.b != cons.b) Lseg = splitk::clamp_len(a.lens[nxt.b], cap);
+      }
     }
     cons = nxt;
   }
   if (failed) {
-    issued = __shfl_sync(FULL, issued, 0);
     for (long long j = k; j < issued; ++j)
       mbar_wait_bounded(&bars[j % kStages], static_cast<uint32_t>((j / kStages) & 1), a.err);
   }
