@@ -267,10 +267,12 @@ template <int D, int G, int VB>
 struct SmemMixed {
   uint8_t ring[kWarps][kStages][MixedGeo<D, VB>::STAGE];
   float qbuf[kWarps][G][D];
-  // key extraction table per (k step kb, lane group tig): the four codes of coordinates
-  // tig * D/4 + 4 kb + (0..3) lie in one 32-bit window of the bit stream starting at bit off0:
-  // words [0, 4) their offsets in the window, [4, 8) their masks, word 8 off0
-  uint32_t ktab[kWarps][D / 16][4][12];
+  // key extraction table per (k step kb, lane group tig): the four codes c0..c3 of coordinates
+  // tig * D/4 + 4 kb + (0..3) lie in one 32-bit window x of the bit stream starting at bit off0,
+  // at offsets r0 = 0, r1, r2, r3.  Words: m0, m1 << 16, 16 - r1, off0 | r2, m2, m3 << 16,
+  // 16 - (r3 - r2) (m = the code's width mask): (x & m0) | (x << (16 - r1)) & (m1 << 16) is the
+  // pair (c0, c1) in two 16-bit halves, and likewise (c2, c3) from x >> r2.
+  uint32_t ktab[kWarps][D / 16][4][8];
   uint32_t stage_ok[kWarps][kStages];  // 1 when the stage's page id was inside the pool
   uint64_t bar[kWarps][kStages];
 };
@@ -295,6 +297,13 @@ __device__ __forceinline__ uint32_t split_h2(float x0, float x1, bool lo) {
 // two integer codes (< 1024) as the exact fp16 pair (c0, c1): 1024 + c in the 0x6400 exponent, minus 1024
 __device__ __forceinline__ uint32_t codes_h2(uint32_t c0, uint32_t c1) {
   const uint32_t h = prmt(c0, c1, 0x5410u) | 0x64006400u;
+  __half2 v = *reinterpret_cast<const __half2*>(&h);
+  v = __hsub2(v, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// (1024 + c0, 1024 + c1) with the 0x6400 exponent in both halves -> the exact fp16 pair (c0, c1)
+__device__ __forceinline__ uint32_t magic_pair(uint32_t h) {
   __half2 v = *reinterpret_cast<const __half2*>(&h);
   v = __hsub2(v, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
   return *reinterpret_cast<uint32_t*>(&v);
@@ -394,7 +403,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
   uint32_t qf[NK][2];
   float cst = 0.f, inv_scale = 1.f;
   float* qb = &sm.qbuf[warp][0][0];
-  uint32_t* ktab = &sm.ktab[warp][0][0][0];
+  uint32_t* ktab = &sm.ktab[warp][0][0][0];  // [kb][tig][8]
   auto load_query = [&](int b, int g) {
     const float* sig = rec_sigma<D>(a.alloc, g);
     const uint8_t* wid8 = rec_width<D>(a.alloc, g);
@@ -423,12 +432,24 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
       const int w = wv[c];
       const int off = (j >= NB ? run : 0) + pre[c];
       const int off0 = __shfl_sync(FULL, off, lane & ~3);  // first coordinate of the group of four
+      const int off2 = __shfl_sync(FULL, off, (lane & ~3) + 2);
       {
         const int r = j % Q4, kb = r >> 2, e = r & 3;
-        uint32_t* ent = ktab + (kb * 4 + j / Q4) * 12;
-        ent[e] = static_cast<uint32_t>(off - off0);
-        ent[4 + e] = (1u << w) - 1u;
-        if (e == 0) ent[8] = static_cast<uint32_t>(off);
+        uint32_t* ent = ktab + (kb * 4 + j / Q4) * 8;
+        const uint32_t m = (1u << w) - 1u;
+        if (e == 0) {
+          ent[0] = m;
+          ent[3] = static_cast<uint32_t>(off);
+        } else if (e == 1) {
+          ent[1] = m << 16;
+          ent[2] = static_cast<uint32_t>(16 - (off - off0));
+        } else if (e == 2) {
+          ent[4] = static_cast<uint32_t>(off - off0);
+          ent[5] = m;
+        } else {
+          ent[6] = m << 16;
+          ent[7] = static_cast<uint32_t>(16 - (off - off2));
+        }
       }
       const float sgm = sig[j % NB];
 #pragma unroll
@@ -545,16 +566,17 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
     float S[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kb = 0; kb < NK; ++kb) {
-      const uint32_t* ent = ktab + (kb * 4 + tig) * 12;
-      const uint4 R = *reinterpret_cast<const uint4*>(ent);
-      const uint4 M = *reinterpret_cast<const uint4*>(ent + 4);
-      const uint32_t off0 = ent[8];
-      const int wi = static_cast<int>(off0 >> 5), sh = static_cast<int>(off0 & 31u);
+      const uint32_t* ent = ktab + (kb * 4 + tig) * 8;
+      const uint4 E0 = *reinterpret_cast<const uint4*>(ent);      // m0, m1 << 16, 16 - r1, off0
+      const uint4 E1 = *reinterpret_cast<const uint4*>(ent + 4);  // r2, m2, m3 << 16, 16 - (r3 - r2)
+      const int wi = static_cast<int>(E0.w >> 5), sh = static_cast<int>(E0.w & 31u);
       const uint32_t x0 = __funnelshift_r(r0w[wi], r0w[wi + 1], sh);
       const uint32_t x1 = __funnelshift_r(r1w[wi], r1w[wi + 1], sh);
-      mma_f16(S, codes_h2(x0 & M.x, (x0 >> R.y) & M.y), codes_h2(x1 & M.x, (x1 >> R.y) & M.y),
-              codes_h2((x0 >> R.z) & M.z, (x0 >> R.w) & M.w), codes_h2((x1 >> R.z) & M.z, (x1 >> R.w) & M.w),
-              qf[kb][0], qf[kb][1]);
+      const uint32_t z0 = x0 >> E1.x, z1 = x1 >> E1.x;
+      mma_f16(S, magic_pair(((x0 & E0.x) | 0x64006400u) | ((x0 << E0.z) & E0.y)),
+              magic_pair(((x1 & E0.x) | 0x64006400u) | ((x1 << E0.z) & E0.y)),
+              magic_pair(((z0 & E1.y) | 0x64006400u) | ((z0 << E1.w) & E1.z)),
+              magic_pair(((z1 & E1.y) | 0x64006400u) | ((z1 << E1.w) & E1.z)), qf[kb][0], qf[kb][1]);
     }
     const __half* prm = reinterpret_cast<const __half*>(buf + MG::PO);
     const float s0 = v0 ? __half2float(prm[4 * gq]) : 0.f, s1 = v1 ? __half2float(prm[4 * (gq + 8)]) : 0.f;
