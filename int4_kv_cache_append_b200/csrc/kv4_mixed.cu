@@ -341,6 +341,19 @@ __device__ __forceinline__ uint32_t swar_pair(const uint32_t (&w0)[NW], const ui
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// (code of dim d of token t0, same of t1) as an exact fp16 pair, for any value width: a field
+// inside one word takes a shift and a mask with the 0x6400 exponent for t0, one shift for t1 and
+// one mask-or to join them; a field across two words goes through take_bits.
+template <int VB, int NW>
+__device__ __forceinline__ uint32_t field_pair(const uint32_t (&w0)[NW], const uint32_t (&w1)[NW], int d) {
+  const int p = d * VB, wi = p >> 5, sh = p & 31;
+  if (sh + VB > 32) return codes_h2(take_bits(w0, p, VB), take_bits(w1, p, VB));
+  const uint32_t m = (1u << VB) - 1u;
+  const uint32_t lo = ((w0[wi] >> sh) & m) | 0x64006400u;
+  const uint32_t hi = sh <= 16 ? (w1[wi] << (16 - sh)) : (w1[wi] >> (sh - 16));
+  return magic_pair(lo | (hi & (m << 16)));
+}
+
 template <int D, int G, int VB>
 __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const DecodeArgs a) {
   using MG = MixedGeo<D, VB>;
@@ -652,11 +665,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
         mma_f16(oacc[mb], swar_pair<VB>(aw[0], aw[1], 2 * mb), swar_pair<VB>(aw[0], aw[1], 2 * mb + 1),
                 swar_pair<VB>(aw[2], aw[3], 2 * mb), swar_pair<VB>(aw[2], aw[3], 2 * mb + 1), b0, b1);
       } else {
-        const int p0 = 2 * mb * VB, p1 = p0 + VB;
-        mma_f16(oacc[mb], codes_h2(take_bits(aw[0], p0, VB), take_bits(aw[1], p0, VB)),
-                codes_h2(take_bits(aw[0], p1, VB), take_bits(aw[1], p1, VB)),
-                codes_h2(take_bits(aw[2], p0, VB), take_bits(aw[3], p0, VB)),
-                codes_h2(take_bits(aw[2], p1, VB), take_bits(aw[3], p1, VB)), b0, b1);
+        mma_f16(oacc[mb], field_pair<VB>(aw[0], aw[1], 2 * mb), field_pair<VB>(aw[0], aw[1], 2 * mb + 1),
+                field_pair<VB>(aw[2], aw[3], 2 * mb), field_pair<VB>(aw[2], aw[3], 2 * mb + 1), b0, b1);
       }
     }
     __syncwarp();
