@@ -128,7 +128,8 @@ size_t align16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 int decode_ctas_full(const kv4_cache* c, int sms) {
   if (c->format == FMT_INT4) return kv4::decode_ctas_per_sm() * sms;
   if (c->format == FMT_MIXED)
-    return kv4::mixed_decode_ctas_per_sm(c->cfg.head_dim, c->cfg.num_q_heads / c->cfg.num_kv_heads, c->cfg.value_bits) * sms;
+    return kv4::mixed_decode_ctas_per_sm(c->cfg.head_dim, c->cfg.num_q_heads / c->cfg.num_kv_heads, c->cfg.value_bits,
+                                         c->cfg.key_bits) * sms;
   return sms;
 }
 

@@ -91,7 +91,7 @@ cudaError_t launch_decode_bf16(DecodeArgs a, int D, int G, int ctas, cudaStream_
 cudaError_t launch_mixed_score(const ScoreArgs& a, int D, cudaStream_t st);
 cudaError_t launch_append_mixed(const AppendArgs& a, int D, cudaStream_t st);
 int mixed_decode_warps_per_cta();
-int mixed_decode_ctas_per_sm(int D, int G, int value_bits);
+int mixed_decode_ctas_per_sm(int D, int G, int value_bits, int key_bits);
 cudaError_t launch_decode_mixed(DecodeArgs a, int D, int G, int ctas, cudaStream_t st);
 
 // Counts every kernel launch the library issues.

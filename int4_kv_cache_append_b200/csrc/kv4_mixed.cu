@@ -248,24 +248,24 @@ __global__ void __launch_bounds__(kAppendThreads) append_mixed_kernel(AppendArgs
 // ------------------------------------------------------------------ decode
 
 constexpr int kWarps = 8;
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 
 template <int D, int VB>
 struct MixedGeo {
   static constexpr int NK = D / 16;              // k steps of QK^T, m blocks of PV
   static constexpr int VR = VB * D / 8;          // value row bytes
-  static constexpr int VO = 16 * D;              // value rows in a stage (key rows hold <= D bytes)
-  static constexpr int PO = VO + 16 * VR;        // parameter records in a stage
-  static constexpr int STAGE = PO + 128;
   static constexpr int DPL = D / 8;              // value dims per lane (PV rows gq, gq + 8)
   static constexpr int WIN = DPL * VB;           // value bits per lane and token
   static constexpr int NWA = (WIN + 31) / 32;    // aligned window words
-  static_assert(STAGE % 16 == 0, "stage size");
 };
 
-template <int D, int G, int VB>
-struct SmemMixed {
-  uint8_t ring[kWarps][kStages][MixedGeo<D, VB>::STAGE];
+// A ring stage holds one 16-position slice of a (page, KV head) tile in the page's own layout:
+// 16 key rows of KR bytes, 16 value rows of VR bytes, 16 records of 8 bytes.  With P = 16 the
+// slice is the whole tile, so one bulk copy fills the stage.
+__host__ __device__ inline int mixed_stage_bytes(int KR, int VR) { return 16 * (KR + VR) + 128; }
+
+template <int D, int G>
+struct SmemMixedFixed {
   float qbuf[kWarps][G][D];
   // key extraction table per (k step kb, lane group tig): the four codes c0..c3 of coordinates
   // tig * D/4 + 4 kb + (0..3) lie in one 32-bit window x of the bit stream starting at bit off0,
@@ -276,6 +276,15 @@ struct SmemMixed {
   uint32_t stage_ok[kWarps][kStages];  // 1 when the stage's page id was inside the pool
   uint64_t bar[kWarps][kStages];
 };
+
+// the per-warp rings follow the fixed part, sized at launch from the row widths
+template <int D, int G>
+constexpr size_t kMixedFixedBytes = (sizeof(SmemMixedFixed<D, G>) + 127) & ~static_cast<size_t>(127);
+
+template <int D, int G>
+size_t mixed_smem_bytes(int KR, int VR) {
+  return kMixedFixedBytes<D, G> + static_cast<size_t>(kWarps) * kStages * mixed_stage_bytes(KR, VR);
+}
 
 __device__ __forceinline__ float exp2_fast(float x) {
   float y;
@@ -359,12 +368,14 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
   using MG = MixedGeo<D, VB>;
   constexpr int NK = MG::NK, NB = D / 2, Q4 = D / 4;
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  SmemMixed<D, G, VB>& sm = *reinterpret_cast<SmemMixed<D, G, VB>*>(smem_raw);
+  SmemMixedFixed<D, G>& sm = *reinterpret_cast<SmemMixedFixed<D, G>*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tig = lane & 3;
   const int wid = blockIdx.x * kWarps + warp;
   const int cap = a.stride * a.P;
   const int KR = a.kbits * D / 8;
+  const int SB = mixed_stage_bytes(KR, MG::VR), VO = 16 * KR, PO = 16 * (KR + MG::VR);
+  uint8_t* const ring = smem_raw + kMixedFixedBytes<D, G> + static_cast<size_t>(warp) * kStages * SB;
   const size_t tile_bytes = static_cast<size_t>(a.P) * (KR + MG::VR + 8);
   uint64_t* bars = sm.bar[warp];
   if (lane == 0) {
@@ -381,7 +392,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
   splitk::Cur cons = splitk::cursor_at(a, cap, lane, c0);
   splitk::Cur prod = cons;
   const long long nslots = c1 - c0;
-  const uint32_t stage_tx = static_cast<uint32_t>(16 * KR + 16 * MG::VR + 128);
+  const uint32_t stage_tx = static_cast<uint32_t>(SB);
 
   // Called by the whole warp: every lane reads the same page-table entry (one request); lane 0
   // arms the barrier and records whether the page is valid, then lanes 0, 1 and 2 each start one
@@ -396,17 +407,18 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
       mbar_arrive_expect_tx(&bars[st], ok ? stage_tx : 0u);
     }
     __syncwarp();
-    if (ok && lane < 3) {
+    if (ok && lane < (a.P == 16 ? 1 : 3)) {
       const int r0 = c.i * 16 - lp * a.P;
       const uint8_t* tile = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(c.g) * tile_bytes;
-      uint8_t* dst = sm.ring[warp][st];
+      uint8_t* dst = ring + st * SB;
       const uint64_t pol = l2_policy_evict_first();
-      if (lane == 0) bulk_g2s_hint(dst, tile + static_cast<size_t>(r0) * KR, 16 * KR, &bars[st], pol);
+      if (a.P == 16) bulk_g2s_hint(dst, tile, static_cast<uint32_t>(SB), &bars[st], pol);  // the whole tile
+      else if (lane == 0) bulk_g2s_hint(dst, tile + static_cast<size_t>(r0) * KR, 16 * KR, &bars[st], pol);
       else if (lane == 1)
-        bulk_g2s_hint(dst + MG::VO, tile + static_cast<size_t>(a.P) * KR + static_cast<size_t>(r0) * MG::VR,
+        bulk_g2s_hint(dst + VO, tile + static_cast<size_t>(a.P) * KR + static_cast<size_t>(r0) * MG::VR,
                       16 * MG::VR, &bars[st], pol);
       else
-        bulk_g2s_hint(dst + MG::PO, tile + static_cast<size_t>(a.P) * (KR + MG::VR) + static_cast<size_t>(r0) * 8, 128,
+        bulk_g2s_hint(dst + PO, tile + static_cast<size_t>(a.P) * (KR + MG::VR) + static_cast<size_t>(r0) * 8, 128,
                       &bars[st], pol);
     }
   };
@@ -565,7 +577,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
       failed = true;
       break;
     }
-    const uint8_t* buf = sm.ring[warp][st];
+    const uint8_t* buf = ring + st * SB;
     const bool page_ok = sm.stage_ok[warp][st] != 0u;
     const int L = Lseg;
     const int i0 = cons.i * 16;
@@ -591,7 +603,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
               magic_pair(((z0 & E1.y) | 0x64006400u) | ((z0 << E1.w) & E1.z)),
               magic_pair(((z1 & E1.y) | 0x64006400u) | ((z1 << E1.w) & E1.z)), qf[kb][0], qf[kb][1]);
     }
-    const __half* prm = reinterpret_cast<const __half*>(buf + MG::PO);
+    const __half* prm = reinterpret_cast<const __half*>(buf + PO);
     const float s0 = v0 ? __half2float(prm[4 * gq]) : 0.f, s1 = v1 ? __half2float(prm[4 * (gq + 8)]) : 0.f;
     const float lg0 = v0 ? s0 * fmaf(S[0] + S[1], inv_scale, cst) : kNegInf;
     const float lg1 = v1 ? s1 * fmaf(S[2] + S[3], inv_scale, cst) : kNegInf;
@@ -648,7 +660,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
     const int bit0 = gq * MG::WIN;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const uint32_t* vr = reinterpret_cast<const uint32_t*>(buf + MG::VO + tk[u] * MG::VR);
+      const uint32_t* vr = reinterpret_cast<const uint32_t*>(buf + VO + tk[u] * MG::VR);
       uint32_t raw[MG::NWA + 1];
 #pragma unroll
       for (int x = 0; x <= MG::NWA; ++x) raw[x] = vr[(bit0 >> 5) + x];
@@ -693,9 +705,11 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
 
 template <int D, int G, int VB>
 cudaError_t launch_dgv(const DecodeArgs& a, int ctas, cudaStream_t st) {
-  const int smem = static_cast<int>(sizeof(SmemMixed<D, G, VB>));
+  const int smem = static_cast<int>(mixed_smem_bytes<D, G>(a.kbits * D / 8, VB * D / 8));
+  // the attribute is raised once, to the size of the widest key rows (8 bits per dimension)
   static std::atomic<uint64_t> done;
-  cudaError_t e = ensure_smem_limit(decode_mixed_kernel<D, G, VB>, smem, done);
+  cudaError_t e = ensure_smem_limit(decode_mixed_kernel<D, G, VB>, static_cast<int>(mixed_smem_bytes<D, G>(D, VB * D / 8)),
+                                    done);
   if (e != cudaSuccess) return e;
   decode_mixed_kernel<D, G, VB><<<ctas, kWarps * 32, smem, st>>>(a);
   e = cudaGetLastError();
@@ -739,24 +753,13 @@ cudaError_t launch_append_mixed(const AppendArgs& a, int D, cudaStream_t st) {
 
 int mixed_decode_warps_per_cta() { return kWarps; }
 
-// Two CTAs per SM where their shared memory fits (it does for value_bits <= 4), else one.
-int mixed_decode_ctas_per_sm(int D, int G, int VB) {
+// Two CTAs per SM where their shared memory fits (rows of up to 12 bytes per dimension pair at
+// D = 128, e.g. K3V3 or K4V4), else one.
+int mixed_decode_ctas_per_sm(int D, int G, int VB, int KB) {
+  const int KR = KB * D / 8, VR = VB * D / 8;
   size_t bytes = 0;
-  auto pick = [&](auto d, auto g) {
-    constexpr int DD = decltype(d)::value, GG = decltype(g)::value;
-    bytes = VB == 2 ? sizeof(SmemMixed<DD, GG, 2>) : VB == 3 ? sizeof(SmemMixed<DD, GG, 3>)
-            : VB == 4 ? sizeof(SmemMixed<DD, GG, 4>) : sizeof(SmemMixed<DD, GG, 8>);
-  };
-  using I128 = std::integral_constant<int, 128>;
-  using I64 = std::integral_constant<int, 64>;
-  using G1 = std::integral_constant<int, 1>;
-  using G2 = std::integral_constant<int, 2>;
-  using G4 = std::integral_constant<int, 4>;
-  if (D == 128) {
-    if (G == 4) pick(I128{}, G4{}); else if (G == 2) pick(I128{}, G2{}); else pick(I128{}, G1{});
-  } else {
-    if (G == 4) pick(I64{}, G4{}); else if (G == 2) pick(I64{}, G2{}); else pick(I64{}, G1{});
-  }
+  if (D == 128) bytes = G == 4 ? mixed_smem_bytes<128, 4>(KR, VR) : G == 2 ? mixed_smem_bytes<128, 2>(KR, VR) : mixed_smem_bytes<128, 1>(KR, VR);
+  else bytes = G == 4 ? mixed_smem_bytes<64, 4>(KR, VR) : G == 2 ? mixed_smem_bytes<64, 2>(KR, VR) : mixed_smem_bytes<64, 1>(KR, VR);
   return 2 * (bytes + 1024) <= 227u * 1024u ? 2 : 1;
 }
 
