@@ -126,7 +126,8 @@ typedef struct kv4_cache kv4_cache;  /* opaque host handle */
  * bf16 V) and 3D + 2 in the side cache (INT8 K and its scale, bf16 V).
  * With KV4_KEYS_MIXED a position takes key_bits*D/8 + value_bits*D/8 + 8 bytes in a page (the
  * packed key and value codes and four fp16: key scale, 0, value zero, value range; a page of one
- * KV head holds P key rows, then P value rows, then P records, heads in order), the side cache is
+ * KV head is P/16 slices of 16 positions, each holding its 16 key rows, then 16 value rows, then
+ * 16 records; heads in order), the side cache is
  * empty, and the page pool ends with num_layers * Hkv block-allocation records of
  * ceil16(5 D / 2) bytes (D/2 fp32 block scales, then D/2 uint8 block widths).
  * Both must be 16-byte aligned.  Returns KV4_ERR_UNSUPPORTED for geometries outside the list.

@@ -19,11 +19,12 @@
 //   - a value gets the per-token affine code of the INT4 cache at value_bits bits: fp16 zero
 //     rounded down, fp16 range rounded up, code = rint((x - zero) / (range / (2^b - 1)));
 //   - codes are packed in coordinate order, least significant bit first, as one little-endian
-//     bit stream per vector; a page tile of one KV head holds P key rows, P value rows and P
-//     8-byte records (key scale, 0, value zero, value range), tiles ordered (page, head).
+//     bit stream per vector; a page tile of one KV head is P/16 slices of 16 positions, each
+//     holding its 16 key rows, 16 value rows and 16 8-byte records (key scale, 0, value zero,
+//     value range), so that a slice is one contiguous block; tiles ordered (page, head).
 //
 // Decode: the same flattened split-K as the BF16 baseline (16-position tiles of one (sequence, KV
-// head), three bulk copies per tile into a per-warp ring, LSE merge).  QK^T runs on m16n8k16 fp16
+// head), one bulk copy per tile into a per-warp ring, LSE merge).  QK^T runs on m16n8k16 fp16
 // MMAs: the integer codes are exact fp16 A operands, the query enters as q_j sigma_j 2^(1-w_j) in
 // hi/lo fp16 halves (columns 2h, 2h+1 of the 8 N columns), and the code-independent part
 // sum_j q_j sigma_j (2^-w_j - 1) is added per head; the MMA's k index is permuted so that each
@@ -229,11 +230,13 @@ __global__ void __launch_bounds__(kAppendThreads) append_mixed_kernel(AppendArgs
   if (lane == 0 && (kbad || vbad)) atomicOr(a.err, KV4_DEVERR_RANGE);
   __syncwarp();
 
-  const int KR = a.kbits * D / 8, VR = a.vbits * D / 8, pp = pos % a.P;
-  uint8_t* tile = a.pool + static_cast<size_t>(page) * a.page_bytes +
-                  static_cast<size_t>(g) * static_cast<size_t>(a.P) * (KR + VR + 8);
-  uint32_t* kdst = reinterpret_cast<uint32_t*>(tile + static_cast<size_t>(pp) * KR);
-  uint32_t* vdst = reinterpret_cast<uint32_t*>(tile + static_cast<size_t>(a.P) * KR + static_cast<size_t>(pp) * VR);
+  const int KR = a.kbits * D / 8, VR = a.vbits * D / 8, pp = pos % a.P, rr = pp & 15;
+  // the position's 16-position slice: 16 key rows, 16 value rows, 16 records
+  uint8_t* slice = a.pool + static_cast<size_t>(page) * a.page_bytes +
+                   static_cast<size_t>(g) * static_cast<size_t>(a.P) * (KR + VR + 8) +
+                   static_cast<size_t>(pp >> 4) * 16 * (KR + VR + 8);
+  uint32_t* kdst = reinterpret_cast<uint32_t*>(slice + static_cast<size_t>(rr) * KR);
+  uint32_t* vdst = reinterpret_cast<uint32_t*>(slice + 16 * static_cast<size_t>(KR) + static_cast<size_t>(rr) * VR);
   for (int i = lane; i < KR / 4; i += 32) kdst[i] = krow[i];
   for (int i = lane; i < VR / 4; i += 32) vdst[i] = vrow[i];
   if (lane == 0) {
@@ -241,7 +244,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_mixed_kernel(AppendArgs
         static_cast<unsigned long long>(__half_as_ushort(ksh)) |
         (static_cast<unsigned long long>(__half_as_ushort(vzh)) << 32) |
         (static_cast<unsigned long long>(__half_as_ushort(vrh)) << 48);
-    *reinterpret_cast<unsigned long long*>(tile + static_cast<size_t>(a.P) * (KR + VR) + static_cast<size_t>(pp) * 8) = rec;
+    *reinterpret_cast<unsigned long long*>(slice + 16 * static_cast<size_t>(KR + VR) + static_cast<size_t>(rr) * 8) = rec;
   }
 }
 
@@ -260,8 +263,7 @@ struct MixedGeo {
 };
 
 // A ring stage holds one 16-position slice of a (page, KV head) tile in the page's own layout:
-// 16 key rows of KR bytes, 16 value rows of VR bytes, 16 records of 8 bytes.  With P = 16 the
-// slice is the whole tile, so one bulk copy fills the stage.
+// 16 key rows of KR bytes, 16 value rows of VR bytes, 16 records of 8 bytes; one bulk copy.
 __host__ __device__ inline int mixed_stage_bytes(int KR, int VR) { return 16 * (KR + VR) + 128; }
 
 template <int D, int G>
@@ -394,32 +396,21 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
   const long long nslots = c1 - c0;
   const uint32_t stage_tx = static_cast<uint32_t>(SB);
 
-  // Called by the whole warp: every lane reads the same page-table entry (one request); lane 0
-  // arms the barrier and records whether the page is valid, then lanes 0, 1 and 2 each start one
-  // of the tile's three bulk copies (keys, values, parameter records).
+  // Lane 0 arms the stage's barrier, records whether the page is valid and starts the bulk copy
+  // of the 16-position slice (16 key rows, 16 value rows, 16 records: one contiguous block).
   auto issue = [&](const splitk::Cur& c, int st) {
+    if (lane != 0) return;
     const int lp = (c.i * 16) / a.P;
     const int page = a.page_table[static_cast<size_t>(c.b) * a.stride + lp];
     const bool ok = page >= 0 && page < a.max_pages;
-    if (lane == 0) {
-      sm.stage_ok[warp][st] = ok ? 1u : 0u;
-      if (!ok) atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
-      mbar_arrive_expect_tx(&bars[st], ok ? stage_tx : 0u);
-    }
-    __syncwarp();
-    if (ok && lane < (a.P == 16 ? 1 : 3)) {
+    sm.stage_ok[warp][st] = ok ? 1u : 0u;
+    if (!ok) atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
+    mbar_arrive_expect_tx(&bars[st], ok ? stage_tx : 0u);
+    if (ok) {
       const int r0 = c.i * 16 - lp * a.P;
-      const uint8_t* tile = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(c.g) * tile_bytes;
-      uint8_t* dst = ring + st * SB;
-      const uint64_t pol = l2_policy_evict_first();
-      if (a.P == 16) bulk_g2s_hint(dst, tile, static_cast<uint32_t>(SB), &bars[st], pol);  // the whole tile
-      else if (lane == 0) bulk_g2s_hint(dst, tile + static_cast<size_t>(r0) * KR, 16 * KR, &bars[st], pol);
-      else if (lane == 1)
-        bulk_g2s_hint(dst + VO, tile + static_cast<size_t>(a.P) * KR + static_cast<size_t>(r0) * MG::VR,
-                      16 * MG::VR, &bars[st], pol);
-      else
-        bulk_g2s_hint(dst + PO, tile + static_cast<size_t>(a.P) * (KR + MG::VR) + static_cast<size_t>(r0) * 8, 128,
-                      &bars[st], pol);
+      const uint8_t* src = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(c.g) * tile_bytes +
+                           static_cast<size_t>(r0 >> 4) * SB;
+      bulk_g2s_hint(ring + st * SB, src, static_cast<uint32_t>(SB), &bars[st], l2_policy_evict_first());
     }
   };
 

@@ -181,21 +181,24 @@ size_t orc_gtq_page_bytes(const orc_gtq_config* c) { return (size_t)c->num_kv_he
 static size_t tile_base(const orc_gtq_config* c, int page, int g) {
   return ((size_t)page * (size_t)c->num_kv_heads + (size_t)g) * orc_gtq_tile_bytes(c);
 }
+/* the 16-position slice of position pp: its 16 key rows, 16 value rows and 16 records */
+static size_t slice_base(const orc_gtq_config* c, int page, int g, int pp) {
+  return tile_base(c, page, g) +
+         (size_t)(pp / 16) * 16u * (orc_gtq_key_row_bytes(c) + orc_gtq_value_row_bytes(c) + 8u);
+}
 size_t orc_gtq_key_row(const orc_gtq_config* c, int page, int g, int pp) {
-  return tile_base(c, page, g) + (size_t)pp * orc_gtq_key_row_bytes(c);
+  return slice_base(c, page, g, pp) + (size_t)(pp % 16) * orc_gtq_key_row_bytes(c);
 }
 size_t orc_gtq_value_row(const orc_gtq_config* c, int page, int g, int pp) {
-  return tile_base(c, page, g) + (size_t)c->page_size * orc_gtq_key_row_bytes(c) +
-         (size_t)pp * orc_gtq_value_row_bytes(c);
+  return slice_base(c, page, g, pp) + 16u * orc_gtq_key_row_bytes(c) + (size_t)(pp % 16) * orc_gtq_value_row_bytes(c);
 }
 size_t orc_gtq_param(const orc_gtq_config* c, int page, int g, int pp) {
-  return tile_base(c, page, g) + (size_t)c->page_size * (orc_gtq_key_row_bytes(c) + orc_gtq_value_row_bytes(c)) +
-         (size_t)pp * 8;
+  return slice_base(c, page, g, pp) + 16u * (orc_gtq_key_row_bytes(c) + orc_gtq_value_row_bytes(c)) + (size_t)(pp % 16) * 8u;
 }
 
 static int gtq_config_ok(const orc_gtq_config* c) {
   return c->num_kv_heads > 0 && c->num_q_heads % c->num_kv_heads == 0 && c->head_dim > 0 &&
-         c->head_dim % 2 == 0 && c->page_size > 0 && c->key_bits >= 1 && c->key_bits <= 8 &&
+         c->head_dim % 2 == 0 && c->page_size > 0 && c->page_size % 16 == 0 && c->key_bits >= 1 && c->key_bits <= 8 &&
          c->value_bits >= 1 && c->value_bits <= 8 && (c->key_bits * c->head_dim) % 8 == 0 &&
          (c->value_bits * c->head_dim) % 8 == 0;
 }

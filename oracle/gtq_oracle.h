@@ -44,9 +44,11 @@
  *   G6 packing: the codes of one vector in coordinate order, each in its width, least
  *      significant bit first, as one little-endian bit stream (bit n of the stream is bit n & 7
  *      of byte n >> 3): key_bits * D / 8 bytes per key, value_bits * D / 8 per value.
- *   G7 page tile of one (page, KV head), P positions: P key rows, then P value rows, then P
- *      parameter records of four fp16 (key scale, a zero pad, value zero, value range); tiles ordered
- *      (page, head).  No rotation, no side cache: the abstract's method needs neither.
+ *   G7 page tile of one (page, KV head), P positions (P a multiple of 16): P/16 slices of 16
+ *      positions, each holding its 16 key rows, then its 16 value rows, then 16 parameter records
+ *      of four fp16 (key scale, a zero pad, value zero, value range); tiles ordered (page, head).
+ *      A slice is one contiguous block whatever P is.  No rotation, no side cache: the
+ *      abstract's method needs neither.
  *   G8 attention: as for the INT4 cache, q head j reads KV head j / (Hq/Hkv), softmax scale
  *      1/sqrt(D), one softmax over [0, L), in fp64 on the dequantised cache.
  */
@@ -63,7 +65,7 @@ typedef struct {
   int num_q_heads;   /* Hq                                   */
   int num_kv_heads;  /* Hkv, Hq % Hkv == 0                   */
   int head_dim;      /* D, even, D * key_bits % 8 == 0 ...   */
-  int page_size;     /* P                                    */
+  int page_size;     /* P, a multiple of 16                  */
   int key_bits;      /* average key bits per dimension, 1..8 */
   int value_bits;    /* value bits per dimension, 1..8       */
 } orc_gtq_config;

@@ -306,11 +306,13 @@ def _brute_gtq_decode(wl, cfg, widths, sigma, pool, q, lens):
             vh = np.zeros((L, D))
             for t in range(L):
                 page = int(wl.page_table[b, t // P])
-                base = (page * wl.Hkv + g) * tile
                 pp = t % P
-                prm = pool[base + P * (kr + vr) + 8 * pp: base + P * (kr + vr) + 8 * pp + 8].view(np.float16).astype(float)
-                kint = int.from_bytes(pool[base + pp * kr: base + (pp + 1) * kr].tobytes(), "little")
-                vint = int.from_bytes(pool[base + P * kr + pp * vr: base + P * kr + (pp + 1) * vr].tobytes(), "little")
+                # slice of 16 positions: 16 key rows, 16 value rows, 16 records of 8 bytes
+                base = (page * wl.Hkv + g) * tile + (pp // 16) * 16 * (kr + vr + 8)
+                rr = pp % 16
+                prm = pool[base + 16 * (kr + vr) + 8 * rr: base + 16 * (kr + vr) + 8 * rr + 8].view(np.float16).astype(float)
+                kint = int.from_bytes(pool[base + rr * kr: base + (rr + 1) * kr].tobytes(), "little")
+                vint = int.from_bytes(pool[base + 16 * kr + rr * vr: base + 16 * kr + (rr + 1) * vr].tobytes(), "little")
                 o = 0
                 for i in range(D):
                     w = wk[i]
@@ -333,8 +335,9 @@ def _brute_gtq_decode(wl, cfg, widths, sigma, pool, q, lens):
 
 
 def pin_gtq_brute_force_decode():
-    for kb, vb, lens, D in ((3, 3, (12, 7, 40), 32), (2, 4, (1, 33, 16), 32), (5, 2, (17, 3, 9), 16)):
-        wl = gtq_workload(D=D, lens=lens)
+    for kb, vb, lens, D, P in ((3, 3, (12, 7, 40), 32, 16), (2, 4, (1, 33, 16), 32, 16), (5, 2, (17, 3, 9), 16, 16),
+                               (3, 3, (70, 5, 33), 32, 32), (4, 2, (100, 49, 17), 16, 48)):
+        wl = gtq_workload(D=D, lens=lens, P=P)
         cfg, widths, sigma, pool = gtq_oracle_cache(wl, kb, vb)
         assert int(widths.sum()) == kb * D // 2 * wl.Hkv
         q = wl.q_input(0)

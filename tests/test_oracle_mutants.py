@@ -80,8 +80,10 @@ GTQ_MUTANTS = [
     ("gtq-value-levels-2w", "const int top = (1 << bits) - 1;", "const int top = (1 << bits);", 0),
     ("gtq-value-zero-round-nearest", "const uint16_t zb = orc_f32_to_f16(mn, ORC_RD);", "const uint16_t zb = orc_f32_to_f16(mn, ORC_RN);", None),
     ("gtq-pack-msb-first", "row[n >> 3] |= (uint8_t)(1u << (n & 7));", "row[n >> 3] |= (uint8_t)(0x80u >> (n & 7));", None),
-    ("gtq-value-rows-after-params", "return tile_base(c, page, g) + (size_t)c->page_size * orc_gtq_key_row_bytes(c) +\n         (size_t)pp * orc_gtq_value_row_bytes(c);",
-     "return tile_base(c, page, g) + (size_t)c->page_size * (orc_gtq_key_row_bytes(c) + 8) +\n         (size_t)pp * orc_gtq_value_row_bytes(c);", None),
+    ("gtq-value-rows-after-params", "return slice_base(c, page, g, pp) + 16u * orc_gtq_key_row_bytes(c) + (size_t)(pp % 16) * orc_gtq_value_row_bytes(c);",
+     "return slice_base(c, page, g, pp) + 16u * (orc_gtq_key_row_bytes(c) + 8u) + (size_t)(pp % 16) * orc_gtq_value_row_bytes(c);", None),
+    ("gtq-page-major-not-slice-major", "(size_t)(pp / 16) * 16u * (orc_gtq_key_row_bytes(c) + orc_gtq_value_row_bytes(c) + 8u);",
+     "0u; (void)pp;", None),
     ("gtq-param-order", "put16(pool + orc_gtq_param(c, page, g, pp) + 4, z);", "put16(pool + orc_gtq_param(c, page, g, pp) + 6, z);", None),
     ("gtq-block-of-coordinate", "wc[i] = widths[(size_t)g * (size_t)nb + (size_t)(i % nb)];", "wc[i] = widths[(size_t)g * (size_t)nb + (size_t)(i / 2)];", None),
     ("gtq-softmax-scale", "const double tau = 1.0 / sqrt((double)D);", "const double tau = 1.0 / (double)D;", None),
