@@ -262,18 +262,28 @@ struct MixedGeo {
   static constexpr int NWA = (WIN + 31) / 32;    // aligned window words
 };
 
-// A ring stage holds one 16-position slice of a (page, KV head) tile in the page's own layout:
-// 16 key rows of KR bytes, 16 value rows of VR bytes, 16 records of 8 bytes; one bulk copy.
-__host__ __device__ inline int mixed_stage_bytes(int KR, int VR) { return 16 * (KR + VR) + 128; }
+// A 16-position slice of a (page, KV head) tile in the page's own layout: 16 key rows of KR bytes,
+// 16 value rows of VR bytes, 16 records of 8 bytes; one bulk copy.
+__host__ __device__ inline int mixed_slice_bytes(int KR, int VR) { return 16 * (KR + VR) + 128; }
+
+// A ring stage: 16 guard bytes, then the slice.  A key window may start up to 10 bits before its
+// row (see the extraction table), so row 0 reads the word before it: the guard keeps that read
+// inside the stage, off the previous stage, whose copy may still be landing.  Its bits are masked.
+constexpr int kStageGuard = 16;
+__host__ __device__ inline int mixed_stage_bytes(int KR, int VR) { return kStageGuard + mixed_slice_bytes(KR, VR); }
 
 template <int D, int G>
 struct SmemMixedFixed {
   float qbuf[kWarps][G][D];
-  // key extraction table per (k step kb, lane group tig): the four codes c0..c3 of coordinates
-  // tig * D/4 + 4 kb + (0..3) lie in one 32-bit window x of the bit stream starting at bit off0,
-  // at offsets r0 = 0, r1, r2, r3.  Words: m0, m1 << 16, 16 - r1, off0 | r2, m2, m3 << 16,
-  // 16 - (r3 - r2) (m = the code's width mask): (x & m0) | (x << (16 - r1)) & (m1 << 16) is the
-  // pair (c0, c1) in two 16-bit halves, and likewise (c2, c3) from x >> r2.
+  // key extraction table per (k step kb, lane group tig).  The four codes c0..c3 (widths w0..w3,
+  // sum W <= 32) of coordinates tig * D/4 + 4 kb + (0..3) follow each other in the bit stream from
+  // bit off0.  The 32-bit window x starts t0 = min(10 - w0, 32 - W) bits before off0, so c0 sits
+  // at the top of a mantissa field, or at most two bits below it when the four are wide.  Then
+  // (x & M0) | (x 2^(26 - w1 - t0 - w0) & M1) is the subnormal pair (c0, c1) with M0 = (2^w0 - 1)
+  // << t0 and M1 = (2^w1 - 1) << (26 - w1); z = x >> (t0 + w0 + w1 - 10 + w2) puts c2 at the top
+  // of the low field and c3 at bit 10, and (z & M2) | (z 2^(16 - w3) & M3) is (c2, c3).  Words:
+  // M0, M1, 2^(26 - w1 - t0 - w0), off0 - t0 (may be negative), the shift of z, M2, M3,
+  // 2^(16 - w3).  The shifts into the high half are multiplies, which run on the FMA pipe.
   uint32_t ktab[kWarps][D / 16][4][8];
   uint32_t stage_ok[kWarps][kStages];  // 1 when the stage's page id was inside the pool
   uint64_t bar[kWarps][kStages];
@@ -305,19 +315,22 @@ __device__ __forceinline__ uint32_t split_h2(float x0, float x1, bool lo) {
   return static_cast<uint32_t>(__half_as_ushort(r0)) | (static_cast<uint32_t>(__half_as_ushort(r1)) << 16);
 }
 
-// two integer codes (< 1024) as the exact fp16 pair (c0, c1): 1024 + c in the 0x6400 exponent, minus 1024
-__device__ __forceinline__ uint32_t codes_h2(uint32_t c0, uint32_t c1) {
-  const uint32_t h = prmt(c0, c1, 0x5410u) | 0x64006400u;
-  __half2 v = *reinterpret_cast<const __half2*>(&h);
-  v = __hsub2(v, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
-  return *reinterpret_cast<uint32_t*>(&v);
-}
+// Integer codes enter the fp16 MMAs as subnormal halves.  A w-bit code c placed at the top of the
+// 10-bit mantissa field, bit pattern c 2^(10 - w), is the half c 2^(10 - w) 2^-24 exactly, and a
+// pair of them is built from the packed bits with shifts (or multiplies) and masks alone.  The
+// tensor cores take subnormal operands, but a product keeps fewer low bits the more leading zeros
+// its subnormal operand has; at the top of the field the sums come out as those of the same codes
+// given as normal halves.  The constant 2^(10 - w - 24) goes into the query weights (keys) and
+// the partial's scale (values).
+constexpr int kSubTop = 10;
 
-// (1024 + c0, 1024 + c1) with the 0x6400 exponent in both halves -> the exact fp16 pair (c0, c1)
-__device__ __forceinline__ uint32_t magic_pair(uint32_t h) {
-  __half2 v = *reinterpret_cast<const __half2*>(&h);
-  v = __hsub2(v, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
-  return *reinterpret_cast<uint32_t*>(&v);
+// x shifted left by n bits (right by -n when n < 0); n is compile-time after unrolling
+__device__ __forceinline__ uint32_t shift_to(uint32_t x, int n) { return n >= 0 ? x << n : x >> -n; }
+
+// value codes c0, c1 (< 2^VB) -> the subnormal pair (c0 2^(10 - VB), c1 2^(10 - VB))
+template <int VB>
+__device__ __forceinline__ uint32_t codes_h2(uint32_t c0, uint32_t c1) {
+  return prmt(c0, c1, 0x5410u) << (kSubTop - VB);
 }
 
 // bits [p, p + w) of a bit array held in words aw (p and w compile-time after unrolling)
@@ -330,39 +343,45 @@ __device__ __forceinline__ uint32_t take_bits(const uint32_t (&aw)[NW], int p, i
 }
 
 // Value widths whose fields never straddle a byte: the PV operands are cut out with byte
-// permutes and masks, each field keeping its position s within its byte (code * 2^s), and the
-// partial's rows are scaled back by 2^-s at the flush.
+// permutes and masks.
 template <int VB>
 constexpr bool kSwarV = VB == 2 || VB == 4 || VB == 8;
 
-// bit position within its byte of the value field of lane dim d
+// Bit position of the value field of lane dim d within its half once it is cut out.  A field at bit
+// s of its byte whose top bit is at bit 7 (two leading zeros in the mantissa field at most) stays
+// where it is; a lower one is lifted to the top of the field.  Odd widths always go to the top.
 template <int VB>
-__host__ __device__ constexpr int swar_shift(int d) { return (d * VB) & 7; }
-
-// (code of dim d of token t0, same of t1) * 2^swar_shift(d) as an exact fp16 pair
-template <int VB, int NW>
-__device__ __forceinline__ uint32_t swar_pair(const uint32_t (&w0)[NW], const uint32_t (&w1)[NW], int d) {
-  const int byte = (d * VB) >> 3, sh = swar_shift<VB>(d);
-  const uint32_t sel = static_cast<uint32_t>((byte & 3) | ((4 + (byte & 3)) << 8));
-  const uint32_t x = prmt(w0[byte >> 2], w1[byte >> 2], sel);
-  const uint32_t m = ((1u << VB) - 1u) << sh;
-  const uint32_t h = (x & (m | (m << 16))) | 0x64006400u;
-  __half2 v = *reinterpret_cast<const __half2*>(&h);
-  v = __hsub2(v, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
-  return *reinterpret_cast<uint32_t*>(&v);
+__host__ __device__ constexpr int value_field_pos(int d) {
+  return !kSwarV<VB> ? kSubTop - VB : (((d * VB) & 7) + VB >= 8 ? (d * VB) & 7 : kSubTop - VB);
 }
 
-// (code of dim d of token t0, same of t1) as an exact fp16 pair, for any value width: a field
-// inside one word takes a shift and a mask with the 0x6400 exponent for t0, one shift for t1 and
-// one mask-or to join them; a field across two words goes through take_bits.
+// the value codes of lane dim d entered the MMAs as c 2^(value_field_pos(d) - 24)
+template <int VB>
+__host__ __device__ constexpr float value_unscale(int d) {
+  return static_cast<float>(1 << (24 - value_field_pos<VB>(d)));
+}
+
+// (code of dim d of token t0, same of t1) as a subnormal pair, byte-aligned widths: one permute
+// puts the field's byte of both tokens into the two halves, a low field is shifted up, one mask
+// keeps both fields
+template <int VB, int NW>
+__device__ __forceinline__ uint32_t swar_pair(const uint32_t (&w0)[NW], const uint32_t (&w1)[NW], int d) {
+  const int byte = (d * VB) >> 3, sh = (d * VB) & 7, pos = value_field_pos<VB>(d);
+  const uint32_t sel = static_cast<uint32_t>((byte & 3) | ((4 + (byte & 3)) << 8));
+  const uint32_t x = prmt(w0[byte >> 2], w1[byte >> 2], sel);
+  const uint32_t m = ((1u << VB) - 1u) << pos;
+  return (pos > sh ? x << (pos - sh) : x) & (m | (m << 16));
+}
+
+// (code of dim d of token t0, same of t1) as a subnormal pair, any value width: a field inside one
+// word takes one shift per token and a mask-or to join them; a field across two words goes
+// through take_bits.
 template <int VB, int NW>
 __device__ __forceinline__ uint32_t field_pair(const uint32_t (&w0)[NW], const uint32_t (&w1)[NW], int d) {
   const int p = d * VB, wi = p >> 5, sh = p & 31;
-  if (sh + VB > 32) return codes_h2(take_bits(w0, p, VB), take_bits(w1, p, VB));
-  const uint32_t m = (1u << VB) - 1u;
-  const uint32_t lo = ((w0[wi] >> sh) & m) | 0x64006400u;
-  const uint32_t hi = sh <= 16 ? (w1[wi] << (16 - sh)) : (w1[wi] >> (sh - 16));
-  return magic_pair(lo | (hi & (m << 16)));
+  if (sh + VB > 32) return codes_h2<VB>(take_bits(w0, p, VB), take_bits(w1, p, VB));
+  const uint32_t m = ((1u << VB) - 1u) << (kSubTop - VB);
+  return (shift_to(w0[wi], kSubTop - VB - sh) & m) | (shift_to(w1[wi], kSubTop + 16 - VB - sh) & (m << 16));
 }
 
 template <int D, int G, int VB>
@@ -376,7 +395,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
   const int wid = blockIdx.x * kWarps + warp;
   const int cap = a.stride * a.P;
   const int KR = a.kbits * D / 8;
-  const int SB = mixed_stage_bytes(KR, MG::VR), VO = 16 * KR, PO = 16 * (KR + MG::VR);
+  const int SB = mixed_stage_bytes(KR, MG::VR), SL = mixed_slice_bytes(KR, MG::VR);
+  const int VO = 16 * KR, PO = 16 * (KR + MG::VR);
   uint8_t* const ring = smem_raw + kMixedFixedBytes<D, G> + static_cast<size_t>(warp) * kStages * SB;
   const size_t tile_bytes = static_cast<size_t>(a.P) * (KR + MG::VR + 8);
   uint64_t* bars = sm.bar[warp];
@@ -394,7 +414,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
   splitk::Cur cons = splitk::cursor_at(a, cap, lane, c0);
   splitk::Cur prod = cons;
   const long long nslots = c1 - c0;
-  const uint32_t stage_tx = static_cast<uint32_t>(SB);
+  const uint32_t stage_tx = static_cast<uint32_t>(SL);
 
   // Lane 0 arms the stage's barrier, records whether the page is valid and starts the bulk copy
   // of the 16-position slice (16 key rows, 16 value rows, 16 records: one contiguous block).
@@ -409,8 +429,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
     if (ok) {
       const int r0 = c.i * 16 - lp * a.P;
       const uint8_t* src = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(c.g) * tile_bytes +
-                           static_cast<size_t>(r0 >> 4) * SB;
-      bulk_g2s_hint(ring + st * SB, src, static_cast<uint32_t>(SB), &bars[st], l2_policy_evict_first());
+                           static_cast<size_t>(r0 >> 4) * SL;
+      bulk_g2s_hint(ring + st * SB + kStageGuard, src, static_cast<uint32_t>(SL), &bars[st], l2_policy_evict_first());
     }
   };
 
@@ -447,24 +467,31 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
       const int j = lane + 32 * i, c = (j % NB) / 32;
       const int w = wv[c];
       const int off = (j >= NB ? run : 0) + pre[c];
-      const int off0 = __shfl_sync(FULL, off, lane & ~3);  // first coordinate of the group of four
-      const int off2 = __shfl_sync(FULL, off, (lane & ~3) + 2);
+      // the group of four coordinates is four consecutive lanes
+      const int g0 = lane & ~3;
+      const int off0 = __shfl_sync(FULL, off, g0);
+      const int w0 = __shfl_sync(FULL, w, g0), w1 = __shfl_sync(FULL, w, g0 + 1);
+      const int w2 = __shfl_sync(FULL, w, g0 + 2), w3 = __shfl_sync(FULL, w, g0 + 3);
+      // the code's field sits at bit 10 - w of its half, except c0 of a wide group, which sits at t0
+      float lift = 1.f;
       {
         const int r = j % Q4, kb = r >> 2, e = r & 3;
         uint32_t* ent = ktab + (kb * 4 + j / Q4) * 8;
+        const int t0 = min(kSubTop - w0, 32 - (w0 + w1 + w2 + w3));
         const uint32_t m = (1u << w) - 1u;
         if (e == 0) {
-          ent[0] = m;
-          ent[3] = static_cast<uint32_t>(off);
+          lift = static_cast<float>(1 << (kSubTop - w0 - t0));
+          ent[0] = m << t0;
+          ent[3] = static_cast<uint32_t>(off0 - t0);
         } else if (e == 1) {
-          ent[1] = m << 16;
-          ent[2] = static_cast<uint32_t>(16 - (off - off0));
+          ent[1] = m << (kSubTop + 16 - w);
+          ent[2] = 1u << (kSubTop + 16 - w - t0 - w0);
         } else if (e == 2) {
-          ent[4] = static_cast<uint32_t>(off - off0);
-          ent[5] = m;
+          ent[4] = static_cast<uint32_t>(t0 + w0 + w1 - (kSubTop - w));
+          ent[5] = m << (kSubTop - w);
         } else {
-          ent[6] = m << 16;
-          ent[7] = static_cast<uint32_t>(16 - (off - off2));
+          ent[6] = m << (kSubTop + 16 - w);
+          ent[7] = 1u << (16 - w);
         }
       }
       const float sgm = sig[j % NB];
@@ -472,7 +499,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
       for (int h = 0; h < G; ++h) {
         const size_t qi = (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G + h) * D + j;
         const float qs = load_elem(a.q, a.q_dtype, qi) * sgm * a.qscale;
-        const float qq = w > 0 ? qs * __int_as_float((128 - w) << 23) : 0.f;      // qs 2^(1-w)
+        // the weight of code c is qs 2^(1 - w); the code enters as c 2^(10 - w - 24) / lift, and
+        // the remaining 2^(1 - w) / 2^(10 - w - 24) = 2^15 is in inv_scale
+        const float qq = w > 0 ? qs * lift : 0.f;
         if (w > 0) csum[h] += qs * (__int_as_float((127 - w) << 23) - 1.0f);      // qs (2^-w - 1)
         qb[h * D + j] = qq;
         amax = fmaxf(amax, fabsf(qq));
@@ -492,7 +521,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
     int ex = 0;
     if (amax > 0.f) frexpf(amax, &ex);
     const float scale = ldexpf(1.f, 8 - ex);
-    inv_scale = ldexpf(1.f, ex - 8);
+    inv_scale = ldexpf(1.f, ex - 8 + 15);
     __syncwarp();
     const int hh = gq >> 1;
     const bool lo = gq & 1;
@@ -532,9 +561,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
 #pragma unroll
       for (int mb = 0; mb < NK; ++mb) {
         const int d = MG::DPL * gq + 2 * mb;
-        // byte-aligned value widths left the codes of dims 2 mb, 2 mb + 1 at 2^s (exact)
-        const float f0 = kSwarV<VB> ? 1.0f / static_cast<float>(1 << swar_shift<VB>(2 * mb)) : 1.0f;
-        const float f1 = kSwarV<VB> ? 1.0f / static_cast<float>(1 << swar_shift<VB>(2 * mb + 1)) : 1.0f;
+        const float f0 = value_unscale<VB>(2 * mb), f1 = value_unscale<VB>(2 * mb + 1);
         *reinterpret_cast<float2*>(p + d) =
             make_float2(fmaf(oacc[mb][0] + oacc[mb][1], f0, z), fmaf(oacc[mb][2] + oacc[mb][3], f1, z));
       }
@@ -568,7 +595,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
       failed = true;
       break;
     }
-    const uint8_t* buf = ring + st * SB;
+    const uint8_t* buf = ring + st * SB + kStageGuard;
     const bool page_ok = sm.stage_ok[warp][st] != 0u;
     const int L = Lseg;
     const int i0 = cons.i * 16;
@@ -583,16 +610,14 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
 #pragma unroll
     for (int kb = 0; kb < NK; ++kb) {
       const uint32_t* ent = ktab + (kb * 4 + tig) * 8;
-      const uint4 E0 = *reinterpret_cast<const uint4*>(ent);      // m0, m1 << 16, 16 - r1, off0
-      const uint4 E1 = *reinterpret_cast<const uint4*>(ent + 4);  // r2, m2, m3 << 16, 16 - (r3 - r2)
-      const int wi = static_cast<int>(E0.w >> 5), sh = static_cast<int>(E0.w & 31u);
+      const uint4 E0 = *reinterpret_cast<const uint4*>(ent);      // M0, M1, multiplier of c1, window start
+      const uint4 E1 = *reinterpret_cast<const uint4*>(ent + 4);  // shift of z, M2, M3, multiplier of c3
+      const int wi = static_cast<int>(E0.w) >> 5, sh = static_cast<int>(E0.w & 31u);  // wi = -1 reads the guard
       const uint32_t x0 = __funnelshift_r(r0w[wi], r0w[wi + 1], sh);
       const uint32_t x1 = __funnelshift_r(r1w[wi], r1w[wi + 1], sh);
       const uint32_t z0 = x0 >> E1.x, z1 = x1 >> E1.x;
-      mma_f16(S, magic_pair(((x0 & E0.x) | 0x64006400u) | ((x0 << E0.z) & E0.y)),
-              magic_pair(((x1 & E0.x) | 0x64006400u) | ((x1 << E0.z) & E0.y)),
-              magic_pair(((z0 & E1.y) | 0x64006400u) | ((z0 << E1.w) & E1.z)),
-              magic_pair(((z1 & E1.y) | 0x64006400u) | ((z1 << E1.w) & E1.z)), qf[kb][0], qf[kb][1]);
+      mma_f16(S, (x0 & E0.x) | ((x0 * E0.z) & E0.y), (x1 & E0.x) | ((x1 * E0.z) & E0.y),
+              (z0 & E1.y) | ((z0 * E1.w) & E1.z), (z1 & E1.y) | ((z1 * E1.w) & E1.z), qf[kb][0], qf[kb][1]);
     }
     const __half* prm = reinterpret_cast<const __half*>(buf + PO);
     const float s0 = v0 ? __half2float(prm[4 * gq]) : 0.f, s1 = v1 ? __half2float(prm[4 * (gq + 8)]) : 0.f;
@@ -663,8 +688,6 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
 #pragma unroll
     for (int mb = 0; mb < NK; ++mb) {
       if constexpr (kSwarV<VB>) {
-        // byte-aligned fields: one prmt puts byte k of two tokens' windows into the two halves,
-        // one mask keeps a field with the 0x6400 exponent, one subtraction leaves code * 2^s
         mma_f16(oacc[mb], swar_pair<VB>(aw[0], aw[1], 2 * mb), swar_pair<VB>(aw[0], aw[1], 2 * mb + 1),
                 swar_pair<VB>(aw[2], aw[3], 2 * mb), swar_pair<VB>(aw[2], aw[3], 2 * mb + 1), b0, b1);
       } else {
