@@ -30,8 +30,11 @@
 // sum_j q_j sigma_j (2^-w_j - 1) is added per head; the MMA's k index is permuted so that each
 // lane reads one contiguous bit range of a key row.  PV multiplies the value codes (exact fp16)
 // by p * step in hi/lo halves and adds sum_t p_t zero_t.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+#include <cstring>
 #include <math.h>
 
 #include <type_traits>
@@ -263,20 +266,48 @@ struct MixedGeo {
 };
 
 // A 16-position slice of a (page, KV head) tile in the page's own layout: 16 key rows of KR bytes,
-// 16 value rows of VR bytes, 16 records of 8 bytes; one bulk copy.
+// 16 value rows of VR bytes, 16 records of 8 bytes.
 __host__ __device__ inline int mixed_slice_bytes(int KR, int VR) { return 16 * (KR + VR) + 128; }
 
-// A ring stage: 16 guard bytes, then the slice.  A key window may start up to 10 bits before its
-// row (see the extraction table), so row 0 reads the word before it: the guard keeps that read
-// inside the stage, off the previous stage, whose copy may still be landing.  Its bits are masked.
-constexpr int kStageGuard = 16;
-__host__ __device__ inline int mixed_stage_bytes(int KR, int VR) { return kStageGuard + mixed_slice_bytes(KR, VR); }
+// The 8 lanes of one lane group read the same word offset of 8 key rows at once.  Rows of KR bytes
+// with KR / 4 a multiple of 16 words fall into two banks' worth of offsets (4-way conflicts at
+// 4-bit keys, for D = 128; with the old row-per-lane coordinate map, 8-way at 8-bit).  In shared
+// memory those rows are given 16 more bytes, which spreads the 8 rows over the banks.  The padded
+// rows arrive by one tensor copy whose box starts 16 bytes before each row (the tensor's fill
+// value, no memory traffic); the others by a bulk copy.  Two-way conflicts (KR / 4 = 8 mod 16)
+// cost less than the row-by-row tensor copy and stay.
+__host__ __device__ inline int mixed_key_pad(int KR) { return (KR / 4) % 16 == 0 ? 16 : 0; }
+
+// A ring stage: [16 bytes][16 key rows of KRP = KR + pad bytes][16 value rows][16 records]; with
+// padded rows, rounded up to 128 bytes (the tensor copy's destination is 128-byte aligned).  A key window may start up to 10 bits before its row (see
+// the extraction table), so row 0 reads the word before it: the first 16 bytes keep that read
+// inside the stage, off the previous one, whose copy may still be landing; with padded rows they
+// are row 0's pad.  The bits read there are masked off.
+constexpr int kStageLead = 16;
+__host__ __device__ inline int mixed_stage_bytes_padded(int KR, int VR, int pad) {
+  const int b = kStageLead + 16 * (KR + pad) + 16 * VR + 128;
+  return pad ? (b + 127) & ~127 : b;
+}
+__host__ __device__ inline int mixed_stage_bytes(int KR, int VR) {
+  return mixed_stage_bytes_padded(KR, VR, mixed_key_pad(KR));
+}
+
+// One 4-D tensor copy global -> shared (box of the tensor map at coordinates x..w); completion is
+// signalled on `bar` as the box's bytes.  Never multicast.
+__device__ __forceinline__ void tensor_g2s_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
+                                              uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
 
 template <int D, int G>
 struct SmemMixedFixed {
   float qbuf[kWarps][G][D];
   // key extraction table per (k step kb, lane group tig).  The four codes c0..c3 (widths w0..w3,
-  // sum W <= 32) of coordinates tig * D/4 + 4 kb + (0..3) follow each other in the bit stream from
+  // sum W <= 32) of coordinates 16 kb + 4 tig + (0..3) follow each other in the bit stream from
   // bit off0.  The 32-bit window x starts t0 = min(10 - w0, 32 - W) bits before off0, so c0 sits
   // at the top of a mantissa field, or at most two bits below it when the four are wide.  Then
   // (x & M0) | (x 2^(26 - w1 - t0 - w0) & M1) is the subnormal pair (c0, c1) with M0 = (2^w0 - 1)
@@ -384,10 +415,15 @@ __device__ __forceinline__ uint32_t field_pair(const uint32_t (&w0)[NW], const u
   return (shift_to(w0[wi], kSubTop - VB - sh) & m) | (shift_to(w1[wi], kSubTop + 16 - VB - sh) & (m << 16));
 }
 
-template <int D, int G, int VB>
-__global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const DecodeArgs a) {
+// Key rows: PAD = false, unpadded, the slice in one bulk copy; PAD = true, padded rows, kmode 1:
+// one tensor copy through kmap (the layer's key rows as the tensor [pages][Hkv P / 16 slices][16
+// rows][KR bytes]), kmode 2: one bulk copy per row (16 lanes).  Mode 1 falls back to 2 if shared
+// memory is not 128-byte aligned, which the tensor copy needs.
+template <int D, int G, int VB, bool PAD>
+__global__ void __launch_bounds__(kWarps * 32, 2)
+    decode_mixed_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap, const int kmode) {
   using MG = MixedGeo<D, VB>;
-  constexpr int NK = MG::NK, NB = D / 2, Q4 = D / 4;
+  constexpr int NK = MG::NK, NB = D / 2;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   SmemMixedFixed<D, G>& sm = *reinterpret_cast<SmemMixedFixed<D, G>*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -395,8 +431,11 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
   const int wid = blockIdx.x * kWarps + warp;
   const int cap = a.stride * a.P;
   const int KR = a.kbits * D / 8;
-  const int SB = mixed_stage_bytes(KR, MG::VR), SL = mixed_slice_bytes(KR, MG::VR);
-  const int VO = 16 * KR, PO = 16 * (KR + MG::VR);
+  const int mode = !PAD ? 0 : (kmode == 1 && (smem_u32(smem_raw) & 127u) != 0u) ? 2 : 1;
+  constexpr int kpad = PAD ? 16 : 0;
+  const int KRP = KR + kpad;  // key row stride in shared memory
+  const int SB = mixed_stage_bytes_padded(KR, MG::VR, kpad), SL = mixed_slice_bytes(KR, MG::VR);
+  const int VO = kStageLead + 16 * KRP, PO = VO + 16 * MG::VR;
   uint8_t* const ring = smem_raw + kMixedFixedBytes<D, G> + static_cast<size_t>(warp) * kStages * SB;
   const size_t tile_bytes = static_cast<size_t>(a.P) * (KR + MG::VR + 8);
   uint64_t* bars = sm.bar[warp];
@@ -414,23 +453,41 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
   splitk::Cur cons = splitk::cursor_at(a, cap, lane, c0);
   splitk::Cur prod = cons;
   const long long nslots = c1 - c0;
-  const uint32_t stage_tx = static_cast<uint32_t>(SL);
+  const uint32_t stage_tx = static_cast<uint32_t>(16 * KRP + 16 * MG::VR + 128);
 
-  // Lane 0 arms the stage's barrier, records whether the page is valid and starts the bulk copy
-  // of the 16-position slice (16 key rows, 16 value rows, 16 records: one contiguous block).
+  // Lane 0 arms the stage's barrier, records whether the page is valid and starts the copies of
+  // the 16-position slice: unpadded, the whole slice in one bulk copy (it lands in the stage's
+  // layout); padded, the key rows by the tensor copy and the value rows with the records by one
+  // bulk copy.  In mode 2 the first 16 lanes copy a key row each.  Called by the whole warp.
   auto issue = [&](const splitk::Cur& c, int st) {
-    if (lane != 0) return;
+    const bool one_lane = mode != 2;  // warp-uniform
+    if (one_lane && lane != 0) return;
     const int lp = (c.i * 16) / a.P;
-    const int page = a.page_table[static_cast<size_t>(c.b) * a.stride + lp];
-    const bool ok = page >= 0 && page < a.max_pages;
-    sm.stage_ok[warp][st] = ok ? 1u : 0u;
-    if (!ok) atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
-    mbar_arrive_expect_tx(&bars[st], ok ? stage_tx : 0u);
-    if (ok) {
-      const int r0 = c.i * 16 - lp * a.P;
-      const uint8_t* src = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(c.g) * tile_bytes +
-                           static_cast<size_t>(r0 >> 4) * SL;
-      bulk_g2s_hint(ring + st * SB + kStageGuard, src, static_cast<uint32_t>(SL), &bars[st], l2_policy_evict_first());
+    int page = 0;
+    if (lane == 0) {
+      page = a.page_table[static_cast<size_t>(c.b) * a.stride + lp];
+      const bool ok = page >= 0 && page < a.max_pages;
+      sm.stage_ok[warp][st] = ok ? 1u : 0u;
+      if (!ok) atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
+      mbar_arrive_expect_tx(&bars[st], ok ? stage_tx : 0u);
+    }
+    if (!one_lane) page = __shfl_sync(FULL, page, 0);
+    if (page < 0 || page >= a.max_pages) return;
+    const int r0 = c.i * 16 - lp * a.P;
+    const uint8_t* src = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(c.g) * tile_bytes +
+                         static_cast<size_t>(r0 >> 4) * SL;
+    uint8_t* dst = ring + st * SB;
+    const uint64_t pol = l2_policy_evict_first();
+    if constexpr (!PAD) {
+      bulk_g2s_hint(dst + kStageLead, src, static_cast<uint32_t>(SL), &bars[st], pol);
+    } else {
+      if (mode == 1) {
+        // box from x = -16: each row lands as [16 bytes of fill][KR bytes]
+        tensor_g2s_4d(dst, &kmap, -16, 0, c.g * (a.P >> 4) + (r0 >> 4), page, &bars[st], pol);
+      } else if (lane < 16) {
+        bulk_g2s_hint(dst + kStageLead + lane * KRP, src + lane * KR, static_cast<uint32_t>(KR), &bars[st], pol);
+      }
+      if (lane == 0) bulk_g2s_hint(dst + VO, src + 16 * KR, static_cast<uint32_t>(16 * MG::VR + 128), &bars[st], pol);
     }
   };
 
@@ -475,8 +532,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
       // the code's field sits at bit 10 - w of its half, except c0 of a wide group, which sits at t0
       float lift = 1.f;
       {
-        const int r = j % Q4, kb = r >> 2, e = r & 3;
-        uint32_t* ent = ktab + (kb * 4 + j / Q4) * 8;
+        const int e = j & 3;
+        uint32_t* ent = ktab + (j >> 2) * 8;  // entry (kb, tig = (j / 4) % 4)
         const int t0 = min(kSubTop - w0, 32 - (w0 + w1 + w2 + w3));
         const uint32_t m = (1u << w) - 1u;
         if (e == 0) {
@@ -527,7 +584,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
     const bool lo = gq & 1;
 #pragma unroll
     for (int kb = 0; kb < NK; ++kb) {
-      const int j0 = tig * Q4 + 4 * kb;
+      const int j0 = 16 * kb + 4 * tig;
       if (hh < G) {
         const float* qh = qb + hh * D;
         qf[kb][0] = split_h2(qh[j0] * scale, qh[j0 + 1] * scale, lo);
@@ -595,24 +652,25 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
       failed = true;
       break;
     }
-    const uint8_t* buf = ring + st * SB + kStageGuard;
+    const uint8_t* buf = ring + st * SB;
     const bool page_ok = sm.stage_ok[warp][st] != 0u;
     const int L = Lseg;
     const int i0 = cons.i * 16;
     const bool v0 = page_ok && tig < G && i0 + gq < L, v1 = page_ok && tig < G && i0 + gq + 8 < L;
 
-    // QK^T.  Lane (gq, tig) reads, in rows gq and gq + 8, the coordinates tig * D/4 + [0, D/4):
-    // k index (2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9) of step kb is coordinate tig * D/4 + 4 kb
-    // + (0, 1, 2, 3), and the query fragments use the same map.
-    const uint32_t* r0w = reinterpret_cast<const uint32_t*>(buf + gq * KR);
-    const uint32_t* r1w = reinterpret_cast<const uint32_t*>(buf + (gq + 8) * KR);
+    // QK^T.  k index (2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9) of step kb is coordinate 16 kb +
+    // 4 tig + (0, 1, 2, 3), and the query fragments use the same map: the four lanes of a row read
+    // neighbouring windows of one 16-coordinate stretch, so with row strides of 4 words mod 8 the
+    // 32 lanes fall into distinct banks (or share a word).
+    const uint32_t* r0w = reinterpret_cast<const uint32_t*>(buf + kStageLead + gq * KRP);
+    const uint32_t* r1w = reinterpret_cast<const uint32_t*>(buf + kStageLead + (gq + 8) * KRP);
     float S[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kb = 0; kb < NK; ++kb) {
       const uint32_t* ent = ktab + (kb * 4 + tig) * 8;
       const uint4 E0 = *reinterpret_cast<const uint4*>(ent);      // M0, M1, multiplier of c1, window start
       const uint4 E1 = *reinterpret_cast<const uint4*>(ent + 4);  // shift of z, M2, M3, multiplier of c3
-      const int wi = static_cast<int>(E0.w) >> 5, sh = static_cast<int>(E0.w & 31u);  // wi = -1 reads the guard
+      const int wi = static_cast<int>(E0.w) >> 5, sh = static_cast<int>(E0.w & 31u);  // wi = -1: the stage's lead bytes
       const uint32_t x0 = __funnelshift_r(r0w[wi], r0w[wi + 1], sh);
       const uint32_t x1 = __funnelshift_r(r1w[wi], r1w[wi + 1], sh);
       const uint32_t z0 = x0 >> E1.x, z1 = x1 >> E1.x;
@@ -717,15 +775,55 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_mixed_kernel(const Deco
   }
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link against the driver
+// library); null when it cannot be had
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// The layer's key rows as the 4-D byte tensor [max_pages][Hkv P / 16][16][KR] (strides KR, the slice
+// bytes, the page bytes) with a box of one slice's 16 rows, KR + 16 bytes wide.  False when the
+// encoder is missing or refuses; the decode then copies unpadded rows.
+bool encode_key_map(CUtensorMap* m, const DecodeArgs& a, int KR, int VR) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(KR), 16u, static_cast<cuuint64_t>(a.Hkv) * (a.P / 16),
+                              static_cast<cuuint64_t>(a.max_pages)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(KR), static_cast<cuuint64_t>(mixed_slice_bytes(KR, VR)),
+                                 static_cast<cuuint64_t>(a.page_bytes)};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(KR + 16), 16u, 1u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<uint8_t*>(a.pool), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, int G, int VB>
 cudaError_t launch_dgv(const DecodeArgs& a, int ctas, cudaStream_t st) {
-  const int smem = static_cast<int>(mixed_smem_bytes<D, G>(a.kbits * D / 8, VB * D / 8));
-  // the attribute is raised once, to the size of the widest key rows (8 bits per dimension)
-  static std::atomic<uint64_t> done;
-  cudaError_t e = ensure_smem_limit(decode_mixed_kernel<D, G, VB>, static_cast<int>(mixed_smem_bytes<D, G>(D, VB * D / 8)),
-                                    done);
+  const int KR = a.kbits * D / 8;
+  CUtensorMap kmap;
+  memset(&kmap, 0, sizeof(kmap));
+  const bool pad = mixed_key_pad(KR) != 0;
+  const int kmode = pad ? (encode_key_map(&kmap, a, KR, VB * D / 8) ? 1 : 2) : 0;
+  const int smem = static_cast<int>(mixed_smem_bytes<D, G>(KR, VB * D / 8));
+  // the attribute is raised once per kernel, to the size of the widest key rows (8 bits per dimension)
+  const int smem_max = static_cast<int>(mixed_smem_bytes<D, G>(D, VB * D / 8));
+  static std::atomic<uint64_t> done_pad, done_flat;
+  cudaError_t e = pad ? ensure_smem_limit(decode_mixed_kernel<D, G, VB, true>, smem_max, done_pad)
+                      : ensure_smem_limit(decode_mixed_kernel<D, G, VB, false>, smem_max, done_flat);
   if (e != cudaSuccess) return e;
-  decode_mixed_kernel<D, G, VB><<<ctas, kWarps * 32, smem, st>>>(a);
+  if (pad)
+    decode_mixed_kernel<D, G, VB, true><<<ctas, kWarps * 32, smem, st>>>(a, kmap, kmode);
+  else
+    decode_mixed_kernel<D, G, VB, false><<<ctas, kWarps * 32, smem, st>>>(a, kmap, kmode);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   splitk::merge_kernel<D, G><<<(a.B * a.Hq + 7) / 8, 256, 0, st>>>(a);
