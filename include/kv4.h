@@ -251,6 +251,16 @@ kv4_status kv4_set_decode_overlap(kv4_cache* cache, int enable);
 kv4_status kv4_debug_force_wait_timeout(kv4_cache* cache, int enable);
 
 /*
+ * kv4_debug_mixed_row_copies: a test hook for the mixed bit-width key cache (default 0).  Key rows
+ * whose word count is a multiple of 16 (4- and 8-bit keys at D = 128, 8-bit at D = 64) are
+ * padded in shared memory and normally arrive by one tensor copy per 16-position slice; that
+ * copy needs a tensor map from the driver's encoder.  With 1, kv4_decode_attn takes the path used
+ * when the encoder is missing or refuses: one bulk copy per key row.  Results are the same either
+ * way.  Returns KV4_ERR_INVALID_ARG for a NULL cache or one of another format.
+ */
+kv4_status kv4_debug_mixed_row_copies(kv4_cache* cache, int enable);
+
+/*
  * Mixed bit-width keys (KV4_KEYS_MIXED): the block allocation of one layer.  "RoPE-Aware Bit
  * Allocation for KV-Cache Quantization" (searcharxiv abstract): under RoPE a key's share of a
  * later logit is a sum over its two-dimensional frequency blocks, so for every layer and KV head a

@@ -43,6 +43,7 @@ struct kv4_cache {
   uint32_t signs[4];  // kv4_set_rotation_signs
   int rotate_v;       // kv4_set_value_rotation
   int stall_test;     // kv4_debug_force_wait_timeout
+  int mixed_rows;     // kv4_debug_mixed_row_copies
   // mixed bit-width keys: per-layer block-allocation records after the pages, and which layers
   // have one
   uint8_t* alloc_base;
@@ -285,7 +286,7 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
   const int G = c->cfg.num_q_heads / c->cfg.num_kv_heads;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const cudaError_t e = fmt == FMT_INT4    ? kv4::launch_decode_int4(a, c->cfg.head_dim, G, ctas, st)
-                        : fmt == FMT_MIXED ? kv4::launch_decode_mixed(a, c->cfg.head_dim, G, ctas, st)
+                        : fmt == FMT_MIXED ? kv4::launch_decode_mixed(a, c->cfg.head_dim, G, ctas, st, c->mixed_rows != 0)
                                            : kv4::launch_decode_bf16(a, c->cfg.head_dim, G, ctas, st);
   return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
@@ -403,6 +404,12 @@ kv4_status kv4_set_decode_overlap(kv4_cache* cache, int enable) {
 kv4_status kv4_debug_force_wait_timeout(kv4_cache* cache, int enable) {
   if (!cache || cache->format != FMT_INT4) return KV4_ERR_INVALID_ARG;
   cache->stall_test = enable ? 1 : 0;
+  return KV4_OK;
+}
+
+kv4_status kv4_debug_mixed_row_copies(kv4_cache* cache, int enable) {
+  if (!cache || cache->format != FMT_MIXED) return KV4_ERR_INVALID_ARG;
+  cache->mixed_rows = enable ? 1 : 0;
   return KV4_OK;
 }
 

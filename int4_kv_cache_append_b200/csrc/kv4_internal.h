@@ -92,7 +92,8 @@ cudaError_t launch_mixed_score(const ScoreArgs& a, int D, cudaStream_t st);
 cudaError_t launch_append_mixed(const AppendArgs& a, int D, cudaStream_t st);
 int mixed_decode_warps_per_cta();
 int mixed_decode_ctas_per_sm(int D, int G, int value_bits, int key_bits);
-cudaError_t launch_decode_mixed(DecodeArgs a, int D, int G, int ctas, cudaStream_t st);
+// row_copies: padded key rows by one bulk copy per row instead of the tensor copy (a test hook)
+cudaError_t launch_decode_mixed(DecodeArgs a, int D, int G, int ctas, cudaStream_t st, bool row_copies);
 
 // Counts every kernel launch the library issues.
 void note_launches(int n);

@@ -431,7 +431,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   const int wid = blockIdx.x * kWarps + warp;
   const int cap = a.stride * a.P;
   const int KR = a.kbits * D / 8;
-  const int mode = !PAD ? 0 : (kmode == 1 && (smem_u32(smem_raw) & 127u) != 0u) ? 2 : 1;
+  const int mode = !PAD ? 0 : (kmode == 1 && (smem_u32(smem_raw) & 127u) == 0u) ? 1 : 2;
   constexpr int kpad = PAD ? 16 : 0;
   const int KRP = KR + kpad;  // key row stride in shared memory
   const int SB = mixed_stage_bytes_padded(KR, MG::VR, kpad), SL = mixed_slice_bytes(KR, MG::VR);
@@ -453,7 +453,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   splitk::Cur cons = splitk::cursor_at(a, cap, lane, c0);
   splitk::Cur prod = cons;
   const long long nslots = c1 - c0;
-  const uint32_t stage_tx = static_cast<uint32_t>(16 * KRP + 16 * MG::VR + 128);
+  // the tensor copy delivers the padded rows (fill included), the other copies the rows' bytes
+  const uint32_t stage_tx = static_cast<uint32_t>(16 * (mode == 1 ? KRP : KR) + 16 * MG::VR + 128);
 
   // Lane 0 arms the stage's barrier, records whether the page is valid and starts the copies of
   // the 16-position slice: unpadded, the whole slice in one bulk copy (it lands in the stage's
@@ -807,12 +808,12 @@ bool encode_key_map(CUtensorMap* m, const DecodeArgs& a, int KR, int VR) {
 }
 
 template <int D, int G, int VB>
-cudaError_t launch_dgv(const DecodeArgs& a, int ctas, cudaStream_t st) {
+cudaError_t launch_dgv(const DecodeArgs& a, int ctas, cudaStream_t st, bool row_copies) {
   const int KR = a.kbits * D / 8;
   CUtensorMap kmap;
   memset(&kmap, 0, sizeof(kmap));
   const bool pad = mixed_key_pad(KR) != 0;
-  const int kmode = pad ? (encode_key_map(&kmap, a, KR, VB * D / 8) ? 1 : 2) : 0;
+  const int kmode = pad ? (!row_copies && encode_key_map(&kmap, a, KR, VB * D / 8) ? 1 : 2) : 0;
   const int smem = static_cast<int>(mixed_smem_bytes<D, G>(KR, VB * D / 8));
   // the attribute is raised once per kernel, to the size of the widest key rows (8 bits per dimension)
   const int smem_max = static_cast<int>(mixed_smem_bytes<D, G>(D, VB * D / 8));
@@ -831,12 +832,12 @@ cudaError_t launch_dgv(const DecodeArgs& a, int ctas, cudaStream_t st) {
 }
 
 template <int D, int G>
-cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
+cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st, bool rows) {
   switch (a.vbits) {
-    case 2: return launch_dgv<D, G, 2>(a, ctas, st);
-    case 3: return launch_dgv<D, G, 3>(a, ctas, st);
-    case 4: return launch_dgv<D, G, 4>(a, ctas, st);
-    case 8: return launch_dgv<D, G, 8>(a, ctas, st);
+    case 2: return launch_dgv<D, G, 2>(a, ctas, st, rows);
+    case 3: return launch_dgv<D, G, 3>(a, ctas, st, rows);
+    case 4: return launch_dgv<D, G, 4>(a, ctas, st, rows);
+    case 8: return launch_dgv<D, G, 8>(a, ctas, st, rows);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -875,17 +876,17 @@ int mixed_decode_ctas_per_sm(int D, int G, int VB, int KB) {
   return 2 * (bytes + 1024) <= 227u * 1024u ? 2 : 1;
 }
 
-cudaError_t launch_decode_mixed(DecodeArgs a, int D, int G, int ctas, cudaStream_t st) {
+cudaError_t launch_decode_mixed(DecodeArgs a, int D, int G, int ctas, cudaStream_t st, bool row_copies) {
   a.W = ctas * kWarps;
   note_launches(2);
   if (D == 128) {
-    if (G == 4) return launch_dg<128, 4>(a, ctas, st);
-    if (G == 2) return launch_dg<128, 2>(a, ctas, st);
-    return launch_dg<128, 1>(a, ctas, st);
+    if (G == 4) return launch_dg<128, 4>(a, ctas, st, row_copies);
+    if (G == 2) return launch_dg<128, 2>(a, ctas, st, row_copies);
+    return launch_dg<128, 1>(a, ctas, st, row_copies);
   }
-  if (G == 4) return launch_dg<64, 4>(a, ctas, st);
-  if (G == 2) return launch_dg<64, 2>(a, ctas, st);
-  return launch_dg<64, 1>(a, ctas, st);
+  if (G == 4) return launch_dg<64, 4>(a, ctas, st, row_copies);
+  if (G == 2) return launch_dg<64, 2>(a, ctas, st, row_copies);
+  return launch_dg<64, 1>(a, ctas, st, row_copies);
 }
 
 }  // namespace kv4

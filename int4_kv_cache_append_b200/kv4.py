@@ -31,7 +31,7 @@ SYMBOLS = (
     "kv4_set_rotation_signs", "kv4_set_value_rotation", "kv4_bf16_query_sizes", "kv4_bf16_cache_init",
     "kv4_bf16_append", "kv4_bf16_decode_workspace_bytes", "kv4_bf16_decode_attn", "kv4_get_device_error",
     "kv4_launch_count", "kv4_status_string", "kv4_version", "kv4_allocate_key_bits", "kv4_set_key_allocation",
-    "kv4_get_key_allocation",
+    "kv4_get_key_allocation", "kv4_debug_mixed_row_copies",
 )
 
 
@@ -67,6 +67,7 @@ def _load():
         "kv4_decode_attn_static": (I, [P, I, I, P, I, i32p, I, i32p, I, P, P, P]),
         "kv4_set_decode_overlap": (I, [P, I]),
         "kv4_debug_force_wait_timeout": (I, [P, I]),
+        "kv4_debug_mixed_row_copies": (I, [P, I]),
         "kv4_set_rotation_signs": (I, [P, P]),
         "kv4_set_value_rotation": (I, [P, I]),
         "kv4_bf16_query_sizes": (I, [cfgp, ctypes.POINTER(S)]),
@@ -194,6 +195,12 @@ def kv4_set_decode_overlap(handle, enable: bool):
     """With enable, the decode kernel builds its schedule from lens and page_table while the
     preceding kernel on the stream runs (they must not be written by that kernel)."""
     _check("kv4_set_decode_overlap", lib.kv4_set_decode_overlap(handle, 1 if enable else 0))
+
+
+def kv4_debug_mixed_row_copies(handle, enable: bool):
+    """Test hook (mixed bit-width keys): padded key rows by one bulk copy per row instead of the
+    tensor copy, the path taken when the driver's tensor-map encoder is not available."""
+    _check("kv4_debug_mixed_row_copies", lib.kv4_debug_mixed_row_copies(handle, 1 if enable else 0))
 
 
 def kv4_debug_force_wait_timeout(handle, enable: bool):

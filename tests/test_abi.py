@@ -156,9 +156,13 @@ def test_mixed_host_validation_without_gpu(lib):
             assert e.value.status == 1
         # setters of the INT4 cache do not apply
         assert lib.kv4_set_value_rotation(v(h), 1) == 1
+        # the row-copy test hook applies to this format only
+        assert lib.kv4_debug_mixed_row_copies(v(h), 1) == 0 and lib.kv4_debug_mixed_row_copies(v(h), 0) == 0
+        assert lib.kv4_debug_mixed_row_copies(None, 1) == 1
         # the INT4 entry points refuse an allocation call
         h4 = kv4.kv4_cache_init(_cfg(), 1 << 20, 1 << 21)
         assert lib.kv4_allocate_key_bits(v(h4), 0, 0, None, 1, None) == 1
+        assert lib.kv4_debug_mixed_row_copies(v(h4), 1) == 1
         kv4.kv4_cache_destroy(h4)
     finally:
         kv4.kv4_cache_destroy(h)

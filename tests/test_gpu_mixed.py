@@ -37,6 +37,9 @@ CASES = [
     # smallest rows (8-byte keys, 16-byte values) and an odd width on every block
     (mixed_workload("m-k1v2-d64", 108, 2, 4, 2, 64, 16, [33, 500]), 1, 2),
     (mixed_workload("m-k7v8-p32", 109, 2, 2, 4, 128, 32, [70, 301], dt=W.F32), 7, 8),
+    # key rows of 16 and 32 words at D = 128: padded in shared memory, brought in by the tensor copy
+    (mixed_workload("m-k4v4-d128", 110, 3, 4, 4, 128, 16, [260, 33, 129]), 4, 4),
+    (mixed_workload("m-k8v8-p48", 111, 2, 2, 2, 128, 48, [200, 97], dt=W.F32), 8, 8),
 ]
 IDS = [c[0].name for c in CASES]
 
@@ -218,6 +221,25 @@ def test_decode_split_count_invariance():
     assert np.abs(o1 - o2).max() <= 1e-5 and np.abs(l1 - l2).max() <= 1e-5
 
 
+@pytest.mark.parametrize("name", ["m-k4v4-d128", "m-k8v8-p48", "m-k8v3"])
+def test_row_copies_match_tensor_copy(name):
+    """Padded key rows arrive by one tensor copy, or by one bulk copy per row when the tensor map
+    cannot be had (forced here through the test hook); the decode must be bit-identical."""
+    from int4_kv_cache_append_b200 import kv4
+    wl, kb, vb = next(c for c in CASES if c[0].name == name)
+    cache = gpu_cache(wl, kb, vb)
+    q = wl.q_input(0)
+    o1, l1 = T.gpu_decode(cache, wl, q)
+    kv4.kv4_debug_mixed_row_copies(cache.handle, True)
+    try:
+        o2, l2 = T.gpu_decode(cache, wl, q)
+    finally:
+        kv4.kv4_debug_mixed_row_copies(cache.handle, False)
+    assert kv4.kv4_get_device_error() == 0
+    assert np.array_equal(o1.view(np.uint32), o2.view(np.uint32)) and np.array_equal(l1.view(np.uint32),
+                                                                                     l2.view(np.uint32))
+
+
 def test_range_overflow_sets_error_bit():
     """A key beyond the fp16 range is stored with zero codes and reported, as in the oracle."""
     from int4_kv_cache_append_b200 import kv4
@@ -268,13 +290,12 @@ def _oracle_one_mixed(wl, kb, vb, widths, sigma, b, g):
     return cfg, pool, out[0], lse[0]
 
 
-@pytest.mark.parametrize("name", ["async-refill", "long-context"])
-def test_fullsize_mixed_sampled_parity(name):
-    """The bench's K3V3 workloads at full size, in its launch configuration: the allocation from
+@pytest.mark.parametrize("name,kb,vb", [("async-refill", 3, 3), ("async-refill", 4, 4), ("long-context", 3, 3)])
+def test_fullsize_mixed_sampled_parity(name, kb, vb):
+    """The bench's mixed workloads at full size, in its launch configuration: the allocation from
     4096 host-drawn keys equals the oracle's; sampled (sequence, KV head) pairs are recomputed by
     the oracle one by one (page bytes bit-exact, outputs within the tolerance)."""
     from int4_kv_cache_append_b200 import harness as H, kv4
-    kb, vb = 3, 3
     wl = dataclasses.replace(W.WORKLOADS[name](), s=0, w=0, h=1, value_format=2, key_bits=kb, value_bits=vb,
                              rope_outliers=True)
     cache = kv4.Cache(H.geometry(wl, value_format=kv4.KV4_KEYS_MIXED), fill=0xA5)
