@@ -415,13 +415,14 @@ __device__ __forceinline__ uint32_t field_pair(const uint32_t (&w0)[NW], const u
   return (shift_to(w0[wi], kSubTop - VB - sh) & m) | (shift_to(w1[wi], kSubTop + 16 - VB - sh) & (m << 16));
 }
 
-// Key rows: PAD = false, unpadded, the slice in one bulk copy; PAD = true, padded rows, kmode 1:
-// one tensor copy through kmap (the layer's key rows as the tensor [pages][Hkv P / 16 slices][16
-// rows][KR bytes]), kmode 2: one bulk copy per row (16 lanes).  Mode 1 falls back to 2 if shared
-// memory is not 128-byte aligned, which the tensor copy needs.
-template <int D, int G, int VB, bool PAD>
+// Key rows (KMODE): 0, unpadded, the slice in one bulk copy; 1, padded rows by one tensor copy
+// through kmap (the layer's key rows as the tensor [pages][Hkv P / 16 slices][16 rows][KR bytes]);
+// 2, padded rows by one bulk copy per row (16 lanes), for when the tensor map cannot be had.  The
+// tensor copy's destination is 128-byte aligned: the dynamic shared memory is declared so, and the
+// kernel has no static shared memory.
+template <int D, int G, int VB, int KMODE>
 __global__ void __launch_bounds__(kWarps * 32, 2)
-    decode_mixed_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap, const int kmode) {
+    decode_mixed_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap) {
   using MG = MixedGeo<D, VB>;
   constexpr int NK = MG::NK, NB = D / 2;
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -431,7 +432,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   const int wid = blockIdx.x * kWarps + warp;
   const int cap = a.stride * a.P;
   const int KR = a.kbits * D / 8;
-  const int mode = !PAD ? 0 : (kmode == 1 && (smem_u32(smem_raw) & 127u) == 0u) ? 1 : 2;
+  constexpr bool PAD = KMODE != 0;
   constexpr int kpad = PAD ? 16 : 0;
   const int KRP = KR + kpad;  // key row stride in shared memory
   const int SB = mixed_stage_bytes_padded(KR, MG::VR, kpad), SL = mixed_slice_bytes(KR, MG::VR);
@@ -454,14 +455,14 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   splitk::Cur prod = cons;
   const long long nslots = c1 - c0;
   // the tensor copy delivers the padded rows (fill included), the other copies the rows' bytes
-  const uint32_t stage_tx = static_cast<uint32_t>(16 * (mode == 1 ? KRP : KR) + 16 * MG::VR + 128);
+  const uint32_t stage_tx = static_cast<uint32_t>(16 * (KMODE == 1 ? KRP : KR) + 16 * MG::VR + 128);
 
   // Lane 0 arms the stage's barrier, records whether the page is valid and starts the copies of
   // the 16-position slice: unpadded, the whole slice in one bulk copy (it lands in the stage's
   // layout); padded, the key rows by the tensor copy and the value rows with the records by one
   // bulk copy.  In mode 2 the first 16 lanes copy a key row each.  Called by the whole warp.
   auto issue = [&](const splitk::Cur& c, int st) {
-    const bool one_lane = mode != 2;  // warp-uniform
+    constexpr bool one_lane = KMODE != 2;
     if (one_lane && lane != 0) return;
     const int lp = (c.i * 16) / a.P;
     int page = 0;
@@ -472,7 +473,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
       if (!ok) atomicOr(a.err, KV4_DEVERR_PAGE_RANGE);
       mbar_arrive_expect_tx(&bars[st], ok ? stage_tx : 0u);
     }
-    if (!one_lane) page = __shfl_sync(FULL, page, 0);
+    if constexpr (!one_lane) page = __shfl_sync(FULL, page, 0);
     if (page < 0 || page >= a.max_pages) return;
     const int r0 = c.i * 16 - lp * a.P;
     const uint8_t* src = a.pool + static_cast<size_t>(page) * a.page_bytes + static_cast<size_t>(c.g) * tile_bytes +
@@ -482,7 +483,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     if constexpr (!PAD) {
       bulk_g2s_hint(dst + kStageLead, src, static_cast<uint32_t>(SL), &bars[st], pol);
     } else {
-      if (mode == 1) {
+      if constexpr (KMODE == 1) {
         // box from x = -16: each row lands as [16 bytes of fill][KR bytes]
         tensor_g2s_4d(dst, &kmap, -16, 0, c.g * (a.P >> 4) + (r0 >> 4), page, &bars[st], pol);
       } else if (lane < 16) {
@@ -817,14 +818,17 @@ cudaError_t launch_dgv(const DecodeArgs& a, int ctas, cudaStream_t st, bool row_
   const int smem = static_cast<int>(mixed_smem_bytes<D, G>(KR, VB * D / 8));
   // the attribute is raised once per kernel, to the size of the widest key rows (8 bits per dimension)
   const int smem_max = static_cast<int>(mixed_smem_bytes<D, G>(D, VB * D / 8));
-  static std::atomic<uint64_t> done_pad, done_flat;
-  cudaError_t e = pad ? ensure_smem_limit(decode_mixed_kernel<D, G, VB, true>, smem_max, done_pad)
-                      : ensure_smem_limit(decode_mixed_kernel<D, G, VB, false>, smem_max, done_flat);
+  static std::atomic<uint64_t> done0, done1, done2;
+  cudaError_t e = kmode == 1   ? ensure_smem_limit(decode_mixed_kernel<D, G, VB, 1>, smem_max, done1)
+                  : kmode == 2 ? ensure_smem_limit(decode_mixed_kernel<D, G, VB, 2>, smem_max, done2)
+                               : ensure_smem_limit(decode_mixed_kernel<D, G, VB, 0>, smem_max, done0);
   if (e != cudaSuccess) return e;
-  if (pad)
-    decode_mixed_kernel<D, G, VB, true><<<ctas, kWarps * 32, smem, st>>>(a, kmap, kmode);
+  if (kmode == 1)
+    decode_mixed_kernel<D, G, VB, 1><<<ctas, kWarps * 32, smem, st>>>(a, kmap);
+  else if (kmode == 2)
+    decode_mixed_kernel<D, G, VB, 2><<<ctas, kWarps * 32, smem, st>>>(a, kmap);
   else
-    decode_mixed_kernel<D, G, VB, false><<<ctas, kWarps * 32, smem, st>>>(a, kmap, kmode);
+    decode_mixed_kernel<D, G, VB, 0><<<ctas, kWarps * 32, smem, st>>>(a, kmap);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   splitk::merge_kernel<D, G><<<(a.B * a.Hq + 7) / 8, 256, 0, st>>>(a);
