@@ -245,7 +245,10 @@ kv4_status kv4_set_decode_overlap(kv4_cache* cache, int enable);
  * out, the warp sets KV4_DEVERR_WAIT_LIMIT, waits (bounded) for the bulk copies it already has
  * in flight, and returns.  The merge kernel then finds no fresh partial records: records that
  * point outside the workspace are skipped with KV4_DEVERR_RECORD.  That call's out and lse are
- * undefined; the context stays usable, and a call with 0 decodes normally.  Returns
+ * undefined; the context stays usable, and a call with 0 decodes normally.  The mixed
+ * bit-width key cache takes the same path: each decode warp's first wait is on a barrier nothing
+ * arrives on, runs out after 1 ms, sets KV4_DEVERR_WAIT_LIMIT, and the warp waits (bounded) for
+ * its copies in flight and returns; that call's out and lse are undefined.  Returns
  * KV4_ERR_INVALID_ARG for a NULL or BF16 cache.
  */
 kv4_status kv4_debug_force_wait_timeout(kv4_cache* cache, int enable);

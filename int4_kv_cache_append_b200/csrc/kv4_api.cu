@@ -276,7 +276,7 @@ kv4_status decode_common(kv4_cache* c, int fmt, int layer, int B, const void* q,
   const int tpp = c->cfg.page_size / 16;
   a.tp_shift = pow2(tpp) ? __builtin_ctz(static_cast<unsigned>(tpp)) : -1;
   // The wait-limit test runs every warp's first wait out after 1 ms; the normal limit is 2 s.
-  a.stall_test = (fmt == FMT_INT4 && c->stall_test) ? 1 : 0;
+  a.stall_test = ((fmt == FMT_INT4 || fmt == FMT_MIXED) && c->stall_test) ? 1 : 0;
   a.wait_ns = a.stall_test ? 1000000ull : 2000000000ull;
   if (fmt == FMT_MIXED) {
     a.alloc = c->alloc_base + static_cast<size_t>(layer) * c->alloc_layer_bytes;
@@ -402,7 +402,7 @@ kv4_status kv4_set_decode_overlap(kv4_cache* cache, int enable) {
 }
 
 kv4_status kv4_debug_force_wait_timeout(kv4_cache* cache, int enable) {
-  if (!cache || cache->format != FMT_INT4) return KV4_ERR_INVALID_ARG;
+  if (!cache || (cache->format != FMT_INT4 && cache->format != FMT_MIXED)) return KV4_ERR_INVALID_ARG;
   cache->stall_test = enable ? 1 : 0;
   return KV4_OK;
 }

@@ -318,6 +318,7 @@ struct SmemMixedFixed {
   uint32_t ktab[kWarps][D / 16][4][8];
   uint32_t stage_ok[kWarps][kStages];  // 1 when the stage's page id was inside the pool
   uint64_t bar[kWarps][kStages];
+  uint64_t stall[kWarps];  // never arrived on (the wait-limit test hook)
 };
 
 // the per-warp rings follow the fixed part, sized at launch from the row widths
@@ -442,6 +443,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   uint64_t* bars = sm.bar[warp];
   if (lane == 0) {
     for (int i = 0; i < kStages; ++i) mbar_init(&bars[i], 1);
+    mbar_init(&sm.stall[warp], 1);
     fence_mbar_init();
   }
   __syncwarp();
@@ -638,9 +640,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   reset();
   load_query(cons.b, cons.g);
   int Lseg = splitk::clamp_len(a.lens[cons.b], cap);  // length of the consumer's sequence
-  bool failed = false;
+  // the wait-limit test hook: a first wait on a barrier nothing arrives on, which runs out
+  bool failed = a.stall_test && !mbar_wait_bounded(&sm.stall[warp], 0u, a.err, a.wait_ns);
   long long k = 0;
-  for (; k < nslots; ++k) {
+  for (; !failed && k < nslots; ++k) {
     if (issued < nslots) {
       fence_proxy_async_smem();
       issue(prod, static_cast<int>((k + kStages - 1) % kStages));
@@ -649,7 +652,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
       ++issued;
     }
     const int st = static_cast<int>(k % kStages);
-    const bool ok = mbar_wait_bounded(&bars[st], static_cast<uint32_t>((k / kStages) & 1), a.err);
+    const bool ok = mbar_wait_bounded(&bars[st], static_cast<uint32_t>((k / kStages) & 1), a.err, a.wait_ns);
     if (__any_sync(FULL, !ok)) {
       failed = true;
       break;
@@ -773,7 +776,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   }
   if (failed) {
     for (long long j = k; j < issued; ++j)
-      mbar_wait_bounded(&bars[j % kStages], static_cast<uint32_t>((j / kStages) & 1), a.err);
+      mbar_wait_bounded(&bars[j % kStages], static_cast<uint32_t>((j / kStages) & 1), a.err, a.wait_ns);
   }
 }
 

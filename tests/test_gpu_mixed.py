@@ -240,6 +240,33 @@ def test_row_copies_match_tensor_copy(name):
                                                                                      l2.view(np.uint32))
 
 
+def test_wait_limit_failure_path_reports_and_recovers():
+    """The device-side failure path of the decode's bounded waits, made to run with the test hook
+    (no invalid copy involved): every warp's first wait is on a barrier that nothing arrives on,
+    runs out after its 1 ms limit, sets KV4_DEVERR_WAIT_LIMIT, waits for its copies in flight and
+    returns.  The context stays usable: with the hook off the next decode matches the oracle."""
+    from int4_kv_cache_append_b200 import kv4
+    wl, kb, vb = CASES[0]
+    cache = gpu_cache(wl, kb, vb)
+    assert kv4.kv4_get_device_error() == 0
+    q = wl.q_input(0)
+    kv4.kv4_debug_force_wait_timeout(cache.handle, True)
+    try:
+        T.gpu_decode(cache, wl, q)
+    finally:
+        kv4.kv4_debug_force_wait_timeout(cache.handle, False)
+    err = kv4.kv4_get_device_error()
+    assert err & kv4.KV4_DEVERR_WAIT_LIMIT, hex(err)
+    _, _, K, _ = prefill(wl)
+    widths, sigma = oracle_allocation(wl, kb, K)
+    cfg, pool = oracle_pool(wl, kb, vb, widths, sigma)
+    out, lse = T.gpu_decode(cache, wl, q)
+    qd = O.BF16 if q.dtype == np.uint16 else O.F32
+    ro, rl = O.gtq_decode(cfg, widths, sigma, pool, q, wl.page_table, np.asarray(wl.lens, np.int32), q_dtype=qd)
+    T.assert_close(out, ro, lse, rl, what="decode after the wait-limit path")
+    assert kv4.kv4_get_device_error() == 0
+
+
 def test_range_overflow_sets_error_bit():
     """A key beyond the fp16 range is stored with zero codes and reported, as in the oracle."""
     from int4_kv_cache_append_b200 import kv4
