@@ -405,15 +405,29 @@ __device__ __forceinline__ uint32_t swar_pair(const uint32_t (&w0)[NW], const ui
   return (pos > sh ? x << (pos - sh) : x) & (m | (m << 16));
 }
 
-// (code of dim d of token t0, same of t1) as a subnormal pair, any value width: a field inside one
-// word takes one shift per token and a mask-or to join them; a field across two words goes
-// through take_bits.
+// The 16-bit chunk an odd-width value field is cut from: the lowest byte b whose bits
+// [8 b, 8 b + 16) hold the field, with bytes b and b + 1 in one word (b % 4 <= 2); -1 when there is
+// none (a field across two words).
+template <int VB>
+__host__ __device__ constexpr int field_chunk(int d) {
+  for (int b = 0; 8 * b <= d * VB; ++b)
+    if (b % 4 <= 2 && d * VB + VB <= 8 * b + 16) return b;
+  return -1;
+}
+
+// (code of dim d of token t0, same of t1) as a subnormal pair, any value width.  One byte permute
+// puts the field's 16-bit chunk of both tokens into the two halves (shared by every field of that
+// chunk), one shift takes both fields to the top of their mantissa fields, one mask keeps them:
+// bits that cross between the halves land outside the mask (a field ends at most at bit 16 of its
+// chunk).  A field across two words goes through take_bits.
 template <int VB, int NW>
 __device__ __forceinline__ uint32_t field_pair(const uint32_t (&w0)[NW], const uint32_t (&w1)[NW], int d) {
-  const int p = d * VB, wi = p >> 5, sh = p & 31;
-  if (sh + VB > 32) return codes_h2<VB>(take_bits(w0, p, VB), take_bits(w1, p, VB));
+  const int b = field_chunk<VB>(d);
+  if (b < 0) return codes_h2<VB>(take_bits(w0, d * VB, VB), take_bits(w1, d * VB, VB));
+  const uint32_t s = static_cast<uint32_t>(b & 3);
+  const uint32_t x = prmt(w0[b >> 2], w1[b >> 2], s | ((s + 1u) << 4) | ((s + 4u) << 8) | ((s + 5u) << 12));
   const uint32_t m = ((1u << VB) - 1u) << (kSubTop - VB);
-  return (shift_to(w0[wi], kSubTop - VB - sh) & m) | (shift_to(w1[wi], kSubTop + 16 - VB - sh) & (m << 16));
+  return shift_to(x, kSubTop - VB - (d * VB - 8 * b)) & (m | (m << 16));
 }
 
 // Key rows (KMODE): 0, unpadded, the slice in one bulk copy; 1, padded rows by one tensor copy
