@@ -480,7 +480,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   auto issue = [&](const splitk::Cur& c, int st) {
     constexpr bool one_lane = KMODE != 2;
     if (one_lane && lane != 0) return;
-    const int lp = (c.i * 16) / a.P;
+    // the page of slice c.i, and the slice within it (a shift when P / 16 is a power of two)
+    const int lp = a.tp_shift >= 0 ? c.i >> a.tp_shift : (c.i * 16) / a.P;
     int page = 0;
     if (lane == 0) {
       page = a.page_table[static_cast<size_t>(c.b) * a.stride + lp];
