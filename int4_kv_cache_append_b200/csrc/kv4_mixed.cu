@@ -24,12 +24,14 @@
 //     value range), so that a slice is one contiguous block; tiles ordered (page, head).
 //
 // Decode: the same flattened split-K as the BF16 baseline (16-position tiles of one (sequence, KV
-// head), one bulk copy per tile into a per-warp ring, LSE merge).  QK^T runs on m16n8k16 fp16
-// MMAs: the integer codes are exact fp16 A operands, the query enters as q_j sigma_j 2^(1-w_j) in
-// hi/lo fp16 halves (columns 2h, 2h+1 of the 8 N columns), and the code-independent part
-// sum_j q_j sigma_j (2^-w_j - 1) is added per head; the MMA's k index is permuted so that each
-// lane reads one contiguous bit range of a key row.  PV multiplies the value codes (exact fp16)
-// by p * step in hi/lo halves and adds sum_t p_t zero_t.
+// head) copied into a per-warp ring, LSE merge).  QK^T runs on m16n8k16 fp16 MMAs: the integer
+// codes enter as exact subnormal fp16 A operands (placed at the top of the mantissa field), the
+// query as q_j sigma_j in hi/lo fp16 halves (columns 2h, 2h+1 of the 8 N columns) with the
+// remaining power of two in the logit scale, and the code-independent part
+// sum_j q_j sigma_j (2^-w_j - 1) is added per head.  The MMA's k index is permuted so that the
+// four lanes of a key row read neighbouring windows of its bit stream; key rows that would put
+// the row lanes on the same shared-memory banks are padded in shared memory.  PV multiplies the
+// value codes (subnormal fp16 likewise) by p * step in hi/lo halves and adds sum_t p_t zero_t.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -334,6 +336,11 @@ __device__ __forceinline__ float exp2_fast(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// the fp16 in the low half of a word, as a float
+__device__ __forceinline__ float low_half(uint32_t w) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu)));
 }
 
 // fp16 pair (x0, x1) or the pair of their fp16 rounding remainders
@@ -698,7 +705,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
               (z0 & E1.y) | ((z0 * E1.w) & E1.z), (z1 & E1.y) | ((z1 * E1.w) & E1.z), qf[kb][0], qf[kb][1]);
     }
     const __half* prm = reinterpret_cast<const __half*>(buf + PO);
-    const float s0 = v0 ? __half2float(prm[4 * gq]) : 0.f, s1 = v1 ? __half2float(prm[4 * (gq + 8)]) : 0.f;
+    // records (key scale, 0, value zero, value range) of rows gq and gq + 8, 8 bytes each
+    const uint2 rec0 = *reinterpret_cast<const uint2*>(prm + 4 * gq);
+    const uint2 rec1 = *reinterpret_cast<const uint2*>(prm + 4 * (gq + 8));
+    const float s0 = v0 ? low_half(rec0.x) : 0.f, s1 = v1 ? low_half(rec1.x) : 0.f;
     const float lg0 = v0 ? s0 * fmaf(S[0] + S[1], inv_scale, cst) : kNegInf;
     const float lg1 = v1 ? s1 * fmaf(S[2] + S[3], inv_scale, cst) : kNegInf;
 
@@ -724,8 +734,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     const float mu = m_run == kNegInf ? 0.f : m_run;
     const float p0 = v0 ? exp2_fast(lg0 - mu) : 0.f, p1 = v1 ? exp2_fast(lg1 - mu) : 0.f;
     l_part += p0 + p1;
-    if (v0) pz = fmaf(p0, __half2float(prm[4 * gq + 2]), pz);
-    if (v1) pz = fmaf(p1, __half2float(prm[4 * (gq + 8) + 2]), pz);
+    if (v0) pz = fmaf(p0, low_half(rec0.y), pz);
+    if (v1) pz = fmaf(p1, low_half(rec1.y), pz);
 
     // PV.  B: p * step of tokens (2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9) for column gq = (head
     // gq / 2, hi or lo half); A: value codes of dims gq * D/8 + [0, D/8) (rows gq and gq + 8 of
