@@ -697,9 +697,11 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
       const uint32_t* ent = ktab + (kb * 4 + tig) * 8;
       const uint4 E0 = *reinterpret_cast<const uint4*>(ent);      // M0, M1, multiplier of c1, window start
       const uint4 E1 = *reinterpret_cast<const uint4*>(ent + 4);  // shift of z, M2, M3, multiplier of c3
-      const int wi = static_cast<int>(E0.w) >> 5, sh = static_cast<int>(E0.w & 31u);  // wi = -1: the stage's lead bytes
-      const uint32_t x0 = __funnelshift_r(r0w[wi], r0w[wi + 1], sh);
-      const uint32_t x1 = __funnelshift_r(r1w[wi], r1w[wi + 1], sh);
+      // word of the window start (-1: the stage's lead bytes); the funnel shift takes the start
+      // mod 32 itself
+      const int wi = static_cast<int>(E0.w) >> 5;
+      const uint32_t x0 = __funnelshift_r(r0w[wi], r0w[wi + 1], E0.w);
+      const uint32_t x1 = __funnelshift_r(r1w[wi], r1w[wi + 1], E0.w);
       const uint32_t z0 = x0 >> E1.x, z1 = x1 >> E1.x;
       mma_f16(S, (x0 & E0.x) | ((x0 * E0.z) & E0.y), (x1 & E0.x) | ((x1 * E0.z) & E0.y),
               (z0 & E1.y) | ((z0 * E1.w) & E1.z), (z1 & E1.y) | ((z1 * E1.w) & E1.z), qf[kb][0], qf[kb][1]);
