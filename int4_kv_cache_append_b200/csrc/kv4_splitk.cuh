@@ -103,15 +103,37 @@ __device__ __forceinline__ Cur cursor_at(const DecodeArgs& a, int cap, int lane,
 // One warp per (sequence, query head): combine the partials of the warps that covered the pair.
 template <int D, int G>
 __global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a) {
-  const int lane = threadIdx.x & 31;
+  // The tile offsets of the warps' sequences and the total, from one pass of the CTA over the
+  // sequences' lengths (256 at a time, block-wide scan) instead of two scans per warp.
+  __shared__ long long incl_s[256];
+  __shared__ long long wsum_s[8];
+  __shared__ long long carry_s;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int item = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
-  if (item >= a.B * a.Hq) return;
-  const int b = item / a.Hq, j = item - b * a.Hq;
-  const int g = j / G, hi = j - g * G;
+  const bool valid = item < a.B * a.Hq;
+  const int b = valid ? item / a.Hq : 0, j = valid ? item - b * a.Hq : 0;
   const int cap = a.stride * a.P;
-  const long long total = prefix_cost(a, cap, lane, a.B);
+  long long bstart = 0;
+  if (threadIdx.x == 0) carry_s = 0;
+  __syncthreads();
+  for (int base = 0; base < a.B; base += 256) {
+    const int bt = base + static_cast<int>(threadIdx.x);
+    const long long c = bt < a.B ? seq_cost(a, clamp_len(a.lens[bt], cap)) : 0;
+    const long long wi = warp_incl_scan(c, lane);
+    if (lane == 31) wsum_s[warp] = wi;
+    __syncthreads();
+    long long off = carry_s;
+    for (int w = 0; w < warp; ++w) off += wsum_s[w];
+    incl_s[threadIdx.x] = off + wi;
+    __syncthreads();
+    if (valid && b >= base && b < base + 256) bstart = incl_s[b - base] - (b < a.B ? seq_cost(a, clamp_len(a.lens[b], cap)) : 0);
+    if (threadIdx.x == 255) carry_s = incl_s[255];
+    __syncthreads();
+  }
+  const long long total = carry_s;
+  if (!valid) return;
+  const int g = j / G, hi = j - g * G;
   const long long Q = quota(total, a.W);
-  const long long bstart = prefix_cost(a, cap, lane, b);
   const int L = clamp_len(a.lens[b], cap);
   const long long n = (L + 15) >> 4;
   constexpr int PER = D / 32;
