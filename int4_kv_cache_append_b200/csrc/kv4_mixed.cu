@@ -272,19 +272,19 @@ struct MixedGeo {
 __host__ __device__ inline int mixed_slice_bytes(int KR, int VR) { return 16 * (KR + VR) + 128; }
 
 // The 8 lanes of one lane group read the same word offset of 8 key rows at once.  Rows of KR bytes
-// with KR / 4 a multiple of 16 words fall into two banks' worth of offsets (4-way conflicts at
-// 4-bit keys, for D = 128; with the old row-per-lane coordinate map, 8-way at 8-bit).  In shared
-// memory those rows are given 16 more bytes, which spreads the 8 rows over the banks.  The padded
-// rows arrive by one tensor copy whose box starts 16 bytes before each row (the tensor's fill
-// value, no memory traffic); the others by a bulk copy.  Two-way conflicts (KR / 4 = 8 mod 16)
-// cost less than the row-by-row tensor copy and stay.
+// with KR / 4 a multiple of 16 words put those reads on two banks' worth of offsets (4-way
+// conflicts at 4-bit keys for D = 128).  In shared memory such rows get 16 more bytes, which
+// spreads the 8 rows over the banks.  The padded rows arrive by one tensor copy whose box starts
+// 16 bytes before each row (the tensor's fill value, no memory traffic); the others by a bulk
+// copy.  Two-way conflicts (KR / 4 = 8 mod 16) cost less than the row-by-row tensor copy and stay.
 __host__ __device__ inline int mixed_key_pad(int KR) { return (KR / 4) % 16 == 0 ? 16 : 0; }
 
 // A ring stage: [16 bytes][16 key rows of KRP = KR + pad bytes][16 value rows][16 records]; with
-// padded rows, rounded up to 128 bytes (the tensor copy's destination is 128-byte aligned).  A key window may start up to 10 bits before its row (see
-// the extraction table), so row 0 reads the word before it: the first 16 bytes keep that read
-// inside the stage, off the previous one, whose copy may still be landing; with padded rows they
-// are row 0's pad.  The bits read there are masked off.
+// padded rows it is rounded up to 128 bytes (the tensor copy's destination is 128-byte aligned).
+// A key window may start up to 10 bits before its row (see the extraction table), so row 0 reads
+// the word before it: the first 16 bytes keep that read inside the stage, off the previous one,
+// whose copy may still be landing; with padded rows they are row 0's pad.  The bits read there
+// are masked off.
 constexpr int kStageLead = 16;
 __host__ __device__ inline int mixed_stage_bytes_padded(int KR, int VR, int pad) {
   const int b = kStageLead + 16 * (KR + pad) + 16 * VR + 128;
@@ -905,8 +905,12 @@ int mixed_decode_warps_per_cta() { return kWarps; }
 int mixed_decode_ctas_per_sm(int D, int G, int VB, int KB) {
   const int KR = KB * D / 8, VR = VB * D / 8;
   size_t bytes = 0;
-  if (D == 128) bytes = G == 4 ? mixed_smem_bytes<128, 4>(KR, VR) : G == 2 ? mixed_smem_bytes<128, 2>(KR, VR) : mixed_smem_bytes<128, 1>(KR, VR);
-  else bytes = G == 4 ? mixed_smem_bytes<64, 4>(KR, VR) : G == 2 ? mixed_smem_bytes<64, 2>(KR, VR) : mixed_smem_bytes<64, 1>(KR, VR);
+  if (D == 128)
+    bytes = G == 4 ? mixed_smem_bytes<128, 4>(KR, VR) : G == 2 ? mixed_smem_bytes<128, 2>(KR, VR)
+                                                       : mixed_smem_bytes<128, 1>(KR, VR);
+  else
+    bytes = G == 4 ? mixed_smem_bytes<64, 4>(KR, VR) : G == 2 ? mixed_smem_bytes<64, 2>(KR, VR)
+                                                     : mixed_smem_bytes<64, 1>(KR, VR);
   return 2 * (bytes + 1024) <= 227u * 1024u ? 2 : 1;
 }
 

@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a) {
     for (int w = 0; w < warp; ++w) off += wsum_s[w];
     incl_s[threadIdx.x] = off + wi;
     __syncthreads();
-    if (valid && b >= base && b < base + 256) bstart = incl_s[b - base] - (b < a.B ? seq_cost(a, clamp_len(a.lens[b], cap)) : 0);
+    if (valid && b >= base && b < base + 256)  // exclusive prefix of sequence b (b < B when valid)
+      bstart = incl_s[b - base] - seq_cost(a, clamp_len(a.lens[b], cap));
     if (threadIdx.x == 255) carry_s = incl_s[255];
     __syncthreads();
   }
