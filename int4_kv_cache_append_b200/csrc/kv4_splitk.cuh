@@ -101,8 +101,10 @@ __device__ __forceinline__ Cur cursor_at(const DecodeArgs& a, int cap, int lane,
 }
 
 // One warp per (sequence, query head): combine the partials of the warps that covered the pair.
+// At most 64 registers (4 CTAs per SM): the batched loads of long runs would otherwise halve the
+// occupancy that the short runs of large batches need.
 template <int D, int G>
-__global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(256, 4) merge_kernel(const DecodeArgs a) {
   // The tile offsets of the warps' sequences and the total, from one pass of the CTA over the
   // sequences' lengths (256 at a time, block-wide scan) instead of two scans per warp.
   __shared__ long long incl_s[256];
@@ -145,16 +147,42 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a) {
   if (n > 0) {
     const long long cs = bstart + g * n, ce = cs + n;
     const long long sid = static_cast<long long>(b) * a.Hkv + g;
-    for (long long w = cs / Q; w <= (ce - 1) / Q; ++w) {
-      const float* p = a.part + (static_cast<size_t>(w + sid) * G + hi) * kPartRow<D>;
-      const float pm = p[D], pl = p[D + 1];
-      if (!(pl > 0.f)) continue;
+    const long long w0 = cs / Q, w1 = (ce - 1) / Q;  // the warps that covered the pair
+    auto fold = [&](float pm, float pl, const float (&pr)[PER]) {
+      if (!(pl > 0.f)) return;
       const float mn = fmaxf(m, pm);
       const float fo = m == kNegInfF ? 0.f : exp2f(m - mn), fp = exp2f(pm - mn);
       l = l * fo + pl * fp;
 #pragma unroll
-      for (int e = 0; e < PER; ++e) o[e] = o[e] * fo + p[lane * PER + e] * fp;
+      for (int e = 0; e < PER; ++e) o[e] = o[e] * fo + pr[e] * fp;
       m = mn;
+    };
+    auto row = [&](long long w) { return a.part + (static_cast<size_t>(w + sid) * G + hi) * kPartRow<D>; };
+    // Long runs of partials kBatch at a time: their loads are issued together (one memory round
+    // trip per batch), then folded in warp order; the rest one by one.
+    constexpr int kBatch = 8;
+    long long w = w0;
+    for (; w + kBatch - 1 <= w1; w += kBatch) {
+      float2 ml[kBatch];
+      float pv[kBatch][PER];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const float* p = row(w + u);
+        ml[u] = *reinterpret_cast<const float2*>(p + D);
+#pragma unroll
+        for (int e = 0; e < PER; ++e) pv[u][e] = p[lane * PER + e];
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) fold(ml[u].x, ml[u].y, pv[u]);
+    }
+    for (; w <= w1; ++w) {
+      const float* p = row(w);
+      const float pm = p[D], pl = p[D + 1];
+      if (!(pl > 0.f)) continue;
+      float pr[PER];
+#pragma unroll
+      for (int e = 0; e < PER; ++e) pr[e] = p[lane * PER + e];
+      fold(pm, pl, pr);
     }
   }
   float* out = a.out + (static_cast<size_t>(b) * a.Hq + j) * D + lane * PER;
