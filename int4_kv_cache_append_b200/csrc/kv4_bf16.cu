@@ -284,8 +284,7 @@ cudaError_t launch_dg(const DecodeArgs& a, int ctas, cudaStream_t st) {
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  splitk::merge_kernel<D, G><<<(a.B * a.Hq + 7) / 8, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return splitk::launch_merge<D, G>(a, st);
 }
 
 }  // namespace

@@ -861,8 +861,7 @@ cudaError_t launch_dgv(const DecodeArgs& a, int ctas, cudaStream_t st, bool row_
     decode_mixed_kernel<D, G, VB, 0><<<ctas, kWarps * 32, smem, st>>>(a, kmap);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  splitk::merge_kernel<D, G><<<(a.B * a.Hq + 7) / 8, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return splitk::launch_merge<D, G>(a, st);
 }
 
 template <int D, int G>

@@ -100,18 +100,24 @@ __device__ __forceinline__ Cur cursor_at(const DecodeArgs& a, int cap, int lane,
   return c;
 }
 
-// One warp per (sequence, query head): combine the partials of the warps that covered the pair.
-// At most 64 registers (4 CTAs per SM): the batched loads of long runs would otherwise halve the
-// occupancy that the short runs of large batches need.
-template <int D, int G>
+// Combine the partials of the warps that covered a (sequence, query head) pair.  MW = 1: one warp
+// per pair, 8 pairs per CTA.  MW = 8, for batches with few pairs (and long runs of partials each):
+// one pair per CTA, its partials split in 8 consecutive runs folded by the 8 warps, whose states
+// warp 0 then combines.  At most 64 registers (4 CTAs per SM): the batched loads of long runs would
+// otherwise halve the occupancy that short runs need.
+template <int D, int G, int MW>
 __global__ void __launch_bounds__(256, 4) merge_kernel(const DecodeArgs a) {
+  static_assert(MW == 1 || MW == 8, "one warp per pair, or a CTA of 8 warps per pair");
   // The tile offsets of the warps' sequences and the total, from one pass of the CTA over the
   // sequences' lengths (256 at a time, block-wide scan) instead of two scans per warp.
   __shared__ long long incl_s[256];
   __shared__ long long wsum_s[8];
   __shared__ long long carry_s;
+  __shared__ float smo[MW][D];
+  __shared__ float smM[MW], smL[MW];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int item = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int item = MW == 1 ? static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5) : static_cast<int>(blockIdx.x);
+  const int sub = MW == 1 ? 0 : warp;  // this warp's run of the pair's partials
   const bool valid = item < a.B * a.Hq;
   const int b = valid ? item / a.Hq : 0, j = valid ? item - b * a.Hq : 0;
   const int cap = a.stride * a.P;
@@ -134,7 +140,7 @@ __global__ void __launch_bounds__(256, 4) merge_kernel(const DecodeArgs a) {
     __syncthreads();
   }
   const long long total = carry_s;
-  if (!valid) return;
+  if (!valid) return;  // uniform over the CTA when MW = 8
   const int g = j / G, hi = j - g * G;
   const long long Q = quota(total, a.W);
   const int L = clamp_len(a.lens[b], cap);
@@ -147,7 +153,9 @@ __global__ void __launch_bounds__(256, 4) merge_kernel(const DecodeArgs a) {
   if (n > 0) {
     const long long cs = bstart + g * n, ce = cs + n;
     const long long sid = static_cast<long long>(b) * a.Hkv + g;
-    const long long w0 = cs / Q, w1 = (ce - 1) / Q;  // the warps that covered the pair
+    const long long f0 = cs / Q, f1 = (ce - 1) / Q;  // the warps that covered the pair
+    const long long cnt = f1 - f0 + 1;
+    const long long w0 = f0 + sub * cnt / MW, w1 = f0 + (sub + 1) * cnt / MW - 1;  // this warp's run
     auto fold = [&](float pm, float pl, const float (&pr)[PER]) {
       if (!(pl > 0.f)) return;
       const float mn = fmaxf(m, pm);
@@ -185,11 +193,50 @@ __global__ void __launch_bounds__(256, 4) merge_kernel(const DecodeArgs a) {
       fold(pm, pl, pr);
     }
   }
+  if constexpr (MW > 1) {
+    // warp 0 combines the 8 runs' (m, l, o), in run order
+#pragma unroll
+    for (int e = 0; e < PER; ++e) smo[sub][lane * PER + e] = o[e];
+    if (lane == 0) {
+      smM[sub] = m;
+      smL[sub] = l;
+    }
+    __syncthreads();
+    if (sub != 0) return;
+    m = kNegInfF;
+#pragma unroll
+    for (int w = 0; w < MW; ++w)
+      if (smL[w] > 0.f) m = fmaxf(m, smM[w]);
+    l = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) o[e] = 0.f;
+#pragma unroll
+    for (int w = 0; w < MW; ++w) {
+      const float f = smL[w] > 0.f ? exp2f(smM[w] - m) : 0.f;
+      l += f * smL[w];
+#pragma unroll
+      for (int e = 0; e < PER; ++e) o[e] = fmaf(f, smo[w][lane * PER + e], o[e]);
+    }
+  }
   float* out = a.out + (static_cast<size_t>(b) * a.Hq + j) * D + lane * PER;
   const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
   for (int e = 0; e < PER; ++e) out[e] = o[e] * inv;
   if (a.lse && lane == 0) a.lse[static_cast<size_t>(b) * a.Hq + j] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : kNegInfF;
+}
+
+// Pairs below which the merge gives each pair a CTA of 8 warps: fewer pairs than about one wave
+// of warps on 148 SMs leave most of the GPU idle with one warp per pair.
+constexpr int kWideMergePairs = 1024;
+
+template <int D, int G>
+cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t st) {
+  const int items = a.B * a.Hq;
+  if (items < kWideMergePairs)
+    merge_kernel<D, G, 8><<<items, 256, 0, st>>>(a);
+  else
+    merge_kernel<D, G, 1><<<(items + 7) / 8, 256, 0, st>>>(a);
+  return cudaGetLastError();
 }
 
 }  // namespace splitk
